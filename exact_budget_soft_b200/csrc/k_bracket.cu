@@ -1,0 +1,598 @@
+// k_bracket.cu -- probabilistic bracketing and the streaming passes
+// ("Fast LapSum: Exact Differentiable Top-k at Million Scale": technical
+// summary section 2.2 steps 1-4, and the abstract).
+//
+//   sample_kernel   kernel-noised sample y_j = r_{I_j} + t L_j (Philox4x64-10)
+//   select_kernel   exact order statistics y_(jR), y_(jL) by 3-round radix select
+//   stream_kernel   one pass over r: counts and stable tail sums of the scores
+//                   outside [a_L, a_R), band compaction (warp ballots)
+//   certify_kernel  one pass over r: G(a_L), G(a_R) and the verdict
+//   p_kernel        p = F((r - b)/t)
+//   vjp_*_kernel    <g,f>/sum f, then grad = (f/t)(g - <g,f>/sum f)
+//
+// The long passes are persistent grid-stride loops over 16-byte vectors with a
+// fixed grid, so every per-block partial covers a fixed set of elements and the
+// "last block" combine (one atomic ticket, fixed summation order) makes every
+// reduction bitwise reproducible.
+#include <cstdint>
+
+#include "lapsum_device.cuh"
+#include "lapsum_kernels.h"
+
+namespace lapsum {
+
+constexpr int SBLOCK = 256;     // threads per block of the streaming passes
+constexpr int SBLOCKS_PER_SM = 4;
+
+static int g_num_sms = 0;
+int stream_grid() {
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (g_num_sms <= 0) g_num_sms = 148;
+    }
+    return g_num_sms * SBLOCKS_PER_SM;
+}
+
+// ------------------------------------------------------ last-block combine --
+// Every block contributes NV doubles (valid in thread 0).  The block that
+// arrives last sums the partials in a fixed order; returns true there, with the
+// totals in thread 0's v[].
+template <int BLOCK, int NV>
+__device__ bool last_block_sum(double (&v)[NV], double *partials, unsigned *ticket,
+                               double *scratch) {
+    __shared__ bool s_last;
+    const int tid = threadIdx.x;
+    const int G = gridDim.x;
+    if (tid == 0) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) partials[(size_t)i * G + blockIdx.x] = v[i];
+        __threadfence();
+        unsigned tk = atomicAdd(ticket, 1u);
+        s_last = (tk == (unsigned)G - 1);
+    }
+    __syncthreads();
+    if (!s_last) return false;
+    __threadfence();
+    double w[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        double s = 0.0;
+        for (int j = tid; j < G; j += BLOCK) s += __ldcg(partials + (size_t)i * G + j);
+        w[i] = s;
+    }
+    block_sum<BLOCK, NV>(w, scratch);
+    if (tid == 0) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) v[i] = w[i];
+        *ticket = 0u;
+    }
+    return true;
+}
+
+// ================================================================ sample --
+// Philox4x64-10 (Salmon et al., SC'11): per round, multiply words 0 and 2 by the
+// round multipliers, cross the high halves over and xor in the key; the key is
+// bumped by two Weyl constants between rounds.
+__device__ __forceinline__ void philox4x64_10(uint64_t &x0, uint64_t &x1, uint64_t &x2,
+                                              uint64_t &x3, uint64_t k0, uint64_t k1) {
+    const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        uint64_t h0 = __umul64hi(M0, x0), l0 = M0 * x0;
+        uint64_t h1 = __umul64hi(M1, x2), l1 = M1 * x2;
+        uint64_t y0 = h1 ^ x1 ^ k0, y2 = h0 ^ x3 ^ k1;
+        x0 = y0;
+        x1 = l1;
+        x2 = y2;
+        x3 = l0;
+        k0 += W0;
+        k1 += W1;
+    }
+}
+
+// ln x for the sampler, from ln m = 2 atanh((m-1)/(m+1)), x = m 2^e with m in
+// [sqrt(1/2), sqrt(2)): atanh(s)/s = sum_j s^{2j}/(2j+1), 11 terms (|s| <= 0.1716),
+// ln x = e ln2 + ln m.  Written with explicitly rounded IEEE operations only, so
+// a CPU evaluating the same formula in the same order gets the same bits.
+__device__ __forceinline__ double sample_ln(double x) {
+    uint64_t bits = (uint64_t)__double_as_longlong(x);
+    int64_t e = (int64_t)((bits >> 52) & 0x7ff) - 1022;
+    double m = __longlong_as_double((long long)((bits & 0x800FFFFFFFFFFFFFull) | (0x3FEull << 52)));
+    if (m < 0x1.6a09e667f3bcdp-1) {
+        m = __dadd_rn(m, m);
+        e -= 1;
+    }
+    double s = __ddiv_rn(__dsub_rn(m, 1.0), __dadd_rn(m, 1.0));
+    double z = __dmul_rn(s, s);
+    double p = __ddiv_rn(1.0, 21.0);
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 19.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 17.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 15.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 13.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 11.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 9.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 7.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 5.0));
+    p = __fma_rn(p, z, __ddiv_rn(1.0, 3.0));
+    p = __fma_rn(p, z, 1.0);
+    double lnm = __dmul_rn(__dadd_rn(s, s), p);
+    return __fma_rn((double)e, 0x1.62e42fefa39efp-1, lnm);
+}
+
+constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
+
+// y_j = r_{I_j} + t L_j: I_j uniform on [0, n) (high word of u0 * n), L_j ~
+// Laplace(0,1) = a random sign times -ln U, U = ((u1 >> 11) + 1) 2^-53 in (0, 1].
+// This is the operator's own noise kernel, so P(y_j > b) = k/n.  The key kept
+// is the fp32 value rounded toward -inf (monotone, so order statistics commute
+// with it), in the descending-order key space.
+__global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
+    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= P.s) return;
+    uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
+    philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
+    const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
+    const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
+    const double E = -sample_ln(U);
+    const double L = (x1 & 1ull) ? E : -E;
+    const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
+    P.keys[j] = desc_key(__double2float_rd(y));
+}
+
+// ================================================================ select --
+// The jR-th and jL-th smallest sample keys (= the jR-th and jL-th largest
+// values) by a radix select over bits [31:20], [19:8], [7:0]; the first round's
+// histogram is shared by both targets.  Bracket ends rounded outward:
+//   a_R = nextup(y_(jR) rounded down) (> y_(jR)),  a_L = y_(jL) rounded down;
+//   jR = 0 -> a_R = +inf,  jL = s + 1 -> a_L = -inf.
+__device__ __forceinline__ uint32_t block_incl_scan_u32(uint32_t v, uint32_t *s_w) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t p = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += p;
+    }
+    if (lane == 31) s_w[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = lane < (int)(blockDim.x >> 5) ? s_w[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t p = __shfl_up_sync(FULL, w, o);
+            if (lane >= o) w += p;
+        }
+        s_w[lane] = w;
+    }
+    __syncthreads();
+    uint32_t r = x + (warp > 0 ? s_w[warp - 1] : 0u);
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
+    __shared__ uint32_t hist[2][4096];
+    __shared__ uint32_t s_w[32];
+    __shared__ uint32_t s_pref[2], s_rank[2];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int s = (int)P.s;
+    const bool valid0 = P.jR >= 1, valid1 = P.jL <= P.s;
+    if (tid == 0) {
+        s_pref[0] = 0; s_pref[1] = 0;
+        s_rank[0] = (uint32_t)(valid0 ? P.jR : 1);
+        s_rank[1] = (uint32_t)(valid1 ? P.jL : 1);
+    }
+    uint32_t mask = 0;
+    const int shifts[3] = {20, 8, 0};
+    const int widths[3] = {12, 12, 8};
+#pragma unroll 1
+    for (int rd = 0; rd < 3; ++rd) {
+        const int sh = shifts[rd];
+        const uint32_t bm = (1u << widths[rd]) - 1u;
+        const int nb = 1 << widths[rd];
+        for (int i = tid; i < 2 * 4096; i += 1024) (&hist[0][0])[i] = 0;
+        __syncthreads();
+        const uint32_t p0 = s_pref[0], p1 = s_pref[1];
+        for (int i0 = 0; i0 < s; i0 += 1024) {
+            const int i = i0 + tid;
+            const bool in = i < s;
+            const uint32_t key = in ? P.keys[i] : 0u;
+            const uint32_t bin = (key >> sh) & bm;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                if (rd == 0 && q == 1) break;                       // shared first round
+                const bool m = in && (rd == 0 ? (valid0 || valid1)
+                                              : ((key & mask) == (q ? p1 : p0)) && (q ? valid1 : valid0));
+                const unsigned act = __ballot_sync(FULL, m);
+                if (!act) continue;
+                const unsigned peers = __match_any_sync(FULL, m ? bin : 0xffffffffu) & act;
+                if (m && lane == __ffs(peers) - 1) atomicAdd(&hist[q][bin], (uint32_t)__popc(peers));
+            }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t *h = (rd == 0) ? hist[0] : hist[q];
+            // thread tid owns bins [4 tid, 4 tid + 4)
+            uint32_t c[4], loc = 0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int bi = tid * 4 + u;
+                c[u] = bi < nb ? h[bi] : 0u;
+                loc += c[u];
+            }
+            const uint32_t inc = block_incl_scan_u32(loc, s_w);
+            const uint32_t ex = inc - loc;
+            const uint32_t want = s_rank[q];
+            const bool vq = q ? valid1 : valid0;
+            __syncthreads();
+            if (vq && ex < want && want <= inc) {
+                uint32_t cum = ex;
+                for (int u = 0; u < 4; ++u) {
+                    if (cum + c[u] >= want) {
+                        s_pref[q] |= (uint32_t)(tid * 4 + u) << sh;
+                        s_rank[q] = want - cum;
+                        break;
+                    }
+                    cum += c[u];
+                }
+            }
+            __syncthreads();
+        }
+        mask |= bm << sh;
+    }
+    if (tid == 0) {
+        Ctl *c = P.ctl;
+        const float yR = desc_key_to_float(s_pref[0]);
+        const float yL = desc_key_to_float(s_pref[1]);
+        c->a_R = valid0 ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
+        c->a_L = valid1 ? yL : -CUDART_INF_F;
+        c->jR = P.jR;
+        c->jL = P.jL;
+        c->s = P.s;
+        c->path = 2;
+        c->verdict = -1;
+    }
+}
+
+// ================================================================ stream --
+struct StreamAcc {
+    unsigned long long cL, cR;
+    double SL, SR;
+    bool bad;
+};
+
+__device__ __forceinline__ double tier_term(double z) {
+    return z <= EXP_TIER ? exp(-z) : (z < 104.0 ? (double)expf(-(float)z) : 0.0);
+}
+
+// One score of the streaming pass (technical summary section 2.2, step 2):
+// at or above a_R -> count, S_R += e^{-(r-a_R)/t}; below a_L -> count,
+// S_L += e^{(r-a_L)/t}; otherwise append to the band (warp-aggregated slot).
+__device__ __forceinline__ void stream_one(float x, bool valid, float aL, float aR, double daL,
+                                           double daR, double inv_t, StreamAcc &acc, float *band,
+                                           unsigned long long cap, unsigned long long *band_ctr,
+                                           int lane) {
+    const bool above = valid && x >= aR;
+    const bool below = valid && x < aL;
+    const bool inb = valid && x >= aL && x < aR;
+    acc.bad |= valid && !isfinite(x);
+    if (above || below) {
+        const double z = above ? ((double)x - daR) * inv_t : (daL - (double)x) * inv_t;
+        const double e = tier_term(z);
+        if (above) { acc.cR += 1; acc.SR += e; }
+        else       { acc.cL += 1; acc.SL += e; }
+    }
+    const unsigned m = __ballot_sync(FULL, inb);
+    if (m) {
+        const int leader = __ffs(m) - 1;
+        unsigned long long base = 0;
+        if (lane == leader) base = atomicAdd(band_ctr, (unsigned long long)__popc(m));
+        base = __shfl_sync(FULL, base, leader) + __popc(m & ((1u << lane) - 1u));
+        if (inb && base < cap) band[base] = x;
+    }
+}
+
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) stream_kernel(BracketParams P) {
+    __shared__ double s_red[4 * (SBLOCK / 32)];
+    Ctl *ctl = P.ctl;
+    const float aL = ctl->a_L, aR = ctl->a_R;
+    const double daL = aL, daR = aR, inv_t = P.inv_t;
+    const int lane = threadIdx.x & 31;
+    const unsigned long long cap = (unsigned long long)P.band_cap;
+    StreamAcc acc{0, 0, 0.0, 0.0, false};
+    const int64_t n = P.n;
+    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
+    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
+    const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
+    const int64_t n4 = aligned ? n / 4 : 0;
+    const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
+    // whole warps iterate together (the ballot needs every lane)
+    const int64_t n4w = (n4 + gstride - 1) / gstride * gstride;
+    for (int64_t i = gtid; i < n4w; i += gstride) {
+        const bool ok = i < n4;
+        float4 v = ok ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        stream_one(v.x, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+        stream_one(v.y, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+        stream_one(v.z, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+        stream_one(v.w, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+    }
+    const int64_t rem0 = n4 * 4;
+    const int64_t remw = rem0 + ((n - rem0 + gstride - 1) / gstride) * gstride;
+    for (int64_t i = rem0 + gtid; i < remw; i += gstride) {
+        const bool ok = i < n;
+        stream_one(ok ? P.r[i] : 0.f, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+    }
+    if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
+    double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL, acc.SR};
+    block_sum<SBLOCK, 4>(v, s_red);
+    if (last_block_sum<SBLOCK, 4>(v, P.partials, &ctl->ticket[0], s_red) && threadIdx.x == 0) {
+        ctl->c_L = (unsigned long long)v[0];
+        ctl->c_R = (unsigned long long)v[1];
+        ctl->S_L = v[2];
+        ctl->S_R = v[3];
+    }
+}
+
+// ============================================================ certificate --
+// One more linear pass (abstract: "a certification pass ... at the cost of one
+// additional linear pass"; technical summary section 2.2 step 4):
+//   G(a) = #{r >= a} - 1/2 sum_{r>=a} e^{-(r-a)/t} + 1/2 sum_{r<a} e^{(r-a)/t}
+// for a = a_L and a = a_R.  Scores outside the band share one exponential
+// between the two ends (e^{-(r-a_L)/t} = e^{-(r-a_R)/t} e^{-(a_R-a_L)/t}, and the
+// mirror image below), band scores take two.  Verdict: G(a_L) >= k > G(a_R),
+// the band fits its buffer, and both passes agree on every membership count.
+struct CertAcc {
+    unsigned long long cntL, cntR, cntB;   // >= a_L, >= a_R, < a_L
+    double above, below, hiLband, loRband;
+    bool bad;
+};
+
+__device__ __forceinline__ void cert_one(float x, bool valid, float aL, float aR, double daL,
+                                         double daR, double inv_t, CertAcc &a) {
+    if (!valid) return;
+    a.bad |= !isfinite(x);
+    if (x >= aR) {
+        a.cntR += 1;
+        a.cntL += 1;
+        a.above += tier_term(((double)x - daR) * inv_t);
+    } else if (x >= aL) {
+        a.cntL += 1;
+        a.hiLband += tier_term(((double)x - daL) * inv_t);
+        a.loRband += tier_term((daR - (double)x) * inv_t);
+    } else if (x < aL) {
+        a.cntB += 1;
+        a.below += tier_term((daL - (double)x) * inv_t);
+    }
+}
+
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) certify_kernel(BracketParams P) {
+    __shared__ double s_red[7 * (SBLOCK / 32)];
+    Ctl *ctl = P.ctl;
+    const float aL = ctl->a_L, aR = ctl->a_R;
+    const double daL = aL, daR = aR, inv_t = P.inv_t;
+    CertAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, false};
+    const int64_t n = P.n;
+    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
+    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
+    const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
+    const int64_t n4 = aligned ? n / 4 : 0;
+    const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
+    for (int64_t i = gtid; i < n4; i += gstride) {
+        const float4 v = r4[i];
+        cert_one(v.x, true, aL, aR, daL, daR, inv_t, acc);
+        cert_one(v.y, true, aL, aR, daL, daR, inv_t, acc);
+        cert_one(v.z, true, aL, aR, daL, daR, inv_t, acc);
+        cert_one(v.w, true, aL, aR, daL, daR, inv_t, acc);
+    }
+    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) cert_one(P.r[i], true, aL, aR, daL, daR, inv_t, acc);
+    if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
+    double v[7] = {(double)acc.cntL, (double)acc.cntR, (double)acc.cntB, acc.above,
+                   acc.below, acc.hiLband, acc.loRband};
+    block_sum<SBLOCK, 7>(v, s_red);
+    if (last_block_sum<SBLOCK, 7>(v, P.partials + 8 * (size_t)gridDim.x, &ctl->ticket[1], s_red) &&
+        threadIdx.x == 0) {
+        const double cntL = v[0], cntR = v[1], cntB = v[2];
+        const double rho = (aR == CUDART_INF_F || aL == -CUDART_INF_F) ? 0.0 : exp(-(daR - daL) * inv_t);
+        const double GaL = cntL - 0.5 * fma(rho, v[3], v[5]) + 0.5 * v[4];
+        const double GaR = cntR - 0.5 * v[3] + 0.5 * fma(rho, v[4], v[6]);
+        ctl->G_aL = GaL;
+        ctl->G_aR = GaR;
+        const unsigned long long cL = ctl->c_L, cR = ctl->c_R, cb = ctl->c_band;
+        const bool ok = (cb <= (unsigned long long)P.band_cap) && (GaL >= P.k) && (GaR < P.k) &&
+                        (cL + cb + cR == (unsigned long long)n) &&
+                        ((unsigned long long)cntR == cR) && ((unsigned long long)(cntL - cntR) == cb) &&
+                        ((unsigned long long)cntB == cL) && ((ctl->status & ST_NONFINITE) == 0);
+        ctl->verdict = ok ? 1 : 0;
+        if (!ok) ctl->fallback_ran = 1;
+        if (cb > (unsigned long long)P.band_cap) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
+    }
+}
+
+// ================================================================= p pass --
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
+p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict__ p,
+         double *__restrict__ b_out, Ctl *ctl, double *partials) {
+    __shared__ double s_red[SBLOCK / 32];
+    const double b = ctl->b;
+    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
+    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(p)) & 15) == 0;
+    const int64_t n4 = aligned ? n / 4 : 0;
+    const float4 *r4 = reinterpret_cast<const float4 *>(r);
+    float4 *p4 = reinterpret_cast<float4 *>(p);
+    double ps = 0.0;
+    for (int64_t i = gtid; i < n4; i += gstride) {
+        const float4 v = __ldcs(r4 + i);
+        float4 o;
+        o.x = laplace_cdf_f((float)(((double)v.x - b) * inv_t));
+        o.y = laplace_cdf_f((float)(((double)v.y - b) * inv_t));
+        o.z = laplace_cdf_f((float)(((double)v.z - b) * inv_t));
+        o.w = laplace_cdf_f((float)(((double)v.w - b) * inv_t));
+        ps += ((double)o.x + (double)o.y) + ((double)o.z + (double)o.w);
+        __stcs(p4 + i, o);
+    }
+    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
+        const float o = laplace_cdf_f((float)(((double)r[i] - b) * inv_t));
+        ps += (double)o;
+        p[i] = o;
+    }
+    double v[1] = {ps};
+    block_sum<SBLOCK, 1>(v, s_red);
+    if (last_block_sum<SBLOCK, 1>(v, partials + 16 * (size_t)gridDim.x, &ctl->ticket[2], s_red) &&
+        threadIdx.x == 0) {
+        ctl->sum_p = v[0];
+        if (b_out) *b_out = b;
+    }
+}
+
+// =================================================================== VJP --
+struct ShiftSumG {
+    float m;
+    double sf, sgf;
+};
+__device__ __forceinline__ void ss_add(ShiftSumG &s, float ax, float g) {
+    if (ax < s.m) {
+        const double sc = (double)expf(ax - s.m);
+        s.sf *= sc;
+        s.sgf *= sc;
+        s.m = ax;
+    }
+    const double e = (double)expf(s.m - ax);
+    s.sf += e;
+    s.sgf = fma((double)g, e, s.sgf);
+}
+__device__ __forceinline__ ShiftSumG ss_merge(ShiftSumG a, ShiftSumG b) {
+    if (b.sf == 0.0) return a;
+    if (a.sf == 0.0) return b;
+    ShiftSumG r;
+    r.m = fminf(a.m, b.m);
+    const double fa = (double)expf(r.m - a.m), fb = (double)expf(r.m - b.m);
+    r.sf = a.sf * fa + b.sf * fb;
+    r.sgf = a.sgf * fa + b.sgf * fb;
+    return r;
+}
+
+// <g,f> and sum f of one long row, shifted by the running min |x| (the ratio is
+// shift-free); per-block partials merged in block order by the last block.
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
+vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
+                  const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
+    __shared__ ShiftSumG s_w[SBLOCK / 32];
+    __shared__ bool s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const double b = *b_in;
+    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + tid;
+    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(g)) & 15) == 0;
+    const int64_t n4 = aligned ? n / 4 : 0;
+    const float4 *r4 = reinterpret_cast<const float4 *>(r);
+    const float4 *g4 = reinterpret_cast<const float4 *>(g);
+    ShiftSumG ss{CUDART_INF_F, 0.0, 0.0};
+    for (int64_t i = gtid; i < n4; i += gstride) {
+        const float4 v = __ldcs(r4 + i), w = __ldcs(g4 + i);
+        ss_add(ss, fabsf((float)(((double)v.x - b) * inv_t)), w.x);
+        ss_add(ss, fabsf((float)(((double)v.y - b) * inv_t)), w.y);
+        ss_add(ss, fabsf((float)(((double)v.z - b) * inv_t)), w.z);
+        ss_add(ss, fabsf((float)(((double)v.w - b) * inv_t)), w.w);
+    }
+    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
+        ss_add(ss, fabsf((float)(((double)r[i] - b) * inv_t)), g[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ShiftSumG q{__shfl_xor_sync(FULL, ss.m, o), __shfl_xor_sync(FULL, ss.sf, o),
+                    __shfl_xor_sync(FULL, ss.sgf, o)};
+        ss = ss_merge(ss, q);
+    }
+    if (lane == 0) s_w[warp] = ss;
+    __syncthreads();
+    const int G = gridDim.x;
+    if (tid == 0) {
+        ShiftSumG a = s_w[0];
+        for (int w = 1; w < SBLOCK / 32; ++w) a = ss_merge(a, s_w[w]);
+        partials[blockIdx.x] = (double)a.m;
+        partials[G + blockIdx.x] = a.sf;
+        partials[2 * G + blockIdx.x] = a.sgf;
+        __threadfence();
+        s_last = atomicAdd(&ctl->ticket[3], 1u) == (unsigned)G - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid == 0) {
+        ShiftSumG a{CUDART_INF_F, 0.0, 0.0};
+        for (int j = 0; j < G; ++j) {
+            ShiftSumG q{(float)__ldcg(partials + j), __ldcg(partials + G + j), __ldcg(partials + 2 * G + j)};
+            a = ss_merge(a, q);
+        }
+        ctl->vjp_lambda = a.sgf / a.sf;
+        ctl->ticket[3] = 0u;
+    }
+}
+
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
+vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
+                 const float *__restrict__ g, int64_t n, double inv_t, const Ctl *ctl,
+                 float *__restrict__ grad) {
+    const double b = *b_in;
+    const float lam = (float)ctl->vjp_lambda;
+    const float it = (float)inv_t;
+    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
+    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(g) |
+                           reinterpret_cast<uintptr_t>(grad)) & 15) == 0;
+    const int64_t n4 = aligned ? n / 4 : 0;
+    const float4 *r4 = reinterpret_cast<const float4 *>(r);
+    const float4 *g4 = reinterpret_cast<const float4 *>(g);
+    float4 *o4 = reinterpret_cast<float4 *>(grad);
+    for (int64_t i = gtid; i < n4; i += gstride) {
+        const float4 v = __ldcs(r4 + i), w = __ldcs(g4 + i);
+        float4 o;
+        o.x = 0.5f * expf(-fabsf((float)(((double)v.x - b) * inv_t))) * it * (w.x - lam);
+        o.y = 0.5f * expf(-fabsf((float)(((double)v.y - b) * inv_t))) * it * (w.y - lam);
+        o.z = 0.5f * expf(-fabsf((float)(((double)v.z - b) * inv_t))) * it * (w.z - lam);
+        o.w = 0.5f * expf(-fabsf((float)(((double)v.w - b) * inv_t))) * it * (w.w - lam);
+        __stcs(o4 + i, o);
+    }
+    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
+        grad[i] = 0.5f * expf(-fabsf((float)(((double)r[i] - b) * inv_t))) * it * (g[i] - lam);
+}
+
+// ============================================================= launchers --
+cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
+    const unsigned blocks = (unsigned)((P.s + 255) / 256);
+    sample_kernel<<<blocks, 256, 0, st>>>(P);
+    return cudaGetLastError();
+}
+cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
+    select_kernel<<<1, 1024, 0, st>>>(P);
+    return cudaGetLastError();
+}
+cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
+    stream_kernel<<<stream_grid(), SBLOCK, 0, st>>>(P);
+    return cudaGetLastError();
+}
+cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
+    certify_kernel<<<stream_grid(), SBLOCK, 0, st>>>(P);
+    return cudaGetLastError();
+}
+cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
+                          double *partials, cudaStream_t st) {
+    p_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, n, 1.0 / t, p, b_out, ctl, partials);
+    return cudaGetLastError();
+}
+cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
+                              Ctl *ctl, double *partials, cudaStream_t st) {
+    vjp_reduce_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, partials);
+    return cudaGetLastError();
+}
+cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
+                             const Ctl *ctl, float *grad, cudaStream_t st) {
+    vjp_apply_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, grad);
+    return cudaGetLastError();
+}
+
+}  // namespace lapsum

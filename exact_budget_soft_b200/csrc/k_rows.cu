@@ -1,0 +1,288 @@
+// k_rows.cu -- full-sort solver inside one CTA ("Fast LapSum: Exact
+// Differentiable Top-k at Million Scale", technical summary section 2.2,
+// full-sort solver): sort the row, one stable prefix/suffix scan of the
+// threshold curve, interval search, closed-form root; then p = F((r-b)/t).
+//
+// One CTA owns one row of up to BLOCK*KPT scores (32768 at 1024 x 32):
+//  * LSD radix sort of the order-preserving uint32 keys, 8-bit digits, keys in
+//    registers (warp-striped), a shared-memory scatter buffer, per-warp digit
+//    histograms and __match_any_sync ranking (stable); digits on which every
+//    key agrees are skipped;
+//  * each thread then owns a run of KPT consecutive sorted scores: it forms the
+//    links d_j and the run's two affine maps (prefix P and suffix Q), a block
+//    scan composes them, G is evaluated at every run end, the crossing run is
+//    found by a max-reduction and re-scanned lane-per-element by one warp, and
+//    the closed-form root gives b;
+//  * the same CTA streams its row again to write p (the row is L2-resident).
+// The band mode solves the sorted band of the bracketing path with the tail
+// sums as seeds (same page, step 3 "exact solve on the band only").
+#include <cstdint>
+
+#include "lapsum_device.cuh"
+#include "lapsum_kernels.h"
+#include "scan_solve.cuh"
+
+namespace lapsum {
+
+template <int BLOCK, int KPT, bool BAND>
+__global__ void __launch_bounds__(BLOCK, 1)
+rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, double t, double inv_t,
+                float *__restrict__ p_out, double *__restrict__ b_out, Ctl *ctl, int64_t band_cap) {
+    using C = RowCfg<BLOCK, KPT>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + C::SMEM_KEYS);
+    uint32_t *s_dbase = s_hist + C::NW * 256;
+    __shared__ double s_b;
+    __shared__ unsigned s_and, s_or;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int n;
+    const float *row;
+    double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
+    if (BAND) {
+        unsigned long long cb = ctl->c_band;
+        if (cb > (unsigned long long)band_cap) {
+            if (tid == 0) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
+            return;
+        }
+        if (cb > (unsigned long long)C::CAP) return;   // the device-wide sort takes it
+        n = (int)cb;
+        row = scores;
+        m0 = (double)ctl->c_R;
+        top = (double)ctl->a_R;
+        P_top = ctl->S_R;
+        bot = (double)ctl->a_L;
+        Q_bot = ctl->S_L;
+    } else {
+        n = (int)n_arg;
+        row = scores + (int64_t)blockIdx.x * n_arg;
+    }
+
+    if (n == 0) {   // band mode only: one interval [a_L, a_R] with no score inside
+        if (tid == 0) {
+            double ed = (top == CUDART_INF || bot == -CUDART_INF) ? 0.0 : exp((bot - top) * inv_t);
+            double Gt = m0 - 0.5 * P_top + 0.5 * ed * Q_bot;
+            double Gb = m0 - 0.5 * ed * P_top + 0.5 * Q_bot;
+            if (!(Gt < k) || !(Gb >= k)) atomicOr(&ctl->status, ST_NO_ROOT);
+            ctl->b = solve_interval(top, bot, m0, P_top, Q_bot, ed, k, t);
+            ctl->j_star = -1;
+        }
+        return;
+    }
+
+    // ---- load keys (warp-striped), pad with the largest key (sorts last)
+    uint32_t key[KPT];
+    uint32_t kand = 0xffffffffu, kor = 0u;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        int idx = warp * C::SEG + i * 32 + lane;
+        uint32_t kk = 0xffffffffu;
+        if (idx < n) {
+            float v = row[idx];
+            bad |= !isfinite(v);
+            kk = desc_key(v);
+        }
+        key[i] = kk;
+        kand &= kk;
+        kor |= kk;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kand &= __shfl_xor_sync(FULL, kand, o);
+        kor |= __shfl_xor_sync(FULL, kor, o);
+    }
+    if (tid == 0) { s_and = 0xffffffffu; s_or = 0u; }
+    __syncthreads();
+    if (lane == 0) { atomicAnd(&s_and, kand); atomicOr(&s_or, kor); }
+    if (__syncthreads_or(bad) && tid == 0 && ctl) atomicOr(&ctl->status, ST_NONFINITE);
+    const uint32_t diff = s_and ^ s_or;
+
+    block_radix_sort<BLOCK, KPT>(key, s_keys, s_hist, s_dbase, diff);
+
+    int64_t jstar = 0;
+    int32_t *st = ctl ? &ctl->status : nullptr;
+    double b = block_scan_solve<BLOCK, KPT>(s_keys, n, k, t, inv_t, m0, top, P_top, bot, Q_bot,
+                                            s_hist, (BAND || blockIdx.x == 0) ? &jstar : nullptr, st);
+    if (tid == 0) {
+        s_b = b;
+        if (BAND) {
+            ctl->b = b;
+            ctl->j_star = jstar;
+        } else {
+            b_out[blockIdx.x] = b;
+            if (blockIdx.x == 0 && ctl) { ctl->b = b; ctl->j_star = jstar; }
+        }
+    }
+    __syncthreads();
+    if (BAND) return;
+
+    // ---- p = F((r - b)/t) for the row
+    b = s_b;
+    float *prow = p_out + (int64_t)blockIdx.x * n_arg;
+    const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(row) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(prow) & 15) == 0);
+    double psum = 0.0;
+    if (vec) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(row);
+        float4 *p4 = reinterpret_cast<float4 *>(prow);
+        for (int i = tid; i < n / 4; i += BLOCK) {
+            float4 v = r4[i], o;
+            o.x = laplace_cdf_f((float)(((double)v.x - b) * inv_t));
+            o.y = laplace_cdf_f((float)(((double)v.y - b) * inv_t));
+            o.z = laplace_cdf_f((float)(((double)v.z - b) * inv_t));
+            o.w = laplace_cdf_f((float)(((double)v.w - b) * inv_t));
+            psum += ((double)o.x + (double)o.y) + ((double)o.z + (double)o.w);
+            p4[i] = o;
+        }
+    } else {
+        for (int i = tid; i < n; i += BLOCK) {
+            float o = laplace_cdf_f((float)(((double)row[i] - b) * inv_t));
+            psum += (double)o;
+            prow[i] = o;
+        }
+    }
+    if (blockIdx.x == 0 && ctl) {
+        double v[1] = {psum};
+        block_sum<BLOCK, 1>(v, reinterpret_cast<double *>(s_hist));
+        if (tid == 0) ctl->sum_p = v[0];
+    }
+}
+
+// ------------------------------------------------------------------ VJP --
+// Per-row analytic VJP (technical summary section 2.1):
+//   grad_i = (f_i/t)(g_i - lambda),  lambda = <g,f>/sum f,  f_i = e^{-|x_i|}/2.
+// lambda is accumulated from terms shifted by the running minimum of |x|
+// (the shift cancels in the ratio), so it stays defined when every f_i
+// underflows.  Sums in fp64 with a fixed-order block combine.  The second
+// sweep re-reads the row from L2.
+struct ShiftSum {
+    float m;       // running min |x| (terms are e^{m - |x|} <= 1)
+    double sf, sgf;
+};
+__device__ __forceinline__ void shift_add(ShiftSum &s, float ax, float g) {
+    if (ax < s.m) {
+        double sc = (double)expf(ax - s.m);   // 0 when s.m = +inf
+        s.sf *= sc;
+        s.sgf *= sc;
+        s.m = ax;
+    }
+    double e = (double)expf(s.m - ax);
+    s.sf += e;
+    s.sgf = fma((double)g, e, s.sgf);
+}
+__device__ __forceinline__ ShiftSum shift_merge(ShiftSum a, ShiftSum b) {
+    if (b.sf == 0.0) return a;
+    if (a.sf == 0.0) return b;
+    ShiftSum r;
+    r.m = fminf(a.m, b.m);
+    double fa = (double)expf(r.m - a.m), fb = (double)expf(r.m - b.m);
+    r.sf = a.sf * fa + b.sf * fb;
+    r.sgf = a.sgf * fa + b.sgf * fb;
+    return r;
+}
+__device__ __forceinline__ ShiftSum shfl_xor_ss(ShiftSum s, int o) {
+    return {__shfl_xor_sync(FULL, s.m, o), __shfl_xor_sync(FULL, s.sf, o),
+            __shfl_xor_sync(FULL, s.sgf, o)};
+}
+
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK)
+rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
+              const float *__restrict__ g, int64_t n, double inv_t, float *__restrict__ grad) {
+    __shared__ ShiftSum s_ss[BLOCK / 32];
+    __shared__ float s_lam;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t off = (int64_t)blockIdx.x * n;
+    const float *r = scores + off;
+    const float *gg = g + off;
+    float *out = grad + off;
+    const double b = b_in[blockIdx.x];
+    const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(r) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(gg) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
+    ShiftSum ss{CUDART_INF_F, 0.0, 0.0};
+    if (vec) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(r);
+        const float4 *g4 = reinterpret_cast<const float4 *>(gg);
+        for (int64_t i = tid; i < n / 4; i += BLOCK) {
+            float4 v = r4[i], w = g4[i];
+            shift_add(ss, fabsf((float)(((double)v.x - b) * inv_t)), w.x);
+            shift_add(ss, fabsf((float)(((double)v.y - b) * inv_t)), w.y);
+            shift_add(ss, fabsf((float)(((double)v.z - b) * inv_t)), w.z);
+            shift_add(ss, fabsf((float)(((double)v.w - b) * inv_t)), w.w);
+        }
+    } else {
+        for (int64_t i = tid; i < n; i += BLOCK)
+            shift_add(ss, fabsf((float)(((double)r[i] - b) * inv_t)), gg[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss = shift_merge(ss, shfl_xor_ss(ss, o));
+    if (lane == 0) s_ss[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+        ShiftSum a = s_ss[0];
+        for (int w = 1; w < BLOCK / 32; ++w) a = shift_merge(a, s_ss[w]);
+        s_lam = (float)(a.sgf / a.sf);
+    }
+    __syncthreads();
+    const float lam = s_lam;
+    const float it = (float)inv_t;
+    if (vec) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(r);
+        const float4 *g4 = reinterpret_cast<const float4 *>(gg);
+        float4 *o4 = reinterpret_cast<float4 *>(out);
+        for (int64_t i = tid; i < n / 4; i += BLOCK) {
+            float4 v = r4[i], w = g4[i], o;
+            o.x = 0.5f * expf(-fabsf((float)(((double)v.x - b) * inv_t))) * it * (w.x - lam);
+            o.y = 0.5f * expf(-fabsf((float)(((double)v.y - b) * inv_t))) * it * (w.y - lam);
+            o.z = 0.5f * expf(-fabsf((float)(((double)v.z - b) * inv_t))) * it * (w.z - lam);
+            o.w = 0.5f * expf(-fabsf((float)(((double)v.w - b) * inv_t))) * it * (w.w - lam);
+            o4[i] = o;
+        }
+    } else {
+        for (int64_t i = tid; i < n; i += BLOCK)
+            out[i] = 0.5f * expf(-fabsf((float)(((double)r[i] - b) * inv_t))) * it * (gg[i] - lam);
+    }
+}
+
+// ------------------------------------------------------------ launchers --
+template <int BLOCK, int KPT, bool BAND>
+static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n, double k, double t,
+                                   float *p, double *b, Ctl *ctl, int64_t band_cap,
+                                   cudaStream_t st) {
+    using C = RowCfg<BLOCK, KPT>;
+    auto kern = rowsolve_kernel<BLOCK, KPT, BAND>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    kern<<<(unsigned)rows, BLOCK, C::SMEM, st>>>(scores, n, k, t, 1.0 / t, p, b, ctl, band_cap);
+    return cudaGetLastError();
+}
+
+int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
+
+cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
+                                 float *p, double *b, Ctl *ctl, cudaStream_t st) {
+    if (n <= RowCfg<256, 16>::CAP)
+        return launch_rowsolve<256, 16, false>(scores, rows, n, k, t, p, b, ctl, 0, st);
+    return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, st);
+}
+
+cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
+                                 cudaStream_t st) {
+    return launch_rowsolve<1024, 32, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap, st);
+}
+
+cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
+                          int64_t n, double t, float *grad, cudaStream_t st) {
+    rowvjp_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, b, g, n, 1.0 / t, grad);
+    return cudaGetLastError();
+}
+
+}  // namespace lapsum

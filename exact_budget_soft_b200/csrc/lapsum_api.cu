@@ -1,0 +1,510 @@
+// lapsum_api.cu -- the C ABI (include/lapsum.h): argument checks, per-stream
+// workspace, the launch sequence of each solver path, diagnostics, timing.
+//
+// Paths ("Fast LapSum: Exact Differentiable Top-k at Million Scale",
+// technical summary section 2.2, and the abstract):
+//   full sort, n <= 32768      one launch: one CTA per row sorts, scans, solves
+//                              and writes p
+//   full sort, longer rows     device radix sort -> locate-scan -> p pass
+//   bracketing (rows == 1,     sample -> select -> streaming pass -> band solve
+//   n >= 2^20 by default)      (one CTA, or device sort + locate) -> certification
+//                              -> gated full-sort fallback -> p pass
+// No step synchronises the host: the band size and the verdict live in device
+// memory and every gated kernel returns at once when it has nothing to do.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "../../include/lapsum.h"
+#include "lapsum_internal.h"
+#include "lapsum_kernels.h"
+
+using namespace lapsum;
+
+namespace {
+
+// ------------------------------------------------------------ profiling --
+struct ProfRec {
+    const char *name;
+    cudaEvent_t e0, e1;
+};
+struct ProfAcc {
+    int64_t launches = 0;
+    double ms = 0.0;
+};
+std::mutex g_prof_mu;
+int g_prof_mode = 0;
+std::vector<ProfRec> g_prof_pending;
+std::vector<std::pair<std::string, ProfAcc>> g_prof_acc;
+std::vector<cudaEvent_t> g_event_pool;
+int64_t g_launches = 0;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// RAII: counts one kernel launch and, when profiling, brackets it with events.
+struct Launch {
+    const char *name;
+    cudaStream_t st;
+    cudaEvent_t e0 = nullptr;
+    Launch(const char *nm, cudaStream_t s) : name(nm), st(s) {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        ++g_launches;
+        if (g_prof_mode) {
+            e0 = take_event();
+            cudaEventRecord(e0, st);
+        }
+    }
+    ~Launch() {
+        if (!e0) return;
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        cudaEvent_t e1 = take_event();
+        cudaEventRecord(e1, st);
+        g_prof_pending.push_back({name, e0, e1});
+    }
+};
+
+// ------------------------------------------------------------ workspace --
+template <typename T>
+cudaError_t grow(T *&p, size_t &have, size_t need) {
+    if (need <= have && p) return cudaSuccess;
+    if (p) {
+        cudaFree(p);
+        p = nullptr;
+        have = 0;
+    }
+    size_t n = need < 64 ? 64 : need;
+    cudaError_t e = cudaMalloc(reinterpret_cast<void **>(&p), n * sizeof(T));
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(p, 0, n * sizeof(T));
+    have = n;
+    return e;
+}
+
+struct Workspace {
+    Ctl *ctl = nullptr;               size_t ctl_n = 0;
+    double *partials = nullptr;       size_t partials_n = 0;
+    uint32_t *skeys = nullptr;        size_t skeys_n = 0;
+    float *band = nullptr;            size_t band_n = 0;
+    uint32_t *keys0 = nullptr;        size_t keys0_n = 0;
+    uint32_t *keys1 = nullptr;        size_t keys1_n = 0;
+    unsigned long long *hist = nullptr; size_t hist_n = 0;
+    uint32_t *dbase = nullptr;        size_t dbase_n = 0;
+    unsigned long long *lookback = nullptr; size_t lookback_n = 0;
+    double *tilebuf = nullptr;        size_t tilebuf_n = 0;
+    uint32_t epoch = 1;
+
+    void release() {
+        cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(band);
+        cudaFree(keys0); cudaFree(keys1); cudaFree(hist); cudaFree(dbase);
+        cudaFree(lookback); cudaFree(tilebuf);
+        *this = Workspace();
+    }
+};
+
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace *> g_ws;
+
+Workspace *get_ws(cudaStream_t st) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    auto key = std::make_pair(dev, st);
+    auto it = g_ws.find(key);
+    if (it != g_ws.end()) return it->second;
+    Workspace *w = new Workspace();
+    g_ws[key] = w;
+    return w;
+}
+
+cudaError_t ws_base(Workspace *w) {
+    cudaError_t e = grow(w->ctl, w->ctl_n, 1);
+    if (e == cudaSuccess) e = grow(w->partials, w->partials_n, (size_t)stream_grid() * 24 + 64);
+    return e;
+}
+
+cudaError_t ws_sort(Workspace *w, int64_t cap) {
+    cudaError_t e = grow(w->keys0, w->keys0_n, (size_t)cap);
+    if (e == cudaSuccess) e = grow(w->keys1, w->keys1_n, (size_t)cap);
+    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256);
+    if (e == cudaSuccess) e = grow(w->dbase, w->dbase_n, 4 * 256);
+    const size_t rt = (size_t)((cap + radix_tile() - 1) / radix_tile()) + 1;
+    if (e == cudaSuccess) e = grow(w->lookback, w->lookback_n, rt * 256);
+    const size_t lt = (size_t)((cap + locate_tile() - 1) / locate_tile()) + 1;
+    if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, lt * 8);
+    return e;
+}
+
+SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32_t gate,
+                   int32_t spin_cap) {
+    SortArgs A{};
+    A.src = src;
+    A.n_host = n;
+    A.cap = cap;
+    A.keys[0] = w->keys0;
+    A.keys[1] = w->keys1;
+    A.hist = w->hist;
+    A.dbase = w->dbase;
+    A.lookback = w->lookback;
+    A.tilebuf = w->tilebuf;
+    A.ctl = w->ctl;
+    A.gate = gate;
+    A.spin_cap = spin_cap;
+    A.epoch = w->epoch++;
+    A.small_cap = rowsolve_capacity();
+    return A;
+}
+
+int map_err(cudaError_t e) {
+    if (e == cudaSuccess) return LAPSUM_OK;
+    if (e == cudaErrorMemoryAllocation) return LAPSUM_ERR_ALLOC;
+    return LAPSUM_ERR_CUDA;
+}
+
+#define LAPSUM_TRY(expr)                            \
+    do {                                            \
+        cudaError_t _e = (expr);                    \
+        if (_e != cudaSuccess) return map_err(_e);  \
+    } while (0)
+
+// ---------------------------------------------------- binomial ranks --
+// Ranks of the binomial order-statistic bracket ("Fast LapSum" abstract and
+// technical summary section 2.2 step 1): X = #{y_j > b} ~ Binomial(s, pi = k/n).
+//   jR = largest j with P(X < j) <= delta/2 (0 -> a_R = +inf),
+//   jL = smallest j with P(X >= j) <= delta/2 (s+1 -> a_L = -inf).
+// The pmf is built outward from the mode by the ratio recurrence
+// pmf(j+1)/pmf(j) = (s-j)/(j+1) * pi/(1-pi), in log space, normalised at the mode.
+void binomial_ranks(int64_t s, double pi, double delta, int64_t &jR, int64_t &jL) {
+    const int64_t mode = (int64_t)std::floor((double)(s + 1) * pi) > s ? s
+                         : (int64_t)std::floor((double)(s + 1) * pi);
+    const double lmode = std::lgamma((double)s + 1.0) - std::lgamma((double)mode + 1.0) -
+                         std::lgamma((double)(s - mode) + 1.0) + (double)mode * std::log(pi) +
+                         (double)(s - mode) * std::log1p(-pi);
+    const double lodds = std::log(pi) - std::log1p(-pi);
+    std::vector<double> lp((size_t)s + 1);
+    lp[(size_t)mode] = lmode;
+    for (int64_t j = mode; j < s; ++j)
+        lp[(size_t)j + 1] = lp[(size_t)j] + std::log((double)(s - j) / (double)(j + 1)) + lodds;
+    for (int64_t j = mode; j > 0; --j)
+        lp[(size_t)j - 1] = lp[(size_t)j] - std::log((double)(s - j + 1) / (double)j) - lodds;
+    const double half = 0.5 * delta;
+    // lower tail, smallest terms first
+    double acc = 0.0, comp = 0.0;
+    jR = 0;
+    for (int64_t j = 1; j <= s; ++j) {
+        const double term = std::exp(lp[(size_t)j - 1]);
+        const double y = term - comp, tt = acc + y;
+        comp = (tt - acc) - y;
+        acc = tt;                                  // acc = P(X < j)
+        if (acc <= half) jR = j; else break;
+    }
+    acc = 0.0; comp = 0.0;
+    jL = s + 1;
+    for (int64_t j = s; j >= 0; --j) {
+        const double term = std::exp(lp[(size_t)j]);
+        const double y = term - comp, tt = acc + y;
+        comp = (tt - acc) - y;
+        acc = tt;                                  // acc = P(X >= j)
+        if (acc <= half) jL = j; else break;
+    }
+}
+
+int check_args(const float *scores, int64_t rows, int64_t n, double k, double t) {
+    if (!scores || rows < 1 || n < 1 || n >= (int64_t(1) << 31)) return LAPSUM_ERR_ARG;
+    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_ERR_ARG;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_ERR_ARG;
+    return LAPSUM_OK;
+}
+
+// Full sort of one long row on the device (also the certification fallback).
+int full_sort_row(Workspace *w, const float *r, int64_t n, double k, double t, int32_t gate,
+                  int32_t spin_cap, cudaStream_t st) {
+    LAPSUM_TRY(ws_sort(w, n));
+    SortArgs A = sort_args(w, r, n, n, gate, spin_cap);
+    {
+        Launch L("radix_sort(5 kernels)", st);
+        g_launches += 4;
+        LAPSUM_TRY(launch_radix_sort(A, k, t, st));
+    }
+    {
+        Launch L("locate", st);
+        LAPSUM_TRY(launch_locate(A, k, t, st));
+    }
+    return LAPSUM_OK;
+}
+
+}  // namespace
+
+// ===================================================================== ABI --
+extern "C" {
+
+const char *lapsum_strerror(int code) {
+    switch (code) {
+        case LAPSUM_OK: return "ok";
+        case LAPSUM_ERR_ARG: return "invalid argument";
+        case LAPSUM_ERR_NONFINITE: return "non-finite score";
+        case LAPSUM_ERR_ALLOC: return "workspace allocation failed";
+        case LAPSUM_ERR_DEVICE_TIMEOUT: return "an inter-block wait gave up (spin cap)";
+        case LAPSUM_ERR_CUDA: return "CUDA runtime error";
+        case LAPSUM_ERR_NO_ROOT: return "no crossing found";
+        default: return "unknown error";
+    }
+}
+
+int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, double t,
+                      float *p_out, double *b_out, const lapsum_options *opt_in,
+                      struct CUstream_st *stream_in) {
+    int rc = check_args(scores, rows, n, k, t);
+    if (rc) return rc;
+    if (!p_out || !b_out) return LAPSUM_ERR_ARG;
+    lapsum_options opt{};
+    if (opt_in) opt = *opt_in;
+    if (opt.delta != 0.0 && !(opt.delta > 0.0 && opt.delta < 1.0)) return LAPSUM_ERR_ARG;
+    if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < 0) return LAPSUM_ERR_ARG;
+    if (opt.force_path < 0 || opt.force_path > 2) return LAPSUM_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    const int32_t spin_cap = opt.spin_cap ? opt.spin_cap : (1 << 20);
+    Workspace *w = get_ws(st);
+    LAPSUM_TRY(ws_base(w));
+
+    int path = opt.force_path;
+    if (path == LAPSUM_PATH_AUTO)
+        path = (rows == 1 && n >= (int64_t(1) << 20)) ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
+    if (path == LAPSUM_PATH_BRACKET && rows != 1) {
+        // one bracket per row: rows are solved one after another
+        for (int64_t r = 0; r < rows; ++r) {
+            rc = lapsum_forward_ex(scores + r * n, 1, n, k, t, p_out + r * n, b_out + r, &opt, stream_in);
+            if (rc) return rc;
+        }
+        return LAPSUM_OK;
+    }
+
+    if (path == LAPSUM_PATH_FULLSORT) {
+        if (n <= rowsolve_capacity()) {
+            LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
+            Launch L("rowsolve", st);
+            LAPSUM_TRY(launch_rowsolve_rows(scores, rows, n, k, t, p_out, b_out, w->ctl, st));
+            return LAPSUM_OK;
+        }
+        for (int64_t r = 0; r < rows; ++r) {
+            const float *row = scores + r * n;
+            LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
+            rc = full_sort_row(w, row, n, k, t, GATE_ALWAYS, spin_cap, st);
+            if (rc) return rc;
+            Launch L("p_pass", st);
+            LAPSUM_TRY(launch_p_pass(row, n, t, p_out + r * n, b_out + r, w->ctl, w->partials, st));
+        }
+        return LAPSUM_OK;
+    }
+
+    // ---------------------------------------------------- bracketing --
+    BracketParams P{};
+    P.r = scores;
+    P.n = n;
+    P.k = k;
+    P.t = t;
+    P.inv_t = 1.0 / t;
+    P.seed = opt.seed;
+    P.row = 0;
+    int64_t s = 0, band_cap = 0;
+    rc = lapsum_bracket_plan(n, k, &opt, &s, &P.jR, &P.jL, &band_cap);
+    if (rc) return rc;
+    P.s = s;
+    P.band_cap = band_cap;
+    P.spin_cap = spin_cap;
+    LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
+    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_cap));
+    LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort the whole row
+    P.band = w->band;
+    P.keys = w->skeys;
+    P.partials = w->partials;
+    P.ctl = w->ctl;
+
+    LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
+    { Launch L("sample", st); LAPSUM_TRY(launch_sample(P, st)); }
+    { Launch L("select", st); LAPSUM_TRY(launch_select(P, st)); }
+    { Launch L("stream_pass", st); LAPSUM_TRY(launch_stream_pass(P, st)); }
+    { Launch L("band_rowsolve", st); LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st)); }
+    if (band_cap > rowsolve_capacity()) {
+        SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap);
+        {
+            Launch L("band_radix_sort(5 kernels)", st);
+            g_launches += 4;
+            LAPSUM_TRY(launch_radix_sort(A, k, t, st));
+        }
+        { Launch L("band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
+    }
+    { Launch L("certify", st); LAPSUM_TRY(launch_certify(P, st)); }
+    rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, st);
+    if (rc) return rc;
+    { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, st)); }
+    return LAPSUM_OK;
+}
+
+int lapsum_bracket_plan(int64_t n, double k, const lapsum_options *opt_in, int64_t *s_out,
+                        int64_t *jR, int64_t *jL, int64_t *band_cap_out) {
+    if (n < 1 || !(k > 0.0) || !(k < (double)n) || !s_out || !jR || !jL || !band_cap_out)
+        return LAPSUM_ERR_ARG;
+    lapsum_options opt{};
+    if (opt_in) opt = *opt_in;
+    if (opt.delta != 0.0 && !(opt.delta > 0.0 && opt.delta < 1.0)) return LAPSUM_ERR_ARG;
+    if (opt.sample_size < 0 || opt.band_cap < 0) return LAPSUM_ERR_ARG;
+    int64_t s = opt.sample_size;
+    if (s == 0) {
+        int64_t pw = 1;
+        while (pw * 2 <= n / 64) pw *= 2;
+        s = std::min<int64_t>(65536, std::max<int64_t>(4096, pw));
+    }
+    if (s > (int64_t(1) << 24)) return LAPSUM_ERR_ARG;
+    const double delta = opt.delta != 0.0 ? opt.delta : 1e-6;
+    binomial_ranks(s, k / (double)n, delta, *jR, *jL);
+    int64_t band_cap = opt.band_cap;
+    if (band_cap == 0) {
+        const double want = 4.0 * (double)n * (double)(*jL - *jR + 2) / (double)s;
+        band_cap = std::max<int64_t>(65536, (int64_t)std::ceil(want));
+    }
+    *band_cap_out = std::min<int64_t>(band_cap, n);
+    *s_out = s;
+    return LAPSUM_OK;
+}
+
+int lapsum_forward(const float *scores, int64_t rows, int64_t n, double k, double t, float *p_out,
+                   double *b_out, struct CUstream_st *stream) {
+    return lapsum_forward_ex(scores, rows, n, k, t, p_out, b_out, nullptr, stream);
+}
+
+int lapsum_backward(const float *scores, const double *b, const float *g, int64_t rows, int64_t n,
+                    double t, float *grad_out, struct CUstream_st *stream_in) {
+    if (!scores || !b || !g || !grad_out || rows < 1 || n < 1 || n >= (int64_t(1) << 31))
+        return LAPSUM_ERR_ARG;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    if (rows > 1 || n <= 65536) {
+        Launch L("rowvjp", st);
+        LAPSUM_TRY(launch_rowvjp(scores, b, g, rows, n, t, grad_out, st));
+        return LAPSUM_OK;
+    }
+    Workspace *w = get_ws(st);
+    LAPSUM_TRY(ws_base(w));
+    { Launch L("vjp_reduce", st); LAPSUM_TRY(launch_vjp_reduce(scores, b, g, n, t, w->ctl, w->partials, st)); }
+    { Launch L("vjp_apply", st); LAPSUM_TRY(launch_vjp_apply(scores, b, g, n, t, w->ctl, grad_out, st)); }
+    return LAPSUM_OK;
+}
+
+int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream_in) {
+    if (!out) return LAPSUM_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    Workspace *w = get_ws(st);
+    std::memset(out, 0, sizeof(*out));
+    if (!w->ctl) return LAPSUM_OK;
+    LAPSUM_TRY(cudaStreamSynchronize(st));
+    Ctl c;
+    LAPSUM_TRY(cudaMemcpy(&c, w->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost));
+    out->path = c.path == 2 ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
+    out->verdict = c.path == 2 ? c.verdict : -1;
+    out->status = c.status;
+    out->fallback = c.fallback_ran;
+    out->s = c.s;
+    out->jR = c.jR;
+    out->jL = c.jL;
+    out->c_L = (int64_t)c.c_L;
+    out->c_band = (int64_t)c.c_band;
+    out->c_R = (int64_t)c.c_R;
+    out->a_L = c.a_L;
+    out->a_R = c.a_R;
+    out->S_L = c.S_L;
+    out->S_R = c.S_R;
+    out->G_aL = c.G_aL;
+    out->G_aR = c.G_aR;
+    out->b = c.b;
+    out->sum_p = c.sum_p;
+    out->j_star = c.j_star;
+    if (c.status & ST_NONFINITE) return LAPSUM_ERR_NONFINITE;
+    if (c.status & ST_TIMEOUT) return LAPSUM_ERR_DEVICE_TIMEOUT;
+    if ((c.status & ST_NO_ROOT) && !(c.path == 2 && c.fallback_ran)) return LAPSUM_ERR_NO_ROOT;
+    return LAPSUM_OK;
+}
+
+int lapsum_release(void) {
+    cudaDeviceSynchronize();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    for (auto it = g_ws.begin(); it != g_ws.end();) {
+        if (it->first.first == dev) {
+            it->second->release();
+            delete it->second;
+            it = g_ws.erase(it);
+        } else {
+            ++it;
+        }
+    }
+    return LAPSUM_OK;
+}
+
+int lapsum_profile_enable(int mode) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (mode == 2) {
+        for (auto &r : g_prof_pending) {
+            g_event_pool.push_back(r.e0);
+            g_event_pool.push_back(r.e1);
+        }
+        g_prof_pending.clear();
+        g_prof_acc.clear();
+        mode = g_prof_mode;
+    }
+    g_prof_mode = mode ? 1 : 0;
+    return LAPSUM_OK;
+}
+
+int lapsum_profile_read(const char **names, int64_t *launches, double *total_ms, int max) {
+    cudaDeviceSynchronize();
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto &r : g_prof_pending) {
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, r.e0, r.e1);
+        bool found = false;
+        for (auto &a : g_prof_acc) {
+            if (a.first == r.name) {
+                a.second.launches += 1;
+                a.second.ms += ms;
+                found = true;
+                break;
+            }
+        }
+        if (!found) g_prof_acc.push_back({std::string(r.name), ProfAcc{1, (double)ms}});
+        g_event_pool.push_back(r.e0);
+        g_event_pool.push_back(r.e1);
+    }
+    g_prof_pending.clear();
+    int i = 0;
+    for (auto &a : g_prof_acc) {
+        if (i >= max) break;
+        if (names) names[i] = a.first.c_str();
+        if (launches) launches[i] = a.second.launches;
+        if (total_ms) total_ms[i] = a.second.ms;
+        ++i;
+    }
+    return (int)g_prof_acc.size();
+}
+
+int64_t lapsum_launch_count(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    return g_launches;
+}
+
+}  // extern "C"

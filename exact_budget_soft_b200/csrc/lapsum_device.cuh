@@ -1,0 +1,205 @@
+// lapsum_device.cuh -- device building blocks shared by the kernels.
+//
+// Notation ("Fast LapSum: Exact Differentiable Top-k at Million Scale",
+// technical summary sections 2.1-2.2): scores sorted descending
+// c_0 >= c_1 >= ... >= c_{n-1}, temperature t, budget k, Laplace CDF F,
+// G(b) = sum_i F((c_i - b)/t) (continuous, strictly decreasing).
+//
+// Stable threshold curve (the "single stable prefix/suffix scan" of the
+// full-sort solver): with links d_j = e^{(c_{j+1} - c_j)/t} <= 1,
+//   P_j = sum_{i<=j} e^{(c_j - c_i)/t} = 1 + d_{j-1} P_{j-1}      (prefix)
+//   Q_j = sum_{i>=j} e^{(c_i - c_j)/t} = 1 + d_j Q_{j+1}          (suffix)
+//   G(c_j) = m0 + (j+1) - P_j/2 + d_j Q_{j+1}/2
+// where m0 scores lie above c_0 (0 for a full row; the count above a_R for a
+// band).  Every factor is <= 1, so nothing overflows ("max-shifted"), and each
+// recurrence is an affine map x -> a x + s, composed associatively in scans.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "lapsum_internal.h"
+
+namespace lapsum {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// ---------------------------------------------------------------- keys --
+// Order-preserving map float -> uint32 whose ASCENDING order is the DESCENDING
+// order of the floats (largest score first).
+__device__ __forceinline__ uint32_t desc_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? u : (u ^ 0x7fffffffu);
+}
+__device__ __forceinline__ float desc_key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? k : (k ^ 0x7fffffffu));
+}
+
+// ------------------------------------------------------------ exp tiers --
+// e^{-z}, z >= 0.  Terms that can move G by more than ~1e-7 relative to one
+// unit (z <= 16) are formed in fp64; farther terms (< 1.2e-7 each) in fp32,
+// whose error is then below ~1.4e-14 absolute per term.
+constexpr double EXP_TIER = 16.0;
+__device__ __forceinline__ double exp_neg_tiered(double z) {
+    return z <= EXP_TIER ? exp(-z) : (double)expf(-(float)z);
+}
+
+// ------------------------------------------------------- affine maps --
+struct Aff {
+    double a, s;   // x -> a x + s
+};
+__device__ __forceinline__ Aff aff_id() { return {1.0, 0.0}; }
+// first f, then g
+__device__ __forceinline__ Aff aff_then(Aff f, Aff g) { return {g.a * f.a, fma(g.a, f.s, g.s)}; }
+__device__ __forceinline__ Aff shfl_up_aff(Aff v, int o) {
+    return {__shfl_up_sync(FULL, v.a, o), __shfl_up_sync(FULL, v.s, o)};
+}
+__device__ __forceinline__ Aff shfl_down_aff(Aff v, int o) {
+    return {__shfl_down_sync(FULL, v.a, o), __shfl_down_sync(FULL, v.s, o)};
+}
+__device__ __forceinline__ Aff shfl_aff(Aff v, int src) {
+    return {__shfl_sync(FULL, v.a, src), __shfl_sync(FULL, v.s, src)};
+}
+// Inclusive warp scan in lane order: lane l gets map_0 then ... then map_l.
+__device__ __forceinline__ Aff warp_scan_fwd(Aff v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        Aff p = shfl_up_aff(v, o);
+        if (lane >= o) v = aff_then(p, v);
+    }
+    return v;
+}
+// Inclusive warp scan in reverse lane order: lane l gets map_31 then ... then map_l.
+__device__ __forceinline__ Aff warp_scan_bwd(Aff v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        Aff p = shfl_down_aff(v, o);
+        if (lane + o < 32) v = aff_then(p, v);
+    }
+    return v;
+}
+
+// Block-wide EXCLUSIVE scans of one affine map per thread (thread order).
+// fwd: thread i gets map_0 then ... then map_{i-1};
+// bwd: thread i gets map_{NT-1} then ... then map_{i+1}.
+// scratch: 2*NW Aff in shared memory.  Contains __syncthreads.
+template <int BLOCK>
+__device__ __forceinline__ void block_scan_excl_both(Aff fwd, Aff bwd, Aff &fwd_ex, Aff &bwd_ex,
+                                                     Aff *scratch) {
+    constexpr int NW = BLOCK / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    Aff fi = warp_scan_fwd(fwd, lane);
+    Aff bi = warp_scan_bwd(bwd, lane);
+    if (lane == 31) scratch[warp] = fi;
+    if (lane == 0) scratch[NW + warp] = bi;
+    __syncthreads();
+    if (warp == 0) {
+        Aff wf = lane < NW ? scratch[lane] : aff_id();
+        Aff wb = lane < NW ? scratch[NW + lane] : aff_id();
+        wf = warp_scan_fwd(wf, lane);
+        // reverse order over the NW warps: lanes >= NW carry the identity
+        wb = warp_scan_bwd(wb, lane);
+        __syncwarp();
+        if (lane < NW) {
+            scratch[lane] = wf;        // inclusive over warps 0..lane
+            scratch[NW + lane] = wb;   // inclusive over warps lane..NW-1
+        }
+    }
+    __syncthreads();
+    Aff fe = shfl_up_aff(fi, 1);
+    if (lane == 0) fe = aff_id();
+    if (warp > 0) fe = aff_then(scratch[warp - 1], fe);
+    Aff be = shfl_down_aff(bi, 1);
+    if (lane == 31) be = aff_id();
+    if (warp < NW - 1) be = aff_then(scratch[NW + warp + 1], be);
+    fwd_ex = fe;
+    bwd_ex = be;
+    __syncthreads();
+}
+
+// ------------------------------------------------------- reductions --
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+__device__ __forceinline__ int warp_max_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+
+// Fixed-order block sum of up to 4 doubles (result valid in thread 0).
+template <int BLOCK, int N>
+__device__ __forceinline__ void block_sum(double (&v)[N], double *scratch /* N*NW */) {
+    constexpr int NW = BLOCK / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = warp_sum(v[i]);
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) scratch[i * NW + warp] = v[i];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            double s = 0.0;
+            for (int w = 0; w < NW; ++w) s += scratch[i * NW + w];
+            v[i] = s;
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------- closed-form root --
+// Root of G(b) = k inside one interval [L, U] between consecutive sorted
+// values ("closed-form root within the interval where the budget equation
+// balances", technical summary section 2.2).  In the interval
+//   G(b) = A - (P_U/2) e^{(b-U)/t} + (Q_L/2) e^{(L-b)/t},
+// A = #scores >= U, P_U = sum_{r>=U} e^{(U-r)/t}, Q_L = sum_{r<=L} e^{(r-L)/t},
+// e_d = e^{(L-U)/t}.  With v = e^{(b-L)/t} in [1, 1/e_d] this is the quadratic
+//   (P_U e_d / 2) v^2 + (k - A) v - Q_L/2 = 0,
+// (the unshifted form is 1/2 S- u^2 + (k-m) u - 1/2 S+ = 0, u = e^{b/t}),
+// whose positive root is taken in the cancellation-free form for the sign of
+// k - A.  L = -inf (nothing below) uses w = e^{(b-U)/t}: A - P_U w/2 = k.
+__device__ __forceinline__ double solve_interval(double U, double L, double A, double P_U,
+                                                 double Q_L, double e_d, double k, double t) {
+    if (L == -CUDART_INF) {
+        double w = 2.0 * (A - k) / P_U;
+        return U + t * log(w);
+    }
+    double a2 = P_U * e_d;
+    double bq = k - A;
+    double sq = sqrt(fma(bq, bq, a2 * Q_L));
+    double v;
+    if (bq >= 0.0) v = (bq + sq) > 0.0 ? Q_L / (bq + sq) : 1.0;
+    else           v = (sq - bq) / a2;
+    if (!(v >= 1.0)) v = 1.0;
+    double b = L + t * log(v);
+    if (b > U) b = U;
+    return b;
+}
+
+// Laplace CDF of an fp32 argument, F(x) = e^x/2 (x < 0), 1 - e^{-x}/2 (x >= 0).
+__device__ __forceinline__ float laplace_cdf_f(float x) {
+    float e = 0.5f * expf(-fabsf(x));
+    return x < 0.0f ? e : 1.0f - e;
+}
+
+// ------------------------------------------------ bounded device waits --
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+}  // namespace lapsum

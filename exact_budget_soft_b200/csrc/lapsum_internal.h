@@ -1,0 +1,63 @@
+// lapsum_internal.h -- state shared by the host orchestration and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lapsum {
+
+// Device error bits (lapsum_stats.status).
+enum : int32_t {
+    ST_NONFINITE = 1,
+    ST_TIMEOUT = 2,
+    ST_BAND_OVERFLOW = 4,
+    ST_NO_ROOT = 8,
+};
+
+// Device-resident control block of one single-row solve.  Every field is
+// written by a kernel and read by a later kernel on the same stream; the host
+// only clears it (one memset per call) and copies it back for diagnostics.
+struct Ctl {
+    // bracket (sample + select)
+    float a_L, a_R;
+    int64_t jR, jL, s;
+    // streaming pass
+    unsigned long long c_L, c_R, c_band;
+    double S_L, S_R;
+    // certification pass
+    double G_aL, G_aR;
+    int32_t verdict;          // 1 certified, 0 not (fallback must run), -1 n/a
+    int32_t status;           // ST_* bits
+    int32_t path;
+    int32_t fallback_ran;
+    // solution
+    double b;
+    int64_t j_star;
+    double sum_p;
+    // single-pass "last block" tickets (zeroed with the block)
+    unsigned int ticket[8];
+    // radix sort: which buffer holds the current keys (-1: the fp32 source)
+    int32_t sort_cur;
+    int32_t sort_skip;        // bit d: every key agrees on digit d (pass skipped)
+    unsigned int tile_ctr[4];
+    // backward
+    double vjp_lambda;
+};
+
+// Kernel-facing parameters of a bracketing solve.
+struct BracketParams {
+    const float *r;
+    int64_t n;
+    double k, t, inv_t;
+    uint64_t seed;
+    int64_t row;
+    int64_t s;
+    int64_t jR, jL;
+    int64_t band_cap;
+    float *band;              // band buffer [band_cap]
+    uint32_t *keys;           // sample keys [s]
+    double *partials;         // per-block partials
+    Ctl *ctl;
+    int32_t spin_cap;
+};
+
+}  // namespace lapsum

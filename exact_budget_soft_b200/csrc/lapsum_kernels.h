@@ -1,0 +1,54 @@
+// lapsum_kernels.h -- host-side launchers of the kernels (internal).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lapsum_internal.h"
+
+namespace lapsum {
+
+// in-CTA full-sort solver (k_rows.cu)
+int rowsolve_capacity();
+cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
+                                 float *p, double *b, Ctl *ctl, cudaStream_t st);
+cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
+                                 cudaStream_t st);
+cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
+                          int64_t n, double t, float *grad, cudaStream_t st);
+
+// bracketing pipeline and streaming passes (k_bracket.cu)
+int stream_grid();
+cudaError_t launch_sample(const BracketParams &P, cudaStream_t st);
+cudaError_t launch_select(const BracketParams &P, cudaStream_t st);
+cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st);
+cudaError_t launch_certify(const BracketParams &P, cudaStream_t st);
+cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
+                          double *partials, cudaStream_t st);
+cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
+                              Ctl *ctl, double *partials, cudaStream_t st);
+cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
+                             const Ctl *ctl, float *grad, cudaStream_t st);
+
+// device-wide radix sort + locate-scan (k_radix.cu)
+enum Gate : int32_t { GATE_ALWAYS = 0, GATE_BAND = 1, GATE_FALLBACK = 2 };
+struct SortArgs {
+    const float *src;          // fp32 scores (keys made on the fly)
+    int64_t n_host;            // element count when gate != GATE_BAND
+    int64_t cap;               // upper bound of the element count (grid sizing)
+    uint32_t *keys[2];         // ping-pong key buffers [cap]
+    unsigned long long *hist;  // [4][256]
+    uint32_t *dbase;           // [4][256]
+    unsigned long long *lookback;  // [tiles][256]
+    double *tilebuf;           // locate per-tile data
+    Ctl *ctl;
+    int32_t gate;
+    int32_t spin_cap;
+    uint32_t epoch;            // distinct per launch sequence (look-back tags)
+    int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
+};
+int radix_tile();
+int locate_tile();
+cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st);
+cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st);
+
+}  // namespace lapsum

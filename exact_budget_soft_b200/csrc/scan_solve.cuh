@@ -1,0 +1,253 @@
+// scan_solve.cuh -- in-CTA radix sort and the threshold-curve scan/solve
+// (full-sort solver of "Fast LapSum: Exact Differentiable Top-k at Million
+// Scale", technical summary section 2.2), shared by the one-CTA row solver and
+// the last CTA of the device-wide locate kernel.
+#pragma once
+#include <cstdint>
+
+#include "lapsum_device.cuh"
+
+namespace lapsum {
+
+template <int BLOCK, int KPT>
+struct RowCfg {
+    static constexpr int NW = BLOCK / 32;
+    static constexpr int CAP = BLOCK * KPT;
+    static constexpr int SEG = 32 * KPT;   // keys per warp segment
+    static constexpr size_t SMEM_KEYS = size_t(CAP) * 4;
+    static constexpr size_t SMEM_HIST = size_t(NW) * 256 * 4;
+    static constexpr size_t SMEM = SMEM_KEYS + SMEM_HIST + 256 * 4 + 2048;
+};
+
+// Block-wide LSD radix sort of warp-striped register keys (ascending).  On
+// return the sorted keys are in s_keys[0 .. CAP).
+template <int BLOCK, int KPT>
+__device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t *s_keys,
+                                                 uint32_t *s_hist, uint32_t *s_dbase,
+                                                 uint32_t diff) {
+    using C = RowCfg<BLOCK, KPT>;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    uint32_t *my_hist = s_hist + warp * 256;
+    bool sorted_in_smem = false;
+#pragma unroll 1
+    for (int sh = 0; sh < 32; sh += 8) {
+        if (((diff >> sh) & 0xffu) == 0u) continue;   // every key has this digit
+        for (int i = tid; i < C::NW * 256; i += BLOCK) s_hist[i] = 0;
+        __syncthreads();
+        // count: per-warp digit histograms (one shared update per group of equal digits)
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) {
+            const uint32_t d = (key[i] >> sh) & 0xffu;
+            const unsigned peers = __match_any_sync(FULL, d);
+            if (lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
+            __syncwarp();
+        }
+        __syncthreads();
+        if (tid < 256) {   // per digit: exclusive prefix over warps, and total
+            uint32_t sum = 0;
+            for (int w = 0; w < C::NW; ++w) {
+                uint32_t c = s_hist[w * 256 + tid];
+                s_hist[w * 256 + tid] = sum;
+                sum += c;
+            }
+            s_dbase[tid] = sum;
+        }
+        __syncthreads();
+        if (warp == 0) {   // exclusive scan of the 256 digit totals
+            uint32_t v[8], run = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { v[j] = s_dbase[lane * 8 + j]; run += v[j]; }
+            uint32_t inc = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                uint32_t p = __shfl_up_sync(FULL, inc, o);
+                if (lane >= o) inc += p;
+            }
+            uint32_t ex = inc - run;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { uint32_t c = v[j]; s_dbase[lane * 8 + j] = ex; ex += c; }
+        }
+        __syncthreads();
+        for (int i = tid; i < C::NW * 256; i += BLOCK) s_hist[i] += s_dbase[i & 255];
+        __syncthreads();
+        // scatter: the same traversal again hands out consecutive slots (stable)
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) {
+            const uint32_t d = (key[i] >> sh) & 0xffu;
+            const unsigned peers = __match_any_sync(FULL, d);
+            const int leader = __ffs(peers) - 1;
+            uint32_t base = 0;
+            if (lane == leader) {
+                base = my_hist[d];
+                my_hist[d] = base + __popc(peers);
+            }
+            base = __shfl_sync(FULL, base, leader) + __popc(peers & lt_mask);
+            s_keys[base] = key[i];
+            __syncwarp();
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) key[i] = s_keys[warp * C::SEG + i * 32 + lane];
+        sorted_in_smem = true;
+        __syncthreads();
+    }
+    if (!sorted_in_smem) {   // all keys identical: any order is sorted
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) s_keys[warp * C::SEG + i * 32 + lane] = key[i];
+        __syncthreads();
+    }
+}
+
+// Solve the sorted values held in s_keys[0..n) (descending scores).
+//   m0      scores above the first value (band: the count at or above a_R)
+//   top     value above c_0 that P_top refers to (a_R, or +inf)
+//   P_top   sum_{scores above} e^{(top - r)/t}
+//   bot     value below c_{n-1} that Q_bot refers to (a_L, or -inf)
+//   Q_bot   sum_{scores below} e^{(r - bot)/t}
+// Returns b in thread 0 (and j_star = index of the last value >= b, -1 if none).
+// Requires n >= 1.
+template <int BLOCK, int KPT>
+__device__ double block_scan_solve(const uint32_t *s_keys, int n, double k, double t, double inv_t,
+                                   double m0, double top, double P_top, double bot, double Q_bot,
+                                   void *scratch_v, int64_t *j_star_out, int32_t *status) {
+    constexpr int R = KPT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    Aff *sc = reinterpret_cast<Aff *>(scratch_v);               // 2*NW Aff
+    int *s_int = reinterpret_cast<int *>(sc + 2 * (BLOCK / 32)); // [0]: r*, [1..NW]: per warp
+    double *s_dbl = reinterpret_cast<double *>(s_int + 40);      // handoff
+
+    auto val = [&](int j) -> double {
+        if (j < 0) return top;
+        if (j >= n) return bot;
+        return (double)desc_key_to_float(s_keys[j]);
+    };
+    // link d_j = e^{(c_{j+1} - c_j)/t}, j in [-1, n-1] (virtual top/bottom at the ends)
+    auto link = [&](int j) -> double {
+        double hi = val(j), lo = val(j + 1);
+        if (hi == CUDART_INF || lo == -CUDART_INF) return 0.0;
+        return exp((lo - hi) * inv_t);
+    };
+
+    const int j0 = tid * R;
+    const int j1 = min(j0 + R, n) - 1;   // run [j0, j1], empty if j1 < j0
+    Aff mp = aff_id(), mq = aff_id();
+    double d_out = 0.0;
+    if (j0 < n) {
+        // P: x -> 1 + d_{j-1} x for j = j0..j1; Q: x -> 1 + d_j x, composed right-to-left
+        double dprev = link(j0 - 1);
+        double cprev = val(j0);
+        for (int j = j0; j <= j1; ++j) {
+            mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
+            double cn = val(j + 1);
+            double d = (cprev == CUDART_INF || cn == -CUDART_INF) ? 0.0 : exp((cn - cprev) * inv_t);
+            // append Q-map of j on the right: T(x) = A(1 + d x) + S
+            mq = {mq.a * d, mq.s + mq.a};
+            dprev = d;
+            cprev = cn;
+        }
+        d_out = dprev;   // d_{j1}
+    }
+    Aff pe, qe;
+    block_scan_excl_both<BLOCK>(mp, mq, pe, qe, sc);
+    const double P_in = fma(pe.a, P_top, pe.s);        // P_{j0-1}
+    const double Q_after = fma(qe.a, Q_bot, qe.s);     // Q_{j1+1}
+    const double P_end = fma(mp.a, P_in, mp.s);        // P_{j1}
+    // G at the run end
+    int cand = -1;
+    if (j0 < n) {
+        double G = (m0 + (double)(j1 + 1)) - 0.5 * P_end + 0.5 * d_out * Q_after;
+        if (G <= k) cand = tid;
+    }
+    // r* = max candidate run
+    cand = warp_max_int(cand);
+    if (lane == 0) s_int[1 + warp] = cand;
+    __syncthreads();
+    if (tid == 0) {
+        int m = -1;
+        for (int w = 0; w < BLOCK / 32; ++w) m = max(m, s_int[1 + w]);
+        s_int[0] = m;
+    }
+    __syncthreads();
+    const int rstar = s_int[0];
+    const int nruns = (n + R - 1) / R;
+    const int rr = rstar + 1;   // run holding the crossing (== nruns: below the last value)
+    if (tid == rr) {
+        s_dbl[0] = P_in;
+        s_dbl[1] = Q_after;
+    }
+    if (rr == nruns && tid == nruns - 1) {   // crossing between c_{n-1} and the bottom
+        s_dbl[0] = P_end;
+    }
+    __syncthreads();
+    double b = 0.0;
+    if (warp == 0) {
+        double U, L, A, PU, QL, ed;
+        int jstar;
+        if (rr >= nruns) {
+            jstar = n - 1;
+            U = val(n - 1);
+            L = bot;
+            A = m0 + n;
+            PU = s_dbl[0];
+            QL = Q_bot;
+            ed = link(n - 1);
+        } else {
+            const int r0 = rr * R;
+            const int cnt = min(R, n - r0);
+            const double Pin = s_dbl[0], Qaft = s_dbl[1];
+            const int j = r0 + lane;
+            const bool act = lane < cnt;
+            double din = act ? link(j - 1) : 1.0;       // d_{j-1}
+            double dj = act ? link(j) : 1.0;            // d_j
+            Aff pm = act ? Aff{din, 1.0} : aff_id();
+            Aff qm = act ? Aff{dj, 1.0} : aff_id();
+            pm = warp_scan_fwd(pm, lane);
+            qm = warp_scan_bwd(qm, lane);
+            double Pj = fma(pm.a, Pin, pm.s);           // P_j
+            double Qj = fma(qm.a, Qaft, qm.s);          // Q_j
+            double Qn = __shfl_down_sync(FULL, Qj, 1);  // Q_{j+1}
+            if (lane == cnt - 1) Qn = Qaft;
+            double G = (m0 + (double)(j + 1)) - 0.5 * Pj + 0.5 * dj * Qn;
+            unsigned bal = __ballot_sync(FULL, act && G <= k);
+            int hl = bal ? 31 - __clz(bal) : -1;         // last lane with G_j <= k
+            double Q0 = __shfl_sync(FULL, Qj, 0);
+            double d0 = __shfl_sync(FULL, din, 0);
+            double Ph = __shfl_sync(FULL, Pj, hl < 0 ? 0 : hl);
+            double Qh = __shfl_sync(FULL, Qn, hl < 0 ? 0 : hl);
+            double dh = __shfl_sync(FULL, dj, hl < 0 ? 0 : hl);
+            if (hl < 0) {   // crossing between c_{r0-1} (or the top) and c_{r0}
+                jstar = r0 - 1;
+                U = val(r0 - 1);
+                L = val(r0);
+                A = m0 + r0;
+                PU = Pin;
+                QL = Q0;
+                ed = d0;
+            } else {
+                jstar = r0 + hl;
+                U = val(jstar);
+                L = val(jstar + 1);
+                A = m0 + jstar + 1;
+                PU = Ph;
+                QL = Qh;
+                ed = dh;
+            }
+        }
+        if (lane == 0) {
+            if (jstar == -1 && U != CUDART_INF) {
+                // G(top) > k: the root lies above the band (bracket missed)
+                if (status) atomicOr(status, ST_NO_ROOT);
+            }
+            if (jstar == n - 1 && L != -CUDART_INF) {
+                double Gb = (m0 + n) - 0.5 * ed * PU + 0.5 * Q_bot;
+                if (Gb < k && status) atomicOr(status, ST_NO_ROOT);
+            }
+            b = solve_interval(U, L, A, PU, QL, ed, k, t);
+            if (j_star_out) *j_star_out = jstar;
+        }
+    }
+    return b;
+}
+
+}  // namespace lapsum

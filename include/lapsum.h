@@ -1,0 +1,186 @@
+/*
+ * lapsum.h -- C ABI of the B200 (sm_100a) Fast LapSum exact-budget soft top-k.
+ *
+ * The operator ("Fast LapSum: Exact Differentiable Top-k at Million Scale",
+ * technical summary section 2.1): for each row of scores r (length n), a
+ * temperature t > 0 and a budget 0 < k < n, find the scalar threshold b with
+ *
+ *     sum_i F((r_i - b)/t) = k,      F = standard Laplace CDF,
+ *
+ * return p_i = F((r_i - b)/t), and give the analytic vector-Jacobian product
+ *
+ *     grad_i = (f_i/t) (g_i - <g,f>/sum f),   f_i = exp(-|r_i - b|/t)/2.
+ *
+ * Two solvers sit behind lapsum_forward (same page, section 2.2, and the
+ * abstract): the full-sort solver (sort, stable prefix/suffix scan, interval
+ * search, closed-form root) and, for long rows, probabilistic bracketing
+ * (kernel-noised sample, binomial order-statistic bracket [a_L, a_R), one
+ * streaming pass folding out-of-band scores into tail sums, a sort of the
+ * band only, a certification pass, and a full-sort fallback when the
+ * certification fails).  Every step runs in this library's CUDA kernels.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are DEVICE memory, owned by the caller, on the
+ *    current CUDA device; rows are contiguous, row-major [rows][n] with row
+ *    stride n elements.  Nothing is retained after the call returns except the
+ *    library's own workspace.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued on it; no entry point synchronises the host except
+ *    lapsum_get_stats / lapsum_profile_read (documented) and the first call on
+ *    a stream, which may allocate the workspace with cudaMalloc.
+ *  - Return value: LAPSUM_OK (0) or a negative LAPSUM_ERR_* code.  Argument
+ *    errors are detected on the host before anything is enqueued.  Errors
+ *    found on the device (non-finite scores, a look-back wait that gave up)
+ *    are reported by lapsum_get_stats.
+ *  - The library keeps one workspace per (device, stream); calls on the same
+ *    stream are ordered, calls on different streams use different
+ *    workspaces.  Not thread-safe for concurrent calls on the same stream.
+ */
+#ifndef LAPSUM_H
+#define LAPSUM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                       /* cudaStream_t == struct CUstream_st* */
+
+#if defined(__GNUC__)
+#define LAPSUM_API __attribute__((visibility("default")))
+#else
+#define LAPSUM_API
+#endif
+
+#define LAPSUM_OK                   0
+#define LAPSUM_ERR_ARG             -1     /* bad size, budget, temperature or null pointer */
+#define LAPSUM_ERR_NONFINITE       -2     /* a score is NaN or +-inf (device-detected)      */
+#define LAPSUM_ERR_ALLOC           -3     /* workspace allocation failed                    */
+#define LAPSUM_ERR_DEVICE_TIMEOUT  -4     /* an inter-block wait gave up (spin cap)         */
+#define LAPSUM_ERR_CUDA            -5     /* a CUDA runtime call failed                     */
+#define LAPSUM_ERR_NO_ROOT         -6     /* solver found no crossing (internal)            */
+
+/* Solver paths */
+#define LAPSUM_PATH_AUTO     0
+#define LAPSUM_PATH_FULLSORT 1
+#define LAPSUM_PATH_BRACKET  2
+
+/*
+ * Tuning of lapsum_forward_ex.  Zero in any field selects its default.
+ *   seed        key of the Philox4x64-10 stream that draws the bracketing
+ *               sample (default 0).
+ *   sample_size s, the number of kernel-noised samples (default
+ *               min(65536, max(4096, 2^floor(log2(n/64))))).
+ *   delta       bracket miss probability bound (default 1e-6).
+ *   band_cap    capacity of the band buffer in scores (default
+ *               max(65536, 4 n (jL - jR + 2)/s), at most n).  A larger band
+ *               fails certification and takes the full-sort fallback.
+ *   spin_cap    polls before an inter-block wait gives up (default 2^20).
+ *   force_path  LAPSUM_PATH_* (default AUTO: bracketing when rows == 1 and
+ *               n >= 2^20, else full sort).
+ */
+typedef struct {
+    uint64_t seed;
+    int64_t  sample_size;
+    double   delta;
+    int64_t  band_cap;
+    int32_t  spin_cap;
+    int32_t  force_path;
+    int32_t  reserved[4];
+} lapsum_options;
+
+/*
+ * Diagnostics of the last lapsum_forward* call on a stream (row 0 for the
+ * batched full-sort path).  Read with lapsum_get_stats.
+ *   path      LAPSUM_PATH_FULLSORT or LAPSUM_PATH_BRACKET
+ *   verdict   bracketing: 1 certified, 0 not certified (fallback ran); -1 n/a
+ *   status    device error bits: 1 non-finite score, 2 wait timeout,
+ *             4 band overflow, 8 no crossing found
+ *   s, jR, jL sample size and order-statistic ranks of the bracket
+ *   a_L, a_R  bracket ends (fp32, rounded outward)
+ *   c_L, c_band, c_R   scores below a_L, in [a_L, a_R), at or above a_R
+ *   S_L, S_R  tail sums sum_{r<a_L} e^{(r-a_L)/t}, sum_{r>=a_R} e^{-(r-a_R)/t}
+ *   G_aL, G_aR  certification values G(a_L), G(a_R)
+ *   b         the threshold of row 0
+ *   sum_p     sum of the fp32 p of row 0, accumulated in fp64
+ */
+typedef struct {
+    int32_t path, verdict, status, fallback;
+    int64_t s, jR, jL;
+    int64_t c_L, c_band, c_R;
+    float   a_L, a_R;
+    double  S_L, S_R;
+    double  G_aL, G_aR;
+    double  b;
+    double  sum_p;
+    int64_t j_star;
+    int64_t reserved[4];
+} lapsum_stats;
+
+/*
+ * Forward: p_out_dev[rows][n] = F((scores - b)/t), b_out_dev[rows] = b (fp64).
+ *   scores_dev  fp32 [rows][n], finite
+ *   rows >= 1, n >= 1, 0 < k < n (real), t > 0 finite
+ *   p_out_dev   fp32 [rows][n] (may not alias scores_dev)
+ *   b_out_dev   fp64 [rows]
+ * Path: "Fast LapSum", technical summary section 2.2 (full-sort solver;
+ * probabilistic bracketing for n > 1e6) and abstract (certification, fallback).
+ */
+LAPSUM_API int lapsum_forward(const float *scores_dev, int64_t rows, int64_t n, double k, double t,
+                   float *p_out_dev, double *b_out_dev, struct CUstream_st *stream);
+
+/* As lapsum_forward, with tuning options (opt may be NULL: defaults). */
+LAPSUM_API int lapsum_forward_ex(const float *scores_dev, int64_t rows, int64_t n, double k, double t,
+                      float *p_out_dev, double *b_out_dev, const lapsum_options *opt,
+                      struct CUstream_st *stream);
+
+/*
+ * Backward (analytic VJP, technical summary section 2.1):
+ *   grad_out_dev[i] = (f_i/t)(g_i - <g,f>/sum f),  f_i = exp(-|scores_i - b|/t)/2,
+ * per row, with b_dev[rows] the thresholds returned by the forward.
+ * Pure function of (scores, b, g).  grad_out_dev may alias g_dev.
+ */
+LAPSUM_API int lapsum_backward(const float *scores_dev, const double *b_dev, const float *g_dev,
+                    int64_t rows, int64_t n, double t, float *grad_out_dev,
+                    struct CUstream_st *stream);
+
+/* Copies the last forward's diagnostics to *out. Synchronises `stream`.
+ * Returns the device error as a LAPSUM_ERR_* code (LAPSUM_OK if none). */
+LAPSUM_API int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream);
+
+/* Static string for a return code. */
+LAPSUM_API const char *lapsum_strerror(int code);
+
+/* Frees every workspace of the current device (synchronises the device). */
+LAPSUM_API int lapsum_release(void);
+
+/*
+ * Per-kernel timing.  lapsum_profile_enable(1) makes every later launch record
+ * a CUDA event pair on its stream; lapsum_profile_read synchronises the device,
+ * folds the pending pairs and copies up to `max` entries (kernel name, number
+ * of launches, total milliseconds) into the arrays; it returns the number of
+ * distinct kernels.  lapsum_profile_enable(0) stops recording; (2) also clears.
+ */
+LAPSUM_API int lapsum_profile_enable(int mode);
+LAPSUM_API int lapsum_profile_read(const char **names, int64_t *launches, double *total_ms, int max);
+
+/*
+ * Plan of the bracketing path for one row of n scores (host only, no device
+ * work): the sample size s, the order-statistic ranks jR, jL and the band
+ * capacity that lapsum_forward_ex would use with `opt` (NULL: defaults).
+ * The ranks follow the binomial bound of the abstract / technical summary
+ * section 2.2 step 1: X = #{y_j > b} ~ Binomial(s, k/n),
+ *   jR = max{j : P(X < j) <= delta/2},  jL = min{j : P(X >= j) <= delta/2}.
+ */
+LAPSUM_API int lapsum_bracket_plan(int64_t n, double k, const lapsum_options *opt, int64_t *s,
+                                   int64_t *jR, int64_t *jL, int64_t *band_cap);
+
+/* Number of kernel launches enqueued by this library since load (a counter). */
+LAPSUM_API int64_t lapsum_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAPSUM_H */

@@ -296,7 +296,7 @@ double orc_ln(double x)
     uint64_t mb = (bits & 0x800FFFFFFFFFFFFFULL) | (0x3FEULL << 52);
     double m;
     memcpy(&m, &mb, sizeof m);
-    if (m < 0.70710678118654752440) { m = m + m; e -= 1; }         /* m in [sqrt(1/2), sqrt(2)) */
+    if (m < 0x1.6a09e667f3bcdp-1) { m = m + m; e -= 1; }           /* m in [sqrt(1/2), sqrt(2)) */
     double s = (m - 1.0) / (m + 1.0);
     double z = s * s;
     double p = 1.0 / 21.0;

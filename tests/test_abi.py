@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds for
+sm_100a, loads, exports every entry point include/lapsum.h declares, rejects
+bad arguments before touching a device, and plans the bracket (sample size,
+binomial ranks, band capacity) exactly as the oracle's restatement does."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lapsum.h")
+
+
+def _lib_path():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("lapsum_build",
+                                                  os.path.join(ROOT, "exact_budget_soft_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return C.CDLL(_lib_path())
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LAPSUM_API\s+[\w\s\*]+?\b(lapsum_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for must in ("lapsum_forward", "lapsum_backward", "lapsum_forward_ex", "lapsum_get_stats"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", _lib_path()]).decode()
+    exported = set(re.findall(r"\sT\s(lapsum_\w+)", out))
+    missing = [s for s in declared_symbols() if s not in exported]
+    assert not missing, missing
+    for s in declared_symbols():
+        assert getattr(lib, s)
+
+
+def test_strerror(lib):
+    lib.lapsum_strerror.restype = C.c_char_p
+    assert lib.lapsum_strerror(0) == b"ok"
+    assert b"argument" in lib.lapsum_strerror(-1)
+
+
+@pytest.mark.parametrize("rows,n,k,t", [(0, 10, 1.0, 1.0), (1, 0, 1.0, 1.0), (1, 10, 0.0, 1.0),
+                                        (1, 10, 10.0, 1.0), (1, 10, 2.0, 0.0), (1, 10, 2.0, -1.0),
+                                        (1, 10, float("nan"), 1.0), (1, 10, 2.0, float("inf"))])
+def test_bad_arguments_rejected_on_host(lib, rows, n, k, t):
+    lib.lapsum_forward.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_double, C.c_double,
+                                   C.c_void_p, C.c_void_p, C.c_void_p]
+    fake = C.c_void_p(0x1000)   # never dereferenced: the check comes first
+    assert lib.lapsum_forward(fake, rows, n, k, t, fake, fake, None) == -1
+    lib.lapsum_backward.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64,
+                                    C.c_double, C.c_void_p, C.c_void_p]
+    if rows < 1 or n < 1 or not (t > 0) or t == float("inf"):
+        assert lib.lapsum_backward(fake, fake, fake, rows, n, t, fake, None) == -1
+
+
+def test_null_pointers_rejected(lib):
+    lib.lapsum_forward.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_double, C.c_double,
+                                   C.c_void_p, C.c_void_p, C.c_void_p]
+    assert lib.lapsum_forward(None, 1, 10, 2.0, 1.0, None, None, None) == -1
+
+
+class Options(C.Structure):
+    _fields_ = [("seed", C.c_uint64), ("sample_size", C.c_int64), ("delta", C.c_double),
+                ("band_cap", C.c_int64), ("spin_cap", C.c_int32), ("force_path", C.c_int32),
+                ("reserved", C.c_int32 * 4)]
+
+
+def _plan(lib, n, k, s=0, delta=0.0):
+    lib.lapsum_bracket_plan.argtypes = [C.c_int64, C.c_double, C.POINTER(Options)] + [C.POINTER(C.c_int64)] * 4
+    o = Options()
+    o.sample_size, o.delta = s, delta
+    out = [C.c_int64() for _ in range(4)]
+    rc = lib.lapsum_bracket_plan(n, k, C.byref(o), *[C.byref(x) for x in out])
+    assert rc == 0
+    return [x.value for x in out]
+
+
+@pytest.mark.parametrize("n,k,s,delta", [(1_048_576, 210, 0, 0.0), (10_000_000, 1e5, 0, 0.0),
+                                         (100_000_000, 1e6, 0, 0.0), (100_000_000, 1e6, 4096, 0.5),
+                                         (5000, 60, 512, 0.2), (3000, 60.0, 512, 0.2),
+                                         (2_000_000, 1.5, 0, 1e-3), (2_000_000, 1999999.0, 0, 1e-9)])
+def test_bracket_plan_matches_oracle_ranks(lib, orc, n, k, s, delta):
+    s_, jR, jL, cap = _plan(lib, n, k, s, delta)
+    if s == 0:
+        pw = 1
+        while pw * 2 <= n // 64:
+            pw *= 2
+        assert s_ == min(65536, max(4096, pw))
+    assert (jR, jL) == orc.binom_ranks(s_, k / n, delta or 1e-6)
+    assert 0 < cap <= n
