@@ -538,7 +538,7 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                  const float *__restrict__ g, int64_t n, double inv_t, const Ctl *ctl,
                  float *__restrict__ grad) {
     const double b = *b_in;
-    const float lam = (float)ctl->vjp_lambda;
+    const double lam = ctl->vjp_lambda;
     const float it = (float)inv_t;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
@@ -551,14 +551,14 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
     for (int64_t i = gtid; i < n4; i += gstride) {
         const float4 v = __ldcs(r4 + i), w = __ldcs(g4 + i);
         float4 o;
-        o.x = 0.5f * expf(-fabsf((float)(((double)v.x - b) * inv_t))) * it * (w.x - lam);
-        o.y = 0.5f * expf(-fabsf((float)(((double)v.y - b) * inv_t))) * it * (w.y - lam);
-        o.z = 0.5f * expf(-fabsf((float)(((double)v.z - b) * inv_t))) * it * (w.z - lam);
-        o.w = 0.5f * expf(-fabsf((float)(((double)v.w - b) * inv_t))) * it * (w.w - lam);
+        o.x = vjp_term(v.x, w.x, b, inv_t, it, lam);
+        o.y = vjp_term(v.y, w.y, b, inv_t, it, lam);
+        o.z = vjp_term(v.z, w.z, b, inv_t, it, lam);
+        o.w = vjp_term(v.w, w.w, b, inv_t, it, lam);
         __stcs(o4 + i, o);
     }
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
-        grad[i] = 0.5f * expf(-fabsf((float)(((double)r[i] - b) * inv_t))) * it * (g[i] - lam);
+        grad[i] = vjp_term(r[i], g[i], b, inv_t, it, lam);
 }
 
 // ============================================================= launchers --

@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(BLOCK)
 rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
               const float *__restrict__ g, int64_t n, double inv_t, float *__restrict__ grad) {
     __shared__ ShiftSum s_ss[BLOCK / 32];
-    __shared__ float s_lam;
+    __shared__ double s_lam;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t off = (int64_t)blockIdx.x * n;
     const float *r = scores + off;
@@ -224,10 +224,10 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
     if (tid == 0) {
         ShiftSum a = s_ss[0];
         for (int w = 1; w < BLOCK / 32; ++w) a = shift_merge(a, s_ss[w]);
-        s_lam = (float)(a.sgf / a.sf);
+        s_lam = a.sgf / a.sf;
     }
     __syncthreads();
-    const float lam = s_lam;
+    const double lam = s_lam;
     const float it = (float)inv_t;
     if (vec) {
         const float4 *r4 = reinterpret_cast<const float4 *>(r);
@@ -235,15 +235,15 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
         float4 *o4 = reinterpret_cast<float4 *>(out);
         for (int64_t i = tid; i < n / 4; i += BLOCK) {
             float4 v = r4[i], w = g4[i], o;
-            o.x = 0.5f * expf(-fabsf((float)(((double)v.x - b) * inv_t))) * it * (w.x - lam);
-            o.y = 0.5f * expf(-fabsf((float)(((double)v.y - b) * inv_t))) * it * (w.y - lam);
-            o.z = 0.5f * expf(-fabsf((float)(((double)v.z - b) * inv_t))) * it * (w.z - lam);
-            o.w = 0.5f * expf(-fabsf((float)(((double)v.w - b) * inv_t))) * it * (w.w - lam);
+            o.x = vjp_term(v.x, w.x, b, inv_t, it, lam);
+            o.y = vjp_term(v.y, w.y, b, inv_t, it, lam);
+            o.z = vjp_term(v.z, w.z, b, inv_t, it, lam);
+            o.w = vjp_term(v.w, w.w, b, inv_t, it, lam);
             o4[i] = o;
         }
     } else {
         for (int64_t i = tid; i < n; i += BLOCK)
-            out[i] = 0.5f * expf(-fabsf((float)(((double)r[i] - b) * inv_t))) * it * (gg[i] - lam);
+            out[i] = vjp_term(r[i], gg[i], b, inv_t, it, lam);
     }
 }
 

@@ -192,6 +192,15 @@ __device__ __forceinline__ float laplace_cdf_f(float x) {
     return x < 0.0f ? e : 1.0f - e;
 }
 
+// One VJP output, (f/t)(g - lambda) with f = e^{-|x|}/2.  g - lambda is formed in
+// fp64: when a few scores carry almost all of sum f, lambda sits within an fp32
+// ulp of their g and the difference would cancel.
+__device__ __forceinline__ float vjp_term(float r, float g, double b, double inv_t, float it,
+                                          double lam) {
+    const float f = 0.5f * expf(-fabsf((float)(((double)r - b) * inv_t)));
+    return (float)((double)(f * it) * ((double)g - lam));
+}
+
 // ------------------------------------------------ bounded device waits --
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
     unsigned long long v;
