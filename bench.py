@@ -49,56 +49,54 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled every few ms (NVML, read-only) in a
+    background thread while the timed region runs."""
+    HW_SLOWDOWN, SW_THERMAL, HW_THERMAL, SW_POWER = 0x8, 0x20, 0x40, 0x4
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines: list[str] = []
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples: list[tuple[float, int]] = []
+        self.max_mhz = None
+        self.ok = False
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception:
+            return self
+        self.stop = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        if self.ok:
+            self.stop.set()
+            self.t.join(timeout=2)
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        names = {self.HW_SLOWDOWN: "hw_slowdown", self.HW_THERMAL: "hw_thermal_slowdown",
+                 self.SW_THERMAL: "sw_thermal_slowdown", self.SW_POWER: "sw_power_cap"}
+        reasons = sorted({nm for _, rs in self.samples for bit, nm in names.items() if rs & bit})
+        sm = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": "NVML" if self.ok else "unavailable"}
 
 
 def dist_setup(n_gpus: int):
@@ -134,6 +132,9 @@ def run_ours(args):
     import exact_budget_soft_b200 as L
 
     w = W.WORKLOADS[args.workload]
+    if args.scale_n:
+        # same distribution and budget fraction at another length (profiling runs)
+        w = W.Workload(f"{w.name}@n={args.scale_n}", 1, args.scale_n, w.k * args.scale_n / w.n, w.t, w.dist, w.path)
     r_np = W.scores(w, seed=rank)[0]
     g_np = W.upstream_grad(w, seed=rank)[0]
     r = torch.from_numpy(r_np).cuda()
@@ -192,7 +193,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(tot / args.steps, 4), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32 (f64 threshold, sums and near-threshold exps)",
         "data": "synthetic (seeded numpy: 256 levels of U(-4,4) sorted descending; g ~ N(0,1))",
-        "config": {"workload": f"{w.name}: 1 row x n=1e8 fp32, k=1e6, t=0.1",
+        "config": {"workload": f"{w.name}: 1 row x n={w.n:.0e} fp32, k={w.k:g}, t={w.t:g}",
                    "l2": "inputs (r, g: 800 MB) larger than the 126 MB L2; no flush",
                    "parallelism": f"replicas x{world} (one row per GPU, no data exchange)"},
         "fwd_ms": round(med_f, 4),
@@ -315,6 +316,7 @@ def main():
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--scale-n", type=int, default=0, help="profiling: same workload at another n")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -139,7 +139,13 @@ __global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
     const double E = -sample_ln(U);
     const double L = (x1 & 1ull) ? E : -E;
     const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
-    P.keys[j] = desc_key(__double2float_rd(y));
+    const uint32_t key = desc_key(__double2float_rd(y));
+    P.keys[j] = key;
+    // first radix-select round: histogram of the top 12 key bits (warp-aggregated)
+    const uint32_t bin = key >> 20;
+    const unsigned act = __activemask();
+    const unsigned peers = __match_any_sync(act, bin);
+    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
 }
 
 // ================================================================ select --
@@ -173,50 +179,64 @@ __device__ __forceinline__ uint32_t block_incl_scan_u32(uint32_t v, uint32_t *s_
     return r;
 }
 
+constexpr int SEL_CAND = 8192;   // candidates per target kept in shared memory
+constexpr size_t SEL_SMEM = (2 * 4096 + 2 * SEL_CAND) * sizeof(uint32_t);
+
 __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
-    __shared__ uint32_t hist[2][4096];
+    extern __shared__ __align__(16) unsigned char sel_smem[];
+    uint32_t (*hist)[4096] = reinterpret_cast<uint32_t (*)[4096]>(sel_smem);
+    uint32_t (*cand)[SEL_CAND] = reinterpret_cast<uint32_t (*)[SEL_CAND]>(sel_smem + 2 * 4096 * sizeof(uint32_t));
     __shared__ uint32_t s_w[32];
-    __shared__ uint32_t s_pref[2], s_rank[2];
-    const int tid = threadIdx.x, lane = tid & 31;
+    __shared__ uint32_t s_pref[2], s_rank[2], s_cnt[2];
+    const int tid = threadIdx.x;
     const int s = (int)P.s;
-    const bool valid0 = P.jR >= 1, valid1 = P.jL <= P.s;
+    const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
     if (tid == 0) {
         s_pref[0] = 0; s_pref[1] = 0;
-        s_rank[0] = (uint32_t)(valid0 ? P.jR : 1);
-        s_rank[1] = (uint32_t)(valid1 ? P.jL : 1);
+        s_rank[0] = (uint32_t)(valid[0] ? P.jR : 1);
+        s_rank[1] = (uint32_t)(valid[1] ? P.jL : 1);
+        s_cnt[0] = 0; s_cnt[1] = 0;
     }
+    // round 1 (bits 31..20): histogram built by the sample kernel; rearm it
+    for (int i = tid; i < 4096; i += 1024) {
+        hist[0][i] = P.hist1[i];
+        P.hist1[i] = 0u;
+    }
+    __syncthreads();
     uint32_t mask = 0;
     const int shifts[3] = {20, 8, 0};
     const int widths[3] = {12, 12, 8};
+    bool fast[2] = {false, false};
 #pragma unroll 1
     for (int rd = 0; rd < 3; ++rd) {
         const int sh = shifts[rd];
         const uint32_t bm = (1u << widths[rd]) - 1u;
         const int nb = 1 << widths[rd];
-        for (int i = tid; i < 2 * 4096; i += 1024) (&hist[0][0])[i] = 0;
-        __syncthreads();
-        const uint32_t p0 = s_pref[0], p1 = s_pref[1];
-        for (int i0 = 0; i0 < s; i0 += 1024) {
-            const int i = i0 + tid;
-            const bool in = i < s;
-            const uint32_t key = in ? P.keys[i] : 0u;
-            const uint32_t bin = (key >> sh) & bm;
+        if (rd > 0) {
+            for (int i = tid; i < 2 * 4096; i += 1024) (&hist[0][0])[i] = 0;
+            __syncthreads();
+            const uint32_t pf[2] = {s_pref[0], s_pref[1]};
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                if (rd == 0 && q == 1) break;                       // shared first round
-                const bool m = in && (rd == 0 ? (valid0 || valid1)
-                                              : ((key & mask) == (q ? p1 : p0)) && (q ? valid1 : valid0));
-                const unsigned act = __ballot_sync(FULL, m);
-                if (!act) continue;
-                const unsigned peers = __match_any_sync(FULL, m ? bin : 0xffffffffu) & act;
-                if (m && lane == __ffs(peers) - 1) atomicAdd(&hist[q][bin], (uint32_t)__popc(peers));
+                if (!valid[q]) continue;
+                if (fast[q]) {
+                    const int c = (int)s_cnt[q];
+                    for (int i = tid; i < c; i += 1024) {
+                        const uint32_t key = cand[q][i];
+                        if ((key & mask) == pf[q]) atomicAdd(&hist[q][(key >> sh) & bm], 1u);
+                    }
+                } else {
+                    for (int i = tid; i < s; i += 1024) {
+                        const uint32_t key = P.keys[i];
+                        if ((key & mask) == pf[q]) atomicAdd(&hist[q][(key >> sh) & bm], 1u);
+                    }
+                }
             }
+            __syncthreads();
         }
-        __syncthreads();
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
             const uint32_t *h = (rd == 0) ? hist[0] : hist[q];
-            // thread tid owns bins [4 tid, 4 tid + 4)
             uint32_t c[4], loc = 0;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -227,9 +247,8 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
             const uint32_t inc = block_incl_scan_u32(loc, s_w);
             const uint32_t ex = inc - loc;
             const uint32_t want = s_rank[q];
-            const bool vq = q ? valid1 : valid0;
             __syncthreads();
-            if (vq && ex < want && want <= inc) {
+            if (valid[q] && ex < want && want <= inc) {
                 uint32_t cum = ex;
                 for (int u = 0; u < 4; ++u) {
                     if (cum + c[u] >= want) {
@@ -243,13 +262,30 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
             __syncthreads();
         }
         mask |= bm << sh;
+        if (rd == 0) {
+            // keep the keys under each target's 12-bit prefix in shared memory
+            const uint32_t pf[2] = {s_pref[0], s_pref[1]};
+            for (int i = tid; i < s; i += 1024) {
+                const uint32_t key = P.keys[i];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    if (valid[q] && (key & mask) == pf[q]) {
+                        const uint32_t pos = atomicAdd(&s_cnt[q], 1u);
+                        if (pos < SEL_CAND) cand[q][pos] = key;
+                    }
+                }
+            }
+            __syncthreads();
+            fast[0] = s_cnt[0] <= SEL_CAND;
+            fast[1] = s_cnt[1] <= SEL_CAND;
+        }
     }
     if (tid == 0) {
         Ctl *c = P.ctl;
         const float yR = desc_key_to_float(s_pref[0]);
         const float yL = desc_key_to_float(s_pref[1]);
-        c->a_R = valid0 ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
-        c->a_L = valid1 ? yL : -CUDART_INF_F;
+        c->a_R = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
+        c->a_L = valid[1] ? yL : -CUDART_INF_F;
         c->jR = P.jR;
         c->jL = P.jL;
         c->s = P.s;
@@ -260,74 +296,92 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
 
 // ================================================================ stream --
 struct StreamAcc {
-    unsigned long long cL, cR;
-    double SL, SR;
+    uint32_t cL, cR;
+    double SL, SR;      // near terms (fp64)
+    float SL2, SR2;     // far terms (fp32)
     bool bad;
 };
-
-__device__ __forceinline__ double tier_term(double z) {
-    return z <= EXP_TIER ? exp(-z) : (z < 104.0 ? (double)expf(-(float)z) : 0.0);
-}
+struct Ends {
+    float aL, aR, itf;
+    double daL, daR, inv_t;
+};
 
 // One score of the streaming pass (technical summary section 2.2, step 2):
 // at or above a_R -> count, S_R += e^{-(r-a_R)/t}; below a_L -> count,
-// S_L += e^{(r-a_L)/t}; otherwise append to the band (warp-aggregated slot).
-__device__ __forceinline__ void stream_one(float x, bool valid, float aL, float aR, double daL,
-                                           double daR, double inv_t, StreamAcc &acc, float *band,
-                                           unsigned long long cap, unsigned long long *band_ctr,
-                                           int lane) {
-    const bool above = valid && x >= aR;
-    const bool below = valid && x < aL;
-    const bool inb = valid && x >= aL && x < aR;
+// S_L += e^{(r-a_L)/t}; returns whether it belongs to the band [a_L, a_R).
+__device__ __forceinline__ bool stream_one(float x, bool valid, const Ends &E, StreamAcc &acc) {
+    const bool above = valid && x >= E.aR;
+    const bool below = valid && x < E.aL;
     acc.bad |= valid && !isfinite(x);
-    if (above || below) {
-        const double z = above ? ((double)x - daR) * inv_t : (daL - (double)x) * inv_t;
-        const double e = tier_term(z);
-        if (above) { acc.cR += 1; acc.SR += e; }
-        else       { acc.cL += 1; acc.SL += e; }
+    if (above) {
+        acc.cR += 1;
+        tier_add(x, E.aR, (double)x, E.daR, E.itf, E.inv_t, acc.SR, acc.SR2);
+    } else if (below) {
+        acc.cL += 1;
+        tier_add(E.aL, x, E.daL, (double)x, E.itf, E.inv_t, acc.SL, acc.SL2);
     }
+    return valid && !above && !below && x == x;
+}
+
+// Append a band score at a warp-aggregated slot of the band buffer (the count
+// keeps going past the capacity so the overflow is visible).
+__device__ __forceinline__ void band_push(float x, bool inb, float *band, unsigned long long cap,
+                                          unsigned long long *ctr, int lane) {
     const unsigned m = __ballot_sync(FULL, inb);
-    if (m) {
-        const int leader = __ffs(m) - 1;
-        unsigned long long base = 0;
-        if (lane == leader) base = atomicAdd(band_ctr, (unsigned long long)__popc(m));
-        base = __shfl_sync(FULL, base, leader) + __popc(m & ((1u << lane) - 1u));
-        if (inb && base < cap) band[base] = x;
-    }
+    if (!m) return;
+    const int leader = __ffs(m) - 1;
+    unsigned long long base = 0;
+    if (lane == leader) base = atomicAdd(ctr, (unsigned long long)__popc(m));
+    base = __shfl_sync(FULL, base, leader) + __popc(m & ((1u << lane) - 1u));
+    if (inb && base < cap) band[base] = x;
 }
 
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) stream_kernel(BracketParams P) {
     __shared__ double s_red[4 * (SBLOCK / 32)];
     Ctl *ctl = P.ctl;
-    const float aL = ctl->a_L, aR = ctl->a_R;
-    const double daL = aL, daR = aR, inv_t = P.inv_t;
+    Ends E;
+    E.aL = ctl->a_L;
+    E.aR = ctl->a_R;
+    E.daL = E.aL;
+    E.daR = E.aR;
+    E.inv_t = P.inv_t;
+    E.itf = (float)P.inv_t;
     const int lane = threadIdx.x & 31;
     const unsigned long long cap = (unsigned long long)P.band_cap;
-    StreamAcc acc{0, 0, 0.0, 0.0, false};
+    unsigned long long *ctr = &ctl->c_band;
+    StreamAcc acc{0, 0, 0.0, 0.0, 0.f, 0.f, false};
     const int64_t n = P.n;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
     const int64_t n4 = aligned ? n / 4 : 0;
     const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
-    // whole warps iterate together (the ballot needs every lane)
+    // whole warps iterate together (the ballots need every lane)
     const int64_t n4w = (n4 + gstride - 1) / gstride * gstride;
     for (int64_t i = gtid; i < n4w; i += gstride) {
         const bool ok = i < n4;
-        float4 v = ok ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        stream_one(v.x, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
-        stream_one(v.y, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
-        stream_one(v.z, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
-        stream_one(v.w, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+        const float4 v = ok ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool b0 = stream_one(v.x, ok, E, acc);
+        const bool b1 = stream_one(v.y, ok, E, acc);
+        const bool b2 = stream_one(v.z, ok, E, acc);
+        const bool b3 = stream_one(v.w, ok, E, acc);
+        if (__any_sync(FULL, b0 | b1 | b2 | b3)) {
+            band_push(v.x, b0, P.band, cap, ctr, lane);
+            band_push(v.y, b1, P.band, cap, ctr, lane);
+            band_push(v.z, b2, P.band, cap, ctr, lane);
+            band_push(v.w, b3, P.band, cap, ctr, lane);
+        }
     }
     const int64_t rem0 = n4 * 4;
     const int64_t remw = rem0 + ((n - rem0 + gstride - 1) / gstride) * gstride;
     for (int64_t i = rem0 + gtid; i < remw; i += gstride) {
         const bool ok = i < n;
-        stream_one(ok ? P.r[i] : 0.f, ok, aL, aR, daL, daR, inv_t, acc, P.band, cap, &ctl->c_band, lane);
+        const float x = ok ? P.r[i] : 0.f;
+        const bool bb = stream_one(x, ok, E, acc);
+        band_push(x, bb, P.band, cap, ctr, lane);
     }
     if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
-    double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL, acc.SR};
+    double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2};
     block_sum<SBLOCK, 4>(v, s_red);
     if (last_block_sum<SBLOCK, 4>(v, P.partials, &ctl->ticket[0], s_red) && threadIdx.x == 0) {
         ctl->c_L = (unsigned long long)v[0];
@@ -346,57 +400,64 @@ __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) stream_kernel(BracketP
 // mirror image below), band scores take two.  Verdict: G(a_L) >= k > G(a_R),
 // the band fits its buffer, and both passes agree on every membership count.
 struct CertAcc {
-    unsigned long long cntL, cntR, cntB;   // >= a_L, >= a_R, < a_L
-    double above, below, hiLband, loRband;
+    uint32_t cntL, cntR, cntB;   // >= a_L, >= a_R, < a_L
+    double above, below, hiL, loR;
+    float above2, below2, hiL2, loR2;
     bool bad;
 };
 
-__device__ __forceinline__ void cert_one(float x, bool valid, float aL, float aR, double daL,
-                                         double daR, double inv_t, CertAcc &a) {
-    if (!valid) return;
+__device__ __forceinline__ void cert_one(float x, const Ends &E, CertAcc &a) {
     a.bad |= !isfinite(x);
-    if (x >= aR) {
+    if (x >= E.aR) {
         a.cntR += 1;
         a.cntL += 1;
-        a.above += tier_term(((double)x - daR) * inv_t);
-    } else if (x >= aL) {
+        tier_add(x, E.aR, (double)x, E.daR, E.itf, E.inv_t, a.above, a.above2);
+    } else if (x >= E.aL) {
         a.cntL += 1;
-        a.hiLband += tier_term(((double)x - daL) * inv_t);
-        a.loRband += tier_term((daR - (double)x) * inv_t);
-    } else if (x < aL) {
+        tier_add(x, E.aL, (double)x, E.daL, E.itf, E.inv_t, a.hiL, a.hiL2);
+        tier_add(E.aR, x, E.daR, (double)x, E.itf, E.inv_t, a.loR, a.loR2);
+    } else if (x < E.aL) {
         a.cntB += 1;
-        a.below += tier_term((daL - (double)x) * inv_t);
+        tier_add(E.aL, x, E.daL, (double)x, E.itf, E.inv_t, a.below, a.below2);
     }
 }
 
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) certify_kernel(BracketParams P) {
     __shared__ double s_red[7 * (SBLOCK / 32)];
     Ctl *ctl = P.ctl;
-    const float aL = ctl->a_L, aR = ctl->a_R;
-    const double daL = aL, daR = aR, inv_t = P.inv_t;
-    CertAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, false};
+    Ends E;
+    E.aL = ctl->a_L;
+    E.aR = ctl->a_R;
+    E.daL = E.aL;
+    E.daR = E.aR;
+    E.inv_t = P.inv_t;
+    E.itf = (float)P.inv_t;
+    CertAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
     const int64_t n = P.n;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
     const int64_t n4 = aligned ? n / 4 : 0;
     const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
+    // the second pass walks the row from the end, so it starts on the part the
+    // streaming pass left in L2
     for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = r4[i];
-        cert_one(v.x, true, aL, aR, daL, daR, inv_t, acc);
-        cert_one(v.y, true, aL, aR, daL, daR, inv_t, acc);
-        cert_one(v.z, true, aL, aR, daL, daR, inv_t, acc);
-        cert_one(v.w, true, aL, aR, daL, daR, inv_t, acc);
+        const float4 v = r4[n4 - 1 - i];
+        cert_one(v.x, E, acc);
+        cert_one(v.y, E, acc);
+        cert_one(v.z, E, acc);
+        cert_one(v.w, E, acc);
     }
-    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) cert_one(P.r[i], true, aL, aR, daL, daR, inv_t, acc);
+    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) cert_one(P.r[i], E, acc);
     if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
-    double v[7] = {(double)acc.cntL, (double)acc.cntR, (double)acc.cntB, acc.above,
-                   acc.below, acc.hiLband, acc.loRband};
+    double v[7] = {(double)acc.cntL, (double)acc.cntR, (double)acc.cntB,
+                   acc.above + (double)acc.above2, acc.below + (double)acc.below2,
+                   acc.hiL + (double)acc.hiL2, acc.loR + (double)acc.loR2};
     block_sum<SBLOCK, 7>(v, s_red);
     if (last_block_sum<SBLOCK, 7>(v, P.partials + 8 * (size_t)gridDim.x, &ctl->ticket[1], s_red) &&
         threadIdx.x == 0) {
         const double cntL = v[0], cntR = v[1], cntB = v[2];
-        const double rho = (aR == CUDART_INF_F || aL == -CUDART_INF_F) ? 0.0 : exp(-(daR - daL) * inv_t);
+        const double rho = (E.aR == CUDART_INF_F || E.aL == -CUDART_INF_F) ? 0.0 : exp(-(E.daR - E.daL) * E.inv_t);
         const double GaL = cntL - 0.5 * fma(rho, v[3], v[5]) + 0.5 * v[4];
         const double GaR = cntR - 0.5 * v[3] + 0.5 * fma(rho, v[4], v[6]);
         ctl->G_aL = GaL;
@@ -413,11 +474,14 @@ __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) certify_kernel(Bracket
 }
 
 // ================================================================= p pass --
+// p = F((r - b)/t), walking forward (the certification pass left the head of
+// the row in L2).  Also sum p (fp64) for the diagnostics.
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict__ p,
          double *__restrict__ b_out, Ctl *ctl, double *partials) {
     __shared__ double s_red[SBLOCK / 32];
     const double b = ctl->b;
+    const XForm xf = make_xform(b, inv_t * LOG2E);
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(p)) & 15) == 0;
@@ -426,17 +490,17 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
     float4 *p4 = reinterpret_cast<float4 *>(p);
     double ps = 0.0;
     for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = __ldcs(r4 + i);
+        const float4 v = r4[i];
         float4 o;
-        o.x = laplace_cdf_f((float)(((double)v.x - b) * inv_t));
-        o.y = laplace_cdf_f((float)(((double)v.y - b) * inv_t));
-        o.z = laplace_cdf_f((float)(((double)v.z - b) * inv_t));
-        o.w = laplace_cdf_f((float)(((double)v.w - b) * inv_t));
+        o.x = laplace_cdf2(xf(v.x));
+        o.y = laplace_cdf2(xf(v.y));
+        o.z = laplace_cdf2(xf(v.z));
+        o.w = laplace_cdf2(xf(v.w));
         ps += ((double)o.x + (double)o.y) + ((double)o.z + (double)o.w);
         __stcs(p4 + i, o);
     }
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
-        const float o = laplace_cdf_f((float)(((double)r[i] - b) * inv_t));
+        const float o = laplace_cdf2(xf(r[i]));
         ps += (double)o;
         p[i] = o;
     }
@@ -450,18 +514,60 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
 }
 
 // =================================================================== VJP --
+// <g,f> and sum f of one long row (walking backward: the p pass left the tail
+// in L2).  Terms are e^{-|x|} in fp32 (denormals kept), summed in fp64.  If
+// every term underflows (all scores farther than ~100 t from b), the last block
+// raises a flag and vjp_shifted_kernel recomputes the ratio from terms shifted
+// by the running minimum of |x| (the shift cancels in <g,f>/sum f).
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
+vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
+                  const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
+    __shared__ double s_red[2 * (SBLOCK / 32)];
+    const double b = *b_in;
+    const XForm xf = make_xform(b, inv_t * LOG2E);
+    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
+    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(g)) & 15) == 0;
+    const int64_t n4 = aligned ? n / 4 : 0;
+    const float4 *r4 = reinterpret_cast<const float4 *>(r);
+    const float4 *g4 = reinterpret_cast<const float4 *>(g);
+    double sf = 0.0, sgf = 0.0;
+    for (int64_t i = gtid; i < n4; i += gstride) {
+        const int64_t j = n4 - 1 - i;
+        const float4 v = r4[j], w = g4[j];
+        const float e0 = exp2f(-fabsf(xf(v.x))), e1 = exp2f(-fabsf(xf(v.y)));
+        const float e2 = exp2f(-fabsf(xf(v.z))), e3 = exp2f(-fabsf(xf(v.w)));
+        sf += ((double)e0 + (double)e1) + ((double)e2 + (double)e3);
+        sgf = fma((double)w.x, (double)e0, sgf);
+        sgf = fma((double)w.y, (double)e1, sgf);
+        sgf = fma((double)w.z, (double)e2, sgf);
+        sgf = fma((double)w.w, (double)e3, sgf);
+    }
+    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
+        const float e = exp2f(-fabsf(xf(r[i])));
+        sf += (double)e;
+        sgf = fma((double)g[i], (double)e, sgf);
+    }
+    double v[2] = {sf, sgf};
+    block_sum<SBLOCK, 2>(v, s_red);
+    if (last_block_sum<SBLOCK, 2>(v, partials, &ctl->ticket[3], s_red) && threadIdx.x == 0) {
+        ctl->vjp_lambda = v[1] / v[0];
+        ctl->vjp_shift = !(v[0] >= 1e-300);
+    }
+}
+
 struct ShiftSumG {
     float m;
     double sf, sgf;
 };
 __device__ __forceinline__ void ss_add(ShiftSumG &s, float ax, float g) {
     if (ax < s.m) {
-        const double sc = (double)expf(ax - s.m);
+        const double sc = (double)exp2f(ax - s.m);
         s.sf *= sc;
         s.sgf *= sc;
         s.m = ax;
     }
-    const double e = (double)expf(s.m - ax);
+    const double e = (double)exp2f(s.m - ax);
     s.sf += e;
     s.sgf = fma((double)g, e, s.sgf);
 }
@@ -470,37 +576,24 @@ __device__ __forceinline__ ShiftSumG ss_merge(ShiftSumG a, ShiftSumG b) {
     if (a.sf == 0.0) return b;
     ShiftSumG r;
     r.m = fminf(a.m, b.m);
-    const double fa = (double)expf(r.m - a.m), fb = (double)expf(r.m - b.m);
+    const double fa = (double)exp2f(r.m - a.m), fb = (double)exp2f(r.m - b.m);
     r.sf = a.sf * fa + b.sf * fb;
     r.sgf = a.sgf * fa + b.sgf * fb;
     return r;
 }
 
-// <g,f> and sum f of one long row, shifted by the running min |x| (the ratio is
-// shift-free); per-block partials merged in block order by the last block.
-__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
-vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
-                  const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
+// Rare path: every f_i underflowed in vjp_reduce_kernel.
+__global__ void __launch_bounds__(SBLOCK)
+vjp_shifted_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
+                   const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
     __shared__ ShiftSumG s_w[SBLOCK / 32];
     __shared__ bool s_last;
+    if (!ctl->vjp_shift) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const double b = *b_in;
-    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + tid;
-    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
-    const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(g)) & 15) == 0;
-    const int64_t n4 = aligned ? n / 4 : 0;
-    const float4 *r4 = reinterpret_cast<const float4 *>(r);
-    const float4 *g4 = reinterpret_cast<const float4 *>(g);
+    const XForm xf = make_xform(*b_in, inv_t * LOG2E);
     ShiftSumG ss{CUDART_INF_F, 0.0, 0.0};
-    for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = __ldcs(r4 + i), w = __ldcs(g4 + i);
-        ss_add(ss, fabsf((float)(((double)v.x - b) * inv_t)), w.x);
-        ss_add(ss, fabsf((float)(((double)v.y - b) * inv_t)), w.y);
-        ss_add(ss, fabsf((float)(((double)v.z - b) * inv_t)), w.z);
-        ss_add(ss, fabsf((float)(((double)v.w - b) * inv_t)), w.w);
-    }
-    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
-        ss_add(ss, fabsf((float)(((double)r[i] - b) * inv_t)), g[i]);
+    for (int64_t i = (int64_t)blockIdx.x * SBLOCK + tid; i < n; i += (int64_t)gridDim.x * SBLOCK)
+        ss_add(ss, fabsf(xf(r[i])), g[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         ShiftSumG q{__shfl_xor_sync(FULL, ss.m, o), __shfl_xor_sync(FULL, ss.sf, o),
@@ -517,7 +610,7 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
         partials[G + blockIdx.x] = a.sf;
         partials[2 * G + blockIdx.x] = a.sgf;
         __threadfence();
-        s_last = atomicAdd(&ctl->ticket[3], 1u) == (unsigned)G - 1;
+        s_last = atomicAdd(&ctl->ticket[7], 1u) == (unsigned)G - 1;
     }
     __syncthreads();
     if (!s_last) return;
@@ -529,7 +622,7 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
             a = ss_merge(a, q);
         }
         ctl->vjp_lambda = a.sgf / a.sf;
-        ctl->ticket[3] = 0u;
+        ctl->ticket[7] = 0u;
     }
 }
 
@@ -537,9 +630,10 @@ __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                  const float *__restrict__ g, int64_t n, double inv_t, const Ctl *ctl,
                  float *__restrict__ grad) {
-    const double b = *b_in;
+    const XForm xf = make_xform(*b_in, inv_t * LOG2E);
     const double lam = ctl->vjp_lambda;
-    const float it = (float)inv_t;
+    const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
+    const float hit = (float)(0.5 * inv_t);
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(g) |
@@ -549,16 +643,16 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
     const float4 *g4 = reinterpret_cast<const float4 *>(g);
     float4 *o4 = reinterpret_cast<float4 *>(grad);
     for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = __ldcs(r4 + i), w = __ldcs(g4 + i);
+        const float4 v = r4[i], w = g4[i];
         float4 o;
-        o.x = vjp_term(v.x, w.x, b, inv_t, it, lam);
-        o.y = vjp_term(v.y, w.y, b, inv_t, it, lam);
-        o.z = vjp_term(v.z, w.z, b, inv_t, it, lam);
-        o.w = vjp_term(v.w, w.w, b, inv_t, it, lam);
+        o.x = vjp_term2(xf(v.x), w.x, hit, lam_hi, lam_lo);
+        o.y = vjp_term2(xf(v.y), w.y, hit, lam_hi, lam_lo);
+        o.z = vjp_term2(xf(v.z), w.z, hit, lam_hi, lam_lo);
+        o.w = vjp_term2(xf(v.w), w.w, hit, lam_hi, lam_lo);
         __stcs(o4 + i, o);
     }
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
-        grad[i] = vjp_term(r[i], g[i], b, inv_t, it, lam);
+        grad[i] = vjp_term2(xf(r[i]), g[i], hit, lam_hi, lam_lo);
 }
 
 // ============================================================= launchers --
@@ -568,7 +662,14 @@ cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
     return cudaGetLastError();
 }
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
-    select_kernel<<<1, 1024, 0, st>>>(P);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SEL_SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    select_kernel<<<1, 1024, SEL_SMEM, st>>>(P);
     return cudaGetLastError();
 }
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
@@ -587,6 +688,9 @@ cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double 
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st) {
     vjp_reduce_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    vjp_shifted_kernel<<<stream_grid() / SBLOCKS_PER_SM, SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, partials);
     return cudaGetLastError();
 }
 cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,

@@ -149,14 +149,16 @@ __global__ void __launch_bounds__(RB, 1) radix_pass_kernel(SortArgs A, int pass,
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sh = 8 * pass;
     const int64_t ntiles = (n + RTILE - 1) / RTILE;
-    if (tid == 0) {
-        s_tile = (int)atomicAdd(&ctl->tile_ctr[pass], 1u);
-        s_cur = ctl->sort_cur;
-    }
+    if (tid == 0) s_cur = ctl->sort_cur;
     __syncthreads();
-    const int tile = s_tile;
     const int cur = s_cur;
-    if (tile < ntiles) {
+    // persistent: tiles are claimed in order from one counter, so a tile only
+    // ever waits on tiles already claimed by running CTAs
+    for (;;) {
+        if (tid == 0) s_tile = (int)atomicAdd(&ctl->tile_ctr[pass], 1u);
+        __syncthreads();
+        const int tile = s_tile;
+        if (tile >= ntiles) break;
         const uint32_t *src = cur >= 0 ? A.keys[cur] : nullptr;
         uint32_t *dst = A.keys[cur >= 0 ? (cur ^ 1) : 0];
         const int64_t base = (int64_t)tile * RTILE;
@@ -258,6 +260,7 @@ __global__ void __launch_bounds__(RB, 1) radix_pass_kernel(SortArgs A, int pass,
             const uint32_t kk = s_keys[i];
             dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
         }
+        __syncthreads();
     }
     // the last CTA to finish publishes the new key buffer and rearms the counters
     __threadfence();
@@ -312,8 +315,7 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
         if (j >= n) return bot;
         return sorted_val(A, cur, j);
     };
-    const int64_t tile = blockIdx.x;
-    if (tile < ntiles) {
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int64_t j0 = tile * LTILE + (int64_t)tid * LK;
         const int64_t j1 = min(j0 + LK, n) - 1;
         Aff mp = aff_id(), mq = aff_id();
@@ -452,13 +454,15 @@ cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) 
         attr = true;
     }
     int64_t hg = (cap + HB * 16 - 1) / (HB * 16);
-    if (hg > (int64_t)num_sms() * 8) hg = (int64_t)num_sms() * 8;
+    if (hg > (int64_t)num_sms() * 2) hg = (int64_t)num_sms() * 2;
     int hgrid = (int)hg;
     if (hgrid < 1) hgrid = 1;
     radix_hist_kernel<<<hgrid, HB, 0, st>>>(A);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const unsigned ptiles = (unsigned)((cap + RTILE - 1) / RTILE);
+    int64_t pt = (cap + RTILE - 1) / RTILE;
+    if (pt > num_sms()) pt = num_sms();   // persistent: one CTA per SM claims tiles in order
+    const unsigned ptiles = (unsigned)pt;
     for (int pass = 0; pass < 4; ++pass) {
         radix_pass_kernel<<<ptiles, RB, smem, st>>>(A, pass, A.epoch * 4u + (uint32_t)pass);
         e = cudaGetLastError();
@@ -476,7 +480,9 @@ cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    const unsigned grid = (unsigned)((A.cap + LTILE - 1) / LTILE);
+    int64_t lg = (A.cap + LTILE - 1) / LTILE;
+    if (lg > num_sms()) lg = num_sms();
+    const unsigned grid = (unsigned)lg;
     locate_kernel<<<grid, LB, smem, st>>>(A, k, t, 1.0 / t);
     return cudaGetLastError();
 }

@@ -120,6 +120,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
 
     // ---- p = F((r - b)/t) for the row
     b = s_b;
+    const XForm xf = make_xform(b, inv_t * LOG2E);
     float *prow = p_out + (int64_t)blockIdx.x * n_arg;
     const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(row) & 15) == 0) &&
                      ((reinterpret_cast<uintptr_t>(prow) & 15) == 0);
@@ -129,16 +130,16 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
         float4 *p4 = reinterpret_cast<float4 *>(prow);
         for (int i = tid; i < n / 4; i += BLOCK) {
             float4 v = r4[i], o;
-            o.x = laplace_cdf_f((float)(((double)v.x - b) * inv_t));
-            o.y = laplace_cdf_f((float)(((double)v.y - b) * inv_t));
-            o.z = laplace_cdf_f((float)(((double)v.z - b) * inv_t));
-            o.w = laplace_cdf_f((float)(((double)v.w - b) * inv_t));
+            o.x = laplace_cdf2(xf(v.x));
+            o.y = laplace_cdf2(xf(v.y));
+            o.z = laplace_cdf2(xf(v.z));
+            o.w = laplace_cdf2(xf(v.w));
             psum += ((double)o.x + (double)o.y) + ((double)o.z + (double)o.w);
             p4[i] = o;
         }
     } else {
         for (int i = tid; i < n; i += BLOCK) {
-            float o = laplace_cdf_f((float)(((double)row[i] - b) * inv_t));
+            float o = laplace_cdf2(xf(row[i]));
             psum += (double)o;
             prow[i] = o;
         }
@@ -154,6 +155,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
 // Per-row analytic VJP (technical summary section 2.1):
 //   grad_i = (f_i/t)(g_i - lambda),  lambda = <g,f>/sum f,  f_i = e^{-|x_i|}/2.
 // lambda is accumulated from terms shifted by the running minimum of |x|
+// (in base-2 units, x log2 e)
 // (the shift cancels in the ratio), so it stays defined when every f_i
 // underflows.  Sums in fp64 with a fixed-order block combine.  The second
 // sweep re-reads the row from L2.
@@ -163,12 +165,12 @@ struct ShiftSum {
 };
 __device__ __forceinline__ void shift_add(ShiftSum &s, float ax, float g) {
     if (ax < s.m) {
-        double sc = (double)expf(ax - s.m);   // 0 when s.m = +inf
+        double sc = (double)exp2f(ax - s.m);   // 0 when s.m = +inf
         s.sf *= sc;
         s.sgf *= sc;
         s.m = ax;
     }
-    double e = (double)expf(s.m - ax);
+    double e = (double)exp2f(s.m - ax);
     s.sf += e;
     s.sgf = fma((double)g, e, s.sgf);
 }
@@ -177,7 +179,7 @@ __device__ __forceinline__ ShiftSum shift_merge(ShiftSum a, ShiftSum b) {
     if (a.sf == 0.0) return b;
     ShiftSum r;
     r.m = fminf(a.m, b.m);
-    double fa = (double)expf(r.m - a.m), fb = (double)expf(r.m - b.m);
+    double fa = (double)exp2f(r.m - a.m), fb = (double)exp2f(r.m - b.m);
     r.sf = a.sf * fa + b.sf * fb;
     r.sgf = a.sgf * fa + b.sgf * fb;
     return r;
@@ -198,7 +200,7 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
     const float *r = scores + off;
     const float *gg = g + off;
     float *out = grad + off;
-    const double b = b_in[blockIdx.x];
+    const XForm xf = make_xform(b_in[blockIdx.x], inv_t * LOG2E);
     const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(r) & 15) == 0) &&
                      ((reinterpret_cast<uintptr_t>(gg) & 15) == 0) &&
                      ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
@@ -208,14 +210,13 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
         const float4 *g4 = reinterpret_cast<const float4 *>(gg);
         for (int64_t i = tid; i < n / 4; i += BLOCK) {
             float4 v = r4[i], w = g4[i];
-            shift_add(ss, fabsf((float)(((double)v.x - b) * inv_t)), w.x);
-            shift_add(ss, fabsf((float)(((double)v.y - b) * inv_t)), w.y);
-            shift_add(ss, fabsf((float)(((double)v.z - b) * inv_t)), w.z);
-            shift_add(ss, fabsf((float)(((double)v.w - b) * inv_t)), w.w);
+            shift_add(ss, fabsf(xf(v.x)), w.x);
+            shift_add(ss, fabsf(xf(v.y)), w.y);
+            shift_add(ss, fabsf(xf(v.z)), w.z);
+            shift_add(ss, fabsf(xf(v.w)), w.w);
         }
     } else {
-        for (int64_t i = tid; i < n; i += BLOCK)
-            shift_add(ss, fabsf((float)(((double)r[i] - b) * inv_t)), gg[i]);
+        for (int64_t i = tid; i < n; i += BLOCK) shift_add(ss, fabsf(xf(r[i])), gg[i]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss = shift_merge(ss, shfl_xor_ss(ss, o));
@@ -228,22 +229,22 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
     }
     __syncthreads();
     const double lam = s_lam;
-    const float it = (float)inv_t;
+    const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
+    const float hit = (float)(0.5 * inv_t);
     if (vec) {
         const float4 *r4 = reinterpret_cast<const float4 *>(r);
         const float4 *g4 = reinterpret_cast<const float4 *>(gg);
         float4 *o4 = reinterpret_cast<float4 *>(out);
         for (int64_t i = tid; i < n / 4; i += BLOCK) {
             float4 v = r4[i], w = g4[i], o;
-            o.x = vjp_term(v.x, w.x, b, inv_t, it, lam);
-            o.y = vjp_term(v.y, w.y, b, inv_t, it, lam);
-            o.z = vjp_term(v.z, w.z, b, inv_t, it, lam);
-            o.w = vjp_term(v.w, w.w, b, inv_t, it, lam);
+            o.x = vjp_term2(xf(v.x), w.x, hit, lam_hi, lam_lo);
+            o.y = vjp_term2(xf(v.y), w.y, hit, lam_hi, lam_lo);
+            o.z = vjp_term2(xf(v.z), w.z, hit, lam_hi, lam_lo);
+            o.w = vjp_term2(xf(v.w), w.w, hit, lam_hi, lam_lo);
             o4[i] = o;
         }
     } else {
-        for (int64_t i = tid; i < n; i += BLOCK)
-            out[i] = vjp_term(r[i], gg[i], b, inv_t, it, lam);
+        for (int64_t i = tid; i < n; i += BLOCK) out[i] = vjp_term2(xf(r[i]), gg[i], hit, lam_hi, lam_lo);
     }
 }
 

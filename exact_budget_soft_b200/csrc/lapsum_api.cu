@@ -99,6 +99,7 @@ struct Workspace {
     Ctl *ctl = nullptr;               size_t ctl_n = 0;
     double *partials = nullptr;       size_t partials_n = 0;
     uint32_t *skeys = nullptr;        size_t skeys_n = 0;
+    uint32_t *hist1 = nullptr;        size_t hist1_n = 0;
     float *band = nullptr;            size_t band_n = 0;
     uint32_t *keys0 = nullptr;        size_t keys0_n = 0;
     uint32_t *keys1 = nullptr;        size_t keys1_n = 0;
@@ -109,7 +110,7 @@ struct Workspace {
     uint32_t epoch = 1;
 
     void release() {
-        cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(band);
+        cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(hist1); cudaFree(band);
         cudaFree(keys0); cudaFree(keys1); cudaFree(hist); cudaFree(dbase);
         cudaFree(lookback); cudaFree(tilebuf);
         *this = Workspace();
@@ -327,10 +328,12 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     P.band_cap = band_cap;
     P.spin_cap = spin_cap;
     LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, 4096));
     LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_cap));
     LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort the whole row
     P.band = w->band;
     P.keys = w->skeys;
+    P.hist1 = w->hist1;
     P.partials = w->partials;
     P.ctl = w->ctl;
 

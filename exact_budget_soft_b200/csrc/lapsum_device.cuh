@@ -192,13 +192,55 @@ __device__ __forceinline__ float laplace_cdf_f(float x) {
     return x < 0.0f ? e : 1.0f - e;
 }
 
-// One VJP output, (f/t)(g - lambda) with f = e^{-|x|}/2.  g - lambda is formed in
-// fp64: when a few scores carry almost all of sum f, lambda sits within an fp32
-// ulp of their g and the difference would cancel.
-__device__ __forceinline__ float vjp_term(float r, float g, double b, double inv_t, float it,
-                                          double lam) {
-    const float f = 0.5f * expf(-fabsf((float)(((double)r - b) * inv_t)));
-    return (float)((double)(f * it) * ((double)g - lam));
+// ----------------------------------------------- fp32 elementwise math --
+constexpr float LOG2E_F = 1.4426950408889634f;
+constexpr double LOG2E = 1.4426950408889634;
+
+// x = (r - b)/t in fp32 from a hi/lo split of the fp64 threshold b:
+//   x = ((r - b_hi) - b_lo) * s.
+// Near the threshold r - b_hi is exact (Sterbenz), so x keeps fp32 relative
+// accuracy however close r is to b; s = log2(e)/t gives x in base-2 units.
+struct XForm {
+    float b_hi, b_lo, s;
+    __device__ __forceinline__ float operator()(float r) const { return ((r - b_hi) - b_lo) * s; }
+};
+__device__ __forceinline__ XForm make_xform(double b, double scale) {
+    XForm f;
+    f.b_hi = (float)b;
+    f.b_lo = (float)(b - (double)f.b_hi);
+    f.s = (float)scale;
+    return f;
+}
+
+// Laplace CDF from the base-2 argument x2 = x log2(e):
+// F = 2^{x2}/2 (x2 < 0), 1 - 2^{-x2}/2 (x2 >= 0).
+__device__ __forceinline__ float laplace_cdf2(float x2) {
+    const float e = 0.5f * exp2f(-fabsf(x2));
+    return x2 < 0.0f ? e : 1.0f - e;
+}
+
+// One VJP output, (f/t)(g - lambda), f = e^{-|x|}/2, from the base-2 argument.
+// g - lambda uses a hi/lo split of the fp64 lambda: when a few scores carry
+// almost all of sum f, lambda sits within an fp32 ulp of their g, and the split
+// keeps the difference exact.
+__device__ __forceinline__ float vjp_term2(float x2, float g, float half_inv_t, float lam_hi,
+                                           float lam_lo) {
+    return (half_inv_t * exp2f(-fabsf(x2))) * ((g - lam_hi) - lam_lo);
+}
+
+// Tiered accumulation of e^{-z}, z = (hi - lo)/t >= 0, where (hi, lo) is
+// (x, a) or (a, x) for a score x and a bracket end a.  Terms that can move the
+// budget by more than ~1e-7 (z <= 16) are formed in fp64 from an fp64 z;
+// terms down to e^{-40} in fp32; smaller ones (< 4.3e-18 each, so < 1e-8 for
+// 2^31 scores) are dropped.
+__device__ __forceinline__ void tier_add(float hi, float lo, double dhi, double dlo, float itf,
+                                         double inv_t, double &acc64, float &acc32) {
+    const float zf = (hi - lo) * itf;
+    if (zf <= 16.0f) {
+        acc64 += exp(-(dhi - dlo) * inv_t);
+    } else if (zf <= 40.0f) {
+        acc32 += exp2f(-zf * LOG2E_F);
+    }
 }
 
 // ------------------------------------------------ bounded device waits --

@@ -41,6 +41,7 @@ struct Ctl {
     unsigned int tile_ctr[4];
     // backward
     double vjp_lambda;
+    int32_t vjp_shift;        // every f underflowed: recompute lambda shifted
 };
 
 // Kernel-facing parameters of a bracketing solve.
@@ -55,6 +56,7 @@ struct BracketParams {
     int64_t band_cap;
     float *band;              // band buffer [band_cap]
     uint32_t *keys;           // sample keys [s]
+    uint32_t *hist1;          // [4096] first-round select histogram (kept zeroed)
     double *partials;         // per-block partials
     Ctl *ctl;
     int32_t spin_cap;
