@@ -4,9 +4,9 @@
 //
 //   sample_kernel   kernel-noised sample y_j = r_{I_j} + t L_j (Philox4x64-10)
 //   select_kernel   exact order statistics y_(jR), y_(jL) by 3-round radix select
-//   stream_kernel   one pass over r: counts and stable tail sums of the scores
-//                   outside [a_L, a_R), band compaction (warp ballots)
-//   certify_kernel  one pass over r: G(a_L), G(a_R) and the verdict
+//   oob_kernel<false>  streaming pass: counts and stable tail sums of the scores
+//                      outside [a_L, a_R), band compaction (warp ballots)
+//   oob_kernel<true>   certification pass: G(a_L), G(a_R) and the verdict
 //   p_kernel        p = F((r - b)/t)
 //   vjp_*_kernel    <g,f>/sum f, then grad = (f/t)(g - <g,f>/sum f)
 //
@@ -294,34 +294,63 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
     }
 }
 
-// ================================================================ stream --
-struct StreamAcc {
-    uint32_t cL, cR;
-    double SL, SR;      // near terms (fp64)
-    float SL2, SR2;     // far terms (fp32)
-    bool bad;
-};
+// ===================================================== out-of-band passes --
+// The streaming pass (technical summary section 2.2, step 2) and the
+// certification pass (step 4, abstract) walk every score once and, for each
+// score outside [a_L, a_R), add its tail term
+//   below a_L:  e^{(r - a_L)/t},    at or above a_R:  e^{-(r - a_R)/t}.
+// Terms come in three tiers by z = |r - a|/t: z <= 16 (can move the budget by
+// more than ~1e-7): fp64 from an fp64 z; 16 < z <= 40: fp32 ex2; z > 40
+// (< 4.3e-18 each): dropped.  A warp whose 128 scores all lie at z > 16 below
+// a_L takes a fast path (count, or count + fp32 terms) -- the bulk of a long
+// row -- so the pass stays memory-bound.  Non-finite scores never take it
+// (the float4 bounds use NaN-propagating max and a finite-min check).
+constexpr float NEAR2 = 23.083120654223414f;   // 16 log2(e)
+constexpr float FAR2 = 57.707801635558535f;    // 40 log2(e)
+
 struct Ends {
-    float aL, aR, itf;
+    float aL, aR, s2;          // s2 = log2(e)/t
+    float midL, farL;          // x < midL: z > 16 below a_L; x < farL: z > 40
     double daL, daR, inv_t;
 };
-
-// One score of the streaming pass (technical summary section 2.2, step 2):
-// at or above a_R -> count, S_R += e^{-(r-a_R)/t}; below a_L -> count,
-// S_L += e^{(r-a_L)/t}; returns whether it belongs to the band [a_L, a_R).
-__device__ __forceinline__ bool stream_one(float x, bool valid, const Ends &E, StreamAcc &acc) {
-    const bool above = valid && x >= E.aR;
-    const bool below = valid && x < E.aL;
-    acc.bad |= valid && !isfinite(x);
-    if (above) {
-        acc.cR += 1;
-        tier_add(x, E.aR, (double)x, E.daR, E.itf, E.inv_t, acc.SR, acc.SR2);
-    } else if (below) {
-        acc.cL += 1;
-        tier_add(E.aL, x, E.daL, (double)x, E.itf, E.inv_t, acc.SL, acc.SL2);
-    }
-    return valid && !above && !below && x == x;
+__device__ __forceinline__ Ends make_ends(const Ctl *ctl, double inv_t) {
+    Ends E;
+    E.aL = ctl->a_L;
+    E.aR = ctl->a_R;
+    E.daL = E.aL;
+    E.daR = E.aR;
+    E.inv_t = inv_t;
+    E.s2 = (float)(inv_t * LOG2E);
+    // thresholds in score space, rounded toward a_L (the fast paths then only
+    // ever take scores at or beyond their tier bound, up to fp32 rounding)
+    E.midL = (float)(E.daL - 16.0 / inv_t);
+    E.farL = (float)(E.daL - 40.0 / inv_t);
+    return E;
 }
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float y;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+    return y;
+}
+// tiered e^{-z} with z = (hi - lo)/t
+__device__ __forceinline__ void tier2(float hi, float lo, double dhi, double dlo, const Ends &E,
+                                      double &acc64, float &acc32) {
+    const float z2 = (hi - lo) * E.s2;
+    if (z2 <= NEAR2) acc64 += exp(-(dhi - dlo) * E.inv_t);
+    else acc32 += ex2_ftz(-z2);
+}
+
+struct OobAcc {
+    uint32_t cL, cR, cB;        // stream: below, above; certify: >= a_L, >= a_R, < a_L
+    double SL, SR, hL, lR;      // near terms: below, above, band vs a_L, band vs a_R
+    float SL2, SR2, hL2, lR2;   // far terms
+    bool bad;
+};
 
 // Append a band score at a warp-aggregated slot of the band buffer (the count
 // keeps going past the capacity so the overflow is visible).
@@ -336,123 +365,124 @@ __device__ __forceinline__ void band_push(float x, bool inb, float *band, unsign
     if (inb && base < cap) band[base] = x;
 }
 
-__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) stream_kernel(BracketParams P) {
-    __shared__ double s_red[4 * (SBLOCK / 32)];
+// General path, one score.  Returns "in the band" (streaming mode).
+template <bool CERT>
+__device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobAcc &a) {
+    if (!valid) return false;
+    a.bad |= !(fabsf(x) < CUDART_INF_F);
+    if (x >= E.aR) {
+        if (CERT) { a.cL += 1; a.cR += 1; } else { a.cR += 1; }
+        tier2(x, E.aR, (double)x, E.daR, E, a.SR, a.SR2);
+        return false;
+    }
+    if (x < E.aL) {
+        if (CERT) a.cB += 1; else a.cL += 1;
+        tier2(E.aL, x, E.daL, (double)x, E, a.SL, a.SL2);
+        return false;
+    }
+    if (CERT && x == x) {
+        a.cL += 1;
+        tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
+        tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
+    }
+    return x == x;
+}
+
+// One float4 of the pass; `ok` false for padding lanes (whole warps iterate).
+template <bool CERT>
+__device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, OobAcc &a,
+                                        const BracketParams &P, unsigned long long cap, int lane) {
+    const float mx = max_nan(max_nan(v.x, v.y), max_nan(v.z, v.w));
+    const float mn = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
+    const bool fin = mn > -CUDART_INF_F;
+    const bool far = !ok || (mx < E.farL && fin);
+    const bool mid = !ok || (mx < E.midL && fin);
+    if (__all_sync(FULL, far)) {
+        if (ok) { if (CERT) a.cB += 4; else a.cL += 4; }
+        return;
+    }
+    if (__all_sync(FULL, mid)) {
+        if (ok) {
+            if (CERT) a.cB += 4; else a.cL += 4;
+            a.SL2 += (ex2_ftz((v.x - E.aL) * E.s2) + ex2_ftz((v.y - E.aL) * E.s2)) +
+                     (ex2_ftz((v.z - E.aL) * E.s2) + ex2_ftz((v.w - E.aL) * E.s2));
+        }
+        return;
+    }
+    const bool b0 = oob_one<CERT>(v.x, ok, E, a);
+    const bool b1 = oob_one<CERT>(v.y, ok, E, a);
+    const bool b2 = oob_one<CERT>(v.z, ok, E, a);
+    const bool b3 = oob_one<CERT>(v.w, ok, E, a);
+    if (!CERT && __any_sync(FULL, b0 | b1 | b2 | b3)) {
+        unsigned long long *ctr = &P.ctl->c_band;
+        band_push(v.x, b0, P.band, cap, ctr, lane);
+        band_push(v.y, b1, P.band, cap, ctr, lane);
+        band_push(v.z, b2, P.band, cap, ctr, lane);
+        band_push(v.w, b3, P.band, cap, ctr, lane);
+    }
+}
+
+// CERT = false: streaming pass (forward over the row): c_L, c_R, S_L, S_R and
+//               the band.
+// CERT = true:  certification pass (backward over the row, starting on what
+//               the streaming pass left in L2):
+//   G(a) = #{r >= a} - 1/2 sum_{r>=a} e^{-(r-a)/t} + 1/2 sum_{r<a} e^{(r-a)/t}
+// at a = a_L and a = a_R.  Scores outside the band share one exponential
+// between the two ends (e^{-(r-a_L)/t} = e^{-(r-a_R)/t} e^{-(a_R-a_L)/t} and its
+// mirror image below); band scores take two.  Verdict: G(a_L) >= k > G(a_R),
+// the band fits its buffer, both passes agree on every membership count, and
+// every score is finite.
+template <bool CERT>
+__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) oob_kernel(BracketParams P) {
+    __shared__ double s_red[7 * (SBLOCK / 32)];
     Ctl *ctl = P.ctl;
-    Ends E;
-    E.aL = ctl->a_L;
-    E.aR = ctl->a_R;
-    E.daL = E.aL;
-    E.daR = E.aR;
-    E.inv_t = P.inv_t;
-    E.itf = (float)P.inv_t;
+    const Ends E = make_ends(ctl, P.inv_t);
     const int lane = threadIdx.x & 31;
     const unsigned long long cap = (unsigned long long)P.band_cap;
-    unsigned long long *ctr = &ctl->c_band;
-    StreamAcc acc{0, 0, 0.0, 0.0, 0.f, 0.f, false};
+    OobAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
     const int64_t n = P.n;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
     const int64_t n4 = aligned ? n / 4 : 0;
     const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
-    // whole warps iterate together (the ballots need every lane)
-    const int64_t n4w = (n4 + gstride - 1) / gstride * gstride;
-    for (int64_t i = gtid; i < n4w; i += gstride) {
+    const int64_t n4w = (n4 + gstride - 1) / gstride * gstride;   // whole warps iterate together
+    int64_t i = gtid;
+    for (; i + gstride < n4w; i += 2 * gstride) {   // two loads in flight
+        const int64_t i0 = CERT ? n4 - 1 - i : i, i1 = CERT ? n4 - 1 - (i + gstride) : i + gstride;
+        const bool ok0 = i < n4, ok1 = i + gstride < n4;
+        const float4 v0 = ok0 ? r4[i0] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v1 = ok1 ? r4[i1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        oob_vec<CERT>(v0, ok0, E, acc, P, cap, lane);
+        oob_vec<CERT>(v1, ok1, E, acc, P, cap, lane);
+    }
+    for (; i < n4w; i += gstride) {
         const bool ok = i < n4;
-        const float4 v = ok ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const bool b0 = stream_one(v.x, ok, E, acc);
-        const bool b1 = stream_one(v.y, ok, E, acc);
-        const bool b2 = stream_one(v.z, ok, E, acc);
-        const bool b3 = stream_one(v.w, ok, E, acc);
-        if (__any_sync(FULL, b0 | b1 | b2 | b3)) {
-            band_push(v.x, b0, P.band, cap, ctr, lane);
-            band_push(v.y, b1, P.band, cap, ctr, lane);
-            band_push(v.z, b2, P.band, cap, ctr, lane);
-            band_push(v.w, b3, P.band, cap, ctr, lane);
-        }
+        const float4 v = ok ? r4[CERT ? n4 - 1 - i : i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        oob_vec<CERT>(v, ok, E, acc, P, cap, lane);
     }
     const int64_t rem0 = n4 * 4;
     const int64_t remw = rem0 + ((n - rem0 + gstride - 1) / gstride) * gstride;
-    for (int64_t i = rem0 + gtid; i < remw; i += gstride) {
-        const bool ok = i < n;
-        const float x = ok ? P.r[i] : 0.f;
-        const bool bb = stream_one(x, ok, E, acc);
-        band_push(x, bb, P.band, cap, ctr, lane);
+    for (int64_t j = rem0 + gtid; j < remw; j += gstride) {
+        const bool ok = j < n;
+        const float x = ok ? P.r[j] : 0.f;
+        const bool bb = oob_one<CERT>(x, ok, E, acc);
+        if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane);
     }
     if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
-    double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2};
-    block_sum<SBLOCK, 4>(v, s_red);
-    if (last_block_sum<SBLOCK, 4>(v, P.partials, &ctl->ticket[0], s_red) && threadIdx.x == 0) {
-        ctl->c_L = (unsigned long long)v[0];
-        ctl->c_R = (unsigned long long)v[1];
-        ctl->S_L = v[2];
-        ctl->S_R = v[3];
+    if (!CERT) {
+        double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2};
+        block_sum<SBLOCK, 4>(v, s_red);
+        if (last_block_sum<SBLOCK, 4>(v, P.partials, &ctl->ticket[0], s_red) && threadIdx.x == 0) {
+            ctl->c_L = (unsigned long long)v[0];
+            ctl->c_R = (unsigned long long)v[1];
+            ctl->S_L = v[2];
+            ctl->S_R = v[3];
+        }
+        return;
     }
-}
-
-// ============================================================ certificate --
-// One more linear pass (abstract: "a certification pass ... at the cost of one
-// additional linear pass"; technical summary section 2.2 step 4):
-//   G(a) = #{r >= a} - 1/2 sum_{r>=a} e^{-(r-a)/t} + 1/2 sum_{r<a} e^{(r-a)/t}
-// for a = a_L and a = a_R.  Scores outside the band share one exponential
-// between the two ends (e^{-(r-a_L)/t} = e^{-(r-a_R)/t} e^{-(a_R-a_L)/t}, and the
-// mirror image below), band scores take two.  Verdict: G(a_L) >= k > G(a_R),
-// the band fits its buffer, and both passes agree on every membership count.
-struct CertAcc {
-    uint32_t cntL, cntR, cntB;   // >= a_L, >= a_R, < a_L
-    double above, below, hiL, loR;
-    float above2, below2, hiL2, loR2;
-    bool bad;
-};
-
-__device__ __forceinline__ void cert_one(float x, const Ends &E, CertAcc &a) {
-    a.bad |= !isfinite(x);
-    if (x >= E.aR) {
-        a.cntR += 1;
-        a.cntL += 1;
-        tier_add(x, E.aR, (double)x, E.daR, E.itf, E.inv_t, a.above, a.above2);
-    } else if (x >= E.aL) {
-        a.cntL += 1;
-        tier_add(x, E.aL, (double)x, E.daL, E.itf, E.inv_t, a.hiL, a.hiL2);
-        tier_add(E.aR, x, E.daR, (double)x, E.itf, E.inv_t, a.loR, a.loR2);
-    } else if (x < E.aL) {
-        a.cntB += 1;
-        tier_add(E.aL, x, E.daL, (double)x, E.itf, E.inv_t, a.below, a.below2);
-    }
-}
-
-__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) certify_kernel(BracketParams P) {
-    __shared__ double s_red[7 * (SBLOCK / 32)];
-    Ctl *ctl = P.ctl;
-    Ends E;
-    E.aL = ctl->a_L;
-    E.aR = ctl->a_R;
-    E.daL = E.aL;
-    E.daR = E.aR;
-    E.inv_t = P.inv_t;
-    E.itf = (float)P.inv_t;
-    CertAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
-    const int64_t n = P.n;
-    const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
-    const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
-    const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
-    const int64_t n4 = aligned ? n / 4 : 0;
-    const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
-    // the second pass walks the row from the end, so it starts on the part the
-    // streaming pass left in L2
-    for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = r4[n4 - 1 - i];
-        cert_one(v.x, E, acc);
-        cert_one(v.y, E, acc);
-        cert_one(v.z, E, acc);
-        cert_one(v.w, E, acc);
-    }
-    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) cert_one(P.r[i], E, acc);
-    if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
-    double v[7] = {(double)acc.cntL, (double)acc.cntR, (double)acc.cntB,
-                   acc.above + (double)acc.above2, acc.below + (double)acc.below2,
-                   acc.hiL + (double)acc.hiL2, acc.loR + (double)acc.loR2};
+    double v[7] = {(double)acc.cL, (double)acc.cR, (double)acc.cB, acc.SR + (double)acc.SR2,
+                   acc.SL + (double)acc.SL2, acc.hL + (double)acc.hL2, acc.lR + (double)acc.lR2};
     block_sum<SBLOCK, 7>(v, s_red);
     if (last_block_sum<SBLOCK, 7>(v, P.partials + 8 * (size_t)gridDim.x, &ctl->ticket[1], s_red) &&
         threadIdx.x == 0) {
@@ -475,7 +505,16 @@ __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) certify_kernel(Bracket
 
 // ================================================================= p pass --
 // p = F((r - b)/t), walking forward (the certification pass left the head of
-// the row in L2).  Also sum p (fp64) for the diagnostics.
+// the row in L2).  Also sum p (fp64 over fp32 float4 partials) for diagnostics.
+__device__ __forceinline__ float4 p_vec(const float4 v, const XForm &xf) {
+    float4 o;
+    o.x = laplace_cdf2(xf(v.x));
+    o.y = laplace_cdf2(xf(v.y));
+    o.z = laplace_cdf2(xf(v.z));
+    o.w = laplace_cdf2(xf(v.w));
+    return o;
+}
+
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict__ p,
          double *__restrict__ b_out, Ctl *ctl, double *partials) {
@@ -489,20 +528,23 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
     const float4 *r4 = reinterpret_cast<const float4 *>(r);
     float4 *p4 = reinterpret_cast<float4 *>(p);
     double ps = 0.0;
-    for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = r4[i];
-        float4 o;
-        o.x = laplace_cdf2(xf(v.x));
-        o.y = laplace_cdf2(xf(v.y));
-        o.z = laplace_cdf2(xf(v.z));
-        o.w = laplace_cdf2(xf(v.w));
-        ps += ((double)o.x + (double)o.y) + ((double)o.z + (double)o.w);
-        __stcs(p4 + i, o);
+    int64_t i = gtid;
+    for (; i + gstride < n4; i += 2 * gstride) {
+        const float4 v0 = r4[i], v1 = r4[i + gstride];
+        const float4 o0 = p_vec(v0, xf), o1 = p_vec(v1, xf);
+        __stcs(p4 + i, o0);
+        __stcs(p4 + i + gstride, o1);
+        ps += (double)(((o0.x + o0.y) + (o0.z + o0.w)) + ((o1.x + o1.y) + (o1.z + o1.w)));
     }
-    for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
-        const float o = laplace_cdf2(xf(r[i]));
+    for (; i < n4; i += gstride) {
+        const float4 o = p_vec(r4[i], xf);
+        __stcs(p4 + i, o);
+        ps += (double)((o.x + o.y) + (o.z + o.w));
+    }
+    for (int64_t j = n4 * 4 + gtid; j < n; j += gstride) {
+        const float o = laplace_cdf2(xf(r[j]));
         ps += (double)o;
-        p[i] = o;
+        p[j] = o;
     }
     double v[1] = {ps};
     block_sum<SBLOCK, 1>(v, s_red);
@@ -532,9 +574,7 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
     const float4 *r4 = reinterpret_cast<const float4 *>(r);
     const float4 *g4 = reinterpret_cast<const float4 *>(g);
     double sf = 0.0, sgf = 0.0;
-    for (int64_t i = gtid; i < n4; i += gstride) {
-        const int64_t j = n4 - 1 - i;
-        const float4 v = r4[j], w = g4[j];
+    auto acc4 = [&](const float4 v, const float4 w) {
         const float e0 = exp2f(-fabsf(xf(v.x))), e1 = exp2f(-fabsf(xf(v.y)));
         const float e2 = exp2f(-fabsf(xf(v.z))), e3 = exp2f(-fabsf(xf(v.w)));
         sf += ((double)e0 + (double)e1) + ((double)e2 + (double)e3);
@@ -542,7 +582,15 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
         sgf = fma((double)w.y, (double)e1, sgf);
         sgf = fma((double)w.z, (double)e2, sgf);
         sgf = fma((double)w.w, (double)e3, sgf);
+    };
+    int64_t i = gtid;
+    for (; i + gstride < n4; i += 2 * gstride) {
+        const int64_t j0 = n4 - 1 - i, j1 = n4 - 1 - (i + gstride);
+        const float4 v0 = r4[j0], w0 = g4[j0], v1 = r4[j1], w1 = g4[j1];
+        acc4(v0, w0);
+        acc4(v1, w1);
     }
+    for (; i < n4; i += gstride) acc4(r4[n4 - 1 - i], g4[n4 - 1 - i]);
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
         const float e = exp2f(-fabsf(xf(r[i])));
         sf += (double)e;
@@ -642,15 +690,21 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
     const float4 *r4 = reinterpret_cast<const float4 *>(r);
     const float4 *g4 = reinterpret_cast<const float4 *>(g);
     float4 *o4 = reinterpret_cast<float4 *>(grad);
-    for (int64_t i = gtid; i < n4; i += gstride) {
-        const float4 v = r4[i], w = g4[i];
+    auto apply4 = [&](const float4 v, const float4 w) {
         float4 o;
         o.x = vjp_term2(xf(v.x), w.x, hit, lam_hi, lam_lo);
         o.y = vjp_term2(xf(v.y), w.y, hit, lam_hi, lam_lo);
         o.z = vjp_term2(xf(v.z), w.z, hit, lam_hi, lam_lo);
         o.w = vjp_term2(xf(v.w), w.w, hit, lam_hi, lam_lo);
-        __stcs(o4 + i, o);
+        return o;
+    };
+    int64_t i = gtid;
+    for (; i + gstride < n4; i += 2 * gstride) {
+        const float4 v0 = r4[i], w0 = g4[i], v1 = r4[i + gstride], w1 = g4[i + gstride];
+        __stcs(o4 + i, apply4(v0, w0));
+        __stcs(o4 + i + gstride, apply4(v1, w1));
     }
+    for (; i < n4; i += gstride) __stcs(o4 + i, apply4(r4[i], g4[i]));
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
         grad[i] = vjp_term2(xf(r[i]), g[i], hit, lam_hi, lam_lo);
 }
@@ -673,11 +727,11 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     return cudaGetLastError();
 }
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
-    stream_kernel<<<stream_grid(), SBLOCK, 0, st>>>(P);
+    oob_kernel<false><<<stream_grid(), SBLOCK, 0, st>>>(P);
     return cudaGetLastError();
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
-    certify_kernel<<<stream_grid(), SBLOCK, 0, st>>>(P);
+    oob_kernel<true><<<stream_grid(), SBLOCK, 0, st>>>(P);
     return cudaGetLastError();
 }
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,

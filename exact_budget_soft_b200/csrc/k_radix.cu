@@ -102,20 +102,28 @@ __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // exclusive digit bases; a digit whose histogram has one bin holding every key is skipped
-    if (tid < 4) {
-        const int d = tid;
-        unsigned long long run = 0;
-        bool trivial = false;
-        for (int b = 0; b < 256; ++b) {
-            const unsigned long long c = __ldcg(A.hist + d * 256 + b);
-            A.dbase[d * 256 + b] = (uint32_t)run;
-            run += c;
-            if (c == (unsigned long long)n) trivial = true;
+    // exclusive digit bases (thread tid owns bin tid of every digit); a digit
+    // whose histogram has one bin holding every key is skipped
+    static_assert(HB == 256, "one thread per bin");
+    __shared__ uint32_t s_wsum[HB / 32];
+    for (int d = 0; d < 4; ++d) {
+        const uint32_t c = (uint32_t)__ldcg(A.hist + d * 256 + tid);
+        const int lane = tid & 31, warp = tid >> 5;
+        uint32_t inc = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t p = __shfl_up_sync(FULL, inc, o);
+            if (lane >= o) inc += p;
         }
-        s_trivial[d] = trivial ? 1 : 0;
+        if (lane == 31) s_wsum[warp] = inc;
+        __syncthreads();
+        uint32_t off = 0;
+        for (int w = 0; w < warp; ++w) off += s_wsum[w];
+        A.dbase[d * 256 + tid] = off + inc - c;
+        const int triv = __syncthreads_or(c == (uint32_t)n);
+        if (tid == 0) s_trivial[d] = triv;
+        __syncthreads();
     }
-    __syncthreads();
     for (int i = tid; i < 4 * 256; i += HB) A.hist[i] = 0ull;   // ready for the next sort
     if (tid == 0) {
         A.ctl->sort_skip = s_trivial[0] | (s_trivial[1] << 1) | (s_trivial[2] << 2) | (s_trivial[3] << 3);
