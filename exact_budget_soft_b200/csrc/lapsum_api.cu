@@ -188,40 +188,86 @@ int map_err(cudaError_t e) {
 //   jR = largest j with P(X < j) <= delta/2 (0 -> a_R = +inf),
 //   jL = smallest j with P(X >= j) <= delta/2 (s+1 -> a_L = -inf).
 // The pmf is built outward from the mode by the ratio recurrence
-// pmf(j+1)/pmf(j) = (s-j)/(j+1) * pi/(1-pi), in log space, normalised at the mode.
-void binomial_ranks(int64_t s, double pi, double delta, int64_t &jR, int64_t &jL) {
-    const int64_t mode = (int64_t)std::floor((double)(s + 1) * pi) > s ? s
-                         : (int64_t)std::floor((double)(s + 1) * pi);
+// pmf(j+1)/pmf(j) = (s-j)/(j+1) * pi/(1-pi), relative to the mode (no logs per
+// term), until terms fall below 1e-300 of the mode; the mode's own value comes
+// from lgamma.  Results are memoised per (s, pi, delta).
+void binomial_ranks_compute(int64_t s, double pi, double delta, int64_t &jR, int64_t &jL) {
+    int64_t mode = (int64_t)std::floor((double)(s + 1) * pi);
+    if (mode > s) mode = s;
     const double lmode = std::lgamma((double)s + 1.0) - std::lgamma((double)mode + 1.0) -
                          std::lgamma((double)(s - mode) + 1.0) + (double)mode * std::log(pi) +
                          (double)(s - mode) * std::log1p(-pi);
-    const double lodds = std::log(pi) - std::log1p(-pi);
-    std::vector<double> lp((size_t)s + 1);
-    lp[(size_t)mode] = lmode;
-    for (int64_t j = mode; j < s; ++j)
-        lp[(size_t)j + 1] = lp[(size_t)j] + std::log((double)(s - j) / (double)(j + 1)) + lodds;
-    for (int64_t j = mode; j > 0; --j)
-        lp[(size_t)j - 1] = lp[(size_t)j] - std::log((double)(s - j + 1) / (double)j) - lodds;
-    const double half = 0.5 * delta;
-    // lower tail, smallest terms first
+    const double pmode = std::exp(lmode);
+    const double odds = pi / (1.0 - pi);
+    std::vector<double> up, down;   // relative pmf above / below the mode
+    double w = 1.0;
+    for (int64_t j = mode; j < s && w > 1e-300; ++j) {
+        w *= ((double)(s - j) / (double)(j + 1)) * odds;
+        up.push_back(w);            // pmf(j+1)/pmf(mode)
+    }
+    w = 1.0;
+    for (int64_t j = mode; j > 0 && w > 1e-300; --j) {
+        w *= ((double)j / (double)(s - j + 1)) / odds;
+        down.push_back(w);          // pmf(j-1)/pmf(mode)
+    }
+    const int64_t lo = mode - (int64_t)down.size();   // smallest j with a stored term
+    const int64_t hi = mode + (int64_t)up.size();
+    auto rel = [&](int64_t j) -> double {
+        if (j == mode) return 1.0;
+        if (j > mode) return up[(size_t)(j - mode - 1)];
+        return down[(size_t)(mode - j - 1)];
+    };
+    const double half = 0.5 * delta / pmode;   // thresholds in units of pmf(mode)
+    // lower tail P(X < j), smallest terms first (Kahan)
     double acc = 0.0, comp = 0.0;
-    jR = 0;
-    for (int64_t j = 1; j <= s; ++j) {
-        const double term = std::exp(lp[(size_t)j - 1]);
-        const double y = term - comp, tt = acc + y;
+    jR = lo;                                       // P(X < lo) is negligible
+    for (int64_t j = lo + 1; j <= s + 1 && j - 1 <= hi; ++j) {
+        const double y = rel(j - 1) - comp, tt = acc + y;
         comp = (tt - acc) - y;
-        acc = tt;                                  // acc = P(X < j)
+        acc = tt;                                  // acc = P(X < j) / pmf(mode)
         if (acc <= half) jR = j; else break;
     }
+    if (jR > s) jR = s;
     acc = 0.0; comp = 0.0;
-    jL = s + 1;
-    for (int64_t j = s; j >= 0; --j) {
-        const double term = std::exp(lp[(size_t)j]);
-        const double y = term - comp, tt = acc + y;
+    jL = hi + 1;                                   // P(X >= hi+1) is negligible
+    for (int64_t j = hi; j >= lo; --j) {
+        const double y = rel(j) - comp, tt = acc + y;
         comp = (tt - acc) - y;
-        acc = tt;                                  // acc = P(X >= j)
+        acc = tt;                                  // acc = P(X >= j) / pmf(mode)
         if (acc <= half) jL = j; else break;
     }
+    if (jL > s + 1) jL = s + 1;
+}
+
+struct RankKey {
+    int64_t s;
+    uint64_t pi_bits, delta_bits;
+    bool operator<(const RankKey &o) const {
+        if (s != o.s) return s < o.s;
+        if (pi_bits != o.pi_bits) return pi_bits < o.pi_bits;
+        return delta_bits < o.delta_bits;
+    }
+};
+std::mutex g_rank_mu;
+std::map<RankKey, std::pair<int64_t, int64_t>> g_rank_cache;
+
+void binomial_ranks(int64_t s, double pi, double delta, int64_t &jR, int64_t &jL) {
+    RankKey key{s, 0, 0};
+    std::memcpy(&key.pi_bits, &pi, 8);
+    std::memcpy(&key.delta_bits, &delta, 8);
+    {
+        std::lock_guard<std::mutex> lk(g_rank_mu);
+        auto it = g_rank_cache.find(key);
+        if (it != g_rank_cache.end()) {
+            jR = it->second.first;
+            jL = it->second.second;
+            return;
+        }
+    }
+    binomial_ranks_compute(s, pi, delta, jR, jL);
+    std::lock_guard<std::mutex> lk(g_rank_mu);
+    if (g_rank_cache.size() > 4096) g_rank_cache.clear();
+    g_rank_cache[key] = {jR, jL};
 }
 
 int check_args(const float *scores, int64_t rows, int64_t n, double k, double t) {

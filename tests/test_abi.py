@@ -102,3 +102,16 @@ def test_bracket_plan_matches_oracle_ranks(lib, orc, n, k, s, delta):
         assert s_ == min(65536, max(4096, pw))
     assert (jR, jL) == orc.binom_ranks(s_, k / n, delta or 1e-6)
     assert 0 < cap <= n
+
+
+def test_bracket_plan_ranks_fuzz(lib, orc):
+    # the library's log-free ratio recurrence and the oracle's lgamma sums pick the same ranks
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for _ in range(400):
+        s = int(rng.choice([50, 512, 1000, 4096, 16384, 65536]))
+        pi = float(10 ** rng.uniform(-6, -0.01))
+        delta = float(10 ** rng.uniform(-9, -0.3))
+        n = 10 ** 9
+        _, jR, jL, _ = _plan(lib, n, pi * n, s, delta)
+        assert (jR, jL) == orc.binom_ranks(s, pi, delta)
