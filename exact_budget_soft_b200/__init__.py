@@ -54,7 +54,7 @@ class Stats(C.Structure):
 
 EXPORTS = ["lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats",
            "lapsum_strerror", "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read",
-           "lapsum_bracket_plan", "lapsum_launch_count"]
+           "lapsum_bracket_plan", "lapsum_profile_filter", "lapsum_selftest_math", "lapsum_launch_count"]
 
 
 def _load() -> C.CDLL:
@@ -76,6 +76,10 @@ def _load() -> C.CDLL:
     lib.lapsum_bracket_plan.argtypes = [i64, dbl, C.POINTER(Options), C.POINTER(i64), C.POINTER(i64),
                                         C.POINTER(i64), C.POINTER(i64)]
     lib.lapsum_bracket_plan.restype = C.c_int
+    lib.lapsum_profile_filter.argtypes = [C.c_char_p]
+    lib.lapsum_profile_filter.restype = C.c_int
+    lib.lapsum_selftest_math.argtypes = [C.c_int, vp, vp, vp, i64, vp]
+    lib.lapsum_selftest_math.restype = C.c_int
     for name in ("lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats",
                  "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read"):
         getattr(lib, name).restype = C.c_int
@@ -182,6 +186,19 @@ def launch_count() -> int:
 
 def profile_enable(mode: int = 1):
     lib.lapsum_profile_enable(int(mode))
+
+
+def profile_filter(substring: str | None = None):
+    lib.lapsum_profile_filter(substring.encode() if substring else None)
+
+
+def selftest_math(which: int, x: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """(ours, CUDA library) for which = 0: 2^{-x} near-tier exp; 1: the sampler's ln."""
+    _need(x, "x", torch.float64)
+    out, ref = torch.empty_like(x), torch.empty_like(x)
+    _check(lib.lapsum_selftest_math(int(which), x.data_ptr(), out.data_ptr(), ref.data_ptr(), x.numel(),
+                                    _stream(None)), "lapsum_selftest_math")
+    return out, ref
 
 
 def profile_read() -> dict:

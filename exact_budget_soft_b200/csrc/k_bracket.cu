@@ -311,7 +311,8 @@ constexpr float FAR2 = 57.707801635558535f;    // 40 log2(e)
 struct Ends {
     float aL, aR, s2;          // s2 = log2(e)/t
     float midL, farL;          // x < midL: z > 16 below a_L; x < farL: z > 40
-    double daL, daR, inv_t;
+    double daL, daR, inv_t, s2d;
+    const double *tab;         // 2^{-j/32}, shared memory
 };
 __device__ __forceinline__ Ends make_ends(const Ctl *ctl, double inv_t) {
     Ends E;
@@ -320,7 +321,8 @@ __device__ __forceinline__ Ends make_ends(const Ctl *ctl, double inv_t) {
     E.daL = E.aL;
     E.daR = E.aR;
     E.inv_t = inv_t;
-    E.s2 = (float)(inv_t * LOG2E);
+    E.s2d = inv_t * LOG2E;
+    E.s2 = (float)E.s2d;
     // thresholds in score space, rounded toward a_L (the fast paths then only
     // ever take scores at or beyond their tier bound, up to fp32 rounding)
     E.midL = (float)(E.daL - 16.0 / inv_t);
@@ -341,7 +343,7 @@ __device__ __forceinline__ float max_nan(float a, float b) {
 __device__ __forceinline__ void tier2(float hi, float lo, double dhi, double dlo, const Ends &E,
                                       double &acc64, float &acc32) {
     const float z2 = (hi - lo) * E.s2;
-    if (z2 <= NEAR2) acc64 += exp(-(dhi - dlo) * E.inv_t);
+    if (z2 <= NEAR2) acc64 += exp2_neg((dhi - dlo) * E.s2d, E.tab);
     else acc32 += ex2_ftz(-z2);
 }
 
@@ -435,8 +437,12 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
 template <bool CERT>
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) oob_kernel(BracketParams P) {
     __shared__ double s_red[7 * (SBLOCK / 32)];
+    __shared__ double s_tab[32];
+    exp2_table_init(s_tab);
     Ctl *ctl = P.ctl;
-    const Ends E = make_ends(ctl, P.inv_t);
+    Ends E = make_ends(ctl, P.inv_t);
+    E.tab = s_tab;
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const unsigned long long cap = (unsigned long long)P.band_cap;
     OobAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
@@ -709,7 +715,29 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
         grad[i] = vjp_term2(xf(r[i]), g[i], hit, lam_hi, lam_lo);
 }
 
+// ============================================================= self-test --
+__global__ void selftest_math_kernel(int which, const double *in, double *out, double *ref, int64_t n) {
+    __shared__ double s_tab[32];
+    exp2_table_init(s_tab);
+    __syncthreads();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const double x = in[i];
+        if (which == 0) {
+            out[i] = exp2_neg(x, s_tab);
+            ref[i] = exp2(-x);
+        } else {
+            out[i] = sample_ln(x);
+            ref[i] = log(x);
+        }
+    }
+}
+
 // ============================================================= launchers --
+cudaError_t launch_selftest_math(int which, const double *in, double *out, double *ref, int64_t n,
+                                 cudaStream_t st) {
+    selftest_math_kernel<<<148, 256, 0, st>>>(which, in, out, ref, n);
+    return cudaGetLastError();
+}
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
     const unsigned blocks = (unsigned)((P.s + 255) / 256);
     sample_kernel<<<blocks, 256, 0, st>>>(P);

@@ -40,6 +40,7 @@ struct ProfAcc {
 };
 std::mutex g_prof_mu;
 int g_prof_mode = 0;
+std::string g_prof_filter;
 std::vector<ProfRec> g_prof_pending;
 std::vector<std::pair<std::string, ProfAcc>> g_prof_acc;
 std::vector<cudaEvent_t> g_event_pool;
@@ -64,7 +65,7 @@ struct Launch {
     Launch(const char *nm, cudaStream_t s) : name(nm), st(s) {
         std::lock_guard<std::mutex> lk(g_prof_mu);
         ++g_launches;
-        if (g_prof_mode) {
+        if (g_prof_mode && (g_prof_filter.empty() || std::strstr(nm, g_prof_filter.c_str()))) {
             e0 = take_event();
             cudaEventRecord(e0, st);
         }
@@ -517,6 +518,21 @@ int lapsum_profile_enable(int mode) {
         mode = g_prof_mode;
     }
     g_prof_mode = mode ? 1 : 0;
+    return LAPSUM_OK;
+}
+
+int lapsum_profile_filter(const char *substring) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_filter = substring ? substring : "";
+    return LAPSUM_OK;
+}
+
+int lapsum_selftest_math(int which, const double *in, double *out, double *ref, int64_t n,
+                         struct CUstream_st *stream_in) {
+    if (!in || !out || !ref || n < 1 || (which != 0 && which != 1)) return LAPSUM_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    LAPSUM_TRY(launch_selftest_math(which, in, out, ref, n, st));
+    LAPSUM_TRY(cudaStreamSynchronize(st));
     return LAPSUM_OK;
 }
 

@@ -228,19 +228,42 @@ __device__ __forceinline__ float vjp_term2(float x2, float g, float half_inv_t, 
     return (half_inv_t * exp2f(-fabsf(x2))) * ((g - lam_hi) - lam_lo);
 }
 
-// Tiered accumulation of e^{-z}, z = (hi - lo)/t >= 0, where (hi, lo) is
-// (x, a) or (a, x) for a score x and a bracket end a.  Terms that can move the
-// budget by more than ~1e-7 (z <= 16) are formed in fp64 from an fp64 z;
-// terms down to e^{-40} in fp32; smaller ones (< 4.3e-18 each, so < 1e-8 for
-// 2^31 scores) are dropped.
-__device__ __forceinline__ void tier_add(float hi, float lo, double dhi, double dlo, float itf,
-                                         double inv_t, double &acc64, float &acc32) {
-    const float zf = (hi - lo) * itf;
-    if (zf <= 16.0f) {
-        acc64 += exp(-(dhi - dlo) * inv_t);
-    } else if (zf <= 40.0f) {
-        acc32 += exp2f(-zf * LOG2E_F);
-    }
+// ----------------------------------------------------- near-tier exp --
+// 2^{-w} for 0 <= w <= 1000, the fp64 terms of the tail sums.  Table-driven
+// reduction after P. T. P. Tang, "Table-driven implementation of the
+// exponential function in IEEE floating-point arithmetic", ACM TOMS 15 (1989):
+//   N = rint(32 w) = 32 m + j,  r = w - N/32 in [-1/64, 1/64],
+//   2^{-w} = 2^{-m} * 2^{-j/32} * 2^{-r},
+// 2^{-r} = e^{-r ln 2} by its Taylor polynomial to degree 6 (remainder
+// < 4e-18), the 32 table values 2^{-j/32} from the library exp2 (computed once
+// per block into shared memory), 2^{-m} applied to the exponent field.  About
+// 11 fp64 operations; relative error a few ulp (tested against exp).
+constexpr double EXP_LN2 = 0x1.62e42fefa39efp-1;
+constexpr double EXP_C1 = -EXP_LN2;
+constexpr double EXP_C2 = EXP_LN2 * EXP_LN2 / 2.0;
+constexpr double EXP_C3 = -EXP_LN2 * EXP_LN2 * EXP_LN2 / 6.0;
+constexpr double EXP_C4 = EXP_LN2 * EXP_LN2 * EXP_LN2 * EXP_LN2 / 24.0;
+constexpr double EXP_C5 = -EXP_LN2 * EXP_LN2 * EXP_LN2 * EXP_LN2 * EXP_LN2 / 120.0;
+constexpr double EXP_C6 = EXP_LN2 * EXP_LN2 * EXP_LN2 * EXP_LN2 * EXP_LN2 * EXP_LN2 / 720.0;
+
+// Fill a 32-entry shared table with 2^{-j/32} (call before use, then sync).
+__device__ __forceinline__ void exp2_table_init(double *tab) {
+    if (threadIdx.x < 32) tab[threadIdx.x] = exp2(-(double)threadIdx.x / 32.0);
+}
+__device__ __forceinline__ double exp2_neg(double w, const double *tab) {
+    const double big = 0x1.8p52;
+    const double tt = fma(w, 32.0, big);                   // N in the low mantissa bits
+    const int N = (int)(uint32_t)__double_as_longlong(tt);
+    const double r = fma(tt - big, -0.03125, w);           // w - N/32, exact
+    double p = EXP_C6;
+    p = fma(p, r, EXP_C5);
+    p = fma(p, r, EXP_C4);
+    p = fma(p, r, EXP_C3);
+    p = fma(p, r, EXP_C2);
+    p = fma(p, r, EXP_C1);
+    p = fma(p, r, 1.0);
+    const double v = tab[N & 31] * p;
+    return __longlong_as_double(__double_as_longlong(v) - ((long long)(N >> 5) << 52));
 }
 
 // ------------------------------------------------ bounded device waits --

@@ -26,6 +26,8 @@ cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double 
                           double *partials, cudaStream_t st);
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st);
+cudaError_t launch_selftest_math(int which, const double *in, double *out, double *ref, int64_t n,
+                                cudaStream_t st);
 cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st);
 

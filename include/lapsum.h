@@ -163,6 +163,8 @@ LAPSUM_API int lapsum_release(void);
  * distinct kernels.  lapsum_profile_enable(0) stops recording; (2) also clears.
  */
 LAPSUM_API int lapsum_profile_enable(int mode);
+/* Record only launches whose kernel name contains `substring` (NULL or "": all). */
+LAPSUM_API int lapsum_profile_filter(const char *substring);
 LAPSUM_API int lapsum_profile_read(const char **names, int64_t *launches, double *total_ms, int max);
 
 /*
@@ -175,6 +177,16 @@ LAPSUM_API int lapsum_profile_read(const char **names, int64_t *launches, double
  */
 LAPSUM_API int lapsum_bracket_plan(int64_t n, double k, const lapsum_options *opt, int64_t *s,
                                    int64_t *jR, int64_t *jL, int64_t *band_cap);
+
+/*
+ * Self-test of two device math helpers against the CUDA math library, on n
+ * device doubles (no other state touched; synchronous on `stream`):
+ *   which = 0: out = 2^{-in} by the table-driven near-tier exponential used in
+ *              the tail sums (valid for 0 <= in <= 1000), ref = exp2(-in);
+ *   which = 1: out = the sampler's own ln(in) (in > 0, normal), ref = log(in).
+ */
+LAPSUM_API int lapsum_selftest_math(int which, const double *in_dev, double *out_dev,
+                                    double *ref_dev, int64_t n, struct CUstream_st *stream);
 
 /* Number of kernel launches enqueued by this library since load (a counter). */
 LAPSUM_API int64_t lapsum_launch_count(void);
