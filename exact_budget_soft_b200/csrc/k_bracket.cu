@@ -306,7 +306,6 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
 // row -- so the pass stays memory-bound.  Non-finite scores never take it
 // (the float4 bounds use NaN-propagating max and a finite-min check).
 constexpr float NEAR2 = 23.083120654223414f;   // 16 log2(e)
-constexpr float FAR2 = 57.707801635558535f;    // 40 log2(e)
 
 struct Ends {
     float aL, aR, s2;          // s2 = log2(e)/t
@@ -436,6 +435,8 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
 // every score is finite.
 template <bool CERT>
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) oob_kernel(BracketParams P) {
+    static_assert(2 * SBLOCK == BULK_F4, "two vectors per thread per chunk");
+    extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[7 * (SBLOCK / 32)];
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
@@ -452,19 +453,20 @@ __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) oob_kernel(BracketPara
     const bool aligned = (reinterpret_cast<uintptr_t>(P.r) & 15) == 0;
     const int64_t n4 = aligned ? n / 4 : 0;
     const float4 *r4 = reinterpret_cast<const float4 *>(P.r);
-    const int64_t n4w = (n4 + gstride - 1) / gstride * gstride;   // whole warps iterate together
-    int64_t i = gtid;
-    for (; i + gstride < n4w; i += 2 * gstride) {   // two loads in flight
-        const int64_t i0 = CERT ? n4 - 1 - i : i, i1 = CERT ? n4 - 1 - (i + gstride) : i + gstride;
-        const bool ok0 = i < n4, ok1 = i + gstride < n4;
-        const float4 v0 = ok0 ? r4[i0] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 v1 = ok1 ? r4[i1] : make_float4(0.f, 0.f, 0.f, 0.f);
-        oob_vec<CERT>(v0, ok0, E, acc, P, cap, lane);
-        oob_vec<CERT>(v1, ok1, E, acc, P, cap, lane);
+    int64_t done4 = 0;
+    if (aligned) {
+        const float4 *src[1] = {r4};
+        done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
+            oob_vec<CERT>(ch[0][threadIdx.x], true, E, acc, P, cap, lane);
+            oob_vec<CERT>(ch[0][threadIdx.x + SBLOCK], true, E, acc, P, cap, lane);
+        });
     }
-    for (; i < n4w; i += gstride) {
-        const bool ok = i < n4;
-        const float4 v = ok ? r4[CERT ? n4 - 1 - i : i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    // vectors after the last full chunk (whole warps iterate together)
+    const int64_t tv = n4 - done4;
+    const int64_t tvw = (tv + gstride - 1) / gstride * gstride;
+    for (int64_t i = gtid; i < tvw; i += gstride) {
+        const bool ok = i < tv;
+        const float4 v = ok ? r4[done4 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
         oob_vec<CERT>(v, ok, E, acc, P, cap, lane);
     }
     const int64_t rem0 = n4 * 4;
@@ -524,6 +526,7 @@ __device__ __forceinline__ float4 p_vec(const float4 v, const XForm &xf) {
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict__ p,
          double *__restrict__ b_out, Ctl *ctl, double *partials) {
+    extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[SBLOCK / 32];
     const double b = ctl->b;
     const XForm xf = make_xform(b, inv_t * LOG2E);
@@ -534,15 +537,17 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
     const float4 *r4 = reinterpret_cast<const float4 *>(r);
     float4 *p4 = reinterpret_cast<float4 *>(p);
     double ps = 0.0;
-    int64_t i = gtid;
-    for (; i + gstride < n4; i += 2 * gstride) {
-        const float4 v0 = r4[i], v1 = r4[i + gstride];
-        const float4 o0 = p_vec(v0, xf), o1 = p_vec(v1, xf);
-        __stcs(p4 + i, o0);
-        __stcs(p4 + i + gstride, o1);
-        ps += (double)(((o0.x + o0.y) + (o0.z + o0.w)) + ((o1.x + o1.y) + (o1.z + o1.w)));
+    int64_t done4 = 0;
+    if (aligned) {
+        const float4 *src[1] = {r4};
+        done4 = bulk_stream<1>(src, n4, false, dsm, &ctl->status, [&](const float4 *const *ch, int64_t base4) {
+            const float4 o0 = p_vec(ch[0][threadIdx.x], xf), o1 = p_vec(ch[0][threadIdx.x + SBLOCK], xf);
+            __stcs(p4 + base4 + threadIdx.x, o0);
+            __stcs(p4 + base4 + threadIdx.x + SBLOCK, o1);
+            ps += (double)(((o0.x + o0.y) + (o0.z + o0.w)) + ((o1.x + o1.y) + (o1.z + o1.w)));
+        });
     }
-    for (; i < n4; i += gstride) {
+    for (int64_t i = done4 + gtid; i < n4; i += gstride) {
         const float4 o = p_vec(r4[i], xf);
         __stcs(p4 + i, o);
         ps += (double)((o.x + o.y) + (o.z + o.w));
@@ -570,6 +575,7 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                   const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
+    extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[2 * (SBLOCK / 32)];
     const double b = *b_in;
     const XForm xf = make_xform(b, inv_t * LOG2E);
@@ -589,14 +595,15 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
         sgf = fma((double)w.z, (double)e2, sgf);
         sgf = fma((double)w.w, (double)e3, sgf);
     };
-    int64_t i = gtid;
-    for (; i + gstride < n4; i += 2 * gstride) {
-        const int64_t j0 = n4 - 1 - i, j1 = n4 - 1 - (i + gstride);
-        const float4 v0 = r4[j0], w0 = g4[j0], v1 = r4[j1], w1 = g4[j1];
-        acc4(v0, w0);
-        acc4(v1, w1);
+    int64_t done4 = 0;
+    if (aligned) {
+        const float4 *src[2] = {r4, g4};
+        done4 = bulk_stream<2>(src, n4, true, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
+            acc4(ch[0][threadIdx.x], ch[1][threadIdx.x]);
+            acc4(ch[0][threadIdx.x + SBLOCK], ch[1][threadIdx.x + SBLOCK]);
+        });
     }
-    for (; i < n4; i += gstride) acc4(r4[n4 - 1 - i], g4[n4 - 1 - i]);
+    for (int64_t i = done4 + gtid; i < n4; i += gstride) acc4(r4[i], g4[i]);
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
         const float e = exp2f(-fabsf(xf(r[i])));
         sf += (double)e;
@@ -684,6 +691,7 @@ __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                  const float *__restrict__ g, int64_t n, double inv_t, const Ctl *ctl,
                  float *__restrict__ grad) {
+    extern __shared__ __align__(128) unsigned char dsm[];
     const XForm xf = make_xform(*b_in, inv_t * LOG2E);
     const double lam = ctl->vjp_lambda;
     const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
@@ -704,13 +712,17 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
         o.w = vjp_term2(xf(v.w), w.w, hit, lam_hi, lam_lo);
         return o;
     };
-    int64_t i = gtid;
-    for (; i + gstride < n4; i += 2 * gstride) {
-        const float4 v0 = r4[i], w0 = g4[i], v1 = r4[i + gstride], w1 = g4[i + gstride];
-        __stcs(o4 + i, apply4(v0, w0));
-        __stcs(o4 + i + gstride, apply4(v1, w1));
+    int64_t done4 = 0;
+    if (aligned) {
+        const float4 *src[2] = {r4, g4};
+        done4 = bulk_stream<2>(src, n4, false, dsm, const_cast<int32_t *>(&ctl->status),
+                               [&](const float4 *const *ch, int64_t base4) {
+            __stcs(o4 + base4 + threadIdx.x, apply4(ch[0][threadIdx.x], ch[1][threadIdx.x]));
+            __stcs(o4 + base4 + threadIdx.x + SBLOCK,
+                   apply4(ch[0][threadIdx.x + SBLOCK], ch[1][threadIdx.x + SBLOCK]));
+        });
     }
-    for (; i < n4; i += gstride) __stcs(o4 + i, apply4(r4[i], g4[i]));
+    for (int64_t i = done4 + gtid; i < n4; i += gstride) __stcs(o4 + i, apply4(r4[i], g4[i]));
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride)
         grad[i] = vjp_term2(xf(r[i]), g[i], hit, lam_hi, lam_lo);
 }
@@ -754,22 +766,35 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     select_kernel<<<1, 1024, SEL_SMEM, st>>>(P);
     return cudaGetLastError();
 }
+template <typename K>
+static cudaError_t set_smem(K kern, size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
-    oob_kernel<false><<<stream_grid(), SBLOCK, 0, st>>>(P);
+    static cudaError_t once = set_smem(oob_kernel<false>, bulk_smem_bytes<1>());
+    if (once != cudaSuccess) return once;
+    oob_kernel<false><<<stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st>>>(P);
     return cudaGetLastError();
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
-    oob_kernel<true><<<stream_grid(), SBLOCK, 0, st>>>(P);
+    static cudaError_t once = set_smem(oob_kernel<true>, bulk_smem_bytes<1>());
+    if (once != cudaSuccess) return once;
+    oob_kernel<true><<<stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st>>>(P);
     return cudaGetLastError();
 }
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
                           double *partials, cudaStream_t st) {
-    p_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, n, 1.0 / t, p, b_out, ctl, partials);
+    static cudaError_t once = set_smem(p_kernel, bulk_smem_bytes<1>());
+    if (once != cudaSuccess) return once;
+    p_kernel<<<stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st>>>(r, n, 1.0 / t, p, b_out, ctl, partials);
     return cudaGetLastError();
 }
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st) {
-    vjp_reduce_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, partials);
+    static cudaError_t once = set_smem(vjp_reduce_kernel, bulk_smem_bytes<2>());
+    if (once != cudaSuccess) return once;
+    vjp_reduce_kernel<<<stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st>>>(r, b, g, n, 1.0 / t, ctl, partials);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     vjp_shifted_kernel<<<stream_grid() / SBLOCKS_PER_SM, SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, partials);
@@ -777,7 +802,9 @@ cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, i
 }
 cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st) {
-    vjp_apply_kernel<<<stream_grid(), SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, grad);
+    static cudaError_t once = set_smem(vjp_apply_kernel, bulk_smem_bytes<2>());
+    if (once != cudaSuccess) return once;
+    vjp_apply_kernel<<<stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st>>>(r, b, g, n, 1.0 / t, ctl, grad);
     return cudaGetLastError();
 }
 

@@ -266,6 +266,121 @@ __device__ __forceinline__ double exp2_neg(double w, const double *tab) {
     return __longlong_as_double(__double_as_longlong(v) - ((long long)(N >> 5) << 52));
 }
 
+// ------------------------------------------------ bulk-copy pipeline --
+// Streaming passes move the row through shared memory with 1D bulk copies
+// (cp.async.bulk, completion counted in bytes on an mbarrier): each CTA keeps
+// STAGES chunks in flight however many registers its threads need, so the
+// read rate does not hinge on occupancy.  Chunks go to CTAs round-robin (or in
+// reverse, to start on the part of the row a previous pass left in L2); the
+// ragged tail is left to plain loads.  Every wait is bounded.
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait; returns false (and leaves the error to the caller) on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int cap) {
+    for (int it = 0; it < cap; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+constexpr int BULK_F4 = 512;                    // float4 per source per chunk (8 KB)
+constexpr int BULK_WAIT_CAP = 1 << 22;
+// stages in flight: 4 chunks of one source, 3 of two (48 KB per CTA, so four
+// CTAs of either kind fit one SM's shared memory)
+template <int NSRC>
+constexpr int bulk_stages() { return NSRC == 1 ? 4 : 3; }
+
+// Shared memory of a pipeline with NSRC sources (dynamic, 16-byte aligned).
+template <int NSRC>
+constexpr size_t bulk_smem_bytes() {
+    return (size_t)bulk_stages<NSRC>() * NSRC * BULK_F4 * 16 + 64;
+}
+
+// Streams the full chunks of NSRC float4 arrays of n4 vectors through shared
+// memory and calls body(const float4 *chunk[NSRC], int64_t first_vector) once
+// per chunk, by every thread of the CTA (each thread reads its own vectors of
+// the chunk).  Returns the number of vectors covered by full chunks (the rest
+// is the caller's tail).  On a wait that gives up it sets ST_TIMEOUT.
+template <int NSRC, typename Body>
+__device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC], int64_t n4, bool reverse,
+                                               unsigned char *smem, int32_t *status, Body &&body) {
+    constexpr int BULK_STAGES = bulk_stages<NSRC>();
+    float4 *buf = reinterpret_cast<float4 *>(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)BULK_STAGES * NSRC * BULK_F4 * 16);
+    const int64_t nch = n4 / BULK_F4;
+    const int64_t G = gridDim.x;
+    const int64_t mine = nch > blockIdx.x ? (nch - 1 - blockIdx.x) / G + 1 : 0;
+    auto chunk_of = [&](int64_t i) -> int64_t {
+        const int64_t c = blockIdx.x + i * G;
+        return reverse ? nch - 1 - c : c;
+    };
+    constexpr uint32_t BYTES = BULK_F4 * 16;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < BULK_STAGES; ++s) mbar_init(&bars[s], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < BULK_STAGES && s < mine; ++s) {
+            mbar_expect_tx(&bars[s], BYTES * NSRC);
+            const int64_t c = chunk_of(s);
+#pragma unroll
+            for (int q = 0; q < NSRC; ++q)
+                bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &bars[s]);
+        }
+    }
+    bool ok = true;
+    for (int64_t i = 0; i < mine; ++i) {
+        const int s = (int)(i % BULK_STAGES);
+        const uint32_t parity = (uint32_t)((i / BULK_STAGES) & 1);
+        if (!mbar_wait(&bars[s], parity, BULK_WAIT_CAP)) ok = false;
+        const float4 *chunk[NSRC];
+#pragma unroll
+        for (int q = 0; q < NSRC; ++q) chunk[q] = buf + ((size_t)s * NSRC + q) * BULK_F4;
+        body(chunk, chunk_of(i) * BULK_F4);
+        __syncthreads();   // every thread is done with stage s
+        if (threadIdx.x == 0 && i + BULK_STAGES < mine) {
+            fence_proxy_async_smem();
+            mbar_expect_tx(&bars[s], BYTES * NSRC);
+            const int64_t c = chunk_of(i + BULK_STAGES);
+#pragma unroll
+            for (int q = 0; q < NSRC; ++q)
+                bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &bars[s]);
+        }
+    }
+    if (!ok && status) atomicOr(status, ST_TIMEOUT);
+    return nch * BULK_F4;
+}
+
 // ------------------------------------------------ bounded device waits --
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
     unsigned long long v;
