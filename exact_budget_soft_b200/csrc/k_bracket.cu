@@ -25,15 +25,16 @@ constexpr int SBLOCK = 256;     // threads per block of the streaming passes
 constexpr int SBLOCKS_PER_SM = 4;
 
 static int g_num_sms = 0;
-int stream_grid() {
+int stream_grid(int per_sm) {
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (g_num_sms <= 0) g_num_sms = 148;
     }
-    return g_num_sms * SBLOCKS_PER_SM;
+    return g_num_sms * per_sm;
 }
+int stream_grid() { return stream_grid(SBLOCKS_PER_SM); }
 
 // ------------------------------------------------------ last-block combine --
 // Every block contributes NV doubles (valid in thread 0).  The block that
@@ -130,6 +131,7 @@ constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
 // is the fp32 value rounded toward -inf (monotone, so order statistics commute
 // with it), in the descending-order key space.
 __global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
+    pdl_enter();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= P.s) return;
     uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
@@ -186,6 +188,7 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
     extern __shared__ __align__(16) unsigned char sel_smem[];
     uint32_t (*hist)[4096] = reinterpret_cast<uint32_t (*)[4096]>(sel_smem);
     uint32_t (*cand)[SEL_CAND] = reinterpret_cast<uint32_t (*)[SEL_CAND]>(sel_smem + 2 * 4096 * sizeof(uint32_t));
+    pdl_enter();
     __shared__ uint32_t s_w[32];
     __shared__ uint32_t s_pref[2], s_rank[2], s_cnt[2];
     const int tid = threadIdx.x;
@@ -410,6 +413,21 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
         }
         return;
     }
+    // every score of the warp below a_L, some near it: tiered terms only
+    if (__all_sync(FULL, !ok || (mx < E.aL && fin))) {
+        if (ok) {
+            if (CERT) a.cB += 4; else a.cL += 4;
+            double s01 = 0.0, s23 = 0.0;
+            float f01 = 0.f, f23 = 0.f;
+            tier2(E.aL, v.x, E.daL, (double)v.x, E, s01, f01);
+            tier2(E.aL, v.y, E.daL, (double)v.y, E, s01, f01);
+            tier2(E.aL, v.z, E.daL, (double)v.z, E, s23, f23);
+            tier2(E.aL, v.w, E.daL, (double)v.w, E, s23, f23);
+            a.SL += s01 + s23;
+            a.SL2 += f01 + f23;
+        }
+        return;
+    }
     const bool b0 = oob_one<CERT>(v.x, ok, E, a);
     const bool b1 = oob_one<CERT>(v.y, ok, E, a);
     const bool b2 = oob_one<CERT>(v.z, ok, E, a);
@@ -434,12 +452,13 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
 // the band fits its buffer, both passes agree on every membership count, and
 // every score is finite.
 template <bool CERT>
-__global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM) oob_kernel(BracketParams P) {
+__global__ void __launch_bounds__(SBLOCK, CERT ? 3 : SBLOCKS_PER_SM) oob_kernel(BracketParams P) {
     static_assert(2 * SBLOCK == BULK_F4, "two vectors per thread per chunk");
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[7 * (SBLOCK / 32)];
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
+    pdl_enter();
     Ctl *ctl = P.ctl;
     Ends E = make_ends(ctl, P.inv_t);
     E.tab = s_tab;
@@ -528,6 +547,7 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
          double *__restrict__ b_out, Ctl *ctl, double *partials) {
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[SBLOCK / 32];
+    pdl_enter();
     const double b = ctl->b;
     const XForm xf = make_xform(b, inv_t * LOG2E);
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
@@ -577,6 +597,7 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                   const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[2 * (SBLOCK / 32)];
+    pdl_enter();
     const double b = *b_in;
     const XForm xf = make_xform(b, inv_t * LOG2E);
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
@@ -649,6 +670,7 @@ vjp_shifted_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                    const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
     __shared__ ShiftSumG s_w[SBLOCK / 32];
     __shared__ bool s_last;
+    pdl_enter();
     if (!ctl->vjp_shift) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const XForm xf = make_xform(*b_in, inv_t * LOG2E);
@@ -692,6 +714,7 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
                  const float *__restrict__ g, int64_t n, double inv_t, const Ctl *ctl,
                  float *__restrict__ grad) {
     extern __shared__ __align__(128) unsigned char dsm[];
+    pdl_enter();
     const XForm xf = make_xform(*b_in, inv_t * LOG2E);
     const double lam = ctl->vjp_lambda;
     const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
@@ -752,8 +775,7 @@ cudaError_t launch_selftest_math(int which, const double *in, double *out, doubl
 }
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
     const unsigned blocks = (unsigned)((P.s + 255) / 256);
-    sample_kernel<<<blocks, 256, 0, st>>>(P);
-    return cudaGetLastError();
+    return launch_k(sample_kernel, blocks, 256, 0, st, P);
 }
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     static bool attr = false;
@@ -763,8 +785,7 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    select_kernel<<<1, 1024, SEL_SMEM, st>>>(P);
-    return cudaGetLastError();
+    return launch_k(select_kernel, 1, 1024, SEL_SMEM, st, P);
 }
 template <typename K>
 static cudaError_t set_smem(K kern, size_t bytes) {
@@ -774,38 +795,34 @@ static cudaError_t set_smem(K kern, size_t bytes) {
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
     static cudaError_t once = set_smem(oob_kernel<false>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    oob_kernel<false><<<stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st>>>(P);
-    return cudaGetLastError();
+    return launch_k(oob_kernel<false>, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
     static cudaError_t once = set_smem(oob_kernel<true>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    oob_kernel<true><<<stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st>>>(P);
-    return cudaGetLastError();
+    return launch_k(oob_kernel<true>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
                           double *partials, cudaStream_t st) {
     static cudaError_t once = set_smem(p_kernel, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    p_kernel<<<stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st>>>(r, n, 1.0 / t, p, b_out, ctl, partials);
-    return cudaGetLastError();
+    return launch_k(p_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, r, n, 1.0 / t, p, b_out, ctl, partials);
 }
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st) {
     static cudaError_t once = set_smem(vjp_reduce_kernel, bulk_smem_bytes<2>());
     if (once != cudaSuccess) return once;
-    vjp_reduce_kernel<<<stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st>>>(r, b, g, n, 1.0 / t, ctl, partials);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_k(vjp_reduce_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g, n,
+                             1.0 / t, ctl, partials);
     if (e != cudaSuccess) return e;
-    vjp_shifted_kernel<<<stream_grid() / SBLOCKS_PER_SM, SBLOCK, 0, st>>>(r, b, g, n, 1.0 / t, ctl, partials);
-    return cudaGetLastError();
+    return launch_k(vjp_shifted_kernel, stream_grid() / SBLOCKS_PER_SM, SBLOCK, 0, st, r, b, g, n, 1.0 / t, ctl,
+                    partials);
 }
 cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st) {
     static cudaError_t once = set_smem(vjp_apply_kernel, bulk_smem_bytes<2>());
     if (once != cudaSuccess) return once;
-    vjp_apply_kernel<<<stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st>>>(r, b, g, n, 1.0 / t, ctl, grad);
-    return cudaGetLastError();
+    return launch_k(vjp_apply_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g, n, 1.0 / t, ctl, grad);
 }
 
 }  // namespace lapsum

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
     __shared__ uint32_t h[4][256];
     __shared__ bool s_last;
     __shared__ int s_trivial[4];
+    pdl_enter();
     const int64_t n = gated_n(A);
     if (n < 0) return;
     const int tid = threadIdx.x;
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(RB, 1) radix_pass_kernel(SortArgs A, int pass,
     __shared__ int s_tile, s_cur;
     __shared__ bool s_last;
 
+    pdl_enter();
     const int64_t n = gated_n(A);
     if (n < 0) return;
     Ctl *ctl = A.ctl;
@@ -303,6 +305,7 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
     __shared__ bool s_last;
     __shared__ int s_tstar;
 
+    pdl_enter();
     const int64_t n = gated_n(A);
     if (n < 0) return;
     Ctl *ctl = A.ctl;
@@ -465,15 +468,13 @@ cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) 
     if (hg > (int64_t)num_sms() * 2) hg = (int64_t)num_sms() * 2;
     int hgrid = (int)hg;
     if (hgrid < 1) hgrid = 1;
-    radix_hist_kernel<<<hgrid, HB, 0, st>>>(A);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_k(radix_hist_kernel, hgrid, HB, 0, st, A);
     if (e != cudaSuccess) return e;
     int64_t pt = (cap + RTILE - 1) / RTILE;
     if (pt > num_sms()) pt = num_sms();   // persistent: one CTA per SM claims tiles in order
     const unsigned ptiles = (unsigned)pt;
     for (int pass = 0; pass < 4; ++pass) {
-        radix_pass_kernel<<<ptiles, RB, smem, st>>>(A, pass, A.epoch * 4u + (uint32_t)pass);
-        e = cudaGetLastError();
+        e = launch_k(radix_pass_kernel, ptiles, RB, smem, st, A, pass, A.epoch * 4u + (uint32_t)pass);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -491,8 +492,7 @@ cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st
     int64_t lg = (A.cap + LTILE - 1) / LTILE;
     if (lg > num_sms()) lg = num_sms();
     const unsigned grid = (unsigned)lg;
-    locate_kernel<<<grid, LB, smem, st>>>(A, k, t, 1.0 / t);
-    return cudaGetLastError();
+    return launch_k(locate_kernel, grid, LB, smem, st, A, k, t, 1.0 / t);
 }
 
 }  // namespace lapsum

@@ -35,6 +35,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     uint32_t *s_dbase = s_hist + C::NW * 256;
     __shared__ double s_b;
     __shared__ unsigned s_and, s_or;
+    pdl_enter();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int n;
@@ -195,6 +196,7 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
               const float *__restrict__ g, int64_t n, double inv_t, float *__restrict__ grad) {
     __shared__ ShiftSum s_ss[BLOCK / 32];
     __shared__ double s_lam;
+    pdl_enter();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t off = (int64_t)blockIdx.x * n;
     const float *r = scores + off;
@@ -262,8 +264,7 @@ static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n,
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    kern<<<(unsigned)rows, BLOCK, C::SMEM, st>>>(scores, n, k, t, 1.0 / t, p, b, ctl, band_cap);
-    return cudaGetLastError();
+    return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl, band_cap);
 }
 
 int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
@@ -282,8 +283,7 @@ cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl
 
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
                           int64_t n, double t, float *grad, cudaStream_t st) {
-    rowvjp_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, b, g, n, 1.0 / t, grad);
-    return cudaGetLastError();
+    return launch_k(rowvjp_kernel<1024>, (unsigned)rows, 1024, 0, st, scores, b, g, n, 1.0 / t, grad);
 }
 
 }  // namespace lapsum

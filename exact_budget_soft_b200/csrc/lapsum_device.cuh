@@ -381,6 +381,18 @@ __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC],
     return nch * BULK_F4;
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// Every kernel of a solve is launched with programmatic stream serialization:
+// it may be scheduled while its predecessor drains, so it first waits for the
+// predecessor's results (griddepcontrol.wait; a no-op when launched plainly)
+// and then lets its own successor start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+    pdl_wait();
+    pdl_trigger();
+}
+
 // ------------------------------------------------ bounded device waits --
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
     unsigned long long v;
