@@ -40,6 +40,16 @@ EXTRA = ["pixels1m", "laplace1e7"]
 KERNEL_BYTES = {"stream_pass": 4, "certify": 4, "p_pass": 8, "vjp_reduce": 8, "vjp_apply": 12}
 
 
+def kernel_sources_sha() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "exact_budget_soft_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -198,7 +208,9 @@ def run_ours(args):
     traffic = None
     tf = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tf):
-        traffic = json.load(open(tf)).get(dom)
+        rec = json.load(open(tf))
+        if rec.get("sources_sha") == kernel_sources_sha():   # counters only valid for the kernels they came from
+            traffic = rec["kernels"].get(dom)
     model_bytes = sum(KERNEL_BYTES.values()) * w.n
     out = {
         "metric": METRIC, "value": round(med, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
