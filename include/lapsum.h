@@ -188,6 +188,39 @@ LAPSUM_API int lapsum_bracket_plan(int64_t n, double k, const lapsum_options *op
 LAPSUM_API int lapsum_selftest_math(int which, const double *in_dev, double *out_dev,
                                     double *ref_dev, int64_t n, struct CUstream_st *stream);
 
+/*
+ * Backward without any device allocation.  The method's pages have no
+ * counterpart of this entry point: it exists for callers that may not call
+ * cudaMalloc while they run -- for instance code recording work into a CUDA
+ * graph under a strict capture mode (allocation is illegal there), a plugin
+ * inside a host framework that owns all device memory, or a process held to a
+ * fixed memory budget.  lapsum_backward grows a per-stream workspace with
+ * cudaMalloc on first use; this variant keeps its scratch (per-block partial
+ * sums, one lambda and one counter per row) in a single array compiled into
+ * the library, LAPSUM_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ * Result: the same VJP as lapsum_backward, grad_out[i] = (f_i/t)(g_i -
+ * <g,f>/sum f) per row, to within fp32 rounding (not bit-identical: the partial
+ * sums are grouped differently).  Arguments as lapsum_backward; every pointer is
+ * caller-owned device memory; nothing is allocated or freed.
+ *
+ * Limit: rows <= 7281 per call (any n < 2^31).  A call needs about
+ * rows * (24 B + 12 B) of scratch with one block per row, more blocks per row
+ * (and the same total) for fewer rows; a call that would not fit returns
+ * LAPSUM_ERR_ARG before anything is enqueued.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * All calls on a device share the one array: each call clears the counters it
+ * needs, but two calls that overlap on the GPU (different streams, or host
+ * threads) race on it -- order them on one stream.
+ */
+#define LAPSUM_NOALLOC_SCRATCH_BYTES 262144
+LAPSUM_API int lapsum_backward_noalloc(const float *scores_dev, const double *b_dev,
+                                       const float *g_dev, int64_t rows, int64_t n, double t,
+                                       float *grad_out_dev, struct CUstream_st *stream);
+
 /* Number of kernel launches enqueued by this library since load (a counter). */
 LAPSUM_API int64_t lapsum_launch_count(void);
 
