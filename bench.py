@@ -253,6 +253,25 @@ def run_ours(args):
             by_n[f"{we.n:.0e}"] = {"workload": name, "median_ms_fwd_vjp": round(statistics.median(mse), 4)}
         by_n["1e+08"] = {"workload": w.name, "median_ms_fwd_vjp": round(med, 4), "fwd_ms": round(med_f, 4)}
         out["by_n"] = by_n
+    # the same step with the certification folded into the streaming pass
+    opt_fused = L.options(certify=L.CERTIFY_FUSED)
+
+    def step_fused():
+        L.forward(r, w.k, w.t, p_out=p, b_out=b, opts=opt_fused)
+        L.backward(r, b, g, w.t, grad_out=grad)
+
+    ms_fused = time_steps(torch, step_fused, args.steps, args.warmup)
+    st_f = L.get_stats()
+    assert st_f["verdict"] == 1 and st_f["rc"] == 0
+    med_fused = statistics.median(ms_fused)
+    if dist:
+        t = torch.tensor([med_fused], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        med_fused = t.item()
+    out["certify_fused"] = {"median_ms_fwd_vjp": round(med_fused, 4),
+                            "model_frac_of_8TBs": round(32 * w.n / (med_fused * 1e-3) / 8e12, 4),
+                            "note": "option certify=LAPSUM_CERTIFY_FUSED: certification folded into the "
+                                    "streaming pass (32 B/score model)"}
     # end to end through the public API: pinned host buffers in and out every step
     r_h = torch.from_numpy(r_np).pin_memory()
     g_h = torch.from_numpy(g_np).pin_memory()

@@ -24,6 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblapsum.so")
 
 PATH_AUTO, PATH_FULLSORT, PATH_BRACKET = 0, 1, 2
+CERTIFY_PASS, CERTIFY_FUSED = 0, 1
 ERRORS = {0: "ok", -1: "invalid argument", -2: "non-finite score", -3: "workspace allocation failed",
           -4: "device wait timeout", -5: "CUDA runtime error", -6: "no crossing found"}
 
@@ -37,7 +38,7 @@ class LapSumError(RuntimeError):
 class Options(C.Structure):
     _fields_ = [("seed", C.c_uint64), ("sample_size", C.c_int64), ("delta", C.c_double),
                 ("band_cap", C.c_int64), ("spin_cap", C.c_int32), ("force_path", C.c_int32),
-                ("reserved", C.c_int32 * 4)]
+                ("certify", C.c_int32), ("reserved", C.c_int32 * 3)]
 
 
 class Stats(C.Structure):
@@ -116,10 +117,10 @@ def _need(x: torch.Tensor, name: str, dtype=torch.float32):
 
 
 def options(seed: int = 0, sample_size: int = 0, delta: float = 0.0, band_cap: int = 0,
-            spin_cap: int = 0, force_path: int = PATH_AUTO) -> Options:
+            spin_cap: int = 0, force_path: int = PATH_AUTO, certify: int = CERTIFY_PASS) -> Options:
     o = Options()
     o.seed, o.sample_size, o.delta, o.band_cap = seed, sample_size, delta, band_cap
-    o.spin_cap, o.force_path = spin_cap, force_path
+    o.spin_cap, o.force_path, o.certify = spin_cap, force_path, certify
     return o
 
 

@@ -369,9 +369,15 @@ __device__ __forceinline__ void band_push(float x, bool inb, float *band, unsign
     if (inb && base < cap) band[base] = x;
 }
 
-// General path, one score.  Returns "in the band" (streaming mode).
-template <bool CERT>
+// Pass modes: the streaming pass, the certification pass, and the streaming
+// pass with the certification folded in (band scores also add their two
+// certification terms; the verdict comes out of the same pass).
+enum : int { OOB_STREAM = 0, OOB_CERT = 1, OOB_STREAM_CERT = 2 };
+
+// General path, one score.  Returns "in the band" (streaming modes).
+template <int MODE>
 __device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobAcc &a) {
+    constexpr bool CERT = MODE == OOB_CERT;
     if (!valid) return false;
     a.bad |= !(fabsf(x) < CUDART_INF_F);
     if (x >= E.aR) {
@@ -384,8 +390,8 @@ __device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobA
         tier2(E.aL, x, E.daL, (double)x, E, a.SL, a.SL2);
         return false;
     }
-    if (CERT && x == x) {
-        a.cL += 1;
+    if (MODE != OOB_STREAM && x == x) {
+        if (CERT) a.cL += 1;
         tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
         tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
     }
@@ -393,9 +399,10 @@ __device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobA
 }
 
 // One float4 of the pass; `ok` false for padding lanes (whole warps iterate).
-template <bool CERT>
+template <int MODE>
 __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, OobAcc &a,
                                         const BracketParams &P, unsigned long long cap, int lane) {
+    constexpr bool CERT = MODE == OOB_CERT;
     const float mx = max_nan(max_nan(v.x, v.y), max_nan(v.z, v.w));
     const float mn = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
     const bool fin = mn > -CUDART_INF_F;
@@ -428,10 +435,10 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
         }
         return;
     }
-    const bool b0 = oob_one<CERT>(v.x, ok, E, a);
-    const bool b1 = oob_one<CERT>(v.y, ok, E, a);
-    const bool b2 = oob_one<CERT>(v.z, ok, E, a);
-    const bool b3 = oob_one<CERT>(v.w, ok, E, a);
+    const bool b0 = oob_one<MODE>(v.x, ok, E, a);
+    const bool b1 = oob_one<MODE>(v.y, ok, E, a);
+    const bool b2 = oob_one<MODE>(v.z, ok, E, a);
+    const bool b3 = oob_one<MODE>(v.w, ok, E, a);
     if (!CERT && __any_sync(FULL, b0 | b1 | b2 | b3)) {
         unsigned long long *ctr = &P.ctl->c_band;
         band_push(v.x, b0, P.band, cap, ctr, lane);
@@ -451,8 +458,9 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
 // mirror image below); band scores take two.  Verdict: G(a_L) >= k > G(a_R),
 // the band fits its buffer, both passes agree on every membership count, and
 // every score is finite.
-template <bool CERT>
-__global__ void __launch_bounds__(SBLOCK, CERT ? 3 : SBLOCKS_PER_SM) oob_kernel(BracketParams P) {
+template <int MODE>
+__global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 3) oob_kernel(BracketParams P) {
+    constexpr bool CERT = MODE == OOB_CERT;
     static_assert(2 * SBLOCK == BULK_F4, "two vectors per thread per chunk");
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[7 * (SBLOCK / 32)];
@@ -476,8 +484,8 @@ __global__ void __launch_bounds__(SBLOCK, CERT ? 3 : SBLOCKS_PER_SM) oob_kernel(
     if (aligned) {
         const float4 *src[1] = {r4};
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
-            oob_vec<CERT>(ch[0][threadIdx.x], true, E, acc, P, cap, lane);
-            oob_vec<CERT>(ch[0][threadIdx.x + SBLOCK], true, E, acc, P, cap, lane);
+            oob_vec<MODE>(ch[0][threadIdx.x], true, E, acc, P, cap, lane);
+            oob_vec<MODE>(ch[0][threadIdx.x + SBLOCK], true, E, acc, P, cap, lane);
         });
     }
     // vectors after the last full chunk (whole warps iterate together)
@@ -486,18 +494,18 @@ __global__ void __launch_bounds__(SBLOCK, CERT ? 3 : SBLOCKS_PER_SM) oob_kernel(
     for (int64_t i = gtid; i < tvw; i += gstride) {
         const bool ok = i < tv;
         const float4 v = ok ? r4[done4 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        oob_vec<CERT>(v, ok, E, acc, P, cap, lane);
+        oob_vec<MODE>(v, ok, E, acc, P, cap, lane);
     }
     const int64_t rem0 = n4 * 4;
     const int64_t remw = rem0 + ((n - rem0 + gstride - 1) / gstride) * gstride;
     for (int64_t j = rem0 + gtid; j < remw; j += gstride) {
         const bool ok = j < n;
         const float x = ok ? P.r[j] : 0.f;
-        const bool bb = oob_one<CERT>(x, ok, E, acc);
+        const bool bb = oob_one<MODE>(x, ok, E, acc);
         if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane);
     }
     if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
-    if (!CERT) {
+    if constexpr (MODE == OOB_STREAM) {
         double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2};
         block_sum<SBLOCK, 4>(v, s_red);
         if (last_block_sum<SBLOCK, 4>(v, P.partials, &ctl->ticket[0], s_red) && threadIdx.x == 0) {
@@ -505,6 +513,33 @@ __global__ void __launch_bounds__(SBLOCK, CERT ? 3 : SBLOCKS_PER_SM) oob_kernel(
             ctl->c_R = (unsigned long long)v[1];
             ctl->S_L = v[2];
             ctl->S_R = v[3];
+        }
+        return;
+    }
+    if constexpr (MODE == OOB_STREAM_CERT) {
+        double v[6] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2,
+                       acc.hL + (double)acc.hL2, acc.lR + (double)acc.lR2};
+        block_sum<SBLOCK, 6>(v, s_red);
+        if (last_block_sum<SBLOCK, 6>(v, P.partials, &ctl->ticket[0], s_red) && threadIdx.x == 0) {
+            const unsigned long long cL = (unsigned long long)v[0], cR = (unsigned long long)v[1];
+            const unsigned long long cb = ctl->c_band;
+            ctl->c_L = cL;
+            ctl->c_R = cR;
+            ctl->S_L = v[2];
+            ctl->S_R = v[3];
+            // G(a_L), G(a_R) from the same terms: band scores are at or above a_L
+            // and below a_R; out-of-band scores share one term between the ends
+            const double rho = (E.aR == CUDART_INF_F || E.aL == -CUDART_INF_F) ? 0.0
+                                                                               : exp(-(E.daR - E.daL) * E.inv_t);
+            const double GaL = (double)(cb + cR) - 0.5 * fma(rho, v[3], v[4]) + 0.5 * v[2];
+            const double GaR = (double)cR - 0.5 * v[3] + 0.5 * fma(rho, v[2], v[5]);
+            ctl->G_aL = GaL;
+            ctl->G_aR = GaR;
+            const bool ok = (cb <= (unsigned long long)P.band_cap) && (GaL >= P.k) && (GaR < P.k) &&
+                            (cL + cb + cR == (unsigned long long)n) && ((ctl->status & ST_NONFINITE) == 0);
+            ctl->verdict = ok ? 1 : 0;
+            if (!ok) ctl->fallback_ran = 1;
+            if (cb > (unsigned long long)P.band_cap) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
         }
         return;
     }
@@ -793,14 +828,17 @@ static cudaError_t set_smem(K kern, size_t bytes) {
 }
 
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
-    static cudaError_t once = set_smem(oob_kernel<false>, bulk_smem_bytes<1>());
+    static cudaError_t once = set_smem(oob_kernel<OOB_STREAM>, bulk_smem_bytes<1>());
+    static cudaError_t once2 = set_smem(oob_kernel<OOB_STREAM_CERT>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    return launch_k(oob_kernel<false>, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, P);
+    if (once2 != cudaSuccess) return once2;
+    if (P.fused_cert) return launch_k(oob_kernel<OOB_STREAM_CERT>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
+    return launch_k(oob_kernel<OOB_STREAM>, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
-    static cudaError_t once = set_smem(oob_kernel<true>, bulk_smem_bytes<1>());
+    static cudaError_t once = set_smem(oob_kernel<OOB_CERT>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    return launch_k(oob_kernel<true>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
+    return launch_k(oob_kernel<OOB_CERT>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
                           double *partials, cudaStream_t st) {

@@ -324,6 +324,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     if (opt.delta != 0.0 && !(opt.delta > 0.0 && opt.delta < 1.0)) return LAPSUM_ERR_ARG;
     if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < 0) return LAPSUM_ERR_ARG;
     if (opt.force_path < 0 || opt.force_path > 2) return LAPSUM_ERR_ARG;
+    if (opt.certify != LAPSUM_CERTIFY_PASS && opt.certify != LAPSUM_CERTIFY_FUSED) return LAPSUM_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
     const int32_t spin_cap = opt.spin_cap ? opt.spin_cap : (1 << 20);
     Workspace *w = get_ws(st);
@@ -374,6 +375,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     P.s = s;
     P.band_cap = band_cap;
     P.spin_cap = spin_cap;
+    P.fused_cert = opt.certify == LAPSUM_CERTIFY_FUSED;
     LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
     LAPSUM_TRY(grow(w->hist1, w->hist1_n, 4096));
     LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_cap));
@@ -398,7 +400,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         }
         { Launch L("band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
     }
-    { Launch L("certify", st); LAPSUM_TRY(launch_certify(P, st)); }
+    if (!P.fused_cert) { Launch L("certify", st); LAPSUM_TRY(launch_certify(P, st)); }
     rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, st);
     if (rc) return rc;
     { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, st)); }

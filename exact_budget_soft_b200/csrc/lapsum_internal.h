@@ -60,6 +60,7 @@ struct BracketParams {
     double *partials;         // per-block partials
     Ctl *ctl;
     int32_t spin_cap;
+    int32_t fused_cert;       // certification folded into the streaming pass
 };
 
 }  // namespace lapsum

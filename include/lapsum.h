@@ -61,6 +61,10 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
 #define LAPSUM_ERR_CUDA            -5     /* a CUDA runtime call failed                     */
 #define LAPSUM_ERR_NO_ROOT         -6     /* solver found no crossing (internal)            */
 
+/* Certification modes (lapsum_options.certify) */
+#define LAPSUM_CERTIFY_PASS  0
+#define LAPSUM_CERTIFY_FUSED 1
+
 /* Solver paths */
 #define LAPSUM_PATH_AUTO     0
 #define LAPSUM_PATH_FULLSORT 1
@@ -79,6 +83,11 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
  *   spin_cap    polls before an inter-block wait gives up (default 2^20).
  *   force_path  LAPSUM_PATH_* (default AUTO: bracketing when rows == 1 and
  *               n >= 2^20, else full sort).
+ *   certify     LAPSUM_CERTIFY_PASS (default): the certification is its own
+ *               linear pass over the row (the abstract's "one additional linear
+ *               pass"); LAPSUM_CERTIFY_FUSED: the streaming pass also adds the
+ *               band scores' certification terms and decides the verdict, so the
+ *               row is read once less.
  */
 typedef struct {
     uint64_t seed;
@@ -87,7 +96,8 @@ typedef struct {
     int64_t  band_cap;
     int32_t  spin_cap;
     int32_t  force_path;
-    int32_t  reserved[4];
+    int32_t  certify;
+    int32_t  reserved[3];
 } lapsum_options;
 
 /*

@@ -76,7 +76,7 @@ def test_null_pointers_rejected(lib):
 class Options(C.Structure):
     _fields_ = [("seed", C.c_uint64), ("sample_size", C.c_int64), ("delta", C.c_double),
                 ("band_cap", C.c_int64), ("spin_cap", C.c_int32), ("force_path", C.c_int32),
-                ("reserved", C.c_int32 * 4)]
+                ("certify", C.c_int32), ("reserved", C.c_int32 * 3)]
 
 
 def _plan(lib, n, k, s=0, delta=0.0):

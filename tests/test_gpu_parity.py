@@ -124,11 +124,12 @@ def check_bracket_integers(orc, r, k, t, st, seed, s, delta):
     return cert
 
 
+@pytest.mark.parametrize("certify", [0, 1])
 @pytest.mark.parametrize("n,dist,k,t", [(1 << 20, "normal", 1000.0, 0.05), (1_500_001, "laplace", 150.0, 0.01),
                                         (1 << 20, "levels256_desc", 20000.0, 0.1)])
-def test_bracketing_parity(L, orc, n, dist, k, t):
+def test_bracketing_parity(L, orc, n, dist, k, t, certify):
     r, g = W.small_case(dist, 1, n, seed=11)
-    p, b, st, grad = run(L, r, k, t, g_np=g)
+    p, b, st, grad = run(L, r, k, t, opts=L.options(certify=certify), g_np=g)
     assert st["rc"] == 0 and st["path"] == 2
     plan = L.bracket_plan(n, k)
     cert = check_bracket_integers(orc, r[0], k, t, st, 0, plan["s"], 1e-6)
@@ -148,15 +149,17 @@ def test_pixels1m_workload(L, orc):
     check_row(orc, r[0], g[0], w.k, w.t, p[0], b[0], grad[0])
 
 
-def test_forced_fallback_by_band_capacity(L, orc):
+@pytest.mark.parametrize("certify", [0, 1])
+def test_forced_fallback_by_band_capacity(L, orc, certify):
     r, g = W.small_case("normal", 1, 1 << 20, seed=5)
     k, t = 3000.0, 0.05
-    p, b, st, grad = run(L, r, k, t, opts=L.options(band_cap=64), g_np=g)
+    p, b, st, grad = run(L, r, k, t, opts=L.options(band_cap=64, certify=certify), g_np=g)
     assert st["rc"] == 0 and st["verdict"] == 0 and st["fallback"] == 1
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
 
 
-def test_forced_fallback_by_missed_bracket(L, orc):
+@pytest.mark.parametrize("certify", [0, 1])
+def test_forced_fallback_by_missed_bracket(L, orc, certify):
     # a tiny sample with delta = 0.5 misses often; the oracle picks a seed that misses
     r, g = W.small_case("normal", 1, 1 << 20, seed=6)
     k, t, s, delta = 5000.0, 0.05, 256, 0.5
@@ -164,7 +167,8 @@ def test_forced_fallback_by_missed_bracket(L, orc):
     seed = next(sd for sd in range(200)
                 if not (float(orc.bracket(r[0], k, t, sd, s, delta)["a_L"]) <= bref <
                         float(orc.bracket(r[0], k, t, sd, s, delta)["a_R"])))
-    p, b, st, grad = run(L, r, k, t, opts=L.options(seed=seed, sample_size=s, delta=delta), g_np=g)
+    p, b, st, grad = run(L, r, k, t, opts=L.options(seed=seed, sample_size=s, delta=delta, certify=certify),
+                         g_np=g)
     cert = check_bracket_integers(orc, r[0], k, t, st, seed, s, delta)
     assert st["verdict"] == cert["verdict"] == 0 and st["fallback"] == 1
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
