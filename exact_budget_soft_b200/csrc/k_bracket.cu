@@ -108,16 +108,16 @@ __device__ __forceinline__ double sample_ln(double x) {
     }
     double s = __ddiv_rn(__dsub_rn(m, 1.0), __dadd_rn(m, 1.0));
     double z = __dmul_rn(s, s);
-    double p = __ddiv_rn(1.0, 21.0);
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 19.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 17.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 15.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 13.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 11.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 9.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 7.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 5.0));
-    p = __fma_rn(p, z, __ddiv_rn(1.0, 3.0));
+    double p = 1.0 / 21.0;                 // correctly rounded constants, folded by the compiler
+    p = __fma_rn(p, z, 1.0 / 19.0);
+    p = __fma_rn(p, z, 1.0 / 17.0);
+    p = __fma_rn(p, z, 1.0 / 15.0);
+    p = __fma_rn(p, z, 1.0 / 13.0);
+    p = __fma_rn(p, z, 1.0 / 11.0);
+    p = __fma_rn(p, z, 1.0 / 9.0);
+    p = __fma_rn(p, z, 1.0 / 7.0);
+    p = __fma_rn(p, z, 1.0 / 5.0);
+    p = __fma_rn(p, z, 1.0 / 3.0);
     p = __fma_rn(p, z, 1.0);
     double lnm = __dmul_rn(__dadd_rn(s, s), p);
     return __fma_rn((double)e, 0x1.62e42fefa39efp-1, lnm);

@@ -61,6 +61,37 @@ __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
     return A.n_host;
 }
 
+// n copies of one value c, between the seeds of the locate step (the band of a
+// tied level, or a row whose scores are all equal): the threshold curve is
+// constant across the run, G(c) = m0 + n/2 - d_top P_top/2 + d_bot Q_bot/2, and
+// the root lies in [c, top) when G(c) <= k, else in [bot, c).
+__device__ void solve_equal_run(const SortArgs &A, int64_t n) {
+    Ctl *ctl = A.ctl;
+    double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
+    if (A.gate == GATE_BAND) {
+        m0 = (double)ctl->c_R;
+        top = (double)ctl->a_R;
+        P_top = ctl->S_R;
+        bot = (double)ctl->a_L;
+        Q_bot = ctl->S_L;
+    }
+    const double c = (double)A.src[0];
+    const double d_top = top == CUDART_INF ? 0.0 : exp((c - top) / A.t);
+    const double d_bot = bot == -CUDART_INF ? 0.0 : exp((bot - c) / A.t);
+    const double nn = (double)n;
+    const double Gc = m0 + 0.5 * nn - 0.5 * d_top * P_top + 0.5 * d_bot * Q_bot;
+    double b;
+    if (Gc <= A.k) {
+        b = solve_interval(top, c, m0, P_top, nn + d_bot * Q_bot, d_top, A.k, A.t);
+        ctl->j_star = -1;
+    } else {
+        b = solve_interval(c, bot, m0 + nn, nn + d_top * P_top, Q_bot, d_bot, A.k, A.t);
+        ctl->j_star = n - 1;
+    }
+    ctl->b = b;
+    if (A.gate == GATE_FALLBACK) ctl->fallback_ran = 1;
+}
+
 // ------------------------------------------------------------ histogram --
 __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
     __shared__ uint32_t h[4][256];
@@ -128,6 +159,9 @@ __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
     for (int i = tid; i < 4 * 256; i += HB) A.hist[i] = 0ull;   // ready for the next sort
     if (tid == 0) {
         A.ctl->sort_skip = s_trivial[0] | (s_trivial[1] << 1) | (s_trivial[2] << 2) | (s_trivial[3] << 3);
+        const bool all_equal = s_trivial[0] && s_trivial[1] && s_trivial[2] && s_trivial[3];
+        A.ctl->sort_solved = all_equal ? 1 : 0;
+        if (all_equal) solve_equal_run(A, n);
         A.ctl->sort_cur = -1;
         A.ctl->ticket[4] = 0u;
     }
@@ -169,8 +203,8 @@ __global__ void __launch_bounds__(RB, 1) radix_pass_kernel(SortArgs A, int pass,
         __syncthreads();
         const int tile = s_tile;
         if (tile >= ntiles) break;
-        const uint32_t *src = cur >= 0 ? A.keys[cur] : nullptr;
-        uint32_t *dst = A.keys[cur >= 0 ? (cur ^ 1) : 0];
+        const uint32_t *src = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
+        uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
         const int64_t base = (int64_t)tile * RTILE;
         const int cnt_tile = (int)min((int64_t)RTILE, n - base);
         for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
@@ -294,8 +328,8 @@ struct TileRec {
     double pad;
 };
 
-__device__ __forceinline__ double sorted_val(const SortArgs &A, int cur, int64_t j) {
-    return cur >= 0 ? (double)desc_key_to_float(A.keys[cur][j]) : (double)A.src[j];
+__device__ __forceinline__ double sorted_val(const uint32_t *keys, const float *src, int64_t j) {
+    return keys ? (double)desc_key_to_float(keys[j]) : (double)src[j];
 }
 
 __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, double t, double inv_t) {
@@ -304,13 +338,19 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
     void *scratch = smem + LTILE * 4;                                        // >= 6 KB
     __shared__ bool s_last;
     __shared__ int s_tstar;
+    __shared__ double s_tab[32];
+    exp2_table_init(s_tab);
 
     pdl_enter();
     const int64_t n = gated_n(A);
     if (n < 0) return;
     Ctl *ctl = A.ctl;
+    if (ctl->sort_solved) return;   // every key equal: solved by the histogram kernel
     const int tid = threadIdx.x, lane = tid & 31;
     const int cur = ctl->sort_cur;
+    const uint32_t *keys_cur = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
+    const double s2d = inv_t * LOG2E;
+    __syncthreads();   // s_tab
     double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
     if (A.gate == GATE_BAND) {
         m0 = (double)ctl->c_R;
@@ -324,7 +364,7 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
     auto val = [&](int64_t j) -> double {
         if (j < 0) return top;
         if (j >= n) return bot;
-        return sorted_val(A, cur, j);
+        return sorted_val(keys_cur, A.src, j);
     };
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int64_t j0 = tile * LTILE + (int64_t)tid * LK;
@@ -334,11 +374,11 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
         if (j0 < n) {
             double cprev = val(j0 - 1);
             double c = val(j0);
-            double dprev = (cprev == CUDART_INF || c == -CUDART_INF) ? 0.0 : exp((c - cprev) * inv_t);
+            double dprev = (cprev == CUDART_INF || c == -CUDART_INF) ? 0.0 : link_exp((cprev - c) * s2d, s_tab);
             for (int64_t j = j0; j <= j1; ++j) {
                 mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
                 const double cn = val(j + 1);
-                const double d = (c == CUDART_INF || cn == -CUDART_INF) ? 0.0 : exp((cn - c) * inv_t);
+                const double d = (c == CUDART_INF || cn == -CUDART_INF) ? 0.0 : link_exp((c - cn) * s2d, s_tab);
                 mq = {mq.a * d, mq.s + mq.a};
                 dprev = d;
                 c = cn;
@@ -422,7 +462,7 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
     const int64_t t0 = TT * LTILE;
     const int cnt = (int)min((int64_t)LTILE, n - t0);
     for (int i = tid; i < cnt; i += LB) {
-        s_keys[i] = cur >= 0 ? A.keys[cur][t0 + i] : desc_key(A.src[t0 + i]);
+        s_keys[i] = keys_cur ? keys_cur[t0 + i] : desc_key(A.src[t0 + i]);
     }
     __syncthreads();
     const double ptop = TT == 0 ? P_top : __ldcg(&rec[TT - 1].p_end);
@@ -431,7 +471,7 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
     const double vbot = val(t0 + cnt);
     int64_t js = 0;
     const double b = block_scan_solve<LB, LK>(s_keys, cnt, k, t, inv_t, m0 + (double)t0, vtop, ptop,
-                                              vbot, qbot, scratch, &js, &ctl->status);
+                                              vbot, qbot, scratch, &js, &ctl->status, s_tab);
     if (tid == 0) {
         ctl->b = b;
         ctl->j_star = t0 + js;

@@ -35,6 +35,8 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     uint32_t *s_dbase = s_hist + C::NW * 256;
     __shared__ double s_b;
     __shared__ unsigned s_and, s_or;
+    __shared__ double s_tab[32];
+    exp2_table_init(s_tab);
     pdl_enter();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -60,6 +62,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
         row = scores + (int64_t)blockIdx.x * n_arg;
     }
 
+    __syncthreads();   // s_tab
     if (n == 0) {   // band mode only: one interval [a_L, a_R] with no score inside
         if (tid == 0) {
             double ed = (top == CUDART_INF || bot == -CUDART_INF) ? 0.0 : exp((bot - top) * inv_t);
@@ -105,7 +108,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     int64_t jstar = 0;
     int32_t *st = ctl ? &ctl->status : nullptr;
     double b = block_scan_solve<BLOCK, KPT>(s_keys, n, k, t, inv_t, m0, top, P_top, bot, Q_bot,
-                                            s_hist, (BAND || blockIdx.x == 0) ? &jstar : nullptr, st);
+                                            s_hist, (BAND || blockIdx.x == 0) ? &jstar : nullptr, st, s_tab);
     if (tid == 0) {
         s_b = b;
         if (BAND) {

@@ -152,8 +152,10 @@ cudaError_t ws_sort(Workspace *w, int64_t cap) {
 }
 
 SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32_t gate,
-                   int32_t spin_cap) {
+                   int32_t spin_cap, double k, double t) {
     SortArgs A{};
+    A.k = k;
+    A.t = t;
     A.src = src;
     A.n_host = n;
     A.cap = cap;
@@ -282,7 +284,7 @@ int check_args(const float *scores, int64_t rows, int64_t n, double k, double t)
 int full_sort_row(Workspace *w, const float *r, int64_t n, double k, double t, int32_t gate,
                   int32_t spin_cap, cudaStream_t st) {
     LAPSUM_TRY(ws_sort(w, n));
-    SortArgs A = sort_args(w, r, n, n, gate, spin_cap);
+    SortArgs A = sort_args(w, r, n, n, gate, spin_cap, k, t);
     {
         Launch L("radix_sort(5 kernels)", st);
         g_launches += 4;
@@ -392,7 +394,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     { Launch L("stream_pass", st); LAPSUM_TRY(launch_stream_pass(P, st)); }
     { Launch L("band_rowsolve", st); LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st)); }
     if (band_cap > rowsolve_capacity()) {
-        SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap);
+        SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap, k, t);
         {
             Launch L("band_radix_sort(5 kernels)", st);
             g_launches += 4;

@@ -266,6 +266,12 @@ __device__ __forceinline__ double exp2_neg(double w, const double *tab) {
     return __longlong_as_double(__double_as_longlong(v) - ((long long)(N >> 5) << 52));
 }
 
+// A link of the threshold curve, e^{-(hi - lo)/t} = 2^{-w}, w = (hi - lo) log2(e)/t >= 0
+// (w > 1000 is below 2^{-1000}: zero for every sum it enters).
+__device__ __forceinline__ double link_exp(double w, const double *tab) {
+    return w <= 1000.0 ? exp2_neg(w, tab) : 0.0;
+}
+
 // ------------------------------------------------ bulk-copy pipeline --
 // Streaming passes move the row through shared memory with 1D bulk copies
 // (cp.async.bulk, completion counted in bytes on an mbarrier): each CTA keeps

@@ -38,6 +38,7 @@ struct Ctl {
     // radix sort: which buffer holds the current keys (-1: the fp32 source)
     int32_t sort_cur;
     int32_t sort_skip;        // bit d: every key agrees on digit d (pass skipped)
+    int32_t sort_solved;      // every key equal: solved without the locate step
     unsigned int tile_ctr[4];
     // backward
     double vjp_lambda;

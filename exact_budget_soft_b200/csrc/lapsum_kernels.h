@@ -65,6 +65,7 @@ struct SortArgs {
     int32_t spin_cap;
     uint32_t epoch;            // distinct per launch sequence (look-back tags)
     int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
+    double k, t;               // budget and temperature (all-equal shortcut)
 };
 int radix_tile();
 int locate_tile();

@@ -110,7 +110,9 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
 template <int BLOCK, int KPT>
 __device__ double block_scan_solve(const uint32_t *s_keys, int n, double k, double t, double inv_t,
                                    double m0, double top, double P_top, double bot, double Q_bot,
-                                   void *scratch_v, int64_t *j_star_out, int32_t *status) {
+                                   void *scratch_v, int64_t *j_star_out, int32_t *status,
+                                   const double *tab) {
+    const double s2d = inv_t * LOG2E;
     constexpr int R = KPT;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     Aff *sc = reinterpret_cast<Aff *>(scratch_v);               // 2*NW Aff
@@ -126,7 +128,7 @@ __device__ double block_scan_solve(const uint32_t *s_keys, int n, double k, doub
     auto link = [&](int j) -> double {
         double hi = val(j), lo = val(j + 1);
         if (hi == CUDART_INF || lo == -CUDART_INF) return 0.0;
-        return exp((lo - hi) * inv_t);
+        return link_exp((hi - lo) * s2d, tab);
     };
 
     const int j0 = tid * R;
@@ -140,7 +142,7 @@ __device__ double block_scan_solve(const uint32_t *s_keys, int n, double k, doub
         for (int j = j0; j <= j1; ++j) {
             mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
             double cn = val(j + 1);
-            double d = (cprev == CUDART_INF || cn == -CUDART_INF) ? 0.0 : exp((cn - cprev) * inv_t);
+            double d = (cprev == CUDART_INF || cn == -CUDART_INF) ? 0.0 : link_exp((cprev - cn) * s2d, tab);
             // append Q-map of j on the right: T(x) = A(1 + d x) + S
             mq = {mq.a * d, mq.s + mq.a};
             dprev = d;
