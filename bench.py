@@ -164,6 +164,9 @@ def run_ours(args):
     step()
     st = L.get_stats()
     assert st["path"] == 2 and st["rc"] == 0
+    # gross sanity of the timed configuration (exact parity is the tests' job): the
+    # sum of the returned p must be within its fp32 rounding of the budget
+    assert abs(st["sum_p"] - w.k) < 1.0 + 1e-7 * w.n, st
 
     # per-kernel breakdown: a short calibration run with every launch bracketed
     L.profile_filter(None)
@@ -262,7 +265,7 @@ def run_ours(args):
 
     ms_fused = time_steps(torch, step_fused, args.steps, args.warmup)
     st_f = L.get_stats()
-    assert st_f["verdict"] == 1 and st_f["rc"] == 0
+    assert st_f["verdict"] == 1 and st_f["rc"] == 0 and abs(st_f["sum_p"] - w.k) < 1.0 + 1e-7 * w.n
     med_fused = statistics.median(ms_fused)
     if dist:
         t = torch.tensor([med_fused], device="cuda", dtype=torch.float64)

@@ -64,7 +64,7 @@ __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
 // n copies of one value c, between the seeds of the locate step (the band of a
 // tied level, or a row whose scores are all equal): the threshold curve is
 // constant across the run, G(c) = m0 + n/2 - d_top P_top/2 + d_bot Q_bot/2, and
-// the root lies in [c, top) when G(c) <= k, else in [bot, c).
+// (G decreasing) the root lies in [bot, c] when G(c) <= k, else in [c, top).
 __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
     Ctl *ctl = A.ctl;
     double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
@@ -81,12 +81,12 @@ __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
     const double nn = (double)n;
     const double Gc = m0 + 0.5 * nn - 0.5 * d_top * P_top + 0.5 * d_bot * Q_bot;
     double b;
-    if (Gc <= A.k) {
-        b = solve_interval(top, c, m0, P_top, nn + d_bot * Q_bot, d_top, A.k, A.t);
-        ctl->j_star = -1;
-    } else {
+    if (Gc <= A.k) {   // G decreasing: the root is at or below c
         b = solve_interval(c, bot, m0 + nn, nn + d_top * P_top, Q_bot, d_bot, A.k, A.t);
         ctl->j_star = n - 1;
+    } else {
+        b = solve_interval(top, c, m0, P_top, nn + d_bot * Q_bot, d_top, A.k, A.t);
+        ctl->j_star = -1;
     }
     ctl->b = b;
     if (A.gate == GATE_FALLBACK) ctl->fallback_ran = 1;

@@ -249,3 +249,19 @@ def test_levels1e8_workload_and_forced_fallback(L, orc):
     assert np.float32(st2["a_L"]) == np.float32(gold["a_L"]) and np.float32(st2["a_R"]) == np.float32(gold["a_R"])
     assert (st2["c_L"], st2["c_band"], st2["c_R"]) == (gold["c_L"], gold["c_band"], gold["c_R"])
     check_large(orc, r, None, w.k, w.t, p2, b2[0], None, rng)
+
+
+@pytest.mark.parametrize("certify", [0, 1])
+@pytest.mark.parametrize("level", [0, 1, 2])
+def test_bracketing_band_of_one_tied_level(L, orc, level, certify):
+    # sorted, 64 tied levels: the band holds one whole level (or none), which the
+    # histogram kernel solves in closed form when it exceeds one CTA
+    n = 1 << 21
+    vals = (-1.0 + (np.arange(64) + 0.5) / 32).astype(np.float32)
+    r = np.repeat(vals[::-1], n // 64)[None, :].copy()
+    g = np.random.default_rng(level).standard_normal((1, n)).astype(np.float32)
+    k = [n / 64 * 1.5, n / 64 * 3.25, n / 64 * 0.4][level]
+    t = 0.05
+    p, b, st, grad = run(L, r, k, t, opts=L.options(certify=certify), g_np=g)
+    assert st["rc"] == 0 and st["path"] == 2
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0], exact_sum=False)
