@@ -254,13 +254,13 @@ def test_levels1e8_workload_and_forced_fallback(L, orc):
 @pytest.mark.parametrize("certify", [0, 1])
 @pytest.mark.parametrize("level", [0, 1, 2])
 def test_bracketing_band_of_one_tied_level(L, orc, level, certify):
-    # sorted, 64 tied levels: the band holds one whole level (or none), which the
-    # histogram kernel solves in closed form when it exceeds one CTA
+    # sorted, 32 tied levels of 65536 scores: the band holds one whole level (or
+    # none); one level exceeds one CTA, so the histogram kernel solves it in closed form
     n = 1 << 21
-    vals = (-1.0 + (np.arange(64) + 0.5) / 32).astype(np.float32)
-    r = np.repeat(vals[::-1], n // 64)[None, :].copy()
+    vals = (-1.0 + (np.arange(32) + 0.5) / 16).astype(np.float32)
+    r = np.repeat(vals[::-1], n // 32)[None, :].copy()
     g = np.random.default_rng(level).standard_normal((1, n)).astype(np.float32)
-    k = [n / 64 * 1.5, n / 64 * 3.25, n / 64 * 0.4][level]
+    k = [n / 32 * 1.5, n / 32 * 3.25, n / 32 * 0.4][level]
     t = 0.05
     p, b, st, grad = run(L, r, k, t, opts=L.options(certify=certify), g_np=g)
     assert st["rc"] == 0 and st["path"] == 2
