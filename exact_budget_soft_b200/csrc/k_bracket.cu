@@ -426,10 +426,16 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
             if (CERT) a.cB += 4; else a.cL += 4;
             double s01 = 0.0, s23 = 0.0;
             float f01 = 0.f, f23 = 0.f;
-            tier2(E.aL, v.x, E.daL, (double)v.x, E, s01, f01);
-            tier2(E.aL, v.y, E.daL, (double)v.y, E, s01, f01);
-            tier2(E.aL, v.z, E.daL, (double)v.z, E, s23, f23);
-            tier2(E.aL, v.w, E.daL, (double)v.w, E, s23, f23);
+            if (mx == mn) {   // four equal scores (sorted or quantised rows): one term, four times
+                tier2(E.aL, v.x, E.daL, (double)v.x, E, s01, f01);
+                s01 *= 4.0;
+                f01 *= 4.0f;
+            } else {
+                tier2(E.aL, v.x, E.daL, (double)v.x, E, s01, f01);
+                tier2(E.aL, v.y, E.daL, (double)v.y, E, s01, f01);
+                tier2(E.aL, v.z, E.daL, (double)v.z, E, s23, f23);
+                tier2(E.aL, v.w, E.daL, (double)v.w, E, s23, f23);
+            }
             a.SL += s01 + s23;
             a.SL2 += f01 + f23;
         }
