@@ -399,20 +399,75 @@ __device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobA
 }
 
 // One float4 of the pass; `ok` false for padding lanes (whole warps iterate).
+// Tail terms of a float4 against one end a: e^{-(x-a)/t} (UP) or e^{-(a-x)/t};
+// four equal scores take one term.
+template <bool UP>
+__device__ __forceinline__ void tier4(const float4 v, bool equal, float af, double ad, const Ends &E,
+                                      double &acc64, float &acc32) {
+    double s01 = 0.0, s23 = 0.0;
+    float f01 = 0.f, f23 = 0.f;
+    auto one = [&](float x, double &s, float &f) {
+        if (UP) tier2(x, af, (double)x, ad, E, s, f);
+        else    tier2(af, x, ad, (double)x, E, s, f);
+    };
+    if (equal) {
+        one(v.x, s01, f01);
+        s01 *= 4.0;
+        f01 *= 4.0f;
+    } else {
+        one(v.x, s01, f01);
+        one(v.y, s01, f01);
+        one(v.z, s23, f23);
+        one(v.w, s23, f23);
+    }
+    acc64 += s01 + s23;
+    acc32 += f01 + f23;
+}
+
+// Append the band scores of a float4 (bit i of m: component i) at consecutive
+// slots: one warp scan and one atomic per warp (the count keeps going past the
+// capacity so the overflow is visible).
+__device__ __forceinline__ void band_push4(const float4 v, int m, float *band, unsigned long long cap,
+                                           unsigned long long *ctr, int lane) {
+    const int cnt = __popc(m);
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int p = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += p;
+    }
+    const int total = __shfl_sync(FULL, inc, 31);
+    if (total == 0) return;
+    unsigned long long base = 0;
+    if (lane == 31) base = atomicAdd(ctr, (unsigned long long)total);
+    base = __shfl_sync(FULL, base, 31) + (unsigned long long)(inc - cnt);
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (m & (1 << i)) {
+            if (base < cap) band[base] = vv[i];
+            ++base;
+        }
+    }
+}
+
+// One float4 of the pass; `ok` false for padding lanes (whole warps iterate).
+// Warp-uniform fast paths for float4s wholly far below a_L, wholly below it,
+// wholly at or above a_R, or wholly inside the band; the general path otherwise.
 template <int MODE>
 __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, OobAcc &a,
                                         const BracketParams &P, unsigned long long cap, int lane) {
     constexpr bool CERT = MODE == OOB_CERT;
+    constexpr bool BANDTERMS = MODE != OOB_STREAM;
     const float mx = max_nan(max_nan(v.x, v.y), max_nan(v.z, v.w));
     const float mn = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
-    const bool fin = mn > -CUDART_INF_F;
-    const bool far = !ok || (mx < E.farL && fin);
-    const bool mid = !ok || (mx < E.midL && fin);
-    if (__all_sync(FULL, far)) {
+    const bool fin = mn > -CUDART_INF_F && mx < CUDART_INF_F;    // false for NaN too
+    const bool equal = mx == mn;
+    if (__all_sync(FULL, !ok || (mx < E.farL && fin))) {
         if (ok) { if (CERT) a.cB += 4; else a.cL += 4; }
         return;
     }
-    if (__all_sync(FULL, mid)) {
+    if (__all_sync(FULL, !ok || (mx < E.midL && fin))) {
         if (ok) {
             if (CERT) a.cB += 4; else a.cL += 4;
             a.SL2 += (ex2_ftz((v.x - E.aL) * E.s2) + ex2_ftz((v.y - E.aL) * E.s2)) +
@@ -420,37 +475,36 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
         }
         return;
     }
-    // every score of the warp below a_L, some near it: tiered terms only
-    if (__all_sync(FULL, !ok || (mx < E.aL && fin))) {
+    if (__all_sync(FULL, !ok || (mx < E.aL && fin))) {            // below a_L, some near it
         if (ok) {
             if (CERT) a.cB += 4; else a.cL += 4;
-            double s01 = 0.0, s23 = 0.0;
-            float f01 = 0.f, f23 = 0.f;
-            if (mx == mn) {   // four equal scores (sorted or quantised rows): one term, four times
-                tier2(E.aL, v.x, E.daL, (double)v.x, E, s01, f01);
-                s01 *= 4.0;
-                f01 *= 4.0f;
-            } else {
-                tier2(E.aL, v.x, E.daL, (double)v.x, E, s01, f01);
-                tier2(E.aL, v.y, E.daL, (double)v.y, E, s01, f01);
-                tier2(E.aL, v.z, E.daL, (double)v.z, E, s23, f23);
-                tier2(E.aL, v.w, E.daL, (double)v.w, E, s23, f23);
-            }
-            a.SL += s01 + s23;
-            a.SL2 += f01 + f23;
+            tier4<false>(v, equal, E.aL, E.daL, E, a.SL, a.SL2);
         }
+        return;
+    }
+    if (__all_sync(FULL, !ok || (mn >= E.aR && fin))) {           // at or above a_R
+        if (ok) {
+            if (CERT) { a.cL += 4; a.cR += 4; } else a.cR += 4;
+            tier4<true>(v, equal, E.aR, E.daR, E, a.SR, a.SR2);
+        }
+        return;
+    }
+    if (__all_sync(FULL, !ok || (mn >= E.aL && mx < E.aR && fin))) {   // inside the band
+        if (ok && BANDTERMS) {
+            if (CERT) a.cL += 4;
+            tier4<true>(v, equal, E.aL, E.daL, E, a.hL, a.hL2);
+            tier4<false>(v, equal, E.aR, E.daR, E, a.lR, a.lR2);
+        }
+        if (!CERT) band_push4(v, ok ? 0xF : 0, P.band, cap, &P.ctl->c_band, lane);
         return;
     }
     const bool b0 = oob_one<MODE>(v.x, ok, E, a);
     const bool b1 = oob_one<MODE>(v.y, ok, E, a);
     const bool b2 = oob_one<MODE>(v.z, ok, E, a);
     const bool b3 = oob_one<MODE>(v.w, ok, E, a);
-    if (!CERT && __any_sync(FULL, b0 | b1 | b2 | b3)) {
-        unsigned long long *ctr = &P.ctl->c_band;
-        band_push(v.x, b0, P.band, cap, ctr, lane);
-        band_push(v.y, b1, P.band, cap, ctr, lane);
-        band_push(v.z, b2, P.band, cap, ctr, lane);
-        band_push(v.w, b3, P.band, cap, ctr, lane);
+    if (!CERT) {
+        const int m = (b0 ? 1 : 0) | (b1 ? 2 : 0) | (b2 ? 4 : 0) | (b3 ? 8 : 0);
+        if (__any_sync(FULL, m != 0)) band_push4(v, m, P.band, cap, &P.ctl->c_band, lane);
     }
 }
 
