@@ -130,24 +130,32 @@ constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
 // This is the operator's own noise kernel, so P(y_j > b) = k/n.  The key kept
 // is the fp32 value rounded toward -inf (monotone, so order statistics commute
 // with it), in the descending-order key space.
-__global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
+__global__ void __launch_bounds__(1024) sample_kernel(BracketParams P) {
+    __shared__ uint32_t s_hist[4096];   // first radix-select round: top 12 key bits
+    for (int i = threadIdx.x; i < 4096; i += blockDim.x) s_hist[i] = 0u;
     pdl_enter();
+    __syncthreads();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= P.s) return;
-    uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
-    philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
-    const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
-    const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
-    const double E = -sample_ln(U);
-    const double L = (x1 & 1ull) ? E : -E;
-    const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
-    const uint32_t key = desc_key(__double2float_rd(y));
-    P.keys[j] = key;
-    // first radix-select round: histogram of the top 12 key bits (warp-aggregated)
-    const uint32_t bin = key >> 20;
-    const unsigned act = __activemask();
-    const unsigned peers = __match_any_sync(act, bin);
-    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
+    if (j < P.s) {
+        uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
+        philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
+        const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
+        const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
+        const double E = -sample_ln(U);
+        const double L = (x1 & 1ull) ? E : -E;
+        const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
+        const uint32_t key = desc_key(__double2float_rd(y));
+        P.keys[j] = key;
+        const uint32_t bin = key >> 20;
+        const unsigned act = __activemask();
+        const unsigned peers = __match_any_sync(act, bin);
+        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 4096; i += blockDim.x) {
+        const uint32_t c = s_hist[i];
+        if (c) atomicAdd(P.hist1 + i, c);
+    }
 }
 
 // ================================================================ select --
@@ -191,7 +199,7 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
     pdl_enter();
     __shared__ uint32_t s_w[32];
     __shared__ uint32_t s_pref[2], s_rank[2], s_cnt[2];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int s = (int)P.s;
     const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
     if (tid == 0) {
@@ -268,14 +276,18 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
         if (rd == 0) {
             // keep the keys under each target's 12-bit prefix in shared memory
             const uint32_t pf[2] = {s_pref[0], s_pref[1]};
-            for (int i = tid; i < s; i += 1024) {
-                const uint32_t key = P.keys[i];
+            for (int i0 = 0; i0 < s; i0 += 1024) {
+                const int i = i0 + tid;
+                const uint32_t key = i < s ? P.keys[i] : 0u;
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    if (valid[q] && (key & mask) == pf[q]) {
-                        const uint32_t pos = atomicAdd(&s_cnt[q], 1u);
-                        if (pos < SEL_CAND) cand[q][pos] = key;
-                    }
+                    const bool m = i < s && valid[q] && (key & mask) == pf[q];
+                    const unsigned bal = __ballot_sync(FULL, m);
+                    if (!bal) continue;
+                    uint32_t base = 0;
+                    if (lane == __ffs(bal) - 1) base = atomicAdd(&s_cnt[q], (uint32_t)__popc(bal));
+                    base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+                    if (m && base < SEL_CAND) cand[q][base] = key;
                 }
             }
             __syncthreads();
@@ -869,8 +881,8 @@ cudaError_t launch_selftest_math(int which, const double *in, double *out, doubl
     return cudaGetLastError();
 }
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
-    const unsigned blocks = (unsigned)((P.s + 255) / 256);
-    return launch_k(sample_kernel, blocks, 256, 0, st, P);
+    const unsigned blocks = (unsigned)((P.s + 1023) / 1024);
+    return launch_k(sample_kernel, blocks, 1024, 0, st, P);
 }
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     static bool attr = false;
