@@ -276,12 +276,10 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
         if (rd == 0) {
             // keep the keys under each target's 12-bit prefix in shared memory
             const uint32_t pf[2] = {s_pref[0], s_pref[1]};
-            for (int i0 = 0; i0 < s; i0 += 1024) {
-                const int i = i0 + tid;
-                const uint32_t key = i < s ? P.keys[i] : 0u;
+            auto take = [&](uint32_t key, bool in) {
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    const bool m = i < s && valid[q] && (key & mask) == pf[q];
+                    const bool m = in && valid[q] && (key & mask) == pf[q];
                     const unsigned bal = __ballot_sync(FULL, m);
                     if (!bal) continue;
                     uint32_t base = 0;
@@ -289,6 +287,29 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
                     base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
                     if (m && base < SEL_CAND) cand[q][base] = key;
                 }
+            };
+            const uint4 *k4 = reinterpret_cast<const uint4 *>(P.keys);
+            const int s4 = s / 4;
+            for (int i0 = 0; i0 < s4; i0 += 4 * 1024) {   // four 16-byte loads in flight per thread
+                uint4 kv[4];
+                bool in[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + u * 1024 + tid;
+                    in[u] = i < s4;
+                    kv[u] = in[u] ? k4[i] : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    take(kv[u].x, in[u]);
+                    take(kv[u].y, in[u]);
+                    take(kv[u].z, in[u]);
+                    take(kv[u].w, in[u]);
+                }
+            }
+            for (int i0 = 4 * s4; i0 < s; i0 += 1024) {
+                const int i = i0 + tid;
+                take(i < s ? P.keys[i] : 0u, i < s);
             }
             __syncthreads();
             fast[0] = s_cnt[0] <= SEL_CAND;
@@ -556,8 +577,8 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     if (aligned) {
         const float4 *src[1] = {r4};
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
-            oob_vec<MODE>(ch[0][threadIdx.x], true, E, acc, P, cap, lane);
-            oob_vec<MODE>(ch[0][threadIdx.x + SBLOCK], true, E, acc, P, cap, lane);
+            oob_vec<MODE>(lds128(ch[0] + threadIdx.x), true, E, acc, P, cap, lane);
+            oob_vec<MODE>(lds128(ch[0] + threadIdx.x + SBLOCK), true, E, acc, P, cap, lane);
         });
     }
     // vectors after the last full chunk (whole warps iterate together)
@@ -668,7 +689,7 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
     if (aligned) {
         const float4 *src[1] = {r4};
         done4 = bulk_stream<1>(src, n4, false, dsm, &ctl->status, [&](const float4 *const *ch, int64_t base4) {
-            const float4 o0 = p_vec(ch[0][threadIdx.x], xf), o1 = p_vec(ch[0][threadIdx.x + SBLOCK], xf);
+            const float4 o0 = p_vec(lds128(ch[0] + threadIdx.x), xf), o1 = p_vec(lds128(ch[0] + threadIdx.x + SBLOCK), xf);
             __stcs(p4 + base4 + threadIdx.x, o0);
             __stcs(p4 + base4 + threadIdx.x + SBLOCK, o1);
             ps += (double)(((o0.x + o0.y) + (o0.z + o0.w)) + ((o1.x + o1.y) + (o1.z + o1.w)));
@@ -727,8 +748,8 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
     if (aligned) {
         const float4 *src[2] = {r4, g4};
         done4 = bulk_stream<2>(src, n4, true, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
-            acc4(ch[0][threadIdx.x], ch[1][threadIdx.x]);
-            acc4(ch[0][threadIdx.x + SBLOCK], ch[1][threadIdx.x + SBLOCK]);
+            acc4(lds128(ch[0] + threadIdx.x), lds128(ch[1] + threadIdx.x));
+            acc4(lds128(ch[0] + threadIdx.x + SBLOCK), lds128(ch[1] + threadIdx.x + SBLOCK));
         });
     }
     for (int64_t i = done4 + gtid; i < n4; i += gstride) acc4(r4[i], g4[i]);
@@ -847,9 +868,9 @@ vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
         const float4 *src[2] = {r4, g4};
         done4 = bulk_stream<2>(src, n4, false, dsm, const_cast<int32_t *>(&ctl->status),
                                [&](const float4 *const *ch, int64_t base4) {
-            __stcs(o4 + base4 + threadIdx.x, apply4(ch[0][threadIdx.x], ch[1][threadIdx.x]));
+            __stcs(o4 + base4 + threadIdx.x, apply4(lds128(ch[0] + threadIdx.x), lds128(ch[1] + threadIdx.x)));
             __stcs(o4 + base4 + threadIdx.x + SBLOCK,
-                   apply4(ch[0][threadIdx.x + SBLOCK], ch[1][threadIdx.x + SBLOCK]));
+                   apply4(lds128(ch[0] + threadIdx.x + SBLOCK), lds128(ch[1] + threadIdx.x + SBLOCK)));
         });
     }
     for (int64_t i = done4 + gtid; i < n4; i += gstride) __stcs(o4 + i, apply4(r4[i], g4[i]));

@@ -318,6 +318,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int ca
     return false;
 }
 
+// 16-byte shared-memory load through an explicit shared address (chunk pointers
+// handed to a body lambda would otherwise be read with generic loads)
+__device__ __forceinline__ float4 lds128(const float4 *p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_addr(p)));
+    return v;
+}
+
 constexpr int BULK_F4 = 512;                    // float4 per source per chunk (8 KB)
 constexpr int BULK_WAIT_CAP = 1 << 22;
 // stages in flight: 4 chunks of one source, 3 of two (48 KB per CTA, so four
