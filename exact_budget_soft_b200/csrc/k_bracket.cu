@@ -130,38 +130,30 @@ constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
 // This is the operator's own noise kernel, so P(y_j > b) = k/n.  The key kept
 // is the fp32 value rounded toward -inf (monotone, so order statistics commute
 // with it), in the descending-order key space.
-__global__ void __launch_bounds__(1024) sample_kernel(BracketParams P) {
-    __shared__ uint32_t s_hist[4096];   // first radix-select round: top 12 key bits
-    for (int i = threadIdx.x; i < 4096; i += blockDim.x) s_hist[i] = 0u;
+__global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
     pdl_enter();
-    __syncthreads();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (j < P.s) {
-        uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
-        philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
-        const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
-        const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
-        const double E = -sample_ln(U);
-        const double L = (x1 & 1ull) ? E : -E;
-        const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
-        const uint32_t key = desc_key(__double2float_rd(y));
-        P.keys[j] = key;
-        const uint32_t bin = key >> 20;
-        const unsigned act = __activemask();
-        const unsigned peers = __match_any_sync(act, bin);
-        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < 4096; i += blockDim.x) {
-        const uint32_t c = s_hist[i];
-        if (c) atomicAdd(P.hist1 + i, c);
-    }
+    if (j >= P.s) return;
+    uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
+    philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
+    const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
+    const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
+    const double E = -sample_ln(U);
+    const double L = (x1 & 1ull) ? E : -E;
+    const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
+    const uint32_t key = desc_key(__double2float_rd(y));
+    P.keys[j] = key;
+    // first radix-select round: histogram of the top 16 key bits (warp-aggregated)
+    const uint32_t bin = key >> 16;
+    const unsigned peers = __match_any_sync(__activemask(), bin);
+    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
 }
 
 // ================================================================ select --
 // The jR-th and jL-th smallest sample keys (= the jR-th and jL-th largest
-// values) by a radix select over bits [31:20], [19:8], [7:0]; the first round's
-// histogram is shared by both targets.  Bracket ends rounded outward:
+// values) by a radix select over bits [31:16] (histogram built by the sampler,
+// shared by both targets), then [15:8] and [7:0] over the keys under each
+// target's 16-bit prefix, gathered in shared memory.  Bracket ends rounded outward:
 //   a_R = nextup(y_(jR) rounded down) (> y_(jR)),  a_L = y_(jL) rounded down;
 //   jR = 0 -> a_R = +inf,  jL = s + 1 -> a_L = -inf.
 __device__ __forceinline__ uint32_t block_incl_scan_u32(uint32_t v, uint32_t *s_w) {
@@ -189,16 +181,17 @@ __device__ __forceinline__ uint32_t block_incl_scan_u32(uint32_t v, uint32_t *s_
     return r;
 }
 
-constexpr int SEL_CAND = 8192;   // candidates per target kept in shared memory
-constexpr size_t SEL_SMEM = (2 * 4096 + 2 * SEL_CAND) * sizeof(uint32_t);
+constexpr int SEL_BINS = 65536;   // first round: top 16 key bits (histogram from the sampler)
+constexpr int SEL_CAND = 8192;    // candidates per target kept in shared memory
+constexpr size_t SEL_SMEM = (2 * SEL_CAND + 2 * 256) * sizeof(uint32_t);
 
 __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
     extern __shared__ __align__(16) unsigned char sel_smem[];
-    uint32_t (*hist)[4096] = reinterpret_cast<uint32_t (*)[4096]>(sel_smem);
-    uint32_t (*cand)[SEL_CAND] = reinterpret_cast<uint32_t (*)[SEL_CAND]>(sel_smem + 2 * 4096 * sizeof(uint32_t));
-    pdl_enter();
+    uint32_t (*cand)[SEL_CAND] = reinterpret_cast<uint32_t (*)[SEL_CAND]>(sel_smem);
+    uint32_t (*h8)[256] = reinterpret_cast<uint32_t (*)[256]>(sel_smem + 2 * SEL_CAND * sizeof(uint32_t));
     __shared__ uint32_t s_w[32];
     __shared__ uint32_t s_pref[2], s_rank[2], s_cnt[2];
+    pdl_enter();
     const int tid = threadIdx.x, lane = tid & 31;
     const int s = (int)P.s;
     const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
@@ -208,113 +201,125 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
         s_rank[1] = (uint32_t)(valid[1] ? P.jL : 1);
         s_cnt[0] = 0; s_cnt[1] = 0;
     }
-    // round 1 (bits 31..20): histogram built by the sample kernel; rearm it
-    for (int i = tid; i < 4096; i += 1024) {
-        hist[0][i] = P.hist1[i];
-        P.hist1[i] = 0u;
-    }
     __syncthreads();
-    uint32_t mask = 0;
-    const int shifts[3] = {20, 8, 0};
-    const int widths[3] = {12, 12, 8};
-    bool fast[2] = {false, false};
-#pragma unroll 1
-    for (int rd = 0; rd < 3; ++rd) {
-        const int sh = shifts[rd];
-        const uint32_t bm = (1u << widths[rd]) - 1u;
-        const int nb = 1 << widths[rd];
-        if (rd > 0) {
-            for (int i = tid; i < 2 * 4096; i += 1024) (&hist[0][0])[i] = 0;
-            __syncthreads();
-            const uint32_t pf[2] = {s_pref[0], s_pref[1]};
+    const uint32_t want0[2] = {s_rank[0], s_rank[1]};   // read before any thread updates them
+    // ---- round 1: thread tid owns bins [64 tid, 64 tid + 64) of the sampler's histogram
+    constexpr int PER = SEL_BINS / 1024;
+    uint4 *h4 = reinterpret_cast<uint4 *>(P.hist1) + tid * (PER / 4);
+    uint32_t loc = 0;
+#pragma unroll
+    for (int u = 0; u < PER / 4; ++u) {
+        const uint4 c = h4[u];
+        loc += (c.x + c.y) + (c.z + c.w);
+    }
+    const uint32_t inc = block_incl_scan_u32(loc, s_w);
+    const uint32_t ex = inc - loc;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint32_t want = want0[q];
+        if (valid[q] && ex < want && want <= inc) {
+            uint32_t cum = ex;
+            for (int bb = 0; bb < PER; ++bb) {
+                const uint32_t c = P.hist1[tid * PER + bb];
+                if (cum + c >= want) {
+                    s_pref[q] = (uint32_t)(tid * PER + bb) << 16;
+                    s_rank[q] = want - cum;
+                    break;
+                }
+                cum += c;
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < PER / 4; ++u) h4[u] = make_uint4(0u, 0u, 0u, 0u);   // rearm for the next call
+    __syncthreads();
+    // ---- collect the keys under each target's 16-bit prefix
+    uint32_t mask = 0xffff0000u;
+    {
+        const uint32_t pf[2] = {s_pref[0], s_pref[1]};
+        auto take = [&](uint32_t key, bool in) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                if (!valid[q]) continue;
-                if (fast[q]) {
-                    const int c = (int)s_cnt[q];
-                    for (int i = tid; i < c; i += 1024) {
-                        const uint32_t key = cand[q][i];
-                        if ((key & mask) == pf[q]) atomicAdd(&hist[q][(key >> sh) & bm], 1u);
-                    }
-                } else {
-                    for (int i = tid; i < s; i += 1024) {
-                        const uint32_t key = P.keys[i];
-                        if ((key & mask) == pf[q]) atomicAdd(&hist[q][(key >> sh) & bm], 1u);
-                    }
-                }
+                const bool m = in && valid[q] && (key & mask) == pf[q];
+                const unsigned bal = __ballot_sync(FULL, m);
+                if (!bal) continue;
+                uint32_t base = 0;
+                if (lane == __ffs(bal) - 1) base = atomicAdd(&s_cnt[q], (uint32_t)__popc(bal));
+                base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+                if (m && base < SEL_CAND) cand[q][base] = key;
             }
-            __syncthreads();
-        }
-#pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-            const uint32_t *h = (rd == 0) ? hist[0] : hist[q];
-            uint32_t c[4], loc = 0;
+        };
+        const uint4 *k4 = reinterpret_cast<const uint4 *>(P.keys);
+        const int s4 = s / 4;
+        for (int i0 = 0; i0 < s4; i0 += 4 * 1024) {   // four 16-byte loads in flight per thread
+            uint4 kv[4];
+            bool in[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int bi = tid * 4 + u;
-                c[u] = bi < nb ? h[bi] : 0u;
-                loc += c[u];
+                const int i = i0 + u * 1024 + tid;
+                in[u] = i < s4;
+                kv[u] = in[u] ? k4[i] : make_uint4(0u, 0u, 0u, 0u);
             }
-            const uint32_t inc = block_incl_scan_u32(loc, s_w);
-            const uint32_t ex = inc - loc;
-            const uint32_t want = s_rank[q];
-            __syncthreads();
-            if (valid[q] && ex < want && want <= inc) {
-                uint32_t cum = ex;
-                for (int u = 0; u < 4; ++u) {
-                    if (cum + c[u] >= want) {
-                        s_pref[q] |= (uint32_t)(tid * 4 + u) << sh;
-                        s_rank[q] = want - cum;
-                        break;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                take(kv[u].x, in[u]);
+                take(kv[u].y, in[u]);
+                take(kv[u].z, in[u]);
+                take(kv[u].w, in[u]);
+            }
+        }
+        for (int i0 = 4 * s4; i0 < s; i0 += 1024) {
+            const int i = i0 + tid;
+            take(i < s ? P.keys[i] : 0u, i < s);
+        }
+    }
+    __syncthreads();
+    const bool fast[2] = {s_cnt[0] <= SEL_CAND, s_cnt[1] <= SEL_CAND};
+    // ---- rounds 2, 3: bits 15..8, 7..0 over the candidates (or every key when
+    //      a prefix holds more keys than the shared buffer)
+#pragma unroll 1
+    for (int sh = 8; sh >= 0; sh -= 8) {
+        for (int i = tid; i < 2 * 256; i += 1024) (&h8[0][0])[i] = 0u;
+        __syncthreads();
+        const uint32_t pf[2] = {s_pref[0], s_pref[1]};
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            if (!valid[q]) continue;
+            const int c = fast[q] ? (int)s_cnt[q] : s;
+            for (int i = tid; i < c; i += 1024) {
+                const uint32_t key = fast[q] ? cand[q][i] : P.keys[i];
+                if ((key & mask) == pf[q]) atomicAdd(&h8[q][(key >> sh) & 0xffu], 1u);
+            }
+        }
+        __syncthreads();
+        if (tid < 64) {   // warp q scans target q's 256 bins (8 per lane)
+            const int q = tid >> 5;
+            if (valid[q]) {
+                uint32_t v[8], run = 0;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { v[u] = h8[q][lane * 8 + u]; run += v[u]; }
+                uint32_t incl = run;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t p = __shfl_up_sync(FULL, incl, o);
+                    if (lane >= o) incl += p;
+                }
+                const uint32_t want = s_rank[q];
+                uint32_t cum = incl - run;
+                if (cum < want && want <= incl) {
+                    for (int u = 0; u < 8; ++u) {
+                        if (cum + v[u] >= want) {
+                            s_pref[q] |= (uint32_t)(lane * 8 + u) << sh;
+                            s_rank[q] = want - cum;
+                            break;
+                        }
+                        cum += v[u];
                     }
-                    cum += c[u];
                 }
             }
-            __syncthreads();
         }
-        mask |= bm << sh;
-        if (rd == 0) {
-            // keep the keys under each target's 12-bit prefix in shared memory
-            const uint32_t pf[2] = {s_pref[0], s_pref[1]};
-            auto take = [&](uint32_t key, bool in) {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const bool m = in && valid[q] && (key & mask) == pf[q];
-                    const unsigned bal = __ballot_sync(FULL, m);
-                    if (!bal) continue;
-                    uint32_t base = 0;
-                    if (lane == __ffs(bal) - 1) base = atomicAdd(&s_cnt[q], (uint32_t)__popc(bal));
-                    base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
-                    if (m && base < SEL_CAND) cand[q][base] = key;
-                }
-            };
-            const uint4 *k4 = reinterpret_cast<const uint4 *>(P.keys);
-            const int s4 = s / 4;
-            for (int i0 = 0; i0 < s4; i0 += 4 * 1024) {   // four 16-byte loads in flight per thread
-                uint4 kv[4];
-                bool in[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int i = i0 + u * 1024 + tid;
-                    in[u] = i < s4;
-                    kv[u] = in[u] ? k4[i] : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    take(kv[u].x, in[u]);
-                    take(kv[u].y, in[u]);
-                    take(kv[u].z, in[u]);
-                    take(kv[u].w, in[u]);
-                }
-            }
-            for (int i0 = 4 * s4; i0 < s; i0 += 1024) {
-                const int i = i0 + tid;
-                take(i < s ? P.keys[i] : 0u, i < s);
-            }
-            __syncthreads();
-            fast[0] = s_cnt[0] <= SEL_CAND;
-            fast[1] = s_cnt[1] <= SEL_CAND;
-        }
+        mask |= 0xffu << sh;
+        __syncthreads();
     }
     if (tid == 0) {
         Ctl *c = P.ctl;
@@ -902,8 +907,8 @@ cudaError_t launch_selftest_math(int which, const double *in, double *out, doubl
     return cudaGetLastError();
 }
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
-    const unsigned blocks = (unsigned)((P.s + 1023) / 1024);
-    return launch_k(sample_kernel, blocks, 1024, 0, st, P);
+    const unsigned blocks = (unsigned)((P.s + 255) / 256);
+    return launch_k(sample_kernel, blocks, 256, 0, st, P);
 }
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     static bool attr = false;

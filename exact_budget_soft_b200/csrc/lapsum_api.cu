@@ -379,7 +379,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     P.spin_cap = spin_cap;
     P.fused_cert = opt.certify == LAPSUM_CERTIFY_FUSED;
     LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
-    LAPSUM_TRY(grow(w->hist1, w->hist1_n, 4096));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, 65536));
     LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_cap));
     LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort the whole row
     P.band = w->band;

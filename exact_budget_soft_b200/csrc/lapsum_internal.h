@@ -57,7 +57,7 @@ struct BracketParams {
     int64_t band_cap;
     float *band;              // band buffer [band_cap]
     uint32_t *keys;           // sample keys [s]
-    uint32_t *hist1;          // [4096] first-round select histogram (kept zeroed)
+    uint32_t *hist1;          // [65536] first-round select histogram (kept zeroed)
     double *partials;         // per-block partials
     Ctl *ctl;
     int32_t spin_cap;
