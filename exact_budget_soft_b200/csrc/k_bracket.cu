@@ -185,7 +185,7 @@ constexpr int SEL_BINS = 65536;   // first round: top 16 key bits (histogram fro
 constexpr int SEL_CAND = 8192;    // candidates per target kept in shared memory
 constexpr size_t SEL_SMEM = (2 * SEL_CAND + 2 * 256) * sizeof(uint32_t);
 
-__global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
+__global__ void __launch_bounds__(1024, 1) select_kernel(BracketParams P) {
     extern __shared__ __align__(16) unsigned char sel_smem[];
     uint32_t (*cand)[SEL_CAND] = reinterpret_cast<uint32_t (*)[SEL_CAND]>(sel_smem);
     uint32_t (*h8)[256] = reinterpret_cast<uint32_t (*)[256]>(sel_smem + 2 * SEL_CAND * sizeof(uint32_t));
@@ -206,11 +206,13 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
     // ---- round 1: thread tid owns bins [64 tid, 64 tid + 64) of the sampler's histogram
     constexpr int PER = SEL_BINS / 1024;
     uint4 *h4 = reinterpret_cast<uint4 *>(P.hist1) + tid * (PER / 4);
+    uint32_t part[PER / 4];   // bin sums of each of the thread's 16-byte vectors
     uint32_t loc = 0;
 #pragma unroll
     for (int u = 0; u < PER / 4; ++u) {
         const uint4 c = h4[u];
-        loc += (c.x + c.y) + (c.z + c.w);
+        part[u] = (c.x + c.y) + (c.z + c.w);
+        loc += part[u];
     }
     const uint32_t inc = block_incl_scan_u32(loc, s_w);
     const uint32_t ex = inc - loc;
@@ -218,16 +220,22 @@ __global__ void __launch_bounds__(1024) select_kernel(BracketParams P) {
     for (int q = 0; q < 2; ++q) {
         const uint32_t want = want0[q];
         if (valid[q] && ex < want && want <= inc) {
-            uint32_t cum = ex;
-            for (int bb = 0; bb < PER; ++bb) {
-                const uint32_t c = P.hist1[tid * PER + bb];
-                if (cum + c >= want) {
-                    s_pref[q] = (uint32_t)(tid * PER + bb) << 16;
-                    s_rank[q] = want - cum;
-                    break;
-                }
-                cum += c;
+            uint32_t cum = ex, at = ex;
+            int u = -1;
+#pragma unroll
+            for (int v = 0; v < PER / 4; ++v) {   // the vector holding the target
+                if (u < 0 && cum + part[v] >= want) { u = v; at = cum; }
+                cum += part[v];
             }
+            cum = at;
+            const uint4 c = h4[u];
+            int e = 3;
+            if (cum + c.x >= want) e = 0;
+            else if (cum + c.x + c.y >= want) { e = 1; cum += c.x; }
+            else if (cum + c.x + c.y + c.z >= want) { e = 2; cum += c.x + c.y; }
+            else cum += c.x + c.y + c.z;
+            s_pref[q] = (uint32_t)(tid * PER + u * 4 + e) << 16;
+            s_rank[q] = want - cum;
         }
     }
 #pragma unroll
