@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(1024, 1) select_kernel(BracketParams P) {
     pdl_enter();
     const int tid = threadIdx.x, lane = tid & 31;
     const int s = (int)P.s;
+    static_assert(SEL_BINS == 32 * 2048, "32 warps x 2048 bins");
     const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
     if (tid == 0) {
         s_pref[0] = 0; s_pref[1] = 0;
@@ -203,43 +204,60 @@ __global__ void __launch_bounds__(1024, 1) select_kernel(BracketParams P) {
     }
     __syncthreads();
     const uint32_t want0[2] = {s_rank[0], s_rank[1]};   // read before any thread updates them
-    // ---- round 1: thread tid owns bins [64 tid, 64 tid + 64) of the sampler's histogram
-    constexpr int PER = SEL_BINS / 1024;
-    uint4 *h4 = reinterpret_cast<uint4 *>(P.hist1) + tid * (PER / 4);
-    uint32_t part[PER / 4];   // bin sums of each of the thread's 16-byte vectors
-    uint32_t loc = 0;
+    // ---- round 1 over the sampler's 16-bit histogram: warp w owns bins
+    //      [2048 w, 2048 w + 2048), read as 16 coalesced rounds of 32 lanes x 4 bins
+    const int warp = tid >> 5;
+    uint4 *hw = reinterpret_cast<uint4 *>(P.hist1) + warp * 512;
+    uint32_t ps[16], rt[16], wtot = 0;
 #pragma unroll
-    for (int u = 0; u < PER / 4; ++u) {
-        const uint4 c = h4[u];
-        part[u] = (c.x + c.y) + (c.z + c.w);
-        loc += part[u];
+    for (int u = 0; u < 16; ++u) {
+        const uint4 c = hw[u * 32 + lane];
+        ps[u] = (c.x + c.y) + (c.z + c.w);
+        uint32_t t = ps[u];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
+        rt[u] = t;
+        wtot += t;
     }
-    const uint32_t inc = block_incl_scan_u32(loc, s_w);
-    const uint32_t ex = inc - loc;
+    if (lane == 0) s_w[warp] = wtot;
+    __syncthreads();
+    uint32_t wbase = 0;
+    for (int w = 0; w < warp; ++w) wbase += s_w[w];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
         const uint32_t want = want0[q];
-        if (valid[q] && ex < want && want <= inc) {
-            uint32_t cum = ex, at = ex;
+        if (valid[q] && wbase < want && want <= wbase + wtot) {     // warp-uniform
+            uint32_t cum = wbase, at = wbase, pu = 0;
             int u = -1;
 #pragma unroll
-            for (int v = 0; v < PER / 4; ++v) {   // the vector holding the target
-                if (u < 0 && cum + part[v] >= want) { u = v; at = cum; }
-                cum += part[v];
+            for (int v = 0; v < 16; ++v) {                           // the round holding the target
+                if (u < 0 && cum + rt[v] >= want) { u = v; at = cum; }
+                if (u < 0) cum += rt[v];
             }
-            cum = at;
-            const uint4 c = h4[u];
-            int e = 3;
-            if (cum + c.x >= want) e = 0;
-            else if (cum + c.x + c.y >= want) { e = 1; cum += c.x; }
-            else if (cum + c.x + c.y + c.z >= want) { e = 2; cum += c.x + c.y; }
-            else cum += c.x + c.y + c.z;
-            s_pref[q] = (uint32_t)(tid * PER + u * 4 + e) << 16;
-            s_rank[q] = want - cum;
+#pragma unroll
+            for (int v = 0; v < 16; ++v) if (v == u) pu = ps[v];
+            uint32_t inc = pu;                                        // lanes of that round
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t p = __shfl_up_sync(FULL, inc, o);
+                if (lane >= o) inc += p;
+            }
+            const uint32_t lo = at + inc - pu;
+            if (lo < want && want <= at + inc) {
+                const uint4 c = hw[u * 32 + lane];
+                uint32_t cc = lo;
+                int e = 3;
+                if (cc + c.x >= want) e = 0;
+                else if (cc + c.x + c.y >= want) { e = 1; cc += c.x; }
+                else if (cc + c.x + c.y + c.z >= want) { e = 2; cc += c.x + c.y; }
+                else cc += c.x + c.y + c.z;
+                s_pref[q] = (uint32_t)(warp * 2048 + u * 128 + lane * 4 + e) << 16;
+                s_rank[q] = want - cc;
+            }
         }
     }
 #pragma unroll
-    for (int u = 0; u < PER / 4; ++u) h4[u] = make_uint4(0u, 0u, 0u, 0u);   // rearm for the next call
+    for (int u = 0; u < 16; ++u) hw[u * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);   // rearm (coalesced)
     __syncthreads();
     // ---- collect the keys under each target's 16-bit prefix
     uint32_t mask = 0xffff0000u;
@@ -268,6 +286,15 @@ __global__ void __launch_bounds__(1024, 1) select_kernel(BracketParams P) {
                 in[u] = i < s4;
                 kv[u] = in[u] ? k4[i] : make_uint4(0u, 0u, 0u, 0u);
             }
+            bool hit = false;   // candidates are rare: one vote for sixteen keys
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t kk[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hit |= in[u] && (((kk[e] & mask) == pf[0] && valid[0]) || ((kk[e] & mask) == pf[1] && valid[1]));
+            }
+            if (!__any_sync(FULL, hit)) continue;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 take(kv[u].x, in[u]);
