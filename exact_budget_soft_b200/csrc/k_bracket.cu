@@ -712,11 +712,10 @@ __device__ __forceinline__ float4 p_vec(const float4 v, const XForm &xf) {
 
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict__ p,
-         double *__restrict__ b_out, Ctl *ctl, double *partials, int only_after_fallback) {
+         double *__restrict__ b_out, Ctl *ctl, double *partials) {
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[SBLOCK / 32];
     pdl_enter();
-    if (only_after_fallback && ctl->verdict != 0) return;   // certified: the first p pass stands
     const double b = ctl->b;
     const XForm xf = make_xform(b, inv_t * LOG2E);
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
@@ -975,11 +974,10 @@ cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
     return launch_k(oob_kernel<OOB_CERT>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
-                          double *partials, int only_after_fallback, cudaStream_t st) {
+                          double *partials, cudaStream_t st) {
     static cudaError_t once = set_smem(p_kernel, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    return launch_k(p_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, r, n, 1.0 / t, p, b_out, ctl, partials,
-                    only_after_fallback);
+    return launch_k(p_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, r, n, 1.0 / t, p, b_out, ctl, partials);
 }
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st) {

@@ -109,13 +109,8 @@ struct Workspace {
     unsigned long long *lookback = nullptr; size_t lookback_n = 0;
     double *tilebuf = nullptr;        size_t tilebuf_n = 0;
     uint32_t epoch = 1;
-    cudaStream_t side = nullptr;      // band solve / fallback run here, overlapped
-    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
 
     void release() {
-        if (side) cudaStreamDestroy(side);
-        for (auto &e : ev)
-            if (e) cudaEventDestroy(e);
         cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(hist1); cudaFree(band);
         cudaFree(keys0); cudaFree(keys1); cudaFree(hist); cudaFree(dbase);
         cudaFree(lookback); cudaFree(tilebuf);
@@ -141,14 +136,6 @@ Workspace *get_ws(cudaStream_t st) {
 cudaError_t ws_base(Workspace *w) {
     cudaError_t e = grow(w->ctl, w->ctl_n, 1);
     if (e == cudaSuccess) e = grow(w->partials, w->partials_n, (size_t)stream_grid() * 24 + 64);
-    return e;
-}
-
-cudaError_t ws_side(Workspace *w) {
-    if (w->side) return cudaSuccess;
-    cudaError_t e = cudaStreamCreateWithFlags(&w->side, cudaStreamNonBlocking);
-    for (auto &ev : w->ev)
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
     return e;
 }
 
@@ -370,7 +357,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
             rc = full_sort_row(w, row, n, k, t, GATE_ALWAYS, spin_cap, st);
             if (rc) return rc;
             Launch L("p_pass", st);
-            LAPSUM_TRY(launch_p_pass(row, n, t, p_out + r * n, b_out + r, w->ctl, w->partials, 0, st));
+            LAPSUM_TRY(launch_p_pass(row, n, t, p_out + r * n, b_out + r, w->ctl, w->partials, st));
         }
         return LAPSUM_OK;
     }
@@ -405,36 +392,20 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     { Launch L("sample", st); LAPSUM_TRY(launch_sample(P, st)); }
     { Launch L("select", st); LAPSUM_TRY(launch_select(P, st)); }
     { Launch L("stream_pass", st); LAPSUM_TRY(launch_stream_pass(P, st)); }
-    // The band solve (latency-bound, a few CTAs) runs on a side stream under the
-    // certification pass (every SM); the gated fallback then runs on the side
-    // stream under the p pass, and a gated second p pass rewrites p when the
-    // certification failed (the first p used the band's threshold).
-    LAPSUM_TRY(ws_side(w));
-    cudaStream_t sd = w->side;
-    LAPSUM_TRY(cudaEventRecord(w->ev[0], st));
-    LAPSUM_TRY(cudaStreamWaitEvent(sd, w->ev[0], 0));
-    { Launch L("band_rowsolve", sd); LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, sd)); }
+    { Launch L("band_rowsolve", st); LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st)); }
     if (band_cap > rowsolve_capacity()) {
         SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap, k, t);
         {
-            Launch L("band_radix_sort(5 kernels)", sd);
+            Launch L("band_radix_sort(5 kernels)", st);
             g_launches += 4;
-            LAPSUM_TRY(launch_radix_sort(A, k, t, sd));
+            LAPSUM_TRY(launch_radix_sort(A, k, t, st));
         }
-        { Launch L("band_locate", sd); LAPSUM_TRY(launch_locate(A, k, t, sd)); }
+        { Launch L("band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
     }
     if (!P.fused_cert) { Launch L("certify", st); LAPSUM_TRY(launch_certify(P, st)); }
-    LAPSUM_TRY(cudaEventRecord(w->ev[1], sd));
-    LAPSUM_TRY(cudaStreamWaitEvent(st, w->ev[1], 0));
-    LAPSUM_TRY(cudaEventRecord(w->ev[2], st));
-    LAPSUM_TRY(cudaStreamWaitEvent(sd, w->ev[2], 0));
-    rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, sd);
+    rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, st);
     if (rc) return rc;
-    { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, 0, st)); }
-    LAPSUM_TRY(cudaEventRecord(w->ev[3], sd));
-    LAPSUM_TRY(cudaStreamWaitEvent(st, w->ev[3], 0));
-    { Launch L("p_pass_after_fallback", st);
-      LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, 1, st)); }
+    { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, st)); }
     return LAPSUM_OK;
 }
 

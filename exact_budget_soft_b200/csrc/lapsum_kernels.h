@@ -41,7 +41,7 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
-                          double *partials, int only_after_fallback, cudaStream_t st);
+                          double *partials, cudaStream_t st);
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st);
 cudaError_t launch_selftest_math(int which, const double *in, double *out, double *ref, int64_t n,
