@@ -118,6 +118,20 @@ def dist_setup(n_gpus: int):
     return dist.get_rank(), dist.get_world_size(), dist
 
 
+def max_over_ranks(dist, values):
+    """Element-wise max of per-rank values (timings), on every rank.
+
+    With N > 1 every rank times its own replica; the job's step time is the
+    slowest rank's.  NCCL reduces on the device, gloo (CPU tests) on the host."""
+    import torch
+    if dist is None:
+        return list(values)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def time_steps(torch, step, K, W_, flush=None):
     for _ in range(W_):
         step()
@@ -199,9 +213,7 @@ def run_ours(args):
     tot = sum(ms)
     dom_ms = prof[dom][1] / max(prof[dom][0], 1)
     if dist:
-        t = torch.tensor([med, tot, med_f, dom_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        med, tot, med_f, dom_ms = t.tolist()
+        med, tot, med_f, dom_ms = max_over_ranks(dist, [med, tot, med_f, dom_ms])
         dist.barrier()
 
     nsteps = 4   # calibration: 1 warm-up + 3 steps
@@ -268,9 +280,7 @@ def run_ours(args):
     assert st_f["verdict"] == 1 and st_f["rc"] == 0 and abs(st_f["sum_p"] - w.k) < 1.0 + 1e-7 * w.n
     med_fused = statistics.median(ms_fused)
     if dist:
-        t = torch.tensor([med_fused], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        med_fused = t.item()
+        med_fused = max_over_ranks(dist, [med_fused])[0]
     out["certify_fused"] = {"median_ms_fwd_vjp": round(med_fused, 4),
                             "model_frac_of_8TBs": round(32 * w.n / (med_fused * 1e-3) / 8e12, 4),
                             "note": "option certify=LAPSUM_CERTIFY_FUSED: certification folded into the "
@@ -294,9 +304,7 @@ def run_ours(args):
     mse2e = time_steps(torch, e2e_step, max(3, args.steps // 4), 1)
     e2e = statistics.median(mse2e)
     if dist:
-        t = torch.tensor([e2e], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = t.item()
+        e2e = max_over_ranks(dist, [e2e])[0]
     out["e2e"] = {"value": round(e2e, 3), "unit": "ms", "h2d_bytes_per_step": 8 * w.n,
                   "d2h_bytes_per_step": 8 * w.n + 8}
     if rank == 0 and world == 1 and not args.no_cpu:
