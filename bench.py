@@ -268,6 +268,40 @@ def run_ours(args):
             by_n[f"{we.n:.0e}"] = {"workload": name, "median_ms_fwd_vjp": round(statistics.median(mse), 4)}
         by_n["1e+08"] = {"workload": w.name, "median_ms_fwd_vjp": round(med, 4), "fwd_ms": round(med_f, 4)}
         out["by_n"] = by_n
+        # the full-sort row path (one CTA per row: sort, scan, root, p) and its VJP
+        rows_out = {}
+        for name in ("n4096", "rows1024"):
+            wr = W.WORKLOADS[name]
+            rr_ = torch.from_numpy(W.scores(wr, seed=rank)).cuda()
+            gr_ = torch.from_numpy(W.upstream_grad(wr, seed=rank)).cuda()
+            pr_, grr_ = torch.empty_like(rr_), torch.empty_like(rr_)
+            br_ = torch.empty(wr.rows, dtype=torch.float64, device="cuda")
+
+            def st_r():
+                L.forward(rr_, wr.k, wr.t, p_out=pr_, b_out=br_)
+                L.backward(rr_, br_, gr_, wr.t, grad_out=grr_)
+
+            msr = time_steps(torch, st_r, max(args.steps, 10), max(args.warmup, 3),
+                             flush=lambda: flushbuf.fill_(1.0))
+            mr = statistics.median(msr)
+            rows_out[name] = {"median_ms_fwd_vjp": round(mr, 4), "rows": wr.rows, "n": wr.n,
+                              "model_gbs": round(20 * wr.units / (mr * 1e-3) / 1e9, 1)}
+        out["full_sort_rows"] = rows_out
+        # forced full-sort fallback on the headline row (certification rejects a weak bracket)
+        gold = json.load(open(os.path.join(ROOT, "tests", "golden", "forced_fallback.json")))
+        if not args.scale_n and gold["workload"] == w.name:
+            of = L.options(seed=gold["seed"], sample_size=gold["sample_size"], delta=gold["delta"])
+
+            def st_fb():
+                L.forward(r, w.k, w.t, p_out=p, b_out=b, opts=of)
+                L.backward(r, b, g, w.t, grad_out=grad)
+
+            msf = time_steps(torch, st_fb, max(5, args.steps // 4), 2)
+            st_fb_stats = L.get_stats()
+            assert st_fb_stats["fallback"] == 1 and st_fb_stats["rc"] == 0
+            out["forced_fallback"] = {"median_ms_fwd_vjp": round(statistics.median(msf), 4),
+                                      "note": "certification fails (seed from tests/golden); the row is "
+                                              "fully sorted on the device"}
     # the same step with the certification folded into the streaming pass
     opt_fused = L.options(certify=L.CERTIFY_FUSED)
 
