@@ -397,6 +397,37 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_case(args):
+    """Profiling driver: time one non-headline case (no JSON line)."""
+    import torch
+    import exact_budget_soft_b200 as L
+    if args.case == "rows":
+        w = W.WORKLOADS["rows1024"]
+        rows = args.case_rows or w.rows
+        w = W.Workload(f"rows{rows}", rows, w.n, w.k, w.t, w.dist, w.path)
+        r = torch.from_numpy(W.scores(w)).cuda()
+        g = torch.from_numpy(W.upstream_grad(w)).cuda()
+        opts = None
+    else:   # forced full-sort fallback on the levels workload (possibly scaled)
+        w = W.WORKLOADS["levels1e8"]
+        if args.scale_n:
+            w = W.Workload(f"{w.name}@n={args.scale_n}", 1, args.scale_n, w.k * args.scale_n / w.n, w.t, w.dist, w.path)
+        r = torch.from_numpy(W.scores(w)[0]).cuda()
+        g = torch.from_numpy(W.upstream_grad(w)[0]).cuda()
+        opts = L.options(band_cap=1)   # any non-empty band overflows: certification fails
+    p, grad = torch.empty_like(r), torch.empty_like(r)
+    b = torch.empty(w.rows, dtype=torch.float64, device="cuda")
+
+    def step():
+        L.forward(r, w.k, w.t, p_out=p, b_out=b, opts=opts)
+        L.backward(r, b, g, w.t, grad_out=grad)
+
+    ms = time_steps(torch, step, args.steps, args.warmup)
+    st = L.get_stats()
+    print(json.dumps({"case": args.case, "workload": w.name, "median_ms_fwd_vjp": statistics.median(ms),
+                      "fallback": st["fallback"], "rc": st["rc"]}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,10 +438,15 @@ def main():
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--scale-n", type=int, default=0, help="profiling: same workload at another n")
+    ap.add_argument("--case", choices=["rows", "fallback"], default=None,
+                    help="profiling driver: time one non-headline case instead of the benchmark")
+    ap.add_argument("--case-rows", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
