@@ -335,7 +335,7 @@ __device__ __forceinline__ double sorted_val(const uint32_t *keys, const float *
 __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, double t, double inv_t) {
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);                 // LTILE
-    void *scratch = smem + LTILE * 4;                                        // >= 6 KB
+    void *scratch = smem + (LTILE + LTILE / 32) * 4;                         // >= 6 KB
     __shared__ bool s_last;
     __shared__ int s_tstar;
     __shared__ double s_tab[32];
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
     const int64_t t0 = TT * LTILE;
     const int cnt = (int)min((int64_t)LTILE, n - t0);
     for (int i = tid; i < cnt; i += LB) {
-        s_keys[i] = keys_cur ? keys_cur[t0 + i] : desc_key(A.src[t0 + i]);
+        s_keys[spad(i)] = keys_cur ? keys_cur[t0 + i] : desc_key(A.src[t0 + i]);
     }
     __syncthreads();
     const double ptop = TT == 0 ? P_top : __ldcg(&rec[TT - 1].p_end);
@@ -522,7 +522,7 @@ cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) 
 
 cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st) {
     static bool attr = false;
-    const size_t smem = (size_t)LTILE * 4 + 16384;
+    const size_t smem = (size_t)(LTILE + LTILE / 32) * 4 + 16384;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(locate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);

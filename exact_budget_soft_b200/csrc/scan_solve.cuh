@@ -9,18 +9,23 @@
 
 namespace lapsum {
 
+// Shared-memory slot of sorted position j: one pad word per 32 keys, so a thread
+// walking its own run of consecutive positions hits a different bank from its
+// neighbours (the scan reads runs; unpadded, all 32 lanes would share a bank).
+__device__ __forceinline__ int spad(int j) { return j + (j >> 5); }
+
 template <int BLOCK, int KPT>
 struct RowCfg {
     static constexpr int NW = BLOCK / 32;
     static constexpr int CAP = BLOCK * KPT;
     static constexpr int SEG = 32 * KPT;   // keys per warp segment
-    static constexpr size_t SMEM_KEYS = size_t(CAP) * 4;
+    static constexpr size_t SMEM_KEYS = size_t(CAP + CAP / 32) * 4;
     static constexpr size_t SMEM_HIST = size_t(NW) * 256 * 4;
     static constexpr size_t SMEM = SMEM_KEYS + SMEM_HIST + 256 * 4 + 2048;
 };
 
 // Block-wide LSD radix sort of warp-striped register keys (ascending).  On
-// return the sorted keys are in s_keys[0 .. CAP).
+// return the sorted keys are in s_keys (position j at spad(j)).
 template <int BLOCK, int KPT>
 __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t *s_keys,
                                                  uint32_t *s_hist, uint32_t *s_dbase,
@@ -83,23 +88,23 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
                 my_hist[d] = base + __popc(peers);
             }
             base = __shfl_sync(FULL, base, leader) + __popc(peers & lt_mask);
-            s_keys[base] = key[i];
+            s_keys[spad((int)base)] = key[i];
             __syncwarp();
         }
         __syncthreads();
 #pragma unroll
-        for (int i = 0; i < KPT; ++i) key[i] = s_keys[warp * C::SEG + i * 32 + lane];
+        for (int i = 0; i < KPT; ++i) key[i] = s_keys[spad(warp * C::SEG + i * 32 + lane)];
         sorted_in_smem = true;
         __syncthreads();
     }
     if (!sorted_in_smem) {   // all keys identical: any order is sorted
 #pragma unroll
-        for (int i = 0; i < KPT; ++i) s_keys[warp * C::SEG + i * 32 + lane] = key[i];
+        for (int i = 0; i < KPT; ++i) s_keys[spad(warp * C::SEG + i * 32 + lane)] = key[i];
         __syncthreads();
     }
 }
 
-// Solve the sorted values held in s_keys[0..n) (descending scores).
+// Solve the sorted values held in s_keys (position j at spad(j); descending scores).
 //   m0      scores above the first value (band: the count at or above a_R)
 //   top     value above c_0 that P_top refers to (a_R, or +inf)
 //   P_top   sum_{scores above} e^{(top - r)/t}
@@ -122,7 +127,7 @@ __device__ double block_scan_solve(const uint32_t *s_keys, int n, double k, doub
     auto val = [&](int j) -> double {
         if (j < 0) return top;
         if (j >= n) return bot;
-        return (double)desc_key_to_float(s_keys[j]);
+        return (double)desc_key_to_float(s_keys[spad(j)]);
     };
     // link d_j = e^{(c_{j+1} - c_j)/t}, j in [-1, n-1] (virtual top/bottom at the ends)
     auto link = [&](int j) -> double {
