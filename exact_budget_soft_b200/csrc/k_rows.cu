@@ -6,7 +6,7 @@
 // One CTA owns one row of up to BLOCK*KPT scores (32768 at 1024 x 32):
 //  * LSD radix sort of the order-preserving uint32 keys, 8-bit digits, keys in
 //    registers (warp-striped), a shared-memory scatter buffer, per-warp digit
-//    histograms and __match_any_sync ranking (stable); digits on which every
+//    histograms and ballot-based digit-peer ranking (stable); digits on which every
 //    key agrees are skipped;
 //  * each thread then owns a run of KPT consecutive sorted scores: it forms the
 //    links d_j and the run's two affine maps (prefix P and suffix Q), a block

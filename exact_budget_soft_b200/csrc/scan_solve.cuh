@@ -14,6 +14,17 @@ namespace lapsum {
 // neighbours (the scan reads runs; unpadded, all 32 lanes would share a bank).
 __device__ __forceinline__ int spad(int j) { return j + (j >> 5); }
 
+// Lanes of the warp holding the same 8-bit digit: eight ballots, one per bit.
+__device__ __forceinline__ unsigned digit_peers(uint32_t d) {
+    unsigned peers = FULL;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+        const unsigned m = __ballot_sync(FULL, (d >> b) & 1u);
+        peers &= ((d >> b) & 1u) ? m : ~m;
+    }
+    return peers;
+}
+
 template <int BLOCK, int KPT>
 struct RowCfg {
     static constexpr int NW = BLOCK / 32;
@@ -44,7 +55,7 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
             const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = __match_any_sync(FULL, d);
+            const unsigned peers = digit_peers(d);
             if (lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
             __syncwarp();
         }
@@ -80,7 +91,7 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
             const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = __match_any_sync(FULL, d);
+            const unsigned peers = digit_peers(d);
             const int leader = __ffs(peers) - 1;
             uint32_t base = 0;
             if (lane == leader) {
