@@ -424,8 +424,15 @@ def run_case(args):
 
     ms = time_steps(torch, step, args.steps, args.warmup)
     st = L.get_stats()
+    # per-kernel CUDA-event averages over a few more steps (events around every launch)
+    L.profile_enable(1)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    per = {k: round(v[1] / v[0], 4) for k, v in L.profile_read().items() if v[0]}
+    L.profile_enable(0)
     print(json.dumps({"case": args.case, "workload": w.name, "median_ms_fwd_vjp": statistics.median(ms),
-                      "fallback": st["fallback"], "rc": st["rc"]}))
+                      "fallback": st["fallback"], "rc": st["rc"], "per_launch_ms": per}))
 
 
 def main():

@@ -5,18 +5,19 @@
 // path (step 3) that exceeds the one-CTA capacity.
 //
 // Sort: keys-only LSD radix sort of the descending-order uint32 keys, 8-bit
-// digits, "onesweep" style:
-//   radix_hist_kernel   one read: all four digit histograms (per-thread run
-//                       length combining, so long runs of tied scores cost one
-//                       shared atomic per run), exclusive digit bases, and the
-//                       set of digits on which every key agrees (those passes
-//                       are skipped);
-//   radix_pass_kernel   per digit: tiles taken in launch order from an atomic
-//                       counter, in-tile stable ranking (per-warp histograms,
-//                       __match_any_sync), decoupled look-back over earlier
-//                       tiles for the global digit offsets (every wait bounded
-//                       by a spin cap), a shared-memory scatter and coalesced
-//                       runs of writes.
+// digits, reduce-then-scan per digit:
+//   radix_hist_kernel     one read: all four digit histograms (per-thread run
+//                         length combining, so long runs of tied scores cost
+//                         one shared atomic per run), exclusive digit bases,
+//                         and the digits on which every key agrees (those
+//                         passes are skipped; all four: solved in closed form);
+//   radix_count_kernel    per 8192-key tile, its 256 digit counts;
+//   radix_scan_kernel     per digit, the counts of earlier tiles -> offsets;
+//   radix_scatter_kernel  per tile, a stable in-tile ranking (per-warp digit
+//                         histograms, __match_any_sync), a shared-memory
+//                         scatter and coalesced runs of writes at the offsets.
+// The count and scatter kernels stage each CTA's next tile in shared memory by
+// one bulk copy while they work on the current one.  No CTA waits on another.
 // Locate: one kernel; every CTA reduces one tile of sorted values to its two
 // affine maps (prefix P, suffix Q); the last CTA scans the tile maps, finds the
 // tile whose end brackets G = k, re-scans that tile in shared memory and takes
@@ -42,6 +43,7 @@ constexpr int HB = 256;             // histogram kernel threads
 constexpr int LB = 1024;            // locate: threads
 constexpr int LK = 16;              // values per thread
 constexpr int LTILE = LB * LK;      // 16384 values per tile
+constexpr int LOC_KEY_WORDS = LTILE + LTILE / 32 + 8;   // padded tile + two halo entries
 
 int radix_tile() { return RTILE; }
 int locate_tile() { return LTILE; }
@@ -105,9 +107,8 @@ __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
     __syncthreads();
     uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
     uint32_t cnt[4] = {0, 0, 0, 0};
-    const int64_t gstride = (int64_t)gridDim.x * HB;
-    for (int64_t i = (int64_t)blockIdx.x * HB + tid; i < n; i += gstride) {
-        const uint32_t key = desc_key(A.src[i]);
+    auto count = [&](float x) {   // run-length combining per digit
+        const uint32_t key = desc_key(x);
 #pragma unroll
         for (int d = 0; d < 4; ++d) {
             const uint32_t bin = (key >> (8 * d)) & 0xffu;
@@ -119,7 +120,35 @@ __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
                 cnt[d] = 1;
             }
         }
+    };
+    // each thread takes chunks of 16 consecutive scores (four 16-byte loads, so
+    // runs of tied scores combine); the next chunk is loaded while this one is
+    // counted (one copy of the counting code: a rotation, not an unrolled batch)
+    const int64_t gstride = (int64_t)gridDim.x * HB;
+    const int64_t nch = (reinterpret_cast<uintptr_t>(A.src) & 15u) == 0 ? n / 16 : 0;
+    const float4 *src4 = reinterpret_cast<const float4 *>(A.src);
+    auto load_chunk = [&](int64_t c, float4 (&v)[4]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = c < nch ? __ldg(src4 + c * 4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 cur4[4];
+    int64_t c = (int64_t)blockIdx.x * HB + tid;
+    load_chunk(c, cur4);
+#pragma unroll 1
+    for (; c < nch; c += gstride) {
+        float4 nxt4[4];
+        load_chunk(c + gstride, nxt4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            count(cur4[q].x);
+            count(cur4[q].y);
+            count(cur4[q].z);
+            count(cur4[q].w);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cur4[q] = nxt4[q];
     }
+    for (int64_t i = nch * 16 + (int64_t)blockIdx.x * HB + tid; i < n; i += gstride) count(__ldg(A.src + i));
 #pragma unroll
     for (int d = 0; d < 4; ++d)
         if (cnt[d]) atomicAdd(&h[d][cur[d]], cnt[d]);
@@ -168,100 +197,254 @@ __global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
 }
 
 // ----------------------------------------------------------- one digit --
-constexpr unsigned long long LB_AGG = 1ull << 62;
-constexpr unsigned long long LB_PREFIX = 2ull << 62;
+// A pass (skipped when every key agrees on its digit) is reduce-then-scan:
+//   radix_count_kernel    each tile's 256 digit counts -> cnt[d][tile]
+//   radix_scan_kernel     per digit d, cnt[d][.] -> global offsets in place:
+//                         dbase[d] + the count of d in all earlier tiles
+//   radix_scatter_kernel  each tile ranks its keys stably in shared memory and
+//                         writes every digit's run at the run's offset
+// No CTA ever waits on another, so the pass has no spin waits at all; the
+// price is one more read of the keys than a single-sweep sort.
 
-__device__ __forceinline__ unsigned long long lb_pack(unsigned long long flag, uint32_t epoch,
-                                                      uint32_t v) {
-    return flag | ((unsigned long long)(epoch & 0x3fffffffu) << 32) | v;
+// Row stride of the count table (a multiple of 4 entries, for 16-byte loads).
+__host__ __device__ __forceinline__ int64_t cnt_stride(int64_t ntiles) { return (ntiles + 3) & ~int64_t(3); }
+
+__device__ __forceinline__ const uint32_t *pass_keys_in(const SortArgs &A, int cur) {
+    return cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
 }
 
-__global__ void __launch_bounds__(RB, 1) radix_pass_kernel(SortArgs A, int pass, uint32_t epoch) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);            // RTILE
-    uint32_t *s_hist = s_keys + RTILE;                                 // RNW * 256
-    uint32_t *s_dstart = s_hist + RNW * 256;                           // 256: in-tile digit start
-    uint32_t *s_gofs = s_dstart + 256;                                 // 256: global base - dstart
-    __shared__ int s_tile, s_cur;
-    __shared__ bool s_last;
+// The tile's keys, warp-striped (key i of lane l of warp w is tile element
+// w*32*RK + i*32 + l), all RK loads in flight at once; keys past the end of the
+// row read as 0xffffffff.  src == nullptr: the first pass, keys from the scores.
+__device__ __forceinline__ void load_tile(const SortArgs &A, const uint32_t *src, int64_t base, int cnt_tile,
+                                          uint32_t (&key)[RK]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int l0 = warp * 32 * RK + lane;
+    if (src) {
+#pragma unroll
+        for (int i = 0; i < RK; ++i)
+            key[i] = l0 + i * 32 < cnt_tile ? __ldcs(src + base + l0 + i * 32) : 0xffffffffu;
+    } else {
+        float x[RK];
+#pragma unroll
+        for (int i = 0; i < RK; ++i) x[i] = l0 + i * 32 < cnt_tile ? __ldg(A.src + base + l0 + i * 32) : 0.0f;
+#pragma unroll
+        for (int i = 0; i < RK; ++i) key[i] = l0 + i * 32 < cnt_tile ? desc_key(x[i]) : 0xffffffffu;
+    }
+}
 
-    pdl_enter();
-    const int64_t n = gated_n(A);
-    if (n < 0) return;
-    Ctl *ctl = A.ctl;
-    if (ctl->sort_skip & (1 << pass)) return;   // every key agrees on this digit
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int sh = 8 * pass;
-    const int64_t ntiles = (n + RTILE - 1) / RTILE;
-    if (tid == 0) s_cur = ctl->sort_cur;
+// Double-buffered tile staging for the pass kernels: tiles are grid-strided, so
+// each CTA knows its next tile and copies it (one bulk copy, completion counted
+// on an mbarrier) while it works on the current one.  Only full tiles of a
+// 16-byte-aligned source are staged; the rest take plain loads.
+struct TileStage {
+    uint32_t *buf;      // 2 * RTILE words
+    uint64_t *bar;      // 2 mbarriers
+    const char *gsrc;   // 4-byte elements: the keys, or the scores on the first pass
+    bool bulk_ok;
+    int64_t n;
+};
+
+__device__ __forceinline__ bool stage_full(const TileStage &S, int64_t tile) {
+    return S.bulk_ok && (tile + 1) * RTILE <= S.n;
+}
+
+// thread 0; the buffer must be free (its last readers are past a barrier)
+__device__ __forceinline__ void stage_issue(const TileStage &S, int slot, int64_t tile) {
+    if (!stage_full(S, tile)) return;
+    fence_proxy_async_smem();
+    mbar_expect_tx(&S.bar[slot], RTILE * 4);
+    bulk_load(S.buf + slot * RTILE, S.gsrc + (size_t)tile * RTILE * 4, RTILE * 4, &S.bar[slot]);
+}
+
+__device__ __forceinline__ void stage_init(TileStage &S, const SortArgs &A, const uint32_t *src, int64_t n,
+                                           unsigned char *smem) {
+    S.buf = reinterpret_cast<uint32_t *>(smem);
+    S.bar = reinterpret_cast<uint64_t *>(smem + 2 * RTILE * 4);
+    S.gsrc = src ? reinterpret_cast<const char *>(src) : reinterpret_cast<const char *>(A.src);
+    S.bulk_ok = (reinterpret_cast<uintptr_t>(S.gsrc) & 15u) == 0;
+    S.n = n;
+    if (threadIdx.x == 0) {
+        mbar_init(&S.bar[0], 1);
+        mbar_init(&S.bar[1], 1);
+        mbar_init_fence();
+    }
     __syncthreads();
-    const int cur = s_cur;
-    // persistent: tiles are claimed in order from one counter, so a tile only
-    // ever waits on tiles already claimed by running CTAs
-    for (;;) {
-        if (tid == 0) s_tile = (int)atomicAdd(&ctl->tile_ctr[pass], 1u);
-        __syncthreads();
-        const int tile = s_tile;
-        if (tile >= ntiles) break;
-        const uint32_t *src = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
-        uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
-        const int64_t base = (int64_t)tile * RTILE;
-        const int cnt_tile = (int)min((int64_t)RTILE, n - base);
+    if (threadIdx.x == 0 && (int64_t)blockIdx.x * RTILE < n) stage_issue(S, 0, blockIdx.x);
+}
+
+// The tile's keys into registers: from its staged copy (waiting, bounded, for
+// the copy) or by plain loads.  Returns false when the wait gave up.
+__device__ __forceinline__ bool stage_keys(const TileStage &S, const SortArgs &A, const uint32_t *src, int slot,
+                                           uint32_t &ph, int64_t tile, int cnt_tile, uint32_t (&key)[RK]) {
+    if (!stage_full(S, tile)) {
+        load_tile(A, src, tile * RTILE, cnt_tile, key);
+        return true;
+    }
+    const bool ok = mbar_wait(&S.bar[slot], (ph >> slot) & 1u, BULK_WAIT_CAP);
+    ph ^= 1u << slot;
+    const uint32_t *sb = S.buf + slot * RTILE;
+    const int l0 = (threadIdx.x >> 5) * 32 * RK + (threadIdx.x & 31);
+    if (src) {
+#pragma unroll
+        for (int i = 0; i < RK; ++i) key[i] = sb[l0 + i * 32];
+    } else {
+#pragma unroll
+        for (int i = 0; i < RK; ++i) key[i] = desc_key(__uint_as_float(sb[l0 + i * 32]));
+    }
+    return ok;
+}
+
+constexpr size_t STAGE_BYTES = 2 * RTILE * 4 + 2 * sizeof(uint64_t);
+
+// Adds this warp's digit counts of the tile to my_hist (the warp's 256 counters).
+__device__ __forceinline__ void warp_count(const uint32_t (&key)[RK], int cnt_tile, int sh, uint32_t *my_hist) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < RK; ++i) {
+        const int li = warp * 32 * RK + i * 32 + lane;
+        const bool v = li < cnt_tile;
+        const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
+        const unsigned peers = __match_any_sync(FULL, d);
+        if (v && lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// Common gate of the three pass kernels: the element count, or < 0 to return.
+__device__ __forceinline__ int64_t pass_n(const SortArgs &A, int pass) {
+    const int64_t n = gated_n(A);
+    if (n < 0) return -1;
+    if (A.ctl->sort_skip & (1 << pass)) return -1;   // every key agrees on this digit
+    return n;
+}
+
+__global__ void __launch_bounds__(RB, 2) radix_count_kernel(SortArgs A, int pass) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + STAGE_BYTES);   // RNW * 256
+    pdl_enter();
+    const int64_t n = pass_n(A, pass);
+    if (n < 0) return;
+    const uint32_t *src = pass_keys_in(A, A.ctl->sort_cur);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t ntiles = (n + RTILE - 1) / RTILE, nts = cnt_stride(ntiles);
+    uint32_t *cnt = A.tilecnt;
+    TileStage S;
+    stage_init(S, A, src, n, smem);
+    uint32_t ph = 0;
+    bool ok = true;
+    int slot = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, slot ^= 1) {
+        if (tid == 0 && tile + gridDim.x < ntiles) stage_issue(S, slot ^ 1, tile + gridDim.x);
+        const int cnt_tile = (int)min((int64_t)RTILE, n - tile * RTILE);
+        uint32_t key[RK];
+        ok &= stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
         for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
         __syncthreads();
-        // load (warp-striped) and count digits per warp
-        uint32_t key[RK];
-        uint32_t *my_hist = s_hist + warp * 256;
-        const unsigned lt_mask = (1u << lane) - 1u;
-#pragma unroll
-        for (int i = 0; i < RK; ++i) {
-            const int li = warp * 32 * RK + i * 32 + lane;
-            const bool v = li < cnt_tile;
-            uint32_t kk = 0xffffffffu;
-            if (v) kk = src ? src[base + li] : desc_key(A.src[base + li]);
-            key[i] = kk;
-            const uint32_t d = v ? ((kk >> sh) & 0xffu) : 0x100u;
-            const unsigned peers = __match_any_sync(FULL, d);
-            if (v && lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
-            __syncwarp();
-        }
+        warp_count(key, cnt_tile, 8 * pass, s_hist + warp * 256);
         __syncthreads();
-        uint32_t tot = 0;
         if (tid < 256) {
+            uint32_t tot = 0;
+#pragma unroll
+            for (int w = 0; w < RNW; ++w) tot += s_hist[w * 256 + tid];
+            cnt[(size_t)tid * nts + tile] = tot;
+        }
+        __syncthreads();   // sums read, staged keys read: both buffers may be reused
+    }
+    if (!ok) atomicOr(&A.ctl->status, ST_TIMEOUT);
+}
+
+constexpr int SB = 1024;   // scan: threads, one CTA per digit
+
+__global__ void __launch_bounds__(SB) radix_scan_kernel(SortArgs A, int pass) {
+    __shared__ uint32_t s_w[SB / 32];
+    pdl_enter();
+    const int64_t n = pass_n(A, pass);
+    if (n < 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t ntiles = (n + RTILE - 1) / RTILE, nts = cnt_stride(ntiles);
+    uint4 *row = reinterpret_cast<uint4 *>(A.tilecnt + (size_t)blockIdx.x * nts);
+    uint32_t carry = A.dbase[pass * 256 + blockIdx.x];
+    const int64_t nv = nts / 4;   // 16-byte vectors of the row (entries past ntiles are never read)
+    for (int64_t v0 = 0; v0 < nv; v0 += SB) {
+        const int64_t vi = v0 + tid;
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (vi < nv) x = row[vi];
+        const uint32_t t4 = x.x + x.y + x.z + x.w;
+        uint32_t inc = t4;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(FULL, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (lane == 31) s_w[warp] = inc;
+        __syncthreads();
+        uint32_t wofs = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < SB / 32; ++w) {
+            const uint32_t c = s_w[w];
+            wofs += w < warp ? c : 0u;
+            total += c;
+        }
+        __syncthreads();   // s_w is rewritten by the next chunk
+        if (vi < nv) {
+            uint32_t e = carry + wofs + inc - t4;
+            uint4 o;
+            o.x = e; e += x.x;
+            o.y = e; e += x.y;
+            o.z = e; e += x.z;
+            o.w = e;
+            row[vi] = o;
+        }
+        carry += total;
+    }
+}
+
+__global__ void __launch_bounds__(RB, 2) radix_scatter_kernel(SortArgs A, int pass) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + STAGE_BYTES);   // RNW * 256
+    uint32_t *s_dstart = s_hist + RNW * 256;                           // 256: in-tile digit start
+    uint32_t *s_gofs = s_dstart + 256;                                 // 256: global offset - dstart
+    __shared__ bool s_last;
+    pdl_enter();
+    const int64_t n = pass_n(A, pass);
+    if (n < 0) return;
+    Ctl *ctl = A.ctl;
+    const int cur = ctl->sort_cur;
+    const uint32_t *src = pass_keys_in(A, cur);
+    uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int sh = 8 * pass;
+    const int64_t ntiles = (n + RTILE - 1) / RTILE, nts = cnt_stride(ntiles);
+    const uint32_t *ofs = A.tilecnt;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    TileStage S;
+    stage_init(S, A, src, n, smem);
+    uint32_t ph = 0;
+    bool ok = true;
+    int slot = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, slot ^= 1) {
+        if (tid == 0 && tile + gridDim.x < ntiles) stage_issue(S, slot ^ 1, tile + gridDim.x);
+        const int cnt_tile = (int)min((int64_t)RTILE, n - tile * RTILE);
+        uint32_t key[RK];
+        ok &= stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
+        // this tile's buffer becomes its scatter buffer once every key is in registers
+        uint32_t *s_keys = S.buf + slot * RTILE;
+        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
+        __syncthreads();
+        uint32_t *my_hist = s_hist + warp * 256;
+        warp_count(key, cnt_tile, sh, my_hist);
+        __syncthreads();
+        if (tid < 256) {   // per digit: exclusive offsets of the warps, tile total
+            uint32_t tot = 0;
+#pragma unroll
             for (int w = 0; w < RNW; ++w) {
                 const uint32_t c = s_hist[w * 256 + tid];
                 s_hist[w * 256 + tid] = tot;
                 tot += c;
             }
-            // publish this tile's digit count, then look back for the exclusive prefix
-            unsigned long long *lb = A.lookback + (size_t)tile * 256 + tid;
-            uint32_t excl = 0;
-            if (tile == 0) {
-                st_release_u64(lb, lb_pack(LB_PREFIX, epoch, tot));
-            } else {
-                st_release_u64(lb, lb_pack(LB_AGG, epoch, tot));
-                for (int p = tile - 1; p >= 0;) {
-                    const unsigned long long *q = A.lookback + (size_t)p * 256 + tid;
-                    unsigned long long v;
-                    int it = 0;
-                    for (;;) {
-                        v = ld_acquire_u64(q);
-                        if (((v >> 32) & 0x3fffffffu) == (epoch & 0x3fffffffu) && (v >> 62) != 0) break;
-                        if (++it > A.spin_cap) {
-                            atomicOr(&ctl->status, ST_TIMEOUT);
-                            v = LB_PREFIX;   // give up: treat as a zero prefix
-                            break;
-                        }
-                        __nanosleep(32);
-                    }
-                    excl += (uint32_t)(v & 0xffffffffu);
-                    if ((v >> 62) == 2) break;
-                    --p;
-                }
-                st_release_u64(lb, lb_pack(LB_PREFIX, epoch, excl + tot));
-            }
-            s_gofs[tid] = A.dbase[pass * 256 + tid] + excl;
-            s_dstart[tid] = tot;   // temporarily the tile total of digit tid
+            s_dstart[tid] = tot;
+            s_gofs[tid] = __ldg(ofs + (size_t)tid * nts + tile);
         }
         __syncthreads();
         if (warp == 0) {   // exclusive scan of the 256 in-tile digit totals
@@ -300,20 +483,21 @@ __global__ void __launch_bounds__(RB, 1) radix_pass_kernel(SortArgs A, int pass,
             __syncwarp();
         }
         __syncthreads();
+        // runs of one digit are consecutive in s_keys and in dst: coalesced writes
         for (int i = tid; i < cnt_tile; i += RB) {
             const uint32_t kk = s_keys[i];
             dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
         }
         __syncthreads();
     }
-    // the last CTA to finish publishes the new key buffer and rearms the counters
+    if (!ok) atomicOr(&ctl->status, ST_TIMEOUT);
+    // the last CTA to finish publishes the new key buffer
     __threadfence();
     __syncthreads();
     if (tid == 0) s_last = atomicAdd(&ctl->ticket[5], 1u) == gridDim.x - 1;
     __syncthreads();
     if (s_last && tid == 0) {
         ctl->sort_cur = cur >= 0 ? (cur ^ 1) : 0;
-        ctl->tile_ctr[pass] = 0u;
         ctl->ticket[5] = 0u;
     }
 }
@@ -335,7 +519,7 @@ __device__ __forceinline__ double sorted_val(const uint32_t *keys, const float *
 __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, double t, double inv_t) {
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);                 // LTILE
-    void *scratch = smem + (LTILE + LTILE / 32) * 4;                         // >= 6 KB
+    void *scratch = smem + LOC_KEY_WORDS * 4;                                // >= 6 KB
     __shared__ bool s_last;
     __shared__ int s_tstar;
     __shared__ double s_tab[32];
@@ -366,18 +550,43 @@ __global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, dou
         if (j >= n) return bot;
         return sorted_val(keys_cur, A.src, j);
     };
+    // staged tile: s_keys[spad(i + 1)] holds sorted position tile*LTILE + i for
+    // i = -1 .. cnt (the two halo entries are the neighbours or the seeds)
+    const uint32_t key_top = desc_key((float)top), key_bot = desc_key((float)bot);
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t j0 = tile * LTILE + (int64_t)tid * LK;
-        const int64_t j1 = min(j0 + LK, n) - 1;
+        const int64_t t0 = tile * LTILE;
+        const int cnt = (int)min((int64_t)LTILE, n - t0);
+        uint32_t kv[LK];
+#pragma unroll
+        for (int u = 0; u < LK; ++u) {   // coalesced, all loads in flight at once
+            const int i = u * LB + tid;
+            kv[u] = 0u;
+            if (i < cnt) kv[u] = keys_cur ? __ldcs(keys_cur + t0 + i) : desc_key(__ldg(A.src + t0 + i));
+        }
+#pragma unroll
+        for (int u = 0; u < LK; ++u) {
+            const int i = u * LB + tid;
+            if (i < cnt) s_keys[spad(i + 1)] = kv[u];
+        }
+        if (tid == 0) {
+            s_keys[spad(0)] = t0 == 0 ? key_top
+                                      : (keys_cur ? keys_cur[t0 - 1] : desc_key(A.src[t0 - 1]));
+            s_keys[spad(cnt + 1)] = t0 + cnt >= n ? key_bot
+                                      : (keys_cur ? keys_cur[t0 + cnt] : desc_key(A.src[t0 + cnt]));
+        }
+        __syncthreads();
+        auto sval = [&](int i) -> double { return (double)desc_key_to_float(s_keys[spad(i + 1)]); };
+        const int l0 = tid * LK;
+        const int l1 = min(l0 + LK, cnt) - 1;
         Aff mp = aff_id(), mq = aff_id();
         double d_last = 0.0;
-        if (j0 < n) {
-            double cprev = val(j0 - 1);
-            double c = val(j0);
+        if (l0 < cnt) {
+            double cprev = sval(l0 - 1);
+            double c = sval(l0);
             double dprev = (cprev == CUDART_INF || c == -CUDART_INF) ? 0.0 : link_exp((cprev - c) * s2d, s_tab);
-            for (int64_t j = j0; j <= j1; ++j) {
+            for (int j = l0; j <= l1; ++j) {
                 mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
-                const double cn = val(j + 1);
+                const double cn = sval(j + 1);
                 const double d = (c == CUDART_INF || cn == -CUDART_INF) ? 0.0 : link_exp((c - cn) * s2d, s_tab);
                 mq = {mq.a * d, mq.s + mq.a};
                 dprev = d;
@@ -497,24 +706,29 @@ cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) 
     (void)t;
     const int64_t cap = A.cap;
     static bool attr = false;
-    const size_t smem = (size_t)RTILE * 4 + (size_t)RNW * 256 * 4 + 2 * 256 * 4;
+    const size_t smem_c = STAGE_BYTES + (size_t)RNW * 256 * 4;
+    const size_t smem = STAGE_BYTES + (size_t)RNW * 256 * 4 + 2 * 256 * 4;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(radix_pass_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(radix_count_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(radix_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    int64_t hg = (cap + HB * 16 - 1) / (HB * 16);
-    if (hg > (int64_t)num_sms() * 2) hg = (int64_t)num_sms() * 2;
+    int64_t hg = (cap + HB * 32 - 1) / (HB * 32);
+    if (hg > (int64_t)num_sms() * 4) hg = (int64_t)num_sms() * 4;
     int hgrid = (int)hg;
     if (hgrid < 1) hgrid = 1;
     cudaError_t e = launch_k(radix_hist_kernel, hgrid, HB, 0, st, A);
     if (e != cudaSuccess) return e;
     int64_t pt = (cap + RTILE - 1) / RTILE;
-    if (pt > num_sms()) pt = num_sms();   // persistent: one CTA per SM claims tiles in order
+    if (pt > 2 * num_sms()) pt = 2 * num_sms();   // two CTAs per SM, tiles grid-strided
     const unsigned ptiles = (unsigned)pt;
     for (int pass = 0; pass < 4; ++pass) {
-        e = launch_k(radix_pass_kernel, ptiles, RB, smem, st, A, pass, A.epoch * 4u + (uint32_t)pass);
+        e = launch_k(radix_count_kernel, ptiles, RB, smem_c, st, A, pass);
+        if (e == cudaSuccess) e = launch_k(radix_scan_kernel, 256u, SB, 0, st, A, pass);
+        if (e == cudaSuccess) e = launch_k(radix_scatter_kernel, ptiles, RB, smem, st, A, pass);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -522,7 +736,7 @@ cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) 
 
 cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st) {
     static bool attr = false;
-    const size_t smem = (size_t)(LTILE + LTILE / 32) * 4 + 16384;
+    const size_t smem = (size_t)LOC_KEY_WORDS * 4 + 16384;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(locate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);

@@ -58,12 +58,10 @@ struct SortArgs {
     uint32_t *keys[2];         // ping-pong key buffers [cap]
     unsigned long long *hist;  // [4][256]
     uint32_t *dbase;           // [4][256]
-    unsigned long long *lookback;  // [tiles][256]
+    uint32_t *tilecnt;         // [256][stride]: per-tile digit counts, then their offsets
     double *tilebuf;           // locate per-tile data
     Ctl *ctl;
     int32_t gate;
-    int32_t spin_cap;
-    uint32_t epoch;            // distinct per launch sequence (look-back tags)
     int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
     double k, t;               // budget and temperature (all-equal shortcut)
 };

@@ -114,6 +114,18 @@ def test_device_sort_path(L, orc, n, dist):
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
 
 
+@pytest.mark.parametrize("rows,n", [(3, 40_001), (2, 65_538)])
+def test_device_sort_path_rows_unaligned(L, orc, rows, n):
+    # rows after the first start off a 16-byte boundary (odd n, or n = 2 mod 4):
+    # the sort's first pass and the histogram take their element-wise paths there
+    r, g = W.small_case("normal", rows, n, seed=11)
+    k, t = n / 50.0, 0.05
+    p, b, st, grad = run(L, r, k, t, opts=L.options(force_path=L.PATH_FULLSORT), g_np=g)
+    assert st["rc"] == 0
+    for i in range(rows):
+        check_row(orc, r[i], g[i], k, t, p[i], b[i], grad[i])
+
+
 # ----------------------------------------------------------- bracketing --
 def check_bracket_integers(orc, r, k, t, st, seed, s, delta):
     br = orc.bracket(r, k, t, seed, s, delta)
