@@ -432,9 +432,10 @@ struct OobAcc {
 // Append a band score at a warp-aggregated slot of the band buffer (the count
 // keeps going past the capacity so the overflow is visible).
 __device__ __forceinline__ void band_push(float x, bool inb, float *band, unsigned long long cap,
-                                          unsigned long long *ctr, int lane) {
+                                          unsigned long long *ctr, int lane, Ctl *ctl) {
     const unsigned m = __ballot_sync(FULL, inb);
     if (!m) return;
+    band_range_update(ctl, inb ? desc_key(x) : 0u, inb ? ~desc_key(x) : 0u);
     const int leader = __ffs(m) - 1;
     unsigned long long base = 0;
     if (lane == leader) base = atomicAdd(ctr, (unsigned long long)__popc(m));
@@ -501,7 +502,7 @@ __device__ __forceinline__ void tier4(const float4 v, bool equal, float af, doub
 // slots: one warp scan and one atomic per warp (the count keeps going past the
 // capacity so the overflow is visible).
 __device__ __forceinline__ void band_push4(const float4 v, int m, float *band, unsigned long long cap,
-                                           unsigned long long *ctr, int lane) {
+                                           unsigned long long *ctr, int lane, Ctl *ctl) {
     const int cnt = __popc(m);
     int inc = cnt;
 #pragma unroll
@@ -511,6 +512,18 @@ __device__ __forceinline__ void band_push4(const float4 v, int m, float *band, u
     }
     const int total = __shfl_sync(FULL, inc, 31);
     if (total == 0) return;
+    {
+        uint32_t kmax = 0u, kinv = 0u;
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (m & (1 << i)) {
+                const uint32_t kk = desc_key(vv[i]);
+                kmax = max(kmax, kk);
+                kinv = max(kinv, ~kk);
+            }
+        band_range_update(ctl, kmax, kinv);
+    }
     unsigned long long base = 0;
     if (lane == 31) base = atomicAdd(ctr, (unsigned long long)total);
     base = __shfl_sync(FULL, base, 31) + (unsigned long long)(inc - cnt);
@@ -568,7 +581,7 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
             tier4<true>(v, equal, E.aL, E.daL, E, a.hL, a.hL2);
             tier4<false>(v, equal, E.aR, E.daR, E, a.lR, a.lR2);
         }
-        if (!CERT) band_push4(v, ok ? 0xF : 0, P.band, cap, &P.ctl->c_band, lane);
+        if (!CERT) band_push4(v, ok ? 0xF : 0, P.band, cap, &P.ctl->c_band, lane, P.ctl);
         return;
     }
     const bool b0 = oob_one<MODE>(v.x, ok, E, a);
@@ -577,7 +590,7 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
     const bool b3 = oob_one<MODE>(v.w, ok, E, a);
     if (!CERT) {
         const int m = (b0 ? 1 : 0) | (b1 ? 2 : 0) | (b2 ? 4 : 0) | (b3 ? 8 : 0);
-        if (__any_sync(FULL, m != 0)) band_push4(v, m, P.band, cap, &P.ctl->c_band, lane);
+        if (__any_sync(FULL, m != 0)) band_push4(v, m, P.band, cap, &P.ctl->c_band, lane, P.ctl);
     }
 }
 
@@ -635,7 +648,7 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
         const bool ok = j < n;
         const float x = ok ? P.r[j] : 0.f;
         const bool bb = oob_one<MODE>(x, ok, E, acc);
-        if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane);
+        if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane, ctl);
     }
     if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
     if constexpr (MODE == OOB_STREAM) {

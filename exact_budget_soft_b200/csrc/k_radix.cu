@@ -5,19 +5,7 @@
 // path (step 3) that exceeds the one-CTA capacity.
 //
 // Sort: keys-only LSD radix sort of the descending-order uint32 keys, 8-bit
-// digits, reduce-then-scan per digit:
-//   radix_hist_kernel     one read: all four digit histograms (per-thread run
-//                         length combining, so long runs of tied scores cost
-//                         one shared atomic per run), exclusive digit bases,
-//                         and the digits on which every key agrees (those
-//                         passes are skipped; all four: solved in closed form);
-//   radix_count_kernel    per 8192-key tile, its 256 digit counts;
-//   radix_scan_kernel     per digit, the counts of earlier tiles -> offsets;
-//   radix_scatter_kernel  per tile, a stable in-tile ranking (per-warp digit
-//                         histograms, __match_any_sync), a shared-memory
-//                         scatter and coalesced runs of writes at the offsets.
-// The count and scatter kernels stage each CTA's next tile in shared memory by
-// one bulk copy while they work on the current one.  No CTA waits on another.
+// digits, in one cooperative kernel (radix_sort_kernel, described below).
 // Locate: one kernel; every CTA reduces one tile of sorted values to its two
 // affine maps (prefix P, suffix Q); the last CTA scans the tile maps, finds the
 // tile whose end brackets G = k, re-scans that tile in shared memory and takes
@@ -55,6 +43,7 @@ __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
         if (c->path != 2) return -1;
         const unsigned long long cb = c->c_band;
         if (cb <= (unsigned long long)A.small_cap || cb > (unsigned long long)A.cap) return -1;
+        if (band_tied(c)) return -1;   // one tied value: the band solver takes it in closed form
         return (int64_t)cb;
     }
     if (A.gate == GATE_FALLBACK) {
@@ -63,10 +52,8 @@ __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
     return A.n_host;
 }
 
-// n copies of one value c, between the seeds of the locate step (the band of a
-// tied level, or a row whose scores are all equal): the threshold curve is
-// constant across the run, G(c) = m0 + n/2 - d_top P_top/2 + d_bot Q_bot/2, and
-// (G decreasing) the root lies in [bot, c] when G(c) <= k, else in [c, top).
+// n copies of one value c, between the seeds of the locate step (a row whose
+// scores are all equal, or the band of one tied level): closed form.
 __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
     Ctl *ctl = A.ctl;
     double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
@@ -77,141 +64,33 @@ __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
         bot = (double)ctl->a_L;
         Q_bot = ctl->S_L;
     }
-    const double c = (double)A.src[0];
-    const double d_top = top == CUDART_INF ? 0.0 : exp((c - top) / A.t);
-    const double d_bot = bot == -CUDART_INF ? 0.0 : exp((bot - c) / A.t);
-    const double nn = (double)n;
-    const double Gc = m0 + 0.5 * nn - 0.5 * d_top * P_top + 0.5 * d_bot * Q_bot;
-    double b;
-    if (Gc <= A.k) {   // G decreasing: the root is at or below c
-        b = solve_interval(c, bot, m0 + nn, nn + d_top * P_top, Q_bot, d_bot, A.k, A.t);
-        ctl->j_star = n - 1;
-    } else {
-        b = solve_interval(top, c, m0, P_top, nn + d_bot * Q_bot, d_top, A.k, A.t);
-        ctl->j_star = -1;
-    }
-    ctl->b = b;
+    bool above = false;
+    ctl->b = solve_equal_run_values((double)A.src[0], (double)n, m0, top, P_top, bot, Q_bot, A.k, A.t, &above);
+    ctl->j_star = above ? n - 1 : -1;
     if (A.gate == GATE_FALLBACK) ctl->fallback_ran = 1;
 }
 
-// ------------------------------------------------------------ histogram --
-__global__ void __launch_bounds__(HB) radix_hist_kernel(SortArgs A) {
-    __shared__ uint32_t h[4][256];
-    __shared__ bool s_last;
-    __shared__ int s_trivial[4];
-    pdl_enter();
-    const int64_t n = gated_n(A);
-    if (n < 0) return;
-    const int tid = threadIdx.x;
-    for (int i = tid; i < 4 * 256; i += HB) (&h[0][0])[i] = 0;
-    __syncthreads();
-    uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-    uint32_t cnt[4] = {0, 0, 0, 0};
-    auto count = [&](float x) {   // run-length combining per digit
-        const uint32_t key = desc_key(x);
-#pragma unroll
-        for (int d = 0; d < 4; ++d) {
-            const uint32_t bin = (key >> (8 * d)) & 0xffu;
-            if (bin == cur[d]) {
-                ++cnt[d];
-            } else {
-                if (cnt[d]) atomicAdd(&h[d][cur[d]], cnt[d]);
-                cur[d] = bin;
-                cnt[d] = 1;
-            }
-        }
-    };
-    // each thread takes chunks of 16 consecutive scores (four 16-byte loads, so
-    // runs of tied scores combine); the next chunk is loaded while this one is
-    // counted (one copy of the counting code: a rotation, not an unrolled batch)
-    const int64_t gstride = (int64_t)gridDim.x * HB;
-    const int64_t nch = (reinterpret_cast<uintptr_t>(A.src) & 15u) == 0 ? n / 16 : 0;
-    const float4 *src4 = reinterpret_cast<const float4 *>(A.src);
-    auto load_chunk = [&](int64_t c, float4 (&v)[4]) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = c < nch ? __ldg(src4 + c * 4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-    };
-    float4 cur4[4];
-    int64_t c = (int64_t)blockIdx.x * HB + tid;
-    load_chunk(c, cur4);
-#pragma unroll 1
-    for (; c < nch; c += gstride) {
-        float4 nxt4[4];
-        load_chunk(c + gstride, nxt4);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            count(cur4[q].x);
-            count(cur4[q].y);
-            count(cur4[q].z);
-            count(cur4[q].w);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) cur4[q] = nxt4[q];
-    }
-    for (int64_t i = nch * 16 + (int64_t)blockIdx.x * HB + tid; i < n; i += gstride) count(__ldg(A.src + i));
-#pragma unroll
-    for (int d = 0; d < 4; ++d)
-        if (cnt[d]) atomicAdd(&h[d][cur[d]], cnt[d]);
-    __syncthreads();
-    for (int i = tid; i < 4 * 256; i += HB) {
-        const uint32_t c = (&h[0][0])[i];
-        if (c) atomicAdd(A.hist + i, (unsigned long long)c);
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&A.ctl->ticket[4], 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // exclusive digit bases (thread tid owns bin tid of every digit); a digit
-    // whose histogram has one bin holding every key is skipped
-    static_assert(HB == 256, "one thread per bin");
-    __shared__ uint32_t s_wsum[HB / 32];
-    for (int d = 0; d < 4; ++d) {
-        const uint32_t c = (uint32_t)__ldcg(A.hist + d * 256 + tid);
-        const int lane = tid & 31, warp = tid >> 5;
-        uint32_t inc = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t p = __shfl_up_sync(FULL, inc, o);
-            if (lane >= o) inc += p;
-        }
-        if (lane == 31) s_wsum[warp] = inc;
-        __syncthreads();
-        uint32_t off = 0;
-        for (int w = 0; w < warp; ++w) off += s_wsum[w];
-        A.dbase[d * 256 + tid] = off + inc - c;
-        const int triv = __syncthreads_or(c == (uint32_t)n);
-        if (tid == 0) s_trivial[d] = triv;
-        __syncthreads();
-    }
-    for (int i = tid; i < 4 * 256; i += HB) A.hist[i] = 0ull;   // ready for the next sort
-    if (tid == 0) {
-        A.ctl->sort_skip = s_trivial[0] | (s_trivial[1] << 1) | (s_trivial[2] << 2) | (s_trivial[3] << 3);
-        const bool all_equal = s_trivial[0] && s_trivial[1] && s_trivial[2] && s_trivial[3];
-        A.ctl->sort_solved = all_equal ? 1 : 0;
-        if (all_equal) solve_equal_run(A, n);
-        A.ctl->sort_cur = -1;
-        A.ctl->ticket[4] = 0u;
-    }
-}
-
-// ----------------------------------------------------------- one digit --
-// A pass (skipped when every key agrees on its digit) is reduce-then-scan:
-//   radix_count_kernel    each tile's 256 digit counts -> cnt[d][tile]
-//   radix_scan_kernel     per digit d, cnt[d][.] -> global offsets in place:
-//                         dbase[d] + the count of d in all earlier tiles
-//   radix_scatter_kernel  each tile ranks its keys stably in shared memory and
-//                         writes every digit's run at the run's offset
-// No CTA ever waits on another, so the pass has no spin waits at all; the
-// price is one more read of the keys than a single-sweep sort.
-
-// Row stride of the count table (a multiple of 4 entries, for 16-byte loads).
-__host__ __device__ __forceinline__ int64_t cnt_stride(int64_t ntiles) { return (ntiles + 3) & ~int64_t(3); }
-
-__device__ __forceinline__ const uint32_t *pass_keys_in(const SortArgs &A, int cur) {
-    return cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
-}
+// ------------------------------------------------------------ sort --
+// One cooperative kernel (every CTA resident, bounded grid barriers between
+// phases).  CTA c owns a contiguous chunk of tiles [t0, t1) in every pass.
+//
+//   phase H   each CTA: the four digit histograms of its chunk (per-thread run
+//             length combining, so long runs of tied scores cost one shared
+//             atomic per run) -> chunk counts of all four digits, and the
+//             global histograms.  Barrier.  Every CTA then derives the digit
+//             bases and the digits on which every key agrees (those passes
+//             are skipped; all four: one value, solved in closed form).
+//   pass p    count (not for the first pass run: phase H counted the input
+//             order): the chunk's digit-p counts.  Barrier.  Each CTA sums the
+//             counts of the chunks before its own (its global start of every
+//             digit), then walks its tiles in order: a stable in-tile ranking
+//             (per-warp digit histograms, __match_any_sync), a shared-memory
+//             scatter and coalesced runs of writes, each digit's running
+//             offset advanced by the tile's count.  Barrier.
+//
+// Each CTA stages its next tile in shared memory by one bulk copy while it
+// works on the current one.  Data written inside the kernel by other CTAs is
+// read through L2 (ld.global.cg or bulk copies), never through L1.
 
 // The tile's keys, warp-striped (key i of lane l of warp w is tile element
 // w*32*RK + i*32 + l), all RK loads in flight at once; keys past the end of the
@@ -223,7 +102,7 @@ __device__ __forceinline__ void load_tile(const SortArgs &A, const uint32_t *src
     if (src) {
 #pragma unroll
         for (int i = 0; i < RK; ++i)
-            key[i] = l0 + i * 32 < cnt_tile ? __ldcs(src + base + l0 + i * 32) : 0xffffffffu;
+            key[i] = l0 + i * 32 < cnt_tile ? __ldcg(src + base + l0 + i * 32) : 0xffffffffu;
     } else {
         float x[RK];
 #pragma unroll
@@ -233,14 +112,13 @@ __device__ __forceinline__ void load_tile(const SortArgs &A, const uint32_t *src
     }
 }
 
-// Double-buffered tile staging for the pass kernels: tiles are grid-strided, so
-// each CTA knows its next tile and copies it (one bulk copy, completion counted
-// on an mbarrier) while it works on the current one.  Only full tiles of a
-// 16-byte-aligned source are staged; the rest take plain loads.
+// Double-buffered tile staging: only full tiles of a 16-byte-aligned source
+// are copied (one bulk copy each, completion counted on an mbarrier); the
+// ragged last tile takes plain loads.
 struct TileStage {
     uint32_t *buf;      // 2 * RTILE words
     uint64_t *bar;      // 2 mbarriers
-    const char *gsrc;   // 4-byte elements: the keys, or the scores on the first pass
+    const char *gsrc;   // 4-byte elements: the keys, or the scores
     bool bulk_ok;
     int64_t n;
 };
@@ -257,20 +135,9 @@ __device__ __forceinline__ void stage_issue(const TileStage &S, int slot, int64_
     bulk_load(S.buf + slot * RTILE, S.gsrc + (size_t)tile * RTILE * 4, RTILE * 4, &S.bar[slot]);
 }
 
-__device__ __forceinline__ void stage_init(TileStage &S, const SortArgs &A, const uint32_t *src, int64_t n,
-                                           unsigned char *smem) {
-    S.buf = reinterpret_cast<uint32_t *>(smem);
-    S.bar = reinterpret_cast<uint64_t *>(smem + 2 * RTILE * 4);
+__device__ __forceinline__ void stage_source(TileStage &S, const SortArgs &A, const uint32_t *src) {
     S.gsrc = src ? reinterpret_cast<const char *>(src) : reinterpret_cast<const char *>(A.src);
     S.bulk_ok = (reinterpret_cast<uintptr_t>(S.gsrc) & 15u) == 0;
-    S.n = n;
-    if (threadIdx.x == 0) {
-        mbar_init(&S.bar[0], 1);
-        mbar_init(&S.bar[1], 1);
-        mbar_init_fence();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && (int64_t)blockIdx.x * RTILE < n) stage_issue(S, 0, blockIdx.x);
 }
 
 // The tile's keys into registers: from its staged copy (waiting, bounded, for
@@ -311,195 +178,242 @@ __device__ __forceinline__ void warp_count(const uint32_t (&key)[RK], int cnt_ti
     }
 }
 
-// Common gate of the three pass kernels: the element count, or < 0 to return.
-__device__ __forceinline__ int64_t pass_n(const SortArgs &A, int pass) {
-    const int64_t n = gated_n(A);
-    if (n < 0) return -1;
-    if (A.ctl->sort_skip & (1 << pass)) return -1;   // every key agrees on this digit
-    return n;
-}
-
-__global__ void __launch_bounds__(RB, 2) radix_count_kernel(SortArgs A, int pass) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + STAGE_BYTES);   // RNW * 256
-    pdl_enter();
-    const int64_t n = pass_n(A, pass);
-    if (n < 0) return;
-    const uint32_t *src = pass_keys_in(A, A.ctl->sort_cur);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int64_t ntiles = (n + RTILE - 1) / RTILE, nts = cnt_stride(ntiles);
-    uint32_t *cnt = A.tilecnt;
-    TileStage S;
-    stage_init(S, A, src, n, smem);
-    uint32_t ph = 0;
+// Walks the CTA's chunk of tiles in order with one tile staged ahead, calling
+// body(tile, cnt_tile, key) with every thread's keys; a barrier follows each
+// body, so the staging buffers are free again.  Returns false if a wait gave up.
+template <typename Body>
+__device__ __forceinline__ bool walk_chunk(TileStage &S, const SortArgs &A, const uint32_t *src, int64_t t0,
+                                           int64_t t1, uint32_t &ph, Body &&body) {
     bool ok = true;
+    stage_source(S, A, src);
+    if (threadIdx.x == 0 && t0 < t1) stage_issue(S, 0, t0);
     int slot = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, slot ^= 1) {
-        if (tid == 0 && tile + gridDim.x < ntiles) stage_issue(S, slot ^ 1, tile + gridDim.x);
-        const int cnt_tile = (int)min((int64_t)RTILE, n - tile * RTILE);
+    for (int64_t tile = t0; tile < t1; ++tile, slot ^= 1) {
+        if (threadIdx.x == 0 && tile + 1 < t1) stage_issue(S, slot ^ 1, tile + 1);
+        const int cnt_tile = (int)min((int64_t)RTILE, S.n - tile * RTILE);
         uint32_t key[RK];
         ok &= stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
-        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
+        body(tile, cnt_tile, key, S.buf + slot * RTILE);
         __syncthreads();
-        warp_count(key, cnt_tile, 8 * pass, s_hist + warp * 256);
-        __syncthreads();
-        if (tid < 256) {
-            uint32_t tot = 0;
-#pragma unroll
-            for (int w = 0; w < RNW; ++w) tot += s_hist[w * 256 + tid];
-            cnt[(size_t)tid * nts + tile] = tot;
-        }
-        __syncthreads();   // sums read, staged keys read: both buffers may be reused
     }
-    if (!ok) atomicOr(&A.ctl->status, ST_TIMEOUT);
+    return ok;
 }
 
-constexpr int SB = 1024;   // scan: threads, one CTA per digit
+constexpr size_t SORT_SMEM = STAGE_BYTES + (size_t)(RNW * 256 + 4 * 256 + 4 * 256) * 4;
+constexpr int SORT_GMAX = 320;   // CTAs of the sort grid at most (chunk counts per digit)
 
-__global__ void __launch_bounds__(SB) radix_scan_kernel(SortArgs A, int pass) {
-    __shared__ uint32_t s_w[SB / 32];
-    pdl_enter();
-    const int64_t n = pass_n(A, pass);
-    if (n < 0) return;
+__global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + STAGE_BYTES);   // RNW * 256: per-warp digit counts
+    uint32_t *s_dstart = s_hist + RNW * 256;   // 256: in-tile digit start
+    uint32_t *s_gofs = s_dstart + 256;         // 256: global offset - in-tile start
+    uint32_t *s_run = s_gofs + 256;            // 256: running global offset of each digit
+    uint32_t *s_tot = s_run + 256;             // 256: scratch (tile totals)
+    uint32_t *s_h4 = s_tot + 256;              // 4 * 256: phase-H histograms, then digit bases
+    __shared__ int s_skip, s_solved;
+    pdl_wait();
+    const int64_t n = gated_n(A);
+    if (n < 0) return;   // the gate reads the same control words in every CTA
+    Ctl *ctl = A.ctl;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t ntiles = (n + RTILE - 1) / RTILE, nts = cnt_stride(ntiles);
-    uint4 *row = reinterpret_cast<uint4 *>(A.tilecnt + (size_t)blockIdx.x * nts);
-    uint32_t carry = A.dbase[pass * 256 + blockIdx.x];
-    const int64_t nv = nts / 4;   // 16-byte vectors of the row (entries past ntiles are never read)
-    for (int64_t v0 = 0; v0 < nv; v0 += SB) {
-        const int64_t vi = v0 + tid;
-        uint4 x = make_uint4(0u, 0u, 0u, 0u);
-        if (vi < nv) x = row[vi];
-        const uint32_t t4 = x.x + x.y + x.z + x.w;
-        uint32_t inc = t4;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int64_t ntiles = (n + RTILE - 1) / RTILE;
+    const int64_t t0 = (int64_t)c * ntiles / G, t1 = (int64_t)(c + 1) * ntiles / G;
+    uint32_t *csum = A.chunkcnt;   // [4][256][G]
+    auto bar = [&]() { grid_sync(&ctl->gbar_count, &ctl->gbar_gen, A.spin_cap, &ctl->status); };
+    TileStage S;
+    S.buf = reinterpret_cast<uint32_t *>(smem);
+    S.bar = reinterpret_cast<uint64_t *>(smem + 2 * RTILE * 4);
+    S.n = n;
+    if (tid == 0) {
+        mbar_init(&S.bar[0], 1);
+        mbar_init(&S.bar[1], 1);
+        mbar_init_fence();
+    }
+    for (int i = tid; i < 4 * 256; i += RB) s_h4[i] = 0;
+    __syncthreads();
+    uint32_t ph = 0;
+    bool ok = true;
+
+    // ---- phase H: the chunk's four digit histograms
+    {
+        uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        uint32_t cnt[4] = {0, 0, 0, 0};
+        ok &= walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[RK], uint32_t *) {
+            const int l0 = warp * 32 * RK + lane;
+#pragma unroll
+            for (int i = 0; i < RK; ++i) {
+                if (l0 + i * 32 >= cnt_tile) break;
+#pragma unroll
+                for (int d = 0; d < 4; ++d) {
+                    const uint32_t bin = (key[i] >> (8 * d)) & 0xffu;
+                    if (bin == cur[d]) {
+                        ++cnt[d];
+                    } else {
+                        if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
+                        cur[d] = bin;
+                        cnt[d] = 1;
+                    }
+                }
+            }
+        });
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
+            if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
+        __syncthreads();
+        for (int i = tid; i < 4 * 256; i += RB) {
+            const uint32_t v = s_h4[i];
+            csum[(size_t)i * G + c] = v;
+            if (v) atomicAdd(A.hist + i, (unsigned long long)v);
+        }
+    }
+    bar();
+    // digit bases and skip flags, the same in every CTA (thread d owns bin d)
+    if (tid == 0) { s_skip = 0; s_solved = 0; }
+    __syncthreads();
+    for (int d4 = 0; d4 < 4; ++d4) {
+        uint32_t v = 0;
+        if (tid < 256) v = (uint32_t)__ldcg(A.hist + d4 * 256 + tid);
+        uint32_t inc = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(FULL, inc, o);
             if (lane >= o) inc += y;
         }
-        if (lane == 31) s_w[warp] = inc;
+        if (lane == 31 && tid < 256) s_tot[warp] = inc;
         __syncthreads();
-        uint32_t wofs = 0, total = 0;
-#pragma unroll
-        for (int w = 0; w < SB / 32; ++w) {
-            const uint32_t c = s_w[w];
-            wofs += w < warp ? c : 0u;
-            total += c;
+        if (tid < 256) {
+            uint32_t off = 0;
+            for (int w = 0; w < warp; ++w) off += s_tot[w];
+            s_h4[d4 * 256 + tid] = off + inc - v;   // exclusive base of bin tid
+            if (v == (uint32_t)n) atomicOr(&s_skip, 1 << d4);
         }
-        __syncthreads();   // s_w is rewritten by the next chunk
-        if (vi < nv) {
-            uint32_t e = carry + wofs + inc - t4;
-            uint4 o;
-            o.x = e; e += x.x;
-            o.y = e; e += x.y;
-            o.z = e; e += x.z;
-            o.w = e;
-            row[vi] = o;
-        }
-        carry += total;
+        __syncthreads();
     }
-}
-
-__global__ void __launch_bounds__(RB, 2) radix_scatter_kernel(SortArgs A, int pass) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + STAGE_BYTES);   // RNW * 256
-    uint32_t *s_dstart = s_hist + RNW * 256;                           // 256: in-tile digit start
-    uint32_t *s_gofs = s_dstart + 256;                                 // 256: global offset - dstart
-    __shared__ bool s_last;
-    pdl_enter();
-    const int64_t n = pass_n(A, pass);
-    if (n < 0) return;
-    Ctl *ctl = A.ctl;
-    const int cur = ctl->sort_cur;
-    const uint32_t *src = pass_keys_in(A, cur);
-    uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int sh = 8 * pass;
-    const int64_t ntiles = (n + RTILE - 1) / RTILE, nts = cnt_stride(ntiles);
-    const uint32_t *ofs = A.tilecnt;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    TileStage S;
-    stage_init(S, A, src, n, smem);
-    uint32_t ph = 0;
-    bool ok = true;
-    int slot = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, slot ^= 1) {
-        if (tid == 0 && tile + gridDim.x < ntiles) stage_issue(S, slot ^ 1, tile + gridDim.x);
-        const int cnt_tile = (int)min((int64_t)RTILE, n - tile * RTILE);
-        uint32_t key[RK];
-        ok &= stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
-        // this tile's buffer becomes its scatter buffer once every key is in registers
-        uint32_t *s_keys = S.buf + slot * RTILE;
-        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
-        __syncthreads();
-        uint32_t *my_hist = s_hist + warp * 256;
-        warp_count(key, cnt_tile, sh, my_hist);
-        __syncthreads();
-        if (tid < 256) {   // per digit: exclusive offsets of the warps, tile total
-            uint32_t tot = 0;
+    const int skip = s_skip;
+    int cur = -1;   // key buffer of the current order (-1: the scores)
+    if (skip == 15) {   // every key equal
+        if (c == 0 && tid == 0) solve_equal_run(A, n);
+    } else {
+        bool first = true;
+        for (int pass = 0; pass < 4; ++pass) {
+            if (skip & (1 << pass)) continue;
+            const int sh = 8 * pass;
+            const uint32_t *src = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
+            uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
+            uint32_t *crow = csum + (size_t)pass * 256 * G;   // [256][G] of this digit
+            if (!first) {   // the chunk's digit counts in the current order
+                for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
+                __syncthreads();
+                ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[RK], uint32_t *) {
+                    warp_count(key, cnt_tile, sh, s_hist + warp * 256);
+                });
+                if (tid < 256) {
+                    uint32_t tot = 0;
 #pragma unroll
-            for (int w = 0; w < RNW; ++w) {
-                const uint32_t c = s_hist[w * 256 + tid];
-                s_hist[w * 256 + tid] = tot;
-                tot += c;
+                    for (int w = 0; w < RNW; ++w) tot += s_hist[w * 256 + tid];
+                    crow[(size_t)tid * G + c] = tot;
+                }
+                bar();
             }
-            s_dstart[tid] = tot;
-            s_gofs[tid] = __ldg(ofs + (size_t)tid * nts + tile);
-        }
-        __syncthreads();
-        if (warp == 0) {   // exclusive scan of the 256 in-tile digit totals
-            uint32_t v[8], run = 0;
+            // global start of every digit in this chunk: base + counts of earlier
+            // chunks (a warp per digit, four digits' loads in flight at once)
+            for (int j = 0; j < 256 / RNW; j += 4) {
+                uint32_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { v[j] = s_dstart[lane * 8 + j]; run += v[j]; }
-            uint32_t inc = run;
+                for (int u = 0; u < SORT_GMAX / 32; ++u) {
+                    const int q = lane + 32 * u;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t p = __shfl_up_sync(FULL, inc, o);
-                if (lane >= o) inc += p;
+                    for (int jj = 0; jj < 4; ++jj)
+                        if (q < c) acc[jj] += __ldcg(crow + (size_t)(warp * (256 / RNW) + j + jj) * G + q);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t a = acc[jj];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+                    const int d = warp * (256 / RNW) + j + jj;
+                    if (lane == 0) s_run[d] = s_h4[pass * 256 + d] + a;
+                }
             }
-            uint32_t ex = inc - run;
+            __syncthreads();
+            ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[RK], uint32_t *s_keys) {
+                for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
+                __syncthreads();   // every key is in registers: s_keys is free too
+                uint32_t *my_hist = s_hist + warp * 256;
+                warp_count(key, cnt_tile, sh, my_hist);
+                __syncthreads();
+                if (tid < 256) {   // per digit: exclusive offsets of the warps, tile total
+                    uint32_t tot = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { const uint32_t c = v[j]; s_dstart[lane * 8 + j] = ex; ex += c; }
-        }
-        __syncthreads();
-        if (tid < 256) s_gofs[tid] -= s_dstart[tid];
-        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] += s_dstart[i & 255];
-        __syncthreads();
-        // scatter into shared memory by (digit, warp, traversal order): stable
+                    for (int w = 0; w < RNW; ++w) {
+                        const uint32_t cw = s_hist[w * 256 + tid];
+                        s_hist[w * 256 + tid] = tot;
+                        tot += cw;
+                    }
+                    s_tot[tid] = tot;
+                    s_gofs[tid] = s_run[tid];
+                    s_run[tid] += tot;
+                }
+                __syncthreads();
+                if (warp == 0) {   // exclusive scan of the 256 tile totals
+                    uint32_t v[8], run = 0;
 #pragma unroll
-        for (int i = 0; i < RK; ++i) {
-            const int li = warp * 32 * RK + i * 32 + lane;
-            const bool v = li < cnt_tile;
-            const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
-            const unsigned peers = __match_any_sync(FULL, d);
-            const int leader = __ffs(peers) - 1;
-            uint32_t bs = 0;
-            if (v && lane == leader) {
-                bs = my_hist[d];
-                my_hist[d] = bs + __popc(peers);
-            }
-            bs = __shfl_sync(FULL, bs, leader) + __popc(peers & lt_mask);
-            if (v) s_keys[bs] = key[i];
-            __syncwarp();
+                    for (int jj = 0; jj < 8; ++jj) { v[jj] = s_tot[lane * 8 + jj]; run += v[jj]; }
+                    uint32_t inc = run;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t y = __shfl_up_sync(FULL, inc, o);
+                        if (lane >= o) inc += y;
+                    }
+                    uint32_t ex = inc - run;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) { const uint32_t cc = v[jj]; s_dstart[lane * 8 + jj] = ex; ex += cc; }
+                }
+                __syncthreads();
+                if (tid < 256) s_gofs[tid] -= s_dstart[tid];
+                for (int i = tid; i < RNW * 256; i += RB) s_hist[i] += s_dstart[i & 255];
+                __syncthreads();
+                // scatter into shared memory by (digit, warp, traversal order): stable
+                const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+                for (int i = 0; i < RK; ++i) {
+                    const int li = warp * 32 * RK + i * 32 + lane;
+                    const bool v = li < cnt_tile;
+                    const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
+                    const unsigned peers = __match_any_sync(FULL, d);
+                    const int leader = __ffs(peers) - 1;
+                    uint32_t bs = 0;
+                    if (v && lane == leader) {
+                        bs = my_hist[d];
+                        my_hist[d] = bs + __popc(peers);
+                    }
+                    bs = __shfl_sync(FULL, bs, leader) + __popc(peers & lt_mask);
+                    if (v) s_keys[bs] = key[i];
+                    __syncwarp();
+                }
+                __syncthreads();
+                // runs of one digit are consecutive in s_keys and in dst: coalesced writes
+                for (int i = tid; i < cnt_tile; i += RB) {
+                    const uint32_t kk = s_keys[i];
+                    dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
+                }
+            });
+            bar();   // the pass's keys are all written before the next pass reads them
+            cur = cur == 0 ? 1 : 0;
+            first = false;
         }
-        __syncthreads();
-        // runs of one digit are consecutive in s_keys and in dst: coalesced writes
-        for (int i = tid; i < cnt_tile; i += RB) {
-            const uint32_t kk = s_keys[i];
-            dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
-        }
-        __syncthreads();
     }
     if (!ok) atomicOr(&ctl->status, ST_TIMEOUT);
-    // the last CTA to finish publishes the new key buffer
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&ctl->ticket[5], 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (s_last && tid == 0) {
-        ctl->sort_cur = cur >= 0 ? (cur ^ 1) : 0;
-        ctl->ticket[5] = 0u;
+    bar();   // every CTA has read the global histograms
+    if (c == 0) {
+        for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
+        if (tid == 0) {
+            ctl->sort_cur = cur;
+            ctl->sort_solved = skip == 15 ? 1 : 0;
+        }
     }
+    pdl_trigger();
 }
 
 // --------------------------------------------------------------- locate --
@@ -701,37 +615,27 @@ static int num_sms() {
     return sms;
 }
 
+int sort_grid_max() { return SORT_GMAX; }
+
 cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) {
     (void)k;
     (void)t;
-    const int64_t cap = A.cap;
-    static bool attr = false;
-    const size_t smem_c = STAGE_BYTES + (size_t)RNW * 256 * 4;
-    const size_t smem = STAGE_BYTES + (size_t)RNW * 256 * 4 + 2 * 256 * 4;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(radix_count_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(radix_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int resident = 0;   // CTAs of the sort kernel that fit the device at once
+    if (!resident) {
+        cudaError_t e = cudaFuncSetAttribute(radix_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SORT_SMEM);
         if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    int64_t hg = (cap + HB * 32 - 1) / (HB * 32);
-    if (hg > (int64_t)num_sms() * 4) hg = (int64_t)num_sms() * 4;
-    int hgrid = (int)hg;
-    if (hgrid < 1) hgrid = 1;
-    cudaError_t e = launch_k(radix_hist_kernel, hgrid, HB, 0, st, A);
-    if (e != cudaSuccess) return e;
-    int64_t pt = (cap + RTILE - 1) / RTILE;
-    if (pt > 2 * num_sms()) pt = 2 * num_sms();   // two CTAs per SM, tiles grid-strided
-    const unsigned ptiles = (unsigned)pt;
-    for (int pass = 0; pass < 4; ++pass) {
-        e = launch_k(radix_count_kernel, ptiles, RB, smem_c, st, A, pass);
-        if (e == cudaSuccess) e = launch_k(radix_scan_kernel, 256u, SB, 0, st, A, pass);
-        if (e == cudaSuccess) e = launch_k(radix_scatter_kernel, ptiles, RB, smem, st, A, pass);
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, radix_sort_kernel, RB, SORT_SMEM);
         if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        resident = per_sm * num_sms();
     }
-    return cudaSuccess;
+    int64_t g = (A.cap + RTILE - 1) / RTILE;
+    if (g > resident) g = resident;
+    if (g > SORT_GMAX) g = SORT_GMAX;
+    if (g < 1) g = 1;
+    return launch_coop(radix_sort_kernel, (unsigned)g, RB, SORT_SMEM, st, A);
 }
 
 cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st) {

@@ -49,6 +49,16 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
             if (tid == 0) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
             return;
         }
+        if (band_tied(ctl)) {   // one tied value, of any count: closed form
+            if (tid == 0) {
+                bool above = false;
+                ctl->b = solve_equal_run_values((double)desc_key_to_float(ctl->band_kmax), (double)cb,
+                                                (double)ctl->c_R, (double)ctl->a_R, ctl->S_R, (double)ctl->a_L,
+                                                ctl->S_L, k, t, &above);
+                ctl->j_star = above ? (int64_t)cb - 1 : -1;
+            }
+            return;
+        }
         if (cb > (unsigned long long)C::CAP) return;   // the device-wide sort takes it
         n = (int)cb;
         row = scores;

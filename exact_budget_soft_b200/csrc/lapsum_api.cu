@@ -105,14 +105,13 @@ struct Workspace {
     uint32_t *keys0 = nullptr;        size_t keys0_n = 0;
     uint32_t *keys1 = nullptr;        size_t keys1_n = 0;
     unsigned long long *hist = nullptr; size_t hist_n = 0;
-    uint32_t *dbase = nullptr;        size_t dbase_n = 0;
-    uint32_t *tilecnt = nullptr; size_t tilecnt_n = 0;
+    uint32_t *chunkcnt = nullptr; size_t chunkcnt_n = 0;
     double *tilebuf = nullptr;        size_t tilebuf_n = 0;
 
     void release() {
         cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(hist1); cudaFree(band);
-        cudaFree(keys0); cudaFree(keys1); cudaFree(hist); cudaFree(dbase);
-        cudaFree(tilecnt); cudaFree(tilebuf);
+        cudaFree(keys0); cudaFree(keys1); cudaFree(hist);
+        cudaFree(chunkcnt); cudaFree(tilebuf);
         *this = Workspace();
     }
 };
@@ -142,16 +141,14 @@ cudaError_t ws_sort(Workspace *w, int64_t cap) {
     cudaError_t e = grow(w->keys0, w->keys0_n, (size_t)cap);
     if (e == cudaSuccess) e = grow(w->keys1, w->keys1_n, (size_t)cap);
     if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256);
-    if (e == cudaSuccess) e = grow(w->dbase, w->dbase_n, 4 * 256);
-    const size_t rt = (size_t)((cap + radix_tile() - 1) / radix_tile() + 3) & ~size_t(3);
-    if (e == cudaSuccess) e = grow(w->tilecnt, w->tilecnt_n, rt * 256);
+    if (e == cudaSuccess) e = grow(w->chunkcnt, w->chunkcnt_n, (size_t)4 * 256 * sort_grid_max());
     const size_t lt = (size_t)((cap + locate_tile() - 1) / locate_tile()) + 1;
     if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, lt * 8);
     return e;
 }
 
-SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32_t gate, double k,
-                   double t) {
+SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32_t gate, int32_t spin_cap,
+                   double k, double t) {
     SortArgs A{};
     A.k = k;
     A.t = t;
@@ -161,11 +158,11 @@ SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32
     A.keys[0] = w->keys0;
     A.keys[1] = w->keys1;
     A.hist = w->hist;
-    A.dbase = w->dbase;
-    A.tilecnt = w->tilecnt;
+    A.chunkcnt = w->chunkcnt;
     A.tilebuf = w->tilebuf;
     A.ctl = w->ctl;
     A.gate = gate;
+    A.spin_cap = spin_cap;
     A.small_cap = rowsolve_capacity();
     return A;
 }
@@ -279,12 +276,11 @@ int check_args(const float *scores, int64_t rows, int64_t n, double k, double t)
 
 // Full sort of one long row on the device (also the certification fallback).
 int full_sort_row(Workspace *w, const float *r, int64_t n, double k, double t, int32_t gate,
-                  cudaStream_t st) {
+                  int32_t spin_cap, cudaStream_t st) {
     LAPSUM_TRY(ws_sort(w, n));
-    SortArgs A = sort_args(w, r, n, n, gate, k, t);
+    SortArgs A = sort_args(w, r, n, n, gate, spin_cap, k, t);
     {
-        Launch L("radix_sort(13 kernels)", st);
-        g_launches += 12;
+        Launch L("radix_sort", st);
         LAPSUM_TRY(launch_radix_sort(A, k, t, st));
     }
     {
@@ -351,7 +347,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         for (int64_t r = 0; r < rows; ++r) {
             const float *row = scores + r * n;
             LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
-            rc = full_sort_row(w, row, n, k, t, GATE_ALWAYS, st);
+            rc = full_sort_row(w, row, n, k, t, GATE_ALWAYS, spin_cap, st);
             if (rc) return rc;
             Launch L("p_pass", st);
             LAPSUM_TRY(launch_p_pass(row, n, t, p_out + r * n, b_out + r, w->ctl, w->partials, st));
@@ -391,16 +387,15 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     { Launch L("stream_pass", st); LAPSUM_TRY(launch_stream_pass(P, st)); }
     { Launch L("band_rowsolve", st); LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st)); }
     if (band_cap > rowsolve_capacity()) {
-        SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, k, t);
+        SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap, k, t);
         {
-            Launch L("band_radix_sort(13 kernels)", st);
-            g_launches += 12;
+            Launch L("band_radix_sort", st);
             LAPSUM_TRY(launch_radix_sort(A, k, t, st));
         }
         { Launch L("band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
     }
     if (!P.fused_cert) { Launch L("certify", st); LAPSUM_TRY(launch_certify(P, st)); }
-    rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, st);
+    rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, st);
     if (rc) return rc;
     { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, st)); }
     return LAPSUM_OK;

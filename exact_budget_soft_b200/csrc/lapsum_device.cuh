@@ -35,6 +35,23 @@ __device__ __forceinline__ float desc_key_to_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? k : (k ^ 0x7fffffffu));
 }
 
+// Band of one tied value: its largest and smallest keys agree (the streaming
+// pass keeps the largest key and the largest complemented key of the band).
+__device__ __forceinline__ bool band_tied(const Ctl *c) {
+    return c->c_band > 0 && (c->band_kmax ^ c->band_kinv) == 0xffffffffu;
+}
+
+// Folds a warp's band keys into those two maxima (all lanes call it; lanes
+// holding no band score pass kmax = 0, kinv = 0).
+__device__ __forceinline__ void band_range_update(Ctl *c, uint32_t kmax, uint32_t kinv) {
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    kinv = __reduce_max_sync(0xffffffffu, kinv);
+    if ((threadIdx.x & 31) == 0 && (kmax | kinv)) {
+        atomicMax(&c->band_kmax, kmax);
+        atomicMax(&c->band_kinv, kinv);
+    }
+}
+
 // ------------------------------------------------------------ exp tiers --
 // e^{-z}, z >= 0.  Terms that can move G by more than ~1e-7 relative to one
 // unit (z <= 16) are formed in fp64; farther terms (< 1.2e-7 each) in fp32,
@@ -186,6 +203,26 @@ __device__ __forceinline__ double solve_interval(double U, double L, double A, d
     return b;
 }
 
+// nn copies of one value c between the seeds of a solve (m0 scores above, the
+// sum P_top of e^{(top-r)/t} over them ending at value top, Q_bot likewise below
+// from bot): the threshold curve is flat across the run,
+//   G(c) = m0 + nn/2 - d_top P_top/2 + d_bot Q_bot/2,
+// and (G decreasing) the root lies in [bot, c] when G(c) <= k, else in [c, top).
+// *above_run: whether the run is above the root (j* = last of the run) or not.
+__device__ __forceinline__ double solve_equal_run_values(double c, double nn, double m0, double top,
+                                                         double P_top, double bot, double Q_bot, double k,
+                                                         double t, bool *above_run) {
+    const double d_top = top == CUDART_INF ? 0.0 : exp((c - top) / t);
+    const double d_bot = bot == -CUDART_INF ? 0.0 : exp((bot - c) / t);
+    const double Gc = m0 + 0.5 * nn - 0.5 * d_top * P_top + 0.5 * d_bot * Q_bot;
+    if (Gc <= k) {
+        *above_run = true;
+        return solve_interval(c, bot, m0 + nn, nn + d_top * P_top, Q_bot, d_bot, k, t);
+    }
+    *above_run = false;
+    return solve_interval(top, c, m0, P_top, nn + d_bot * Q_bot, d_top, k, t);
+}
+
 // Laplace CDF of an fp32 argument, F(x) = e^x/2 (x < 0), 1 - e^{-x}/2 (x >= 0).
 __device__ __forceinline__ float laplace_cdf_f(float x) {
     float e = 0.5f * expf(-fabsf(x));
@@ -267,8 +304,10 @@ __device__ __forceinline__ double exp2_neg(double w, const double *tab) {
 }
 
 // A link of the threshold curve, e^{-(hi - lo)/t} = 2^{-w}, w = (hi - lo) log2(e)/t >= 0
-// (w > 1000 is below 2^{-1000}: zero for every sum it enters).
+// (w > 1000 is below 2^{-1000}: zero for every sum it enters; w = 0, a tie, is
+// exactly 1, which exp2_neg also returns -- the branch only skips the work).
 __device__ __forceinline__ double link_exp(double w, const double *tab) {
+    if (w == 0.0) return 1.0;
     return w <= 1000.0 ? exp2_neg(w, tab) : 0.0;
 }
 
@@ -418,6 +457,43 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 __device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Grid-wide barrier of a cooperative launch (every CTA is resident): an
+// arrival counter and a generation word in device memory; the last CTA to
+// arrive resets the counter and advances the generation.  The wait is bounded:
+// after cap polls the CTA sets ST_TIMEOUT in *status and goes on.
+__device__ __forceinline__ void grid_sync(unsigned *count, unsigned *gen, int cap, int32_t *status) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned g = ld_acquire_u32(gen);   // read before arriving: it cannot advance yet
+        __threadfence();
+        if (atomicAdd(count, 1u) == gridDim.x - 1) {
+            atomicExch(count, 0u);
+            __threadfence();
+            st_release_u32(gen, g + 1u);
+        } else {
+            int it = 0;
+            while (ld_acquire_u32(gen) == g) {
+                if (++it > cap) {
+                    atomicOr(status, ST_TIMEOUT);
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
 // Relaxed (but coherent at GPU scope) 64-bit accesses, for words that carry their
 // own flag and value and guard no other data.
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {

@@ -23,6 +23,8 @@ struct Ctl {
     // streaming pass
     unsigned long long c_L, c_R, c_band;
     double S_L, S_R;
+    unsigned int band_kmax;   // largest descending-order key in the band (every band score,
+    unsigned int band_kinv;   //   past the capacity too) and the largest complemented key
     // certification pass
     double G_aL, G_aR;
     int32_t verdict;          // 1 certified, 0 not (fallback must run), -1 n/a
@@ -37,9 +39,9 @@ struct Ctl {
     unsigned int ticket[8];
     // radix sort: which buffer holds the current keys (-1: the fp32 source)
     int32_t sort_cur;
-    int32_t sort_skip;        // bit d: every key agrees on digit d (pass skipped)
     int32_t sort_solved;      // every key equal: solved without the locate step
-    unsigned int tile_ctr[4];
+    unsigned int gbar_count;  // grid barrier of the cooperative sort: arrivals
+    unsigned int gbar_gen;    //   and generation
     // backward
     double vjp_lambda;
     int32_t vjp_shift;        // every f underflowed: recompute lambda shifted

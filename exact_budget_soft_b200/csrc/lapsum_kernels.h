@@ -25,6 +25,24 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// A cooperative launch (every CTA resident at once, so CTAs may wait on one
+// another at grid barriers); ordinary stream order, no early launch.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // in-CTA full-sort solver (k_rows.cu)
 int rowsolve_capacity();
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
@@ -57,15 +75,16 @@ struct SortArgs {
     int64_t cap;               // upper bound of the element count (grid sizing)
     uint32_t *keys[2];         // ping-pong key buffers [cap]
     unsigned long long *hist;  // [4][256]
-    uint32_t *dbase;           // [4][256]
-    uint32_t *tilecnt;         // [256][stride]: per-tile digit counts, then their offsets
+    uint32_t *chunkcnt;        // [4][256][grid]: digit counts of each CTA's chunk of tiles
     double *tilebuf;           // locate per-tile data
     Ctl *ctl;
     int32_t gate;
+    int32_t spin_cap;          // grid-barrier polls before a wait gives up
     int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
     double k, t;               // budget and temperature (all-equal shortcut)
 };
 int radix_tile();
+int sort_grid_max();
 int locate_tile();
 cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st);
 cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st);
