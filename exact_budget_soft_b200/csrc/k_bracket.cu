@@ -4,6 +4,7 @@
 //
 //   sample_kernel   kernel-noised sample y_j = r_{I_j} + t L_j (Philox4x64-10)
 //   select_kernel   exact order statistics y_(jR), y_(jL) by 3-round radix select
+//                   over a grid (last CTA finishes)
 //   oob_kernel<false>  streaming pass: counts and stable tail sums of the scores
 //                      outside [a_L, a_R), band compaction (warp ballots)
 //   oob_kernel<true>   certification pass: G(a_L), G(a_R) and the verdict
@@ -124,6 +125,7 @@ __device__ __forceinline__ double sample_ln(double x) {
 }
 
 constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
+constexpr int SEL_BINS = 65536;   // select histogram of the top 16 key bits (then 256 of the top 8)
 
 // y_j = r_{I_j} + t L_j: I_j uniform on [0, n) (high word of u0 * n), L_j ~
 // Laplace(0,1) = a random sign times -ln U, U = ((u1 >> 11) + 1) 2^-53 in (0, 1].
@@ -131,22 +133,32 @@ constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
 // is the fp32 value rounded toward -inf (monotone, so order statistics commute
 // with it), in the descending-order key space.
 __global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
+    __shared__ uint32_t s_h0[256];
+    s_h0[threadIdx.x] = 0u;
     pdl_enter();
+    __syncthreads();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= P.s) return;
-    uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
-    philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
-    const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
-    const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
-    const double E = -sample_ln(U);
-    const double L = (x1 & 1ull) ? E : -E;
-    const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
-    const uint32_t key = desc_key(__double2float_rd(y));
-    P.keys[j] = key;
-    // first radix-select round: histogram of the top 16 key bits (warp-aggregated)
-    const uint32_t bin = key >> 16;
-    const unsigned peers = __match_any_sync(__activemask(), bin);
-    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
+    if (j < P.s) {
+        uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
+        philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
+        const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
+        const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
+        const double E = -sample_ln(U);
+        const double L = (x1 & 1ull) ? E : -E;
+        const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
+        const uint32_t key = desc_key(__double2float_rd(y));
+        P.keys[j] = key;
+        // histograms of the top 16 bits (global, warp-aggregated) and top 8 bits
+        const uint32_t bin = key >> 16;
+        const unsigned peers = __match_any_sync(__activemask(), bin);
+        if ((threadIdx.x & 31) == __ffs(peers) - 1) {
+            atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
+            atomicAdd(&s_h0[bin >> 8], (uint32_t)__popc(peers));
+        }
+    }
+    __syncthreads();
+    const uint32_t c = s_h0[threadIdx.x];
+    if (c) atomicAdd(P.hist1 + SEL_BINS + threadIdx.x, c);
 }
 
 // ================================================================ select --
@@ -181,149 +193,112 @@ __device__ __forceinline__ uint32_t block_incl_scan_u32(uint32_t v, uint32_t *s_
     return r;
 }
 
-constexpr int SEL_BINS = 65536;   // first round: top 16 key bits (histogram from the sampler)
-constexpr int SEL_CAND = 8192;    // candidates per target kept in shared memory
-constexpr size_t SEL_SMEM = (2 * SEL_CAND + 2 * 256) * sizeof(uint32_t);
 
-__global__ void __launch_bounds__(1024, 1) select_kernel(BracketParams P) {
-    extern __shared__ __align__(16) unsigned char sel_smem[];
-    uint32_t (*cand)[SEL_CAND] = reinterpret_cast<uint32_t (*)[SEL_CAND]>(sel_smem);
-    uint32_t (*h8)[256] = reinterpret_cast<uint32_t (*)[256]>(sel_smem + 2 * SEL_CAND * sizeof(uint32_t));
-    __shared__ uint32_t s_w[32];
-    __shared__ uint32_t s_pref[2], s_rank[2], s_cnt[2];
+constexpr int SEL_CAND = 8192;   // candidate keys per target kept (global buffer)
+constexpr int SEL_GRID = 64;     // select CTAs
+constexpr int SEL_BLOCK = 256;
+
+// Radix select over a grid: every CTA finds the two targets' 16-bit prefixes
+// from the sampler's histograms (top 8 bits, then the 256 bins of the top-16
+// histogram under the chosen byte), gathers the keys of its share of the sample
+// that carry one of the prefixes into a global candidate buffer, and the last
+// CTA to finish runs rounds 2 and 3 (bits 15..8, 7..0) over the candidates (or
+// over every key when a prefix holds more than the buffer).
+__global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams P) {
+    __shared__ uint32_t s_w[SEL_BLOCK / 32];
+    __shared__ uint32_t h8[2][256];
+    __shared__ uint32_t s_pref[2], s_rank[2], s_bin0[2];
+    __shared__ bool s_last;
     pdl_enter();
     const int tid = threadIdx.x, lane = tid & 31;
-    const int s = (int)P.s;
-    static_assert(SEL_BINS == 32 * 2048, "32 warps x 2048 bins");
+    const int64_t s = P.s;
+    Ctl *ctl = P.ctl;
     const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
-    if (tid == 0) {
-        s_pref[0] = 0; s_pref[1] = 0;
-        s_rank[0] = (uint32_t)(valid[0] ? P.jR : 1);
-        s_rank[1] = (uint32_t)(valid[1] ? P.jL : 1);
-        s_cnt[0] = 0; s_cnt[1] = 0;
-    }
-    __syncthreads();
-    const uint32_t want0[2] = {s_rank[0], s_rank[1]};   // read before any thread updates them
-    // ---- round 1 over the sampler's 16-bit histogram: warp w owns bins
-    //      [2048 w, 2048 w + 2048), read as 16 coalesced rounds of 32 lanes x 4 bins
-    const int warp = tid >> 5;
-    uint4 *hw = reinterpret_cast<uint4 *>(P.hist1) + warp * 512;
-    uint32_t ps[16], rt[16], wtot = 0;
+    const uint32_t want0[2] = {(uint32_t)(valid[0] ? P.jR : 1), (uint32_t)(valid[1] ? P.jL : 1)};
+    if (tid < 2) { s_bin0[tid] = 0u; s_rank[tid] = 1u; s_pref[tid] = 0u; }
+    // ---- round 1a: the top byte of each target (thread t owns bin t)
+    {
+        const uint32_t c = __ldcg(P.hist1 + SEL_BINS + tid);
+        const uint32_t incl = block_incl_scan_u32(c, s_w);
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        const uint4 c = hw[u * 32 + lane];
-        ps[u] = (c.x + c.y) + (c.z + c.w);
-        uint32_t t = ps[u];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
-        rt[u] = t;
-        wtot += t;
+        for (int q = 0; q < 2; ++q)
+            if (incl - c < want0[q] && want0[q] <= incl) {
+                s_bin0[q] = (uint32_t)tid;
+                s_rank[q] = want0[q] - (incl - c);
+            }
+        __syncthreads();
     }
-    if (lane == 0) s_w[warp] = wtot;
-    __syncthreads();
-    uint32_t wbase = 0;
-    for (int w = 0; w < warp; ++w) wbase += s_w[w];
+    // ---- round 1b: the second byte, from the 256 top-16 bins under the first
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-        const uint32_t want = want0[q];
-        if (valid[q] && wbase < want && want <= wbase + wtot) {     // warp-uniform
-            uint32_t cum = wbase, at = wbase, pu = 0;
-            int u = -1;
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {                           // the round holding the target
-                if (u < 0 && cum + rt[v] >= want) { u = v; at = cum; }
-                if (u < 0) cum += rt[v];
-            }
-#pragma unroll
-            for (int v = 0; v < 16; ++v) if (v == u) pu = ps[v];
-            uint32_t inc = pu;                                        // lanes of that round
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t p = __shfl_up_sync(FULL, inc, o);
-                if (lane >= o) inc += p;
-            }
-            const uint32_t lo = at + inc - pu;
-            if (lo < want && want <= at + inc) {
-                const uint4 c = hw[u * 32 + lane];
-                uint32_t cc = lo;
-                int e = 3;
-                if (cc + c.x >= want) e = 0;
-                else if (cc + c.x + c.y >= want) { e = 1; cc += c.x; }
-                else if (cc + c.x + c.y + c.z >= want) { e = 2; cc += c.x + c.y; }
-                else cc += c.x + c.y + c.z;
-                s_pref[q] = (uint32_t)(warp * 2048 + u * 128 + lane * 4 + e) << 16;
-                s_rank[q] = want - cc;
-            }
+        const uint32_t b0 = s_bin0[q], want = s_rank[q];
+        const uint32_t c = __ldcg(P.hist1 + b0 * 256 + tid);
+        const uint32_t incl = block_incl_scan_u32(c, s_w);
+        if (incl - c < want && want <= incl) {
+            s_pref[q] = ((b0 << 8) | (uint32_t)tid) << 16;
+            s_rank[q] = want - (incl - c);
         }
+        __syncthreads();
     }
-#pragma unroll
-    for (int u = 0; u < 16; ++u) hw[u * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);   // rearm (coalesced)
-    __syncthreads();
-    // ---- collect the keys under each target's 16-bit prefix
-    uint32_t mask = 0xffff0000u;
+    // ---- gather this CTA's keys under either prefix
+    const uint32_t pf[2] = {s_pref[0], s_pref[1]};
     {
-        const uint32_t pf[2] = {s_pref[0], s_pref[1]};
         auto take = [&](uint32_t key, bool in) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                const bool m = in && valid[q] && (key & mask) == pf[q];
+                const bool m = in && valid[q] && (key & 0xffff0000u) == pf[q];
                 const unsigned bal = __ballot_sync(FULL, m);
                 if (!bal) continue;
                 uint32_t base = 0;
-                if (lane == __ffs(bal) - 1) base = atomicAdd(&s_cnt[q], (uint32_t)__popc(bal));
+                if (lane == __ffs(bal) - 1) base = atomicAdd(&ctl->sel_cnt[q], (uint32_t)__popc(bal));
                 base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
-                if (m && base < SEL_CAND) cand[q][base] = key;
+                if (m && base < SEL_CAND) P.cand[q * SEL_CAND + base] = key;
             }
         };
         const uint4 *k4 = reinterpret_cast<const uint4 *>(P.keys);
-        const int s4 = s / 4;
-        for (int i0 = 0; i0 < s4; i0 += 4 * 1024) {   // four 16-byte loads in flight per thread
-            uint4 kv[4];
-            bool in[4];
+        const int64_t s4 = s / 4;
+        const int64_t stride = (int64_t)gridDim.x * SEL_BLOCK;
+        for (int64_t i0 = (int64_t)blockIdx.x * SEL_BLOCK; i0 < s4; i0 += stride) {
+            const int64_t i = i0 + tid;
+            const bool in = i < s4;
+            const uint4 kv = in ? k4[i] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+            bool hit = false;   // candidates are rare: one vote for four keys
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * 1024 + tid;
-                in[u] = i < s4;
-                kv[u] = in[u] ? k4[i] : make_uint4(0u, 0u, 0u, 0u);
-            }
-            bool hit = false;   // candidates are rare: one vote for sixteen keys
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t kk[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    hit |= in[u] && (((kk[e] & mask) == pf[0] && valid[0]) || ((kk[e] & mask) == pf[1] && valid[1]));
-            }
+            for (int e = 0; e < 4; ++e)
+                hit |= in && (((kk[e] & 0xffff0000u) == pf[0] && valid[0]) || ((kk[e] & 0xffff0000u) == pf[1] && valid[1]));
             if (!__any_sync(FULL, hit)) continue;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                take(kv[u].x, in[u]);
-                take(kv[u].y, in[u]);
-                take(kv[u].z, in[u]);
-                take(kv[u].w, in[u]);
+            for (int e = 0; e < 4; ++e) take(kk[e], in);
+        }
+        if (blockIdx.x == 0)
+            for (int64_t i0 = 4 * s4; i0 < s; i0 += SEL_BLOCK) {
+                const int64_t i = i0 + tid;
+                take(i < s ? P.keys[i] : 0u, i < s);
             }
-        }
-        for (int i0 = 4 * s4; i0 < s; i0 += 1024) {
-            const int i = i0 + tid;
-            take(i < s ? P.keys[i] : 0u, i < s);
-        }
     }
+    __threadfence();
     __syncthreads();
-    const bool fast[2] = {s_cnt[0] <= SEL_CAND, s_cnt[1] <= SEL_CAND};
-    // ---- rounds 2, 3: bits 15..8, 7..0 over the candidates (or every key when
-    //      a prefix holds more keys than the shared buffer)
+    if (tid == 0) s_last = atomicAdd(&ctl->ticket[5], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // ---- last CTA: rounds 2, 3 over the candidates
+    const uint32_t cnt[2] = {__ldcg(&ctl->sel_cnt[0]), __ldcg(&ctl->sel_cnt[1])};
+    const bool fast[2] = {cnt[0] <= SEL_CAND, cnt[1] <= SEL_CAND};
+    uint32_t mask = 0xffff0000u;
 #pragma unroll 1
     for (int sh = 8; sh >= 0; sh -= 8) {
-        for (int i = tid; i < 2 * 256; i += 1024) (&h8[0][0])[i] = 0u;
+        for (int i = tid; i < 2 * 256; i += SEL_BLOCK) (&h8[0][0])[i] = 0u;
         __syncthreads();
-        const uint32_t pf[2] = {s_pref[0], s_pref[1]};
+        const uint32_t pq[2] = {s_pref[0], s_pref[1]};
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             if (!valid[q]) continue;
-            const int c = fast[q] ? (int)s_cnt[q] : s;
-            for (int i = tid; i < c; i += 1024) {
-                const uint32_t key = fast[q] ? cand[q][i] : P.keys[i];
-                if ((key & mask) == pf[q]) atomicAdd(&h8[q][(key >> sh) & 0xffu], 1u);
+            const int64_t c = fast[q] ? (int64_t)cnt[q] : s;
+            for (int64_t i = tid; i < c; i += SEL_BLOCK) {
+                const uint32_t key = fast[q] ? __ldcg(P.cand + q * SEL_CAND + i) : P.keys[i];
+                if ((key & mask) == pq[q]) atomicAdd(&h8[q][(key >> sh) & 0xffu], 1u);
             }
         }
         __syncthreads();
@@ -356,17 +331,18 @@ __global__ void __launch_bounds__(1024, 1) select_kernel(BracketParams P) {
         mask |= 0xffu << sh;
         __syncthreads();
     }
+    P.hist1[SEL_BINS + tid] = 0u;   // the top-byte histogram; the streaming pass clears the rest
     if (tid == 0) {
-        Ctl *c = P.ctl;
         const float yR = desc_key_to_float(s_pref[0]);
         const float yL = desc_key_to_float(s_pref[1]);
-        c->a_R = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
-        c->a_L = valid[1] ? yL : -CUDART_INF_F;
-        c->jR = P.jR;
-        c->jL = P.jL;
-        c->s = P.s;
-        c->path = 2;
-        c->verdict = -1;
+        ctl->a_R = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
+        ctl->a_L = valid[1] ? yL : -CUDART_INF_F;
+        ctl->jR = P.jR;
+        ctl->jL = P.jL;
+        ctl->s = P.s;
+        ctl->path = 2;
+        ctl->verdict = -1;
+        ctl->ticket[5] = 0u;
     }
 }
 
@@ -613,6 +589,11 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
     pdl_enter();
+    if (!CERT) {   // the select histogram is spent: clear it for the next solve
+        uint4 *h = reinterpret_cast<uint4 *>(P.hist1);
+        for (int64_t i = (int64_t)blockIdx.x * SBLOCK + threadIdx.x; i < SEL_BINS / 4; i += (int64_t)gridDim.x * SBLOCK)
+            h[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     Ctl *ctl = P.ctl;
     Ends E = make_ends(ctl, P.inv_t);
     E.tab = s_tab;
@@ -959,15 +940,9 @@ cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
     return launch_k(sample_kernel, blocks, 256, 0, st, P);
 }
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SEL_SMEM);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    return launch_k(select_kernel, 1, 1024, SEL_SMEM, st, P);
+    return launch_k(select_kernel, SEL_GRID, SEL_BLOCK, 0, st, P);
 }
+int select_cand_capacity() { return SEL_CAND; }
 template <typename K>
 static cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);

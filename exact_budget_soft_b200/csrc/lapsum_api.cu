@@ -101,6 +101,7 @@ struct Workspace {
     double *partials = nullptr;       size_t partials_n = 0;
     uint32_t *skeys = nullptr;        size_t skeys_n = 0;
     uint32_t *hist1 = nullptr;        size_t hist1_n = 0;
+    uint32_t *selcand = nullptr;      size_t selcand_n = 0;
     float *band = nullptr;            size_t band_n = 0;
     uint32_t *keys0 = nullptr;        size_t keys0_n = 0;
     uint32_t *keys1 = nullptr;        size_t keys1_n = 0;
@@ -109,7 +110,7 @@ struct Workspace {
     double *tilebuf = nullptr;        size_t tilebuf_n = 0;
 
     void release() {
-        cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(hist1); cudaFree(band);
+        cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(hist1); cudaFree(selcand); cudaFree(band);
         cudaFree(keys0); cudaFree(keys1); cudaFree(hist);
         cudaFree(chunkcnt); cudaFree(tilebuf);
         *this = Workspace();
@@ -372,12 +373,14 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     P.spin_cap = spin_cap;
     P.fused_cert = opt.certify == LAPSUM_CERTIFY_FUSED;
     LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
-    LAPSUM_TRY(grow(w->hist1, w->hist1_n, 65536));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, 65536 + 256));
+    LAPSUM_TRY(grow(w->selcand, w->selcand_n, (size_t)2 * select_cand_capacity()));
     LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_cap));
     LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort the whole row
     P.band = w->band;
     P.keys = w->skeys;
     P.hist1 = w->hist1;
+    P.cand = w->selcand;
     P.partials = w->partials;
     P.ctl = w->ctl;
 

@@ -38,6 +38,7 @@ struct Ctl {
     // single-pass "last block" tickets (zeroed with the block)
     unsigned int ticket[8];
     // radix sort: which buffer holds the current keys (-1: the fp32 source)
+    unsigned int sel_cnt[2];  // select: keys under each target's 16-bit prefix
     int32_t sort_cur;
     int32_t sort_solved;      // every key equal: solved without the locate step
     unsigned int gbar_count;  // grid barrier of the cooperative sort: arrivals
@@ -59,7 +60,9 @@ struct BracketParams {
     int64_t band_cap;
     float *band;              // band buffer [band_cap]
     uint32_t *keys;           // sample keys [s]
-    uint32_t *hist1;          // [65536] first-round select histogram (kept zeroed)
+    uint32_t *hist1;          // [65536 + 256] select histograms of the top 16 and top 8 key
+                              //   bits (zero between solves: the streaming pass clears them)
+    uint32_t *cand;           // [2][SEL_CAND] keys under each target's 16-bit prefix
     double *partials;         // per-block partials
     Ctl *ctl;
     int32_t spin_cap;

@@ -56,6 +56,7 @@ cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, 
 int stream_grid();
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st);
+int select_cand_capacity();
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,

@@ -162,6 +162,20 @@ def test_pixels1m_workload(L, orc):
 
 
 @pytest.mark.parametrize("certify", [0, 1])
+def test_bracketing_large_band_device_sort(L, orc, certify):
+    # a small sample leaves a wide bracket: the band (~1e5 scores, untied) is
+    # too long for one CTA and goes through the device-wide sort and locate
+    n = (1 << 21) + 12345
+    r, g = W.small_case("laplace", 1, n, seed=12)
+    k, t, s = n / 10.0, 0.05, 4096
+    p, b, st, grad = run(L, r, k, t, opts=L.options(sample_size=s, certify=certify), g_np=g)
+    assert st["rc"] == 0 and st["path"] == 2 and st["verdict"] == 1 and st["fallback"] == 0
+    assert st["c_band"] > 32768
+    check_bracket_integers(orc, r[0], k, t, st, 0, s, 1e-6)
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+@pytest.mark.parametrize("certify", [0, 1])
 def test_forced_fallback_by_band_capacity(L, orc, certify):
     r, g = W.small_case("normal", 1, 1 << 20, seed=5)
     k, t = 3000.0, 0.05
