@@ -750,7 +750,10 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
 
 // =================================================================== VJP --
 // <g,f> and sum f of one long row (walking backward: the p pass left the tail
-// in L2).  Terms are e^{-|x|} in fp32 (denormals kept), summed in fp64.  If
+// in L2).  Terms are e^{-|x|} in fp32 (denormals kept); each thread sums the
+// terms of one chunk (eight scores: positive terms, and g e products whose
+// fp32 rounding is ~1e-7 of their magnitudes) in fp32 and adds that partial to
+// fp64 accumulators, so the fp64 pipe sees two adds per eight scores.  If
 // every term underflows (all scores farther than ~100 t from b), the last block
 // raises a flag and vjp_shifted_kernel recomputes the ratio from terms shifted
 // by the running minimum of |x| (the shift cancels in <g,f>/sum f).
@@ -769,24 +772,32 @@ vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
     const float4 *r4 = reinterpret_cast<const float4 *>(r);
     const float4 *g4 = reinterpret_cast<const float4 *>(g);
     double sf = 0.0, sgf = 0.0;
-    auto acc4 = [&](const float4 v, const float4 w) {
+    auto part4 = [&](const float4 v, const float4 w, float &f32, float &gf32) {
         const float e0 = exp2f(-fabsf(xf(v.x))), e1 = exp2f(-fabsf(xf(v.y)));
         const float e2 = exp2f(-fabsf(xf(v.z))), e3 = exp2f(-fabsf(xf(v.w)));
-        sf += ((double)e0 + (double)e1) + ((double)e2 + (double)e3);
-        sgf = fma((double)w.x, (double)e0, sgf);
-        sgf = fma((double)w.y, (double)e1, sgf);
-        sgf = fma((double)w.z, (double)e2, sgf);
-        sgf = fma((double)w.w, (double)e3, sgf);
+        f32 += (e0 + e1) + (e2 + e3);
+        gf32 = fmaf(w.x, e0, gf32);
+        gf32 = fmaf(w.y, e1, gf32);
+        gf32 = fmaf(w.z, e2, gf32);
+        gf32 = fmaf(w.w, e3, gf32);
     };
     int64_t done4 = 0;
     if (aligned) {
         const float4 *src[2] = {r4, g4};
         done4 = bulk_stream<2>(src, n4, true, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
-            acc4(lds128(ch[0] + threadIdx.x), lds128(ch[1] + threadIdx.x));
-            acc4(lds128(ch[0] + threadIdx.x + SBLOCK), lds128(ch[1] + threadIdx.x + SBLOCK));
+            float f32 = 0.f, gf32 = 0.f;
+            part4(lds128(ch[0] + threadIdx.x), lds128(ch[1] + threadIdx.x), f32, gf32);
+            part4(lds128(ch[0] + threadIdx.x + SBLOCK), lds128(ch[1] + threadIdx.x + SBLOCK), f32, gf32);
+            sf += (double)f32;
+            sgf += (double)gf32;
         });
     }
-    for (int64_t i = done4 + gtid; i < n4; i += gstride) acc4(r4[i], g4[i]);
+    for (int64_t i = done4 + gtid; i < n4; i += gstride) {
+        float f32 = 0.f, gf32 = 0.f;
+        part4(r4[i], g4[i], f32, gf32);
+        sf += (double)f32;
+        sgf += (double)gf32;
+    }
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
         const float e = exp2f(-fabsf(xf(r[i])));
         sf += (double)e;
