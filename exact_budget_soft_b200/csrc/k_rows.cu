@@ -27,7 +27,8 @@ namespace lapsum {
 template <int BLOCK, int KPT, bool BAND>
 __global__ void __launch_bounds__(BLOCK, 1)
 rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, double t, double inv_t,
-                float *__restrict__ p_out, double *__restrict__ b_out, Ctl *ctl, int64_t band_cap) {
+                float *__restrict__ p_out, double *__restrict__ b_out, Ctl *ctl, int64_t band_cap,
+                int64_t band_lo) {
     using C = RowCfg<BLOCK, KPT>;
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);
@@ -49,8 +50,8 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
             if (tid == 0) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
             return;
         }
-        if (band_tied(ctl)) {   // one tied value, of any count: closed form
-            if (tid == 0) {
+        if (band_tied(ctl)) {   // one tied value, of any count: closed form (first variant)
+            if (band_lo == 0 && tid == 0) {
                 bool above = false;
                 ctl->b = solve_equal_run_values((double)desc_key_to_float(ctl->band_kmax), (double)cb,
                                                 (double)ctl->c_R, (double)ctl->a_R, ctl->S_R, (double)ctl->a_L,
@@ -59,6 +60,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
             }
             return;
         }
+        if (band_lo > 0 && cb <= (unsigned long long)band_lo) return;   // a smaller variant takes it
         if (cb > (unsigned long long)C::CAP) return;   // the device-wide sort takes it
         n = (int)cb;
         row = scores;
@@ -113,7 +115,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     if (__syncthreads_or(bad) && tid == 0 && ctl) atomicOr(&ctl->status, ST_NONFINITE);
     const uint32_t diff = s_and ^ s_or;
 
-    block_radix_sort<BLOCK, KPT>(key, s_keys, s_hist, s_dbase, diff);
+    block_radix_sort<BLOCK, KPT, BAND>(key, s_keys, s_hist, s_dbase, diff);
 
     int64_t jstar = 0;
     int32_t *st = ctl ? &ctl->status : nullptr;
@@ -266,7 +268,7 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
 // ------------------------------------------------------------ launchers --
 template <int BLOCK, int KPT, bool BAND>
 static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n, double k, double t,
-                                   float *p, double *b, Ctl *ctl, int64_t band_cap,
+                                   float *p, double *b, Ctl *ctl, int64_t band_cap, int64_t band_lo,
                                    cudaStream_t st) {
     using C = RowCfg<BLOCK, KPT>;
     auto kern = rowsolve_kernel<BLOCK, KPT, BAND>;
@@ -277,7 +279,8 @@ static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n,
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl, band_cap);
+    return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl, band_cap,
+                    band_lo);
 }
 
 int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
@@ -285,13 +288,19 @@ int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st) {
     if (n <= RowCfg<256, 16>::CAP)
-        return launch_rowsolve<256, 16, false>(scores, rows, n, k, t, p, b, ctl, 0, st);
-    return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, st);
+        return launch_rowsolve<256, 16, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, st);
+    return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, st);
 }
 
+// Two variants, each gated on the band size the streaming pass counted: bands
+// of up to 4096 scores (and tied or empty bands) in a 256-thread CTA, larger
+// ones up to 32768 in a 1024-thread CTA.
 cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
                                  cudaStream_t st) {
-    return launch_rowsolve<1024, 32, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap, st);
+    cudaError_t e = launch_rowsolve<256, 16, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, st);
+    if (e != cudaSuccess) return e;
+    return launch_rowsolve<1024, 32, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap,
+                                           RowCfg<256, 16>::CAP, st);
 }
 
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,

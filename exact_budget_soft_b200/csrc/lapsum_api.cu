@@ -388,7 +388,11 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     { Launch L("sample", st); LAPSUM_TRY(launch_sample(P, st)); }
     { Launch L("select", st); LAPSUM_TRY(launch_select(P, st)); }
     { Launch L("stream_pass", st); LAPSUM_TRY(launch_stream_pass(P, st)); }
-    { Launch L("band_rowsolve", st); LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st)); }
+    {
+        Launch L("band_rowsolve", st);
+        ++g_launches;   // two size-gated variants
+        LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st));
+    }
     if (band_cap > rowsolve_capacity()) {
         SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap, k, t);
         {

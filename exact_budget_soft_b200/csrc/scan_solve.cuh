@@ -15,7 +15,11 @@ namespace lapsum {
 __device__ __forceinline__ int spad(int j) { return j + (j >> 5); }
 
 // Lanes of the warp holding the same 8-bit digit: eight ballots, one per bit.
+// UNIFORM: first one vote for a warp that agrees throughout (padding, sorted or
+// tied keys: the mostly-padded band) -- a loss on full rows of random keys.
+template <bool UNIFORM>
 __device__ __forceinline__ unsigned digit_peers(uint32_t d) {
+    if (UNIFORM && __all_sync(FULL, d == __shfl_sync(FULL, d, 0))) return FULL;
     unsigned peers = FULL;
 #pragma unroll
     for (int b = 0; b < 8; ++b) {
@@ -37,7 +41,7 @@ struct RowCfg {
 
 // Block-wide LSD radix sort of warp-striped register keys (ascending).  On
 // return the sorted keys are in s_keys (position j at spad(j)).
-template <int BLOCK, int KPT>
+template <int BLOCK, int KPT, bool UNIFORM = false>
 __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t *s_keys,
                                                  uint32_t *s_hist, uint32_t *s_dbase,
                                                  uint32_t diff) {
@@ -55,7 +59,7 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
             const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = digit_peers(d);
+            const unsigned peers = digit_peers<UNIFORM>(d);
             if (lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
             __syncwarp();
         }
@@ -91,7 +95,7 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
             const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = digit_peers(d);
+            const unsigned peers = digit_peers<UNIFORM>(d);
             const int leader = __ffs(peers) - 1;
             uint32_t base = 0;
             if (lane == leader) {
