@@ -400,6 +400,7 @@ __device__ __forceinline__ void tier2(float hi, float lo, double dhi, double dlo
 
 struct OobAcc {
     uint32_t cL, cR, cB;        // stream: below, above; certify: >= a_L, >= a_R, < a_L
+    uint32_t kmax, kinv;        // stream: largest band key and largest complemented band key
     double SL, SR, hL, lR;      // near terms: below, above, band vs a_L, band vs a_R
     float SL2, SR2, hL2, lR2;   // far terms
     bool bad;
@@ -408,10 +409,13 @@ struct OobAcc {
 // Append a band score at a warp-aggregated slot of the band buffer (the count
 // keeps going past the capacity so the overflow is visible).
 __device__ __forceinline__ void band_push(float x, bool inb, float *band, unsigned long long cap,
-                                          unsigned long long *ctr, int lane, Ctl *ctl) {
+                                          unsigned long long *ctr, int lane, OobAcc &a) {
     const unsigned m = __ballot_sync(FULL, inb);
     if (!m) return;
-    band_range_update(ctl, inb ? desc_key(x) : 0u, inb ? ~desc_key(x) : 0u);
+    if (inb) {
+        a.kmax = max(a.kmax, desc_key(x));
+        a.kinv = max(a.kinv, ~desc_key(x));
+    }
     const int leader = __ffs(m) - 1;
     unsigned long long base = 0;
     if (lane == leader) base = atomicAdd(ctr, (unsigned long long)__popc(m));
@@ -478,7 +482,7 @@ __device__ __forceinline__ void tier4(const float4 v, bool equal, float af, doub
 // slots: one warp scan and one atomic per warp (the count keeps going past the
 // capacity so the overflow is visible).
 __device__ __forceinline__ void band_push4(const float4 v, int m, float *band, unsigned long long cap,
-                                           unsigned long long *ctr, int lane, Ctl *ctl) {
+                                           unsigned long long *ctr, int lane, OobAcc &a) {
     const int cnt = __popc(m);
     int inc = cnt;
 #pragma unroll
@@ -489,16 +493,14 @@ __device__ __forceinline__ void band_push4(const float4 v, int m, float *band, u
     const int total = __shfl_sync(FULL, inc, 31);
     if (total == 0) return;
     {
-        uint32_t kmax = 0u, kinv = 0u;
         const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             if (m & (1 << i)) {
                 const uint32_t kk = desc_key(vv[i]);
-                kmax = max(kmax, kk);
-                kinv = max(kinv, ~kk);
+                a.kmax = max(a.kmax, kk);
+                a.kinv = max(a.kinv, ~kk);
             }
-        band_range_update(ctl, kmax, kinv);
     }
     unsigned long long base = 0;
     if (lane == 31) base = atomicAdd(ctr, (unsigned long long)total);
@@ -557,7 +559,7 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
             tier4<true>(v, equal, E.aL, E.daL, E, a.hL, a.hL2);
             tier4<false>(v, equal, E.aR, E.daR, E, a.lR, a.lR2);
         }
-        if (!CERT) band_push4(v, ok ? 0xF : 0, P.band, cap, &P.ctl->c_band, lane, P.ctl);
+        if (!CERT) band_push4(v, ok ? 0xF : 0, P.band, cap, &P.ctl->c_band, lane, a);
         return;
     }
     const bool b0 = oob_one<MODE>(v.x, ok, E, a);
@@ -566,7 +568,7 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
     const bool b3 = oob_one<MODE>(v.w, ok, E, a);
     if (!CERT) {
         const int m = (b0 ? 1 : 0) | (b1 ? 2 : 0) | (b2 ? 4 : 0) | (b3 ? 8 : 0);
-        if (__any_sync(FULL, m != 0)) band_push4(v, m, P.band, cap, &P.ctl->c_band, lane, P.ctl);
+        if (__any_sync(FULL, m != 0)) band_push4(v, m, P.band, cap, &P.ctl->c_band, lane, a);
     }
 }
 
@@ -600,7 +602,7 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const unsigned long long cap = (unsigned long long)P.band_cap;
-    OobAcc acc{0, 0, 0, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
+    OobAcc acc{0, 0, 0, 0u, 0u, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
     const int64_t n = P.n;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
@@ -629,9 +631,13 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
         const bool ok = j < n;
         const float x = ok ? P.r[j] : 0.f;
         const bool bb = oob_one<MODE>(x, ok, E, acc);
-        if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane, ctl);
+        if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane, acc);
     }
     if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
+    if (!CERT) {
+        __shared__ uint32_t s_two[2];
+        band_range_flush(ctl, acc.kmax, acc.kinv, s_two);
+    }
     if constexpr (MODE == OOB_STREAM) {
         double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2};
         block_sum<SBLOCK, 4>(v, s_red);

@@ -23,8 +23,11 @@
 namespace lapsum {
 
 constexpr int RB = 512;             // radix pass: threads
-constexpr int RK = 16;              // keys per thread
-constexpr int RTILE = RB * RK;      // 8192 keys per tile
+// keys per thread K: 16 (8192-key tiles) for long rows, 4 (2048-key tiles, more
+// CTAs in parallel) when the sort holds at most SMALL_SORT keys
+#define TILE_K(K) (RB * (K))
+constexpr int RK_BIG = 16, RK_SMALL = 4;
+constexpr int64_t SMALL_SORT = int64_t(1) << 20;
 constexpr int RNW = RB / 32;
 constexpr int HB = 256;             // histogram kernel threads
 
@@ -33,7 +36,7 @@ constexpr int LK = 16;              // values per thread
 constexpr int LTILE = LB * LK;      // 16384 values per tile
 constexpr int LOC_KEY_WORDS = LTILE + LTILE / 32 + 8;   // padded tile + two halo entries
 
-int radix_tile() { return RTILE; }
+int radix_tile() { return TILE_K(RK_BIG); }
 int locate_tile() { return LTILE; }
 
 // Element count behind a gate; < 0 means "nothing to do".
@@ -93,83 +96,91 @@ __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
 // read through L2 (ld.global.cg or bulk copies), never through L1.
 
 // The tile's keys, warp-striped (key i of lane l of warp w is tile element
-// w*32*RK + i*32 + l), all RK loads in flight at once; keys past the end of the
+// w*32*K + i*32 + l), all K loads in flight at once; keys past the end of the
 // row read as 0xffffffff.  src == nullptr: the first pass, keys from the scores.
+template <int K>
 __device__ __forceinline__ void load_tile(const SortArgs &A, const uint32_t *src, int64_t base, int cnt_tile,
-                                          uint32_t (&key)[RK]) {
+                                          uint32_t (&key)[K]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int l0 = warp * 32 * RK + lane;
+    const int l0 = warp * 32 * K + lane;
     if (src) {
 #pragma unroll
-        for (int i = 0; i < RK; ++i)
+        for (int i = 0; i < K; ++i)
             key[i] = l0 + i * 32 < cnt_tile ? __ldcg(src + base + l0 + i * 32) : 0xffffffffu;
     } else {
-        float x[RK];
+        float x[K];
 #pragma unroll
-        for (int i = 0; i < RK; ++i) x[i] = l0 + i * 32 < cnt_tile ? __ldg(A.src + base + l0 + i * 32) : 0.0f;
+        for (int i = 0; i < K; ++i) x[i] = l0 + i * 32 < cnt_tile ? __ldg(A.src + base + l0 + i * 32) : 0.0f;
 #pragma unroll
-        for (int i = 0; i < RK; ++i) key[i] = l0 + i * 32 < cnt_tile ? desc_key(x[i]) : 0xffffffffu;
+        for (int i = 0; i < K; ++i) key[i] = l0 + i * 32 < cnt_tile ? desc_key(x[i]) : 0xffffffffu;
     }
 }
 
 // Double-buffered tile staging: only full tiles of a 16-byte-aligned source
 // are copied (one bulk copy each, completion counted on an mbarrier); the
 // ragged last tile takes plain loads.
+template <int K>
 struct TileStage {
-    uint32_t *buf;      // 2 * RTILE words
+    uint32_t *buf;      // 2 * TILE_K(K) words
     uint64_t *bar;      // 2 mbarriers
     const char *gsrc;   // 4-byte elements: the keys, or the scores
     bool bulk_ok;
     int64_t n;
 };
 
-__device__ __forceinline__ bool stage_full(const TileStage &S, int64_t tile) {
-    return S.bulk_ok && (tile + 1) * RTILE <= S.n;
+template <int K>
+__device__ __forceinline__ bool stage_full(const TileStage<K> &S, int64_t tile) {
+    return S.bulk_ok && (tile + 1) * TILE_K(K) <= S.n;
 }
 
 // thread 0; the buffer must be free (its last readers are past a barrier)
-__device__ __forceinline__ void stage_issue(const TileStage &S, int slot, int64_t tile) {
+template <int K>
+__device__ __forceinline__ void stage_issue(const TileStage<K> &S, int slot, int64_t tile) {
     if (!stage_full(S, tile)) return;
     fence_proxy_async_smem();
-    mbar_expect_tx(&S.bar[slot], RTILE * 4);
-    bulk_load(S.buf + slot * RTILE, S.gsrc + (size_t)tile * RTILE * 4, RTILE * 4, &S.bar[slot]);
+    mbar_expect_tx(&S.bar[slot], TILE_K(K) * 4);
+    bulk_load(S.buf + slot * TILE_K(K), S.gsrc + (size_t)tile * TILE_K(K) * 4, TILE_K(K) * 4, &S.bar[slot]);
 }
 
-__device__ __forceinline__ void stage_source(TileStage &S, const SortArgs &A, const uint32_t *src) {
+template <int K>
+__device__ __forceinline__ void stage_source(TileStage<K> &S, const SortArgs &A, const uint32_t *src) {
     S.gsrc = src ? reinterpret_cast<const char *>(src) : reinterpret_cast<const char *>(A.src);
     S.bulk_ok = (reinterpret_cast<uintptr_t>(S.gsrc) & 15u) == 0;
 }
 
 // The tile's keys into registers: from its staged copy (waiting, bounded, for
 // the copy) or by plain loads.  Returns false when the wait gave up.
-__device__ __forceinline__ bool stage_keys(const TileStage &S, const SortArgs &A, const uint32_t *src, int slot,
-                                           uint32_t &ph, int64_t tile, int cnt_tile, uint32_t (&key)[RK]) {
+template <int K>
+__device__ __forceinline__ bool stage_keys(const TileStage<K> &S, const SortArgs &A, const uint32_t *src, int slot,
+                                           uint32_t &ph, int64_t tile, int cnt_tile, uint32_t (&key)[K]) {
     if (!stage_full(S, tile)) {
-        load_tile(A, src, tile * RTILE, cnt_tile, key);
+        load_tile(A, src, tile * TILE_K(K), cnt_tile, key);
         return true;
     }
     const bool ok = mbar_wait(&S.bar[slot], (ph >> slot) & 1u, BULK_WAIT_CAP);
     ph ^= 1u << slot;
-    const uint32_t *sb = S.buf + slot * RTILE;
-    const int l0 = (threadIdx.x >> 5) * 32 * RK + (threadIdx.x & 31);
+    const uint32_t *sb = S.buf + slot * TILE_K(K);
+    const int l0 = (threadIdx.x >> 5) * 32 * K + (threadIdx.x & 31);
     if (src) {
 #pragma unroll
-        for (int i = 0; i < RK; ++i) key[i] = sb[l0 + i * 32];
+        for (int i = 0; i < K; ++i) key[i] = sb[l0 + i * 32];
     } else {
 #pragma unroll
-        for (int i = 0; i < RK; ++i) key[i] = desc_key(__uint_as_float(sb[l0 + i * 32]));
+        for (int i = 0; i < K; ++i) key[i] = desc_key(__uint_as_float(sb[l0 + i * 32]));
     }
     return ok;
 }
 
-constexpr size_t STAGE_BYTES = 2 * RTILE * 4 + 2 * sizeof(uint64_t);
+template <int K>
+constexpr size_t stage_bytes() { return 2 * TILE_K(K) * 4 + 2 * sizeof(uint64_t); }
 
 // Adds this warp's digit counts of the tile to my_hist (the warp's 256 counters).
-__device__ __forceinline__ void warp_count(const uint32_t (&key)[RK], int cnt_tile, int sh, uint32_t *my_hist) {
+template <int K>
+__device__ __forceinline__ void warp_count(const uint32_t (&key)[K], int cnt_tile, int sh, uint32_t *my_hist) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int i = 0; i < RK; ++i) {
-        const int li = warp * 32 * RK + i * 32 + lane;
+    for (int i = 0; i < K; ++i) {
+        const int li = warp * 32 * K + i * 32 + lane;
         const bool v = li < cnt_tile;
         const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
         const unsigned peers = __match_any_sync(FULL, d);
@@ -181,8 +192,8 @@ __device__ __forceinline__ void warp_count(const uint32_t (&key)[RK], int cnt_ti
 // Walks the CTA's chunk of tiles in order with one tile staged ahead, calling
 // body(tile, cnt_tile, key) with every thread's keys; a barrier follows each
 // body, so the staging buffers are free again.  Returns false if a wait gave up.
-template <typename Body>
-__device__ __forceinline__ bool walk_chunk(TileStage &S, const SortArgs &A, const uint32_t *src, int64_t t0,
+template <int K, typename Body>
+__device__ __forceinline__ bool walk_chunk(TileStage<K> &S, const SortArgs &A, const uint32_t *src, int64_t t0,
                                            int64_t t1, uint32_t &ph, Body &&body) {
     bool ok = true;
     stage_source(S, A, src);
@@ -190,21 +201,23 @@ __device__ __forceinline__ bool walk_chunk(TileStage &S, const SortArgs &A, cons
     int slot = 0;
     for (int64_t tile = t0; tile < t1; ++tile, slot ^= 1) {
         if (threadIdx.x == 0 && tile + 1 < t1) stage_issue(S, slot ^ 1, tile + 1);
-        const int cnt_tile = (int)min((int64_t)RTILE, S.n - tile * RTILE);
-        uint32_t key[RK];
+        const int cnt_tile = (int)min((int64_t)TILE_K(K), S.n - tile * TILE_K(K));
+        uint32_t key[K];
         ok &= stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
-        body(tile, cnt_tile, key, S.buf + slot * RTILE);
+        body(tile, cnt_tile, key, S.buf + slot * TILE_K(K));
         __syncthreads();
     }
     return ok;
 }
 
-constexpr size_t SORT_SMEM = STAGE_BYTES + (size_t)(RNW * 256 + 4 * 256 + 4 * 256) * 4;
+template <int K>
+constexpr size_t sort_smem() { return stage_bytes<K>() + (size_t)(RNW * 256 + 4 * 256 + 4 * 256) * 4; }
 constexpr int SORT_GMAX = 320;   // CTAs of the sort grid at most (chunk counts per digit)
 
+template <int K>
 __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
     extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + STAGE_BYTES);   // RNW * 256: per-warp digit counts
+    uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + stage_bytes<K>());   // RNW * 256: per-warp digit counts
     uint32_t *s_dstart = s_hist + RNW * 256;   // 256: in-tile digit start
     uint32_t *s_gofs = s_dstart + 256;         // 256: global offset - in-tile start
     uint32_t *s_run = s_gofs + 256;            // 256: running global offset of each digit
@@ -217,13 +230,13 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
     Ctl *ctl = A.ctl;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x, c = blockIdx.x;
-    const int64_t ntiles = (n + RTILE - 1) / RTILE;
+    const int64_t ntiles = (n + TILE_K(K) - 1) / TILE_K(K);
     const int64_t t0 = (int64_t)c * ntiles / G, t1 = (int64_t)(c + 1) * ntiles / G;
     uint32_t *csum = A.chunkcnt;   // [4][256][G]
     auto bar = [&]() { grid_sync(&ctl->gbar_count, &ctl->gbar_gen, A.spin_cap, &ctl->status); };
-    TileStage S;
+    TileStage<K> S;
     S.buf = reinterpret_cast<uint32_t *>(smem);
-    S.bar = reinterpret_cast<uint64_t *>(smem + 2 * RTILE * 4);
+    S.bar = reinterpret_cast<uint64_t *>(smem + 2 * TILE_K(K) * 4);
     S.n = n;
     if (tid == 0) {
         mbar_init(&S.bar[0], 1);
@@ -239,10 +252,10 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
     {
         uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         uint32_t cnt[4] = {0, 0, 0, 0};
-        ok &= walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[RK], uint32_t *) {
-            const int l0 = warp * 32 * RK + lane;
+        ok &= walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
+            const int l0 = warp * 32 * K + lane;
 #pragma unroll
-            for (int i = 0; i < RK; ++i) {
+            for (int i = 0; i < K; ++i) {
                 if (l0 + i * 32 >= cnt_tile) break;
 #pragma unroll
                 for (int d = 0; d < 4; ++d) {
@@ -305,7 +318,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
             if (!first) {   // the chunk's digit counts in the current order
                 for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
                 __syncthreads();
-                ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[RK], uint32_t *) {
+                ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
                     warp_count(key, cnt_tile, sh, s_hist + warp * 256);
                 });
                 if (tid < 256) {
@@ -337,7 +350,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
                 }
             }
             __syncthreads();
-            ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[RK], uint32_t *s_keys) {
+            ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *s_keys) {
                 for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
                 __syncthreads();   // every key is in registers: s_keys is free too
                 uint32_t *my_hist = s_hist + warp * 256;
@@ -377,8 +390,8 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
                 // scatter into shared memory by (digit, warp, traversal order): stable
                 const unsigned lt_mask = (1u << lane) - 1u;
 #pragma unroll
-                for (int i = 0; i < RK; ++i) {
-                    const int li = warp * 32 * RK + i * 32 + lane;
+                for (int i = 0; i < K; ++i) {
+                    const int li = warp * 32 * K + i * 32 + lane;
                     const bool v = li < cnt_tile;
                     const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
                     const unsigned peers = __match_any_sync(FULL, d);
@@ -617,25 +630,33 @@ static int num_sms() {
 
 int sort_grid_max() { return SORT_GMAX; }
 
-cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) {
-    (void)k;
-    (void)t;
-    static int resident = 0;   // CTAs of the sort kernel that fit the device at once
+template <int K>
+static cudaError_t launch_sort_k(SortArgs &A, cudaStream_t st) {
+    static int resident = 0;   // CTAs of this sort kernel that fit the device at once
     if (!resident) {
-        cudaError_t e = cudaFuncSetAttribute(radix_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SORT_SMEM);
+        cudaError_t e = cudaFuncSetAttribute(radix_sort_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)sort_smem<K>());
         if (e != cudaSuccess) return e;
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, radix_sort_kernel, RB, SORT_SMEM);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, radix_sort_kernel<K>, RB, sort_smem<K>());
         if (e != cudaSuccess) return e;
         if (per_sm < 1) return cudaErrorInvalidConfiguration;
         resident = per_sm * num_sms();
     }
-    int64_t g = (A.cap + RTILE - 1) / RTILE;
+    int64_t g = (A.cap + TILE_K(K) - 1) / TILE_K(K);
     if (g > resident) g = resident;
     if (g > SORT_GMAX) g = SORT_GMAX;
     if (g < 1) g = 1;
-    return launch_coop(radix_sort_kernel, (unsigned)g, RB, SORT_SMEM, st, A);
+    return launch_coop(radix_sort_kernel<K>, (unsigned)g, RB, sort_smem<K>(), st, A);
+}
+
+// The tile size follows the capacity of the sort (the host does not know the
+// band's size): small sorts take small tiles, so more CTAs share the work.
+cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) {
+    (void)k;
+    (void)t;
+    if (A.cap <= SMALL_SORT) return launch_sort_k<RK_SMALL>(A, st);
+    return launch_sort_k<RK_BIG>(A, st);
 }
 
 cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st) {

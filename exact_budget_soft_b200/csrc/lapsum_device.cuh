@@ -41,14 +41,21 @@ __device__ __forceinline__ bool band_tied(const Ctl *c) {
     return c->c_band > 0 && (c->band_kmax ^ c->band_kinv) == 0xffffffffu;
 }
 
-// Folds a warp's band keys into those two maxima (all lanes call it; lanes
-// holding no band score pass kmax = 0, kinv = 0).
-__device__ __forceinline__ void band_range_update(Ctl *c, uint32_t kmax, uint32_t kinv) {
+// Folds a CTA's band-key maxima (per thread; 0 for none) into those two words:
+// one shared and one global atomic per CTA.  Every thread of the CTA calls it.
+__device__ __forceinline__ void band_range_flush(Ctl *c, uint32_t kmax, uint32_t kinv, uint32_t *s_two) {
+    if (threadIdx.x == 0) { s_two[0] = 0u; s_two[1] = 0u; }
+    __syncthreads();
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     kinv = __reduce_max_sync(0xffffffffu, kinv);
     if ((threadIdx.x & 31) == 0 && (kmax | kinv)) {
-        atomicMax(&c->band_kmax, kmax);
-        atomicMax(&c->band_kinv, kinv);
+        atomicMax(&s_two[0], kmax);
+        atomicMax(&s_two[1], kinv);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && (s_two[0] | s_two[1])) {
+        atomicMax(&c->band_kmax, s_two[0]);
+        atomicMax(&c->band_kinv, s_two[1]);
     }
 }
 

@@ -105,7 +105,7 @@ def test_all_equal_and_ties(L, orc):
 
 # ----------------------------------------------- device-wide full sort --
 @pytest.mark.parametrize("n,dist", [(32769, "normal"), (100_000, "laplace"), (300_001, "normal"),
-                                    (500_000, "levels256_desc")])
+                                    (500_000, "levels256_desc"), (1_100_003, "normal")])
 def test_device_sort_path(L, orc, n, dist):
     r, g = W.small_case(dist, 1, n, seed=7)
     k, t = n / 100.0, 0.05
