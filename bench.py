@@ -302,6 +302,21 @@ def run_ours(args):
             out["forced_fallback"] = {"median_ms_fwd_vjp": round(statistics.median(msf), 4),
                                       "note": "certification fails (seed from tests/golden); the row is "
                                               "fully sorted on the device"}
+            # the same missed bracket with one widening round before the fallback
+            ow = L.options(seed=gold["seed"], sample_size=gold["sample_size"], delta=gold["delta"], widen=1)
+
+            def st_w():
+                L.forward(r, w.k, w.t, p_out=p, b_out=b, opts=ow)
+                L.backward(r, b, g, w.t, grad_out=grad)
+
+            msw = time_steps(torch, st_w, max(5, args.steps // 4), 2)
+            sw = L.get_stats()
+            assert sw["rc"] == 0 and sw["widened"] == 1
+            out["forced_widening"] = {"median_ms_fwd_vjp": round(statistics.median(msw), 4),
+                                      "widened": int(sw["widened"]), "verdict": int(sw["verdict"]),
+                                      "fallback": int(sw["fallback"]), "c_band": int(sw["c_band"]),
+                                      "note": "the forced-fallback bracket with widen=1: the missed side is "
+                                              "re-bracketed from the same sample and the row streamed again"}
     # the same step with the certification folded into the streaming pass
     opt_fused = L.options(certify=L.CERTIFY_FUSED)
 

@@ -38,7 +38,7 @@ class LapSumError(RuntimeError):
 class Options(C.Structure):
     _fields_ = [("seed", C.c_uint64), ("sample_size", C.c_int64), ("delta", C.c_double),
                 ("band_cap", C.c_int64), ("spin_cap", C.c_int32), ("force_path", C.c_int32),
-                ("certify", C.c_int32), ("reserved", C.c_int32 * 3)]
+                ("certify", C.c_int32), ("widen", C.c_int32), ("reserved", C.c_int32 * 2)]
 
 
 class Stats(C.Structure):
@@ -47,7 +47,8 @@ class Stats(C.Structure):
                 ("c_L", C.c_int64), ("c_band", C.c_int64), ("c_R", C.c_int64),
                 ("a_L", C.c_float), ("a_R", C.c_float), ("S_L", C.c_double), ("S_R", C.c_double),
                 ("G_aL", C.c_double), ("G_aR", C.c_double), ("b", C.c_double),
-                ("sum_p", C.c_double), ("j_star", C.c_int64), ("reserved", C.c_int64 * 4)]
+                ("sum_p", C.c_double), ("j_star", C.c_int64), ("widened", C.c_int64),
+                ("reserved", C.c_int64 * 3)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
@@ -117,10 +118,11 @@ def _need(x: torch.Tensor, name: str, dtype=torch.float32):
 
 
 def options(seed: int = 0, sample_size: int = 0, delta: float = 0.0, band_cap: int = 0,
-            spin_cap: int = 0, force_path: int = PATH_AUTO, certify: int = CERTIFY_PASS) -> Options:
+            spin_cap: int = 0, force_path: int = PATH_AUTO, certify: int = CERTIFY_PASS,
+            widen: int = 0) -> Options:
     o = Options()
     o.seed, o.sample_size, o.delta, o.band_cap = seed, sample_size, delta, band_cap
-    o.spin_cap, o.force_path, o.certify = spin_cap, force_path, certify
+    o.spin_cap, o.force_path, o.certify, o.widen = spin_cap, force_path, certify, widen
     return o
 
 

@@ -125,6 +125,15 @@ __device__ __forceinline__ double sample_ln(double x) {
 }
 
 constexpr uint64_t SAMPLE_TAG = 0x4C41505355534D50ull;   // Philox key word 1
+
+// The widening round's first two kernels run only after a missed bracket (the
+// certification left a direction); the rest run once the select has started it.
+__device__ __forceinline__ bool widen_starts(const BracketParams &P) {
+    return P.ctl->verdict == 0 && P.ctl->widen_dir != 0;
+}
+__device__ __forceinline__ bool round_skipped(const BracketParams &P) {
+    return P.round2 && !P.ctl->widened;
+}
 constexpr int SEL_BINS = 65536;   // select histogram of the top 16 key bits (then 256 of the top 8)
 
 // y_j = r_{I_j} + t L_j: I_j uniform on [0, n) (high word of u0 * n), L_j ~
@@ -136,6 +145,10 @@ __global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
     __shared__ uint32_t s_h0[256];
     s_h0[threadIdx.x] = 0u;
     pdl_enter();
+    if (P.round2) {   // the same sample again, for the widened ranks
+        if (!widen_starts(P)) return;
+        if (blockIdx.x == 0 && threadIdx.x < 2) P.ctl->sel_cnt[threadIdx.x] = 0u;
+    }
     __syncthreads();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j < P.s) {
@@ -210,6 +223,7 @@ __global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams P) {
     __shared__ uint32_t s_pref[2], s_rank[2], s_bin0[2];
     __shared__ bool s_last;
     pdl_enter();
+    if (P.round2 && !widen_starts(P)) return;
     const int tid = threadIdx.x, lane = tid & 31;
     const int64_t s = P.s;
     Ctl *ctl = P.ctl;
@@ -335,10 +349,31 @@ __global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams P) {
     if (tid == 0) {
         const float yR = desc_key_to_float(s_pref[0]);
         const float yL = desc_key_to_float(s_pref[1]);
-        ctl->a_R = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
-        ctl->a_L = valid[1] ? yL : -CUDART_INF_F;
-        ctl->jR = P.jR;
-        ctl->jL = P.jL;
+        const float aR = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
+        const float aL = valid[1] ? yL : -CUDART_INF_F;
+        if (P.round2) {   // the missed side becomes the bracket; the stream starts afresh
+            if (ctl->widen_dir > 0) {   // b >= old a_R
+                ctl->a_L = ctl->a_R;
+                ctl->jL = ctl->jR;
+                ctl->a_R = aR;
+                ctl->jR = P.jR;
+            } else {                    // b < old a_L
+                ctl->a_R = ctl->a_L;
+                ctl->jR = ctl->jL;
+                ctl->a_L = aL;
+                ctl->jL = P.jL;
+            }
+            ctl->c_band = 0ull;
+            ctl->band_kmax = 0u;
+            ctl->band_kinv = 0u;
+            atomicAnd(&ctl->status, ~(ST_NO_ROOT | ST_BAND_OVERFLOW));   // the first band solve's misses
+            ctl->widened = 1;
+        } else {
+            ctl->a_R = aR;
+            ctl->a_L = aL;
+            ctl->jR = P.jR;
+            ctl->jL = P.jL;
+        }
         ctl->s = P.s;
         ctl->path = 2;
         ctl->verdict = -1;
@@ -572,6 +607,18 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
     }
 }
 
+// The verdict, and for a failed first round with widening enabled the side the
+// threshold lies on: a bracket whose counts agree and whose band fits, but with
+// G(a_R) >= k (b at or above a_R) or G(a_L) < k (b below a_L), was missed.
+__device__ __forceinline__ void set_verdict(const BracketParams &P, bool ok, bool sound, double GaL,
+                                            double GaR) {
+    Ctl *ctl = P.ctl;
+    ctl->verdict = ok ? 1 : 0;
+    int dir = 0;
+    if (!ok && sound && P.widen && !P.round2) dir = GaR >= P.k ? 1 : (GaL < P.k ? -1 : 0);
+    ctl->widen_dir = dir;
+}
+
 // CERT = false: streaming pass (forward over the row): c_L, c_R, S_L, S_R and
 //               the band.
 // CERT = true:  certification pass (backward over the row, starting on what
@@ -591,6 +638,7 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
     pdl_enter();
+    if (round_skipped(P)) return;
     if (!CERT) {   // the select histogram is spent: clear it for the next solve
         uint4 *h = reinterpret_cast<uint4 *>(P.hist1);
         for (int64_t i = (int64_t)blockIdx.x * SBLOCK + threadIdx.x; i < SEL_BINS / 4; i += (int64_t)gridDim.x * SBLOCK)
@@ -668,10 +716,10 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
             const double GaR = (double)cR - 0.5 * v[3] + 0.5 * fma(rho, v[2], v[5]);
             ctl->G_aL = GaL;
             ctl->G_aR = GaR;
-            const bool ok = (cb <= (unsigned long long)P.band_cap) && (GaL >= P.k) && (GaR < P.k) &&
-                            (cL + cb + cR == (unsigned long long)n) && ((ctl->status & ST_NONFINITE) == 0);
-            ctl->verdict = ok ? 1 : 0;
-            if (!ok) ctl->fallback_ran = 1;
+            const bool sound = (cb <= (unsigned long long)P.band_cap) &&
+                               (cL + cb + cR == (unsigned long long)n) && ((ctl->status & ST_NONFINITE) == 0);
+            const bool ok = sound && (GaL >= P.k) && (GaR < P.k);
+            set_verdict(P, ok, sound, GaL, GaR);
             if (cb > (unsigned long long)P.band_cap) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
         }
         return;
@@ -688,12 +736,11 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
         ctl->G_aL = GaL;
         ctl->G_aR = GaR;
         const unsigned long long cL = ctl->c_L, cR = ctl->c_R, cb = ctl->c_band;
-        const bool ok = (cb <= (unsigned long long)P.band_cap) && (GaL >= P.k) && (GaR < P.k) &&
-                        (cL + cb + cR == (unsigned long long)n) &&
-                        ((unsigned long long)cntR == cR) && ((unsigned long long)(cntL - cntR) == cb) &&
-                        ((unsigned long long)cntB == cL) && ((ctl->status & ST_NONFINITE) == 0);
-        ctl->verdict = ok ? 1 : 0;
-        if (!ok) ctl->fallback_ran = 1;
+        const bool sound = (cb <= (unsigned long long)P.band_cap) && (cL + cb + cR == (unsigned long long)n) &&
+                           ((unsigned long long)cntR == cR) && ((unsigned long long)(cntL - cntR) == cb) &&
+                           ((unsigned long long)cntB == cL) && ((ctl->status & ST_NONFINITE) == 0);
+        const bool ok = sound && (GaL >= P.k) && (GaR < P.k);
+        set_verdict(P, ok, sound, GaL, GaR);
         if (cb > (unsigned long long)P.band_cap) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
     }
 }

@@ -44,6 +44,7 @@ __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
     const Ctl *c = A.ctl;
     if (A.gate == GATE_BAND) {
         if (c->path != 2) return -1;
+        if (A.round2 && !c->widened) return -1;
         const unsigned long long cb = c->c_band;
         if (cb <= (unsigned long long)A.small_cap || cb > (unsigned long long)A.cap) return -1;
         if (band_tied(c)) return -1;   // one tied value: the band solver takes it in closed form

@@ -28,7 +28,7 @@ template <int BLOCK, int KPT, bool BAND>
 __global__ void __launch_bounds__(BLOCK, 1)
 rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, double t, double inv_t,
                 float *__restrict__ p_out, double *__restrict__ b_out, Ctl *ctl, int64_t band_cap,
-                int64_t band_lo) {
+                int64_t band_lo, int32_t round2) {
     using C = RowCfg<BLOCK, KPT>;
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);
@@ -45,6 +45,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     const float *row;
     double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
     if (BAND) {
+        if (round2 && !ctl->widened) return;   // the widening round did not start
         unsigned long long cb = ctl->c_band;
         if (cb > (unsigned long long)band_cap) {
             if (tid == 0) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
@@ -269,7 +270,7 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
 template <int BLOCK, int KPT, bool BAND>
 static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n, double k, double t,
                                    float *p, double *b, Ctl *ctl, int64_t band_cap, int64_t band_lo,
-                                   cudaStream_t st) {
+                                   int32_t round2, cudaStream_t st) {
     using C = RowCfg<BLOCK, KPT>;
     auto kern = rowsolve_kernel<BLOCK, KPT, BAND>;
     static bool attr = false;
@@ -280,7 +281,7 @@ static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n,
         attr = true;
     }
     return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl, band_cap,
-                    band_lo);
+                    band_lo, round2);
 }
 
 int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
@@ -288,19 +289,20 @@ int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st) {
     if (n <= RowCfg<256, 16>::CAP)
-        return launch_rowsolve<256, 16, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, st);
-    return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, st);
+        return launch_rowsolve<256, 16, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, 0, st);
+    return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, 0, st);
 }
 
 // Two variants, each gated on the band size the streaming pass counted: bands
 // of up to 4096 scores (and tied or empty bands) in a 256-thread CTA, larger
 // ones up to 32768 in a 1024-thread CTA.
 cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
-                                 cudaStream_t st) {
-    cudaError_t e = launch_rowsolve<256, 16, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, st);
+                                 int32_t round2, cudaStream_t st) {
+    cudaError_t e =
+        launch_rowsolve<256, 16, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, round2, st);
     if (e != cudaSuccess) return e;
     return launch_rowsolve<1024, 32, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap,
-                                           RowCfg<256, 16>::CAP, st);
+                                           RowCfg<256, 16>::CAP, round2, st);
 }
 
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,

@@ -321,6 +321,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < 0) return LAPSUM_ERR_ARG;
     if (opt.force_path < 0 || opt.force_path > 2) return LAPSUM_ERR_ARG;
     if (opt.certify != LAPSUM_CERTIFY_PASS && opt.certify != LAPSUM_CERTIFY_FUSED) return LAPSUM_ERR_ARG;
+    if (opt.widen != 0 && opt.widen != 1) return LAPSUM_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
     const int32_t spin_cap = opt.spin_cap ? opt.spin_cap : (1 << 20);
     Workspace *w = get_ws(st);
@@ -372,36 +373,69 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     P.band_cap = band_cap;
     P.spin_cap = spin_cap;
     P.fused_cert = opt.certify == LAPSUM_CERTIFY_FUSED;
+    P.widen = opt.widen;
+    // the widening round, on the same sample: the ranks of confidence delta^2,
+    // moved at least one first-round spread (jL - jR, at least 1) beyond the first
+    // round's ranks and clipped to [0, s + 1]; its band lies between a first-round
+    // end and the new end on the side that was missed
+    BracketParams P2{};
+    if (opt.widen) {
+        P2 = P;
+        P2.round2 = 1;
+        const double delta = opt.delta != 0.0 ? opt.delta : 1e-6;
+        binomial_ranks(s, k / (double)n, std::max(delta * delta, 1e-300), P2.jR, P2.jL);
+        const int64_t spread = std::max<int64_t>(1, P.jL - P.jR);
+        P2.jR = std::max<int64_t>(0, std::min(P2.jR, P.jR - spread));
+        P2.jL = std::min<int64_t>(s + 1, std::max(P2.jL, P.jL + spread));
+        int64_t cap2 = opt.band_cap;
+        if (cap2 == 0) {
+            const int64_t gap = std::max(P.jR - P2.jR, P2.jL - P.jL);
+            const double want = 4.0 * (double)n * (double)(gap + 2) / (double)s;
+            cap2 = std::max<int64_t>(65536, (int64_t)std::ceil(want));
+        }
+        P2.band_cap = std::min<int64_t>(cap2, n);
+    }
+    const int64_t band_buf = std::max(band_cap, opt.widen ? P2.band_cap : int64_t(0));
     LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
     LAPSUM_TRY(grow(w->hist1, w->hist1_n, 65536 + 256));
     LAPSUM_TRY(grow(w->selcand, w->selcand_n, (size_t)2 * select_cand_capacity()));
-    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_cap));
+    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_buf));
     LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort the whole row
-    P.band = w->band;
-    P.keys = w->skeys;
-    P.hist1 = w->hist1;
-    P.cand = w->selcand;
-    P.partials = w->partials;
-    P.ctl = w->ctl;
+
+    P2.band = P.band = w->band;
+    P2.keys = P.keys = w->skeys;
+    P2.hist1 = P.hist1 = w->hist1;
+    P2.cand = P.cand = w->selcand;
+    P2.partials = P.partials = w->partials;
+    P2.ctl = P.ctl = w->ctl;
 
     LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
-    { Launch L("sample", st); LAPSUM_TRY(launch_sample(P, st)); }
-    { Launch L("select", st); LAPSUM_TRY(launch_select(P, st)); }
-    { Launch L("stream_pass", st); LAPSUM_TRY(launch_stream_pass(P, st)); }
-    {
-        Launch L("band_rowsolve", st);
-        ++g_launches;   // two size-gated variants
-        LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, band_cap, st));
-    }
-    if (band_cap > rowsolve_capacity()) {
-        SortArgs A = sort_args(w, w->band, 0, band_cap, GATE_BAND, spin_cap, k, t);
+    // one bracketing round: sample, select, stream, band solve, certification
+    auto bracket_round = [&](const BracketParams &Q) -> int {
+        const bool r2 = Q.round2 != 0;   // profiling names are literals (the profiler keeps the pointer)
+        { Launch L(r2 ? "widen_sample" : "sample", st); LAPSUM_TRY(launch_sample(Q, st)); }
+        { Launch L(r2 ? "widen_select" : "select", st); LAPSUM_TRY(launch_select(Q, st)); }
+        { Launch L(r2 ? "widen_stream_pass" : "stream_pass", st); LAPSUM_TRY(launch_stream_pass(Q, st)); }
         {
-            Launch L("band_radix_sort", st);
-            LAPSUM_TRY(launch_radix_sort(A, k, t, st));
+            Launch L(r2 ? "widen_band_rowsolve" : "band_rowsolve", st);
+            ++g_launches;   // two size-gated variants
+            LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, Q.band_cap, Q.round2, st));
         }
-        { Launch L("band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
+        if (Q.band_cap > rowsolve_capacity()) {
+            SortArgs A = sort_args(w, w->band, 0, Q.band_cap, GATE_BAND, spin_cap, k, t);
+            A.round2 = Q.round2;
+            { Launch L(r2 ? "widen_band_radix_sort" : "band_radix_sort", st); LAPSUM_TRY(launch_radix_sort(A, k, t, st)); }
+            { Launch L(r2 ? "widen_band_locate" : "band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
+        }
+        if (!Q.fused_cert) { Launch L(r2 ? "widen_certify" : "certify", st); LAPSUM_TRY(launch_certify(Q, st)); }
+        return LAPSUM_OK;
+    };
+    rc = bracket_round(P);
+    if (rc) return rc;
+    if (opt.widen) {
+        rc = bracket_round(P2);
+        if (rc) return rc;
     }
-    if (!P.fused_cert) { Launch L("certify", st); LAPSUM_TRY(launch_certify(P, st)); }
     rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, st);
     if (rc) return rc;
     { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, st)); }
@@ -486,6 +520,7 @@ int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream_in) {
     out->b = c.b;
     out->sum_p = c.sum_p;
     out->j_star = c.j_star;
+    out->widened = c.widened;
     if (c.status & ST_NONFINITE) return LAPSUM_ERR_NONFINITE;
     if (c.status & ST_TIMEOUT) return LAPSUM_ERR_DEVICE_TIMEOUT;
     if ((c.status & ST_NO_ROOT) && !(c.path == 2 && c.fallback_ran)) return LAPSUM_ERR_NO_ROOT;

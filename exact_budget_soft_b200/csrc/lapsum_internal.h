@@ -28,6 +28,8 @@ struct Ctl {
     // certification pass
     double G_aL, G_aR;
     int32_t verdict;          // 1 certified, 0 not (fallback must run), -1 n/a
+    int32_t widen_dir;        // failed certification: +1 b at or above a_R, -1 below a_L, 0 other
+    int32_t widened;          // the widening round is running (or ran)
     int32_t status;           // ST_* bits
     int32_t path;
     int32_t fallback_ran;
@@ -67,6 +69,8 @@ struct BracketParams {
     Ctl *ctl;
     int32_t spin_cap;
     int32_t fused_cert;       // certification folded into the streaming pass
+    int32_t widen;            // a widening round follows a missed bracket
+    int32_t round2;           // this launch belongs to the widening round
 };
 
 }  // namespace lapsum

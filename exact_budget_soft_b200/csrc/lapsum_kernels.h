@@ -48,7 +48,7 @@ int rowsolve_capacity();
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st);
 cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
-                                 cudaStream_t st);
+                                 int32_t round2, cudaStream_t st);
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
                           int64_t n, double t, float *grad, cudaStream_t st);
 
@@ -80,6 +80,7 @@ struct SortArgs {
     double *tilebuf;           // locate per-tile data
     Ctl *ctl;
     int32_t gate;
+    int32_t round2;            // band gate of the widening round: runs only once it started
     int32_t spin_cap;          // grid-barrier polls before a wait gives up
     int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
     double k, t;               // budget and temperature (all-equal shortcut)

@@ -88,6 +88,18 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
  *               pass"); LAPSUM_CERTIFY_FUSED: the streaming pass also adds the
  *               band scores' certification terms and decides the verdict, so the
  *               row is read once less.
+ *   widen       0 (default): a bracket that fails certification goes straight to
+ *               the full-sort fallback.  1: first one widening round ("Fast
+ *               LapSum", technical summary section 2.2 step 4, the bracket
+ *               "iteratively widened"): when the failure is a miss -- the counts
+ *               agree, the band fits, but G(a_R) >= k (b at or above a_R) or
+ *               G(a_L) < k (b below a_L) -- the same sample is re-selected at the
+ *               ranks of confidence delta^2 and the missed side becomes the new
+ *               bracket: [a_R, y_(jR2)) or [y_(jL2), a_L).  The row is streamed,
+ *               the band solved and the bracket certified again; the full sort
+ *               runs only if that round fails too.  Every decision is taken on
+ *               the device (the round's kernels return at once when it is not
+ *               needed).
  */
 typedef struct {
     uint64_t seed;
@@ -97,7 +109,8 @@ typedef struct {
     int32_t  spin_cap;
     int32_t  force_path;
     int32_t  certify;
-    int32_t  reserved[3];
+    int32_t  widen;
+    int32_t  reserved[2];
 } lapsum_options;
 
 /*
@@ -114,6 +127,7 @@ typedef struct {
  *   G_aL, G_aR  certification values G(a_L), G(a_R)
  *   b         the threshold of row 0
  *   sum_p     sum of the fp32 p of row 0, accumulated in fp64
+ *   widened   1 if the widening round ran (then s..G_aR describe its bracket)
  */
 typedef struct {
     int32_t path, verdict, status, fallback;
@@ -125,7 +139,8 @@ typedef struct {
     double  b;
     double  sum_p;
     int64_t j_star;
-    int64_t reserved[4];
+    int64_t widened;
+    int64_t reserved[3];
 } lapsum_stats;
 
 /*

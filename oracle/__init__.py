@@ -68,6 +68,9 @@ def _load():
                 "orc_sample": (None, [f32p, C.c_int64, C.c_double, C.c_uint64, C.c_int64,
                                       C.c_int64, f64p, i64p]),
                 "orc_binom_ranks": (C.c_int, [C.c_int64, C.c_double, C.c_double, lp, lp]),
+                "orc_widen_ranks": (C.c_int, [C.c_int64, C.c_double, C.c_double, lp, lp]),
+                "orc_bracket_at_ranks": (C.c_int, [f32p, C.c_int64, C.c_double, C.c_uint64, C.c_int64,
+                                                   C.c_int64, C.c_int64, C.c_int64, fp, fp]),
                 "orc_bracket": (C.c_int, [f32p, C.c_int64, C.c_double, C.c_double, C.c_uint64,
                                           C.c_int64, C.c_int64, C.c_double, fp, fp, lp, lp]),
                 "orc_counts": (None, [f32p, C.c_int64, C.c_float, C.c_float, lp, lp, lp]),
@@ -180,6 +183,26 @@ def bracket(r, k: float, t: float, seed: int, s: int, delta: float, row: int = 0
     if rc != 0:
         raise ValueError("bad bracket arguments")
     return {"a_L": np.float32(aL.value), "a_R": np.float32(aR.value), "jR": jr.value, "jL": jl.value}
+
+
+def widen_ranks(s: int, pi: float, delta: float) -> tuple[int, int]:
+    """Ranks (jR2, jL2) of the widening round (delta^2 ranks, moved at least one
+    first-round spread beyond the first round's ranks)."""
+    jr, jl = C.c_int64(), C.c_int64()
+    rc = _load().orc_widen_ranks(int(s), float(pi), float(delta), C.byref(jr), C.byref(jl))
+    if rc != 0:
+        raise ValueError("bad binomial arguments")
+    return jr.value, jl.value
+
+
+def bracket_at_ranks(r, t: float, seed: int, s: int, jR: int, jL: int, row: int = 0) -> dict:
+    r = _f32(r)
+    aL, aR = C.c_float(), C.c_float()
+    rc = _load().orc_bracket_at_ranks(r, r.size, float(t), int(seed), int(row), int(s), int(jR), int(jL),
+                                      C.byref(aL), C.byref(aR))
+    if rc != 0:
+        raise ValueError("bad rank arguments")
+    return {"a_L": np.float32(aL.value), "a_R": np.float32(aR.value), "jR": jR, "jL": jL}
 
 
 def counts(r, a_L: float, a_R: float) -> tuple[int, int, int]:

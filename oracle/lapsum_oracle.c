@@ -416,6 +416,48 @@ int orc_bracket(const float *r, int64_t n, double k, double t, uint64_t seed, in
     return 0;
 }
 
+/*
+ * Bracket ends at given ranks of the same sample (outward fp32 rounding as in
+ * orc_bracket): a_R = nextup(rd(y_(jR))) (+inf for jR = 0), a_L = rd(y_(jL))
+ * (-inf for jL = s + 1).
+ */
+int orc_bracket_at_ranks(const float *r, int64_t n, double t, uint64_t seed, int64_t row, int64_t s,
+                         int64_t jR, int64_t jL, float *aL, float *aR)
+{
+    if (s < 1 || jR < 0 || jR > s || jL < 1 || jL > s + 1) return -1;
+    double *y = malloc((size_t)s * sizeof(double));
+    orc_sample(r, n, t, seed, row, s, y, NULL);
+    qsort(y, (size_t)s, sizeof(double), cmp_desc);
+    *aR = jR >= 1 ? nextafterf(f32_down(y[jR - 1]), INFINITY) : INFINITY;
+    *aL = jL <= s ? f32_down(y[jL - 1]) : -INFINITY;
+    free(y);
+    return 0;
+}
+
+/*
+ * Ranks of the widening round ("iteratively widened" bracket, technical
+ * summary section 2.2 step 4; the rule is this implementation's reading):
+ * start from the ranks of confidence delta^2 and move each at least one
+ * first-round spread (jL - jR, at least 1) beyond the first round's rank,
+ * clipped to [0, s + 1].  A miss above a_R uses jR2, a miss below a_L uses jL2.
+ */
+int orc_widen_ranks(int64_t s, double pi, double delta, int64_t *jR2, int64_t *jL2)
+{
+    int64_t jR, jL, r2, l2;
+    if (orc_binom_ranks(s, pi, delta, &jR, &jL) != 0) return -1;
+    double d2 = delta * delta;
+    if (d2 < 1e-300) d2 = 1e-300;
+    if (orc_binom_ranks(s, pi, d2, &r2, &l2) != 0) return -1;
+    int64_t spread = jL - jR;
+    if (spread < 1) spread = 1;
+    if (r2 > jR - spread) r2 = jR - spread;
+    if (r2 < 0) r2 = 0;
+    if (l2 < jL + spread) l2 = jL + spread;
+    if (l2 > s + 1) l2 = s + 1;
+    *jR2 = r2; *jL2 = l2;
+    return 0;
+}
+
 /* Band membership [FL-2.2 step 2]: above r >= a_R; band a_L <= r < a_R; below r < a_L. */
 void orc_counts(const float *r, int64_t n, float aL, float aR, int64_t *cL, int64_t *cB, int64_t *cR)
 {

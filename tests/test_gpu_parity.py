@@ -291,3 +291,76 @@ def test_bracketing_band_of_one_tied_level(L, orc, level, certify):
     p, b, st, grad = run(L, r, k, t, opts=L.options(certify=certify), g_np=g)
     assert st["rc"] == 0 and st["path"] == 2
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0], exact_sum=False)
+
+
+# ------------------------------------------------ bracket widening (NEXT-1) --
+def widened_bracket(orc, r, k, t, seed, s, delta):
+    """The oracle's prediction of the widening round: first-round bracket, the
+    side it missed (from its certification), and the bracket of the second round
+    (the missed side, up to the delta^2 order statistic of the same sample)."""
+    br1 = orc.bracket(r, k, t, seed, s, delta)
+    c1 = orc.certify(r, k, t, br1["a_L"], br1["a_R"], band_cap=10**12)
+    if c1["verdict"] == 1:
+        return br1, 0, None
+    jR2, jL2 = orc.widen_ranks(s, k / r.size, delta)
+    br2 = orc.bracket_at_ranks(r, t, seed, s, jR2, jL2)
+    if c1["G_aR"] >= k:   # b at or above a_R
+        return br1, 1, {"a_L": br1["a_R"], "a_R": br2["a_R"], "jL": br1["jR"], "jR": br2["jR"]}
+    assert c1["G_aL"] < k
+    return br1, -1, {"a_L": br2["a_L"], "a_R": br1["a_L"], "jL": br2["jL"], "jR": br1["jL"]}
+
+
+def find_widen_seed(orc, r, k, t, s, delta, want_cover):
+    for sd in range(400):
+        _, d, br2 = widened_bracket(orc, r, k, t, sd, s, delta)
+        if d == 0:
+            continue
+        c2 = orc.certify(r, k, t, br2["a_L"], br2["a_R"], band_cap=10**12)
+        if (c2["verdict"] == 1) == want_cover:
+            return sd, d, br2, c2
+    raise AssertionError("no seed found")
+
+
+@pytest.mark.parametrize("certify", [0, 1])
+def test_widening_recovers_a_missed_bracket(L, orc, certify):
+    r, g = W.small_case("normal", 1, 1 << 20, seed=6)
+    k, t, s, delta = 5000.0, 0.05, 256, 0.5
+    seed, d, br2, c2 = find_widen_seed(orc, r[0], k, t, s, delta, want_cover=True)
+    p, b, st, grad = run(L, r, k, t, opts=L.options(seed=seed, sample_size=s, delta=delta, certify=certify,
+                                                     widen=1), g_np=g)
+    assert st["rc"] == 0 and st["widened"] == 1 and st["verdict"] == 1 and st["fallback"] == 0
+    assert np.float32(st["a_L"]) == br2["a_L"] and np.float32(st["a_R"]) == br2["a_R"]
+    assert (st["jR"], st["jL"]) == (br2["jR"], br2["jL"])
+    assert (st["c_L"], st["c_band"], st["c_R"]) == (c2["c_L"], c2["c_band"], c2["c_R"])
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+@pytest.mark.parametrize("certify", [0, 1])
+def test_widening_that_misses_again_falls_back(L, orc, certify):
+    r, g = W.small_case("laplace", 1, 1 << 20, seed=8)
+    k, t, s, delta = 20000.0, 0.05, 64, 0.9
+    seed, d, br2, c2 = find_widen_seed(orc, r[0], k, t, s, delta, want_cover=False)
+    p, b, st, grad = run(L, r, k, t, opts=L.options(seed=seed, sample_size=s, delta=delta, certify=certify,
+                                                     widen=1), g_np=g)
+    assert st["rc"] == 0 and st["widened"] == 1 and st["verdict"] == 0 and st["fallback"] == 1
+    assert np.float32(st["a_L"]) == br2["a_L"] and np.float32(st["a_R"]) == br2["a_R"]
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+def test_widening_not_needed_changes_nothing(L, orc):
+    r, g = W.small_case("normal", 1, 1 << 20, seed=9)
+    k, t = 1000.0, 0.05
+    p0, b0, st0, _ = run(L, r, k, t)
+    p1, b1, st1, grad = run(L, r, k, t, opts=L.options(widen=1), g_np=g)
+    assert st1["widened"] == 0 and st1["verdict"] == 1 and st1["fallback"] == 0
+    assert b1[0] == b0[0] and np.array_equal(p1, p0)
+    check_row(orc, r[0], g[0], k, t, p1[0], b1[0], grad[0])
+
+
+def test_widening_skips_band_overflow(L, orc):
+    # a bracket that holds b but whose band overflows is not widened: full sort
+    r, g = W.small_case("normal", 1, 1 << 20, seed=5)
+    k, t = 3000.0, 0.05
+    p, b, st, grad = run(L, r, k, t, opts=L.options(band_cap=64, widen=1), g_np=g)
+    assert st["widened"] == 0 and st["verdict"] == 0 and st["fallback"] == 1
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])

@@ -311,3 +311,58 @@ def test_counts_partition(orc):
     assert (cl, cb, cr) == (int((ok < -0.5).sum()), int(((ok >= -0.5) & (ok < 1.5)).sum()),
                             int((ok >= 1.5).sum()))
     assert cl + cb + cr == r.size - 1
+
+
+def _scipy_ranks(s, pi, delta):
+    # jR: largest j with P(X < j) <= delta/2; jL: smallest j with P(X >= j) <= delta/2
+    X = st.binom(s, pi)
+    jR = max([j for j in range(0, s + 1) if X.cdf(j - 1) <= delta / 2] + [0])
+    jL = min([j for j in range(0, s + 2) if X.sf(j - 1) <= delta / 2])
+    return jR, jL
+
+
+@pytest.mark.parametrize("s,pi,delta", [(256, 5000 / 2**20, 0.5), (64, 20000 / 2**20, 0.9),
+                                        (4096, 0.01, 1e-3), (65536, 0.01, 1e-6), (512, 0.3, 0.2)])
+def test_widen_ranks_pinned_to_binomial_tails(orc, s, pi, delta):
+    # the widening round's ranks: at least as far out as the delta^2 tails
+    # (scipy), at least one first-round spread beyond the first round, in [0, s+1]
+    jR, jL = _scipy_ranks(s, pi, delta)
+    r2, l2 = _scipy_ranks(s, pi, max(delta * delta, 1e-300))
+    jR2, jL2 = orc.widen_ranks(s, pi, delta)
+    spread = max(1, jL - jR)
+    assert 0 <= jR2 <= min(r2, max(0, jR - spread)) and (jR2 == 0 or jR2 == min(r2, jR - spread))
+    assert max(l2, min(s + 1, jL + spread)) <= jL2 <= s + 1 and (jL2 == s + 1 or jL2 == max(l2, jL + spread))
+    assert jR2 < jR or jR == 0
+    assert jL2 > jL or jL == s + 1
+
+
+def test_widen_ranks_worked_cases(orc):
+    # s = 256, pi = 5000/2^20, delta = 0.5: the first-round ranks are (0, 3) and the
+    # delta^2 ranks are (0, 3) too, so only the one-spread rule moves jL: (0, 6)
+    assert orc.binom_ranks(256, 5000 / 2**20, 0.5) == (0, 3)
+    assert orc.binom_ranks(256, 5000 / 2**20, 0.25) == (0, 3)
+    assert orc.widen_ranks(256, 5000 / 2**20, 0.5) == (0, 6)
+
+
+def test_bracket_at_ranks_is_outward_order_statistics(orc):
+    r = _row(4000, seed=24)
+    t, s, seed = 0.05, 1024, 5
+    y, _ = orc.sample(r, t, seed, s)
+    ys = np.sort(y)[::-1]
+    for jR, jL in [(0, 1), (3, 17), (100, 1025), (1024, 1024)]:
+        br = orc.bracket_at_ranks(r, t, seed, s, jR, jL)
+        if jR == 0:
+            assert br["a_R"] == np.float32(np.inf)
+        else:
+            f = np.float32(ys[jR - 1])
+            down = f if float(f) <= ys[jR - 1] else np.nextafter(f, np.float32(-np.inf))
+            assert br["a_R"] == np.nextafter(down, np.float32(np.inf))
+        if jL == s + 1:
+            assert br["a_L"] == np.float32(-np.inf)
+        else:
+            assert float(br["a_L"]) <= ys[jL - 1] < float(np.nextafter(br["a_L"], np.float32(np.inf)))
+    # at the first-round ranks it is the bracket itself
+    k, delta = 40.0, 1e-3
+    b1 = orc.bracket(r, k, t, seed, s, delta)
+    b2 = orc.bracket_at_ranks(r, t, seed, s, b1["jR"], b1["jL"])
+    assert (b1["a_L"], b1["a_R"]) == (b2["a_L"], b2["a_R"])
