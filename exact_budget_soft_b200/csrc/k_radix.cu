@@ -6,14 +6,14 @@
 //
 // Sort: keys-only LSD radix sort of the descending-order uint32 keys, 8-bit
 // digits, in one cooperative kernel (radix_sort_kernel, described below).
-// Locate: one kernel; every CTA reduces one tile of sorted values to its two
-// affine maps (prefix P, suffix Q); the last CTA scans the tile maps, finds the
-// tile whose end brackets G = k, re-scans that tile in shared memory and takes
-// the closed-form root.
+// Locate (the same kernel, after the last pass): tile and chunk maps of the
+// prefix/suffix scans, then one CTA narrows the crossing down chunk -> tile ->
+// value and takes the closed-form root.
 //
 // The host never learns the band size or the certification verdict: every
 // kernel reads its element count and its gate from the control block and
 // returns at once when it has nothing to do.
+#include <climits>
 #include <cstdint>
 
 #include "lapsum_device.cuh"
@@ -31,13 +31,8 @@ constexpr int64_t SMALL_SORT = int64_t(1) << 20;
 constexpr int RNW = RB / 32;
 constexpr int HB = 256;             // histogram kernel threads
 
-constexpr int LB = 1024;            // locate: threads
-constexpr int LK = 16;              // values per thread
-constexpr int LTILE = LB * LK;      // 16384 values per tile
-constexpr int LOC_KEY_WORDS = LTILE + LTILE / 32 + 8;   // padded tile + two halo entries
 
 int radix_tile() { return TILE_K(RK_BIG); }
-int locate_tile() { return LTILE; }
 
 // Element count behind a gate; < 0 means "nothing to do".
 __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
@@ -211,6 +206,252 @@ __device__ __forceinline__ bool walk_chunk(TileStage<K> &S, const SortArgs &A, c
     return ok;
 }
 
+// ------------------------------------------------------------ locate --
+// After the last pass the sorted values c_0 >= c_1 >= ... sit in one key buffer.
+// The threshold curve is evaluated by affine scans (prefix P_j = 1 + d_{j-1}
+// P_{j-1}, suffix Q_j = 1 + d_j Q_{j+1}, links d_j = e^{(c_{j+1} - c_j)/t}):
+//   1. every CTA reduces each tile of its chunk to its two maps (a tile record)
+//      and composes them into its chunk's maps (a chunk record);   barrier;
+//   2. CTA 0 scans the chunk maps and finds the chunk whose end first has
+//      G > k -- the crossing is in it (or below the last value);
+//   3. CTA 0 scans that chunk's tile maps and finds the crossing tile;
+//   4. CTA 0 re-scans that tile element by element and takes the closed-form
+//      root (block_scan_solve).
+struct TileRec {
+    double pa, ps;     // tile prefix map  P_end = pa * P_before + ps
+    double qa, qs;     // tile suffix map  Q_first = qa * Q_after + qs
+    double d_out;      // link from the tile's last value to the next value
+    double p_end;      // filled by CTA 0 for the tiles of the crossing chunk
+    double q_after;
+    double pad;
+};
+struct ChunkRec {
+    double pa, ps, qa, qs;   // the chunk's composed maps (identity when it has no tile)
+    double d_out;            // link out of the chunk's last value
+    double last;             // index of the chunk's last value, -1 when it has no tile
+    double pad[2];
+};
+
+struct Seeds {   // what lies above and below the sorted values
+    double m0, top, P_top, bot, Q_bot;
+};
+__device__ __forceinline__ Seeds locate_seeds(const SortArgs &A) {
+    Seeds z{0.0, CUDART_INF, 0.0, -CUDART_INF, 0.0};
+    if (A.gate == GATE_BAND) {
+        const Ctl *c = A.ctl;
+        z.m0 = (double)c->c_R;
+        z.top = (double)c->a_R;
+        z.P_top = c->S_R;
+        z.bot = (double)c->a_L;
+        z.Q_bot = c->S_L;
+    }
+    return z;
+}
+
+// Step 1 for one CTA: its tiles' records and its chunk record.  s_t: room for a
+// tile plus two halo values in the padded layout; sc: scan scratch.
+template <int K>
+__device__ void locate_tiles(const SortArgs &A, const uint32_t *sorted, int64_t n, int64_t t0, int64_t t1,
+                             const Seeds &z, TileRec *rec, ChunkRec *crec, uint32_t *s_t, Aff *sc,
+                             const double *tab) {
+    constexpr int TILE = TILE_K(K);
+    const int tid = threadIdx.x;
+    const double s2d = (1.0 / A.t) * LOG2E;
+    const uint32_t key_top = desc_key((float)z.top), key_bot = desc_key((float)z.bot);
+    __shared__ Aff s_map[2];
+    __shared__ double s_dout;
+    Aff Pc = aff_id(), Qc = aff_id();
+    double dc = 0.0;
+    for (int64_t tile = t0; tile < t1; ++tile) {
+        const int64_t base = tile * TILE;
+        const int cnt = (int)min((int64_t)TILE, n - base);
+        // s_t[spad(i + 1)] = sorted position base + i for i = -1 .. cnt
+#pragma unroll
+        for (int u = 0; u < K; ++u) {
+            const int i = u * RB + tid;
+            if (i < cnt) s_t[spad(i + 1)] = __ldcg(sorted + base + i);
+        }
+        if (tid == 0) {
+            s_t[spad(0)] = base == 0 ? key_top : __ldcg(sorted + base - 1);
+            s_t[spad(cnt + 1)] = base + cnt >= n ? key_bot : __ldcg(sorted + base + cnt);
+        }
+        __syncthreads();
+        auto sval = [&](int i) -> double { return (double)desc_key_to_float(s_t[spad(i + 1)]); };
+        const int l0 = tid * K, l1 = min(l0 + K, cnt) - 1;
+        Aff mp = aff_id(), mq = aff_id();
+        double d_last = 0.0;
+        if (l0 < cnt) {
+            double cprev = sval(l0 - 1), c = sval(l0);
+            double dprev = (cprev == CUDART_INF || c == -CUDART_INF) ? 0.0 : link_exp((cprev - c) * s2d, tab);
+            for (int j = l0; j <= l1; ++j) {
+                mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
+                const double cn = sval(j + 1);
+                const double d = (c == CUDART_INF || cn == -CUDART_INF) ? 0.0 : link_exp((c - cn) * s2d, tab);
+                mq = {mq.a * d, mq.s + mq.a};
+                dprev = d;
+                c = cn;
+            }
+            d_last = dprev;
+        }
+        Aff pe, qe;
+        block_scan_excl_both<RB>(mp, mq, pe, qe, sc);
+        const int owner = (cnt - 1) / K;
+        if (tid == owner) {
+            const Aff P = aff_then(pe, mp);
+            rec[tile].pa = P.a;
+            rec[tile].ps = P.s;
+            rec[tile].d_out = d_last;
+            s_map[0] = P;
+            s_dout = d_last;
+        }
+        if (tid == 0) {
+            const Aff Q = aff_then(qe, mq);
+            rec[tile].qa = Q.a;
+            rec[tile].qs = Q.s;
+            s_map[1] = Q;
+        }
+        __syncthreads();
+        if (tid == 0) {   // the chunk's maps: P of the tiles in order, Q the other way round
+            Pc = aff_then(Pc, s_map[0]);
+            Qc = aff_then(s_map[1], Qc);
+            dc = s_dout;
+        }
+        __syncthreads();   // s_t and s_map are reused by the next tile
+    }
+    if (tid == 0) {
+        ChunkRec r;
+        r.pa = Pc.a;
+        r.ps = Pc.s;
+        r.qa = Qc.a;
+        r.qs = Qc.s;
+        r.d_out = dc;
+        r.last = t1 > t0 ? (double)(min(t1 * TILE, n) - 1) : -1.0;
+        r.pad[0] = r.pad[1] = 0.0;
+        crec[blockIdx.x] = r;
+    }
+}
+
+// max (or min, with neg = true) of one int over the CTA
+__device__ __forceinline__ int block_max_int(int v, int *s_w) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(FULL, v, o));
+    if (lane == 0) s_w[warp] = v;
+    __syncthreads();
+    int m = s_w[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = max(m, s_w[w]);
+    __syncthreads();
+    return m;
+}
+
+// Steps 2-4, CTA 0 alone, after the barrier that follows step 1.
+template <int K>
+__device__ void locate_finish(const SortArgs &A, const uint32_t *sorted, int64_t n, const Seeds &z, TileRec *rec,
+                              const ChunkRec *crec, uint32_t *s_t, void *scratch, const double *tab) {
+    constexpr int TILE = TILE_K(K);
+    const int tid = threadIdx.x;
+    const int G = gridDim.x;
+    const int64_t ntiles = (n + TILE - 1) / TILE;
+    Ctl *ctl = A.ctl;
+    Aff *sc = reinterpret_cast<Aff *>(scratch);
+    __shared__ int s_w[RB / 32];
+    __shared__ double s_d[2];
+    // ---- step 2: the chunk maps (G <= RB chunks: one scan)
+    Aff mP = aff_id(), mQ = aff_id();
+    double dO = 0.0, last = -1.0;
+    if (tid < G) {
+        const ChunkRec *r = crec + tid;
+        mP = {__ldcg(&r->pa), __ldcg(&r->ps)};
+        mQ = {__ldcg(&r->qa), __ldcg(&r->qs)};
+        dO = __ldcg(&r->d_out);
+        last = __ldcg(&r->last);
+    }
+    Aff pe, qe;
+    block_scan_excl_both<RB>(mP, mQ, pe, qe, sc);
+    const double Pb = fma(pe.a, z.P_top, pe.s);   // P before the chunk's first value
+    const double Qa = fma(qe.a, z.Q_bot, qe.s);   // Q after the chunk's last value
+    const bool full = tid < G && last >= 0.0;
+    int cand = -1;
+    if (full) {
+        const double Pend = fma(mP.a, Pb, mP.s);
+        const double Gend = (z.m0 + last + 1.0) - 0.5 * Pend + 0.5 * dO * Qa;
+        if (Gend <= A.k) cand = tid;
+    }
+    const int cstar = block_max_int(cand, s_w);
+    // the crossing chunk: the first chunk with tiles after cstar, else the last one with tiles
+    const int nxt = -block_max_int(full && tid > cstar ? -tid : INT_MIN + 1, s_w);
+    const int lastfull = block_max_int(full ? tid : -1, s_w);
+    const int tgt = (nxt != INT_MAX) ? nxt : lastfull;
+    if (tid == tgt) {
+        s_d[0] = Pb;
+        s_d[1] = Qa;
+    }
+    __syncthreads();
+    const double Pin = s_d[0], Qout = s_d[1];
+    const int64_t T0 = (int64_t)tgt * ntiles / G, T1 = (int64_t)(tgt + 1) * ntiles / G;
+    // ---- step 3: the tiles of that chunk (forward P, backward Q, RB tiles at a time)
+    __shared__ double s_carry;
+    double carry_p = Pin;
+    for (int64_t c0 = T0; c0 < T1; c0 += RB) {
+        const int64_t T = c0 + tid;
+        Aff m = aff_id();
+        if (T < T1) m = {__ldcg(&rec[T].pa), __ldcg(&rec[T].ps)};
+        Aff p2, q2;
+        block_scan_excl_both<RB>(m, aff_id(), p2, q2, sc);
+        const Aff inc = aff_then(p2, m);
+        if (T < T1) rec[T].p_end = fma(inc.a, carry_p, inc.s);
+        const int64_t lastT = min(c0 + RB, T1) - 1;
+        if (T == lastT) s_carry = fma(inc.a, carry_p, inc.s);
+        __syncthreads();
+        carry_p = s_carry;
+        __syncthreads();
+    }
+    double carry_q = Qout;
+    int best = -1;   // last tile (offset from T0) with G <= k at its end
+    const int64_t nck = (T1 - T0 + RB - 1) / RB;
+    for (int64_t ci = nck - 1; ci >= 0; --ci) {
+        const int64_t c0 = T0 + ci * RB;
+        const int64_t T = c0 + tid;
+        Aff m = aff_id();
+        if (T < T1) m = {__ldcg(&rec[T].qa), __ldcg(&rec[T].qs)};
+        Aff p2, q2;
+        block_scan_excl_both<RB>(aff_id(), m, p2, q2, sc);
+        const double Qa_t = fma(q2.a, carry_q, q2.s);   // Q after tile T
+        if (T < T1) {
+            rec[T].q_after = Qa_t;
+            const int64_t tend = min((T + 1) * TILE, n) - 1;
+            const double Gt = (z.m0 + (double)(tend + 1)) - 0.5 * rec[T].p_end + 0.5 * __ldcg(&rec[T].d_out) * Qa_t;
+            if (Gt <= A.k) best = max(best, (int)(T - T0));
+        }
+        if (tid == 0) {
+            const Aff all = aff_then(q2, m);
+            s_carry = fma(all.a, carry_q, all.s);
+        }
+        __syncthreads();
+        carry_q = s_carry;
+        __syncthreads();
+    }
+    best = block_max_int(best, s_w);
+    const int64_t TT = min(T0 + best + 1, T1 - 1);
+    // ---- step 4: the crossing tile, element by element
+    const int64_t t0v = TT * TILE;
+    const int cnt = (int)min((int64_t)TILE, n - t0v);
+    for (int i = tid; i < cnt; i += RB) s_t[spad(i)] = __ldcg(sorted + t0v + i);
+    __syncthreads();
+    const double ptop = TT == T0 ? Pin : rec[TT - 1].p_end;
+    const double qbot = rec[TT].q_after;
+    const double vtop = t0v == 0 ? z.top : (double)desc_key_to_float(__ldcg(sorted + t0v - 1));
+    const double vbot = t0v + cnt >= n ? z.bot : (double)desc_key_to_float(__ldcg(sorted + t0v + cnt));
+    int64_t js = 0;
+    const double b = block_scan_solve<RB, K>(s_t, cnt, A.k, A.t, 1.0 / A.t, z.m0 + (double)t0v, vtop, ptop, vbot,
+                                             qbot, scratch, &js, &ctl->status, tab);
+    if (tid == 0) {
+        ctl->b = b;
+        ctl->j_star = t0v + js;
+        if (A.gate == GATE_FALLBACK) ctl->fallback_ran = 1;
+    }
+}
+
 template <int K>
 constexpr size_t sort_smem() { return stage_bytes<K>() + (size_t)(RNW * 256 + 4 * 256 + 4 * 256) * 4; }
 constexpr int SORT_GMAX = 320;   // CTAs of the sort grid at most (chunk counts per digit)
@@ -225,6 +466,8 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
     uint32_t *s_tot = s_run + 256;             // 256: scratch (tile totals)
     uint32_t *s_h4 = s_tot + 256;              // 4 * 256: phase-H histograms, then digit bases
     __shared__ int s_skip, s_solved;
+    __shared__ double s_tab[32];
+    exp2_table_init(s_tab);
     pdl_wait();
     const int64_t n = gated_n(A);
     if (n < 0) return;   // the gate reads the same control words in every CTA
@@ -419,202 +662,22 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs A) {
         }
     }
     if (!ok) atomicOr(&ctl->status, ST_TIMEOUT);
-    bar();   // every CTA has read the global histograms
+    // locate: tile and chunk maps of the sorted values (every CTA, its chunk)
+    const uint32_t *sorted = cur == 0 ? A.keys[0] : A.keys[1];
+    const Seeds z = locate_seeds(A);
+    ChunkRec *crec = reinterpret_cast<ChunkRec *>(A.tilebuf);
+    TileRec *rec = reinterpret_cast<TileRec *>(A.tilebuf + 8 * SORT_GMAX);
+    if (skip != 15) locate_tiles<K>(A, sorted, n, t0, t1, z, rec, crec, S.buf, reinterpret_cast<Aff *>(s_hist), s_tab);
+    bar();   // the maps are complete, and every CTA has read the global histograms
     if (c == 0) {
         for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
         if (tid == 0) {
             ctl->sort_cur = cur;
             ctl->sort_solved = skip == 15 ? 1 : 0;
         }
+        if (skip != 15) locate_finish<K>(A, sorted, n, z, rec, crec, S.buf, s_hist, s_tab);
     }
     pdl_trigger();
-}
-
-// --------------------------------------------------------------- locate --
-struct TileRec {
-    double pa, ps;     // tile prefix map  P_end = pa * P_before + ps
-    double qa, qs;     // tile suffix map  Q_first = qa * Q_after + qs
-    double d_out;      // link from the tile's last value to the next value
-    double p_end;      // filled by the last CTA
-    double q_after;    // filled by the last CTA
-    double pad;
-};
-
-__device__ __forceinline__ double sorted_val(const uint32_t *keys, const float *src, int64_t j) {
-    return keys ? (double)desc_key_to_float(keys[j]) : (double)src[j];
-}
-
-__global__ void __launch_bounds__(LB, 1) locate_kernel(SortArgs A, double k, double t, double inv_t) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);                 // LTILE
-    void *scratch = smem + LOC_KEY_WORDS * 4;                                // >= 6 KB
-    __shared__ bool s_last;
-    __shared__ int s_tstar;
-    __shared__ double s_tab[32];
-    exp2_table_init(s_tab);
-
-    pdl_enter();
-    const int64_t n = gated_n(A);
-    if (n < 0) return;
-    Ctl *ctl = A.ctl;
-    if (ctl->sort_solved) return;   // every key equal: solved by the histogram kernel
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int cur = ctl->sort_cur;
-    const uint32_t *keys_cur = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
-    const double s2d = inv_t * LOG2E;
-    __syncthreads();   // s_tab
-    double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
-    if (A.gate == GATE_BAND) {
-        m0 = (double)ctl->c_R;
-        top = (double)ctl->a_R;
-        P_top = ctl->S_R;
-        bot = (double)ctl->a_L;
-        Q_bot = ctl->S_L;
-    }
-    TileRec *rec = reinterpret_cast<TileRec *>(A.tilebuf);
-    const int64_t ntiles = (n + LTILE - 1) / LTILE;
-    auto val = [&](int64_t j) -> double {
-        if (j < 0) return top;
-        if (j >= n) return bot;
-        return sorted_val(keys_cur, A.src, j);
-    };
-    // staged tile: s_keys[spad(i + 1)] holds sorted position tile*LTILE + i for
-    // i = -1 .. cnt (the two halo entries are the neighbours or the seeds)
-    const uint32_t key_top = desc_key((float)top), key_bot = desc_key((float)bot);
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t t0 = tile * LTILE;
-        const int cnt = (int)min((int64_t)LTILE, n - t0);
-        uint32_t kv[LK];
-#pragma unroll
-        for (int u = 0; u < LK; ++u) {   // coalesced, all loads in flight at once
-            const int i = u * LB + tid;
-            kv[u] = 0u;
-            if (i < cnt) kv[u] = keys_cur ? __ldcs(keys_cur + t0 + i) : desc_key(__ldg(A.src + t0 + i));
-        }
-#pragma unroll
-        for (int u = 0; u < LK; ++u) {
-            const int i = u * LB + tid;
-            if (i < cnt) s_keys[spad(i + 1)] = kv[u];
-        }
-        if (tid == 0) {
-            s_keys[spad(0)] = t0 == 0 ? key_top
-                                      : (keys_cur ? keys_cur[t0 - 1] : desc_key(A.src[t0 - 1]));
-            s_keys[spad(cnt + 1)] = t0 + cnt >= n ? key_bot
-                                      : (keys_cur ? keys_cur[t0 + cnt] : desc_key(A.src[t0 + cnt]));
-        }
-        __syncthreads();
-        auto sval = [&](int i) -> double { return (double)desc_key_to_float(s_keys[spad(i + 1)]); };
-        const int l0 = tid * LK;
-        const int l1 = min(l0 + LK, cnt) - 1;
-        Aff mp = aff_id(), mq = aff_id();
-        double d_last = 0.0;
-        if (l0 < cnt) {
-            double cprev = sval(l0 - 1);
-            double c = sval(l0);
-            double dprev = (cprev == CUDART_INF || c == -CUDART_INF) ? 0.0 : link_exp((cprev - c) * s2d, s_tab);
-            for (int j = l0; j <= l1; ++j) {
-                mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
-                const double cn = sval(j + 1);
-                const double d = (c == CUDART_INF || cn == -CUDART_INF) ? 0.0 : link_exp((c - cn) * s2d, s_tab);
-                mq = {mq.a * d, mq.s + mq.a};
-                dprev = d;
-                c = cn;
-            }
-            d_last = dprev;
-        }
-        Aff pe, qe;
-        block_scan_excl_both<LB>(mp, mq, pe, qe, reinterpret_cast<Aff *>(scratch));
-        const int64_t tile_end = min((tile + 1) * LTILE, n) - 1;
-        const int owner = (int)((tile_end - tile * LTILE) / LK);
-        if (tid == owner) {
-            const Aff P = aff_then(pe, mp);
-            rec[tile].pa = P.a;
-            rec[tile].ps = P.s;
-            rec[tile].d_out = d_last;
-        }
-        if (tid == 0) {
-            const Aff Q = aff_then(qe, mq);
-            rec[tile].qa = Q.a;
-            rec[tile].qs = Q.s;
-        }
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&ctl->ticket[6], 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-
-    // ---- last CTA: scan the tile maps, find the crossing tile, re-scan it
-    Aff *sc = reinterpret_cast<Aff *>(scratch);
-    double carry_p = P_top;
-    for (int64_t c0 = 0; c0 < ntiles; c0 += LB) {
-        const int64_t T = c0 + tid;
-        Aff m = aff_id();
-        if (T < ntiles) m = {__ldcg(&rec[T].pa), __ldcg(&rec[T].ps)};
-        Aff pe, qe;
-        block_scan_excl_both<LB>(m, aff_id(), pe, qe, sc);
-        const Aff inc = aff_then(pe, m);
-        if (T < ntiles) rec[T].p_end = fma(inc.a, carry_p, inc.s);
-        // carry = inclusive of the chunk's last tile
-        __shared__ double s_carry;
-        const int64_t lastT = min(c0 + LB, ntiles) - 1;
-        if (T == lastT) s_carry = fma(inc.a, carry_p, inc.s);
-        __syncthreads();
-        carry_p = s_carry;
-        __syncthreads();
-    }
-    __threadfence_block();
-    double carry_q = Q_bot;
-    int best = -1;
-    const int64_t nchunks = (ntiles + LB - 1) / LB;
-    for (int64_t ci = nchunks - 1; ci >= 0; --ci) {
-        const int64_t c0 = ci * LB;
-        const int64_t T = c0 + tid;
-        Aff m = aff_id();
-        if (T < ntiles) m = {__ldcg(&rec[T].qa), __ldcg(&rec[T].qs)};
-        Aff pe, qe;
-        block_scan_excl_both<LB>(aff_id(), m, pe, qe, sc);
-        // qe: maps of tiles T+1 .. chunk end applied (chunk-relative), then carry
-        const double Qa = fma(qe.a, carry_q, qe.s);     // Q at the value after tile T
-        if (T < ntiles) {
-            rec[T].q_after = Qa;
-            const int64_t tend = min((T + 1) * LTILE, n) - 1;
-            const double G = (m0 + (double)(tend + 1)) - 0.5 * __ldcg(&rec[T].p_end) +
-                             0.5 * __ldcg(&rec[T].d_out) * Qa;
-            if (G <= k) best = max(best, (int)T);
-        }
-        __shared__ double s_cq;
-        if (tid == 0) s_cq = fma(aff_then(qe, m).a, carry_q, aff_then(qe, m).s);
-        __syncthreads();
-        carry_q = s_cq;
-        __syncthreads();
-    }
-    best = warp_max_int(best);
-    if (tid == 0) s_tstar = -1;
-    __syncthreads();
-    if (lane == 0) atomicMax(&s_tstar, best);
-    __syncthreads();
-    const int64_t TT = min((int64_t)s_tstar + 1, ntiles - 1);
-    const int64_t t0 = TT * LTILE;
-    const int cnt = (int)min((int64_t)LTILE, n - t0);
-    for (int i = tid; i < cnt; i += LB) {
-        s_keys[spad(i)] = keys_cur ? keys_cur[t0 + i] : desc_key(A.src[t0 + i]);
-    }
-    __syncthreads();
-    const double ptop = TT == 0 ? P_top : __ldcg(&rec[TT - 1].p_end);
-    const double vtop = val(t0 - 1);
-    const double qbot = __ldcg(&rec[TT].q_after);
-    const double vbot = val(t0 + cnt);
-    int64_t js = 0;
-    const double b = block_scan_solve<LB, LK>(s_keys, cnt, k, t, inv_t, m0 + (double)t0, vtop, ptop,
-                                              vbot, qbot, scratch, &js, &ctl->status, s_tab);
-    if (tid == 0) {
-        ctl->b = b;
-        ctl->j_star = t0 + js;
-        if (A.gate == GATE_FALLBACK) ctl->fallback_ran = 1;
-        ctl->ticket[6] = 0u;
-    }
 }
 
 // ------------------------------------------------------------ launchers --
@@ -630,6 +693,14 @@ static int num_sms() {
 }
 
 int sort_grid_max() { return SORT_GMAX; }
+
+// Doubles of locate records a sort of up to cap keys needs: chunk records, then
+// one record per tile (8192-key tiles, or 2048 when cap <= SMALL_SORT).
+int64_t sort_record_doubles(int64_t cap) {
+    const int64_t tiles = cap <= SMALL_SORT ? (cap + TILE_K(RK_SMALL) - 1) / TILE_K(RK_SMALL)
+                                            : (cap + TILE_K(RK_BIG) - 1) / TILE_K(RK_BIG);
+    return 8 * ((int64_t)SORT_GMAX + tiles + 1);
+}
 
 template <int K>
 static cudaError_t launch_sort_k(SortArgs &A, cudaStream_t st) {
@@ -660,19 +731,5 @@ cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) 
     return launch_sort_k<RK_BIG>(A, st);
 }
 
-cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st) {
-    static bool attr = false;
-    const size_t smem = (size_t)LOC_KEY_WORDS * 4 + 16384;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(locate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    int64_t lg = (A.cap + LTILE - 1) / LTILE;
-    if (lg > num_sms()) lg = num_sms();
-    const unsigned grid = (unsigned)lg;
-    return launch_k(locate_kernel, grid, LB, smem, st, A, k, t, 1.0 / t);
-}
 
 }  // namespace lapsum

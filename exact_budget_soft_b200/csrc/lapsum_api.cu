@@ -143,8 +143,7 @@ cudaError_t ws_sort(Workspace *w, int64_t cap) {
     if (e == cudaSuccess) e = grow(w->keys1, w->keys1_n, (size_t)cap);
     if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256);
     if (e == cudaSuccess) e = grow(w->chunkcnt, w->chunkcnt_n, (size_t)4 * 256 * sort_grid_max());
-    const size_t lt = (size_t)((cap + locate_tile() - 1) / locate_tile()) + 1;
-    if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, lt * 8);
+    if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, (size_t)sort_record_doubles(cap));
     return e;
 }
 
@@ -281,12 +280,8 @@ int full_sort_row(Workspace *w, const float *r, int64_t n, double k, double t, i
     LAPSUM_TRY(ws_sort(w, n));
     SortArgs A = sort_args(w, r, n, n, gate, spin_cap, k, t);
     {
-        Launch L("radix_sort", st);
+        Launch L("radix_sort", st);   // sort and locate, one cooperative kernel
         LAPSUM_TRY(launch_radix_sort(A, k, t, st));
-    }
-    {
-        Launch L("locate", st);
-        LAPSUM_TRY(launch_locate(A, k, t, st));
     }
     return LAPSUM_OK;
 }
@@ -425,7 +420,6 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
             SortArgs A = sort_args(w, w->band, 0, Q.band_cap, GATE_BAND, spin_cap, k, t);
             A.round2 = Q.round2;
             { Launch L(r2 ? "widen_band_radix_sort" : "band_radix_sort", st); LAPSUM_TRY(launch_radix_sort(A, k, t, st)); }
-            { Launch L(r2 ? "widen_band_locate" : "band_locate", st); LAPSUM_TRY(launch_locate(A, k, t, st)); }
         }
         if (!Q.fused_cert) { Launch L(r2 ? "widen_certify" : "certify", st); LAPSUM_TRY(launch_certify(Q, st)); }
         return LAPSUM_OK;

@@ -87,8 +87,7 @@ struct SortArgs {
 };
 int radix_tile();
 int sort_grid_max();
-int locate_tile();
+int64_t sort_record_doubles(int64_t cap);
 cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st);
-cudaError_t launch_locate(const SortArgs &A, double k, double t, cudaStream_t st);
 
 }  // namespace lapsum
