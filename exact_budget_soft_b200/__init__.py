@@ -54,7 +54,7 @@ class Stats(C.Structure):
         return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
 
 
-EXPORTS = ["lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats",
+EXPORTS = ["lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats", "lapsum_get_stats_rows",
            "lapsum_strerror", "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read",
            "lapsum_bracket_plan", "lapsum_profile_filter", "lapsum_selftest_math", "lapsum_launch_count"]
 
@@ -69,6 +69,7 @@ def _load() -> C.CDLL:
     lib.lapsum_forward_ex.argtypes = [vp, i64, i64, dbl, dbl, vp, vp, C.POINTER(Options), vp]
     lib.lapsum_backward.argtypes = [vp, vp, vp, i64, i64, dbl, vp, vp]
     lib.lapsum_get_stats.argtypes = [C.POINTER(Stats), vp]
+    lib.lapsum_get_stats_rows.argtypes = [C.POINTER(Stats), i64, C.POINTER(i64), vp]
     lib.lapsum_strerror.restype = C.c_char_p
     lib.lapsum_strerror.argtypes = [C.c_int]
     lib.lapsum_profile_enable.argtypes = [C.c_int]
@@ -168,6 +169,21 @@ def get_stats(stream=None, check: bool = True) -> dict:
     d = st.as_dict()
     d["rc"] = rc
     return d
+
+
+def get_stats_rows(max_rows: int, stream=None, check: bool = True) -> list[dict]:
+    """Per-row diagnostics of the last forward on `stream` (synchronises it)."""
+    arr = (Stats * max(1, int(max_rows)))()
+    got = C.c_int64()
+    rc = lib.lapsum_get_stats_rows(arr, max(1, int(max_rows)), C.byref(got), _stream(stream))
+    if check:
+        _check(rc, "lapsum_get_stats_rows")
+    out = []
+    for i in range(got.value):
+        d = arr[i].as_dict()
+        d["rc"] = rc
+        out.append(d)
+    return out
 
 
 def bracket_plan(n: int, k: float, opts: Options | None = None) -> dict:

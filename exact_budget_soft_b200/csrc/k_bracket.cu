@@ -141,7 +141,8 @@ constexpr int SEL_BINS = 65536;   // select histogram of the top 16 key bits (th
 // This is the operator's own noise kernel, so P(y_j > b) = k/n.  The key kept
 // is the fp32 value rounded toward -inf (monotone, so order statistics commute
 // with it), in the descending-order key space.
-__global__ void __launch_bounds__(256) sample_kernel(BracketParams P) {
+__global__ void __launch_bounds__(256) sample_kernel(BracketParams Pg) {
+    const BracketParams P = at_row(Pg, blockIdx.y);
     __shared__ uint32_t s_h0[256];
     s_h0[threadIdx.x] = 0u;
     pdl_enter();
@@ -217,7 +218,9 @@ constexpr int SEL_BLOCK = 256;
 // that carry one of the prefixes into a global candidate buffer, and the last
 // CTA to finish runs rounds 2 and 3 (bits 15..8, 7..0) over the candidates (or
 // over every key when a prefix holds more than the buffer).
-__global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams P) {
+__global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams Pg) {
+    static_assert(2 * SEL_CAND == SEL_CAND_WORDS, "candidate buffer stride");
+    const BracketParams P = at_row(Pg, blockIdx.y);
     __shared__ uint32_t s_w[SEL_BLOCK / 32];
     __shared__ uint32_t h8[2][256];
     __shared__ uint32_t s_pref[2], s_rank[2], s_bin0[2];
@@ -630,7 +633,8 @@ __device__ __forceinline__ void set_verdict(const BracketParams &P, bool ok, boo
 // the band fits its buffer, both passes agree on every membership count, and
 // every score is finite.
 template <int MODE>
-__global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 3) oob_kernel(BracketParams P) {
+__global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 3) oob_kernel(BracketParams Pg) {
+    const BracketParams P = at_row(Pg, blockIdx.y);
     constexpr bool CERT = MODE == OOB_CERT;
     static_assert(2 * SBLOCK == BULK_F4, "two vectors per thread per chunk");
     extern __shared__ __align__(128) unsigned char dsm[];
@@ -758,8 +762,14 @@ __device__ __forceinline__ float4 p_vec(const float4 v, const XForm &xf) {
 }
 
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
-p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict__ p,
-         double *__restrict__ b_out, Ctl *ctl, double *partials) {
+p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restrict__ p_,
+         double *__restrict__ b_out_, Ctl *ctl_, double *partials_, int64_t pstride) {
+    const int64_t row = blockIdx.y;   // rows of a batch: one grid.y slice each
+    const float *__restrict__ r = r_ + row * n;
+    float *__restrict__ p = p_ + row * n;
+    double *b_out = b_out_ ? b_out_ + row : nullptr;
+    Ctl *ctl = ctl_ + row;
+    double *partials = partials_ + row * pstride;
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[SBLOCK / 32];
     pdl_enter();
@@ -811,8 +821,15 @@ p_kernel(const float *__restrict__ r, int64_t n, double inv_t, float *__restrict
 // raises a flag and vjp_shifted_kernel recomputes the ratio from terms shifted
 // by the running minimum of |x| (the shift cancels in <g,f>/sum f).
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
-vjp_reduce_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
-                  const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
+vjp_reduce_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_,
+                  const float *__restrict__ g_, int64_t n, double inv_t, Ctl *ctl_, double *partials_,
+                  int64_t pstride) {
+    const int64_t row = blockIdx.y;
+    const float *__restrict__ r = r_ + row * n;
+    const float *__restrict__ g = g_ + row * n;
+    const double *b_in = b_in_ + row;
+    Ctl *ctl = ctl_ + row;
+    double *partials = partials_ + row * pstride;
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[2 * (SBLOCK / 32)];
     pdl_enter();
@@ -892,8 +909,15 @@ __device__ __forceinline__ ShiftSumG ss_merge(ShiftSumG a, ShiftSumG b) {
 
 // Rare path: every f_i underflowed in vjp_reduce_kernel.
 __global__ void __launch_bounds__(SBLOCK)
-vjp_shifted_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
-                   const float *__restrict__ g, int64_t n, double inv_t, Ctl *ctl, double *partials) {
+vjp_shifted_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_,
+                   const float *__restrict__ g_, int64_t n, double inv_t, Ctl *ctl_, double *partials_,
+                   int64_t pstride) {
+    const int64_t row = blockIdx.y;
+    const float *__restrict__ r = r_ + row * n;
+    const float *__restrict__ g = g_ + row * n;
+    const double *b_in = b_in_ + row;
+    Ctl *ctl = ctl_ + row;
+    double *partials = partials_ + row * pstride;
     __shared__ ShiftSumG s_w[SBLOCK / 32];
     __shared__ bool s_last;
     pdl_enter();
@@ -936,9 +960,15 @@ vjp_shifted_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
 }
 
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
-vjp_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_in,
-                 const float *__restrict__ g, int64_t n, double inv_t, const Ctl *ctl,
-                 float *__restrict__ grad) {
+vjp_apply_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_,
+                 const float *__restrict__ g_, int64_t n, double inv_t, const Ctl *ctl_,
+                 float *__restrict__ grad_) {
+    const int64_t row = blockIdx.y;
+    const float *__restrict__ r = r_ + row * n;
+    const float *__restrict__ g = g_ + row * n;
+    const double *b_in = b_in_ + row;
+    const Ctl *ctl = ctl_ + row;
+    float *__restrict__ grad = grad_ + row * n;
     extern __shared__ __align__(128) unsigned char dsm[];
     pdl_enter();
     const XForm xf = make_xform(*b_in, inv_t * LOG2E);
@@ -999,12 +1029,21 @@ cudaError_t launch_selftest_math(int which, const double *in, double *out, doubl
     selftest_math_kernel<<<148, 256, 0, st>>>(which, in, out, ref, n);
     return cudaGetLastError();
 }
+// Streaming grids for a batch: the CTAs of one full-device grid shared out
+// among the rows (grid.y = row), at least one each.
+static dim3 row_grid(int per_sm, int64_t rows) {
+    const int64_t g = stream_grid(per_sm) / rows;
+    return dim3((unsigned)(g < 1 ? 1 : g), (unsigned)rows);
+}
+int64_t partial_stride(int64_t rows) {
+    return 24 * (int64_t)row_grid(SBLOCKS_PER_SM, rows).x + 64;
+}
+
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
-    const unsigned blocks = (unsigned)((P.s + 255) / 256);
-    return launch_k(sample_kernel, blocks, 256, 0, st, P);
+    return launch_k(sample_kernel, dim3((unsigned)((P.s + 255) / 256), (unsigned)P.rows), 256, 0, st, P);
 }
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
-    return launch_k(select_kernel, SEL_GRID, SEL_BLOCK, 0, st, P);
+    return launch_k(select_kernel, dim3(SEL_GRID, (unsigned)P.rows), SEL_BLOCK, 0, st, P);
 }
 int select_cand_capacity() { return SEL_CAND; }
 template <typename K>
@@ -1017,35 +1056,40 @@ cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
     static cudaError_t once2 = set_smem(oob_kernel<OOB_STREAM_CERT>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
     if (once2 != cudaSuccess) return once2;
-    if (P.fused_cert) return launch_k(oob_kernel<OOB_STREAM_CERT>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
-    return launch_k(oob_kernel<OOB_STREAM>, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, P);
+    if (P.fused_cert)
+        return launch_k(oob_kernel<OOB_STREAM_CERT>, row_grid(3, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
+    return launch_k(oob_kernel<OOB_STREAM>, row_grid(SBLOCKS_PER_SM, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
     static cudaError_t once = set_smem(oob_kernel<OOB_CERT>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    return launch_k(oob_kernel<OOB_CERT>, stream_grid(3), SBLOCK, bulk_smem_bytes<1>(), st, P);
+    return launch_k(oob_kernel<OOB_CERT>, row_grid(3, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
-cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
+cudaError_t launch_p_pass(const float *r, int64_t rows, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
                           double *partials, cudaStream_t st) {
     static cudaError_t once = set_smem(p_kernel, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
-    return launch_k(p_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<1>(), st, r, n, 1.0 / t, p, b_out, ctl, partials);
+    return launch_k(p_kernel, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<1>(), st, r, n, 1.0 / t, p,
+                    b_out, ctl, partials, partial_stride(rows));
 }
-cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
+cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st) {
     static cudaError_t once = set_smem(vjp_reduce_kernel, bulk_smem_bytes<2>());
     if (once != cudaSuccess) return once;
-    cudaError_t e = launch_k(vjp_reduce_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g, n,
-                             1.0 / t, ctl, partials);
+    const int64_t ps = partial_stride(rows);
+    cudaError_t e = launch_k(vjp_reduce_kernel, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<2>(), st,
+                             r, b, g, n, 1.0 / t, ctl, partials, ps);
     if (e != cudaSuccess) return e;
-    return launch_k(vjp_shifted_kernel, stream_grid() / SBLOCKS_PER_SM, SBLOCK, 0, st, r, b, g, n, 1.0 / t, ctl,
-                    partials);
+    dim3 gs = row_grid(SBLOCKS_PER_SM, rows);
+    gs.x = gs.x / SBLOCKS_PER_SM < 1 ? 1 : gs.x / SBLOCKS_PER_SM;
+    return launch_k(vjp_shifted_kernel, gs, SBLOCK, 0, st, r, b, g, n, 1.0 / t, ctl, partials, ps);
 }
-cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
+cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st) {
     static cudaError_t once = set_smem(vjp_apply_kernel, bulk_smem_bytes<2>());
     if (once != cudaSuccess) return once;
-    return launch_k(vjp_apply_kernel, stream_grid(), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g, n, 1.0 / t, ctl, grad);
+    return launch_k(vjp_apply_kernel, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g, n,
+                    1.0 / t, ctl, grad);
 }
 
 }  // namespace lapsum

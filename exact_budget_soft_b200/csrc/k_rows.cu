@@ -44,7 +44,8 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     int n;
     const float *row;
     double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
-    if (BAND) {
+    if (BAND) {   // one CTA per row of a batch: its band buffer and control block
+        ctl += blockIdx.x;
         if (round2 && !ctl->widened) return;   // the widening round did not start
         unsigned long long cb = ctl->c_band;
         if (cb > (unsigned long long)band_cap) {
@@ -64,7 +65,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
         if (band_lo > 0 && cb <= (unsigned long long)band_lo) return;   // a smaller variant takes it
         if (cb > (unsigned long long)C::CAP) return;   // the device-wide sort takes it
         n = (int)cb;
-        row = scores;
+        row = scores + (int64_t)blockIdx.x * band_cap;
         m0 = (double)ctl->c_R;
         top = (double)ctl->a_R;
         P_top = ctl->S_R;
@@ -296,12 +297,12 @@ cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, d
 // Two variants, each gated on the band size the streaming pass counted: bands
 // of up to 4096 scores (and tied or empty bands) in a 256-thread CTA, larger
 // ones up to 32768 in a 1024-thread CTA.
-cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
-                                 int32_t round2, cudaStream_t st) {
+cudaError_t launch_rowsolve_band(const float *band, int64_t rows, double k, double t, Ctl *ctl,
+                                 int64_t band_cap, int32_t round2, cudaStream_t st) {
     cudaError_t e =
-        launch_rowsolve<256, 16, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, round2, st);
+        launch_rowsolve<256, 16, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, round2, st);
     if (e != cudaSuccess) return e;
-    return launch_rowsolve<1024, 32, true>(band, 1, 0, k, t, nullptr, nullptr, ctl, band_cap,
+    return launch_rowsolve<1024, 32, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap,
                                            RowCfg<256, 16>::CAP, round2, st);
 }
 

@@ -108,6 +108,7 @@ struct Workspace {
     unsigned long long *hist = nullptr; size_t hist_n = 0;
     uint32_t *chunkcnt = nullptr; size_t chunkcnt_n = 0;
     double *tilebuf = nullptr;        size_t tilebuf_n = 0;
+    int64_t rows = 1;                 // rows of the last solve (their control blocks hold its stats)
 
     void release() {
         cudaFree(ctl); cudaFree(partials); cudaFree(skeys); cudaFree(hist1); cudaFree(selcand); cudaFree(band);
@@ -132,9 +133,10 @@ Workspace *get_ws(cudaStream_t st) {
     return w;
 }
 
-cudaError_t ws_base(Workspace *w) {
-    cudaError_t e = grow(w->ctl, w->ctl_n, 1);
-    if (e == cudaSuccess) e = grow(w->partials, w->partials_n, (size_t)stream_grid() * 24 + 64);
+// Control blocks and per-block partials for a batch of rows.
+cudaError_t ws_base(Workspace *w, int64_t rows) {
+    cudaError_t e = grow(w->ctl, w->ctl_n, (size_t)rows);
+    if (e == cudaSuccess) e = grow(w->partials, w->partials_n, (size_t)(rows * partial_stride(rows)));
     return e;
 }
 
@@ -164,6 +166,8 @@ SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32
     A.gate = gate;
     A.spin_cap = spin_cap;
     A.small_cap = rowsolve_capacity();
+    A.rows = 1;
+    A.src_stride = 0;
     return A;
 }
 
@@ -274,11 +278,14 @@ int check_args(const float *scores, int64_t rows, int64_t n, double k, double t)
     return LAPSUM_OK;
 }
 
-// Full sort of one long row on the device (also the certification fallback).
-int full_sort_row(Workspace *w, const float *r, int64_t n, double k, double t, int32_t gate,
-                  int32_t spin_cap, cudaStream_t st) {
+// Full sort of long rows on the device (also the certification fallback): one
+// cooperative kernel walks the rows, each gated by its own control block.
+int full_sort_rows(Workspace *w, const float *r, int64_t rows, int64_t n, double k, double t, int32_t gate,
+                   int32_t spin_cap, cudaStream_t st) {
     LAPSUM_TRY(ws_sort(w, n));
     SortArgs A = sort_args(w, r, n, n, gate, spin_cap, k, t);
+    A.rows = rows;
+    A.src_stride = n;
     {
         Launch L("radix_sort", st);   // sort and locate, one cooperative kernel
         LAPSUM_TRY(launch_radix_sort(A, k, t, st));
@@ -320,19 +327,13 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
     const int32_t spin_cap = opt.spin_cap ? opt.spin_cap : (1 << 20);
     Workspace *w = get_ws(st);
-    LAPSUM_TRY(ws_base(w));
 
     int path = opt.force_path;
-    if (path == LAPSUM_PATH_AUTO)
-        path = (rows == 1 && n >= (int64_t(1) << 20)) ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
-    if (path == LAPSUM_PATH_BRACKET && rows != 1) {
-        // one bracket per row: rows are solved one after another
-        for (int64_t r = 0; r < rows; ++r) {
-            rc = lapsum_forward_ex(scores + r * n, 1, n, k, t, p_out + r * n, b_out + r, &opt, stream_in);
-            if (rc) return rc;
-        }
-        return LAPSUM_OK;
-    }
+    if (path == LAPSUM_PATH_AUTO)   // long rows bracket, one or many (a batch shares the kernels)
+        path = n >= (int64_t(1) << 20) ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
+    if (path == LAPSUM_PATH_BRACKET && rows > 65535) return LAPSUM_ERR_ARG;   // grid.y holds the row
+    w->rows = path == LAPSUM_PATH_FULLSORT && n <= rowsolve_capacity() ? 1 : rows;
+    LAPSUM_TRY(ws_base(w, w->rows));
 
     if (path == LAPSUM_PATH_FULLSORT) {
         if (n <= rowsolve_capacity()) {
@@ -341,14 +342,11 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
             LAPSUM_TRY(launch_rowsolve_rows(scores, rows, n, k, t, p_out, b_out, w->ctl, st));
             return LAPSUM_OK;
         }
-        for (int64_t r = 0; r < rows; ++r) {
-            const float *row = scores + r * n;
-            LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
-            rc = full_sort_row(w, row, n, k, t, GATE_ALWAYS, spin_cap, st);
-            if (rc) return rc;
-            Launch L("p_pass", st);
-            LAPSUM_TRY(launch_p_pass(row, n, t, p_out + r * n, b_out + r, w->ctl, w->partials, st));
-        }
+        LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl) * (size_t)rows, st));
+        rc = full_sort_rows(w, scores, rows, n, k, t, GATE_ALWAYS, spin_cap, st);
+        if (rc) return rc;
+        Launch L("p_pass", st);
+        LAPSUM_TRY(launch_p_pass(scores, rows, n, t, p_out, b_out, w->ctl, w->partials, st));
         return LAPSUM_OK;
     }
 
@@ -356,6 +354,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     BracketParams P{};
     P.r = scores;
     P.n = n;
+    P.rows = rows;
     P.k = k;
     P.t = t;
     P.inv_t = 1.0 / t;
@@ -391,20 +390,22 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         P2.band_cap = std::min<int64_t>(cap2, n);
     }
     const int64_t band_buf = std::max(band_cap, opt.widen ? P2.band_cap : int64_t(0));
-    LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)s));
-    LAPSUM_TRY(grow(w->hist1, w->hist1_n, 65536 + 256));
-    LAPSUM_TRY(grow(w->selcand, w->selcand_n, (size_t)2 * select_cand_capacity()));
-    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)band_buf));
-    LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort the whole row
+    const size_t R = (size_t)rows;
+    LAPSUM_TRY(grow(w->skeys, w->skeys_n, R * (size_t)s));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, R * (size_t)HIST_WORDS));
+    LAPSUM_TRY(grow(w->selcand, w->selcand_n, R * (size_t)SEL_CAND_WORDS));
+    LAPSUM_TRY(grow(w->band, w->band_n, R * (size_t)band_buf));
+    LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort a whole row (rows one after another)
 
     P2.band = P.band = w->band;
     P2.keys = P.keys = w->skeys;
     P2.hist1 = P.hist1 = w->hist1;
     P2.cand = P.cand = w->selcand;
     P2.partials = P.partials = w->partials;
+    P2.part_stride = P.part_stride = partial_stride(rows);
     P2.ctl = P.ctl = w->ctl;
 
-    LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl), st));
+    LAPSUM_TRY(cudaMemsetAsync(w->ctl, 0, sizeof(Ctl) * R, st));
     // one bracketing round: sample, select, stream, band solve, certification
     auto bracket_round = [&](const BracketParams &Q) -> int {
         const bool r2 = Q.round2 != 0;   // profiling names are literals (the profiler keeps the pointer)
@@ -414,11 +415,13 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         {
             Launch L(r2 ? "widen_band_rowsolve" : "band_rowsolve", st);
             ++g_launches;   // two size-gated variants
-            LAPSUM_TRY(launch_rowsolve_band(w->band, k, t, w->ctl, Q.band_cap, Q.round2, st));
+            LAPSUM_TRY(launch_rowsolve_band(w->band, rows, k, t, w->ctl, Q.band_cap, Q.round2, st));
         }
         if (Q.band_cap > rowsolve_capacity()) {
             SortArgs A = sort_args(w, w->band, 0, Q.band_cap, GATE_BAND, spin_cap, k, t);
             A.round2 = Q.round2;
+            A.rows = rows;
+            A.src_stride = Q.band_cap;
             { Launch L(r2 ? "widen_band_radix_sort" : "band_radix_sort", st); LAPSUM_TRY(launch_radix_sort(A, k, t, st)); }
         }
         if (!Q.fused_cert) { Launch L(r2 ? "widen_certify" : "certify", st); LAPSUM_TRY(launch_certify(Q, st)); }
@@ -430,9 +433,9 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         rc = bracket_round(P2);
         if (rc) return rc;
     }
-    rc = full_sort_row(w, scores, n, k, t, GATE_FALLBACK, spin_cap, st);
+    rc = full_sort_rows(w, scores, rows, n, k, t, GATE_FALLBACK, spin_cap, st);
     if (rc) return rc;
-    { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, n, t, p_out, b_out, w->ctl, w->partials, st)); }
+    { Launch L("p_pass", st); LAPSUM_TRY(launch_p_pass(scores, rows, n, t, p_out, b_out, w->ctl, w->partials, st)); }
     return LAPSUM_OK;
 }
 
@@ -474,27 +477,21 @@ int lapsum_backward(const float *scores, const double *b, const float *g, int64_
         return LAPSUM_ERR_ARG;
     if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
-    if (rows > 1 || n <= 65536) {
+    if (n <= 65536 || rows > 65535) {   // short rows: one CTA per row
         Launch L("rowvjp", st);
         LAPSUM_TRY(launch_rowvjp(scores, b, g, rows, n, t, grad_out, st));
         return LAPSUM_OK;
     }
+    // long rows: the streaming passes, the rows of a batch sharing the grid
     Workspace *w = get_ws(st);
-    LAPSUM_TRY(ws_base(w));
-    { Launch L("vjp_reduce", st); LAPSUM_TRY(launch_vjp_reduce(scores, b, g, n, t, w->ctl, w->partials, st)); }
-    { Launch L("vjp_apply", st); LAPSUM_TRY(launch_vjp_apply(scores, b, g, n, t, w->ctl, grad_out, st)); }
+    LAPSUM_TRY(ws_base(w, rows));
+    { Launch L("vjp_reduce", st); LAPSUM_TRY(launch_vjp_reduce(scores, b, g, rows, n, t, w->ctl, w->partials, st)); }
+    { Launch L("vjp_apply", st); LAPSUM_TRY(launch_vjp_apply(scores, b, g, rows, n, t, w->ctl, grad_out, st)); }
     return LAPSUM_OK;
 }
 
-int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream_in) {
-    if (!out) return LAPSUM_ERR_ARG;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
-    Workspace *w = get_ws(st);
+static void fill_stats(const Ctl &c, lapsum_stats *out) {
     std::memset(out, 0, sizeof(*out));
-    if (!w->ctl) return LAPSUM_OK;
-    LAPSUM_TRY(cudaStreamSynchronize(st));
-    Ctl c;
-    LAPSUM_TRY(cudaMemcpy(&c, w->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost));
     out->path = c.path == 2 ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
     out->verdict = c.path == 2 ? c.verdict : -1;
     out->status = c.status;
@@ -515,10 +512,41 @@ int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream_in) {
     out->sum_p = c.sum_p;
     out->j_star = c.j_star;
     out->widened = c.widened;
+}
+
+static int stats_rc(const Ctl &c) {
     if (c.status & ST_NONFINITE) return LAPSUM_ERR_NONFINITE;
     if (c.status & ST_TIMEOUT) return LAPSUM_ERR_DEVICE_TIMEOUT;
     if ((c.status & ST_NO_ROOT) && !(c.path == 2 && c.fallback_ran)) return LAPSUM_ERR_NO_ROOT;
     return LAPSUM_OK;
+}
+
+int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream_in) {
+    if (!out) return LAPSUM_ERR_ARG;
+    int64_t got = 0;
+    return lapsum_get_stats_rows(out, 1, &got, stream_in);
+}
+
+int lapsum_get_stats_rows(lapsum_stats *out, int64_t max_rows, int64_t *rows_out,
+                          struct CUstream_st *stream_in) {
+    if (!out || !rows_out || max_rows < 1) return LAPSUM_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    Workspace *w = get_ws(st);
+    *rows_out = 0;
+    std::memset(out, 0, sizeof(*out) * (size_t)max_rows);
+    if (!w->ctl) return LAPSUM_OK;
+    LAPSUM_TRY(cudaStreamSynchronize(st));
+    const int64_t rows = std::min<int64_t>(w->rows, (int64_t)w->ctl_n);
+    std::vector<Ctl> c((size_t)rows);
+    LAPSUM_TRY(cudaMemcpy(c.data(), w->ctl, sizeof(Ctl) * (size_t)rows, cudaMemcpyDeviceToHost));
+    int rc = LAPSUM_OK;
+    for (int64_t i = 0; i < rows; ++i) {   // the first error over all rows of the last solve
+        const int ri = stats_rc(c[(size_t)i]);
+        if (rc == LAPSUM_OK) rc = ri;
+        if (i < max_rows) fill_stats(c[(size_t)i], out + i);
+    }
+    *rows_out = std::min(rows, max_rows);
+    return rc;
 }
 
 int lapsum_release(void) {

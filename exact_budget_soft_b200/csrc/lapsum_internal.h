@@ -51,26 +51,48 @@ struct Ctl {
 };
 
 // Kernel-facing parameters of a bracketing solve.
+// Kernel-facing parameters of a bracketing solve of `rows` rows (grid.y = row).
+// Pointers are the bases of row 0; every per-row array has a fixed row stride
+// (see at_row), so a kernel first takes its row's view.
 struct BracketParams {
-    const float *r;
+    const float *r;           // scores [rows][n]
     int64_t n;
+    int64_t rows;
     double k, t, inv_t;
     uint64_t seed;
-    int64_t row;
+    int64_t row;              // the row of this view (the sample's Philox counter word)
     int64_t s;
     int64_t jR, jL;
     int64_t band_cap;
-    float *band;              // band buffer [band_cap]
-    uint32_t *keys;           // sample keys [s]
-    uint32_t *hist1;          // [65536 + 256] select histograms of the top 16 and top 8 key
-                              //   bits (zero between solves: the streaming pass clears them)
-    uint32_t *cand;           // [2][SEL_CAND] keys under each target's 16-bit prefix
-    double *partials;         // per-block partials
-    Ctl *ctl;
+    float *band;              // band buffers [rows][band_cap]
+    uint32_t *keys;           // sample keys [rows][s]
+    uint32_t *hist1;          // [rows][HIST_WORDS] select histograms of the top 16 and top 8
+                              //   key bits (zero between solves: the streaming pass clears them)
+    uint32_t *cand;           // [rows][2][SEL_CAND] keys under each target's 16-bit prefix
+    double *partials;         // per-block partials [rows][part_stride]
+    int64_t part_stride;
+    Ctl *ctl;                 // control blocks [rows]
     int32_t spin_cap;
     int32_t fused_cert;       // certification folded into the streaming pass
     int32_t widen;            // a widening round follows a missed bracket
     int32_t round2;           // this launch belongs to the widening round
 };
+
+constexpr int64_t HIST_WORDS = 65536 + 256;
+constexpr int64_t SEL_CAND_WORDS = 2 * 8192;
+
+// The view of one row: every per-row pointer moved to that row.
+__host__ __device__ inline BracketParams at_row(const BracketParams &P, int64_t row) {
+    BracketParams Q = P;
+    Q.row = row;
+    Q.r = P.r + row * P.n;
+    Q.band = P.band + row * P.band_cap;
+    Q.keys = P.keys + row * P.s;
+    Q.hist1 = P.hist1 + row * HIST_WORDS;
+    Q.cand = P.cand + row * SEL_CAND_WORDS;
+    Q.partials = P.partials + row * P.part_stride;
+    Q.ctl = P.ctl + row;
+    return Q;
+}
 
 }  // namespace lapsum

@@ -47,31 +47,34 @@ inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, si
 int rowsolve_capacity();
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st);
-cudaError_t launch_rowsolve_band(const float *band, double k, double t, Ctl *ctl, int64_t band_cap,
-                                 int32_t round2, cudaStream_t st);
+cudaError_t launch_rowsolve_band(const float *band, int64_t rows, double k, double t, Ctl *ctl,
+                                 int64_t band_cap, int32_t round2, cudaStream_t st);
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
                           int64_t n, double t, float *grad, cudaStream_t st);
 
 // bracketing pipeline and streaming passes (k_bracket.cu)
 int stream_grid();
+int64_t partial_stride(int64_t rows);   // doubles of per-block partials per row
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st);
 int select_cand_capacity();
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st);
-cudaError_t launch_p_pass(const float *r, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
+cudaError_t launch_p_pass(const float *r, int64_t rows, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
                           double *partials, cudaStream_t st);
-cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t n, double t,
+cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st);
 cudaError_t launch_selftest_math(int which, const double *in, double *out, double *ref, int64_t n,
                                 cudaStream_t st);
-cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t n, double t,
+cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st);
 
 // device-wide radix sort + locate-scan (k_radix.cu)
 enum Gate : int32_t { GATE_ALWAYS = 0, GATE_BAND = 1, GATE_FALLBACK = 2 };
 struct SortArgs {
-    const float *src;          // fp32 scores (keys made on the fly)
+    const float *src;          // fp32 scores (keys made on the fly) of row 0
+    int64_t src_stride;        // floats from one row's source to the next
+    int64_t rows;              // rows the kernel walks, one after another (each gated)
     int64_t n_host;            // element count when gate != GATE_BAND
     int64_t cap;               // upper bound of the element count (grid sizing)
     uint32_t *keys[2];         // ping-pong key buffers [cap]

@@ -26,12 +26,12 @@
  *    library's own workspace.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point synchronises the host except
- *    lapsum_get_stats / lapsum_profile_read (documented) and the first call on
+ *    lapsum_get_stats* / lapsum_profile_read (documented) and the first call on
  *    a stream, which may allocate the workspace with cudaMalloc.
  *  - Return value: LAPSUM_OK (0) or a negative LAPSUM_ERR_* code.  Argument
  *    errors are detected on the host before anything is enqueued.  Errors
- *    found on the device (non-finite scores, a look-back wait that gave up)
- *    are reported by lapsum_get_stats.
+ *    found on the device (non-finite scores, a grid-barrier wait that gave
+ *    up) are reported by lapsum_get_stats / lapsum_get_stats_rows.
  *  - The library keeps one workspace per (device, stream); calls on the same
  *    stream are ordered, calls on different streams use different
  *    workspaces.  Not thread-safe for concurrent calls on the same stream.
@@ -81,8 +81,11 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
  *               max(65536, 4 n (jL - jR + 2)/s), at most n).  A larger band
  *               fails certification and takes the full-sort fallback.
  *   spin_cap    polls before an inter-block wait gives up (default 2^20).
- *   force_path  LAPSUM_PATH_* (default AUTO: bracketing when rows == 1 and
- *               n >= 2^20, else full sort).
+ *   force_path  LAPSUM_PATH_* (default AUTO: bracketing when n >= 2^20, else
+ *               full sort).  Bracketing solves the rows of a batch together:
+ *               every kernel takes one slice of its grid per row (rows <=
+ *               65535), each row with its own sample (Philox counter word =
+ *               row), bracket, band, certification and fallback.
  *   certify     LAPSUM_CERTIFY_PASS (default): the certification is its own
  *               linear pass over the row (the abstract's "one additional linear
  *               pass"); LAPSUM_CERTIFY_FUSED: the streaming pass also adds the
@@ -114,8 +117,9 @@ typedef struct {
 } lapsum_options;
 
 /*
- * Diagnostics of the last lapsum_forward* call on a stream (row 0 for the
- * batched full-sort path).  Read with lapsum_get_stats.
+ * Diagnostics of one row of the last lapsum_forward* call on a stream: row 0
+ * with lapsum_get_stats, every row with lapsum_get_stats_rows (the one-CTA
+ * full-sort path of rows <= 32768 scores keeps row 0's only).
  *   path      LAPSUM_PATH_FULLSORT or LAPSUM_PATH_BRACKET
  *   verdict   bracketing: 1 certified, 0 not certified (fallback ran); -1 n/a
  *   status    device error bits: 1 non-finite score, 2 wait timeout,
@@ -173,6 +177,16 @@ LAPSUM_API int lapsum_backward(const float *scores_dev, const double *b_dev, con
 /* Copies the last forward's diagnostics to *out. Synchronises `stream`.
  * Returns the device error as a LAPSUM_ERR_* code (LAPSUM_OK if none). */
 LAPSUM_API int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream);
+
+/*
+ * Per-row diagnostics of the last lapsum_forward* call on a stream: fills
+ * out[0 .. min(rows, max_rows)) (out: host array of max_rows entries), sets
+ * *rows_out to the number filled.  Synchronises the stream.  Returns the first
+ * device-found error over all rows (as lapsum_get_stats does for row 0), else 0;
+ * LAPSUM_ERR_ARG for a null pointer or max_rows < 1.
+ */
+LAPSUM_API int lapsum_get_stats_rows(lapsum_stats *out, int64_t max_rows, int64_t *rows_out,
+                                     struct CUstream_st *stream);
 
 /* Static string for a return code. */
 LAPSUM_API const char *lapsum_strerror(int code);

@@ -364,3 +364,86 @@ def test_widening_skips_band_overflow(L, orc):
     p, b, st, grad = run(L, r, k, t, opts=L.options(band_cap=64, widen=1), g_np=g)
     assert st["widened"] == 0 and st["verdict"] == 0 and st["fallback"] == 1
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+# ------------------------------------------------ batched bracketing (NEXT-3) --
+def run_rows(L, r_np, k, t, opts=None, g_np=None):
+    r = torch.from_numpy(np.ascontiguousarray(r_np)).cuda()
+    p, b = L.forward(r, k, t, opts=opts)
+    sts = L.get_stats_rows(r.shape[0], check=False)
+    grad = None
+    if g_np is not None:
+        g = torch.from_numpy(np.ascontiguousarray(g_np)).cuda()
+        grad = L.backward(r, b, g, t).cpu().numpy()
+    torch.cuda.synchronize()
+    return p.cpu().numpy(), b.cpu().numpy(), sts, grad
+
+
+def expected_row(orc, r, k, t, seed, s, delta, row, widen=False):
+    """The oracle's bracket of one row of a batch (its own Philox counter word),
+    the certification outcome, and -- with widening -- the second round."""
+    br = orc.bracket(r, k, t, seed, s, delta, row=row)
+    c = orc.certify(r, k, t, br["a_L"], br["a_R"], band_cap=10**12)
+    out = {"br": br, "cert": c, "widened": 0}
+    if widen and c["verdict"] == 0:
+        jR2, jL2 = orc.widen_ranks(s, k / r.size, delta)
+        b2 = orc.bracket_at_ranks(r, t, seed, s, jR2, jL2, row=row)
+        if c["G_aR"] >= k:
+            nb = {"a_L": br["a_R"], "a_R": b2["a_R"], "jL": br["jR"], "jR": jR2}
+        else:
+            nb = {"a_L": b2["a_L"], "a_R": br["a_L"], "jL": jL2, "jR": br["jL"]}
+        out.update(br=nb, cert=orc.certify(r, k, t, nb["a_L"], nb["a_R"], band_cap=10**12), widened=1)
+    return out
+
+
+@pytest.mark.parametrize("certify", [0, 1])
+def test_batched_bracketing_rows(L, orc, certify):
+    # three rows of a ragged length (rows start off 16-byte boundaries): one
+    # launch sequence, every row bracketed, certified and solved on its own
+    rows, n = 3, (1 << 20) + 123
+    r, g = W.small_case("laplace", rows, n, seed=13)
+    k, t = 2000.0, 0.05
+    p, b, sts, grad = run_rows(L, r, k, t, opts=L.options(certify=certify), g_np=g)
+    plan = L.bracket_plan(n, k)
+    assert len(sts) == rows
+    for i in range(rows):
+        st = sts[i]
+        assert st["rc"] == 0 and st["path"] == 2 and st["verdict"] == 1 and st["fallback"] == 0
+        e = expected_row(orc, r[i], k, t, 0, plan["s"], 1e-6, i)
+        assert np.float32(st["a_L"]) == e["br"]["a_L"] and np.float32(st["a_R"]) == e["br"]["a_R"]
+        assert (st["c_L"], st["c_band"], st["c_R"]) == (e["cert"]["c_L"], e["cert"]["c_band"], e["cert"]["c_R"])
+        check_row(orc, r[i], g[i], k, t, p[i], b[i], grad[i])
+
+
+@pytest.mark.parametrize("widen", [0, 1])
+def test_batched_rows_with_misses(L, orc, widen):
+    # a weak bracket (s = 256, delta = 0.5) misses on some rows: each row's
+    # verdict, widening and fallback follow that row's own certification
+    # (Philox seed 10: by the oracle, rows 0 and 4 miss; widening recovers row 0
+    # and row 4 misses again)
+    rows, n = 6, 1 << 20
+    r, g = W.small_case("normal", rows, n, seed=14)
+    k, t, s, delta, seed = 5000.0, 0.05, 256, 0.5, 10
+    p, b, sts, grad = run_rows(L, r, k, t, opts=L.options(seed=seed, sample_size=s, delta=delta, widen=widen),
+                               g_np=g)
+    outcomes = set()
+    for i in range(rows):
+        st = sts[i]
+        e = expected_row(orc, r[i], k, t, seed, s, delta, i, widen=bool(widen))
+        assert st["rc"] == 0 and st["widened"] == e["widened"]
+        assert np.float32(st["a_L"]) == e["br"]["a_L"] and np.float32(st["a_R"]) == e["br"]["a_R"]
+        assert st["verdict"] == e["cert"]["verdict"] and st["fallback"] == 1 - e["cert"]["verdict"]
+        outcomes.add((st["verdict"], st["widened"]))
+        check_row(orc, r[i], g[i], k, t, p[i], b[i], grad[i])
+    assert len(outcomes) > 1   # the batch mixes rows that pass and rows that do not
+
+
+def test_batched_rows_all_fall_back(L, orc):
+    # every row's band overflows: the cooperative sort walks all rows
+    rows, n = 3, (1 << 20) + 5
+    r, g = W.small_case("normal", rows, n, seed=15)
+    k, t = 3000.0, 0.05
+    p, b, sts, grad = run_rows(L, r, k, t, opts=L.options(band_cap=64), g_np=g)
+    for i in range(rows):
+        assert sts[i]["verdict"] == 0 and sts[i]["fallback"] == 1 and sts[i]["rc"] == 0
+        check_row(orc, r[i], g[i], k, t, p[i], b[i], grad[i])
