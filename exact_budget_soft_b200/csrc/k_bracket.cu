@@ -466,28 +466,39 @@ __device__ __forceinline__ void band_push(float x, bool inb, float *band, unsign
 // certification terms; the verdict comes out of the same pass).
 enum : int { OOB_STREAM = 0, OOB_CERT = 1, OOB_STREAM_CERT = 2 };
 
-// General path, one score.  Returns "in the band" (streaming modes).
+// General path, one score.  Returns "in the band" (streaming modes).  Written
+// to keep a warp of mixed scores together: every out-of-band score forms its
+// fp32 tail term, and the masks pick where it goes; only the rare scores near
+// an end (fp64 term) and band scores (certification terms) branch.
 template <int MODE>
 __device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobAcc &a) {
     constexpr bool CERT = MODE == OOB_CERT;
     if (!valid) return false;
     a.bad |= !(fabsf(x) < CUDART_INF_F);
-    if (x >= E.aR) {
-        if (CERT) { a.cL += 1; a.cR += 1; } else { a.cR += 1; }
-        tier2(x, E.aR, (double)x, E.daR, E, a.SR, a.SR2);
-        return false;
+    const bool above = x >= E.aR, below = x < E.aL;
+    const bool inb = !above && !below && x == x;
+    if (CERT) {
+        a.cR += above;
+        a.cB += below;
+        a.cL += above || inb;
+    } else {
+        a.cR += above;
+        a.cL += below;
     }
-    if (x < E.aL) {
-        if (CERT) a.cB += 1; else a.cL += 1;
-        tier2(E.aL, x, E.daL, (double)x, E, a.SL, a.SL2);
-        return false;
+    const float z2 = (above ? x - E.aR : E.aL - x) * E.s2;   // tail exponent in base-2 units
+    const bool near = (above || below) && z2 <= NEAR2;
+    const float f = ex2_ftz(-z2);
+    a.SR2 += (above && !near) ? f : 0.f;
+    a.SL2 += (below && !near) ? f : 0.f;
+    if (near) {
+        if (above) a.SR += exp2_neg(((double)x - E.daR) * E.s2d, E.tab);
+        else       a.SL += exp2_neg((E.daL - (double)x) * E.s2d, E.tab);
     }
-    if (MODE != OOB_STREAM && x == x) {
-        if (CERT) a.cL += 1;
+    if (MODE != OOB_STREAM && inb) {
         tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
         tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
     }
-    return x == x;
+    return inb;
 }
 
 // One float4 of the pass; `ok` false for padding lanes (whole warps iterate).
@@ -610,6 +621,115 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
     }
 }
 
+// ---- one chunk per thread (two float4s) at a time --------------------------
+// Sparse band scores of a streaming pass go to a queue in shared memory, written
+// out with one global atomic per CTA at the end (a warp-aggregated global push
+// only if the queue fills).
+constexpr int BQ = 4096;
+
+__device__ __forceinline__ float pick8(const float4 &u, const float4 &w, int i) {
+    const float lo = (i & 2) ? ((i & 1) ? u.w : u.z) : ((i & 1) ? u.y : u.x);
+    const float hi = (i & 2) ? ((i & 1) ? w.w : w.z) : ((i & 1) ? w.y : w.x);
+    return (i & 4) ? hi : lo;
+}
+
+// The common part of the general path for one score: counts and the fp32 tail
+// term; a score near an end (fp64 term) or in the band only sets its bit.
+template <int MODE>
+__device__ __forceinline__ void oob_cheap(float x, int bit, const Ends &E, OobAcc &a, uint32_t &near_m,
+                                          uint32_t &band_m) {
+    constexpr bool CERT = MODE == OOB_CERT;
+    a.bad |= !(fabsf(x) < CUDART_INF_F);
+    const bool above = x >= E.aR, below = x < E.aL;
+    const bool inb = !above && !below && x == x;
+    if (CERT) {
+        a.cR += above;
+        a.cB += below;
+        a.cL += above || inb;
+    } else {
+        a.cR += above;
+        a.cL += below;
+    }
+    const float z2 = (above ? x - E.aR : E.aL - x) * E.s2;
+    const bool near = (above || below) && z2 <= NEAR2;
+    const float f = ex2_ftz(-z2);
+    a.SR2 += (above && !near) ? f : 0.f;
+    a.SL2 += (below && !near) ? f : 0.f;
+    near_m |= near ? (1u << bit) : 0u;
+    band_m |= inb ? (1u << bit) : 0u;
+}
+
+template <int MODE>
+__device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, const Ends &E, OobAcc &a,
+                                          const BracketParams &P, unsigned long long cap, int lane,
+                                          float *s_bq, unsigned *s_bn) {
+    constexpr bool CERT = MODE == OOB_CERT;
+    constexpr bool BANDTERMS = MODE != OOB_STREAM;
+    const float mx = max_nan(max_nan(max_nan(v0.x, v0.y), max_nan(v0.z, v0.w)),
+                             max_nan(max_nan(v1.x, v1.y), max_nan(v1.z, v1.w)));
+    const float mn = fminf(fminf(fminf(v0.x, v0.y), fminf(v0.z, v0.w)), fminf(fminf(v1.x, v1.y), fminf(v1.z, v1.w)));
+    const bool fin = mn > -CUDART_INF_F && mx < CUDART_INF_F;
+    // a whole warp on one side (sorted or clustered scores): the float4 fast paths
+    if (__all_sync(FULL, mx < E.aL && fin) || __all_sync(FULL, mn >= E.aR && fin) ||
+        __all_sync(FULL, mn >= E.aL && mx < E.aR && fin)) {
+        oob_vec<MODE>(v0, true, E, a, P, cap, lane);
+        oob_vec<MODE>(v1, true, E, a, P, cap, lane);
+        return;
+    }
+    // general path: the cheap part for all eight, then the marked ones
+    uint32_t near_m = 0, band_m = 0;
+    oob_cheap<MODE>(v0.x, 0, E, a, near_m, band_m);
+    oob_cheap<MODE>(v0.y, 1, E, a, near_m, band_m);
+    oob_cheap<MODE>(v0.z, 2, E, a, near_m, band_m);
+    oob_cheap<MODE>(v0.w, 3, E, a, near_m, band_m);
+    oob_cheap<MODE>(v1.x, 4, E, a, near_m, band_m);
+    oob_cheap<MODE>(v1.y, 5, E, a, near_m, band_m);
+    oob_cheap<MODE>(v1.z, 6, E, a, near_m, band_m);
+    oob_cheap<MODE>(v1.w, 7, E, a, near_m, band_m);
+    // fp64 tail terms of scores near an end: each warp loops as often as its
+    // busiest lane has such scores
+    while (__any_sync(FULL, near_m != 0)) {
+        if (near_m) {
+            const float x = pick8(v0, v1, __ffs(near_m) - 1);
+            near_m &= near_m - 1;
+            if (x >= E.aR) a.SR += exp2_neg(((double)x - E.daR) * E.s2d, E.tab);
+            else           a.SL += exp2_neg((E.daL - (double)x) * E.s2d, E.tab);
+        }
+    }
+    if (!__any_sync(FULL, band_m != 0)) return;
+    if (BANDTERMS) {   // the band scores' two certification terms
+        uint32_t m = band_m;
+        while (__any_sync(FULL, m != 0)) {
+            if (m) {
+                const float x = pick8(v0, v1, __ffs(m) - 1);
+                m &= m - 1;
+                tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
+                tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
+            }
+        }
+    }
+    if (!CERT) {   // the band scores into the CTA's queue
+        const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool inb = (band_m >> i) & 1u;
+            const unsigned m = __ballot_sync(FULL, inb);
+            if (!m) continue;
+            const int leader = __ffs(m) - 1;
+            unsigned base = 0;
+            if (lane == leader) base = atomicAdd(s_bn, (unsigned)__popc(m));
+            const unsigned slot = __shfl_sync(FULL, base, leader) + __popc(m & lt);
+            const float x = pick8(v0, v1, i);
+            if (inb) {
+                a.kmax = max(a.kmax, desc_key(x));
+                a.kinv = max(a.kinv, ~desc_key(x));
+                if (slot < (unsigned)BQ) s_bq[slot] = x;
+            }
+            band_push(x, inb && slot >= (unsigned)BQ, P.band, cap, &P.ctl->c_band, lane, a);   // queue full
+        }
+    }
+}
+
 // The verdict, and for a failed first round with widening enabled the side the
 // threshold lies on: a bracket whose counts agree and whose band fits, but with
 // G(a_R) >= k (b at or above a_R) or G(a_L) < k (b below a_L), was missed.
@@ -640,7 +760,11 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     extern __shared__ __align__(128) unsigned char dsm[];
     __shared__ double s_red[7 * (SBLOCK / 32)];
     __shared__ double s_tab[32];
+    __shared__ float s_bq[CERT ? 1 : BQ];   // sparse band scores of this CTA
+    __shared__ unsigned s_bn;
+    __shared__ unsigned long long s_bbase;
     exp2_table_init(s_tab);
+    if (threadIdx.x == 0) s_bn = 0u;
     pdl_enter();
     if (round_skipped(P)) return;
     if (!CERT) {   // the select histogram is spent: clear it for the next solve
@@ -665,8 +789,8 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     if (aligned) {
         const float4 *src[1] = {r4};
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
-            oob_vec<MODE>(lds128(ch[0] + threadIdx.x), true, E, acc, P, cap, lane);
-            oob_vec<MODE>(lds128(ch[0] + threadIdx.x + SBLOCK), true, E, acc, P, cap, lane);
+            oob_chunk<MODE>(lds128(ch[0] + threadIdx.x), lds128(ch[0] + threadIdx.x + SBLOCK), E, acc, P, cap,
+                            lane, s_bq, &s_bn);
         });
     }
     // vectors after the last full chunk (whole warps iterate together)
@@ -689,6 +813,16 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     if (!CERT) {
         __shared__ uint32_t s_two[2];
         band_range_flush(ctl, acc.kmax, acc.kinv, s_two);
+        // the queued band scores: one slot range per CTA
+        const unsigned nq = min(s_bn, (unsigned)BQ);
+        if (nq) {
+            if (threadIdx.x == 0) s_bbase = atomicAdd(&ctl->c_band, (unsigned long long)nq);
+            __syncthreads();
+            for (unsigned i = threadIdx.x; i < nq; i += SBLOCK) {
+                const unsigned long long slot = s_bbase + i;
+                if (slot < cap) P.band[slot] = s_bq[i];
+            }
+        }
     }
     if constexpr (MODE == OOB_STREAM) {
         double v[4] = {(double)acc.cL, (double)acc.cR, acc.SL + (double)acc.SL2, acc.SR + (double)acc.SR2};

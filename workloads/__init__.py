@@ -60,6 +60,8 @@ WORKLOADS: dict[str, Workload] = {
                  "bracketing + band sort + certification"),
         Workload("levels1e8", 1, 100_000_000, 1_000_000.0, 0.1, "levels256_desc",
                  "bracketing (+ forced full-sort fallback run)"),
+        Workload("batch64x1m", 64, 1_048_576, 10_486.0, 0.05, "normal",
+                 "batched bracketing (64 rows of 2^20, k = 1% of each row)"),
     ]
 }
 
