@@ -669,11 +669,45 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
                              max_nan(max_nan(v1.x, v1.y), max_nan(v1.z, v1.w)));
     const float mn = fminf(fminf(fminf(v0.x, v0.y), fminf(v0.z, v0.w)), fminf(fminf(v1.x, v1.y), fminf(v1.z, v1.w)));
     const bool fin = mn > -CUDART_INF_F && mx < CUDART_INF_F;
-    // a whole warp on one side (sorted or clustered scores): the float4 fast paths
-    if (__all_sync(FULL, mx < E.aL && fin) || __all_sync(FULL, mn >= E.aR && fin) ||
-        __all_sync(FULL, mn >= E.aL && mx < E.aR && fin)) {
-        oob_vec<MODE>(v0, true, E, a, P, cap, lane);
-        oob_vec<MODE>(v1, true, E, a, P, cap, lane);
+    // a whole warp on one side (sorted or clustered scores): eight scores at once
+    const bool eq0 = v0.x == v0.y && v0.y == v0.z && v0.z == v0.w;
+    const bool eq1 = v1.x == v1.y && v1.y == v1.z && v1.z == v1.w;
+    if (__all_sync(FULL, mx < E.farL && fin)) {            // far below a_L: counts only
+        if (CERT) a.cB += 8; else a.cL += 8;
+        return;
+    }
+    if (__all_sync(FULL, mx < E.midL && fin)) {            // below a_L, fp32 terms
+        if (CERT) a.cB += 8; else a.cL += 8;
+        a.SL2 += ((ex2_ftz((v0.x - E.aL) * E.s2) + ex2_ftz((v0.y - E.aL) * E.s2)) +
+                  (ex2_ftz((v0.z - E.aL) * E.s2) + ex2_ftz((v0.w - E.aL) * E.s2))) +
+                 ((ex2_ftz((v1.x - E.aL) * E.s2) + ex2_ftz((v1.y - E.aL) * E.s2)) +
+                  (ex2_ftz((v1.z - E.aL) * E.s2) + ex2_ftz((v1.w - E.aL) * E.s2)));
+        return;
+    }
+    if (__all_sync(FULL, mx < E.aL && fin)) {              // below a_L, some near it
+        if (CERT) a.cB += 8; else a.cL += 8;
+        tier4<false>(v0, eq0, E.aL, E.daL, E, a.SL, a.SL2);
+        tier4<false>(v1, eq1, E.aL, E.daL, E, a.SL, a.SL2);
+        return;
+    }
+    if (__all_sync(FULL, mn >= E.aR && fin)) {             // at or above a_R
+        if (CERT) { a.cL += 8; a.cR += 8; } else a.cR += 8;
+        tier4<true>(v0, eq0, E.aR, E.daR, E, a.SR, a.SR2);
+        tier4<true>(v1, eq1, E.aR, E.daR, E, a.SR, a.SR2);
+        return;
+    }
+    if (__all_sync(FULL, mn >= E.aL && mx < E.aR && fin)) {   // inside the band
+        if (BANDTERMS) {
+            if (CERT) a.cL += 8;
+            tier4<true>(v0, eq0, E.aL, E.daL, E, a.hL, a.hL2);
+            tier4<false>(v0, eq0, E.aR, E.daR, E, a.lR, a.lR2);
+            tier4<true>(v1, eq1, E.aL, E.daL, E, a.hL, a.hL2);
+            tier4<false>(v1, eq1, E.aR, E.daR, E, a.lR, a.lR2);
+        }
+        if (!CERT) {
+            band_push4(v0, 0xF, P.band, cap, &P.ctl->c_band, lane, a);
+            band_push4(v1, 0xF, P.band, cap, &P.ctl->c_band, lane, a);
+        }
         return;
     }
     // general path: the cheap part for all eight, then the marked ones

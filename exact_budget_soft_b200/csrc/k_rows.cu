@@ -294,16 +294,21 @@ cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, d
     return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, 0, st);
 }
 
-// Two variants, each gated on the band size the streaming pass counted: bands
-// of up to 4096 scores (and tied or empty bands) in a 256-thread CTA, larger
-// ones up to 32768 in a 1024-thread CTA.
+// Three variants, each gated on the band size the streaming pass counted (the
+// sort inside a CTA costs its capacity, not the band): bands of up to 4096
+// scores (and tied or empty bands) in a 256-thread CTA, up to 16384 in a
+// 512-thread CTA, up to 32768 in a 1024-thread CTA.  A launch whose gate is
+// closed returns at once.
 cudaError_t launch_rowsolve_band(const float *band, int64_t rows, double k, double t, Ctl *ctl,
                                  int64_t band_cap, int32_t round2, cudaStream_t st) {
     cudaError_t e =
         launch_rowsolve<256, 16, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, round2, st);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || band_cap <= RowCfg<256, 16>::CAP) return e;
+    e = launch_rowsolve<512, 32, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap,
+                                       RowCfg<256, 16>::CAP, round2, st);
+    if (e != cudaSuccess || band_cap <= RowCfg<512, 32>::CAP) return e;
     return launch_rowsolve<1024, 32, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap,
-                                           RowCfg<256, 16>::CAP, round2, st);
+                                           RowCfg<512, 32>::CAP, round2, st);
 }
 
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,

@@ -414,7 +414,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         { Launch L(r2 ? "widen_stream_pass" : "stream_pass", st); LAPSUM_TRY(launch_stream_pass(Q, st)); }
         {
             Launch L(r2 ? "widen_band_rowsolve" : "band_rowsolve", st);
-            ++g_launches;   // two size-gated variants
+            g_launches += Q.band_cap > 16384 ? 2 : (Q.band_cap > 4096 ? 1 : 0);   // size-gated variants
             LAPSUM_TRY(launch_rowsolve_band(w->band, rows, k, t, w->ctl, Q.band_cap, Q.round2, st));
         }
         if (Q.band_cap > rowsolve_capacity()) {

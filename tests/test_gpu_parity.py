@@ -447,3 +447,18 @@ def test_batched_rows_all_fall_back(L, orc):
     for i in range(rows):
         assert sts[i]["verdict"] == 0 and sts[i]["fallback"] == 1 and sts[i]["rc"] == 0
         check_row(orc, r[i], g[i], k, t, p[i], b[i], grad[i])
+
+
+@pytest.mark.parametrize("s,lo,hi", [(65536, 0, 4096), (16384, 4096, 16384), (2048, 16384, 32768)])
+def test_band_solver_variants(L, orc, s, lo, hi):
+    # the sample size sets the band's size: each one-CTA band solver variant
+    # (<= 4096, <= 16384, <= 32768 scores) solves one of these bands
+    n = 1 << 20
+    r, g = W.small_case("normal", 1, n, seed=16)
+    k, t = n / 100.0, 0.05
+    br = orc.bracket(r[0], k, t, 0, s, 1e-6)
+    cert = orc.certify(r[0], k, t, br["a_L"], br["a_R"], band_cap=10**12)
+    assert lo < cert["c_band"] <= hi
+    p, b, st, grad = run(L, r, k, t, opts=L.options(sample_size=s), g_np=g)
+    assert st["rc"] == 0 and st["verdict"] == 1 and st["c_band"] == cert["c_band"]
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
