@@ -55,13 +55,20 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
         if (((diff >> sh) & 0xffu) == 0u) continue;   // every key has this digit
         for (int i = tid; i < C::NW * 256; i += BLOCK) s_hist[i] = 0;
         __syncthreads();
-        // count: per-warp digit histograms (one shared update per group of equal digits)
+        // count: per-warp digit histograms.  Counts need no order: one shared
+        // atomic per key (lanes on one counter serialise, the rest run in
+        // parallel).  A mostly uniform warp (band mode: padding) takes one
+        // update per group of equal digits instead.
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
             const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = digit_peers<UNIFORM>(d);
-            if (lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
-            __syncwarp();
+            if (UNIFORM) {
+                const unsigned peers = digit_peers<true>(d);
+                if (lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
+                __syncwarp();
+            } else {
+                atomicAdd(&my_hist[d], 1u);
+            }
         }
         __syncthreads();
         if (tid < 256) {   // per digit: exclusive prefix over warps, and total
