@@ -171,6 +171,8 @@ template <int K>
 constexpr size_t stage_bytes() { return 2 * TILE_K(K) * 4 + 2 * sizeof(uint64_t); }
 
 // Adds this warp's digit counts of the tile to my_hist (the warp's 256 counters).
+// Counts need no order: a warp whose keys all share the digit (sorted or tied
+// scores) adds them at once, any other warp takes one shared atomic per key.
 template <int K>
 __device__ __forceinline__ void warp_count(const uint32_t (&key)[K], int cnt_tile, int sh, uint32_t *my_hist) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -179,10 +181,13 @@ __device__ __forceinline__ void warp_count(const uint32_t (&key)[K], int cnt_til
         const int li = warp * 32 * K + i * 32 + lane;
         const bool v = li < cnt_tile;
         const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
-        const unsigned peers = __match_any_sync(FULL, d);
-        if (v && lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
-        __syncwarp();
+        if (__all_sync(FULL, d == __shfl_sync(FULL, d, 0))) {
+            if (lane == 0 && d < 0x100u) my_hist[d] += 32u;
+        } else if (v) {
+            atomicAdd(&my_hist[d], 1u);
+        }
     }
+    __syncwarp();
 }
 
 // Walks the CTA's chunk of tiles in order with one tile staged ahead, calling
