@@ -101,10 +101,10 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
             float v = row[idx];
             bad |= !isfinite(v);
             kk = desc_key(v);
+            kand &= kk;   // digits on which the scores agree (padding excluded: it is the
+            kor |= kk;    //   largest key and starts after every score, so ties keep it last)
         }
         key[i] = kk;
-        kand &= kk;
-        kor |= kk;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
