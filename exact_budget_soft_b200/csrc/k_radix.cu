@@ -32,7 +32,6 @@ constexpr int RNW = RB / 32;
 constexpr int HB = 256;             // histogram kernel threads
 
 
-int radix_tile() { return TILE_K(RK_BIG); }
 
 // Element count behind a gate; < 0 means "nothing to do".
 __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
@@ -470,7 +469,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
     uint32_t *s_run = s_gofs + 256;            // 256: running global offset of each digit
     uint32_t *s_tot = s_run + 256;             // 256: scratch (tile totals)
     uint32_t *s_h4 = s_tot + 256;              // 4 * 256: phase-H histograms, then digit bases
-    __shared__ int s_skip, s_solved;
+    __shared__ int s_skip;
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
     pdl_wait();
@@ -537,7 +536,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
         }
         bar();
         // digit bases and skip flags, the same in every CTA (thread d owns bin d)
-        if (tid == 0) { s_skip = 0; s_solved = 0; }
+        if (tid == 0) s_skip = 0;
         __syncthreads();
         for (int d4 = 0; d4 < 4; ++d4) {
             uint32_t v = 0;
@@ -682,10 +681,6 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
         bar();   // the maps are complete, and every CTA has read the global histograms
         if (c == 0) {
             for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
-            if (tid == 0) {
-                ctl->sort_cur = cur;
-                ctl->sort_solved = skip == 15 ? 1 : 0;
-            }
             if (skip != 15) locate_finish<K>(A, sorted, n, z, rec, crec, S.buf, s_hist, s_tab);
         }
         if (row + 1 < Ag.rows) bar();   // the next row reuses the global scratch

@@ -39,10 +39,8 @@ struct Ctl {
     double sum_p;
     // single-pass "last block" tickets (zeroed with the block)
     unsigned int ticket[8];
-    // radix sort: which buffer holds the current keys (-1: the fp32 source)
     unsigned int sel_cnt[2];  // select: keys under each target's 16-bit prefix
-    int32_t sort_cur;
-    int32_t sort_solved;      // every key equal: solved without the locate step
+    // device-wide sort
     unsigned int gbar_count;  // grid barrier of the cooperative sort: arrivals
     unsigned int gbar_gen;    //   and generation
     // backward

@@ -88,7 +88,6 @@ struct SortArgs {
     int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
     double k, t;               // budget and temperature (all-equal shortcut)
 };
-int radix_tile();
 int sort_grid_max();
 int64_t sort_record_doubles(int64_t cap);
 cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st);
