@@ -25,6 +25,8 @@ LIB_PATH = os.path.join(_HERE, "liblapsum.so")
 
 PATH_AUTO, PATH_FULLSORT, PATH_BRACKET = 0, 1, 2
 CERTIFY_PASS, CERTIFY_FUSED = 0, 1
+# error codes (LAPSUM_ERR_* of the C header)
+ERR_ARG, ERR_NONFINITE, ERR_ALLOC, ERR_DEVICE_TIMEOUT, ERR_CUDA, ERR_NO_ROOT = -1, -2, -3, -4, -5, -6
 ERRORS = {0: "ok", -1: "invalid argument", -2: "non-finite score", -3: "workspace allocation failed",
           -4: "device wait timeout", -5: "CUDA runtime error", -6: "no crossing found"}
 

@@ -462,3 +462,36 @@ def test_band_solver_variants(L, orc, s, lo, hi):
     p, b, st, grad = run(L, r, k, t, opts=L.options(sample_size=s), g_np=g)
     assert st["rc"] == 0 and st["verdict"] == 1 and st["c_band"] == cert["c_band"]
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+# ------------------------------------------------------- bracketing edges --
+@pytest.mark.parametrize("k,t", [(1.5, 0.05), ((1 << 20) - 3.0, 0.05), (1000.0, 1e-4), (300000.0, 50.0)])
+def test_bracketing_extreme_budgets_and_temperatures(L, orc, k, t):
+    # k near 0 (a_R = +inf) and near n (a_L = -inf); a tiny t (nearly hard top-k)
+    # and a large one (p nearly k/n everywhere)
+    n = 1 << 20
+    r, g = W.small_case("normal", 1, n, seed=17)
+    p, b, st, grad = run(L, r, k, t, g_np=g)
+    assert st["rc"] == 0 and st["path"] == 2
+    plan = L.bracket_plan(n, k)
+    check_bracket_integers(orc, r[0], k, t, st, 0, plan["s"], 1e-6)
+    # with t large every p is mid-range and the fp32 p carry a bias of a fraction
+    # of an ulp that adds up over 2^20 scores: the mass tolerance holds for the
+    # exact mass at b (checked in check_row) and the rounded sum keeps within its
+    # rounding bound sum ulp(p_i)/2
+    wide = t > 1.0
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0], exact_sum=not wide)
+    if wide:
+        bound = np.sum(np.spacing(p[0].astype(np.float32)).astype(np.float64)) / 2
+        assert abs(p[0].astype(np.float64).sum() - k) <= bound
+
+
+def test_batched_rows_report_a_nonfinite_row(L):
+    rows, n = 3, 1 << 20
+    r, _ = W.small_case("normal", rows, n, seed=18)
+    r[1, 12345] = np.nan
+    rt = torch.from_numpy(r).cuda()
+    L.forward(rt, 1000.0, 0.05)
+    sts = L.get_stats_rows(rows, check=False)
+    assert sts[0]["rc"] == L.ERR_NONFINITE
+    assert (sts[1]["status"] & 1) and not (sts[0]["status"] & 1) and not (sts[2]["status"] & 1)
