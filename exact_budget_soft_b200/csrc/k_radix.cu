@@ -486,204 +486,230 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
     __syncthreads();
     uint32_t ph = 0;   // mbarrier phases, carried from row to row
     // the rows of a batch, one after another (each gated by its own control block)
-    for (int64_t row = 0; row < Ag.rows; ++row) {
-        SortArgs A = Ag;
-        A.src = Ag.src + row * Ag.src_stride;
-        A.ctl = Ag.ctl + row;
-        const int64_t n = gated_n(A);
-        if (n < 0) continue;   // the gate reads the same control words in every CTA
-        Ctl *ctl = A.ctl;
-        const int64_t ntiles = (n + TILE_K(K) - 1) / TILE_K(K);
-        const int64_t t0 = (int64_t)c * ntiles / G, t1 = (int64_t)(c + 1) * ntiles / G;
-        uint32_t *csum = A.chunkcnt;   // [4][256][G]
-        auto bar = [&]() { grid_sync(&ctl->gbar_count, &ctl->gbar_gen, A.spin_cap, &ctl->status); };
-        S.n = n;
-        for (int i = tid; i < 4 * 256; i += RB) s_h4[i] = 0;
-        __syncthreads();
-        bool ok = true;
-
-        // ---- phase H: the chunk's four digit histograms
+    // The gates of a block of RB rows are read together (one thread per row) and
+    // the open rows listed in row order -- the same list in every CTA.
+    __shared__ int s_open[RB];
+    __shared__ int s_wopen[RNW];
+    for (int64_t r0 = 0; r0 < Ag.rows; r0 += RB) {
+        int nopen = 0;
         {
-            uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-            uint32_t cnt[4] = {0, 0, 0, 0};
-            ok &= walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
-                const int l0 = warp * 32 * K + lane;
-#pragma unroll
-                for (int i = 0; i < K; ++i) {
-                    if (l0 + i * 32 >= cnt_tile) break;
-#pragma unroll
-                    for (int d = 0; d < 4; ++d) {
-                        const uint32_t bin = (key[i] >> (8 * d)) & 0xffu;
-                        if (bin == cur[d]) {
-                            ++cnt[d];
-                        } else {
-                            if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
-                            cur[d] = bin;
-                            cnt[d] = 1;
-                        }
-                    }
-                }
-            });
-#pragma unroll
-            for (int d = 0; d < 4; ++d)
-                if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
+            bool open = false;
+            if (r0 + tid < Ag.rows) {
+                SortArgs A = Ag;
+                A.ctl = Ag.ctl + r0 + tid;
+                open = gated_n(A) >= 0;
+            }
+            const unsigned m = __ballot_sync(FULL, open);
+            if (lane == 0) s_wopen[warp] = __popc(m);
             __syncthreads();
-            for (int i = tid; i < 4 * 256; i += RB) {
-                const uint32_t v = s_h4[i];
-                csum[(size_t)i * G + c] = v;
-                if (v) atomicAdd(A.hist + i, (unsigned long long)v);
+            int before = 0;
+            for (int w = 0; w < RNW; ++w) {
+                before += w < warp ? s_wopen[w] : 0;
+                nopen += s_wopen[w];
             }
-        }
-        bar();
-        // digit bases and skip flags, the same in every CTA (thread d owns bin d)
-        if (tid == 0) s_skip = 0;
-        __syncthreads();
-        for (int d4 = 0; d4 < 4; ++d4) {
-            uint32_t v = 0;
-            if (tid < 256) v = (uint32_t)__ldcg(A.hist + d4 * 256 + tid);
-            uint32_t inc = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(FULL, inc, o);
-                if (lane >= o) inc += y;
-            }
-            if (lane == 31 && tid < 256) s_tot[warp] = inc;
-            __syncthreads();
-            if (tid < 256) {
-                uint32_t off = 0;
-                for (int w = 0; w < warp; ++w) off += s_tot[w];
-                s_h4[d4 * 256 + tid] = off + inc - v;   // exclusive base of bin tid
-                if (v == (uint32_t)n) atomicOr(&s_skip, 1 << d4);
-            }
+            if (open) s_open[before + __popc(m & ((1u << lane) - 1u))] = tid;
             __syncthreads();
         }
-        const int skip = s_skip;
-        int cur = -1;   // key buffer of the current order (-1: the scores)
-        if (skip == 15) {   // every key equal
-            if (c == 0 && tid == 0) solve_equal_run(A, n);
-        } else {
-            bool first = true;
-            for (int pass = 0; pass < 4; ++pass) {
-                if (skip & (1 << pass)) continue;
-                const int sh = 8 * pass;
-                const uint32_t *src = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
-                uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
-                uint32_t *crow = csum + (size_t)pass * 256 * G;   // [256][G] of this digit
-                if (!first) {   // the chunk's digit counts in the current order
-                    for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
-                    __syncthreads();
-                    ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
-                        warp_count(key, cnt_tile, sh, s_hist + warp * 256);
-                    });
-                    if (tid < 256) {
-                        uint32_t tot = 0;
-#pragma unroll
-                        for (int w = 0; w < RNW; ++w) tot += s_hist[w * 256 + tid];
-                        crow[(size_t)tid * G + c] = tot;
-                    }
-                    bar();
-                }
-                // global start of every digit in this chunk: base + counts of earlier
-                // chunks (a warp per digit, four digits' loads in flight at once)
-                for (int j = 0; j < 256 / RNW; j += 4) {
-                    uint32_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-                    for (int u = 0; u < SORT_GMAX / 32; ++u) {
-                        const int q = lane + 32 * u;
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj)
-                            if (q < c) acc[jj] += __ldcg(crow + (size_t)(warp * (256 / RNW) + j + jj) * G + q);
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        uint32_t a = acc[jj];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
-                        const int d = warp * (256 / RNW) + j + jj;
-                        if (lane == 0) s_run[d] = s_h4[pass * 256 + d] + a;
-                    }
-                }
-                __syncthreads();
-                ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *s_keys) {
-                    for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
-                    __syncthreads();   // every key is in registers: s_keys is free too
-                    uint32_t *my_hist = s_hist + warp * 256;
-                    warp_count(key, cnt_tile, sh, my_hist);
-                    __syncthreads();
-                    if (tid < 256) {   // per digit: exclusive offsets of the warps, tile total
-                        uint32_t tot = 0;
-#pragma unroll
-                        for (int w = 0; w < RNW; ++w) {
-                            const uint32_t cw = s_hist[w * 256 + tid];
-                            s_hist[w * 256 + tid] = tot;
-                            tot += cw;
-                        }
-                        s_tot[tid] = tot;
-                        s_gofs[tid] = s_run[tid];
-                        s_run[tid] += tot;
-                    }
-                    __syncthreads();
-                    if (warp == 0) {   // exclusive scan of the 256 tile totals
-                        uint32_t v[8], run = 0;
-#pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) { v[jj] = s_tot[lane * 8 + jj]; run += v[jj]; }
-                        uint32_t inc = run;
-#pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const uint32_t y = __shfl_up_sync(FULL, inc, o);
-                            if (lane >= o) inc += y;
-                        }
-                        uint32_t ex = inc - run;
-#pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) { const uint32_t cc = v[jj]; s_dstart[lane * 8 + jj] = ex; ex += cc; }
-                    }
-                    __syncthreads();
-                    if (tid < 256) s_gofs[tid] -= s_dstart[tid];
-                    for (int i = tid; i < RNW * 256; i += RB) s_hist[i] += s_dstart[i & 255];
-                    __syncthreads();
-                    // scatter into shared memory by (digit, warp, traversal order): stable
-                    const unsigned lt_mask = (1u << lane) - 1u;
+        for (int oi = 0; oi < nopen; ++oi) {
+            const int64_t row = r0 + s_open[oi];
+            SortArgs A = Ag;
+            A.src = Ag.src + row * Ag.src_stride;
+            A.ctl = Ag.ctl + row;
+            const int64_t n = gated_n(A);
+            Ctl *ctl = A.ctl;
+            const int64_t ntiles = (n + TILE_K(K) - 1) / TILE_K(K);
+            const int64_t t0 = (int64_t)c * ntiles / G, t1 = (int64_t)(c + 1) * ntiles / G;
+            uint32_t *csum = A.chunkcnt;   // [4][256][G]
+            auto bar = [&]() { grid_sync(&ctl->gbar_count, &ctl->gbar_gen, A.spin_cap, &ctl->status); };
+            S.n = n;
+            for (int i = tid; i < 4 * 256; i += RB) s_h4[i] = 0;
+            __syncthreads();
+            bool ok = true;
+
+            // ---- phase H: the chunk's four digit histograms
+            {
+                uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+                uint32_t cnt[4] = {0, 0, 0, 0};
+                ok &= walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
+                    const int l0 = warp * 32 * K + lane;
 #pragma unroll
                     for (int i = 0; i < K; ++i) {
-                        const int li = warp * 32 * K + i * 32 + lane;
-                        const bool v = li < cnt_tile;
-                        const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
-                        const unsigned peers = __match_any_sync(FULL, d);
-                        const int leader = __ffs(peers) - 1;
-                        uint32_t bs = 0;
-                        if (v && lane == leader) {
-                            bs = my_hist[d];
-                            my_hist[d] = bs + __popc(peers);
+                        if (l0 + i * 32 >= cnt_tile) break;
+#pragma unroll
+                        for (int d = 0; d < 4; ++d) {
+                            const uint32_t bin = (key[i] >> (8 * d)) & 0xffu;
+                            if (bin == cur[d]) {
+                                ++cnt[d];
+                            } else {
+                                if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
+                                cur[d] = bin;
+                                cnt[d] = 1;
+                            }
                         }
-                        bs = __shfl_sync(FULL, bs, leader) + __popc(peers & lt_mask);
-                        if (v) s_keys[bs] = key[i];
-                        __syncwarp();
-                    }
-                    __syncthreads();
-                    // runs of one digit are consecutive in s_keys and in dst: coalesced writes
-                    for (int i = tid; i < cnt_tile; i += RB) {
-                        const uint32_t kk = s_keys[i];
-                        dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
                     }
                 });
-                bar();   // the pass's keys are all written before the next pass reads them
-                cur = cur == 0 ? 1 : 0;
-                first = false;
+#pragma unroll
+                for (int d = 0; d < 4; ++d)
+                    if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
+                __syncthreads();
+                for (int i = tid; i < 4 * 256; i += RB) {
+                    const uint32_t v = s_h4[i];
+                    csum[(size_t)i * G + c] = v;
+                    if (v) atomicAdd(A.hist + i, (unsigned long long)v);
+                }
             }
+            bar();
+            // digit bases and skip flags, the same in every CTA (thread d owns bin d)
+            if (tid == 0) s_skip = 0;
+            __syncthreads();
+            for (int d4 = 0; d4 < 4; ++d4) {
+                uint32_t v = 0;
+                if (tid < 256) v = (uint32_t)__ldcg(A.hist + d4 * 256 + tid);
+                uint32_t inc = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(FULL, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                if (lane == 31 && tid < 256) s_tot[warp] = inc;
+                __syncthreads();
+                if (tid < 256) {
+                    uint32_t off = 0;
+                    for (int w = 0; w < warp; ++w) off += s_tot[w];
+                    s_h4[d4 * 256 + tid] = off + inc - v;   // exclusive base of bin tid
+                    if (v == (uint32_t)n) atomicOr(&s_skip, 1 << d4);
+                }
+                __syncthreads();
+            }
+            const int skip = s_skip;
+            int cur = -1;   // key buffer of the current order (-1: the scores)
+            if (skip == 15) {   // every key equal
+                if (c == 0 && tid == 0) solve_equal_run(A, n);
+            } else {
+                bool first = true;
+                for (int pass = 0; pass < 4; ++pass) {
+                    if (skip & (1 << pass)) continue;
+                    const int sh = 8 * pass;
+                    const uint32_t *src = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
+                    uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
+                    uint32_t *crow = csum + (size_t)pass * 256 * G;   // [256][G] of this digit
+                    if (!first) {   // the chunk's digit counts in the current order
+                        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
+                        __syncthreads();
+                        ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
+                            warp_count(key, cnt_tile, sh, s_hist + warp * 256);
+                        });
+                        if (tid < 256) {
+                            uint32_t tot = 0;
+#pragma unroll
+                            for (int w = 0; w < RNW; ++w) tot += s_hist[w * 256 + tid];
+                            crow[(size_t)tid * G + c] = tot;
+                        }
+                        bar();
+                    }
+                    // global start of every digit in this chunk: base + counts of earlier
+                    // chunks (a warp per digit, four digits' loads in flight at once)
+                    for (int j = 0; j < 256 / RNW; j += 4) {
+                        uint32_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+                        for (int u = 0; u < SORT_GMAX / 32; ++u) {
+                            const int q = lane + 32 * u;
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+                                if (q < c) acc[jj] += __ldcg(crow + (size_t)(warp * (256 / RNW) + j + jj) * G + q);
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            uint32_t a = acc[jj];
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+                            const int d = warp * (256 / RNW) + j + jj;
+                            if (lane == 0) s_run[d] = s_h4[pass * 256 + d] + a;
+                        }
+                    }
+                    __syncthreads();
+                    ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *s_keys) {
+                        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
+                        __syncthreads();   // every key is in registers: s_keys is free too
+                        uint32_t *my_hist = s_hist + warp * 256;
+                        warp_count(key, cnt_tile, sh, my_hist);
+                        __syncthreads();
+                        if (tid < 256) {   // per digit: exclusive offsets of the warps, tile total
+                            uint32_t tot = 0;
+#pragma unroll
+                            for (int w = 0; w < RNW; ++w) {
+                                const uint32_t cw = s_hist[w * 256 + tid];
+                                s_hist[w * 256 + tid] = tot;
+                                tot += cw;
+                            }
+                            s_tot[tid] = tot;
+                            s_gofs[tid] = s_run[tid];
+                            s_run[tid] += tot;
+                        }
+                        __syncthreads();
+                        if (warp == 0) {   // exclusive scan of the 256 tile totals
+                            uint32_t v[8], run = 0;
+#pragma unroll
+                            for (int jj = 0; jj < 8; ++jj) { v[jj] = s_tot[lane * 8 + jj]; run += v[jj]; }
+                            uint32_t inc = run;
+#pragma unroll
+                            for (int o = 1; o < 32; o <<= 1) {
+                                const uint32_t y = __shfl_up_sync(FULL, inc, o);
+                                if (lane >= o) inc += y;
+                            }
+                            uint32_t ex = inc - run;
+#pragma unroll
+                            for (int jj = 0; jj < 8; ++jj) { const uint32_t cc = v[jj]; s_dstart[lane * 8 + jj] = ex; ex += cc; }
+                        }
+                        __syncthreads();
+                        if (tid < 256) s_gofs[tid] -= s_dstart[tid];
+                        for (int i = tid; i < RNW * 256; i += RB) s_hist[i] += s_dstart[i & 255];
+                        __syncthreads();
+                        // scatter into shared memory by (digit, warp, traversal order): stable
+                        const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+                        for (int i = 0; i < K; ++i) {
+                            const int li = warp * 32 * K + i * 32 + lane;
+                            const bool v = li < cnt_tile;
+                            const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
+                            const unsigned peers = __match_any_sync(FULL, d);
+                            const int leader = __ffs(peers) - 1;
+                            uint32_t bs = 0;
+                            if (v && lane == leader) {
+                                bs = my_hist[d];
+                                my_hist[d] = bs + __popc(peers);
+                            }
+                            bs = __shfl_sync(FULL, bs, leader) + __popc(peers & lt_mask);
+                            if (v) s_keys[bs] = key[i];
+                            __syncwarp();
+                        }
+                        __syncthreads();
+                        // runs of one digit are consecutive in s_keys and in dst: coalesced writes
+                        for (int i = tid; i < cnt_tile; i += RB) {
+                            const uint32_t kk = s_keys[i];
+                            dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
+                        }
+                    });
+                    bar();   // the pass's keys are all written before the next pass reads them
+                    cur = cur == 0 ? 1 : 0;
+                    first = false;
+                }
+            }
+            if (!ok) atomicOr(&ctl->status, ST_TIMEOUT);
+            // locate: tile and chunk maps of the sorted values (every CTA, its chunk)
+            const uint32_t *sorted = cur == 0 ? A.keys[0] : A.keys[1];
+            const Seeds z = locate_seeds(A);
+            ChunkRec *crec = reinterpret_cast<ChunkRec *>(A.tilebuf);
+            TileRec *rec = reinterpret_cast<TileRec *>(A.tilebuf + 8 * SORT_GMAX);
+            if (skip != 15) locate_tiles<K>(A, sorted, n, t0, t1, z, rec, crec, S.buf, reinterpret_cast<Aff *>(s_hist), s_tab);
+            bar();   // the maps are complete, and every CTA has read the global histograms
+            if (c == 0) {
+                for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
+                if (skip != 15) locate_finish<K>(A, sorted, n, z, rec, crec, S.buf, s_hist, s_tab);
+            }
+            bar();   // the next row reuses the global scratch
+            __syncthreads();   // s_open is rewritten by the next block of rows
         }
-        if (!ok) atomicOr(&ctl->status, ST_TIMEOUT);
-        // locate: tile and chunk maps of the sorted values (every CTA, its chunk)
-        const uint32_t *sorted = cur == 0 ? A.keys[0] : A.keys[1];
-        const Seeds z = locate_seeds(A);
-        ChunkRec *crec = reinterpret_cast<ChunkRec *>(A.tilebuf);
-        TileRec *rec = reinterpret_cast<TileRec *>(A.tilebuf + 8 * SORT_GMAX);
-        if (skip != 15) locate_tiles<K>(A, sorted, n, t0, t1, z, rec, crec, S.buf, reinterpret_cast<Aff *>(s_hist), s_tab);
-        bar();   // the maps are complete, and every CTA has read the global histograms
-        if (c == 0) {
-            for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
-            if (skip != 15) locate_finish<K>(A, sorted, n, z, rec, crec, S.buf, s_hist, s_tab);
-        }
-        if (row + 1 < Ag.rows) bar();   // the next row reuses the global scratch
     }
     pdl_trigger();
 }
