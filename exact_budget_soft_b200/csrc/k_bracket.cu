@@ -1210,8 +1210,11 @@ int64_t partial_stride(int64_t rows) {
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st) {
     return launch_k(sample_kernel, dim3((unsigned)((P.s + 255) / 256), (unsigned)P.rows), 256, 0, st, P);
 }
+// 64 CTAs for one row; a batch shares about four CTAs per SM among its rows
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
-    return launch_k(select_kernel, dim3(SEL_GRID, (unsigned)P.rows), SEL_BLOCK, 0, st, P);
+    int64_t per_row = (int64_t)stream_grid() / P.rows;
+    per_row = per_row < 1 ? 1 : (per_row > SEL_GRID ? SEL_GRID : per_row);
+    return launch_k(select_kernel, dim3((unsigned)per_row, (unsigned)P.rows), SEL_BLOCK, 0, st, P);
 }
 int select_cand_capacity() { return SEL_CAND; }
 template <typename K>
