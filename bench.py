@@ -443,6 +443,13 @@ def run_case(args):
         r = torch.from_numpy(W.scores(w)).cuda()
         g = torch.from_numpy(W.upstream_grad(w)).cuda()
         opts = None
+    elif args.case == "batch":   # batched bracketing on normal scores (random order)
+        w = W.WORKLOADS["batch64x1m"]
+        rows = args.case_rows or w.rows
+        w = W.Workload(f"batch{rows}x1m", rows, w.n, w.k, w.t, w.dist, w.path)
+        r = torch.from_numpy(W.scores(w)).cuda()
+        g = torch.from_numpy(W.upstream_grad(w)).cuda()
+        opts = None
     else:   # forced full-sort fallback on the levels workload (possibly scaled)
         w = W.WORKLOADS["levels1e8"]
         if args.scale_n:
@@ -480,7 +487,7 @@ def main():
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--scale-n", type=int, default=0, help="profiling: same workload at another n")
-    ap.add_argument("--case", choices=["rows", "fallback"], default=None,
+    ap.add_argument("--case", choices=["rows", "fallback", "batch"], default=None,
                     help="profiling driver: time one non-headline case instead of the benchmark")
     ap.add_argument("--case-rows", type=int, default=0)
     args = ap.parse_args()

@@ -1,0 +1,307 @@
+// k_band.cu -- the band solve of the bracketing path: the threshold b inside
+// [a_L, a_R) from the band scores and the streaming pass's counts and tail sums
+// ("Fast LapSum: Exact Differentiable Top-k at Million Scale", technical summary
+// section 2.2 step 3; the root of one interval in closed form, section 2.1).
+//
+// One CTA per row.  Instead of sorting the band, the CTA narrows it with a radix
+// select steered by G itself:
+//   * the band's key range is cut into at most 1024 bins of 2^s consecutive keys;
+//     one sweep over the band gives every bin its count, its smallest and largest
+//     key, and two tail sums referenced to the bin's own edges,
+//         A_j = sum_{r in bin j} e^{(r - e_j)/t},  B_j = sum_{r in bin j} e^{(e_{j+1} - r)/t}
+//     (e_j > r >= e_{j+1}, so every term is at most 1);
+//   * affine recurrences over the bins -- the maps of the sorted scan, one per
+//     bin instead of one per score --
+//         U_{j+1} = B_j + d_j U_j,   V_j = A_j + d_j V_{j+1},   d_j = e^{(e_{j+1} - e_j)/t}
+//     give G at every edge, G(e_j) = C_j - U_j/2 + V_j/2 (C_j: scores >= e_j);
+//   * G falls as b rises, so the bin whose top edge has G < k and whose bottom
+//     edge has G >= k holds b; it becomes the new band, the scores above and
+//     below it folded into (C, U) and V.
+// Each step leaves a key range shorter by ten bits, so at most four steps end
+// on a band of one value (any count) or an empty one, where the root has a
+// closed form -- no sort at all.  Steps sweep the band buffer until the band has
+// at most GATHER_CAP scores; it is then copied to shared memory and the later
+// steps sweep that copy.  The sums are fixed point (2^-62 units, exact 96-bit
+// integers), so b does not depend on the order in which threads add.
+#include <cstdint>
+
+#include "lapsum_device.cuh"
+#include "lapsum_kernels.h"
+
+namespace lapsum {
+
+constexpr int BS_BLOCK = 1024;
+constexpr int BS_BITS = 10;
+constexpr int BS_BINS = 1 << BS_BITS;   // one bin per thread in the scan
+constexpr int BS_NW = BS_BLOCK / 32;
+constexpr int GATHER_CAP = 4096;        // bands this small are swept from shared memory
+
+// A band (or sub-band) and what lies outside it.
+struct SubBand {
+    unsigned long long m0;     // scores at or above top
+    unsigned long long n;      // scores inside [bot, top)
+    double top, P_top;         // P_top = sum_{r >= top} e^{(top - r)/t}
+    double bot, Q_bot;         // Q_bot = sum_{r < bot} e^{(r - bot)/t}
+    uint32_t klo, khi;         // smallest and largest descending-order key inside
+};
+
+// Fixed-point sum of terms in [0, 1]: q = round(v 2^62) added to a 96-bit
+// integer held in three 32-bit words (w[0] lowest), each add carrying into the
+// next word itself.  Every word sees the same additions in any order, and each
+// add wraps its word at most once, so the carries -- and the total -- do not
+// depend on the order of the adds.  (Shared-memory atomics are native only at
+// 32 bits.)
+__device__ __forceinline__ void fix_add(unsigned *w, double v) {
+    const unsigned long long q = __double2ull_rn(v * 0x1p62);
+    const unsigned lo = (unsigned)q;
+    const unsigned o0 = atomicAdd(&w[0], lo);
+    const unsigned mid = (unsigned)(q >> 32) + (o0 + lo < o0 ? 1u : 0u);   // <= 2^30 + 1
+    if (mid) {
+        const unsigned o1 = atomicAdd(&w[1], mid);
+        if (o1 + mid < o1) atomicAdd(&w[2], 1u);
+    }
+}
+__device__ __forceinline__ double fix_value(const unsigned *w) {
+    return fma((double)w[2], 4.0, fma((double)w[1], 0x1p-30, (double)w[0] * 0x1p-62));
+}
+
+// Per-bin sums of one step (dynamic shared memory).
+struct BinSums {
+    unsigned cnt[BS_BINS];
+    unsigned kmin[BS_BINS];
+    unsigned kmax[BS_BINS];
+    unsigned fa[BS_BINS][3], fb[BS_BINS][3];   // fixed-point A_j and B_j
+};
+
+// Exclusive block scans of three maps per thread: U-maps forward (thread
+// order), V-maps backward, counts forward.  scratch: 3 * BS_NW Aff.
+__device__ __forceinline__ void block_scan3(Aff mu, Aff mv, unsigned c, Aff &mu_ex, Aff &mv_ex, unsigned &c_ex,
+                                            Aff *scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const Aff fi = warp_scan_fwd(mu, lane);
+    const Aff bi = warp_scan_bwd(mv, lane);
+    unsigned ci = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned p = __shfl_up_sync(FULL, ci, o);
+        if (lane >= o) ci += p;
+    }
+    if (lane == 31) {
+        scratch[warp] = fi;
+        scratch[2 * BS_NW + warp] = Aff{0.0, (double)ci};
+    }
+    if (lane == 0) scratch[BS_NW + warp] = bi;
+    __syncthreads();
+    if (warp == 0) {   // BS_NW == 32: one lane per warp
+        Aff wf = warp_scan_fwd(scratch[lane], lane);
+        Aff wb = warp_scan_bwd(scratch[BS_NW + lane], lane);
+        double wc = scratch[2 * BS_NW + lane].s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double p = __shfl_up_sync(FULL, wc, o);
+            if (lane >= o) wc += p;
+        }
+        __syncwarp();
+        scratch[lane] = wf;                        // warps 0..lane
+        scratch[BS_NW + lane] = wb;                // warps lane..31
+        scratch[2 * BS_NW + lane] = Aff{0.0, wc};  // counts of warps 0..lane
+    }
+    __syncthreads();
+    Aff fe = shfl_up_aff(fi, 1);
+    if (lane == 0) fe = aff_id();
+    if (warp > 0) fe = aff_then(scratch[warp - 1], fe);
+    Aff be = shfl_down_aff(bi, 1);
+    if (lane == 31) be = aff_id();
+    if (warp < BS_NW - 1) be = aff_then(scratch[BS_NW + warp + 1], be);
+    mu_ex = fe;
+    mv_ex = be;
+    c_ex = (ci - c) + (warp > 0 ? (unsigned)scratch[2 * BS_NW + warp - 1].s : 0u);
+}
+
+// Edge e_j of the J bins of 2^s keys over [klo, khi]: e_0 = top, e_J = bot, and
+// between them the value of the largest key of bin j - 1 (so bin j holds the
+// scores r with e_{j+1} <= r < e_j).
+__device__ __forceinline__ double bin_edge(uint32_t klo, int s, unsigned J, unsigned j, double top, double bot) {
+    if (j == 0) return top;
+    if (j >= J) return bot;
+    return (double)desc_key_to_float(klo + (j << s) - 1u);
+}
+
+// One narrowing step, by the whole CTA: bins over the current sub-band S (in
+// shared memory), a block scan over the bins (thread j owns bin j), and S left
+// holding the bin that contains b.  The first step over the whole band also
+// flags a root outside [a_L, a_R) (status non-null); later steps take the bin
+// whose edges straddle k as computed, with no flag, as an edge's G can differ
+// from the step before it by rounding.
+__device__ void band_level(const float *src, int64_t nsrc, SubBand &S, BinSums &B, Aff *scratch, unsigned *hit,
+                           double s2d, double k, const double *tab, int32_t *status) {
+    const int tid = threadIdx.x;
+    const uint32_t klo = S.klo, khi = S.khi;
+    const double top = S.top, bot = S.bot;
+    const int bits = 32 - __clz(khi - klo);
+    const int s = bits > BS_BITS ? bits - BS_BITS : 0;
+    const unsigned J = ((khi - klo) >> s) + 1u;   // <= BS_BINS
+    if (tid < (int)J) {
+        B.cnt[tid] = 0u;
+        B.kmin[tid] = 0xffffffffu;
+        B.kmax[tid] = 0u;
+#pragma unroll
+        for (int q = 0; q < 3; ++q) B.fa[tid][q] = B.fb[tid][q] = 0u;
+    }
+    if (tid == 0) *hit = 0xffffffffu;
+    __syncthreads();
+    auto add = [&](float x) {
+        const uint32_t kk = desc_key(x);
+        if (kk < klo || kk > khi) return;
+        const unsigned j = (kk - klo) >> s;
+        const double xd = (double)x;
+        const double eh = bin_edge(klo, s, J, j, top, bot);
+        const double el = bin_edge(klo, s, J, j + 1, top, bot);
+        atomicAdd(&B.cnt[j], 1u);
+        atomicMin(&B.kmin[j], kk);
+        atomicMax(&B.kmax[j], kk);
+        fix_add(B.fa[j], link_exp((eh - xd) * s2d, tab));   // e^{(r - e_j)/t}
+        fix_add(B.fb[j], link_exp((xd - el) * s2d, tab));   // e^{(e_{j+1} - r)/t}
+    };
+    int64_t i = tid;
+    for (; i + 3 * BS_BLOCK < nsrc; i += 4 * BS_BLOCK) {   // four loads in flight
+        const float x0 = src[i], x1 = src[i + BS_BLOCK], x2 = src[i + 2 * BS_BLOCK], x3 = src[i + 3 * BS_BLOCK];
+        add(x0);
+        add(x1);
+        add(x2);
+        add(x3);
+    }
+    for (; i < nsrc; i += BS_BLOCK) add(src[i]);
+    __syncthreads();
+
+    // thread j: bin j (bins past J carry identity maps)
+    const unsigned j = (unsigned)tid;
+    const double e_hi = bin_edge(klo, s, J, j, top, bot), e_lo = bin_edge(klo, s, J, j + 1, top, bot);
+    unsigned c = 0u;
+    double A = 0.0, Bj = 0.0, d = 1.0;
+    if (j < J) {
+        c = B.cnt[j];
+        A = fix_value(B.fa[j]);
+        Bj = fix_value(B.fb[j]);
+        d = link_exp((e_hi - e_lo) * s2d, tab);   // 0 across an infinite edge
+    }
+    Aff mu_ex, mv_ex;
+    unsigned c_ex;
+    block_scan3(Aff{d, Bj}, Aff{d, A}, c, mu_ex, mv_ex, c_ex, scratch);   // U_{j+1} = d U_j + B, V_j = d V_{j+1} + A
+    const double U = fma(mu_ex.a, S.P_top, mu_ex.s);           // U_j
+    const double Vn = fma(mv_ex.a, S.Q_bot, mv_ex.s);          // V_{j+1}
+    const unsigned long long C = S.m0 + c_ex;                  // C_j
+    const double Gn = (double)(C + c) - 0.5 * fma(d, U, Bj) + 0.5 * Vn;   // G(e_{j+1})
+    if (status && j == 0) {
+        const double G0 = (double)C - 0.5 * U + 0.5 * fma(d, Vn, A);
+        if (!(G0 < k)) atomicOr(status, ST_NO_ROOT);   // G(a_R) >= k: b at or above a_R
+    }
+    if (j < J && (Gn >= k || j + 1 == J)) atomicMin(hit, j);   // the first bin whose bottom edge has G >= k
+    __syncthreads();
+    if (j == *hit) {
+        if (status && !(Gn >= k)) atomicOr(status, ST_NO_ROOT);   // G(a_L) < k: b below a_L
+        S.m0 = C;
+        S.n = c;
+        S.top = e_hi;
+        S.P_top = U;
+        S.bot = e_lo;
+        S.Q_bot = Vn;
+        S.klo = B.kmin[j];
+        S.khi = B.kmax[j];
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(BS_BLOCK, 1)
+band_select_kernel(const float *__restrict__ band_all, int64_t band_cap, double k, double t, double inv_t,
+                   Ctl *ctl_all, int32_t round2) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    BinSums &s_bins = *reinterpret_cast<BinSums *>(dsm);
+    __shared__ Aff s_scan[3 * BS_NW];
+    __shared__ unsigned s_hit;
+    __shared__ SubBand s_sb;
+    __shared__ double s_tab[32];
+    __shared__ float s_buf[GATHER_CAP];
+    __shared__ unsigned s_got;
+    exp2_table_init(s_tab);
+    pdl_enter();
+
+    const int tid = threadIdx.x;
+    Ctl *ctl = ctl_all + blockIdx.x;
+    if (round2 && !ctl->widened) return;   // the widening round did not start
+    const unsigned long long cb = ctl->c_band;
+    if (cb > (unsigned long long)band_cap) {
+        if (tid == 0) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
+        return;
+    }
+    const double s2d = inv_t * LOG2E;
+    const unsigned long long c_R = ctl->c_R;
+    if (tid == 0) {
+        s_sb.m0 = c_R;
+        s_sb.n = cb;
+        s_sb.top = (double)ctl->a_R;
+        s_sb.P_top = ctl->S_R;
+        s_sb.bot = (double)ctl->a_L;
+        s_sb.Q_bot = ctl->S_L;
+        s_sb.klo = ~ctl->band_kinv;   // largest band score
+        s_sb.khi = ctl->band_kmax;    // smallest band score
+        s_got = 0u;
+    }
+    __syncthreads();   // s_tab, s_sb
+    const float *src = band_all + (int64_t)blockIdx.x * band_cap;
+    int64_t nsrc = (int64_t)cb;
+    bool first = true, gathered = false;
+    for (int it = 0; it < 4; ++it) {   // four steps reach a single key
+        if (s_sb.n == 0 || s_sb.klo >= s_sb.khi) break;
+        if (!gathered && s_sb.n <= (unsigned long long)GATHER_CAP) {   // later steps sweep a copy
+            const uint32_t klo = s_sb.klo, khi = s_sb.khi;
+            for (int64_t i = tid; i < nsrc; i += BS_BLOCK) {
+                const float x = src[i];
+                const uint32_t kk = desc_key(x);
+                if (kk >= klo && kk <= khi) {
+                    const unsigned slot = atomicAdd(&s_got, 1u);
+                    if (slot < (unsigned)GATHER_CAP) s_buf[slot] = x;
+                }
+            }
+            __syncthreads();
+            src = s_buf;
+            nsrc = min(s_got, (unsigned)GATHER_CAP);   // the band's count by construction
+            gathered = true;
+        }
+        band_level(src, nsrc, s_sb, s_bins, s_scan, &s_hit, s2d, k, s_tab, first ? &ctl->status : nullptr);
+        first = false;
+    }
+    if (tid != 0) return;
+    const SubBand S = s_sb;
+    const int64_t above = (int64_t)(S.m0 - c_R);   // band scores above the final band
+    if (S.n == 0) {   // no score in [bot, top): one interval
+        const double ed = link_exp((S.top - S.bot) * s2d, s_tab);
+        const double m0 = (double)S.m0;
+        const double Gt = m0 - 0.5 * S.P_top + 0.5 * ed * S.Q_bot;
+        const double Gb = m0 - 0.5 * ed * S.P_top + 0.5 * S.Q_bot;
+        if (first && (!(Gt < k) || !(Gb >= k))) atomicOr(&ctl->status, ST_NO_ROOT);
+        ctl->b = solve_interval(S.top, S.bot, m0, S.P_top, S.Q_bot, ed, k, t);
+        ctl->j_star = above - 1;
+        return;
+    }
+    // one value, of any count (klo == khi once the loop ends)
+    bool at_or_above = false;
+    ctl->b = solve_equal_run_values((double)desc_key_to_float(S.klo), (double)S.n, (double)S.m0, S.top, S.P_top,
+                                    S.bot, S.Q_bot, k, t, &at_or_above);
+    ctl->j_star = at_or_above ? above + (int64_t)S.n - 1 : above - 1;
+}
+
+cudaError_t launch_band_select(const float *band, int64_t rows, double k, double t, Ctl *ctl, int64_t band_cap,
+                               int32_t round2, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(band_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)sizeof(BinSums));
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    return launch_k(band_select_kernel, (unsigned)rows, BS_BLOCK, sizeof(BinSums), st, band, band_cap, k, t,
+                    1.0 / t, ctl, round2);
+}
+
+}  // namespace lapsum

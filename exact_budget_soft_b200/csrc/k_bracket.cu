@@ -730,7 +730,8 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
             else           a.SL += exp2_neg((E.daL - (double)x) * E.s2d, E.tab);
         }
     }
-    if (!__any_sync(FULL, band_m != 0)) return;
+    uint32_t band_any = __reduce_or_sync(FULL, band_m);   // components with a band score in some lane
+    if (!band_any) return;
     if (BANDTERMS) {   // the band scores' two certification terms
         uint32_t m = band_m;
         while (__any_sync(FULL, m != 0)) {
@@ -744,11 +745,11 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
     }
     if (!CERT) {   // the band scores into the CTA's queue
         const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        while (band_any) {
+            const int i = __ffs(band_any) - 1;
+            band_any &= band_any - 1;
             const bool inb = (band_m >> i) & 1u;
             const unsigned m = __ballot_sync(FULL, inb);
-            if (!m) continue;
             const int leader = __ffs(m) - 1;
             unsigned base = 0;
             if (lane == leader) base = atomicAdd(s_bn, (unsigned)__popc(m));

@@ -1,8 +1,7 @@
 // k_radix.cu -- device-wide sort and locate-scan for rows too long for one
 // CTA: the full-sort solver of "Fast LapSum: Exact Differentiable Top-k at
-// Million Scale" (technical summary section 2.2) on a whole row (the fallback
-// of the abstract, when certification fails) or on a band of the bracketing
-// path (step 3) that exceeds the one-CTA capacity.
+// Million Scale" (technical summary section 2.2) on a whole row: the full-sort
+// path for long rows, and the fallback of the abstract when certification fails.
 //
 // Sort: keys-only LSD radix sort of the descending-order uint32 keys, 8-bit
 // digits, in one cooperative kernel (radix_sort_kernel, described below).
@@ -10,9 +9,8 @@
 // prefix/suffix scans, then one CTA narrows the crossing down chunk -> tile ->
 // value and takes the closed-form root.
 //
-// The host never learns the band size or the certification verdict: every
-// kernel reads its element count and its gate from the control block and
-// returns at once when it has nothing to do.
+// The host never learns the certification verdict: the fallback sort reads its
+// gate from each row's control block and skips the rows with nothing to do.
 #include <climits>
 #include <cstdint>
 
@@ -35,35 +33,16 @@ constexpr int HB = 256;             // histogram kernel threads
 
 // Element count behind a gate; < 0 means "nothing to do".
 __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
-    const Ctl *c = A.ctl;
-    if (A.gate == GATE_BAND) {
-        if (c->path != 2) return -1;
-        if (A.round2 && !c->widened) return -1;
-        const unsigned long long cb = c->c_band;
-        if (cb <= (unsigned long long)A.small_cap || cb > (unsigned long long)A.cap) return -1;
-        if (band_tied(c)) return -1;   // one tied value: the band solver takes it in closed form
-        return (int64_t)cb;
-    }
-    if (A.gate == GATE_FALLBACK) {
-        if (c->verdict != 0) return -1;
-    }
+    if (A.gate == GATE_FALLBACK && A.ctl->verdict != 0) return -1;
     return A.n_host;
 }
 
-// n copies of one value c, between the seeds of the locate step (a row whose
-// scores are all equal, or the band of one tied level): closed form.
+// n copies of one value c (a row whose scores are all equal): closed form.
 __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
     Ctl *ctl = A.ctl;
-    double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
-    if (A.gate == GATE_BAND) {
-        m0 = (double)ctl->c_R;
-        top = (double)ctl->a_R;
-        P_top = ctl->S_R;
-        bot = (double)ctl->a_L;
-        Q_bot = ctl->S_L;
-    }
     bool above = false;
-    ctl->b = solve_equal_run_values((double)A.src[0], (double)n, m0, top, P_top, bot, Q_bot, A.k, A.t, &above);
+    ctl->b = solve_equal_run_values((double)A.src[0], (double)n, 0.0, CUDART_INF, 0.0, -CUDART_INF, 0.0, A.k,
+                                    A.t, &above);
     ctl->j_star = above ? n - 1 : -1;
     if (A.gate == GATE_FALLBACK) ctl->fallback_ran = 1;
 }
@@ -239,17 +218,8 @@ struct ChunkRec {
 struct Seeds {   // what lies above and below the sorted values
     double m0, top, P_top, bot, Q_bot;
 };
-__device__ __forceinline__ Seeds locate_seeds(const SortArgs &A) {
-    Seeds z{0.0, CUDART_INF, 0.0, -CUDART_INF, 0.0};
-    if (A.gate == GATE_BAND) {
-        const Ctl *c = A.ctl;
-        z.m0 = (double)c->c_R;
-        z.top = (double)c->a_R;
-        z.P_top = c->S_R;
-        z.bot = (double)c->a_L;
-        z.Q_bot = c->S_L;
-    }
-    return z;
+__device__ __forceinline__ Seeds locate_seeds(const SortArgs &) {
+    return Seeds{0.0, CUDART_INF, 0.0, -CUDART_INF, 0.0};   // a whole row: nothing above or below
 }
 
 // Step 1 for one CTA: its tiles' records and its chunk record.  s_t: room for a

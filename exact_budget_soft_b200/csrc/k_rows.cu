@@ -14,8 +14,8 @@
 //    found by a max-reduction and re-scanned lane-per-element by one warp, and
 //    the closed-form root gives b;
 //  * the same CTA streams its row again to write p (the row is L2-resident).
-// The band mode solves the sorted band of the bracketing path with the tail
-// sums as seeds (same page, step 3 "exact solve on the band only").
+// The band of the bracketing path goes to k_band.cu, which narrows it first
+// and hands only the part holding b to the same block sort and scan.
 #include <cstdint>
 
 #include "lapsum_device.cuh"
@@ -24,11 +24,10 @@
 
 namespace lapsum {
 
-template <int BLOCK, int KPT, bool BAND>
+template <int BLOCK, int KPT>
 __global__ void __launch_bounds__(BLOCK, 1)
 rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, double t, double inv_t,
-                float *__restrict__ p_out, double *__restrict__ b_out, Ctl *ctl, int64_t band_cap,
-                int64_t band_lo, int32_t round2) {
+                float *__restrict__ p_out, double *__restrict__ b_out, Ctl *ctl) {
     using C = RowCfg<BLOCK, KPT>;
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);
@@ -41,53 +40,10 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     pdl_enter();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int n;
-    const float *row;
-    double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
-    if (BAND) {   // one CTA per row of a batch: its band buffer and control block
-        ctl += blockIdx.x;
-        if (round2 && !ctl->widened) return;   // the widening round did not start
-        unsigned long long cb = ctl->c_band;
-        if (cb > (unsigned long long)band_cap) {
-            if (tid == 0) atomicOr(&ctl->status, ST_BAND_OVERFLOW);
-            return;
-        }
-        if (band_tied(ctl)) {   // one tied value, of any count: closed form (first variant)
-            if (band_lo == 0 && tid == 0) {
-                bool above = false;
-                ctl->b = solve_equal_run_values((double)desc_key_to_float(ctl->band_kmax), (double)cb,
-                                                (double)ctl->c_R, (double)ctl->a_R, ctl->S_R, (double)ctl->a_L,
-                                                ctl->S_L, k, t, &above);
-                ctl->j_star = above ? (int64_t)cb - 1 : -1;
-            }
-            return;
-        }
-        if (band_lo > 0 && cb <= (unsigned long long)band_lo) return;   // a smaller variant takes it
-        if (cb > (unsigned long long)C::CAP) return;   // the device-wide sort takes it
-        n = (int)cb;
-        row = scores + (int64_t)blockIdx.x * band_cap;
-        m0 = (double)ctl->c_R;
-        top = (double)ctl->a_R;
-        P_top = ctl->S_R;
-        bot = (double)ctl->a_L;
-        Q_bot = ctl->S_L;
-    } else {
-        n = (int)n_arg;
-        row = scores + (int64_t)blockIdx.x * n_arg;
-    }
-
+    const int n = (int)n_arg;
+    const float *row = scores + (int64_t)blockIdx.x * n_arg;
+    const double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
     __syncthreads();   // s_tab
-    if (n == 0) {   // band mode only: one interval [a_L, a_R] with no score inside
-        if (tid == 0) {
-            double ed = (top == CUDART_INF || bot == -CUDART_INF) ? 0.0 : exp((bot - top) * inv_t);
-            double Gt = m0 - 0.5 * P_top + 0.5 * ed * Q_bot;
-            double Gb = m0 - 0.5 * ed * P_top + 0.5 * Q_bot;
-            if (!(Gt < k) || !(Gb >= k)) atomicOr(&ctl->status, ST_NO_ROOT);
-            ctl->b = solve_interval(top, bot, m0, P_top, Q_bot, ed, k, t);
-            ctl->j_star = -1;
-        }
-        return;
-    }
 
     // ---- load keys (warp-striped), pad with the largest key (sorts last)
     uint32_t key[KPT];
@@ -117,24 +73,18 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     if (__syncthreads_or(bad) && tid == 0 && ctl) atomicOr(&ctl->status, ST_NONFINITE);
     const uint32_t diff = s_and ^ s_or;
 
-    block_radix_sort<BLOCK, KPT, BAND>(key, s_keys, s_hist, s_dbase, diff);
+    block_radix_sort<BLOCK, KPT>(key, s_keys, s_hist, s_dbase, diff);
 
     int64_t jstar = 0;
     int32_t *st = ctl ? &ctl->status : nullptr;
     double b = block_scan_solve<BLOCK, KPT>(s_keys, n, k, t, inv_t, m0, top, P_top, bot, Q_bot,
-                                            s_hist, (BAND || blockIdx.x == 0) ? &jstar : nullptr, st, s_tab);
+                                            s_hist, blockIdx.x == 0 ? &jstar : nullptr, st, s_tab);
     if (tid == 0) {
         s_b = b;
-        if (BAND) {
-            ctl->b = b;
-            ctl->j_star = jstar;
-        } else {
-            b_out[blockIdx.x] = b;
-            if (blockIdx.x == 0 && ctl) { ctl->b = b; ctl->j_star = jstar; }
-        }
+        b_out[blockIdx.x] = b;
+        if (blockIdx.x == 0 && ctl) { ctl->b = b; ctl->j_star = jstar; }
     }
     __syncthreads();
-    if (BAND) return;
 
     // ---- p = F((r - b)/t) for the row
     b = s_b;
@@ -268,12 +218,11 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
 }
 
 // ------------------------------------------------------------ launchers --
-template <int BLOCK, int KPT, bool BAND>
+template <int BLOCK, int KPT>
 static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n, double k, double t,
-                                   float *p, double *b, Ctl *ctl, int64_t band_cap, int64_t band_lo,
-                                   int32_t round2, cudaStream_t st) {
+                                   float *p, double *b, Ctl *ctl, cudaStream_t st) {
     using C = RowCfg<BLOCK, KPT>;
-    auto kern = rowsolve_kernel<BLOCK, KPT, BAND>;
+    auto kern = rowsolve_kernel<BLOCK, KPT>;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -281,34 +230,15 @@ static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n,
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl, band_cap,
-                    band_lo, round2);
+    return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl);
 }
 
 int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
 
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st) {
-    if (n <= RowCfg<256, 16>::CAP)
-        return launch_rowsolve<256, 16, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, 0, st);
-    return launch_rowsolve<1024, 32, false>(scores, rows, n, k, t, p, b, ctl, 0, 0, 0, st);
-}
-
-// Three variants, each gated on the band size the streaming pass counted (the
-// sort inside a CTA costs its capacity, not the band): bands of up to 4096
-// scores (and tied or empty bands) in a 256-thread CTA, up to 16384 in a
-// 512-thread CTA, up to 32768 in a 1024-thread CTA.  A launch whose gate is
-// closed returns at once.
-cudaError_t launch_rowsolve_band(const float *band, int64_t rows, double k, double t, Ctl *ctl,
-                                 int64_t band_cap, int32_t round2, cudaStream_t st) {
-    cudaError_t e =
-        launch_rowsolve<256, 16, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap, 0, round2, st);
-    if (e != cudaSuccess || band_cap <= RowCfg<256, 16>::CAP) return e;
-    e = launch_rowsolve<512, 32, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap,
-                                       RowCfg<256, 16>::CAP, round2, st);
-    if (e != cudaSuccess || band_cap <= RowCfg<512, 32>::CAP) return e;
-    return launch_rowsolve<1024, 32, true>(band, rows, 0, k, t, nullptr, nullptr, ctl, band_cap,
-                                           RowCfg<512, 32>::CAP, round2, st);
+    if (n <= RowCfg<256, 16>::CAP) return launch_rowsolve<256, 16>(scores, rows, n, k, t, p, b, ctl, st);
+    return launch_rowsolve<1024, 32>(scores, rows, n, k, t, p, b, ctl, st);
 }
 
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,

@@ -165,7 +165,6 @@ SortArgs sort_args(Workspace *w, const float *src, int64_t n, int64_t cap, int32
     A.ctl = w->ctl;
     A.gate = gate;
     A.spin_cap = spin_cap;
-    A.small_cap = rowsolve_capacity();
     A.rows = 1;
     A.src_stride = 0;
     return A;
@@ -412,18 +411,7 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
         { Launch L(r2 ? "widen_sample" : "sample", st); LAPSUM_TRY(launch_sample(Q, st)); }
         { Launch L(r2 ? "widen_select" : "select", st); LAPSUM_TRY(launch_select(Q, st)); }
         { Launch L(r2 ? "widen_stream_pass" : "stream_pass", st); LAPSUM_TRY(launch_stream_pass(Q, st)); }
-        {
-            Launch L(r2 ? "widen_band_rowsolve" : "band_rowsolve", st);
-            g_launches += Q.band_cap > 16384 ? 2 : (Q.band_cap > 4096 ? 1 : 0);   // size-gated variants
-            LAPSUM_TRY(launch_rowsolve_band(w->band, rows, k, t, w->ctl, Q.band_cap, Q.round2, st));
-        }
-        if (Q.band_cap > rowsolve_capacity()) {
-            SortArgs A = sort_args(w, w->band, 0, Q.band_cap, GATE_BAND, spin_cap, k, t);
-            A.round2 = Q.round2;
-            A.rows = rows;
-            A.src_stride = Q.band_cap;
-            { Launch L(r2 ? "widen_band_radix_sort" : "band_radix_sort", st); LAPSUM_TRY(launch_radix_sort(A, k, t, st)); }
-        }
+        { Launch L(r2 ? "widen_band_select" : "band_select", st); LAPSUM_TRY(launch_band_select(w->band, rows, k, t, w->ctl, Q.band_cap, Q.round2, st)); }
         if (!Q.fused_cert) { Launch L(r2 ? "widen_certify" : "certify", st); LAPSUM_TRY(launch_certify(Q, st)); }
         return LAPSUM_OK;
     };

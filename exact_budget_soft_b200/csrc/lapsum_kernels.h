@@ -47,8 +47,9 @@ inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, si
 int rowsolve_capacity();
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st);
-cudaError_t launch_rowsolve_band(const float *band, int64_t rows, double k, double t, Ctl *ctl,
-                                 int64_t band_cap, int32_t round2, cudaStream_t st);
+// band solve of the bracketing path, one CTA per row (k_band.cu)
+cudaError_t launch_band_select(const float *band, int64_t rows, double k, double t, Ctl *ctl, int64_t band_cap,
+                               int32_t round2, cudaStream_t st);
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
                           int64_t n, double t, float *grad, cudaStream_t st);
 
@@ -70,12 +71,12 @@ cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, in
                              const Ctl *ctl, float *grad, cudaStream_t st);
 
 // device-wide radix sort + locate-scan (k_radix.cu)
-enum Gate : int32_t { GATE_ALWAYS = 0, GATE_BAND = 1, GATE_FALLBACK = 2 };
+enum Gate : int32_t { GATE_ALWAYS = 0, GATE_FALLBACK = 2 };
 struct SortArgs {
     const float *src;          // fp32 scores (keys made on the fly) of row 0
     int64_t src_stride;        // floats from one row's source to the next
     int64_t rows;              // rows the kernel walks, one after another (each gated)
-    int64_t n_host;            // element count when gate != GATE_BAND
+    int64_t n_host;            // element count
     int64_t cap;               // upper bound of the element count (grid sizing)
     uint32_t *keys[2];         // ping-pong key buffers [cap]
     unsigned long long *hist;  // [4][256]
@@ -83,9 +84,7 @@ struct SortArgs {
     double *tilebuf;           // locate per-tile data
     Ctl *ctl;
     int32_t gate;
-    int32_t round2;            // band gate of the widening round: runs only once it started
     int32_t spin_cap;          // grid-barrier polls before a wait gives up
-    int32_t small_cap;         // band gate: sizes <= small_cap are solved in one CTA
     double k, t;               // budget and temperature (all-equal shortcut)
 };
 int sort_grid_max();

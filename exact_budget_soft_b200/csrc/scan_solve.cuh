@@ -264,9 +264,9 @@ __device__ double block_scan_solve(const uint32_t *s_keys, int n, double k, doub
             }
         }
         if (lane == 0) {
-            if (jstar == -1 && U != CUDART_INF) {
-                // G(top) > k: the root lies above the band (bracket missed)
-                if (status) atomicOr(status, ST_NO_ROOT);
+            if (jstar == -1 && U != CUDART_INF) {   // b between c_0 and top: needs G(top) <= k
+                const double Gt = A - 0.5 * PU + 0.5 * ed * QL;
+                if (Gt > k && status) atomicOr(status, ST_NO_ROOT);
             }
             if (jstar == n - 1 && L != -CUDART_INF) {
                 double Gb = (m0 + n) - 0.5 * ed * PU + 0.5 * Q_bot;
