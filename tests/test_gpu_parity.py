@@ -162,9 +162,9 @@ def test_pixels1m_workload(L, orc):
 
 
 @pytest.mark.parametrize("certify", [0, 1])
-def test_bracketing_large_band_device_sort(L, orc, certify):
-    # a small sample leaves a wide bracket: the band (~1e5 scores, untied) is
-    # too long for one CTA and goes through the device-wide sort and locate
+def test_bracketing_large_band(L, orc, certify):
+    # a small sample leaves a wide bracket: the band (~1e5 scores, untied) takes
+    # narrowing steps over the band buffer before its copy in shared memory
     n = (1 << 21) + 12345
     r, g = W.small_case("laplace", 1, n, seed=12)
     k, t, s = n / 10.0, 0.05, 4096
@@ -450,9 +450,10 @@ def test_batched_rows_all_fall_back(L, orc):
 
 
 @pytest.mark.parametrize("s,lo,hi", [(65536, 0, 4096), (16384, 4096, 16384), (2048, 16384, 32768)])
-def test_band_solver_variants(L, orc, s, lo, hi):
-    # the sample size sets the band's size: each one-CTA band solver variant
-    # (<= 4096, <= 16384, <= 32768 scores) solves one of these bands
+def test_band_select_sizes(L, orc, s, lo, hi):
+    # the sample size sets the band's size: a band of at most 4096 scores is
+    # copied to shared memory before the first narrowing step, a longer one is
+    # narrowed from the band buffer first
     n = 1 << 20
     r, g = W.small_case("normal", 1, n, seed=16)
     k, t = n / 100.0, 0.05
@@ -462,6 +463,64 @@ def test_band_solver_variants(L, orc, s, lo, hi):
     p, b, st, grad = run(L, r, k, t, opts=L.options(sample_size=s), g_np=g)
     assert st["rc"] == 0 and st["verdict"] == 1 and st["c_band"] == cert["c_band"]
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+@pytest.mark.parametrize("certify", [0, 1])
+def test_band_select_band_across_zero(L, orc, certify):
+    # k = n/2 puts the band around 0: its keys span both signs (a 31-bit key
+    # range), which takes the full four narrowing steps
+    n = 1 << 20
+    r, g = W.small_case("normal", 1, n, seed=19)
+    k, t = n / 2.0, 0.05
+    p, b, st, grad = run(L, r, k, t, opts=L.options(certify=certify), g_np=g)
+    assert st["rc"] == 0 and st["path"] == 2 and st["verdict"] == 1
+    plan = L.bracket_plan(n, k)
+    cert = check_bracket_integers(orc, r[0], k, t, st, 0, plan["s"], 1e-6)
+    band = r[0][(r[0] >= np.float32(st["a_L"])) & (r[0] < np.float32(st["a_R"]))]
+    assert band.min() < 0.0 < band.max() and cert["c_band"] > 4096
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
+
+
+def test_band_select_tied_runs_longer_than_the_copy(L, orc):
+    # 256 tied levels of ~16k scores each; a small sample (4096) widens the
+    # bracket so the band holds several whole levels, and the narrowing ends on
+    # one level (more scores than the shared-memory copy holds) or on the gap
+    # between two, both in closed form
+    n = 1 << 22
+    r, g = W.small_case("levels256_desc", 1, n, seed=20)
+    for k in (2.5 * n / 256, 40.0 * n / 256):
+        p, b, st, grad = run(L, r, k, 0.02, opts=L.options(sample_size=4096), g_np=g)
+        assert st["rc"] == 0 and st["path"] == 2 and st["verdict"] == 1
+        band = r[0][(r[0] >= np.float32(st["a_L"])) & (r[0] < np.float32(st["a_R"]))]
+        assert np.unique(band).size >= 2 and band.size > 4096
+        check_row(orc, r[0], g[0], k, 0.02, p[0], b[0], grad[0], exact_sum=False)
+
+
+def test_band_select_root_above_the_band(L, orc):
+    # 3000 scores in [1, 1.1] over a N(0, 0.1^2) bulk, k = 3010, t = 0.2: b lies
+    # above every score of the cluster, and with some seeds the bracket's upper
+    # end lies above b with no band score in [b, a_R) -- the root is in the
+    # band's top interval, a regular case (no NO_ROOT)
+    n = 1 << 20
+    rng = np.random.default_rng(21)
+    r = (0.1 * rng.standard_normal(n)).astype(np.float32)
+    r[:3000] = rng.uniform(1.0, 1.1, 3000).astype(np.float32)
+    rng.shuffle(r)
+    g = rng.standard_normal(n).astype(np.float32)
+    k, t = 3010.0, 0.2
+    bref = orc.solve(r, k, t, method=1)
+    plan = L.bracket_plan(n, k)
+
+    def top_interval(seed):
+        br = orc.bracket(r, k, t, seed, plan["s"], 1e-6)
+        band = r[(r >= br["a_L"]) & (r < br["a_R"])]
+        return br["a_L"] <= bref < br["a_R"] and band.size > 0 and float(band.max()) < bref
+
+    seed = next(sd for sd in range(64) if top_interval(sd))
+    p, b, st, grad = run(L, r[None, :], k, t, opts=L.options(seed=seed), g_np=g[None, :])
+    assert st["rc"] == 0 and st["verdict"] == 1 and st["fallback"] == 0
+    assert not (st["status"] & 8)
+    check_row(orc, r, g, k, t, p[0], b[0], grad[0])
 
 
 # ------------------------------------------------------- bracketing edges --
