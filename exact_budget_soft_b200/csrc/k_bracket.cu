@@ -659,10 +659,54 @@ __device__ __forceinline__ void oob_cheap(float x, int bit, const Ends &E, OobAc
     band_m |= inb ? (1u << bit) : 0u;
 }
 
+// The rare scores of a general chunk -- near an end (fp64 tail term) or in the
+// band (queue slot, or the two certification terms) -- are staged in a per-warp
+// queue in shared memory and handled 32 at a time, one per lane, so a warp no
+// longer loops as often as its busiest lane has such scores.
+constexpr int SQ = 64;   // staged scores per warp (below 32 between chunks, at most 32 added)
+
+// Up to 32 staged scores, one per lane (lanes >= cnt idle).
+template <int MODE>
+__device__ __forceinline__ void special_batch(const float *q, int cnt, const Ends &E, OobAcc &a,
+                                              const BracketParams &P, unsigned long long cap, int lane,
+                                              float *s_bq, unsigned *s_bn) {
+    constexpr bool CERT = MODE == OOB_CERT;
+    constexpr bool BANDTERMS = MODE != OOB_STREAM;
+    const bool act = lane < cnt;
+    const float x = act ? q[lane] : 0.f;
+    const bool above = act && x >= E.aR, below = act && x < E.aL;
+    const bool inb = act && !above && !below;
+    {   // a score out of the band was staged for its fp64 tail term
+        const double w = above ? ((double)x - E.daR) * E.s2d : (below ? (E.daL - (double)x) * E.s2d : 0.0);
+        const double e = exp2_neg(w, E.tab);
+        if (above) a.SR += e;
+        if (below) a.SL += e;
+    }
+    if (BANDTERMS && inb) {   // the band score's two certification terms
+        tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
+        tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
+    }
+    if (!CERT) {   // the band scores into the CTA's queue
+        const unsigned m = __ballot_sync(FULL, inb);
+        if (m) {
+            const int leader = __ffs(m) - 1;
+            unsigned base = 0;
+            if (lane == leader) base = atomicAdd(s_bn, (unsigned)__popc(m));
+            const unsigned slot = __shfl_sync(FULL, base, leader) + __popc(m & ((1u << lane) - 1u));
+            if (inb) {
+                a.kmax = max(a.kmax, desc_key(x));
+                a.kinv = max(a.kinv, ~desc_key(x));
+                if (slot < (unsigned)BQ) s_bq[slot] = x;
+            }
+            band_push(x, inb && slot >= (unsigned)BQ, P.band, cap, &P.ctl->c_band, lane, a);   // queue full
+        }
+    }
+}
+
 template <int MODE>
 __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, const Ends &E, OobAcc &a,
                                           const BracketParams &P, unsigned long long cap, int lane,
-                                          float *s_bq, unsigned *s_bn) {
+                                          float *s_bq, unsigned *s_bn, float *sq, unsigned &sq_n) {
     constexpr bool CERT = MODE == OOB_CERT;
     constexpr bool BANDTERMS = MODE != OOB_STREAM;
     const float mx = max_nan(max_nan(max_nan(v0.x, v0.y), max_nan(v0.z, v0.w)),
@@ -720,8 +764,31 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
     oob_cheap<MODE>(v1.y, 5, E, a, near_m, band_m);
     oob_cheap<MODE>(v1.z, 6, E, a, near_m, band_m);
     oob_cheap<MODE>(v1.w, 7, E, a, near_m, band_m);
-    // fp64 tail terms of scores near an end: each warp loops as often as its
-    // busiest lane has such scores
+    const uint32_t sp = near_m | band_m;
+    const unsigned cnt = __popc(sp);
+    unsigned inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned p = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += p;
+    }
+    const unsigned total = __shfl_sync(FULL, inc, 31);
+    if (total == 0) return;
+    if (total <= 32) {   // stage them; a full batch of 32 goes at once
+        unsigned pos = sq_n + inc - cnt;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if ((sp >> i) & 1u) sq[pos++] = pick8(v0, v1, i);
+        sq_n += total;
+        __syncwarp();
+        if (sq_n >= 32) {
+            sq_n -= 32;
+            special_batch<MODE>(sq + sq_n, 32, E, a, P, cap, lane, s_bq, s_bn);
+        }
+        return;
+    }
+    // a dense chunk: fp64 tail terms of scores near an end, each warp looping as
+    // often as its busiest lane has such scores
     while (__any_sync(FULL, near_m != 0)) {
         if (near_m) {
             const float x = pick8(v0, v1, __ffs(near_m) - 1);
@@ -796,6 +863,7 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     __shared__ double s_red[7 * (SBLOCK / 32)];
     __shared__ double s_tab[32];
     __shared__ float s_bq[CERT ? 1 : BQ];   // sparse band scores of this CTA
+    __shared__ float s_sq[SBLOCK / 32][SQ];   // staged rare scores, per warp
     __shared__ unsigned s_bn;
     __shared__ unsigned long long s_bbase;
     exp2_table_init(s_tab);
@@ -823,10 +891,14 @@ __global__ void __launch_bounds__(SBLOCK, MODE == OOB_STREAM ? SBLOCKS_PER_SM : 
     int64_t done4 = 0;
     if (aligned) {
         const float4 *src[1] = {r4};
+        float *sq = s_sq[threadIdx.x >> 5];
+        unsigned sq_n = 0;   // the same in every lane of a warp
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
             oob_chunk<MODE>(lds128(ch[0] + threadIdx.x), lds128(ch[0] + threadIdx.x + SBLOCK), E, acc, P, cap,
-                            lane, s_bq, &s_bn);
+                            lane, s_bq, &s_bn, sq, sq_n);
         });
+        __syncwarp();
+        if (sq_n) special_batch<MODE>(sq, (int)sq_n, E, acc, P, cap, lane, s_bq, &s_bn);
     }
     // vectors after the last full chunk (whole warps iterate together)
     const int64_t tv = n4 - done4;
