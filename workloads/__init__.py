@@ -57,7 +57,7 @@ WORKLOADS: dict[str, Workload] = {
         Workload("pixels1m", 1, 1_048_576, 210.0, 0.01, "pixel_mix",
                  "bracketing + certification"),
         Workload("laplace1e7", 1, 10_000_000, 100_000.0, 0.05, "laplace",
-                 "bracketing + band sort + certification"),
+                 "bracketing + band select + certification"),
         Workload("levels1e8", 1, 100_000_000, 1_000_000.0, 0.1, "levels256_desc",
                  "bracketing (+ forced full-sort fallback run)"),
         Workload("batch64x1m", 64, 1_048_576, 10_486.0, 0.05, "normal",
