@@ -703,57 +703,72 @@ __device__ __forceinline__ void special_batch(const float *q, int cnt, const End
     }
 }
 
-template <int MODE>
+template <int MODE, bool ADAPT>
 __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, const Ends &E, OobAcc &a,
                                           const BracketParams &P, unsigned long long cap, int lane,
-                                          float *s_bq, unsigned *s_bn, float *sq, unsigned &sq_n) {
+                                          float *s_bq, unsigned *s_bn, float *sq, unsigned &sq_n,
+                                          unsigned &hist, unsigned &tick) {
     constexpr bool CERT = MODE == OOB_CERT;
     constexpr bool BANDTERMS = MODE != OOB_STREAM;
-    const float mx = max_nan(max_nan(max_nan(v0.x, v0.y), max_nan(v0.z, v0.w)),
-                             max_nan(max_nan(v1.x, v1.y), max_nan(v1.z, v1.w)));
-    const float mn = fminf(fminf(fminf(v0.x, v0.y), fminf(v0.z, v0.w)), fminf(fminf(v1.x, v1.y), fminf(v1.z, v1.w)));
-    const bool fin = mn > -CUDART_INF_F && mx < CUDART_INF_F;
-    // a whole warp on one side (sorted or clustered scores): eight scores at once
-    const bool eq0 = v0.x == v0.y && v0.y == v0.z && v0.z == v0.w;
-    const bool eq1 = v1.x == v1.y && v1.y == v1.z && v1.z == v1.w;
-    if (__all_sync(FULL, mx < E.farL && fin)) {            // far below a_L: counts only
-        if (CERT) a.cB += 8; else a.cL += 8;
-        return;
+    // ADAPT: hist records which of the warp's last 16 chunks took the general
+    // path.  When 12 or more did (random score order), the fast-path tests are
+    // skipped, except on every 16th chunk, which keeps the history fresh; every
+    // chunk is correct on the general path.
+    bool try_fast = true;
+    if (ADAPT) {
+        try_fast = __popc(hist & 0xffffu) < 12 || (tick & 15u) == 0u;
+        hist <<= 1;
+        ++tick;
     }
-    if (__all_sync(FULL, mx < E.midL && fin)) {            // below a_L, fp32 terms
-        if (CERT) a.cB += 8; else a.cL += 8;
-        a.SL2 += ((ex2_ftz((v0.x - E.aL) * E.s2) + ex2_ftz((v0.y - E.aL) * E.s2)) +
-                  (ex2_ftz((v0.z - E.aL) * E.s2) + ex2_ftz((v0.w - E.aL) * E.s2))) +
-                 ((ex2_ftz((v1.x - E.aL) * E.s2) + ex2_ftz((v1.y - E.aL) * E.s2)) +
-                  (ex2_ftz((v1.z - E.aL) * E.s2) + ex2_ftz((v1.w - E.aL) * E.s2)));
-        return;
-    }
-    if (__all_sync(FULL, mx < E.aL && fin)) {              // below a_L, some near it
-        if (CERT) a.cB += 8; else a.cL += 8;
-        tier4<false>(v0, eq0, E.aL, E.daL, E, a.SL, a.SL2);
-        tier4<false>(v1, eq1, E.aL, E.daL, E, a.SL, a.SL2);
-        return;
-    }
-    if (__all_sync(FULL, mn >= E.aR && fin)) {             // at or above a_R
-        if (CERT) { a.cL += 8; a.cR += 8; } else a.cR += 8;
-        tier4<true>(v0, eq0, E.aR, E.daR, E, a.SR, a.SR2);
-        tier4<true>(v1, eq1, E.aR, E.daR, E, a.SR, a.SR2);
-        return;
-    }
-    if (__all_sync(FULL, mn >= E.aL && mx < E.aR && fin)) {   // inside the band
-        if (BANDTERMS) {
-            if (CERT) a.cL += 8;
-            tier4<true>(v0, eq0, E.aL, E.daL, E, a.hL, a.hL2);
-            tier4<false>(v0, eq0, E.aR, E.daR, E, a.lR, a.lR2);
-            tier4<true>(v1, eq1, E.aL, E.daL, E, a.hL, a.hL2);
-            tier4<false>(v1, eq1, E.aR, E.daR, E, a.lR, a.lR2);
+    if (try_fast) {
+        const float mx = max_nan(max_nan(max_nan(v0.x, v0.y), max_nan(v0.z, v0.w)),
+                                 max_nan(max_nan(v1.x, v1.y), max_nan(v1.z, v1.w)));
+        const float mn = fminf(fminf(fminf(v0.x, v0.y), fminf(v0.z, v0.w)),
+                               fminf(fminf(v1.x, v1.y), fminf(v1.z, v1.w)));
+        const bool fin = mn > -CUDART_INF_F && mx < CUDART_INF_F;
+        // a whole warp on one side (sorted or clustered scores): eight scores at once
+        const bool eq0 = v0.x == v0.y && v0.y == v0.z && v0.z == v0.w;
+        const bool eq1 = v1.x == v1.y && v1.y == v1.z && v1.z == v1.w;
+        if (__all_sync(FULL, mx < E.farL && fin)) {            // far below a_L: counts only
+            if (CERT) a.cB += 8; else a.cL += 8;
+            return;
         }
-        if (!CERT) {
-            band_push4(v0, 0xF, P.band, cap, &P.ctl->c_band, lane, a);
-            band_push4(v1, 0xF, P.band, cap, &P.ctl->c_band, lane, a);
+        if (__all_sync(FULL, mx < E.midL && fin)) {            // below a_L, fp32 terms
+            if (CERT) a.cB += 8; else a.cL += 8;
+            a.SL2 += ((ex2_ftz((v0.x - E.aL) * E.s2) + ex2_ftz((v0.y - E.aL) * E.s2)) +
+                      (ex2_ftz((v0.z - E.aL) * E.s2) + ex2_ftz((v0.w - E.aL) * E.s2))) +
+                     ((ex2_ftz((v1.x - E.aL) * E.s2) + ex2_ftz((v1.y - E.aL) * E.s2)) +
+                      (ex2_ftz((v1.z - E.aL) * E.s2) + ex2_ftz((v1.w - E.aL) * E.s2)));
+            return;
         }
-        return;
+        if (__all_sync(FULL, mx < E.aL && fin)) {              // below a_L, some near it
+            if (CERT) a.cB += 8; else a.cL += 8;
+            tier4<false>(v0, eq0, E.aL, E.daL, E, a.SL, a.SL2);
+            tier4<false>(v1, eq1, E.aL, E.daL, E, a.SL, a.SL2);
+            return;
+        }
+        if (__all_sync(FULL, mn >= E.aR && fin)) {             // at or above a_R
+            if (CERT) { a.cL += 8; a.cR += 8; } else a.cR += 8;
+            tier4<true>(v0, eq0, E.aR, E.daR, E, a.SR, a.SR2);
+            tier4<true>(v1, eq1, E.aR, E.daR, E, a.SR, a.SR2);
+            return;
+        }
+        if (__all_sync(FULL, mn >= E.aL && mx < E.aR && fin)) {   // inside the band
+            if (BANDTERMS) {
+                if (CERT) a.cL += 8;
+                tier4<true>(v0, eq0, E.aL, E.daL, E, a.hL, a.hL2);
+                tier4<false>(v0, eq0, E.aR, E.daR, E, a.lR, a.lR2);
+                tier4<true>(v1, eq1, E.aL, E.daL, E, a.hL, a.hL2);
+                tier4<false>(v1, eq1, E.aR, E.daR, E, a.lR, a.lR2);
+            }
+            if (!CERT) {
+                band_push4(v0, 0xF, P.band, cap, &P.ctl->c_band, lane, a);
+                band_push4(v1, 0xF, P.band, cap, &P.ctl->c_band, lane, a);
+            }
+            return;
+        }
     }
+    if (ADAPT) hist |= 1u;
     // general path: the cheap part for all eight, then the marked ones
     uint32_t near_m = 0, band_m = 0;
     oob_cheap<MODE>(v0.x, 0, E, a, near_m, band_m);
@@ -858,8 +873,11 @@ __device__ __forceinline__ void set_verdict(const BracketParams &P, bool ok, boo
 // at 64 registers; the certification passes keep more accumulators and were
 // measured faster at three (80 registers) on one row and at four on a batch of
 // random-order rows (195 -> 170 us per 256 MB), so the certification pass is
-// built both ways.
-template <int MODE, int MINB = (MODE == OOB_STREAM ? SBLOCKS_PER_SM : 3)>
+// built both ways.  ADAPT: skip the chunk fast-path tests on random-order runs
+// of chunks (oob_chunk); measured faster on the streaming pass and on the
+// batched certification pass, slower (+3%) on the one-row certification pass
+// of sorted scores.
+template <int MODE, int MINB = (MODE == OOB_STREAM ? SBLOCKS_PER_SM : 3), bool ADAPT = (MODE == OOB_STREAM)>
 __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
     const BracketParams P = at_row(Pg, blockIdx.y);
     constexpr bool CERT = MODE == OOB_CERT;
@@ -897,10 +915,10 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
     if (aligned) {
         const float4 *src[1] = {r4};
         float *sq = s_sq[threadIdx.x >> 5];
-        unsigned sq_n = 0;   // the same in every lane of a warp
+        unsigned sq_n = 0, hist = 0, tick = 0;   // the same in every lane of a warp
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
-            oob_chunk<MODE>(lds128(ch[0] + threadIdx.x), lds128(ch[0] + threadIdx.x + SBLOCK), E, acc, P, cap,
-                            lane, s_bq, &s_bn, sq, sq_n);
+            oob_chunk<MODE, ADAPT>(lds128(ch[0] + threadIdx.x), lds128(ch[0] + threadIdx.x + SBLOCK), E, acc, P, cap,
+                            lane, s_bq, &s_bn, sq, sq_n, hist, tick);
         });
         __syncwarp();
         if (sq_n) special_batch<MODE>(sq, (int)sq_n, E, acc, P, cap, lane, s_bq, &s_bn);
@@ -1311,10 +1329,10 @@ cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
     static cudaError_t once = set_smem(oob_kernel<OOB_CERT, 3>, bulk_smem_bytes<1>());
-    static cudaError_t once4 = set_smem(oob_kernel<OOB_CERT, 4>, bulk_smem_bytes<1>());
+    static cudaError_t once4 = set_smem(oob_kernel<OOB_CERT, 4, true>, bulk_smem_bytes<1>());
     if (once != cudaSuccess || once4 != cudaSuccess) return once != cudaSuccess ? once : once4;
     if (P.rows > 1)
-        return launch_k(oob_kernel<OOB_CERT, 4>, row_grid(4, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
+        return launch_k(oob_kernel<OOB_CERT, 4, true>, row_grid(4, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
     return launch_k(oob_kernel<OOB_CERT, 3>, row_grid(3, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_p_pass(const float *r, int64_t rows, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
