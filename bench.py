@@ -40,12 +40,17 @@ EXTRA = ["pixels1m", "laplace1e7"]
 KERNEL_BYTES = {"stream_pass": 4, "certify": 4, "p_pass": 8, "vjp_reduce": 8, "vjp_apply": 12}
 
 
+# The files the streaming kernels (stream, certify, p, vjp) are built from: the
+# DRAM counters in profiles/traffic.json hold only while these are unchanged.
+STREAM_KERNEL_SOURCES = ["k_bracket.cu", "lapsum_device.cuh", "lapsum_kernels.h", "lapsum_internal.h"]
+
+
 def kernel_sources_sha() -> str:
-    import glob
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "exact_budget_soft_b200", "csrc", "*"))):
-        h.update(os.path.basename(f).encode())
+    for name in STREAM_KERNEL_SOURCES:
+        f = os.path.join(ROOT, "exact_budget_soft_b200", "csrc", name)
+        h.update(name.encode())
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 

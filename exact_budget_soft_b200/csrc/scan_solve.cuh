@@ -15,11 +15,7 @@ namespace lapsum {
 __device__ __forceinline__ int spad(int j) { return j + (j >> 5); }
 
 // Lanes of the warp holding the same 8-bit digit: eight ballots, one per bit.
-// UNIFORM: first one vote for a warp that agrees throughout (padding, sorted or
-// tied keys: the mostly-padded band) -- a loss on full rows of random keys.
-template <bool UNIFORM>
 __device__ __forceinline__ unsigned digit_peers(uint32_t d) {
-    if (UNIFORM && __all_sync(FULL, d == __shfl_sync(FULL, d, 0))) return FULL;
     unsigned peers = FULL;
 #pragma unroll
     for (int b = 0; b < 8; ++b) {
@@ -41,7 +37,7 @@ struct RowCfg {
 
 // Block-wide LSD radix sort of warp-striped register keys (ascending).  On
 // return the sorted keys are in s_keys (position j at spad(j)).
-template <int BLOCK, int KPT, bool UNIFORM = false>
+template <int BLOCK, int KPT>
 __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t *s_keys,
                                                  uint32_t *s_hist, uint32_t *s_dbase,
                                                  uint32_t diff) {
@@ -57,19 +53,9 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
         __syncthreads();
         // count: per-warp digit histograms.  Counts need no order: one shared
         // atomic per key (lanes on one counter serialise, the rest run in
-        // parallel).  A mostly uniform warp (band mode: padding) takes one
-        // update per group of equal digits instead.
+        // parallel).
 #pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const uint32_t d = (key[i] >> sh) & 0xffu;
-            if (UNIFORM) {
-                const unsigned peers = digit_peers<true>(d);
-                if (lane == __ffs(peers) - 1) my_hist[d] += __popc(peers);
-                __syncwarp();
-            } else {
-                atomicAdd(&my_hist[d], 1u);
-            }
-        }
+        for (int i = 0; i < KPT; ++i) atomicAdd(&my_hist[(key[i] >> sh) & 0xffu], 1u);
         __syncthreads();
         if (tid < 256) {   // per digit: exclusive prefix over warps, and total
             uint32_t sum = 0;
@@ -102,7 +88,7 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
             const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = digit_peers<UNIFORM>(d);
+            const unsigned peers = digit_peers(d);
             const int leader = __ffs(peers) - 1;
             uint32_t base = 0;
             if (lane == leader) {
