@@ -476,7 +476,7 @@ band_select_kernel(const float *__restrict__ band_all, int64_t band_cap, double 
         gathered = band_window(src, nsrc, s_sb, s_bins, s_scan, s_win, s_buf, &s_got, s2d, k, s_tab, &ctl->status);
         if (gathered) {
             src = s_buf;
-            nsrc = (int64_t)s_sb.n;
+            nsrc = min(s_got, (unsigned)GATHER_CAP);   // the window's count by construction
         }
         first = false;
     }
