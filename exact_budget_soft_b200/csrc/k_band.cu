@@ -121,9 +121,6 @@ __device__ __forceinline__ void block_scan3(Aff mu, Aff mv, unsigned c, Aff &mu_
     c_ex = (ci - c) + (warp > 0 ? (unsigned)scratch[2 * BS_NW + warp - 1].s : 0u);
 }
 
-// Edge e_j of the J bins of 2^s keys over [klo, khi]: e_0 = top, e_J = bot, and
-// between them the value of the largest key of bin j - 1 (so bin j holds the
-// scores r with e_{j+1} <= r < e_j).
 // Two affine maps with one multiplier, x -> a x + s1 and y -> a y + s2 (the
 // upper and lower bounds of the window step share d_j).
 struct Aff2 {
@@ -178,6 +175,9 @@ __device__ __forceinline__ int bin_shift(uint32_t w) {
     const int bits = 32 - __clz(w);
     return bits > BS_BITS ? bits - BS_BITS : 0;
 }
+// Edge e_j of the J bins of 2^s keys over [klo, khi]: e_0 = top, e_J = bot, and
+// between them the value of the largest key of bin j - 1 (so bin j holds the
+// scores r with e_{j+1} <= r < e_j).
 __device__ __forceinline__ double bin_edge(uint32_t klo, int s, unsigned J, unsigned j, double top, double bot) {
     if (j == 0) return top;
     if (j >= J) return bot;
@@ -190,8 +190,8 @@ __device__ __forceinline__ double bin_edge(uint32_t klo, int s, unsigned J, unsi
 // flags a root outside [a_L, a_R) (status non-null); later steps take the bin
 // whose edges straddle k as computed, with no flag, as an edge's G can differ
 // from the step before it by rounding.
-__device__ __noinline__ void band_level(const float *src, int64_t nsrc, SubBand &S, BinSums &B, Aff *scratch, unsigned *hit,
-                           double s2d, double k, const double *tab, int32_t *status) {
+__device__ __noinline__ void band_level(const float *src, int64_t nsrc, SubBand &S, BinSums &B, Aff *scratch,
+                                       unsigned *hit, double s2d, double k, const double *tab, int32_t *status) {
     const int tid = threadIdx.x;
     const uint32_t klo = S.klo, khi = S.khi;
     const double top = S.top, bot = S.bot;
@@ -304,8 +304,9 @@ struct WinScratch {
 // A second sweep sums the tail terms of the scores above and below that window
 // (per-thread fixed point, no atomics) and copies the window's own scores to
 // shared memory.  S becomes the window; returns true when the copy holds it.
-__device__ __noinline__ bool band_window(const float *src, int64_t nsrc, SubBand &S, BinSums &B, Aff *scratch, WinScratch &W,
-                            float *buf, unsigned *got, double s2d, double k, const double *tab, int32_t *status) {
+__device__ __noinline__ bool band_window(const float *src, int64_t nsrc, SubBand &S, BinSums &B, Aff *scratch,
+                                        WinScratch &W, float *buf, unsigned *got, double s2d, double k,
+                                        const double *tab, int32_t *status) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t klo = S.klo, khi = S.khi;
     const double top = S.top, bot = S.bot;
