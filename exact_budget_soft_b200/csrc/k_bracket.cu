@@ -5,9 +5,9 @@
 //   sample_kernel   kernel-noised sample y_j = r_{I_j} + t L_j (Philox4x64-10)
 //   select_kernel   exact order statistics y_(jR), y_(jL) by 3-round radix select
 //                   over a grid (last CTA finishes)
-//   oob_kernel<false>  streaming pass: counts and stable tail sums of the scores
-//                      outside [a_L, a_R), band compaction (warp ballots)
-//   oob_kernel<true>   certification pass: G(a_L), G(a_R) and the verdict
+//   oob_kernel<OOB_STREAM>  streaming pass: counts and stable tail sums of the
+//                      scores outside [a_L, a_R), band compaction
+//   oob_kernel<OOB_CERT>  certification pass: G(a_L), G(a_R) and the verdict
 //   p_kernel        p = F((r - b)/t)
 //   vjp_*_kernel    <g,f>/sum f, then grad = (f/t)(g - <g,f>/sum f)
 //
