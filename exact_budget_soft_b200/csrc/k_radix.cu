@@ -726,8 +726,8 @@ static cudaError_t launch_sort_k(SortArgs &A, cudaStream_t st) {
     return launch_coop(radix_sort_kernel<K>, (unsigned)g, RB, sort_smem<K>(), st, A);
 }
 
-// The tile size follows the capacity of the sort (the host does not know the
-// band's size): small sorts take small tiles, so more CTAs share the work.
+// The tile size follows the capacity of the sort: small sorts take small
+// tiles, so more CTAs share the work.
 cudaError_t launch_radix_sort(SortArgs &A, double k, double t, cudaStream_t st) {
     (void)k;
     (void)t;

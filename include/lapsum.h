@@ -15,9 +15,11 @@
  * abstract): the full-sort solver (sort, stable prefix/suffix scan, interval
  * search, closed-form root) and, for long rows, probabilistic bracketing
  * (kernel-noised sample, binomial order-statistic bracket [a_L, a_R), one
- * streaming pass folding out-of-band scores into tail sums, a sort of the
- * band only, a certification pass, and a full-sort fallback when the
- * certification fails).  Every step runs in this library's CUDA kernels.
+ * streaming pass folding out-of-band scores into tail sums, an exact solve on
+ * the band only -- narrowed by a radix select steered by the threshold curve,
+ * then the closed-form root -- a certification pass, and a full-sort fallback
+ * when the certification fails).  Every step runs in this library's CUDA
+ * kernels.
  *
  * Conventions for every entry point:
  *  - Pointers named *_dev are DEVICE memory, owned by the caller, on the
