@@ -12,6 +12,8 @@ Every function cites the passage it follows in the C source:
 * ``p``          -- p_i = F((r_i-b)/t).
 * ``vjp``        -- grad = (f/t)(g - <g,f>/sum f).
 * ``G``          -- the budget function itself (and sum f).
+* ``sort_desc``  -- the scores in descending order (fp64).
+* ``tail_sums``  -- the streaming pass's tail sums S_L, S_R from their definition.
 * ``philox``, ``ln``, ``sample``, ``binom_ranks``, ``bracket``, ``counts``,
   ``certify`` -- an independent restatement of the probabilistic bracket, for
   exact comparison of the integer results with the GPU path.
@@ -63,6 +65,7 @@ def _load():
                 "orc_p": (None, [f32p, C.c_int64, C.c_double, C.c_double, f64p]),
                 "orc_vjp": (None, [f32p, f32p, C.c_int64, C.c_double, C.c_double, f64p, dp, dp]),
                 "orc_sort_desc": (None, [f32p, C.c_int64, f64p]),
+                "orc_tail_sums": (None, [f32p, C.c_int64, C.c_float, C.c_float, C.c_double, dp, dp, dp, dp]),
                 "orc_philox4x64_10": (None, [u64p, u64p, u64p]),
                 "orc_ln": (C.c_double, [C.c_double]),
                 "orc_sample": (None, [f32p, C.c_int64, C.c_double, C.c_uint64, C.c_int64,
@@ -144,6 +147,15 @@ def sort_desc(r) -> np.ndarray:
     out = np.empty(r.size, dtype=np.float64)
     _load().orc_sort_desc(r, r.size, out)
     return out
+
+
+def tail_sums(r, a_L: float, a_R: float, t: float) -> dict:
+    """Streaming-pass tail sums S_L, S_R from their definition, and the parts of
+    each made of terms with |r - a|/t > 16."""
+    r = _f32(r)
+    v = [C.c_double() for _ in range(4)]
+    _load().orc_tail_sums(r, r.size, float(a_L), float(a_R), float(t), *[C.byref(x) for x in v])
+    return {"S_L": v[0].value, "S_R": v[1].value, "S_L_far": v[2].value, "S_R_far": v[3].value}
 
 
 def philox(counter, key) -> np.ndarray:

@@ -234,6 +234,49 @@ void orc_vjp(const float *r, const float *g, int64_t n, double b, double t,
     if (sf_out) *sf_out = nsum_val(&S0);
 }
 
+/*
+ * Tail sums of the streaming pass [FL-2.2 step 2], from their definition:
+ *   S_L = sum_{r < a_L} e^{(r - a_L)/t},   S_R = sum_{r >= a_R} e^{-(r - a_R)/t}
+ * (every term at most 1; an infinite end has an empty tail).  Also returns the
+ * part of each sum made of terms with z = |r - a|/t > 16, the terms a fast
+ * solver may form in a lower precision, so a test can bound their error.
+ * Neumaier sums over fixed chunks, combined in chunk order.
+ */
+void orc_tail_sums(const float *r, int64_t n, float aL, float aR, double t,
+                   double *SL, double *SR, double *SL_far, double *SR_far)
+{
+    int64_t nch = (n + ORC_CHUNK - 1) / ORC_CHUNK;
+    double *part = calloc((size_t)(4 * (nch ? nch : 1)), sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < nch; ++c) {
+        int64_t lo = c * ORC_CHUNK, hi = lo + ORC_CHUNK < n ? lo + ORC_CHUNK : n;
+        nsum L = {0, 0}, R = {0, 0}, Lf = {0, 0}, Rf = {0, 0};
+        for (int64_t i = lo; i < hi; ++i) {
+            float v = r[i];
+            if (!isinf(aL) && v < aL) {
+                double z = ((double)aL - (double)v) / t;
+                double e = exp(-z);
+                nsum_add(&L, e);
+                if (z > 16.0) nsum_add(&Lf, e);
+            } else if (!isinf(aR) && v >= aR) {
+                double z = ((double)v - (double)aR) / t;
+                double e = exp(-z);
+                nsum_add(&R, e);
+                if (z > 16.0) nsum_add(&Rf, e);
+            }
+        }
+        part[4 * c + 0] = nsum_val(&L);  part[4 * c + 1] = nsum_val(&R);
+        part[4 * c + 2] = nsum_val(&Lf); part[4 * c + 3] = nsum_val(&Rf);
+    }
+    nsum L = {0, 0}, R = {0, 0}, Lf = {0, 0}, Rf = {0, 0};
+    for (int64_t c = 0; c < nch; ++c) {
+        nsum_add(&L, part[4 * c + 0]);  nsum_add(&R, part[4 * c + 1]);
+        nsum_add(&Lf, part[4 * c + 2]); nsum_add(&Rf, part[4 * c + 3]);
+    }
+    free(part);
+    *SL = nsum_val(&L); *SR = nsum_val(&R); *SL_far = nsum_val(&Lf); *SR_far = nsum_val(&Rf);
+}
+
 static int cmp_desc(const void *a, const void *b)
 {
     double x = *(const double *)a, y = *(const double *)b;

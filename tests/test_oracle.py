@@ -366,3 +366,53 @@ def test_bracket_at_ranks_is_outward_order_statistics(orc):
     b1 = orc.bracket(r, k, t, seed, s, delta)
     b2 = orc.bracket_at_ranks(r, t, seed, s, b1["jR"], b1["jL"])
     assert (b1["a_L"], b1["a_R"]) == (b2["a_L"], b2["a_R"])
+
+
+# ------------------------------------------------- sort and the tail sums
+def test_sort_desc_matches_numpy_sort(orc):
+    r = np.concatenate([RNG.standard_normal(5000), np.repeat([0.5, -0.0, 0.0, 3e-39], 100),
+                        [np.float32(3.4e38), -np.float32(3.4e38)]]).astype(np.float32)
+    RNG.shuffle(r)
+    out = orc.sort_desc(r)
+    ref = np.sort(r.astype(np.float64))[::-1]
+    assert np.array_equal(out, ref)
+
+
+@pytest.mark.parametrize("m,t", [(50, 0.1), (400, 0.1), (3000, 0.02)])
+def test_tail_sums_geometric_closed_form(orc, m, t):
+    # scores on a grid of step D below a_L (i = 1..m) and at or above a_R (i = 0..m-1):
+    # the tail sums are geometric series in q = e^{-D/t}; the terms with z = iD/t > 16
+    # form the tails of those series.  Band scores (a_L <= r < a_R) add nothing.
+    D = 1.0 / 64
+    aL, aR = np.float32(-1.0), np.float32(2.0)
+    i = np.arange(1, m + 1)
+    below = (np.float64(aL) - i * D).astype(np.float32)
+    above = (np.float64(aR) + (i - 1) * D).astype(np.float32)
+    band = np.array([aL, 0.0, np.nextafter(aR, np.float32(0))], np.float32)
+    r = np.concatenate([below, above, band])
+    RNG.shuffle(r)
+    q = math.exp(-D / t)
+    got = orc.tail_sums(r, aL, aR, t)
+    geo = lambda a, b: (q ** a - q ** (b + 1)) / (1 - q)   # sum_{j=a}^{b} q^j
+    far_from = math.floor(16 * t / D) + 1                    # first j with jD/t > 16
+    assert abs(got["S_L"] - geo(1, m)) <= 1e-13 * geo(1, m)
+    assert abs(got["S_R"] - geo(0, m - 1)) <= 1e-13 * geo(0, m - 1)
+    want_far_L = geo(far_from, m) if m >= far_from else 0.0
+    want_far_R = geo(far_from, m - 1) if m - 1 >= far_from else 0.0
+    assert abs(got["S_L_far"] - want_far_L) <= 1e-13 * max(want_far_L, 1e-300)
+    assert abs(got["S_R_far"] - want_far_R) <= 1e-13 * max(want_far_R, 1e-300)
+
+
+def test_tail_sums_match_scipy_logsumexp(orc):
+    from scipy.special import logsumexp
+    r = RNG.laplace(0.0, 1.0, 200_000).astype(np.float32)
+    t = 0.05
+    for aL, aR in ((np.float32(1.5), np.float32(1.75)), (np.float32(-np.inf), np.float32(0.3)),
+                   (np.float32(-0.2), np.float32(np.inf))):
+        got = orc.tail_sums(r, aL, aR, t)
+        lo = r[r < aL].astype(np.float64)
+        hi = r[r >= aR].astype(np.float64)
+        SL = math.exp(logsumexp((lo - float(aL)) / t)) if lo.size else 0.0
+        SR = math.exp(logsumexp(-(hi - float(aR)) / t)) if hi.size else 0.0
+        assert abs(got["S_L"] - SL) <= 1e-12 * max(SL, 1e-300)
+        assert abs(got["S_R"] - SR) <= 1e-12 * max(SR, 1e-300)
