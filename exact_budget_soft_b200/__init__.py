@@ -25,6 +25,8 @@ LIB_PATH = os.path.join(_HERE, "liblapsum.so")
 
 PATH_AUTO, PATH_FULLSORT, PATH_BRACKET = 0, 1, 2
 CERTIFY_PASS, CERTIFY_FUSED = 0, 1
+# lapsum_stats.flags bits (rare routes a solve took)
+FLAG_SELECT_ALL_KEYS = 1
 # error codes (LAPSUM_ERR_* of the C header)
 ERR_ARG, ERR_NONFINITE, ERR_ALLOC, ERR_DEVICE_TIMEOUT, ERR_CUDA, ERR_NO_ROOT = -1, -2, -3, -4, -5, -6
 ERRORS = {0: "ok", -1: "invalid argument", -2: "non-finite score", -3: "workspace allocation failed",
@@ -50,7 +52,7 @@ class Stats(C.Structure):
                 ("a_L", C.c_float), ("a_R", C.c_float), ("S_L", C.c_double), ("S_R", C.c_double),
                 ("G_aL", C.c_double), ("G_aR", C.c_double), ("b", C.c_double),
                 ("sum_p", C.c_double), ("j_star", C.c_int64), ("widened", C.c_int64),
-                ("reserved", C.c_int64 * 3)]
+                ("flags", C.c_int64), ("reserved", C.c_int64 * 2)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
@@ -58,7 +60,10 @@ class Stats(C.Structure):
 
 EXPORTS = ["lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats", "lapsum_get_stats_rows",
            "lapsum_strerror", "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read",
-           "lapsum_bracket_plan", "lapsum_profile_filter", "lapsum_selftest_math", "lapsum_launch_count"]
+           "lapsum_bracket_plan", "lapsum_profile_filter", "lapsum_selftest_math", "lapsum_launch_count",
+           "lapsum_backward_noalloc", "lapsum_shard_plan", "lapsum_shard_sample", "lapsum_shard_stream",
+           "lapsum_shard_solve", "lapsum_shard_p", "lapsum_shard_vjp_partial", "lapsum_shard_vjp_apply"]
+SHARD_PART = 10   # doubles in a slice's streaming-pass record (LAPSUM_SHARD_PART)
 
 
 def _load() -> C.CDLL:
@@ -85,6 +90,17 @@ def _load() -> C.CDLL:
     lib.lapsum_profile_filter.restype = C.c_int
     lib.lapsum_selftest_math.argtypes = [C.c_int, vp, vp, vp, i64, vp]
     lib.lapsum_selftest_math.restype = C.c_int
+    op = C.POINTER(Options)
+    lib.lapsum_shard_plan.argtypes = [i64, dbl, op, C.POINTER(i64), C.POINTER(i64)]
+    lib.lapsum_shard_sample.argtypes = [vp, i64, i64, i64, dbl, dbl, op, vp, vp]
+    lib.lapsum_shard_stream.argtypes = [vp, i64, i64, i64, dbl, dbl, op, vp, vp, vp, vp]
+    lib.lapsum_shard_solve.argtypes = [vp, i64, vp, i64, i64, dbl, dbl, op, vp, vp, vp]
+    lib.lapsum_shard_p.argtypes = [vp, i64, dbl, vp, vp, vp]
+    lib.lapsum_shard_vjp_partial.argtypes = [vp, vp, vp, i64, dbl, dbl, vp, vp]
+    lib.lapsum_shard_vjp_apply.argtypes = [vp, vp, vp, i64, dbl, vp, i64, vp, vp]
+    for name in ("lapsum_shard_plan", "lapsum_shard_sample", "lapsum_shard_stream", "lapsum_shard_solve",
+                 "lapsum_shard_p", "lapsum_shard_vjp_partial", "lapsum_shard_vjp_apply"):
+        getattr(lib, name).restype = C.c_int
     for name in ("lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats",
                  "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read"):
         getattr(lib, name).restype = C.c_int

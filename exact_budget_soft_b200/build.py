@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblapsum.so")
-SOURCES = ["lapsum_api.cu", "k_rows.cu", "k_bracket.cu", "k_radix.cu", "k_band.cu", "k_noalloc.cu"]
+SOURCES = ["lapsum_api.cu", "k_rows.cu", "k_bracket.cu", "k_radix.cu", "k_band.cu", "k_noalloc.cu", "k_shard.cu"]
 HEADERS = ["lapsum_internal.h", "lapsum_kernels.h", "lapsum_device.cuh", "scan_solve.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

@@ -525,13 +525,8 @@ band_select_kernel(const float *__restrict__ band_all, int64_t band_cap, double 
 
 cudaError_t launch_band_select(const float *band, int64_t rows, double k, double t, Ctl *ctl, int64_t band_cap,
                                int32_t round2, cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(band_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)sizeof(BinSums));
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    const cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(band_select_kernel), sizeof(BinSums));
+    if (e != cudaSuccess) return e;
     return launch_k(band_select_kernel, (unsigned)rows, BS_BLOCK, sizeof(BinSums), st, band, band_cap, k, t,
                     1.0 / t, ctl, round2);
 }

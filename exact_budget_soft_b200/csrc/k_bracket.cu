@@ -25,16 +25,7 @@ namespace lapsum {
 constexpr int SBLOCK = 256;     // threads per block of the streaming passes
 constexpr int SBLOCKS_PER_SM = 4;
 
-static int g_num_sms = 0;
-int stream_grid(int per_sm) {
-    if (g_num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (g_num_sms <= 0) g_num_sms = 148;
-    }
-    return g_num_sms * per_sm;
-}
+int stream_grid(int per_sm) { return device_sm_count() * per_sm; }
 int stream_grid() { return stream_grid(SBLOCKS_PER_SM); }
 
 // ------------------------------------------------------ last-block combine --
@@ -152,10 +143,20 @@ __global__ void __launch_bounds__(256) sample_kernel(BracketParams Pg) {
     }
     __syncthreads();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // the index is drawn over the whole row; a rank holding one slice of a split
+    // row keeps the draws that land in its slice (the others hold the rest)
+    bool mine = false;
+    int64_t I = 0;
+    uint64_t x1 = 0;
     if (j < P.s) {
-        uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
+        uint64_t x0 = (uint64_t)j, x2 = 0, x3 = 0;
+        x1 = (uint64_t)P.row;
         philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
-        const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n);
+        I = (int64_t)__umul64hi(x0, (uint64_t)P.n_total) - P.shard_off;
+        mine = I >= 0 && I < P.n;
+        if (!mine) P.keys[j] = 0u;   // a split row's exchange sums the ranks' shares
+    }
+    if (mine) {
         const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
         const double E = -sample_ln(U);
         const double L = (x1 & 1ull) ? E : -E;
@@ -350,6 +351,7 @@ __global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams Pg) {
     }
     P.hist1[SEL_BINS + tid] = 0u;   // the top-byte histogram; the streaming pass clears the rest
     if (tid == 0) {
+        if ((valid[0] && !fast[0]) || (valid[1] && !fast[1])) ctl->flags |= FLAG_SELECT_ALL_KEYS;
         const float yR = desc_key_to_float(s_pref[0]);
         const float yL = desc_key_to_float(s_pref[1]);
         const float aR = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
@@ -984,6 +986,8 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
             const double GaR = (double)cR - 0.5 * v[3] + 0.5 * fma(rho, v[2], v[5]);
             ctl->G_aL = GaL;
             ctl->G_aR = GaR;
+            ctl->hL = v[4];
+            ctl->lR = v[5];
             const bool sound = (cb <= (unsigned long long)P.band_cap) &&
                                (cL + cb + cR == (unsigned long long)n) && ((ctl->status & ST_NONFINITE) == 0);
             const bool ok = sound && (GaL >= P.k) && (GaR < P.k);
@@ -1016,12 +1020,12 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
 // ================================================================= p pass --
 // p = F((r - b)/t), walking forward (the certification pass left the head of
 // the row in L2).  Also sum p (fp64 over fp32 float4 partials) for diagnostics.
-__device__ __forceinline__ float4 p_vec(const float4 v, const XForm &xf) {
+__device__ __forceinline__ float4 p_vec(const float4 v, const PForm &pf) {
     float4 o;
-    o.x = laplace_cdf2(xf(v.x));
-    o.y = laplace_cdf2(xf(v.y));
-    o.z = laplace_cdf2(xf(v.z));
-    o.w = laplace_cdf2(xf(v.w));
+    o.x = pf(v.x);
+    o.y = pf(v.y);
+    o.z = pf(v.z);
+    o.w = pf(v.w);
     return o;
 }
 
@@ -1038,7 +1042,7 @@ p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restric
     __shared__ double s_red[SBLOCK / 32];
     pdl_enter();
     const double b = ctl->b;
-    const XForm xf = make_xform(b, inv_t * LOG2E);
+    const PForm xf = make_pform(b, inv_t * LOG2E);
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(p)) & 15) == 0;
@@ -1062,7 +1066,7 @@ p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restric
         ps += (double)((o.x + o.y) + (o.z + o.w));
     }
     for (int64_t j = n4 * 4 + gtid; j < n; j += gstride) {
-        const float o = laplace_cdf2(xf(r[j]));
+        const float o = xf(r[j]);
         ps += (double)o;
         p[j] = o;
     }
@@ -1077,17 +1081,23 @@ p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restric
 
 // =================================================================== VJP --
 // <g,f> and sum f of one long row (walking backward: the p pass left the tail
-// in L2).  Terms are e^{-|x|} in fp32 (denormals kept); each thread sums the
+// in L2).  Terms are e^{-|x|} in fp32; each thread sums the
 // terms of one chunk (eight scores: positive terms, and g e products whose
 // fp32 rounding is ~1e-7 of their magnitudes) in fp32 and adds that partial to
 // fp64 accumulators, so the fp64 pipe sees two adds per eight scores.  If
-// every term underflows (all scores farther than ~100 t from b), the last block
+// sum e is below 2^-96 (every score farther than ~66 t from b: some terms may
+// have lost significant bits as fp32 denormals, or underflowed), the last block
 // raises a flag and vjp_shifted_kernel recomputes the ratio from terms shifted
 // by the running minimum of |x| (the shift cancels in <g,f>/sum f).
+// SLICE: one slice of a row split across ranks -- the terms are shifted by
+// 2^{sh2} (sh2 = 0, or the smallest |x2| over every rank when the plain sums
+// are too small), and the last block writes {sum e, sum g e, min |x2|} to
+// part_out for the ranks' exchange instead of lambda.
+template <bool SLICE>
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
 vjp_reduce_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_,
                   const float *__restrict__ g_, int64_t n, double inv_t, Ctl *ctl_, double *partials_,
-                  int64_t pstride) {
+                  int64_t pstride, float sh2, double *part_out) {
     const int64_t row = blockIdx.y;
     const float *__restrict__ r = r_ + row * n;
     const float *__restrict__ g = g_ + row * n;
@@ -1106,9 +1116,15 @@ vjp_reduce_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_
     const float4 *r4 = reinterpret_cast<const float4 *>(r);
     const float4 *g4 = reinterpret_cast<const float4 *>(g);
     double sf = 0.0, sgf = 0.0;
+    float amin = CUDART_INF_F;   // SLICE: smallest |x2| of the thread's scores
+    auto term = [&](float r1) {
+        const float a = fabsf(xf(r1));
+        if (SLICE) amin = fminf(amin, a);
+        return SLICE ? exp2f(sh2 - a) : exp2f(-a);
+    };
     auto part4 = [&](const float4 v, const float4 w, float &f32, float &gf32) {
-        const float e0 = exp2f(-fabsf(xf(v.x))), e1 = exp2f(-fabsf(xf(v.y)));
-        const float e2 = exp2f(-fabsf(xf(v.z))), e3 = exp2f(-fabsf(xf(v.w)));
+        const float e0 = term(v.x), e1 = term(v.y);
+        const float e2 = term(v.z), e3 = term(v.w);
         f32 += (e0 + e1) + (e2 + e3);
         gf32 = fmaf(w.x, e0, gf32);
         gf32 = fmaf(w.y, e1, gf32);
@@ -1133,15 +1149,38 @@ vjp_reduce_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_
         sgf += (double)gf32;
     }
     for (int64_t i = n4 * 4 + gtid; i < n; i += gstride) {
-        const float e = exp2f(-fabsf(xf(r[i])));
+        const float e = term(r[i]);
         sf += (double)e;
         sgf = fma((double)g[i], (double)e, sgf);
+    }
+    if (SLICE) {   // the slice's smallest |x2|: block minimum, then one atomic per block
+        __shared__ unsigned s_min;
+        if (threadIdx.x == 0) s_min = 0x7f800000u;
+        __syncthreads();
+        amin = fminf(amin, __shfl_xor_sync(FULL, amin, 16));
+        amin = fminf(amin, __shfl_xor_sync(FULL, amin, 8));
+        amin = fminf(amin, __shfl_xor_sync(FULL, amin, 4));
+        amin = fminf(amin, __shfl_xor_sync(FULL, amin, 2));
+        amin = fminf(amin, __shfl_xor_sync(FULL, amin, 1));
+        if ((threadIdx.x & 31) == 0) atomicMin(&s_min, __float_as_uint(amin));   // amin >= 0: bits order as values
+        __syncthreads();
+        if (threadIdx.x == 0) atomicMin(reinterpret_cast<unsigned *>(&ctl->vjp_min), s_min);
     }
     double v[2] = {sf, sgf};
     block_sum<SBLOCK, 2>(v, s_red);
     if (last_block_sum<SBLOCK, 2>(v, partials, &ctl->ticket[3], s_red) && threadIdx.x == 0) {
+        if (SLICE) {
+            __threadfence();
+            part_out[0] = v[0];
+            part_out[1] = v[1];
+            // the slice's smallest |x| in natural units (|x2| = |x| log2 e)
+            part_out[2] = (double)__uint_as_float(atomicAdd(reinterpret_cast<unsigned *>(&ctl->vjp_min), 0u)) / LOG2E;
+            return;
+        }
         ctl->vjp_lambda = v[1] / v[0];
-        ctl->vjp_shift = !(v[0] >= 1e-300);
+        // below 2^-96 some terms may be denormal in fp32 (fewer significant
+        // bits) or lost; the shifted recomputation keeps every term's precision
+        ctl->vjp_shift = !(v[0] >= 0x1p-96);
     }
 }
 
@@ -1150,6 +1189,7 @@ struct ShiftSumG {
     double sf, sgf;
 };
 __device__ __forceinline__ void ss_add(ShiftSumG &s, float ax, float g) {
+    ax = fminf(ax, 3.0e38f);   // |x| may overflow fp32 (t tiny): keep the shift finite
     if (ax < s.m) {
         const double sc = (double)exp2f(ax - s.m);
         s.sf *= sc;
@@ -1171,7 +1211,7 @@ __device__ __forceinline__ ShiftSumG ss_merge(ShiftSumG a, ShiftSumG b) {
     return r;
 }
 
-// Rare path: every f_i underflowed in vjp_reduce_kernel.
+// Rare path: sum f was below 2^-96 in vjp_reduce_kernel (b far from every score).
 __global__ void __launch_bounds__(SBLOCK)
 vjp_shifted_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_,
                    const float *__restrict__ g_, int64_t n, double inv_t, Ctl *ctl_, double *partials_,
@@ -1238,7 +1278,7 @@ vjp_apply_kernel(const float *__restrict__ r_, const double *__restrict__ b_in_,
     const XForm xf = make_xform(*b_in, inv_t * LOG2E);
     const double lam = ctl->vjp_lambda;
     const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
-    const float hit = (float)(0.5 * inv_t);
+    const float hit = vjp_scale2(inv_t);   // log2(1/(2t))
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
     const bool aligned = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(g) |
@@ -1315,12 +1355,12 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
 int select_cand_capacity() { return SEL_CAND; }
 template <typename K>
 static cudaError_t set_smem(K kern, size_t bytes) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    return set_max_dynamic_smem(reinterpret_cast<const void *>(kern), bytes);
 }
 
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
-    static cudaError_t once = set_smem(oob_kernel<OOB_STREAM>, bulk_smem_bytes<1>());
-    static cudaError_t once2 = set_smem(oob_kernel<OOB_STREAM_CERT>, bulk_smem_bytes<1>());
+    const cudaError_t once = set_smem(oob_kernel<OOB_STREAM>, bulk_smem_bytes<1>());
+    const cudaError_t once2 = set_smem(oob_kernel<OOB_STREAM_CERT>, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
     if (once2 != cudaSuccess) return once2;
     if (P.fused_cert)
@@ -1328,8 +1368,8 @@ cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st) {
     return launch_k(oob_kernel<OOB_STREAM>, row_grid(SBLOCKS_PER_SM, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
 }
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
-    static cudaError_t once = set_smem(oob_kernel<OOB_CERT, 3>, bulk_smem_bytes<1>());
-    static cudaError_t once4 = set_smem(oob_kernel<OOB_CERT, 4, true>, bulk_smem_bytes<1>());
+    const cudaError_t once = set_smem(oob_kernel<OOB_CERT, 3>, bulk_smem_bytes<1>());
+    const cudaError_t once4 = set_smem(oob_kernel<OOB_CERT, 4, true>, bulk_smem_bytes<1>());
     if (once != cudaSuccess || once4 != cudaSuccess) return once != cudaSuccess ? once : once4;
     if (P.rows > 1)
         return launch_k(oob_kernel<OOB_CERT, 4, true>, row_grid(4, P.rows), SBLOCK, bulk_smem_bytes<1>(), st, P);
@@ -1337,26 +1377,33 @@ cudaError_t launch_certify(const BracketParams &P, cudaStream_t st) {
 }
 cudaError_t launch_p_pass(const float *r, int64_t rows, int64_t n, double t, float *p, double *b_out, Ctl *ctl,
                           double *partials, cudaStream_t st) {
-    static cudaError_t once = set_smem(p_kernel, bulk_smem_bytes<1>());
+    const cudaError_t once = set_smem(p_kernel, bulk_smem_bytes<1>());
     if (once != cudaSuccess) return once;
     return launch_k(p_kernel, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<1>(), st, r, n, 1.0 / t, p,
                     b_out, ctl, partials, partial_stride(rows));
 }
 cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                               Ctl *ctl, double *partials, cudaStream_t st) {
-    static cudaError_t once = set_smem(vjp_reduce_kernel, bulk_smem_bytes<2>());
+    const cudaError_t once = set_smem(vjp_reduce_kernel<false>, bulk_smem_bytes<2>());
     if (once != cudaSuccess) return once;
     const int64_t ps = partial_stride(rows);
-    cudaError_t e = launch_k(vjp_reduce_kernel, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<2>(), st,
-                             r, b, g, n, 1.0 / t, ctl, partials, ps);
+    cudaError_t e = launch_k(vjp_reduce_kernel<false>, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<2>(),
+                             st, r, b, g, n, 1.0 / t, ctl, partials, ps, 0.0f, (double *)nullptr);
     if (e != cudaSuccess) return e;
     dim3 gs = row_grid(SBLOCKS_PER_SM, rows);
     gs.x = gs.x / SBLOCKS_PER_SM < 1 ? 1 : gs.x / SBLOCKS_PER_SM;
     return launch_k(vjp_shifted_kernel, gs, SBLOCK, 0, st, r, b, g, n, 1.0 / t, ctl, partials, ps);
 }
+cudaError_t launch_vjp_slice_partial(const float *r, const double *b, const float *g, int64_t n, double t,
+                                     float sh2, Ctl *ctl, double *partials, double *part_out, cudaStream_t st) {
+    const cudaError_t once = set_smem(vjp_reduce_kernel<true>, bulk_smem_bytes<2>());
+    if (once != cudaSuccess) return once;
+    return launch_k(vjp_reduce_kernel<true>, row_grid(SBLOCKS_PER_SM, 1), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g,
+                    n, 1.0 / t, ctl, partials, partial_stride(1), sh2, part_out);
+}
 cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st) {
-    static cudaError_t once = set_smem(vjp_apply_kernel, bulk_smem_bytes<2>());
+    const cudaError_t once = set_smem(vjp_apply_kernel, bulk_smem_bytes<2>());
     if (once != cudaSuccess) return once;
     return launch_k(vjp_apply_kernel, row_grid(SBLOCKS_PER_SM, rows), SBLOCK, bulk_smem_bytes<2>(), st, r, b, g, n,
                     1.0 / t, ctl, grad);

@@ -40,6 +40,7 @@ struct ShiftAcc {
     double sf, sgf;
 };
 __device__ __forceinline__ void sa_add(ShiftAcc &s, float ax, float g) {
+    ax = fminf(ax, 3.0e38f);   // |x| may overflow fp32 (t tiny): keep the shift finite
     if (ax < s.m) {
         const double sc = (double)exp2f(ax - s.m);
         s.sf *= sc;
@@ -125,7 +126,7 @@ noalloc_apply_kernel(const float *__restrict__ r, const double *__restrict__ b_i
     const XForm xf = make_xform(b_in[row], inv_t * LOG2E);
     const double lam = lam_all[row];
     const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
-    const float hit = (float)(0.5 * inv_t);
+    const float hit = vjp_scale2(inv_t);   // log2(1/(2t))
     for (int64_t i = j * NB + threadIdx.x; i < n; i += B * NB)
         out[i] = vjp_term2(xf(rr[i]), gg[i], hit, lam_hi, lam_lo);
 }
@@ -159,7 +160,7 @@ extern "C" int lapsum_backward_noalloc(const float *scores, const double *b, con
                                        struct CUstream_st *stream_in) {
     if (!scores || !b || !g || !grad_out || rows < 1 || n < 1 || n >= (int64_t(1) << 31))
         return LAPSUM_ERR_ARG;
-    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_ERR_ARG;
+    if (!(t >= LAPSUM_T_MIN && t <= LAPSUM_T_MAX)) return LAPSUM_ERR_ARG;
     // blocks per row: about four per SM in total, at least one per row
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -31,6 +31,15 @@ constexpr int HB = 256;             // histogram kernel threads
 
 
 
+// The two words after the four global digit histograms: a count of sorts that
+// gave up (possibly leaving partial counts in the histograms), and the count at
+// the last clean-up.  They differ while the histograms need clearing.
+__device__ __forceinline__ unsigned long long *A_hist_dirty(const SortArgs &A) { return A.hist + 4 * 256; }
+__device__ __forceinline__ unsigned long long *A_hist_cleaned(const SortArgs &A) { return A.hist + 4 * 256 + 1; }
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long *p) {
+    return *reinterpret_cast<const volatile unsigned long long *>(p);
+}
+
 // Element count behind a gate; < 0 means "nothing to do".
 __device__ __forceinline__ int64_t gated_n(const SortArgs &A) {
     if (A.gate == GATE_FALLBACK && A.ctl->verdict != 0) return -1;
@@ -170,11 +179,12 @@ __device__ __forceinline__ void warp_count(const uint32_t (&key)[K], int cnt_til
 
 // Walks the CTA's chunk of tiles in order with one tile staged ahead, calling
 // body(tile, cnt_tile, key) with every thread's keys; a barrier follows each
-// body, so the staging buffers are free again.  Returns false if a wait gave up.
+// body, so the staging buffers are free again.  Returns false if a wait gave up
+// (in any thread): ST_TIMEOUT is set, no further copy is issued, the copies in
+// flight are waited for (bounded), and the caller must return.
 template <int K, typename Body>
 __device__ __forceinline__ bool walk_chunk(TileStage<K> &S, const SortArgs &A, const uint32_t *src, int64_t t0,
                                            int64_t t1, uint32_t &ph, Body &&body) {
-    bool ok = true;
     stage_source(S, A, src);
     if (threadIdx.x == 0 && t0 < t1) stage_issue(S, 0, t0);
     int slot = 0;
@@ -182,11 +192,21 @@ __device__ __forceinline__ bool walk_chunk(TileStage<K> &S, const SortArgs &A, c
         if (threadIdx.x == 0 && tile + 1 < t1) stage_issue(S, slot ^ 1, tile + 1);
         const int cnt_tile = (int)min((int64_t)TILE_K(K), S.n - tile * TILE_K(K));
         uint32_t key[K];
-        ok &= stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
+        const bool ok = stage_keys(S, A, src, slot, ph, tile, cnt_tile, key);
         body(tile, cnt_tile, key, S.buf + slot * TILE_K(K));
-        __syncthreads();
+        if (!__syncthreads_and(ok)) {
+            if (threadIdx.x == 0) {
+                atomicOr(&A.ctl->status, ST_TIMEOUT);
+                // this tile's copy (its phase bit already flipped) and the next one's
+                if (stage_full(S, tile)) mbar_wait(&S.bar[slot], ((ph >> slot) & 1u) ^ 1u, BULK_WAIT_CAP);
+                if (tile + 1 < t1 && stage_full(S, tile + 1))
+                    mbar_wait(&S.bar[slot ^ 1], (ph >> (slot ^ 1)) & 1u, BULK_WAIT_CAP);
+            }
+            __syncthreads();
+            return false;
+        }
     }
-    return ok;
+    return true;
 }
 
 // ------------------------------------------------------------ locate --
@@ -454,6 +474,19 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
         mbar_init_fence();
     }
     __syncthreads();
+    // A sort that gave up on an earlier launch may have left partial counts in the
+    // global digit histograms (the word after them says so; every CTA reads it
+    // before any count is added, so all take the same branch): clear them first.
+    const unsigned long long gave_up = ld_volatile_u64(A_hist_dirty(Ag));
+    if (gave_up != ld_volatile_u64(A_hist_cleaned(Ag))) {
+        if (c == 0)
+            for (int i = tid; i < 4 * 256; i += RB) Ag.hist[i] = 0ull;
+        if (!grid_sync(&Ag.ctl->gbar_count, &Ag.ctl->gbar_gen, Ag.spin_cap, &Ag.ctl->status)) {
+            if (tid == 0) atomicAdd(A_hist_dirty(Ag), 1ull);
+            return;
+        }
+        if (c == 0 && tid == 0) *A_hist_cleaned(Ag) = gave_up;   // a give-up later in this launch counts again
+    }
     uint32_t ph = 0;   // mbarrier phases, carried from row to row
     // the rows of a batch, one after another (each gated by its own control block)
     // The gates of a block of RB rows are read together (one thread per row) and
@@ -490,17 +523,22 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
             const int64_t ntiles = (n + TILE_K(K) - 1) / TILE_K(K);
             const int64_t t0 = (int64_t)c * ntiles / G, t1 = (int64_t)(c + 1) * ntiles / G;
             uint32_t *csum = A.chunkcnt;   // [4][256][G]
-            auto bar = [&]() { grid_sync(&ctl->gbar_count, &ctl->gbar_gen, A.spin_cap, &ctl->status); };
+            // a barrier or copy wait that gives up ends the kernel for this CTA (every
+            // CTA then leaves at its next barrier, each wait bounded)
+            auto bar = [&]() -> bool {
+                const bool ok = grid_sync(&ctl->gbar_count, &ctl->gbar_gen, A.spin_cap, &ctl->status);
+                if (!ok && tid == 0) atomicAdd(A_hist_dirty(A), 1ull);
+                return ok;
+            };
             S.n = n;
             for (int i = tid; i < 4 * 256; i += RB) s_h4[i] = 0;
             __syncthreads();
-            bool ok = true;
 
             // ---- phase H: the chunk's four digit histograms
             {
                 uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
                 uint32_t cnt[4] = {0, 0, 0, 0};
-                ok &= walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
+                const bool walked = walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
                     const int l0 = warp * 32 * K + lane;
 #pragma unroll
                     for (int i = 0; i < K; ++i) {
@@ -518,6 +556,10 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                         }
                     }
                 });
+                if (!walked) {
+                    if (tid == 0) atomicAdd(A_hist_dirty(A), 1ull);
+                    return;
+                }
 #pragma unroll
                 for (int d = 0; d < 4; ++d)
                     if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
@@ -528,7 +570,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                     if (v) atomicAdd(A.hist + i, (unsigned long long)v);
                 }
             }
-            bar();
+            if (!bar()) return;
             // digit bases and skip flags, the same in every CTA (thread d owns bin d)
             if (tid == 0) s_skip = 0;
             __syncthreads();
@@ -566,16 +608,19 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                     if (!first) {   // the chunk's digit counts in the current order
                         for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
                         __syncthreads();
-                        ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
-                            warp_count(key, cnt_tile, sh, s_hist + warp * 256);
-                        });
+                        if (!walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
+                                warp_count(key, cnt_tile, sh, s_hist + warp * 256);
+                            })) {
+                            if (tid == 0) atomicAdd(A_hist_dirty(A), 1ull);
+                            return;
+                        }
                         if (tid < 256) {
                             uint32_t tot = 0;
 #pragma unroll
                             for (int w = 0; w < RNW; ++w) tot += s_hist[w * 256 + tid];
                             crow[(size_t)tid * G + c] = tot;
                         }
-                        bar();
+                        if (!bar()) return;
                     }
                     // global start of every digit in this chunk: base + counts of earlier
                     // chunks (a warp per digit, four digits' loads in flight at once)
@@ -598,7 +643,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                         }
                     }
                     __syncthreads();
-                    ok &= walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *s_keys) {
+                    const bool walked = walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *s_keys) {
                         for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
                         __syncthreads();   // every key is in registers: s_keys is free too
                         uint32_t *my_hist = s_hist + warp * 256;
@@ -660,24 +705,27 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                             dst[(uint32_t)(s_gofs[(kk >> sh) & 0xffu] + (uint32_t)i)] = kk;
                         }
                     });
-                    bar();   // the pass's keys are all written before the next pass reads them
+                    if (!walked) {
+                        if (tid == 0) atomicAdd(A_hist_dirty(A), 1ull);
+                        return;
+                    }
+                    if (!bar()) return;   // the pass's keys are all written before the next pass reads them
                     cur = cur == 0 ? 1 : 0;
                     first = false;
                 }
             }
-            if (!ok) atomicOr(&ctl->status, ST_TIMEOUT);
             // locate: tile and chunk maps of the sorted values (every CTA, its chunk)
             const uint32_t *sorted = cur == 0 ? A.keys[0] : A.keys[1];
             const Seeds z = locate_seeds(A);
             ChunkRec *crec = reinterpret_cast<ChunkRec *>(A.tilebuf);
             TileRec *rec = reinterpret_cast<TileRec *>(A.tilebuf + 8 * SORT_GMAX);
             if (skip != 15) locate_tiles<K>(A, sorted, n, t0, t1, z, rec, crec, S.buf, reinterpret_cast<Aff *>(s_hist), s_tab);
-            bar();   // the maps are complete, and every CTA has read the global histograms
+            if (!bar()) return;   // the maps are complete, and every CTA has read the global histograms
             if (c == 0) {
                 for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
                 if (skip != 15) locate_finish<K>(A, sorted, n, z, rec, crec, S.buf, s_hist, s_tab);
             }
-            bar();   // the next row reuses the global scratch
+            if (!bar()) return;   // the next row reuses the global scratch
             __syncthreads();   // s_open is rewritten by the next block of rows
         }
     }
@@ -685,17 +733,6 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
 }
 
 // ------------------------------------------------------------ launchers --
-static int num_sms() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    return sms;
-}
-
 int sort_grid_max() { return SORT_GMAX; }
 
 // Doubles of locate records a sort of up to cap keys needs: chunk records, then
@@ -708,17 +745,12 @@ int64_t sort_record_doubles(int64_t cap) {
 
 template <int K>
 static cudaError_t launch_sort_k(SortArgs &A, cudaStream_t st) {
-    static int resident = 0;   // CTAs of this sort kernel that fit the device at once
-    if (!resident) {
-        cudaError_t e = cudaFuncSetAttribute(radix_sort_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)sort_smem<K>());
-        if (e != cudaSuccess) return e;
-        int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, radix_sort_kernel<K>, RB, sort_smem<K>());
-        if (e != cudaSuccess) return e;
-        if (per_sm < 1) return cudaErrorInvalidConfiguration;
-        resident = per_sm * num_sms();
-    }
+    const void *kern = reinterpret_cast<const void *>(radix_sort_kernel<K>);
+    cudaError_t e = set_max_dynamic_smem(kern, sort_smem<K>());
+    if (e != cudaSuccess) return e;
+    int resident = 0;   // CTAs of this sort kernel that fit the current device at once
+    e = resident_ctas(kern, RB, sort_smem<K>(), &resident);
+    if (e != cudaSuccess) return e;
     int64_t g = (A.cap + TILE_K(K) - 1) / TILE_K(K);
     if (g > resident) g = resident;
     if (g > SORT_GMAX) g = SORT_GMAX;

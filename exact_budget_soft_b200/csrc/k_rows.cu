@@ -88,7 +88,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
 
     // ---- p = F((r - b)/t) for the row
     b = s_b;
-    const XForm xf = make_xform(b, inv_t * LOG2E);
+    const PForm pf = make_pform(b, inv_t * LOG2E);
     float *prow = p_out + (int64_t)blockIdx.x * n_arg;
     const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(row) & 15) == 0) &&
                      ((reinterpret_cast<uintptr_t>(prow) & 15) == 0);
@@ -98,16 +98,16 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
         float4 *p4 = reinterpret_cast<float4 *>(prow);
         for (int i = tid; i < n / 4; i += BLOCK) {
             float4 v = r4[i], o;
-            o.x = laplace_cdf2(xf(v.x));
-            o.y = laplace_cdf2(xf(v.y));
-            o.z = laplace_cdf2(xf(v.z));
-            o.w = laplace_cdf2(xf(v.w));
+            o.x = pf(v.x);
+            o.y = pf(v.y);
+            o.z = pf(v.z);
+            o.w = pf(v.w);
             psum += ((double)o.x + (double)o.y) + ((double)o.z + (double)o.w);
             p4[i] = o;
         }
     } else {
         for (int i = tid; i < n; i += BLOCK) {
-            float o = laplace_cdf2(xf(row[i]));
+            float o = pf(row[i]);
             psum += (double)o;
             prow[i] = o;
         }
@@ -132,6 +132,7 @@ struct ShiftSum {
     double sf, sgf;
 };
 __device__ __forceinline__ void shift_add(ShiftSum &s, float ax, float g) {
+    ax = fminf(ax, 3.0e38f);   // |x| may overflow fp32 (t tiny): keep the shift finite
     if (ax < s.m) {
         double sc = (double)exp2f(ax - s.m);   // 0 when s.m = +inf
         s.sf *= sc;
@@ -199,7 +200,7 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
     __syncthreads();
     const double lam = s_lam;
     const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
-    const float hit = (float)(0.5 * inv_t);
+    const float hit = vjp_scale2(inv_t);   // log2(1/(2t))
     if (vec) {
         const float4 *r4 = reinterpret_cast<const float4 *>(r);
         const float4 *g4 = reinterpret_cast<const float4 *>(gg);
@@ -223,13 +224,8 @@ static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n,
                                    float *p, double *b, Ctl *ctl, cudaStream_t st) {
     using C = RowCfg<BLOCK, KPT>;
     auto kern = rowsolve_kernel<BLOCK, KPT>;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)C::SMEM);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    const cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), C::SMEM);
+    if (e != cudaSuccess) return e;
     return launch_k(kern, (unsigned)rows, BLOCK, C::SMEM, st, scores, n, k, t, 1.0 / t, p, b, ctl);
 }
 

@@ -18,12 +18,69 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 #include <utility>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/lapsum.h"
 #include "lapsum_internal.h"
 #include "lapsum_kernels.h"
+
+namespace lapsum {
+
+namespace {
+std::mutex g_dev_mu;
+std::map<int, int> g_dev_sms;
+std::map<std::tuple<int, const void *, size_t>, cudaError_t> g_dev_smem;
+std::map<std::tuple<int, const void *, int, size_t>, int> g_dev_resident;
+int current_device() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+}  // namespace
+
+int device_sm_count() {
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    auto it = g_dev_sms.find(dev);
+    if (it != g_dev_sms.end()) return it->second;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    g_dev_sms[dev] = sms;
+    return sms;
+}
+
+cudaError_t set_max_dynamic_smem(const void *kern, size_t bytes) {
+    const auto key = std::make_tuple(current_device(), kern, bytes);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    auto it = g_dev_smem.find(key);
+    if (it != g_dev_smem.end()) return it->second;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    g_dev_smem[key] = e;
+    return e;
+}
+
+cudaError_t resident_ctas(const void *kern, int threads, size_t smem, int *out) {
+    const int sms = device_sm_count();
+    const auto key = std::make_tuple(current_device(), kern, threads, smem);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    auto it = g_dev_resident.find(key);
+    if (it != g_dev_resident.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    int per_sm = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    *out = g_dev_resident[key] = per_sm * sms;
+    return cudaSuccess;
+}
+
+}  // namespace lapsum
 
 using namespace lapsum;
 
@@ -57,12 +114,15 @@ cudaEvent_t take_event() {
     return e;
 }
 
-// RAII: counts one kernel launch and, when profiling, brackets it with events.
+// RAII: counts one kernel launch, names it for tracing tools (an NVTX range
+// around the host-side launch, named after the solver step: free when no tool
+// is attached) and, when profiling, brackets it with events.
 struct Launch {
     const char *name;
     cudaStream_t st;
     cudaEvent_t e0 = nullptr;
     Launch(const char *nm, cudaStream_t s) : name(nm), st(s) {
+        nvtxRangePushA(nm);
         std::lock_guard<std::mutex> lk(g_prof_mu);
         ++g_launches;
         if (g_prof_mode && (g_prof_filter.empty() || std::strstr(nm, g_prof_filter.c_str()))) {
@@ -71,6 +131,7 @@ struct Launch {
         }
     }
     ~Launch() {
+        nvtxRangePop();
         if (!e0) return;
         std::lock_guard<std::mutex> lk(g_prof_mu);
         cudaEvent_t e1 = take_event();
@@ -143,7 +204,7 @@ cudaError_t ws_base(Workspace *w, int64_t rows) {
 cudaError_t ws_sort(Workspace *w, int64_t cap) {
     cudaError_t e = grow(w->keys0, w->keys0_n, (size_t)cap);
     if (e == cudaSuccess) e = grow(w->keys1, w->keys1_n, (size_t)cap);
-    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256);
+    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256 + 2);   // + the give-up and clean-up counts
     if (e == cudaSuccess) e = grow(w->chunkcnt, w->chunkcnt_n, (size_t)4 * 256 * sort_grid_max());
     if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, (size_t)sort_record_doubles(cap));
     return e;
@@ -273,7 +334,7 @@ void binomial_ranks(int64_t s, double pi, double delta, int64_t &jR, int64_t &jL
 int check_args(const float *scores, int64_t rows, int64_t n, double k, double t) {
     if (!scores || rows < 1 || n < 1 || n >= (int64_t(1) << 31)) return LAPSUM_ERR_ARG;
     if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_ERR_ARG;
-    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_ERR_ARG;
+    if (!(t >= LAPSUM_T_MIN && t <= LAPSUM_T_MAX)) return LAPSUM_ERR_ARG;
     return LAPSUM_OK;
 }
 
@@ -293,6 +354,31 @@ int full_sort_rows(Workspace *w, const float *r, int64_t rows, int64_t n, double
 }
 
 }  // namespace
+
+namespace lapsum {
+struct ShardWs {
+    Ctl *ctl;
+    double *partials;
+    uint32_t *skeys, *hist1, *cand;
+    float *band;
+    int64_t band_cap;
+};
+// The stream's workspace for one slice of a split row (k_shard.cu): a control
+// block and partials for one row, sample keys (s), select histograms and
+// candidates, a band buffer of band_cap scores.  Zero sizes keep what is there.
+int shard_workspace(struct CUstream_st *stream, int64_t s, int64_t band_cap, ShardWs *out) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Workspace *w = get_ws(st);
+    w->rows = 1;
+    LAPSUM_TRY(ws_base(w, 1));
+    LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)std::max<int64_t>(s, 1)));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, (size_t)HIST_WORDS));
+    LAPSUM_TRY(grow(w->selcand, w->selcand_n, (size_t)SEL_CAND_WORDS));
+    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)std::max<int64_t>(band_cap, 1)));
+    *out = ShardWs{w->ctl, w->partials, w->skeys, w->hist1, w->selcand, w->band, (int64_t)w->band_n};
+    return LAPSUM_OK;
+}
+}  // namespace lapsum
 
 // ===================================================================== ABI --
 extern "C" {
@@ -319,12 +405,13 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     lapsum_options opt{};
     if (opt_in) opt = *opt_in;
     if (opt.delta != 0.0 && !(opt.delta > 0.0 && opt.delta < 1.0)) return LAPSUM_ERR_ARG;
-    if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < 0) return LAPSUM_ERR_ARG;
+    if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < -1) return LAPSUM_ERR_ARG;
     if (opt.force_path < 0 || opt.force_path > 2) return LAPSUM_ERR_ARG;
     if (opt.certify != LAPSUM_CERTIFY_PASS && opt.certify != LAPSUM_CERTIFY_FUSED) return LAPSUM_ERR_ARG;
     if (opt.widen != 0 && opt.widen != 1) return LAPSUM_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
-    const int32_t spin_cap = opt.spin_cap ? opt.spin_cap : (1 << 20);
+    // spin_cap -1: grid-barrier waits give up at their first poll (exercises the timeout path)
+    const int32_t spin_cap = opt.spin_cap > 0 ? opt.spin_cap : (opt.spin_cap == 0 ? (1 << 20) : 0);
     Workspace *w = get_ws(st);
 
     int path = opt.force_path;
@@ -359,6 +446,8 @@ int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, do
     P.inv_t = 1.0 / t;
     P.seed = opt.seed;
     P.row = 0;
+    P.shard_off = 0;
+    P.n_total = n;
     int64_t s = 0, band_cap = 0;
     rc = lapsum_bracket_plan(n, k, &opt, &s, &P.jR, &P.jL, &band_cap);
     if (rc) return rc;
@@ -463,7 +552,7 @@ int lapsum_backward(const float *scores, const double *b, const float *g, int64_
                     double t, float *grad_out, struct CUstream_st *stream_in) {
     if (!scores || !b || !g || !grad_out || rows < 1 || n < 1 || n >= (int64_t(1) << 31))
         return LAPSUM_ERR_ARG;
-    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_ERR_ARG;
+    if (!(t >= LAPSUM_T_MIN && t <= LAPSUM_T_MAX)) return LAPSUM_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
     if (n <= 65536 || rows > 65535) {   // short rows: one CTA per row
         Launch L("rowvjp", st);
@@ -500,6 +589,7 @@ static void fill_stats(const Ctl &c, lapsum_stats *out) {
     out->sum_p = c.sum_p;
     out->j_star = c.j_star;
     out->widened = c.widened;
+    out->flags = c.flags;
 }
 
 static int stats_rc(const Ctl &c) {

@@ -263,14 +263,51 @@ __device__ __forceinline__ float laplace_cdf2(float x2) {
     return x2 < 0.0f ? e : 1.0f - e;
 }
 
+// The returned p = F((r - b)/t), written so that sum p keeps the budget k over
+// millions of scores (the method's exact-budget property, technical summary
+// section 2.1).  Two systematic errors of a plain fp32 evaluation would add up
+// over the row instead of cancelling:
+//  * the fp32 scale s = log2(e)/t carries one relative rounding error shared by
+//    every score; s is split into s_hi + s_lo and x2 = d s_hi + d s_lo by an fma,
+//    so what is left is each score's own rounding;
+//  * where p is mid-range (|x2| < 1, p in (1/4, 3/4)) every score's p is of the
+//    same size and any bias of the fp32 exponential would add up linearly, so
+//    there p is formed in fp64 from the fp64 threshold and rounded once.
+// Elsewhere p < 1/4 or 1 - p < 1/4 and the fp32 value is used.
+struct PForm {
+    float b_hi, b_lo, s_hi, s_lo;
+    double b, s2d;
+    __device__ __forceinline__ float operator()(float r) const {
+        const float d = (r - b_hi) - b_lo;
+        const float x2 = fmaf(d, s_lo, d * s_hi);
+        if (fabsf(x2) >= 1.0f) return laplace_cdf2(x2);
+        const double xd = ((double)r - b) * s2d;
+        const double e = 0.5 * exp2(-fabs(xd));
+        return (float)(xd < 0.0 ? e : 1.0 - e);
+    }
+};
+__device__ __forceinline__ PForm make_pform(double b, double scale) {
+    PForm f;
+    f.b = b;
+    f.s2d = scale;
+    f.b_hi = (float)b;
+    f.b_lo = (float)(b - (double)f.b_hi);
+    f.s_hi = (float)scale;
+    f.s_lo = (float)(scale - (double)f.s_hi);
+    return f;
+}
+
 // One VJP output, (f/t)(g - lambda), f = e^{-|x|}/2, from the base-2 argument.
+// The factor 1/(2t) enters the exponent, f/t = 2^{l2h - |x2|} with
+// l2h = log2(1/(2t)) (vjp_scale2), so an output that fp32 can hold comes out
+// even where f alone would underflow (t tiny, b far from every score).
 // g - lambda uses a hi/lo split of the fp64 lambda: when a few scores carry
 // almost all of sum f, lambda sits within an fp32 ulp of their g, and the split
 // keeps the difference exact.
-__device__ __forceinline__ float vjp_term2(float x2, float g, float half_inv_t, float lam_hi,
-                                           float lam_lo) {
-    return (half_inv_t * exp2f(-fabsf(x2))) * ((g - lam_hi) - lam_lo);
+__device__ __forceinline__ float vjp_term2(float x2, float g, float l2h, float lam_hi, float lam_lo) {
+    return exp2f(l2h - fabsf(x2)) * ((g - lam_hi) - lam_lo);
 }
+__device__ __forceinline__ float vjp_scale2(double inv_t) { return (float)log2(0.5 * inv_t); }
 
 // ----------------------------------------------------- near-tier exp --
 // 2^{-w} for 0 <= w <= 1000, the fp64 terms of the tail sums.  Table-driven
@@ -391,7 +428,10 @@ constexpr size_t bulk_smem_bytes() {
 // memory and calls body(const float4 *chunk[NSRC], int64_t first_vector) once
 // per chunk, by every thread of the CTA (each thread reads its own vectors of
 // the chunk).  Returns the number of vectors covered by full chunks (the rest
-// is the caller's tail).  On a wait that gives up it sets ST_TIMEOUT.
+// is the caller's tail).  If a wait gives up (in any thread), the CTA sets
+// ST_TIMEOUT, issues no further copy, waits (bounded again) for the copies it
+// has in flight and stops streaming; the caller's result is then invalid and
+// the error reaches the host through the status word.
 template <int NSRC, typename Body>
 __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC], int64_t n4, bool reverse,
                                                unsigned char *smem, int32_t *status, Body &&body) {
@@ -420,16 +460,24 @@ __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC],
                 bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &bars[s]);
         }
     }
-    bool ok = true;
     for (int64_t i = 0; i < mine; ++i) {
         const int s = (int)(i % BULK_STAGES);
         const uint32_t parity = (uint32_t)((i / BULK_STAGES) & 1);
-        if (!mbar_wait(&bars[s], parity, BULK_WAIT_CAP)) ok = false;
+        const bool ok = mbar_wait(&bars[s], parity, BULK_WAIT_CAP);
         const float4 *chunk[NSRC];
 #pragma unroll
         for (int q = 0; q < NSRC; ++q) chunk[q] = buf + ((size_t)s * NSRC + q) * BULK_F4;
         body(chunk, chunk_of(i) * BULK_F4);
-        __syncthreads();   // every thread is done with stage s
+        if (!__syncthreads_and(ok)) {   // every thread is done with stage s; a wait gave up
+            if (threadIdx.x == 0) {
+                if (status) atomicOr(status, ST_TIMEOUT);
+                // the copies issued and not yet consumed: chunks i .. i + STAGES - 1
+                for (int64_t j = i; j < i + BULK_STAGES && j < mine; ++j)
+                    mbar_wait(&bars[j % BULK_STAGES], (uint32_t)((j / BULK_STAGES) & 1), BULK_WAIT_CAP);
+            }
+            __syncthreads();
+            return nch * BULK_F4;
+        }
         if (threadIdx.x == 0 && i + BULK_STAGES < mine) {
             fence_proxy_async_smem();
             mbar_expect_tx(&bars[s], BYTES * NSRC);
@@ -439,7 +487,6 @@ __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC],
                 bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &bars[s]);
         }
     }
-    if (!ok && status) atomicOr(status, ST_TIMEOUT);
     return nch * BULK_F4;
 }
 
@@ -476,29 +523,44 @@ __device__ __forceinline__ void st_release_u32(unsigned *p, unsigned v) {
 // Grid-wide barrier of a cooperative launch (every CTA is resident): an
 // arrival counter and a generation word in device memory; the last CTA to
 // arrive resets the counter and advances the generation.  The wait is bounded:
-// after cap polls the CTA sets ST_TIMEOUT in *status and goes on.
-__device__ __forceinline__ void grid_sync(unsigned *count, unsigned *gen, int cap, int32_t *status) {
+// after cap polls (or as soon as another CTA has given up: ST_TIMEOUT in
+// *status) the CTA sets ST_TIMEOUT and the barrier returns false.  The caller
+// then returns at once, so no CTA runs a phase after a barrier that did not
+// complete; the CTAs still waiting give up in turn (the one that left never
+// arrives again), each after a bounded wait.  A CTA also skips arriving when
+// the status already carries ST_TIMEOUT.
+__device__ __forceinline__ int32_t ld_volatile_s32(const int32_t *p) {
+    return *reinterpret_cast<const volatile int32_t *>(p);
+}
+__device__ __forceinline__ bool grid_sync(unsigned *count, unsigned *gen, int cap, int32_t *status) {
+    __shared__ int s_gave_up;
     __syncthreads();
     if (threadIdx.x == 0) {
-        const unsigned g = ld_acquire_u32(gen);   // read before arriving: it cannot advance yet
-        __threadfence();
-        if (atomicAdd(count, 1u) == gridDim.x - 1) {
-            atomicExch(count, 0u);
+        int gave_up = (ld_volatile_s32(status) & ST_TIMEOUT) != 0;
+        if (!gave_up) {
+            const unsigned g = ld_acquire_u32(gen);   // read before arriving: it cannot advance yet
             __threadfence();
-            st_release_u32(gen, g + 1u);
-        } else {
-            int it = 0;
-            while (ld_acquire_u32(gen) == g) {
-                if (++it > cap) {
-                    atomicOr(status, ST_TIMEOUT);
-                    break;
+            if (atomicAdd(count, 1u) == gridDim.x - 1) {
+                atomicExch(count, 0u);
+                __threadfence();
+                st_release_u32(gen, g + 1u);
+            } else {
+                int it = 0;
+                while (ld_acquire_u32(gen) == g) {
+                    if (++it > cap || (ld_volatile_s32(status) & ST_TIMEOUT)) {
+                        atomicOr(status, ST_TIMEOUT);
+                        gave_up = 1;
+                        break;
+                    }
+                    __nanosleep(64);
                 }
-                __nanosleep(64);
             }
+            __threadfence();
         }
-        __threadfence();
+        s_gave_up = gave_up;
     }
     __syncthreads();
+    return s_gave_up == 0;
 }
 
 // Relaxed (but coherent at GPU scope) 64-bit accesses, for words that carry their

@@ -44,8 +44,16 @@ struct Ctl {
     unsigned int gbar_count;  // grid barrier of the cooperative sort: arrivals
     unsigned int gbar_gen;    //   and generation
     // backward
+    double hL, lR;            // fused certification: band terms vs a_L and vs a_R
     double vjp_lambda;
-    int32_t vjp_shift;        // every f underflowed: recompute lambda shifted
+    float vjp_min;            // split rows: the slice's smallest |x| (base 2; cleared to +inf)
+    int32_t vjp_shift;        // sum f too small for fp32 terms: recompute lambda shifted
+    int32_t flags;            // FLAG_* bits: which rare routes ran
+};
+
+// Rare routes a solve took (lapsum_stats.flags).
+enum : int32_t {
+    FLAG_SELECT_ALL_KEYS = 1,   // the select's candidate buffer overflowed: it walked every sample key
 };
 
 // Kernel-facing parameters of a bracketing solve.
@@ -74,6 +82,10 @@ struct BracketParams {
     int32_t fused_cert;       // certification folded into the streaming pass
     int32_t widen;            // a widening round follows a missed bracket
     int32_t round2;           // this launch belongs to the widening round
+    // a row split across ranks: this rank holds scores [shard_off, shard_off + n) of
+    // a row of n_total (the sample draws global indices; 0 and n for a whole row)
+    int64_t shard_off;
+    int64_t n_total;
 };
 
 constexpr int64_t HIST_WORDS = 65536 + 256;

@@ -43,6 +43,13 @@ inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, si
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// Per-device launch set-up (lapsum_api.cu), cached per (device, kernel) under a
+// lock, so a process that drives several GPUs configures each one:
+int device_sm_count();   // SMs of the current device
+cudaError_t set_max_dynamic_smem(const void *kern, size_t bytes);   // once per (device, kernel, size)
+// CTAs of `kern` (block threads, dynamic smem bytes) resident on the current device at once
+cudaError_t resident_ctas(const void *kern, int threads, size_t smem, int *out);
+
 // in-CTA full-sort solver (k_rows.cu)
 int rowsolve_capacity();
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
@@ -67,6 +74,10 @@ cudaError_t launch_vjp_reduce(const float *r, const double *b, const float *g, i
                               Ctl *ctl, double *partials, cudaStream_t st);
 cudaError_t launch_selftest_math(int which, const double *in, double *out, double *ref, int64_t n,
                                 cudaStream_t st);
+// one slice of a split row: {sum e, sum g e, min |x2|} with terms 2^{sh2 - |x2|}
+// (ctl->vjp_min and ticket[3] of the row's control block must start at +inf / 0)
+cudaError_t launch_vjp_slice_partial(const float *r, const double *b, const float *g, int64_t n, double t,
+                                     float sh2, Ctl *ctl, double *partials, double *part_out, cudaStream_t st);
 cudaError_t launch_vjp_apply(const float *r, const double *b, const float *g, int64_t rows, int64_t n, double t,
                              const Ctl *ctl, float *grad, cudaStream_t st);
 
@@ -79,7 +90,7 @@ struct SortArgs {
     int64_t n_host;            // element count
     int64_t cap;               // upper bound of the element count (grid sizing)
     uint32_t *keys[2];         // ping-pong key buffers [cap]
-    unsigned long long *hist;  // [4][256]
+    unsigned long long *hist;  // [4][256], then two words: sorts that gave up, and that count at the last clean-up
     uint32_t *chunkcnt;        // [4][256][grid]: digit counts of each CTA's chunk of tiles
     double *tilebuf;           // locate per-tile data
     Ctl *ctl;

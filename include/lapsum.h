@@ -63,6 +63,12 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
 #define LAPSUM_ERR_CUDA            -5     /* a CUDA runtime call failed                     */
 #define LAPSUM_ERR_NO_ROOT         -6     /* solver found no crossing (internal)            */
 
+/* Temperatures accepted by every entry point: LAPSUM_T_MIN <= t <= LAPSUM_T_MAX.
+ * The kernels form x = (r - b)/t in fp32 with the scale log2(e)/t; outside this
+ * range that scale (or its inverse) is not a finite, normal fp32 number. */
+#define LAPSUM_T_MIN 1e-36
+#define LAPSUM_T_MAX 1e36
+
 /* Certification modes (lapsum_options.certify) */
 #define LAPSUM_CERTIFY_PASS  0
 #define LAPSUM_CERTIFY_FUSED 1
@@ -82,7 +88,11 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
  *   band_cap    capacity of the band buffer in scores (default
  *               max(65536, 4 n (jL - jR + 2)/s), at most n).  A larger band
  *               fails certification and takes the full-sort fallback.
- *   spin_cap    polls before an inter-block wait gives up (default 2^20).
+ *   spin_cap    polls before a grid-barrier wait of the device-wide sort gives up
+ *               (default 2^20).  -1: give up at the first poll that finds the
+ *               barrier still closed -- a way to exercise the timeout path, which then
+ *               reports LAPSUM_ERR_DEVICE_TIMEOUT through lapsum_get_stats and
+ *               leaves the library ready for the next call.
  *   force_path  LAPSUM_PATH_* (default AUTO: bracketing when n >= 2^20, else
  *               full sort).  Bracketing solves the rows of a batch together:
  *               every kernel takes one slice of its grid per row (rows <=
@@ -134,6 +144,8 @@ typedef struct {
  *   b         the threshold of row 0
  *   sum_p     sum of the fp32 p of row 0, accumulated in fp64
  *   widened   1 if the widening round ran (then s..G_aR describe its bracket)
+ *   flags     rare routes taken: 1 = more than 8192 sample keys shared a target's
+ *             16-bit prefix, so the bracket select walked the whole sample
  */
 typedef struct {
     int32_t path, verdict, status, fallback;
@@ -146,13 +158,14 @@ typedef struct {
     double  sum_p;
     int64_t j_star;
     int64_t widened;
-    int64_t reserved[3];
+    int64_t flags;
+    int64_t reserved[2];
 } lapsum_stats;
 
 /*
  * Forward: p_out_dev[rows][n] = F((scores - b)/t), b_out_dev[rows] = b (fp64).
  *   scores_dev  fp32 [rows][n], finite
- *   rows >= 1, n >= 1, 0 < k < n (real), t > 0 finite
+ *   rows >= 1, n >= 1, 0 < k < n (real), LAPSUM_T_MIN <= t <= LAPSUM_T_MAX
  *   p_out_dev   fp32 [rows][n] (may not alias scores_dev)
  *   b_out_dev   fp64 [rows]
  * Path: "Fast LapSum", technical summary section 2.2 (full-sort solver;
@@ -261,6 +274,87 @@ LAPSUM_API int lapsum_selftest_math(int which, const double *in_dev, double *out
 LAPSUM_API int lapsum_backward_noalloc(const float *scores_dev, const double *b_dev,
                                        const float *g_dev, int64_t rows, int64_t n, double t,
                                        float *grad_out_dev, struct CUstream_st *stream);
+
+/*
+ * One row split across GPUs ("Fast LapSum", technical summary section 4.1:
+ * rows of 1e8 scores and beyond, past one GPU's memory).  The row of n_total
+ * scores is cut into contiguous slices, one per rank (one process per GPU);
+ * rank q holds scores [offset_q, offset_q + n_local_q).  Every rank calls the
+ * entry points below on its slice, in this order, on one stream, and exchanges
+ * the small device buffers they produce with its collective library between the
+ * calls (exact_budget_soft_b200.sharded does it with torch.distributed/NCCL):
+ *
+ *   lapsum_shard_plan        sizes of the exchange buffers (host only)
+ *   lapsum_shard_sample      this rank's share of the bracketing sample
+ *       -> all-reduce (sum) of the xbuf words over the ranks (as int32 or uint32)
+ *   lapsum_shard_stream      bracket (identical on every rank) and the streaming
+ *                            pass over the slice, certification terms folded in
+ *       -> all-gather of the LAPSUM_SHARD_PART-double records, rank order;
+ *          all-gather of each slice's band scores (record[2] of them), rank order
+ *   lapsum_shard_solve       the row's counts and sums, the verdict, b
+ *       (verdict 0: the bracket failed certification; the caller gathers the
+ *        whole row and solves it with lapsum_forward_ex, force_path FULLSORT)
+ *   lapsum_shard_p           p of the slice at b
+ * and for the VJP:
+ *   lapsum_shard_vjp_partial {sum e, sum g e, min |x|} of the slice, e = e^{shift-|x|}
+ *       -> all-gather of the 3-double records, rank order; if the summed e is
+ *          below 2^-96 (every score far from b), call it again with shift =
+ *          the smallest min |x| over the ranks and all-gather again
+ *   lapsum_shard_vjp_apply   grad of the slice
+ *
+ * The sample is the one-GPU sample of the whole row (same Philox counters, the
+ * index drawn over n_total; each rank fills the draws that land in its slice),
+ * so the bracket, the counts and the verdict equal those of lapsum_forward_ex on
+ * the whole row (certify = LAPSUM_CERTIFY_FUSED).  Sums are combined in rank
+ * order on every rank, so every rank gets the same b.  Options as for
+ * lapsum_forward_ex, except widen and force_path (LAPSUM_ERR_ARG).  Pointers
+ * are device memory on the rank's GPU; the library's per-stream workspace
+ * carries state from one call to the next (lapsum_get_stats after
+ * lapsum_shard_solve reports the whole row's bracket, counts and verdict).
+ */
+#define LAPSUM_SHARD_PART 10   /* c_L c_R c_band S_L S_R hL lR kmax kinv status (doubles) */
+
+/* xbuf_words: uint32 words of the sample exchange buffer; band_cap: capacity of
+ * every band buffer (a slice's, and the gathered band's: more fails certification). */
+LAPSUM_API int lapsum_shard_plan(int64_t n_total, double k, const lapsum_options *opt,
+                                 int64_t *xbuf_words, int64_t *band_cap);
+
+/* Fills xbuf_dev[xbuf_words] with this slice's share of the sample (zero where
+ * another rank owns the draw) and its select histograms; clears the workspace. */
+LAPSUM_API int lapsum_shard_sample(const float *scores_dev, int64_t n_local, int64_t offset, int64_t n_total,
+                                   double k, double t, const lapsum_options *opt, uint32_t *xbuf_dev,
+                                   struct CUstream_st *stream);
+
+/* From the summed xbuf: the bracket; then the slice's streaming pass.  Writes its
+ * record part_dev[LAPSUM_SHARD_PART] and its band scores to band_dev[band_cap]
+ * (record[2] of them; a count above band_cap keeps counting, and fails the row). */
+LAPSUM_API int lapsum_shard_stream(const float *scores_dev, int64_t n_local, int64_t offset, int64_t n_total,
+                                   double k, double t, const lapsum_options *opt, const uint32_t *xbuf_dev,
+                                   double *part_dev, float *band_dev, struct CUstream_st *stream);
+
+/* parts_dev[ranks][LAPSUM_SHARD_PART] in rank order; band_all_dev: the ranks'
+ * band scores concatenated (band_total of them).  Writes b_out_dev[0] (fp64) and
+ * verdict_out_dev[0] (1 certified; 0: use the full-sort fallback). */
+LAPSUM_API int lapsum_shard_solve(const double *parts_dev, int64_t ranks, const float *band_all_dev,
+                                  int64_t band_total, int64_t n_total, double k, double t,
+                                  const lapsum_options *opt, double *b_out_dev, int32_t *verdict_out_dev,
+                                  struct CUstream_st *stream);
+
+/* p_out_dev[n_local] = F((scores - b)/t) for the slice, b = b_dev[0]. */
+LAPSUM_API int lapsum_shard_p(const float *scores_dev, int64_t n_local, double t, const double *b_dev,
+                              float *p_out_dev, struct CUstream_st *stream);
+
+/* part_dev[3] = {sum_i e_i, sum_i g_i e_i, min_i |x_i|} over the slice,
+ * e_i = e^{shift - |x_i|}, x_i = (scores_i - b)/t; shift >= 0. */
+LAPSUM_API int lapsum_shard_vjp_partial(const float *scores_dev, const double *b_dev, const float *g_dev,
+                                        int64_t n_local, double t, double shift, double *part_dev,
+                                        struct CUstream_st *stream);
+
+/* lambda = sum(sum g e)/sum(sum e) over parts_dev[ranks][3] (one shift for all,
+ * rank order); grad_out_dev[n_local] = (f_i/t)(g_i - lambda) for the slice. */
+LAPSUM_API int lapsum_shard_vjp_apply(const float *scores_dev, const double *b_dev, const float *g_dev,
+                                      int64_t n_local, double t, const double *parts_dev, int64_t ranks,
+                                      float *grad_out_dev, struct CUstream_st *stream);
 
 /* Number of kernel launches enqueued by this library since load (a counter). */
 LAPSUM_API int64_t lapsum_launch_count(void);

@@ -55,7 +55,8 @@ def test_strerror(lib):
 
 @pytest.mark.parametrize("rows,n,k,t", [(0, 10, 1.0, 1.0), (1, 0, 1.0, 1.0), (1, 10, 0.0, 1.0),
                                         (1, 10, 10.0, 1.0), (1, 10, 2.0, 0.0), (1, 10, 2.0, -1.0),
-                                        (1, 10, float("nan"), 1.0), (1, 10, 2.0, float("inf"))])
+                                        (1, 10, float("nan"), 1.0), (1, 10, 2.0, float("inf")),
+                                        (1, 10, 2.0, 1e-37), (1, 10, 2.0, 1e37)])
 def test_bad_arguments_rejected_on_host(lib, rows, n, k, t):
     lib.lapsum_forward.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_double, C.c_double,
                                    C.c_void_p, C.c_void_p, C.c_void_p]
@@ -63,8 +64,10 @@ def test_bad_arguments_rejected_on_host(lib, rows, n, k, t):
     assert lib.lapsum_forward(fake, rows, n, k, t, fake, fake, None) == -1
     lib.lapsum_backward.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64,
                                     C.c_double, C.c_void_p, C.c_void_p]
-    if rows < 1 or n < 1 or not (t > 0) or t == float("inf"):
+    if rows < 1 or n < 1 or not (1e-36 <= t <= 1e36):
         assert lib.lapsum_backward(fake, fake, fake, rows, n, t, fake, None) == -1
+        lib.lapsum_backward_noalloc.argtypes = lib.lapsum_backward.argtypes
+        assert lib.lapsum_backward_noalloc(fake, fake, fake, rows, n, t, fake, None) == -1
 
 
 def test_null_pointers_rejected(lib):

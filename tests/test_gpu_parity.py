@@ -534,15 +534,9 @@ def test_bracketing_extreme_budgets_and_temperatures(L, orc, k, t):
     assert st["rc"] == 0 and st["path"] == 2
     plan = L.bracket_plan(n, k)
     check_bracket_integers(orc, r[0], k, t, st, 0, plan["s"], 1e-6)
-    # with t large every p is mid-range and the fp32 p carry a bias of a fraction
-    # of an ulp that adds up over 2^20 scores: the mass tolerance holds for the
-    # exact mass at b (checked in check_row) and the rounded sum keeps within its
-    # rounding bound sum ulp(p_i)/2
-    wide = t > 1.0
-    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0], exact_sum=not wide)
-    if wide:
-        bound = np.sum(np.spacing(p[0].astype(np.float32)).astype(np.float64)) / 2
-        assert abs(p[0].astype(np.float64).sum() - k) <= bound
+    # with t large every p is mid-range (p ~ k/n): the plain sum of the returned
+    # fp32 p keeps the budget too (no bias adds up over the 2^20 scores)
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
 
 
 def test_batched_rows_report_a_nonfinite_row(L):
