@@ -232,6 +232,13 @@ def run_ours(args):
         if rec.get("sources_sha") == kernel_sources_sha():   # counters only valid for the kernels they came from
             traffic = rec["kernels"].get(dom)
     model_bytes = sum(KERNEL_BYTES.values()) * w.n
+    # bytes actually moved (ncu DRAM counters of the streaming kernels, one launch each per step), when
+    # they were taken on the kernels as built now
+    dram_step = None
+    if os.path.exists(tf):
+        rec = json.load(open(tf))
+        if rec.get("sources_sha") == kernel_sources_sha() and all(k in rec["kernels"] for k in KERNEL_BYTES):
+            dram_step = int(sum(rec["kernels"][k] for k in KERNEL_BYTES))
     out = {
         "metric": METRIC, "value": round(med, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(tot / args.steps, 4), "higher_is_better": False,
@@ -245,6 +252,8 @@ def run_ours(args):
         "model_bytes_per_step": model_bytes,
         "model_gbs": round(model_bytes / (med * 1e-3) / 1e9, 1),
         "model_frac_of_8TBs": round(model_bytes / (med * 1e-3) / 8e12, 4),
+        "dram_bytes_per_step": dram_step,
+        "dram_frac_of_8TBs": round(dram_step / (med * 1e-3) / 8e12, 4) if dram_step else None,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "alg_bytes_per_launch": alg_bytes},
@@ -265,14 +274,43 @@ def run_ours(args):
             ge_ = torch.from_numpy(W.upstream_grad(we, seed=rank)[0]).cuda()
             pe_, be_, gre_ = torch.empty_like(re_), torch.empty(1, dtype=torch.float64, device="cuda"), torch.empty_like(re_)
 
-            def st_e():
+            def fw_e():
                 L.forward(re_, we.k, we.t, p_out=pe_, b_out=be_)
+
+            def st_e():
+                fw_e()
                 L.backward(re_, be_, ge_, we.t, grad_out=gre_)
 
             mse = time_steps(torch, st_e, max(args.steps, 10), max(args.warmup, 3), flush=lambda: flushbuf.fill_(1.0))
-            by_n[f"{we.n:.0e}"] = {"workload": name, "median_ms_fwd_vjp": round(statistics.median(mse), 4)}
-        by_n["1e+08"] = {"workload": w.name, "median_ms_fwd_vjp": round(med, 4), "fwd_ms": round(med_f, 4)}
+            msf = time_steps(torch, fw_e, max(args.steps, 10), max(args.warmup, 3), flush=lambda: flushbuf.fill_(1.0))
+            me, mf = statistics.median(mse), statistics.median(msf)
+            by_n[f"{we.n:.0e}"] = {"workload": name, "median_ms_fwd_vjp": round(me, 4), "fwd_ms": round(mf, 4),
+                                   "scores_per_s_fwd_vjp": round(we.n / (me * 1e-3)),
+                                   "scores_per_s_fwd": round(we.n / (mf * 1e-3))}
+        by_n["1e+08"] = {"workload": w.name, "median_ms_fwd_vjp": round(med, 4), "fwd_ms": round(med_f, 4),
+                         "scores_per_s_fwd_vjp": round(w.n / (med * 1e-3)),
+                         "scores_per_s_fwd": round(w.n / (med_f * 1e-3))}
         out["by_n"] = by_n
+        # the same 1e8 scores in random order: no chunk of the row lies wholly on one side of the bracket
+        wr = W.WORKLOADS["levels1e8_shuffled"]
+        rr = torch.from_numpy(W.scores(wr, seed=rank)[0]).cuda()
+
+        def st_rand():
+            L.forward(rr, wr.k, wr.t, p_out=p, b_out=b)
+            L.backward(rr, b, g, wr.t, grad_out=grad)
+
+        def fw_rand():
+            L.forward(rr, wr.k, wr.t, p_out=p, b_out=b)
+
+        msr = time_steps(torch, st_rand, args.steps, args.warmup)
+        msrf = time_steps(torch, fw_rand, args.steps, args.warmup)
+        st_r = L.get_stats()
+        assert st_r["rc"] == 0 and st_r["path"] == 2
+        out["random_order_1e8"] = {"workload": f"{wr.name}: 1 row x n=1e8, k=1e6, t=0.1, scores in random order",
+                                   "median_ms_fwd_vjp": round(statistics.median(msr), 4),
+                                   "fwd_ms": round(statistics.median(msrf), 4), "verdict": int(st_r["verdict"]),
+                                   "vs_sorted_headline": round(statistics.median(msr) / med, 3)}
+        del rr
         # the full-sort row path (one CTA per row: sort, scan, root, p) and its VJP
         rows_out = {}
         for name in ("n4096", "rows1024"):
@@ -383,6 +421,12 @@ def run_ours(args):
                   "d2h_bytes_per_step": 8 * w.n + 8}
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(w)
+        if not args.headline_only:   # the oracle on every workload of the measurement table
+            out["oracle_by_config"] = {nm: oracle_config(W.WORKLOADS[nm])
+                                       for nm in ("n4096", "rows1024", "pixels1m", "laplace1e7")}
+            out["oracle_by_config"][w.name] = {"fwd_ms": out["cpu_baseline"]["fwd_ms"],
+                                               "fwd_vjp_ms": out["cpu_baseline"]["value"]}
+            out["oracle_by_config"]["host"] = host_cores()
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist:
@@ -405,14 +449,34 @@ def oracle_step(w, n_sample, seed=0):
     return (time.perf_counter() - t0) * 1e3
 
 
-def cpu_baseline(w, n_sample=10_000_000):
+def host_cores() -> dict:
     import oracle
-    ms = oracle_step(w, n_sample)
-    scaled = ms * w.n / n_sample
-    return {"value": round(scaled, 1), "unit": "ms (per 1e8 scores, scaled linearly)", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"one fp64 oracle fwd+VJP (Newton-safeguarded bisection, p, VJP) on {n_sample:.0e} scores "
-                      f"drawn from the workload (k scaled to {w.k * n_sample / w.n:g}), x{w.n // n_sample} to 1e8"}
+    return {"cores": oracle.num_threads(), "nproc": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
+
+
+def oracle_config(w) -> dict:
+    """The oracle on one whole workload (every row): fwd (solve + p) and fwd+VJP, ms."""
+    import oracle
+    r, g = W.scores(w), W.upstream_grad(w)
+    t0 = time.perf_counter()
+    bs = []
+    for i in range(w.rows):
+        b = oracle.solve(r[i], w.k, w.t, method=1)
+        oracle.p(r[i], b, w.t)
+        bs.append(b)
+    t1 = time.perf_counter()
+    for i in range(w.rows):
+        oracle.vjp(r[i], g[i], bs[i], w.t)
+    t2 = time.perf_counter()
+    return {"fwd_ms": round((t1 - t0) * 1e3, 1), "fwd_vjp_ms": round((t2 - t0) * 1e3, 1)}
+
+
+def cpu_baseline(w):
+    t = oracle_config(w)
+    return {"value": t["fwd_vjp_ms"], "unit": "ms", **host_cores(), "kind": "oracle",
+            "fwd_ms": t["fwd_ms"],
+            "sample": f"one fp64 oracle fwd+VJP (Newton-safeguarded bisection, p, VJP) on the whole {w.name} "
+                      f"workload (n = {w.n:.0e}), measured, not scaled"}
 
 
 def run_reference(args):
@@ -421,7 +485,9 @@ def run_reference(args):
         return
     import oracle
     w = W.WORKLOADS[args.workload]
-    n_sample = 2_000_000
+    # each step: the oracle on the whole workload when K + W steps of it fit about two
+    # minutes of host time (about 3 s a step at n = 1e8), else on a sample scaled to n
+    n_sample = w.n if (args.steps + args.warmup) <= 40 else 10_000_000
     for _ in range(args.warmup):
         oracle_step(w, n_sample)
     ms = [oracle_step(w, n_sample) * w.n / n_sample for _ in range(args.steps)]
@@ -430,9 +496,11 @@ def run_reference(args):
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": f"{w.name}: 1 row x n=1e8 fp32, k=1e6, t=0.1"},
-           "cpu_baseline": {"value": round(v, 1), "unit": "ms", "kind": "oracle", "cores": oracle.num_threads(),
-                            "sample": f"each step: fp64 oracle fwd+VJP on {n_sample:.0e} scores of the workload, "
-                                      f"scaled x{w.n // n_sample} to 1e8"},
+           "cpu_baseline": {"value": round(v, 1), "unit": "ms", "kind": "oracle", **host_cores(),
+                            "sample": (f"each step: fp64 oracle fwd+VJP on the whole workload (n = {w.n:.0e})"
+                                       if n_sample == w.n else
+                                       f"each step: fp64 oracle fwd+VJP on {n_sample:.0e} scores of the workload, "
+                                       f"scaled x{w.n // n_sample} to 1e8")},
            "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 

@@ -21,7 +21,10 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblapsum.so")
+# LAPSUM_CHECKED=1 loads the checked build (bounds tests on computed indices,
+# guard words around the workspace; slower, for debugging)
+CHECKED = os.environ.get("LAPSUM_CHECKED") == "1"
+LIB_PATH = os.path.join(_HERE, "liblapsum_checked.so" if CHECKED else "liblapsum.so")
 
 PATH_AUTO, PATH_FULLSORT, PATH_BRACKET = 0, 1, 2
 CERTIFY_PASS, CERTIFY_FUSED = 0, 1
@@ -29,8 +32,10 @@ CERTIFY_PASS, CERTIFY_FUSED = 0, 1
 FLAG_SELECT_ALL_KEYS = 1
 # error codes (LAPSUM_ERR_* of the C header)
 ERR_ARG, ERR_NONFINITE, ERR_ALLOC, ERR_DEVICE_TIMEOUT, ERR_CUDA, ERR_NO_ROOT = -1, -2, -3, -4, -5, -6
+ERR_BOUNDS = -7
 ERRORS = {0: "ok", -1: "invalid argument", -2: "non-finite score", -3: "workspace allocation failed",
-          -4: "device wait timeout", -5: "CUDA runtime error", -6: "no crossing found"}
+          -4: "device wait timeout", -5: "CUDA runtime error", -6: "no crossing found",
+          -7: "index or guard word out of bounds (checked build)"}
 
 
 class LapSumError(RuntimeError):
@@ -69,6 +74,7 @@ SHARD_PART = 10   # doubles in a slice's streaming-pass record (LAPSUM_SHARD_PAR
 def _load() -> C.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_budget_soft_b200.build`"
+                          " (--checked for the checked build)"
                           " (there is no CPU fallback)")
     lib = C.CDLL(LIB_PATH)
     vp, i64, dbl = C.c_void_p, C.c_int64, C.c_double
@@ -161,6 +167,10 @@ def forward(scores: torch.Tensor, k: float, t: float, p_out: torch.Tensor | None
                                b_out.data_ptr(), C.byref(opts) if opts is not None else None,
                                _stream(stream))
     _check(rc, "lapsum_forward")
+    if CHECKED:   # the checked build reports an out-of-bounds index through the device status
+        st = Stats()
+        if lib.lapsum_get_stats(C.byref(st), _stream(stream)) == ERR_BOUNDS:
+            raise LapSumError(ERR_BOUNDS, "lapsum_forward")
     return p_out, b_out
 
 

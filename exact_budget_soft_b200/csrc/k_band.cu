@@ -191,7 +191,8 @@ __device__ __forceinline__ double bin_edge(uint32_t klo, int s, unsigned J, unsi
 // whose edges straddle k as computed, with no flag, as an edge's G can differ
 // from the step before it by rounding.
 __device__ __noinline__ void band_level(const float *src, int64_t nsrc, SubBand &S, BinSums &B, Aff *scratch,
-                                       unsigned *hit, double s2d, double k, const double *tab, int32_t *status) {
+                                       unsigned *hit, double s2d, double k, const double *tab, int32_t *status,
+                                       int32_t *bstatus) {
     const int tid = threadIdx.x;
     const uint32_t klo = S.klo, khi = S.khi;
     const double top = S.top, bot = S.bot;
@@ -210,6 +211,7 @@ __device__ __noinline__ void band_level(const float *src, int64_t nsrc, SubBand 
         const uint32_t kk = desc_key(x);
         if (kk < klo || kk > khi) return;
         const unsigned j = (kk - klo) >> s;
+        if (!in_bounds(j < J && J <= (unsigned)BS_BINS, bstatus)) return;
         const double xd = (double)x;
         const double eh = bin_edge(klo, s, J, j, top, bot);
         const double el = bin_edge(klo, s, J, j + 1, top, bot);
@@ -500,7 +502,8 @@ band_select_kernel(const float *__restrict__ band_all, int64_t band_cap, double 
             nsrc = min(s_got, (unsigned)GATHER_CAP);   // the band's count by construction
             gathered = true;
         }
-        band_level(src, nsrc, s_sb, s_bins, s_scan, &s_hit, s2d, k, s_tab, first ? &ctl->status : nullptr);
+        band_level(src, nsrc, s_sb, s_bins, s_scan, &s_hit, s2d, k, s_tab, first ? &ctl->status : nullptr,
+                   &ctl->status);
         first = false;
     }
     if (tid != 0) return;

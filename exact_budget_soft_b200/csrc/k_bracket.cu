@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(256) sample_kernel(BracketParams Pg) {
         philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
         I = (int64_t)__umul64hi(x0, (uint64_t)P.n_total) - P.shard_off;
         mine = I >= 0 && I < P.n;
+        if (mine && !in_bounds(I < P.n && P.s <= (int64_t)gridDim.x * blockDim.x, &P.ctl->status)) mine = false;
         if (!mine) P.keys[j] = 0u;   // a split row's exchange sums the ranks' shares
     }
     if (mine) {
@@ -795,7 +796,10 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
         unsigned pos = sq_n + inc - cnt;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            if ((sp >> i) & 1u) sq[pos++] = pick8(v0, v1, i);
+            if ((sp >> i) & 1u) {
+                if (in_bounds(pos < (unsigned)SQ, &P.ctl->status)) sq[pos] = pick8(v0, v1, i);
+                ++pos;
+            }
         sq_n += total;
         __syncwarp();
         if (sq_n >= 32) {

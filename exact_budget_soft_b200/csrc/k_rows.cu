@@ -218,6 +218,127 @@ rowvjp_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
     }
 }
 
+// One row of up to BLOCK * EPT scores per CTA, read from HBM once: each thread
+// keeps |x2| of its EPT scores in registers and the row's g in shared memory.
+//   1. m = min |x2| over the row (block minimum);
+//   2. e_i = 2^{m - |x2_i|} (the largest is 1: no underflow however far b is),
+//      lambda = sum g e / sum e (fp32 per thread, fp64 across the block);
+//   3. grad_i = e_i 2^{l2h - m} (g_i - lambda), l2h = log2(1/(2t)) -- or, when
+//      2^{l2h - m} is not a normal fp32 number (b farther than ~87 t from every
+//      score and t not small), from 2^{l2h - |x2_i|} directly, re-reading r.
+template <int BLOCK, int EPT>
+__global__ void __launch_bounds__(BLOCK, 1)
+rowvjp_reg_kernel(const float *__restrict__ scores, const double *__restrict__ b_in,
+                  const float *__restrict__ g, int64_t n_arg, double inv_t, float *__restrict__ grad) {
+    static_assert(EPT % 4 == 0, "float4 slots");
+    extern __shared__ __align__(16) float s_g[];
+    __shared__ float s_min[BLOCK / 32];
+    __shared__ double s_red[2 * (BLOCK / 32)];
+    pdl_enter();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = (int)n_arg;
+    const int64_t off = (int64_t)blockIdx.x * n_arg;
+    const float *r = scores + off;
+    const float *gg = g + off;
+    float *out = grad + off;
+    const XForm xf = make_xform(b_in[blockIdx.x], inv_t * LOG2E);
+    const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(gg) |
+                                         reinterpret_cast<uintptr_t>(out)) & 15) == 0;
+    // slot i of thread t: element 4 (t + (i/4) BLOCK) + i%4 (vector rows), else t + i BLOCK
+    auto elem = [&](int i) -> int { return vec ? 4 * (tid + (i >> 2) * BLOCK) + (i & 3) : tid + i * BLOCK; };
+    float ax[EPT];
+    float amin = CUDART_INF_F;
+    if (vec) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(r);
+        const float4 *g4 = reinterpret_cast<const float4 *>(gg);
+        float4 *sg4 = reinterpret_cast<float4 *>(s_g);
+#pragma unroll
+        for (int q = 0; q < EPT / 4; ++q) {
+            const int i4 = tid + q * BLOCK;
+            if (4 * i4 < n) {
+                const float4 v = r4[i4];
+                sg4[i4] = g4[i4];
+                ax[4 * q + 0] = fabsf(xf(v.x));
+                ax[4 * q + 1] = fabsf(xf(v.y));
+                ax[4 * q + 2] = fabsf(xf(v.z));
+                ax[4 * q + 3] = fabsf(xf(v.w));
+            } else {
+                ax[4 * q + 0] = ax[4 * q + 1] = ax[4 * q + 2] = ax[4 * q + 3] = CUDART_INF_F;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPT; ++i) {
+            const int j = tid + i * BLOCK;
+            if (j < n) {
+                s_g[j] = gg[j];
+                ax[i] = fabsf(xf(r[j]));
+            } else {
+                ax[i] = CUDART_INF_F;
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) amin = fminf(amin, fminf(ax[i], 3.0e38f));   // finite: |x| may overflow fp32
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amin = fminf(amin, __shfl_xor_sync(FULL, amin, o));
+    if (lane == 0) s_min[warp] = amin;
+    __syncthreads();   // also: s_g complete
+    float m = s_min[0];
+#pragma unroll
+    for (int w = 1; w < BLOCK / 32; ++w) m = fminf(m, s_min[w]);
+    float sf = 0.f, sgf = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+        const float e = exp2f(m - ax[i]);   // padding slots: 2^-inf = 0
+        const int j = elem(i);
+        const float gj = j < n ? s_g[j] : 0.f;
+        sf += e;
+        sgf = fmaf(gj, e, sgf);
+        ax[i] = e;
+    }
+    double v[2] = {(double)sf, (double)sgf};
+    block_sum<BLOCK, 2>(v, s_red);
+    if (tid == 0) s_red[0] = v[1] / v[0];
+    __syncthreads();
+    const double lam = s_red[0];
+    const float lam_hi = (float)lam, lam_lo = (float)(lam - (double)lam_hi);
+    const float l2h = vjp_scale2(inv_t);
+    const float cexp = l2h - m;
+    if (cexp >= -125.0f) {   // 2^{l2h - m} is a normal fp32 number: scale the kept e_i
+        const float C = exp2f(cexp);
+        if (vec) {
+            float4 *o4 = reinterpret_cast<float4 *>(out);
+            const float4 *sg4 = reinterpret_cast<const float4 *>(s_g);
+#pragma unroll
+            for (int q = 0; q < EPT / 4; ++q) {
+                const int i4 = tid + q * BLOCK;
+                if (4 * i4 < n) {
+                    const float4 w = sg4[i4];
+                    float4 o;
+                    o.x = (ax[4 * q + 0] * C) * ((w.x - lam_hi) - lam_lo);
+                    o.y = (ax[4 * q + 1] * C) * ((w.y - lam_hi) - lam_lo);
+                    o.z = (ax[4 * q + 2] * C) * ((w.z - lam_hi) - lam_lo);
+                    o.w = (ax[4 * q + 3] * C) * ((w.w - lam_hi) - lam_lo);
+                    o4[i4] = o;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < EPT; ++i) {
+                const int j = tid + i * BLOCK;
+                if (j < n) out[j] = (ax[i] * C) * ((s_g[j] - lam_hi) - lam_lo);
+            }
+        }
+    } else {   // every output is below 2^-125 |g - lambda|: each from its own exponent
+#pragma unroll
+        for (int i = 0; i < EPT; ++i) {
+            const int j = elem(i);
+            if (j < n) out[j] = vjp_term2(xf(r[j]), s_g[j], l2h, lam_hi, lam_lo);
+        }
+    }
+}
+
 // ------------------------------------------------------------ launchers --
 template <int BLOCK, int KPT>
 static cudaError_t launch_rowsolve(const float *scores, int64_t rows, int64_t n, double k, double t,
@@ -239,6 +360,13 @@ cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, d
 
 cudaError_t launch_rowvjp(const float *scores, const double *b, const float *g, int64_t rows,
                           int64_t n, double t, float *grad, cudaStream_t st) {
+    if (n <= 1024 * 32) {   // the row's |x| in registers and its g in shared memory: one read
+        auto kern = rowvjp_reg_kernel<1024, 32>;
+        const size_t smem = (size_t)((n + 3) & ~int64_t(3)) * sizeof(float);
+        const cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), 1024 * 32 * sizeof(float));
+        if (e != cudaSuccess) return e;
+        return launch_k(kern, (unsigned)rows, 1024, smem, st, scores, b, g, n, 1.0 / t, grad);
+    }
     return launch_k(rowvjp_kernel<1024>, (unsigned)rows, 1024, 0, st, scores, b, g, n, 1.0 / t, grad);
 }
 

@@ -141,6 +141,15 @@ struct Launch {
 };
 
 // ------------------------------------------------------------ workspace --
+// The checked build (-DLAPSUM_CHECKED) puts GUARD_BYTES of a fixed pattern after
+// every workspace buffer and verifies them at the end of every call.
+#ifdef LAPSUM_CHECKED
+constexpr size_t GUARD_BYTES = 256;
+#else
+constexpr size_t GUARD_BYTES = 0;
+#endif
+constexpr unsigned char GUARD_FILL = 0xA5;
+
 template <typename T>
 cudaError_t grow(T *&p, size_t &have, size_t need) {
     if (need <= have && p) return cudaSuccess;
@@ -150,9 +159,11 @@ cudaError_t grow(T *&p, size_t &have, size_t need) {
         have = 0;
     }
     size_t n = need < 64 ? 64 : need;
-    cudaError_t e = cudaMalloc(reinterpret_cast<void **>(&p), n * sizeof(T));
+    cudaError_t e = cudaMalloc(reinterpret_cast<void **>(&p), n * sizeof(T) + GUARD_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaMemset(p, 0, n * sizeof(T));
+    if (e == cudaSuccess && GUARD_BYTES)
+        e = cudaMemset(reinterpret_cast<char *>(p) + n * sizeof(T), GUARD_FILL, GUARD_BYTES);
     have = n;
     return e;
 }
@@ -176,6 +187,28 @@ struct Workspace {
         cudaFree(keys0); cudaFree(keys1); cudaFree(hist);
         cudaFree(chunkcnt); cudaFree(tilebuf);
         *this = Workspace();
+    }
+
+    // checked build: every buffer's guard bytes still hold the fill pattern
+    // (synchronises the stream); LAPSUM_ERR_BOUNDS otherwise
+    int verify_guards(cudaStream_t st) const {
+        if (!GUARD_BYTES) return LAPSUM_OK;
+        const std::pair<const void *, size_t> bufs[] = {
+            {ctl, ctl_n * sizeof(Ctl)}, {partials, partials_n * sizeof(double)},
+            {skeys, skeys_n * 4}, {hist1, hist1_n * 4}, {selcand, selcand_n * 4}, {band, band_n * 4},
+            {keys0, keys0_n * 4}, {keys1, keys1_n * 4}, {hist, hist_n * 8}, {chunkcnt, chunkcnt_n * 4},
+            {tilebuf, tilebuf_n * 8}};
+        if (cudaStreamSynchronize(st) != cudaSuccess) return LAPSUM_ERR_CUDA;
+        unsigned char g[GUARD_BYTES ? GUARD_BYTES : 1];
+        for (const auto &b : bufs) {
+            if (!b.first) continue;
+            if (cudaMemcpy(g, static_cast<const char *>(b.first) + b.second, GUARD_BYTES, cudaMemcpyDeviceToHost) !=
+                cudaSuccess)
+                return LAPSUM_ERR_CUDA;
+            for (size_t i = 0; i < GUARD_BYTES; ++i)
+                if (g[i] != GUARD_FILL) return LAPSUM_ERR_BOUNDS;
+        }
+        return LAPSUM_OK;
     }
 };
 
@@ -392,13 +425,27 @@ const char *lapsum_strerror(int code) {
         case LAPSUM_ERR_DEVICE_TIMEOUT: return "an inter-block wait gave up (spin cap)";
         case LAPSUM_ERR_CUDA: return "CUDA runtime error";
         case LAPSUM_ERR_NO_ROOT: return "no crossing found";
+        case LAPSUM_ERR_BOUNDS: return "checked build: an index or a guard word was out of bounds";
         default: return "unknown error";
     }
 }
 
+static int forward_impl(const float *scores, int64_t rows, int64_t n, double k, double t,
+                        float *p_out, double *b_out, const lapsum_options *opt_in,
+                        struct CUstream_st *stream_in);
+
 int lapsum_forward_ex(const float *scores, int64_t rows, int64_t n, double k, double t,
                       float *p_out, double *b_out, const lapsum_options *opt_in,
                       struct CUstream_st *stream_in) {
+    const int rc = forward_impl(scores, rows, n, k, t, p_out, b_out, opt_in, stream_in);
+    if (rc || !GUARD_BYTES) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    return get_ws(st)->verify_guards(st);
+}
+
+static int forward_impl(const float *scores, int64_t rows, int64_t n, double k, double t,
+                        float *p_out, double *b_out, const lapsum_options *opt_in,
+                        struct CUstream_st *stream_in) {
     int rc = check_args(scores, rows, n, k, t);
     if (rc) return rc;
     if (!p_out || !b_out) return LAPSUM_ERR_ARG;
@@ -564,7 +611,7 @@ int lapsum_backward(const float *scores, const double *b, const float *g, int64_
     LAPSUM_TRY(ws_base(w, rows));
     { Launch L("vjp_reduce", st); LAPSUM_TRY(launch_vjp_reduce(scores, b, g, rows, n, t, w->ctl, w->partials, st)); }
     { Launch L("vjp_apply", st); LAPSUM_TRY(launch_vjp_apply(scores, b, g, rows, n, t, w->ctl, grad_out, st)); }
-    return LAPSUM_OK;
+    return w->verify_guards(st);
 }
 
 static void fill_stats(const Ctl &c, lapsum_stats *out) {
@@ -593,6 +640,7 @@ static void fill_stats(const Ctl &c, lapsum_stats *out) {
 }
 
 static int stats_rc(const Ctl &c) {
+    if (c.status & ST_BOUNDS) return LAPSUM_ERR_BOUNDS;
     if (c.status & ST_NONFINITE) return LAPSUM_ERR_NONFINITE;
     if (c.status & ST_TIMEOUT) return LAPSUM_ERR_DEVICE_TIMEOUT;
     if ((c.status & ST_NO_ROOT) && !(c.path == 2 && c.fallback_ran)) return LAPSUM_ERR_NO_ROOT;

@@ -24,6 +24,21 @@ namespace lapsum {
 
 constexpr unsigned FULL = 0xffffffffu;
 
+// ------------------------------------------------------- checked build --
+// Built with -DLAPSUM_CHECKED (liblapsum_checked.so), every computed index of a
+// store or gather below is tested against its buffer before the access: an
+// index outside sets ST_BOUNDS in the row's status word (reported as
+// LAPSUM_ERR_BOUNDS) and the access is skipped -- never a trap.  In the normal
+// build the test compiles away.
+#ifdef LAPSUM_CHECKED
+__device__ __forceinline__ bool in_bounds(bool ok, int32_t *status) {
+    if (!ok && status) atomicOr(status, ST_BOUNDS);
+    return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, int32_t *) { return true; }
+#endif
+
 // ---------------------------------------------------------------- keys --
 // Order-preserving map float -> uint32 whose ASCENDING order is the DESCENDING
 // order of the floats (largest score first).

@@ -11,6 +11,7 @@ enum : int32_t {
     ST_TIMEOUT = 2,
     ST_BAND_OVERFLOW = 4,
     ST_NO_ROOT = 8,
+    ST_BOUNDS = 16,   // checked build: a computed index fell outside its buffer (the access was skipped)
 };
 
 // Device-resident control block of one single-row solve.  Every field is

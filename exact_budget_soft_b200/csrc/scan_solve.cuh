@@ -96,7 +96,7 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
                 my_hist[d] = base + __popc(peers);
             }
             base = __shfl_sync(FULL, base, leader) + __popc(peers & lt_mask);
-            s_keys[spad((int)base)] = key[i];
+            if (in_bounds(base < (uint32_t)C::CAP, nullptr)) s_keys[spad((int)base)] = key[i];
             __syncwarp();
         }
         __syncthreads();

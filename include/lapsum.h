@@ -62,6 +62,7 @@ struct CUstream_st;                       /* cudaStream_t == struct CUstream_st*
 #define LAPSUM_ERR_DEVICE_TIMEOUT  -4     /* an inter-block wait gave up (spin cap)         */
 #define LAPSUM_ERR_CUDA            -5     /* a CUDA runtime call failed                     */
 #define LAPSUM_ERR_NO_ROOT         -6     /* solver found no crossing (internal)            */
+#define LAPSUM_ERR_BOUNDS          -7     /* checked build only: an index or guard word failed */
 
 /* Temperatures accepted by every entry point: LAPSUM_T_MIN <= t <= LAPSUM_T_MAX.
  * The kernels form x = (r - b)/t in fp32 with the scale log2(e)/t; outside this
@@ -135,7 +136,8 @@ typedef struct {
  *   path      LAPSUM_PATH_FULLSORT or LAPSUM_PATH_BRACKET
  *   verdict   bracketing: 1 certified, 0 not certified (fallback ran); -1 n/a
  *   status    device error bits: 1 non-finite score, 2 wait timeout,
- *             4 band overflow, 8 no crossing found
+ *             4 band overflow, 8 no crossing found, 16 index out of bounds
+ *             (checked build)
  *   s, jR, jL sample size and order-statistic ranks of the bracket
  *   a_L, a_R  bracket ends (fp32, rounded outward)
  *   c_L, c_band, c_R   scores below a_L, in [a_L, a_R), at or above a_R

@@ -188,6 +188,7 @@ def test_tail_sums_and_certification_values(L, orc, n, dist, k, t, certify):
 
 
 # ------------------------------------------------------- every row, rows1024 --
+@pytest.mark.slow
 def test_rows1024_every_row(L, orc):
     w = W.WORKLOADS["rows1024"]
     r, g = W.scores(w), W.upstream_grad(w)

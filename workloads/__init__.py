@@ -18,6 +18,7 @@ classifier are not available here):
   laplace1e7    1 x 1e7         Laplace(0,1)                      k=1e5     t=0.05
   levels1e8     1 x 1e8         256 levels of U(-4,4), level i ->  k=1e6     t=0.1
                                 -4+(i+1/2)/32, sorted descending
+  levels1e8_shuffled            the same scores in random order     k=1e6     t=0.1
 
 Every workload draws its scores, its random positions and its upstream
 gradient g ~ N(0,1) from three independent PCG64 streams spawned from one
@@ -62,6 +63,8 @@ WORKLOADS: dict[str, Workload] = {
                  "bracketing (+ forced full-sort fallback run)"),
         Workload("batch64x1m", 64, 1_048_576, 10_486.0, 0.05, "normal",
                  "batched bracketing (64 rows of 2^20, k = 1% of each row)"),
+        Workload("levels1e8_shuffled", 1, 100_000_000, 1_000_000.0, 0.1, "levels256_shuffled",
+                 "the levels1e8 scores in random order (every chunk of the row mixes levels)"),
     ]
 }
 
@@ -97,6 +100,11 @@ def _draw(dist: str, rows: int, n: int, rs: np.random.Generator, rp: np.random.G
         return out
     if dist == "levels256_desc":
         return np.stack([_levels256_desc(rs, n) for _ in range(rows)])
+    if dist == "levels256_shuffled":   # the same multiset of levels, then a random permutation
+        out = np.stack([_levels256_desc(rs, n) for _ in range(rows)])
+        for i in range(rows):
+            rp.shuffle(out[i])
+        return out
     if dist == "uniform":
         return rs.uniform(-1.0, 1.0, (rows, n)).astype(np.float32)
     raise ValueError(f"unknown distribution {dist!r}")
