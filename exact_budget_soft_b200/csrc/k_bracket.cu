@@ -387,6 +387,224 @@ __global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams Pg) {
     }
 }
 
+// ========================================================= sample + select --
+// The sample and the bracket's order statistics in one launch (the one-GPU
+// path): every CTA draws its share of the sample as sample_kernel does; the CTA
+// that finishes last (one ticket per row) runs the whole radix select on it --
+// round 1 from the histograms the sampler built, the keys under each target's
+// 16-bit prefix gathered into shared memory, rounds 2 and 3 there -- so no
+// second launch and no global candidate buffer sit on the critical path.
+constexpr int SS_BLOCK = 1024;
+
+// The bracket ends from the selected keys (and, in the widening round, the new
+// bracket on the missed side); thread 0.
+__device__ __forceinline__ void select_finish(const BracketParams &P, const bool valid[2], uint32_t prefR,
+                                              uint32_t prefL) {
+    Ctl *ctl = P.ctl;
+    const float yR = desc_key_to_float(prefR);
+    const float yL = desc_key_to_float(prefL);
+    const float aR = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
+    const float aL = valid[1] ? yL : -CUDART_INF_F;
+    if (P.round2) {   // the missed side becomes the bracket; the stream starts afresh
+        if (ctl->widen_dir > 0) {   // b >= old a_R
+            ctl->a_L = ctl->a_R;
+            ctl->jL = ctl->jR;
+            ctl->a_R = aR;
+            ctl->jR = P.jR;
+        } else {                    // b < old a_L
+            ctl->a_R = ctl->a_L;
+            ctl->jR = ctl->jL;
+            ctl->a_L = aL;
+            ctl->jL = P.jL;
+        }
+        ctl->c_band = 0ull;
+        ctl->band_kmax = 0u;
+        ctl->band_kinv = 0u;
+        atomicAnd(&ctl->status, ~(ST_NO_ROOT | ST_BAND_OVERFLOW));   // the first band solve's misses
+        ctl->widened = 1;
+    } else {
+        ctl->a_R = aR;
+        ctl->a_L = aL;
+        ctl->jR = P.jR;
+        ctl->jL = P.jL;
+    }
+    ctl->s = P.s;
+    ctl->path = 2;
+    ctl->verdict = -1;
+}
+
+__global__ void __launch_bounds__(SS_BLOCK) sample_select_kernel(BracketParams Pg) {
+    const BracketParams P = at_row(Pg, blockIdx.y);
+    extern __shared__ __align__(16) uint32_t s_cand[];   // [2][SEL_CAND], the last CTA's candidates
+    __shared__ uint32_t s_h0[256];
+    __shared__ uint32_t s_w[SS_BLOCK / 32];
+    __shared__ uint32_t h8[2][256];
+    __shared__ uint32_t s_pref[2], s_rank[2], s_bin0[2], s_cnt[2];
+    __shared__ bool s_last;
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (tid < 256) s_h0[tid] = 0u;
+    pdl_enter();
+    if (P.round2 && !widen_starts(P)) return;   // the same sample again, for the widened ranks
+    __syncthreads();
+    Ctl *ctl = P.ctl;
+    // ---- the sample (as sample_kernel)
+    const int64_t j = (int64_t)blockIdx.x * SS_BLOCK + tid;
+    if (j < P.s) {
+        uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
+        philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
+        const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n_total) - P.shard_off;
+        if (in_bounds(I >= 0 && I < P.n, &ctl->status)) {
+            const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
+            const double E = -sample_ln(U);
+            const double L = (x1 & 1ull) ? E : -E;
+            const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
+            const uint32_t key = desc_key(__double2float_rd(y));
+            P.keys[j] = key;
+            const uint32_t bin = key >> 16;
+            const unsigned peers = __match_any_sync(__activemask(), bin);
+            if (lane == __ffs(peers) - 1) {
+                atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
+                atomicAdd(&s_h0[bin >> 8], (uint32_t)__popc(peers));
+            }
+        }
+    }
+    __syncthreads();
+    if (tid < 256 && s_h0[tid]) atomicAdd(P.hist1 + SEL_BINS + tid, s_h0[tid]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&ctl->ticket[5], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // ---- the last CTA: the radix select over the whole sample
+    const int64_t s = P.s;
+    const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
+    const uint32_t want0[2] = {(uint32_t)(valid[0] ? P.jR : 1), (uint32_t)(valid[1] ? P.jL : 1)};
+    if (tid < 2) { s_bin0[tid] = 0u; s_rank[tid] = 1u; s_pref[tid] = 0u; s_cnt[tid] = 0u; }
+    {   // round 1a: the top byte of each target (thread t < 256 owns bin t)
+        const uint32_t c = tid < 256 ? __ldcg(P.hist1 + SEL_BINS + tid) : 0u;
+        const uint32_t incl = block_incl_scan_u32(c, s_w);
+        if (tid < 256) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                if (incl - c < want0[q] && want0[q] <= incl) {
+                    s_bin0[q] = (uint32_t)tid;
+                    s_rank[q] = want0[q] - (incl - c);
+                }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {   // round 1b: the second byte, from the 256 top-16 bins under the first
+        const uint32_t b0 = s_bin0[q], want = s_rank[q];
+        const uint32_t c = tid < 256 ? __ldcg(P.hist1 + b0 * 256 + tid) : 0u;
+        const uint32_t incl = block_incl_scan_u32(c, s_w);
+        if (tid < 256 && incl - c < want && want <= incl) {
+            s_pref[q] = ((b0 << 8) | (uint32_t)tid) << 16;
+            s_rank[q] = want - (incl - c);
+        }
+        __syncthreads();
+    }
+    const uint32_t pf[2] = {s_pref[0], s_pref[1]};
+    {   // the keys under either prefix, into shared memory (one vote for four keys)
+        auto take = [&](uint32_t key, bool in) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const bool m = in && valid[q] && (key & 0xffff0000u) == pf[q];
+                const unsigned bal = __ballot_sync(FULL, m);
+                if (!bal) continue;
+                uint32_t base = 0;
+                if (lane == __ffs(bal) - 1) base = atomicAdd(&s_cnt[q], (uint32_t)__popc(bal));
+                base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+                if (m && base < SEL_CAND) s_cand[q * SEL_CAND + base] = key;
+            }
+        };
+        const uint4 *k4 = reinterpret_cast<const uint4 *>(P.keys);
+        const int64_t s4 = s / 4;
+        constexpr int INFL = 4;   // vectors per thread in flight
+        for (int64_t i0 = 0; i0 < s4; i0 += INFL * SS_BLOCK) {
+            uint4 kv[INFL];
+#pragma unroll
+            for (int u = 0; u < INFL; ++u) {
+                const int64_t i = i0 + u * SS_BLOCK + tid;
+                kv[u] = i < s4 ? __ldcg(k4 + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < INFL; ++u) {
+                const bool in = i0 + u * SS_BLOCK + tid < s4;
+                const uint32_t kk[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+                bool hit = false;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hit |= in && (((kk[e] & 0xffff0000u) == pf[0] && valid[0]) ||
+                                  ((kk[e] & 0xffff0000u) == pf[1] && valid[1]));
+                if (!__any_sync(FULL, hit)) continue;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) take(kk[e], in);
+            }
+        }
+        for (int64_t i0 = 4 * s4; i0 < s; i0 += SS_BLOCK) {
+            const int64_t i = i0 + tid;
+            take(i < s ? __ldcg(P.keys + i) : 0u, i < s);
+        }
+    }
+    __syncthreads();
+    // ---- rounds 2, 3 (bits 15..8, 7..0) over the candidates, or over every key
+    const uint32_t cnt[2] = {s_cnt[0], s_cnt[1]};
+    const bool fast[2] = {cnt[0] <= SEL_CAND, cnt[1] <= SEL_CAND};
+    uint32_t mask = 0xffff0000u;
+#pragma unroll 1
+    for (int sh = 8; sh >= 0; sh -= 8) {
+        for (int i = tid; i < 2 * 256; i += SS_BLOCK) (&h8[0][0])[i] = 0u;
+        __syncthreads();
+        const uint32_t pq[2] = {s_pref[0], s_pref[1]};
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            if (!valid[q]) continue;
+            const int64_t c = fast[q] ? (int64_t)cnt[q] : s;
+            for (int64_t i = tid; i < c; i += SS_BLOCK) {
+                const uint32_t key = fast[q] ? s_cand[q * SEL_CAND + i] : __ldcg(P.keys + i);
+                if ((key & mask) == pq[q]) atomicAdd(&h8[q][(key >> sh) & 0xffu], 1u);
+            }
+        }
+        __syncthreads();
+        if (tid < 64) {   // warp q scans target q's 256 bins (8 per lane)
+            const int q = tid >> 5;
+            if (valid[q]) {
+                uint32_t v[8], run = 0;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { v[u] = h8[q][lane * 8 + u]; run += v[u]; }
+                uint32_t incl = run;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t pp = __shfl_up_sync(FULL, incl, o);
+                    if (lane >= o) incl += pp;
+                }
+                const uint32_t want = s_rank[q];
+                uint32_t cum = incl - run;
+                if (cum < want && want <= incl) {
+                    for (int u = 0; u < 8; ++u) {
+                        if (cum + v[u] >= want) {
+                            s_pref[q] |= (uint32_t)(lane * 8 + u) << sh;
+                            s_rank[q] = want - cum;
+                            break;
+                        }
+                        cum += v[u];
+                    }
+                }
+            }
+        }
+        mask |= 0xffu << sh;
+        __syncthreads();
+    }
+    if (tid < 256) P.hist1[SEL_BINS + tid] = 0u;   // the top-byte histogram; the streaming pass clears the rest
+    if (tid == 0) {
+        if ((valid[0] && !fast[0]) || (valid[1] && !fast[1])) ctl->flags |= FLAG_SELECT_ALL_KEYS;
+        select_finish(P, valid, s_pref[0], s_pref[1]);
+        ctl->ticket[5] = 0u;
+    }
+}
+
 // ===================================================== out-of-band passes --
 // The streaming pass (technical summary section 2.2, step 2) and the
 // certification pass (step 4, abstract) walk every score once and, for each
@@ -440,11 +658,12 @@ __device__ __forceinline__ void tier2(float hi, float lo, double dhi, double dlo
 }
 
 struct OobAcc {
-    uint32_t cL, cR, cB;        // stream: below, above; certify: >= a_L, >= a_R, < a_L
+    uint32_t cL, cR, cB;        // stream: below, above; certify: (unused), >= a_R, < a_L
+    uint32_t np;                // certify: scores seen (>= a_L is np - cB for a finite row)
     uint32_t kmax, kinv;        // stream: largest band key and largest complemented band key
     double SL, SR, hL, lR;      // near terms: below, above, band vs a_L, band vs a_R
     float SL2, SR2, hL2, lR2;   // far terms
-    bool bad;
+    float mx;                   // max |score|, NaN-propagating: not finite -> a non-finite score
 };
 
 // Append a band score at a warp-aggregated slot of the band buffer (the count
@@ -477,13 +696,13 @@ template <int MODE>
 __device__ __forceinline__ bool oob_one(float x, bool valid, const Ends &E, OobAcc &a) {
     constexpr bool CERT = MODE == OOB_CERT;
     if (!valid) return false;
-    a.bad |= !(fabsf(x) < CUDART_INF_F);
+    a.mx = max_nan(a.mx, fabsf(x));
     const bool above = x >= E.aR, below = x < E.aL;
     const bool inb = !above && !below && x == x;
     if (CERT) {
         a.cR += above;
         a.cB += below;
-        a.cL += above || inb;
+        a.np += 1;
     } else {
         a.cR += above;
         a.cL += below;
@@ -580,12 +799,12 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
     const bool fin = mn > -CUDART_INF_F && mx < CUDART_INF_F;    // false for NaN too
     const bool equal = mx == mn;
     if (__all_sync(FULL, !ok || (mx < E.farL && fin))) {
-        if (ok) { if (CERT) a.cB += 4; else a.cL += 4; }
+        if (ok) { if (CERT) { a.cB += 4; a.np += 4; } else a.cL += 4; }
         return;
     }
     if (__all_sync(FULL, !ok || (mx < E.midL && fin))) {
         if (ok) {
-            if (CERT) a.cB += 4; else a.cL += 4;
+            if (CERT) { a.cB += 4; a.np += 4; } else a.cL += 4;
             a.SL2 += (ex2_ftz((v.x - E.aL) * E.s2) + ex2_ftz((v.y - E.aL) * E.s2)) +
                      (ex2_ftz((v.z - E.aL) * E.s2) + ex2_ftz((v.w - E.aL) * E.s2));
         }
@@ -593,21 +812,21 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
     }
     if (__all_sync(FULL, !ok || (mx < E.aL && fin))) {            // below a_L, some near it
         if (ok) {
-            if (CERT) a.cB += 4; else a.cL += 4;
+            if (CERT) { a.cB += 4; a.np += 4; } else a.cL += 4;
             tier4<false>(v, equal, E.aL, E.daL, E, a.SL, a.SL2);
         }
         return;
     }
     if (__all_sync(FULL, !ok || (mn >= E.aR && fin))) {           // at or above a_R
         if (ok) {
-            if (CERT) { a.cL += 4; a.cR += 4; } else a.cR += 4;
+            if (CERT) { a.cR += 4; a.np += 4; } else a.cR += 4;
             tier4<true>(v, equal, E.aR, E.daR, E, a.SR, a.SR2);
         }
         return;
     }
     if (__all_sync(FULL, !ok || (mn >= E.aL && mx < E.aR && fin))) {   // inside the band
         if (ok && BANDTERMS) {
-            if (CERT) a.cL += 4;
+            if (CERT) a.np += 4;
             tier4<true>(v, equal, E.aL, E.daL, E, a.hL, a.hL2);
             tier4<false>(v, equal, E.aR, E.daR, E, a.lR, a.lR2);
         }
@@ -628,7 +847,7 @@ __device__ __forceinline__ void oob_vec(const float4 v, bool ok, const Ends &E, 
 // Sparse band scores of a streaming pass go to a queue in shared memory, written
 // out with one global atomic per CTA at the end (a warp-aggregated global push
 // only if the queue fills).
-constexpr int BQ = 4096;
+constexpr int BQ = 2048;
 
 __device__ __forceinline__ float pick8(const float4 &u, const float4 &w, int i) {
     const float lo = (i & 2) ? ((i & 1) ? u.w : u.z) : ((i & 1) ? u.y : u.x);
@@ -636,54 +855,54 @@ __device__ __forceinline__ float pick8(const float4 &u, const float4 &w, int i) 
     return (i & 4) ? hi : lo;
 }
 
-// The common part of the general path for one score: counts and the fp32 tail
-// term; a score near an end (fp64 term) or in the band only sets its bit.
+// The common part of the general path for one score: the counts, and the fp32
+// tail term of a score more than 16 t beyond its end (the bulk of a long row);
+// every other score -- near an end (fp64 term), in the band, or not a number --
+// only sets its bit in sp_m for special_one.  About sixteen instructions, with
+// the two ends' sums kept apart by predicated adds.
 template <int MODE>
-__device__ __forceinline__ void oob_cheap(float x, int bit, const Ends &E, OobAcc &a, uint32_t &near_m,
-                                          uint32_t &band_m) {
+__device__ __forceinline__ void oob_cheap(float x, int bit, const Ends &E, OobAcc &a, uint32_t &sp_m) {
     constexpr bool CERT = MODE == OOB_CERT;
-    a.bad |= !(fabsf(x) < CUDART_INF_F);
+    a.mx = max_nan(a.mx, fabsf(x));
     const bool above = x >= E.aR, below = x < E.aL;
-    const bool inb = !above && !below && x == x;
     if (CERT) {
         a.cR += above;
         a.cB += below;
-        a.cL += above || inb;
     } else {
         a.cR += above;
         a.cL += below;
     }
-    const float z2 = (above ? x - E.aR : E.aL - x) * E.s2;
-    const bool near = (above || below) && z2 <= NEAR2;
+    const float z2 = (above ? x - E.aR : E.aL - x) * E.s2;   // base-2 distance beyond the end (band: <= 0)
     const float f = ex2_ftz(-z2);
-    a.SR2 += (above && !near) ? f : 0.f;
-    a.SL2 += (below && !near) ? f : 0.f;
-    near_m |= near ? (1u << bit) : 0u;
-    band_m |= inb ? (1u << bit) : 0u;
+    const bool far = z2 > NEAR2;                             // false for NaN
+    if (far && above) a.SR2 += f;
+    if (far && below) a.SL2 += f;
+    if (!(far && (above || below))) sp_m |= 1u << bit;
 }
 
 // The rare scores of a general chunk -- near an end (fp64 tail term) or in the
 // band (queue slot, or the two certification terms) -- are staged in a per-warp
-// queue in shared memory and handled 32 at a time, one per lane, so a warp no
-// longer loops as often as its busiest lane has such scores.
-constexpr int SQ = 64;   // staged scores per warp (below 32 between chunks, at most 32 added)
+// queue in shared memory and handled 32 at a time, one per lane, so a warp never
+// loops as often as its busiest lane has such scores, and every batch but the
+// last is full however many a chunk has (on tied levels in random order, a
+// large t puts ~40% of the scores within 16 t of an end).
+constexpr int SQ = 32 + 8 * 32;   // staged scores per warp: below 32 between chunks, at most 256 added
 
-// Up to 32 staged scores, one per lane (lanes >= cnt idle).
+// One rare score per lane (act false: nothing), by the whole warp: the fp64 tail
+// term of a score near an end; for a band score its queue slot and/or its two
+// certification terms.  Not-a-number scores take neither (the status reports them).
 template <int MODE>
-__device__ __forceinline__ void special_batch(const float *q, int cnt, const Ends &E, OobAcc &a,
-                                              const BracketParams &P, unsigned long long cap, int lane,
-                                              float *s_bq, unsigned *s_bn) {
+__device__ __forceinline__ void special_one(float x, bool act, const Ends &E, OobAcc &a, const BracketParams &P,
+                                            unsigned long long cap, int lane, float *s_bq, unsigned *s_bn) {
     constexpr bool CERT = MODE == OOB_CERT;
     constexpr bool BANDTERMS = MODE != OOB_STREAM;
-    const bool act = lane < cnt;
-    const float x = act ? q[lane] : 0.f;
     const bool above = act && x >= E.aR, below = act && x < E.aL;
-    const bool inb = act && !above && !below;
-    {   // a score out of the band was staged for its fp64 tail term
-        const double w = above ? ((double)x - E.daR) * E.s2d : (below ? (E.daL - (double)x) * E.s2d : 0.0);
+    const bool inb = act && !above && !below && x == x;
+    if (above || below) {   // a score out of the band was staged for its fp64 tail term
+        const double w = above ? ((double)x - E.daR) * E.s2d : (E.daL - (double)x) * E.s2d;
         const double e = exp2_neg(w, E.tab);
         if (above) a.SR += e;
-        if (below) a.SL += e;
+        else a.SL += e;
     }
     if (BANDTERMS && inb) {   // the band score's two certification terms
         tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
@@ -706,10 +925,19 @@ __device__ __forceinline__ void special_batch(const float *q, int cnt, const End
     }
 }
 
+// Up to 32 staged scores, one per lane (lanes >= cnt idle).
+template <int MODE>
+__device__ __forceinline__ void special_batch(const float *q, int cnt, const Ends &E, OobAcc &a,
+                                              const BracketParams &P, unsigned long long cap, int lane,
+                                              float *s_bq, unsigned *s_bn) {
+    const bool act = lane < cnt;
+    special_one<MODE>(act ? q[lane] : 0.f, act, E, a, P, cap, lane, s_bq, s_bn);
+}
+
 template <int MODE, bool ADAPT>
 __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, const Ends &E, OobAcc &a,
                                           const BracketParams &P, unsigned long long cap, int lane,
-                                          float *s_bq, unsigned *s_bn, float *sq, unsigned &sq_n,
+                                          float *s_bq, unsigned *s_bn, float *sq, unsigned *sqc, unsigned &sq_n,
                                           unsigned &hist, unsigned &tick) {
     constexpr bool CERT = MODE == OOB_CERT;
     constexpr bool BANDTERMS = MODE != OOB_STREAM;
@@ -733,11 +961,11 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
         const bool eq0 = v0.x == v0.y && v0.y == v0.z && v0.z == v0.w;
         const bool eq1 = v1.x == v1.y && v1.y == v1.z && v1.z == v1.w;
         if (__all_sync(FULL, mx < E.farL && fin)) {            // far below a_L: counts only
-            if (CERT) a.cB += 8; else a.cL += 8;
+            if (CERT) { a.cB += 8; a.np += 8; } else a.cL += 8;
             return;
         }
         if (__all_sync(FULL, mx < E.midL && fin)) {            // below a_L, fp32 terms
-            if (CERT) a.cB += 8; else a.cL += 8;
+            if (CERT) { a.cB += 8; a.np += 8; } else a.cL += 8;
             a.SL2 += ((ex2_ftz((v0.x - E.aL) * E.s2) + ex2_ftz((v0.y - E.aL) * E.s2)) +
                       (ex2_ftz((v0.z - E.aL) * E.s2) + ex2_ftz((v0.w - E.aL) * E.s2))) +
                      ((ex2_ftz((v1.x - E.aL) * E.s2) + ex2_ftz((v1.y - E.aL) * E.s2)) +
@@ -745,20 +973,20 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
             return;
         }
         if (__all_sync(FULL, mx < E.aL && fin)) {              // below a_L, some near it
-            if (CERT) a.cB += 8; else a.cL += 8;
+            if (CERT) { a.cB += 8; a.np += 8; } else a.cL += 8;
             tier4<false>(v0, eq0, E.aL, E.daL, E, a.SL, a.SL2);
             tier4<false>(v1, eq1, E.aL, E.daL, E, a.SL, a.SL2);
             return;
         }
         if (__all_sync(FULL, mn >= E.aR && fin)) {             // at or above a_R
-            if (CERT) { a.cL += 8; a.cR += 8; } else a.cR += 8;
+            if (CERT) { a.cR += 8; a.np += 8; } else a.cR += 8;
             tier4<true>(v0, eq0, E.aR, E.daR, E, a.SR, a.SR2);
             tier4<true>(v1, eq1, E.aR, E.daR, E, a.SR, a.SR2);
             return;
         }
         if (__all_sync(FULL, mn >= E.aL && mx < E.aR && fin)) {   // inside the band
             if (BANDTERMS) {
-                if (CERT) a.cL += 8;
+                if (CERT) a.np += 8;
                 tier4<true>(v0, eq0, E.aL, E.daL, E, a.hL, a.hL2);
                 tier4<false>(v0, eq0, E.aR, E.daR, E, a.lR, a.lR2);
                 tier4<true>(v1, eq1, E.aL, E.daL, E, a.hL, a.hL2);
@@ -773,83 +1001,37 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
     }
     if (ADAPT) hist |= 1u;
     // general path: the cheap part for all eight, then the marked ones
-    uint32_t near_m = 0, band_m = 0;
-    oob_cheap<MODE>(v0.x, 0, E, a, near_m, band_m);
-    oob_cheap<MODE>(v0.y, 1, E, a, near_m, band_m);
-    oob_cheap<MODE>(v0.z, 2, E, a, near_m, band_m);
-    oob_cheap<MODE>(v0.w, 3, E, a, near_m, band_m);
-    oob_cheap<MODE>(v1.x, 4, E, a, near_m, band_m);
-    oob_cheap<MODE>(v1.y, 5, E, a, near_m, band_m);
-    oob_cheap<MODE>(v1.z, 6, E, a, near_m, band_m);
-    oob_cheap<MODE>(v1.w, 7, E, a, near_m, band_m);
-    const uint32_t sp = near_m | band_m;
+    uint32_t sp = 0;
+    oob_cheap<MODE>(v0.x, 0, E, a, sp);
+    oob_cheap<MODE>(v0.y, 1, E, a, sp);
+    oob_cheap<MODE>(v0.z, 2, E, a, sp);
+    oob_cheap<MODE>(v0.w, 3, E, a, sp);
+    oob_cheap<MODE>(v1.x, 4, E, a, sp);
+    oob_cheap<MODE>(v1.y, 5, E, a, sp);
+    oob_cheap<MODE>(v1.z, 6, E, a, sp);
+    oob_cheap<MODE>(v1.w, 7, E, a, sp);
+    if (CERT) a.np += 8;
     const unsigned cnt = __popc(sp);
-    unsigned inc = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned p = __shfl_up_sync(FULL, inc, o);
-        if (lane >= o) inc += p;
-    }
-    const unsigned total = __shfl_sync(FULL, inc, 31);
+    const unsigned total = __reduce_add_sync(FULL, cnt);
     if (total == 0) return;
-    if (total <= 32) {   // stage them; a full batch of 32 goes at once
-        unsigned pos = sq_n + inc - cnt;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if ((sp >> i) & 1u) {
-                if (in_bounds(pos < (unsigned)SQ, &P.ctl->status)) sq[pos] = pick8(v0, v1, i);
-                ++pos;
-            }
-        sq_n += total;
-        __syncwarp();
-        if (sq_n >= 32) {
+    // stage them (slots from the warp's counter, in any order), then handle full batches of 32
+    unsigned pos = 0;
+    if (cnt) pos = atomicAdd(sqc, cnt);
+    while (sp) {
+        if (in_bounds(pos < (unsigned)SQ, &P.ctl->status)) sq[pos] = pick8(v0, v1, __ffs(sp) - 1);
+        ++pos;
+        sp &= sp - 1;
+    }
+    __syncwarp();
+    sq_n += total;
+    if (sq_n >= 32) {
+        do {
             sq_n -= 32;
             special_batch<MODE>(sq + sq_n, 32, E, a, P, cap, lane, s_bq, s_bn);
-        }
-        return;
-    }
-    // a dense chunk: fp64 tail terms of scores near an end, each warp looping as
-    // often as its busiest lane has such scores
-    while (__any_sync(FULL, near_m != 0)) {
-        if (near_m) {
-            const float x = pick8(v0, v1, __ffs(near_m) - 1);
-            near_m &= near_m - 1;
-            if (x >= E.aR) a.SR += exp2_neg(((double)x - E.daR) * E.s2d, E.tab);
-            else           a.SL += exp2_neg((E.daL - (double)x) * E.s2d, E.tab);
-        }
-    }
-    uint32_t band_any = __reduce_or_sync(FULL, band_m);   // components with a band score in some lane
-    if (!band_any) return;
-    if (BANDTERMS) {   // the band scores' two certification terms
-        uint32_t m = band_m;
-        while (__any_sync(FULL, m != 0)) {
-            if (m) {
-                const float x = pick8(v0, v1, __ffs(m) - 1);
-                m &= m - 1;
-                tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
-                tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
-            }
-        }
-    }
-    if (!CERT) {   // the band scores into the CTA's queue
-        const unsigned lt = (1u << lane) - 1u;
-        while (band_any) {
-            const int i = __ffs(band_any) - 1;
-            band_any &= band_any - 1;
-            const bool inb = (band_m >> i) & 1u;
-            const unsigned m = __ballot_sync(FULL, inb);
-            const int leader = __ffs(m) - 1;
-            unsigned base = 0;
-            if (lane == leader) base = atomicAdd(s_bn, (unsigned)__popc(m));
-            const unsigned slot = __shfl_sync(FULL, base, leader) + __popc(m & lt);
-            const float x = pick8(v0, v1, i);
-            if (inb) {
-                a.kmax = max(a.kmax, desc_key(x));
-                a.kinv = max(a.kinv, ~desc_key(x));
-                if (slot < (unsigned)BQ) s_bq[slot] = x;
-            }
-            band_push(x, inb && slot >= (unsigned)BQ, P.band, cap, &P.ctl->c_band, lane, a);   // queue full
-        }
+        } while (sq_n >= 32);
+        __syncwarp();
+        if (lane == 0) *sqc = sq_n;
+        __syncwarp();
     }
 }
 
@@ -893,6 +1075,7 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
     __shared__ double s_tab[32];
     __shared__ float s_bq[CERT ? 1 : BQ];   // sparse band scores of this CTA
     __shared__ float s_sq[SBLOCK / 32][SQ];   // staged rare scores, per warp
+    __shared__ unsigned s_sqc[SBLOCK / 32];   // and each warp's count of them
     __shared__ unsigned s_bn;
     __shared__ unsigned long long s_bbase;
     exp2_table_init(s_tab);
@@ -910,7 +1093,9 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const unsigned long long cap = (unsigned long long)P.band_cap;
-    OobAcc acc{0, 0, 0, 0u, 0u, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, false};
+    OobAcc acc{0, 0, 0, 0, 0u, 0u, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (lane == 0) s_sqc[threadIdx.x >> 5] = 0u;
+    __syncwarp();
     const int64_t n = P.n;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
@@ -924,7 +1109,7 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
         unsigned sq_n = 0, hist = 0, tick = 0;   // the same in every lane of a warp
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
             oob_chunk<MODE, ADAPT>(lds128(ch[0] + threadIdx.x), lds128(ch[0] + threadIdx.x + SBLOCK), E, acc, P, cap,
-                            lane, s_bq, &s_bn, sq, sq_n, hist, tick);
+                                   lane, s_bq, &s_bn, sq, &s_sqc[threadIdx.x >> 5], sq_n, hist, tick);
         });
         __syncwarp();
         if (sq_n) special_batch<MODE>(sq, (int)sq_n, E, acc, P, cap, lane, s_bq, &s_bn);
@@ -945,7 +1130,7 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
         const bool bb = oob_one<MODE>(x, ok, E, acc);
         if (!CERT) band_push(x, bb, P.band, cap, &ctl->c_band, lane, acc);
     }
-    if (__syncthreads_or(acc.bad) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
+    if (__syncthreads_or(!(acc.mx < CUDART_INF_F)) && threadIdx.x == 0) atomicOr(&ctl->status, ST_NONFINITE);
     if (!CERT) {
         __shared__ uint32_t s_two[2];
         band_range_flush(ctl, acc.kmax, acc.kinv, s_two);
@@ -1000,7 +1185,7 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
         }
         return;
     }
-    double v[7] = {(double)acc.cL, (double)acc.cR, (double)acc.cB, acc.SR + (double)acc.SR2,
+    double v[7] = {(double)(acc.np - acc.cB), (double)acc.cR, (double)acc.cB, acc.SR + (double)acc.SR2,
                    acc.SL + (double)acc.SL2, acc.hL + (double)acc.hL2, acc.lR + (double)acc.lR2};
     block_sum<SBLOCK, 7>(v, s_red);
     if (last_block_sum<SBLOCK, 7>(v, P.partials + 8 * (size_t)gridDim.x, &ctl->ticket[1], s_red) &&
@@ -1024,12 +1209,17 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
 // ================================================================= p pass --
 // p = F((r - b)/t), walking forward (the certification pass left the head of
 // the row in L2).  Also sum p (fp64 over fp32 float4 partials) for diagnostics.
+// Four p at once: the fp32 value for all, then -- only in warps where some lane
+// has a mid-range p (one vote) -- the fp64 value for those (PForm).
 __device__ __forceinline__ float4 p_vec(const float4 v, const PForm &pf) {
     float4 o;
-    o.x = pf(v.x);
-    o.y = pf(v.y);
-    o.z = pf(v.z);
-    o.w = pf(v.w);
+    const bool m0 = pf.fast(v.x, o.x), m1 = pf.fast(v.y, o.y), m2 = pf.fast(v.z, o.z), m3 = pf.fast(v.w, o.w);
+    if (__any_sync(FULL, m0 || m1 || m2 || m3)) {
+        if (m0) o.x = pf.mid(v.x);
+        if (m1) o.y = pf.mid(v.y);
+        if (m2) o.z = pf.mid(v.z);
+        if (m3) o.w = pf.mid(v.w);
+    }
     return o;
 }
 
@@ -1357,6 +1547,13 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     return launch_k(select_kernel, dim3((unsigned)per_row, (unsigned)P.rows), SEL_BLOCK, 0, st, P);
 }
 int select_cand_capacity() { return SEL_CAND; }
+cudaError_t launch_sample_select(const BracketParams &P, cudaStream_t st) {
+    const size_t smem = 2 * SEL_CAND * sizeof(uint32_t);
+    const cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(sample_select_kernel), smem);
+    if (e != cudaSuccess) return e;
+    return launch_k(sample_select_kernel, dim3((unsigned)((P.s + SS_BLOCK - 1) / SS_BLOCK), (unsigned)P.rows),
+                    SS_BLOCK, smem, st, P);
+}
 template <typename K>
 static cudaError_t set_smem(K kern, size_t bytes) {
     return set_max_dynamic_smem(reinterpret_cast<const void *>(kern), bytes);

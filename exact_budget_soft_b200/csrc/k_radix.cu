@@ -70,7 +70,7 @@ __device__ void solve_equal_run(const SortArgs &A, int64_t n) {
 //             order): the chunk's digit-p counts.  Barrier.  Each CTA sums the
 //             counts of the chunks before its own (its global start of every
 //             digit), then walks its tiles in order: a stable in-tile ranking
-//             (per-warp digit histograms, digit peers from ballots), a shared-memory
+//             (per-warp digit histograms, __match_any_sync), a shared-memory
 //             scatter and coalesced runs of writes, each digit's running
 //             offset advanced by the tile's count.  Barrier.
 //
@@ -687,10 +687,9 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                             const int li = warp * 32 * K + i * 32 + lane;
                             const bool v = li < cnt_tile;
                             const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
-                            // lanes holding the same digit: eight ballots (measured faster than
-                            // __match_any_sync on B200), restricted to the lanes with a key
-                            const unsigned vm = __ballot_sync(FULL, v);
-                            const unsigned peers = digit_peers(d & 0xffu) & (v ? vm : ~vm);
+                            // lanes holding the same digit (eight ballots measured slower here:
+                            // this kernel is bound by the same ALU pipe they use)
+                            const unsigned peers = __match_any_sync(FULL, d);
                             const int leader = __ffs(peers) - 1;
                             uint32_t bs = 0;
                             if (v && lane == leader) {

@@ -4,10 +4,8 @@
 // threshold curve, interval search, closed-form root; then p = F((r-b)/t).
 //
 // One CTA owns one row of up to BLOCK*KPT scores (32768 at 1024 x 32):
-//  * LSD radix sort of the order-preserving uint32 keys, 8-bit digits, keys in
-//    registers (warp-striped), a shared-memory scatter buffer, per-warp digit
-//    histograms and ballot-based digit-peer ranking (stable); digits on which every
-//    key agrees are skipped;
+//  * sort of the order-preserving uint32 keys: a bitonic network on each thread's
+//    keys in registers, then merge-path levels in shared memory (block_merge_sort);
 //  * each thread then owns a run of KPT consecutive sorted scores: it forms the
 //    links d_j and the run's two affine maps (prefix P and suffix Q), a block
 //    scan composes them, G is evaluated at every run end, the crossing run is
@@ -32,9 +30,7 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *s_keys = reinterpret_cast<uint32_t *>(smem);
     uint32_t *s_hist = reinterpret_cast<uint32_t *>(smem + C::SMEM_KEYS);
-    uint32_t *s_dbase = s_hist + C::NW * 256;
     __shared__ double s_b;
-    __shared__ unsigned s_and, s_or;
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
     pdl_enter();
@@ -45,35 +41,26 @@ rowsolve_kernel(const float *__restrict__ scores, int64_t n_arg, double k, doubl
     const double m0 = 0.0, top = CUDART_INF, P_top = 0.0, bot = -CUDART_INF, Q_bot = 0.0;
     __syncthreads();   // s_tab
 
-    // ---- load keys (warp-striped), pad with the largest key (sorts last)
+    // ---- load keys (warp-striped; any order is a valid input order), pad with the
+    // largest key (sorts last), then sort (a bitonic network per thread, merge
+    // levels in shared memory: measured faster than an 8-bit radix sort here)
     uint32_t key[KPT];
-    uint32_t kand = 0xffffffffu, kor = 0u;
     bool bad = false;
 #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        int idx = warp * C::SEG + i * 32 + lane;
+        const int idx = warp * C::SEG + i * 32 + lane;
         uint32_t kk = 0xffffffffu;
         if (idx < n) {
-            float v = row[idx];
+            const float v = row[idx];
             bad |= !isfinite(v);
             kk = desc_key(v);
-            kand &= kk;   // digits on which the scores agree (padding excluded: it is the
-            kor |= kk;    //   largest key and starts after every score, so ties keep it last)
         }
         key[i] = kk;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        kand &= __shfl_xor_sync(FULL, kand, o);
-        kor |= __shfl_xor_sync(FULL, kor, o);
-    }
-    if (tid == 0) { s_and = 0xffffffffu; s_or = 0u; }
-    __syncthreads();
-    if (lane == 0) { atomicAnd(&s_and, kand); atomicOr(&s_or, kor); }
     if (__syncthreads_or(bad) && tid == 0 && ctl) atomicOr(&ctl->status, ST_NONFINITE);
-    const uint32_t diff = s_and ^ s_or;
 
-    block_radix_sort<BLOCK, KPT>(key, s_keys, s_hist, s_dbase, diff);
+    block_merge_sort<BLOCK, KPT>(key, s_keys);
+    __syncthreads();
 
     int64_t jstar = 0;
     int32_t *st = ctl ? &ctl->status : nullptr;
@@ -354,7 +341,15 @@ int rowsolve_capacity() { return RowCfg<1024, 32>::CAP; }
 
 cudaError_t launch_rowsolve_rows(const float *scores, int64_t rows, int64_t n, double k, double t,
                                  float *p, double *b, Ctl *ctl, cudaStream_t st) {
+    // Few rows (at most two per SM): each row's latency is the time, so a row takes
+    // a full 1024-thread CTA with as few keys per thread as it needs (shorter
+    // sequential runs in the sort and the scan).  Many short rows: 256-thread CTAs,
+    // eight per SM.
+    const bool few = rows <= 2 * (int64_t)device_sm_count();
+    if (n <= RowCfg<1024, 4>::CAP && few) return launch_rowsolve<1024, 4>(scores, rows, n, k, t, p, b, ctl, st);
     if (n <= RowCfg<256, 16>::CAP) return launch_rowsolve<256, 16>(scores, rows, n, k, t, p, b, ctl, st);
+    if (n <= RowCfg<1024, 8>::CAP && few) return launch_rowsolve<1024, 8>(scores, rows, n, k, t, p, b, ctl, st);
+    if (n <= RowCfg<1024, 16>::CAP && few) return launch_rowsolve<1024, 16>(scores, rows, n, k, t, p, b, ctl, st);
     return launch_rowsolve<1024, 32>(scores, rows, n, k, t, p, b, ctl, st);
 }
 

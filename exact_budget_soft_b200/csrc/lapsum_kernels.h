@@ -65,6 +65,8 @@ int stream_grid();
 int64_t partial_stride(int64_t rows);   // doubles of per-block partials per row
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st);
+// the sample and its select in one launch (the last CTA of each row selects)
+cudaError_t launch_sample_select(const BracketParams &P, cudaStream_t st);
 int select_cand_capacity();
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st);
@@ -89,7 +91,7 @@ struct SortArgs {
     int64_t rows;              // rows the kernel walks, one after another (each gated)
     int64_t n_host;            // element count
     int64_t cap;               // upper bound of the element count (grid sizing)
-    uint32_t *keys[2];         // ping-pong key buffers [cap]
+    uint32_t *keys[2];         // ping-pong key buffers [cap]: the workspace's, and the caller's p output
     unsigned long long *hist;  // [4][256], then two words: sorts that gave up, and that count at the last clean-up
     uint32_t *chunkcnt;        // [4][256][grid]: digit counts of each CTA's chunk of tiles
     double *tilebuf;           // locate per-tile data

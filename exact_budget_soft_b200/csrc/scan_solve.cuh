@@ -112,6 +112,77 @@ __device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t 
     }
 }
 
+// Ascending sorting network on N keys in registers (bitonic: log2 N (log2 N + 1)/2
+// stages of N/2 compare-exchanges; every index is a compile-time constant).
+template <int N>
+__device__ __forceinline__ void bitonic_regs(uint32_t (&k)[N]) {
+#pragma unroll
+    for (int kk = 2; kk <= N; kk <<= 1) {
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const uint32_t a = k[i], b = k[l];
+                    const uint32_t lo = min(a, b), hi = max(a, b);
+                    if ((i & kk) == 0) { k[i] = lo; k[l] = hi; } else { k[i] = hi; k[l] = lo; }
+                }
+            }
+        }
+    }
+}
+
+// Block-wide merge sort of KPT keys per thread (ascending), the alternative to
+// the radix sort for one CTA's row: each thread sorts its keys in registers,
+// then log2(BLOCK) merge levels double the sorted runs in shared memory.  At a
+// level of runs of L, thread t produces outputs [KPT t, KPT t + KPT) of the
+// merge of its pair of runs: it finds where its outputs start by a binary search
+// on the merge path (the first i with A[i] > B[o - i - 1]) and then merges
+// KPT elements sequentially.  No warp votes: every step is a compare, a select
+// and a shared-memory load.  On return the sorted keys are in s_keys (position
+// j at spad(j)).
+template <int BLOCK, int KPT>
+__device__ __forceinline__ void block_merge_sort(uint32_t (&key)[KPT], uint32_t *s_keys) {
+    constexpr int CAP = BLOCK * KPT;
+    const int tid = threadIdx.x;
+    bitonic_regs<KPT>(key);
+#pragma unroll
+    for (int q = 0; q < KPT; ++q) s_keys[spad(KPT * tid + q)] = key[q];
+    __syncthreads();
+#pragma unroll 1
+    for (int L = KPT; L < CAP; L <<= 1) {
+        const int out0 = KPT * tid;
+        const int base = out0 & ~(2 * L - 1);
+        const int o = out0 - base;                 // output offset within the pair's merge
+        const int A0 = base, B0 = base + L;        // the pair's two sorted runs of L keys
+        int lo = o > L ? o - L : 0, hi = o < L ? o : L;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (s_keys[spad(A0 + mid)] <= s_keys[spad(B0 + o - mid - 1)]) lo = mid + 1;
+            else hi = mid;
+        }
+        int i = lo, j = o - lo;
+        uint32_t a = i < L ? s_keys[spad(A0 + i)] : 0u, b = j < L ? s_keys[spad(B0 + j)] : 0u;
+#pragma unroll
+        for (int q = 0; q < KPT; ++q) {
+            const bool ta = i < L && (j >= L || a <= b);
+            key[q] = ta ? a : b;
+            if (ta) {
+                ++i;
+                a = i < L ? s_keys[spad(A0 + i)] : 0u;
+            } else {
+                ++j;
+                b = j < L ? s_keys[spad(B0 + j)] : 0u;
+            }
+        }
+        __syncthreads();   // every thread has read its inputs
+#pragma unroll
+        for (int q = 0; q < KPT; ++q) s_keys[spad(out0 + q)] = key[q];
+        __syncthreads();
+    }
+}
+
 // Solve the sorted values held in s_keys (position j at spad(j); descending scores).
 //   m0      scores above the first value (band: the count at or above a_R)
 //   top     value above c_0 that P_top refers to (a_R, or +inf)
