@@ -1209,8 +1209,14 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
 // ================================================================= p pass --
 // p = F((r - b)/t), walking forward (the certification pass left the head of
 // the row in L2).  Also sum p (fp64 over fp32 float4 partials) for diagnostics.
+// Four p at once, one lane at a time (any subset of a warp may call it).
+__device__ __forceinline__ float4 p_vec_lane(const float4 v, const PForm &pf) {
+    return make_float4(pf(v.x), pf(v.y), pf(v.z), pf(v.w));
+}
+
 // Four p at once: the fp32 value for all, then -- only in warps where some lane
-// has a mid-range p (one vote) -- the fp64 value for those (PForm).
+// has a mid-range p (one vote) -- the fp64 value for those (PForm).  Every lane
+// of the warp must call it together (the chunks of the bulk pipeline).
 __device__ __forceinline__ float4 p_vec(const float4 v, const PForm &pf) {
     float4 o;
     const bool m0 = pf.fast(v.x, o.x), m1 = pf.fast(v.y, o.y), m2 = pf.fast(v.z, o.z), m3 = pf.fast(v.w, o.w);
@@ -1255,7 +1261,7 @@ p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restric
         });
     }
     for (int64_t i = done4 + gtid; i < n4; i += gstride) {
-        const float4 o = p_vec(r4[i], xf);
+        const float4 o = p_vec_lane(r4[i], xf);   // the tail: not every lane of a warp is here
         __stcs(p4 + i, o);
         ps += (double)((o.x + o.y) + (o.z + o.w));
     }

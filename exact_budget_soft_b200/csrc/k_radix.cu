@@ -687,9 +687,12 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                             const int li = warp * 32 * K + i * 32 + lane;
                             const bool v = li < cnt_tile;
                             const uint32_t d = v ? ((key[i] >> sh) & 0xffu) : 0x100u;
-                            // lanes holding the same digit (eight ballots measured slower here:
-                            // this kernel is bound by the same ALU pipe they use)
-                            const unsigned peers = __match_any_sync(FULL, d);
+                            // lanes holding the same digit: all of them when the warp's keys
+                            // agree on it (sorted or tied scores: one vote), else a match
+                            // (eight ballots measured slower here: this kernel is bound by
+                            // the ALU pipe they use)
+                            const bool uni = __all_sync(FULL, d == __shfl_sync(FULL, d, 0));
+                            const unsigned peers = uni ? FULL : __match_any_sync(FULL, d);
                             const int leader = __ffs(peers) - 1;
                             uint32_t bs = 0;
                             if (v && lane == leader) {

@@ -519,7 +519,7 @@ __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC],
             }
             __syncwarp();
         }
-        if (*reinterpret_cast<volatile int *>(&s_stop)) break;
+        if (__any_sync(FULL, *reinterpret_cast<volatile int *>(&s_stop) != 0)) break;   // warp-uniform
         const int s = (int)(i % ST);
         if (!__all_sync(FULL, mbar_wait(&full[s], (uint32_t)((i / ST) & 1), BULK_WAIT_CAP))) {
             if (lane == 0) s_stop = 1;
