@@ -387,224 +387,6 @@ __global__ void __launch_bounds__(SEL_BLOCK) select_kernel(BracketParams Pg) {
     }
 }
 
-// ========================================================= sample + select --
-// The sample and the bracket's order statistics in one launch (the one-GPU
-// path): every CTA draws its share of the sample as sample_kernel does; the CTA
-// that finishes last (one ticket per row) runs the whole radix select on it --
-// round 1 from the histograms the sampler built, the keys under each target's
-// 16-bit prefix gathered into shared memory, rounds 2 and 3 there -- so no
-// second launch and no global candidate buffer sit on the critical path.
-constexpr int SS_BLOCK = 1024;
-
-// The bracket ends from the selected keys (and, in the widening round, the new
-// bracket on the missed side); thread 0.
-__device__ __forceinline__ void select_finish(const BracketParams &P, const bool valid[2], uint32_t prefR,
-                                              uint32_t prefL) {
-    Ctl *ctl = P.ctl;
-    const float yR = desc_key_to_float(prefR);
-    const float yL = desc_key_to_float(prefL);
-    const float aR = valid[0] ? nextafterf(yR, CUDART_INF_F) : CUDART_INF_F;
-    const float aL = valid[1] ? yL : -CUDART_INF_F;
-    if (P.round2) {   // the missed side becomes the bracket; the stream starts afresh
-        if (ctl->widen_dir > 0) {   // b >= old a_R
-            ctl->a_L = ctl->a_R;
-            ctl->jL = ctl->jR;
-            ctl->a_R = aR;
-            ctl->jR = P.jR;
-        } else {                    // b < old a_L
-            ctl->a_R = ctl->a_L;
-            ctl->jR = ctl->jL;
-            ctl->a_L = aL;
-            ctl->jL = P.jL;
-        }
-        ctl->c_band = 0ull;
-        ctl->band_kmax = 0u;
-        ctl->band_kinv = 0u;
-        atomicAnd(&ctl->status, ~(ST_NO_ROOT | ST_BAND_OVERFLOW));   // the first band solve's misses
-        ctl->widened = 1;
-    } else {
-        ctl->a_R = aR;
-        ctl->a_L = aL;
-        ctl->jR = P.jR;
-        ctl->jL = P.jL;
-    }
-    ctl->s = P.s;
-    ctl->path = 2;
-    ctl->verdict = -1;
-}
-
-__global__ void __launch_bounds__(SS_BLOCK) sample_select_kernel(BracketParams Pg) {
-    const BracketParams P = at_row(Pg, blockIdx.y);
-    extern __shared__ __align__(16) uint32_t s_cand[];   // [2][SEL_CAND], the last CTA's candidates
-    __shared__ uint32_t s_h0[256];
-    __shared__ uint32_t s_w[SS_BLOCK / 32];
-    __shared__ uint32_t h8[2][256];
-    __shared__ uint32_t s_pref[2], s_rank[2], s_bin0[2], s_cnt[2];
-    __shared__ bool s_last;
-    const int tid = threadIdx.x, lane = tid & 31;
-    if (tid < 256) s_h0[tid] = 0u;
-    pdl_enter();
-    if (P.round2 && !widen_starts(P)) return;   // the same sample again, for the widened ranks
-    __syncthreads();
-    Ctl *ctl = P.ctl;
-    // ---- the sample (as sample_kernel)
-    const int64_t j = (int64_t)blockIdx.x * SS_BLOCK + tid;
-    if (j < P.s) {
-        uint64_t x0 = (uint64_t)j, x1 = (uint64_t)P.row, x2 = 0, x3 = 0;
-        philox4x64_10(x0, x1, x2, x3, P.seed, SAMPLE_TAG);
-        const int64_t I = (int64_t)__umul64hi(x0, (uint64_t)P.n_total) - P.shard_off;
-        if (in_bounds(I >= 0 && I < P.n, &ctl->status)) {
-            const double U = (double)((x1 >> 11) + 1ull) * 0x1p-53;
-            const double E = -sample_ln(U);
-            const double L = (x1 & 1ull) ? E : -E;
-            const double y = __dadd_rn((double)__ldg(P.r + I), __dmul_rn(P.t, L));
-            const uint32_t key = desc_key(__double2float_rd(y));
-            P.keys[j] = key;
-            const uint32_t bin = key >> 16;
-            const unsigned peers = __match_any_sync(__activemask(), bin);
-            if (lane == __ffs(peers) - 1) {
-                atomicAdd(P.hist1 + bin, (uint32_t)__popc(peers));
-                atomicAdd(&s_h0[bin >> 8], (uint32_t)__popc(peers));
-            }
-        }
-    }
-    __syncthreads();
-    if (tid < 256 && s_h0[tid]) atomicAdd(P.hist1 + SEL_BINS + tid, s_h0[tid]);
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&ctl->ticket[5], 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // ---- the last CTA: the radix select over the whole sample
-    const int64_t s = P.s;
-    const bool valid[2] = {P.jR >= 1, P.jL <= P.s};
-    const uint32_t want0[2] = {(uint32_t)(valid[0] ? P.jR : 1), (uint32_t)(valid[1] ? P.jL : 1)};
-    if (tid < 2) { s_bin0[tid] = 0u; s_rank[tid] = 1u; s_pref[tid] = 0u; s_cnt[tid] = 0u; }
-    {   // round 1a: the top byte of each target (thread t < 256 owns bin t)
-        const uint32_t c = tid < 256 ? __ldcg(P.hist1 + SEL_BINS + tid) : 0u;
-        const uint32_t incl = block_incl_scan_u32(c, s_w);
-        if (tid < 256) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-                if (incl - c < want0[q] && want0[q] <= incl) {
-                    s_bin0[q] = (uint32_t)tid;
-                    s_rank[q] = want0[q] - (incl - c);
-                }
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {   // round 1b: the second byte, from the 256 top-16 bins under the first
-        const uint32_t b0 = s_bin0[q], want = s_rank[q];
-        const uint32_t c = tid < 256 ? __ldcg(P.hist1 + b0 * 256 + tid) : 0u;
-        const uint32_t incl = block_incl_scan_u32(c, s_w);
-        if (tid < 256 && incl - c < want && want <= incl) {
-            s_pref[q] = ((b0 << 8) | (uint32_t)tid) << 16;
-            s_rank[q] = want - (incl - c);
-        }
-        __syncthreads();
-    }
-    const uint32_t pf[2] = {s_pref[0], s_pref[1]};
-    {   // the keys under either prefix, into shared memory (one vote for four keys)
-        auto take = [&](uint32_t key, bool in) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const bool m = in && valid[q] && (key & 0xffff0000u) == pf[q];
-                const unsigned bal = __ballot_sync(FULL, m);
-                if (!bal) continue;
-                uint32_t base = 0;
-                if (lane == __ffs(bal) - 1) base = atomicAdd(&s_cnt[q], (uint32_t)__popc(bal));
-                base = __shfl_sync(FULL, base, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
-                if (m && base < SEL_CAND) s_cand[q * SEL_CAND + base] = key;
-            }
-        };
-        const uint4 *k4 = reinterpret_cast<const uint4 *>(P.keys);
-        const int64_t s4 = s / 4;
-        constexpr int INFL = 4;   // vectors per thread in flight
-        for (int64_t i0 = 0; i0 < s4; i0 += INFL * SS_BLOCK) {
-            uint4 kv[INFL];
-#pragma unroll
-            for (int u = 0; u < INFL; ++u) {
-                const int64_t i = i0 + u * SS_BLOCK + tid;
-                kv[u] = i < s4 ? __ldcg(k4 + i) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int u = 0; u < INFL; ++u) {
-                const bool in = i0 + u * SS_BLOCK + tid < s4;
-                const uint32_t kk[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
-                bool hit = false;
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    hit |= in && (((kk[e] & 0xffff0000u) == pf[0] && valid[0]) ||
-                                  ((kk[e] & 0xffff0000u) == pf[1] && valid[1]));
-                if (!__any_sync(FULL, hit)) continue;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) take(kk[e], in);
-            }
-        }
-        for (int64_t i0 = 4 * s4; i0 < s; i0 += SS_BLOCK) {
-            const int64_t i = i0 + tid;
-            take(i < s ? __ldcg(P.keys + i) : 0u, i < s);
-        }
-    }
-    __syncthreads();
-    // ---- rounds 2, 3 (bits 15..8, 7..0) over the candidates, or over every key
-    const uint32_t cnt[2] = {s_cnt[0], s_cnt[1]};
-    const bool fast[2] = {cnt[0] <= SEL_CAND, cnt[1] <= SEL_CAND};
-    uint32_t mask = 0xffff0000u;
-#pragma unroll 1
-    for (int sh = 8; sh >= 0; sh -= 8) {
-        for (int i = tid; i < 2 * 256; i += SS_BLOCK) (&h8[0][0])[i] = 0u;
-        __syncthreads();
-        const uint32_t pq[2] = {s_pref[0], s_pref[1]};
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            if (!valid[q]) continue;
-            const int64_t c = fast[q] ? (int64_t)cnt[q] : s;
-            for (int64_t i = tid; i < c; i += SS_BLOCK) {
-                const uint32_t key = fast[q] ? s_cand[q * SEL_CAND + i] : __ldcg(P.keys + i);
-                if ((key & mask) == pq[q]) atomicAdd(&h8[q][(key >> sh) & 0xffu], 1u);
-            }
-        }
-        __syncthreads();
-        if (tid < 64) {   // warp q scans target q's 256 bins (8 per lane)
-            const int q = tid >> 5;
-            if (valid[q]) {
-                uint32_t v[8], run = 0;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) { v[u] = h8[q][lane * 8 + u]; run += v[u]; }
-                uint32_t incl = run;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t pp = __shfl_up_sync(FULL, incl, o);
-                    if (lane >= o) incl += pp;
-                }
-                const uint32_t want = s_rank[q];
-                uint32_t cum = incl - run;
-                if (cum < want && want <= incl) {
-                    for (int u = 0; u < 8; ++u) {
-                        if (cum + v[u] >= want) {
-                            s_pref[q] |= (uint32_t)(lane * 8 + u) << sh;
-                            s_rank[q] = want - cum;
-                            break;
-                        }
-                        cum += v[u];
-                    }
-                }
-            }
-        }
-        mask |= 0xffu << sh;
-        __syncthreads();
-    }
-    if (tid < 256) P.hist1[SEL_BINS + tid] = 0u;   // the top-byte histogram; the streaming pass clears the rest
-    if (tid == 0) {
-        if ((valid[0] && !fast[0]) || (valid[1] && !fast[1])) ctl->flags |= FLAG_SELECT_ALL_KEYS;
-        select_finish(P, valid, s_pref[0], s_pref[1]);
-        ctl->ticket[5] = 0u;
-    }
-}
-
 // ===================================================== out-of-band passes --
 // The streaming pass (technical summary section 2.2, step 2) and the
 // certification pass (step 4, abstract) walk every score once and, for each
@@ -1553,13 +1335,6 @@ cudaError_t launch_select(const BracketParams &P, cudaStream_t st) {
     return launch_k(select_kernel, dim3((unsigned)per_row, (unsigned)P.rows), SEL_BLOCK, 0, st, P);
 }
 int select_cand_capacity() { return SEL_CAND; }
-cudaError_t launch_sample_select(const BracketParams &P, cudaStream_t st) {
-    const size_t smem = 2 * SEL_CAND * sizeof(uint32_t);
-    const cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(sample_select_kernel), smem);
-    if (e != cudaSuccess) return e;
-    return launch_k(sample_select_kernel, dim3((unsigned)((P.s + SS_BLOCK - 1) / SS_BLOCK), (unsigned)P.rows),
-                    SS_BLOCK, smem, st, P);
-}
 template <typename K>
 static cudaError_t set_smem(K kern, size_t bytes) {
     return set_max_dynamic_smem(reinterpret_cast<const void *>(kern), bytes);

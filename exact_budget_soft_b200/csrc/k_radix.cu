@@ -27,7 +27,6 @@ constexpr int RB = 512;             // radix pass: threads
 constexpr int RK_BIG = 16, RK_SMALL = 4;
 constexpr int64_t SMALL_SORT = int64_t(1) << 20;
 constexpr int RNW = RB / 32;
-constexpr int HB = 256;             // histogram kernel threads
 
 
 
@@ -36,6 +35,13 @@ constexpr int HB = 256;             // histogram kernel threads
 // the last clean-up.  They differ while the histograms need clearing.
 __device__ __forceinline__ unsigned long long *A_hist_dirty(const SortArgs &A) { return A.hist + 4 * 256; }
 __device__ __forceinline__ unsigned long long *A_hist_cleaned(const SortArgs &A) { return A.hist + 4 * 256 + 1; }
+// Four more words: for each sign class of the keys (negative scores, then the
+// rest), the OR of the keys and the OR of their complements -- the bits that
+// vary within the class are the AND of the two.  A digit whose bits vary within
+// neither class is decided by the sign, so its pass changes no order among keys
+// that tie on the higher digits: it is skipped like a constant digit.  (Scores
+// quantised to a few mantissa bits -- tied levels -- skip two of four passes.)
+__device__ __forceinline__ unsigned long long *A_sign_bits(const SortArgs &A) { return A.hist + 4 * 256 + 2; }
 __device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long *p) {
     return *reinterpret_cast<const volatile unsigned long long *>(p);
 }
@@ -479,8 +485,10 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
     // before any count is added, so all take the same branch): clear them first.
     const unsigned long long gave_up = ld_volatile_u64(A_hist_dirty(Ag));
     if (gave_up != ld_volatile_u64(A_hist_cleaned(Ag))) {
-        if (c == 0)
+        if (c == 0) {
             for (int i = tid; i < 4 * 256; i += RB) Ag.hist[i] = 0ull;
+            if (tid < 4) A_sign_bits(Ag)[tid] = 0ull;
+        }
         if (!grid_sync(&Ag.ctl->gbar_count, &Ag.ctl->gbar_gen, Ag.spin_cap, &Ag.ctl->status)) {
             if (tid == 0) atomicAdd(A_hist_dirty(Ag), 1ull);
             return;
@@ -538,11 +546,15 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
             {
                 uint32_t cur[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
                 uint32_t cnt[4] = {0, 0, 0, 0};
+                uint32_t sor[2] = {0u, 0u}, snot[2] = {0u, 0u};   // per sign class: OR of keys, of ~keys
                 const bool walked = walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
                     const int l0 = warp * 32 * K + lane;
 #pragma unroll
                     for (int i = 0; i < K; ++i) {
                         if (l0 + i * 32 >= cnt_tile) break;
+                        const int sg = key[i] >> 31;
+                        sor[sg] |= key[i];
+                        snot[sg] |= ~key[i];
 #pragma unroll
                         for (int d = 0; d < 4; ++d) {
                             const uint32_t bin = (key[i] >> (8 * d)) & 0xffu;
@@ -563,6 +575,16 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
 #pragma unroll
                 for (int d = 0; d < 4; ++d)
                     if (cnt[d]) atomicAdd(&s_h4[d * 256 + cur[d]], cnt[d]);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {   // the CTA's varying bits per sign class, then the grid's
+                    sor[q] = __reduce_or_sync(FULL, sor[q]);
+                    snot[q] = __reduce_or_sync(FULL, snot[q]);
+                    if (lane == 0 && (sor[q] | snot[q])) {
+                        atomicOr(reinterpret_cast<unsigned long long *>(A_sign_bits(A) + 2 * q), (unsigned long long)sor[q]);
+                        atomicOr(reinterpret_cast<unsigned long long *>(A_sign_bits(A) + 2 * q + 1),
+                                 (unsigned long long)snot[q]);
+                    }
+                }
                 __syncthreads();
                 for (int i = tid; i < 4 * 256; i += RB) {
                     const uint32_t v = s_h4[i];
@@ -572,7 +594,14 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
             }
             if (!bar()) return;
             // digit bases and skip flags, the same in every CTA (thread d owns bin d)
-            if (tid == 0) s_skip = 0;
+            if (tid == 0) {
+                const unsigned long long *sb = A_sign_bits(A);
+                const uint32_t vary = (uint32_t)(__ldcg(sb) & __ldcg(sb + 1)) | (uint32_t)(__ldcg(sb + 2) & __ldcg(sb + 3));
+                int sk = 0;
+                for (int d4 = 0; d4 < 3; ++d4)   // the top digit holds the sign: skipped only when constant (below)
+                    if (((vary >> (8 * d4)) & 0xffu) == 0u) sk |= 1 << d4;
+                s_skip = sk;
+            }
             __syncthreads();
             for (int d4 = 0; d4 < 4; ++d4) {
                 uint32_t v = 0;
@@ -729,6 +758,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
             if (!bar()) return;   // the maps are complete, and every CTA has read the global histograms
             if (c == 0) {
                 for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort
+                if (tid < 4) A_sign_bits(A)[tid] = 0ull;
                 if (skip != 15) locate_finish<K>(A, sorted, n, z, rec, crec, S.buf, s_hist, s_tab);
             }
             if (!bar()) return;   // the next row reuses the global scratch

@@ -63,6 +63,18 @@ cudaError_t set_max_dynamic_smem(const void *kern, size_t bytes) {
     return e;
 }
 
+std::map<int, bool> g_coop_pdl_refused;
+bool coop_pdl_refused() {
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    return g_coop_pdl_refused.count(dev) != 0;
+}
+void coop_pdl_refuse() {
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    g_coop_pdl_refused[dev] = true;
+}
+
 cudaError_t resident_ctas(const void *kern, int threads, size_t smem, int *out) {
     const int sms = device_sm_count();
     const auto key = std::make_tuple(current_device(), kern, threads, smem);
@@ -198,13 +210,13 @@ struct Workspace {
             {keys0, keys0_n * 4}, {hist, hist_n * 8}, {chunkcnt, chunkcnt_n * 4},
             {tilebuf, tilebuf_n * 8}};
         if (cudaStreamSynchronize(st) != cudaSuccess) return LAPSUM_ERR_CUDA;
-        unsigned char g[GUARD_BYTES ? GUARD_BYTES : 1];
+        constexpr size_t NG = GUARD_BYTES ? GUARD_BYTES : 1;
+        unsigned char g[NG];
         for (const auto &b : bufs) {
             if (!b.first) continue;
-            if (cudaMemcpy(g, static_cast<const char *>(b.first) + b.second, GUARD_BYTES, cudaMemcpyDeviceToHost) !=
-                cudaSuccess)
+            if (cudaMemcpy(g, static_cast<const char *>(b.first) + b.second, NG, cudaMemcpyDeviceToHost) != cudaSuccess)
                 return LAPSUM_ERR_CUDA;
-            for (size_t i = 0; i < GUARD_BYTES; ++i)
+            for (size_t i = 0; i < NG; ++i)
                 if (g[i] != GUARD_FILL) return LAPSUM_ERR_BOUNDS;
         }
         return LAPSUM_OK;
@@ -238,7 +250,7 @@ cudaError_t ws_base(Workspace *w, int64_t rows) {
 // workspace holds one key buffer of the row, not two.
 cudaError_t ws_sort(Workspace *w, int64_t cap) {
     cudaError_t e = grow(w->keys0, w->keys0_n, (size_t)cap);
-    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256 + 2);   // + the give-up and clean-up counts
+    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256 + 6);   // + give-up/clean-up counts, per-sign varying bits
     if (e == cudaSuccess) e = grow(w->chunkcnt, w->chunkcnt_n, (size_t)4 * 256 * sort_grid_max());
     if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, (size_t)sort_record_doubles(cap));
     return e;
@@ -545,7 +557,8 @@ static int forward_impl(const float *scores, int64_t rows, int64_t n, double k, 
     // one bracketing round: sample, select, stream, band solve, certification
     auto bracket_round = [&](const BracketParams &Q) -> int {
         const bool r2 = Q.round2 != 0;   // profiling names are literals (the profiler keeps the pointer)
-        { Launch L(r2 ? "widen_sample_select" : "sample_select", st); LAPSUM_TRY(launch_sample_select(Q, st)); }
+        { Launch L(r2 ? "widen_sample" : "sample", st); LAPSUM_TRY(launch_sample(Q, st)); }
+        { Launch L(r2 ? "widen_select" : "select", st); LAPSUM_TRY(launch_select(Q, st)); }
         { Launch L(r2 ? "widen_stream_pass" : "stream_pass", st); LAPSUM_TRY(launch_stream_pass(Q, st)); }
         { Launch L(r2 ? "widen_band_select" : "band_select", st); LAPSUM_TRY(launch_band_select(w->band, rows, k, t, w->ctl, Q.band_cap, Q.round2, st)); }
         if (!Q.fused_cert) { Launch L(r2 ? "widen_certify" : "certify", st); LAPSUM_TRY(launch_certify(Q, st)); }

@@ -465,8 +465,10 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 // released it, one chunk behind, so a warp slowed by rare scores holds the
 // others back only when it falls a whole ring behind.  If a wait gives up (any
 // of them), the CTA stops at the next chunk, sets ST_TIMEOUT, and waits (bounded
-// again) for the copies it has in flight before returning; the caller's result
-// is then invalid and the error reaches the host through the status word.
+// again) for the copies it has in flight before returning (warps still waiting
+// on a copy that is no longer issued leave when their own bounded wait gives up);
+// the caller's result is then invalid and the error reaches the host through the
+// status word.
 template <int NSRC, typename Body>
 __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC], int64_t n4, bool reverse,
                                                unsigned char *smem, int32_t *status, Body &&body) {
@@ -519,7 +521,6 @@ __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC],
             }
             __syncwarp();
         }
-        if (__any_sync(FULL, *reinterpret_cast<volatile int *>(&s_stop) != 0)) break;   // warp-uniform
         const int s = (int)(i % ST);
         if (!__all_sync(FULL, mbar_wait(&full[s], (uint32_t)((i / ST) & 1), BULK_WAIT_CAP))) {
             if (lane == 0) s_stop = 1;

@@ -26,7 +26,13 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
 }
 
 // A cooperative launch (every CTA resident at once, so CTAs may wait on one
-// another at grid barriers); ordinary stream order, no early launch.
+// another at grid barriers).  With programmatic stream serialization as well
+// when the runtime takes the pair (the kernel's CTAs are then scheduled while
+// its predecessor drains, and wait for it with griddepcontrol.wait before any
+// grid barrier); if it refuses the pair, a plain cooperative launch in stream
+// order (the refusal is remembered per device).
+bool coop_pdl_refused();
+void coop_pdl_refuse();
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                                Args &&...args) {
@@ -35,12 +41,22 @@ inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, si
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+    cfg.numAttrs = coop_pdl_refused() ? 1 : 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+    if (e != cudaSuccess && cfg.numAttrs == 2 &&
+        (e == cudaErrorInvalidValue || e == cudaErrorNotSupported || e == cudaErrorInvalidConfiguration)) {
+        (void)cudaGetLastError();   // the launch did not happen: try without the pair
+        coop_pdl_refuse();
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+    }
+    return e;
 }
 
 // Per-device launch set-up (lapsum_api.cu), cached per (device, kernel) under a
@@ -65,8 +81,6 @@ int stream_grid();
 int64_t partial_stride(int64_t rows);   // doubles of per-block partials per row
 cudaError_t launch_sample(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_select(const BracketParams &P, cudaStream_t st);
-// the sample and its select in one launch (the last CTA of each row selects)
-cudaError_t launch_sample_select(const BracketParams &P, cudaStream_t st);
 int select_cand_capacity();
 cudaError_t launch_stream_pass(const BracketParams &P, cudaStream_t st);
 cudaError_t launch_certify(const BracketParams &P, cudaStream_t st);
@@ -92,7 +106,8 @@ struct SortArgs {
     int64_t n_host;            // element count
     int64_t cap;               // upper bound of the element count (grid sizing)
     uint32_t *keys[2];         // ping-pong key buffers [cap]: the workspace's, and the caller's p output
-    unsigned long long *hist;  // [4][256], then two words: sorts that gave up, and that count at the last clean-up
+    unsigned long long *hist;  // [4][256], then two words: sorts that gave up, and that count at the last clean-up,
+                               // then four: per sign class, the OR of the keys and of their complements
     uint32_t *chunkcnt;        // [4][256][grid]: digit counts of each CTA's chunk of tiles
     double *tilebuf;           // locate per-tile data
     Ctl *ctl;

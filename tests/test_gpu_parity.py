@@ -105,8 +105,11 @@ def test_all_equal_and_ties(L, orc):
 
 # ----------------------------------------------- device-wide full sort --
 @pytest.mark.parametrize("n,dist", [(32769, "normal"), (100_000, "laplace"), (300_001, "normal"),
-                                    (500_000, "levels256_desc"), (1_100_003, "normal")])
+                                    (500_000, "levels256_desc"), (1_100_003, "normal"),
+                                    (300_007, "levels256_shuffled"), (2_000_000, "levels256_shuffled")])
 def test_device_sort_path(L, orc, n, dist):
+    # the shuffled levels (few mantissa bits, both signs) make the sort skip the
+    # two low digits (decided by the sign) and still reorder the row
     r, g = W.small_case(dist, 1, n, seed=7)
     k, t = n / 100.0, 0.05
     p, b, st, grad = run(L, r, k, t, opts=L.options(force_path=L.PATH_FULLSORT), g_np=g)
