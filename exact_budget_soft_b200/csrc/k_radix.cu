@@ -166,9 +166,28 @@ constexpr size_t stage_bytes() { return 2 * TILE_K(K) * 4 + 2 * sizeof(uint64_t)
 // Adds this warp's digit counts of the tile to my_hist (the warp's 256 counters).
 // Counts need no order: a warp whose keys all share the digit (sorted or tied
 // scores) adds them at once, any other warp takes one shared atomic per key.
-template <int K>
+// WHOLE: first test the warp's keys together (one vote for all K of them; the
+// count walks, where no ranking state competes for registers).
+template <int K, bool WHOLE>
 __device__ __forceinline__ void warp_count(const uint32_t (&key)[K], int cnt_tile, int sh, uint32_t *my_hist) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (WHOLE) {   // every key of the warp on the digit of its first key (lane 0's key 0): one add
+        const uint32_t d0 = __shfl_sync(FULL, (key[0] >> sh) & 0xffu, 0);
+        bool same = true;
+        uint32_t nv = 0;
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            const bool v = warp * 32 * K + i * 32 + lane < cnt_tile;
+            same &= !v || ((key[i] >> sh) & 0xffu) == d0;
+            nv += v;
+        }
+        if (__all_sync(FULL, same)) {
+            nv = __reduce_add_sync(FULL, nv);   // 0: the warp lies past the end of the tile
+            if (lane == 0 && nv) my_hist[d0] += nv;
+            __syncwarp();
+            return;
+        }
+    }
 #pragma unroll
     for (int i = 0; i < K; ++i) {
         const int li = warp * 32 * K + i * 32 + lane;
@@ -248,77 +267,154 @@ __device__ __forceinline__ Seeds locate_seeds(const SortArgs &) {
     return Seeds{0.0, CUDART_INF, 0.0, -CUDART_INF, 0.0};   // a whole row: nothing above or below
 }
 
-// Step 1 for one CTA: its tiles' records and its chunk record.  s_t: room for a
-// tile plus two halo values in the padded layout; sc: scan scratch.
+// Step 1 for one CTA: its tiles' records and its chunk record.  The tiles are
+// staged in shared memory one ahead (bulk copies into the sort's two tile
+// buffers; plain loads for a ragged or unaligned tile), and each thread maps
+// its K consecutive values.  A tile's suffix map needs the link out of its last
+// value, which the next tile supplies (its first value's link in): the map is
+// kept up to that link and completed one tile later (the chunk's last tile
+// from one load after the walk), so no tile waits on a value beyond it.
+// Returns false when a copy wait gave up (ST_TIMEOUT set, copies in flight
+// awaited); the caller must return.
 template <int K>
-__device__ void locate_tiles(const SortArgs &A, const uint32_t *sorted, int64_t n, int64_t t0, int64_t t1,
-                             const Seeds &z, TileRec *rec, ChunkRec *crec, uint32_t *s_t, Aff *sc,
+__device__ bool locate_tiles(const SortArgs &A, TileStage<K> &S, uint32_t &ph, const uint32_t *sorted, int64_t n,
+                             int64_t t0, int64_t t1, const Seeds &z, TileRec *rec, ChunkRec *crec, Aff *sc,
                              const double *tab) {
     constexpr int TILE = TILE_K(K);
-    const int tid = threadIdx.x;
+    constexpr int NW = RB / 32;
+    static_assert(K % 4 == 0, "a thread reads its values as uint4");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const double s2d = (1.0 / A.t) * LOG2E;
-    const uint32_t key_top = desc_key((float)z.top), key_bot = desc_key((float)z.bot);
-    __shared__ Aff s_map[2];
-    __shared__ double s_dout;
-    Aff Pc = aff_id(), Qc = aff_id();
-    double dc = 0.0;
-    for (int64_t tile = t0; tile < t1; ++tile) {
+    __shared__ float s_last;              // the last value of the tile just mapped
+    __shared__ float s_wend[2][NW];       // each warp's first and last value
+    // link between neighbours hi >= lo: e^{-(hi - lo)/t}; 0 against an infinite end
+    auto link = [&](double hi, double lo) -> double {
+        return (hi == CUDART_INF || lo == -CUDART_INF) ? 0.0 : link_exp((hi - lo) * s2d, tab);
+    };
+    Aff Pc = aff_id(), Qc = aff_id(), Qprev = aff_id();   // thread 0: chunk maps, last tile's partial Q map
+    double vprev = 0.0;                                    // thread 0: the value before the tile
+    if (tid == 0) vprev = t0 == 0 ? z.top : (double)desc_key_to_float(__ldcg(sorted + t0 * TILE - 1));
+    stage_source(S, A, sorted);
+    if (tid == 0 && t0 < t1) stage_issue(S, 0, t0);
+    int slot = 0;
+    for (int64_t tile = t0; tile < t1; ++tile, slot ^= 1) {
+        if (tid == 0 && tile + 1 < t1) stage_issue(S, slot ^ 1, tile + 1);
         const int64_t base = tile * TILE;
         const int cnt = (int)min((int64_t)TILE, n - base);
-        // s_t[spad(i + 1)] = sorted position base + i for i = -1 .. cnt
+        const int l0 = tid * K;
+        const int nk = max(0, min(K, cnt - l0));   // this thread's values
+        float c[K];   // this thread's values (fp32 scores; links are formed in fp64)
+        bool ok = true;
+        if (stage_full(S, tile)) {
+            ok = mbar_wait(&S.bar[slot], (ph >> slot) & 1u, BULK_WAIT_CAP);
+            ph ^= 1u << slot;
+            const uint4 *q = reinterpret_cast<const uint4 *>(S.buf + slot * TILE + l0);
 #pragma unroll
-        for (int u = 0; u < K; ++u) {
-            const int i = u * RB + tid;
-            if (i < cnt) s_t[spad(i + 1)] = __ldcg(sorted + base + i);
-        }
-        if (tid == 0) {
-            s_t[spad(0)] = base == 0 ? key_top : __ldcg(sorted + base - 1);
-            s_t[spad(cnt + 1)] = base + cnt >= n ? key_bot : __ldcg(sorted + base + cnt);
-        }
-        __syncthreads();
-        auto sval = [&](int i) -> double { return (double)desc_key_to_float(s_t[spad(i + 1)]); };
-        const int l0 = tid * K, l1 = min(l0 + K, cnt) - 1;
-        Aff mp = aff_id(), mq = aff_id();
-        double d_last = 0.0;
-        if (l0 < cnt) {
-            double cprev = sval(l0 - 1), c = sval(l0);
-            double dprev = (cprev == CUDART_INF || c == -CUDART_INF) ? 0.0 : link_exp((cprev - c) * s2d, tab);
-            for (int j = l0; j <= l1; ++j) {
-                mp = {mp.a * dprev, fma(mp.s, dprev, 1.0)};
-                const double cn = sval(j + 1);
-                const double d = (c == CUDART_INF || cn == -CUDART_INF) ? 0.0 : link_exp((c - cn) * s2d, tab);
-                mq = {mq.a * d, mq.s + mq.a};
-                dprev = d;
-                c = cn;
+            for (int v = 0; v < K / 4; ++v) {
+                const uint4 w = q[v];
+                c[4 * v + 0] = desc_key_to_float(w.x);
+                c[4 * v + 1] = desc_key_to_float(w.y);
+                c[4 * v + 2] = desc_key_to_float(w.z);
+                c[4 * v + 3] = desc_key_to_float(w.w);
             }
-            d_last = dprev;
+        } else {
+#pragma unroll
+            for (int u = 0; u < K; ++u) c[u] = u < nk ? desc_key_to_float(__ldcg(sorted + base + l0 + u)) : 0.0f;
         }
-        Aff pe, qe;
-        block_scan_excl_both<RB>(mp, mq, pe, qe, sc);
-        const int owner = (cnt - 1) / K;
-        if (tid == owner) {
-            const Aff P = aff_then(pe, mp);
+        float clast = c[0];
+#pragma unroll
+        for (int u = 1; u < K; ++u) clast = u < nk ? c[u] : clast;
+        if (lane == 0) s_wend[0][warp] = c[0];
+        if (lane == 31) s_wend[1][warp] = clast;
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) {
+                atomicOr(&A.ctl->status, ST_TIMEOUT);
+                if (stage_full(S, tile)) mbar_wait(&S.bar[slot], ((ph >> slot) & 1u) ^ 1u, BULK_WAIT_CAP);
+                if (tile + 1 < t1 && stage_full(S, tile + 1))
+                    mbar_wait(&S.bar[slot ^ 1], (ph >> (slot ^ 1)) & 1u, BULK_WAIT_CAP);
+            }
+            __syncthreads();
+            return false;
+        }
+        // the values either side of this thread's run
+        const float up = __shfl_up_sync(FULL, clast, 1), dn = __shfl_down_sync(FULL, c[0], 1);
+        const double before = tid == 0 ? vprev : (double)(lane > 0 ? up : s_wend[1][warp - 1]);
+        const float after = lane < 31 ? dn : (warp < NW - 1 ? s_wend[0][warp + 1] : 0.0f);
+        // P: x -> 1 + d x over the run in order, d the link into each value; Q:
+        // x -> 1 + d x right to left, d the link out of each value, the tile's last
+        // value taking d = 1 (its link out is applied later)
+        const double din = link(before, (double)c[0]);   // into the run's first value
+        Aff mp = aff_id(), mq = aff_id();
+        bool flat = nk > 0;   // every value of the run equal (tied scores): every inner link is 1
+                              // (a non-finite row is reported, not solved)
+#pragma unroll
+        for (int u = 1; u < K; ++u) flat &= u >= nk || c[u] == c[0];
+        if (flat) {   // P_end = nk + din P_before, Q_first = nk + dout Q_after
+            const double dout = l0 + nk < cnt ? link((double)clast, (double)after) : 1.0;
+            mp = {din, (double)nk};
+            mq = {dout, (double)nk};
+        } else {
+            double dcur = din;
+#pragma unroll
+            for (int u = 0; u < K; ++u) {
+                if (u < nk) {
+                    mp = {mp.a * dcur, fma(mp.s, dcur, 1.0)};
+                    const double dnext = u + 1 < nk ? link((double)c[u], (double)c[(u + 1) % K])
+                                                    : (l0 + nk < cnt ? link((double)c[u], (double)after) : 1.0);
+                    mq = {mq.a * dnext, mq.s + mq.a};
+                    dcur = dnext;
+                }
+            }
+        }
+        // the tile's two maps: a tree over the warp's lanes (P in thread order, Q the
+        // other way round), then thread 0 over the warps
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const Aff pp = shfl_down_aff(mp, o), pq = shfl_down_aff(mq, o);
+            if (lane + o < 32) {   // lane l (a multiple of 2o) takes lanes l + o .. l + 2o - 1
+                mp = aff_then(mp, pp);
+                mq = aff_then(pq, mq);
+            }
+        }
+        if (lane == 0) {
+            sc[warp] = mp;
+            sc[NW + warp] = mq;
+        }
+        if (tid == (cnt - 1) / K) s_last = clast;   // the tile's last value is this thread's
+        __syncthreads();
+        if (tid == 0) {
+            Aff P = sc[0], Q = sc[NW];
+            for (int w = 1; w < NW; ++w) {
+                P = aff_then(P, sc[w]);
+                Q = aff_then(sc[NW + w], Q);
+            }
             rec[tile].pa = P.a;
             rec[tile].ps = P.s;
-            rec[tile].d_out = d_last;
-            s_map[0] = P;
-            s_dout = d_last;
+            if (tile > t0) {   // the link into this tile completes the previous tile's Q map
+                const Aff Qf = {Qprev.a * din, Qprev.s};
+                rec[tile - 1].qa = Qf.a;
+                rec[tile - 1].qs = Qf.s;
+                rec[tile - 1].d_out = din;
+                Qc = aff_then(Qf, Qc);
+            }
+            Pc = aff_then(Pc, P);
+            Qprev = Q;
+            vprev = s_last;
         }
-        if (tid == 0) {
-            const Aff Q = aff_then(qe, mq);
-            rec[tile].qa = Q.a;
-            rec[tile].qs = Q.s;
-            s_map[1] = Q;
-        }
-        __syncthreads();
-        if (tid == 0) {   // the chunk's maps: P of the tiles in order, Q the other way round
-            Pc = aff_then(Pc, s_map[0]);
-            Qc = aff_then(s_map[1], Qc);
-            dc = s_dout;
-        }
-        __syncthreads();   // s_t and s_map are reused by the next tile
+        __syncthreads();   // the stage buffer and the scratch are reused by the next tile
     }
     if (tid == 0) {
+        double dc = 0.0;
+        if (t1 > t0) {   // the chunk's last tile: its link out, to the value after the chunk
+            const int64_t e = min(t1 * TILE, n);
+            const double vnext = e >= n ? z.bot : (double)desc_key_to_float(__ldcg(sorted + e));
+            dc = link(vprev, vnext);
+            const Aff Qf = {Qprev.a * dc, Qprev.s};
+            rec[t1 - 1].qa = Qf.a;
+            rec[t1 - 1].qs = Qf.s;
+            rec[t1 - 1].d_out = dc;
+            Qc = aff_then(Qf, Qc);
+        }
         ChunkRec r;
         r.pa = Pc.a;
         r.ps = Pc.s;
@@ -329,6 +425,7 @@ __device__ void locate_tiles(const SortArgs &A, const uint32_t *sorted, int64_t 
         r.pad[0] = r.pad[1] = 0.0;
         crec[blockIdx.x] = r;
     }
+    return true;
 }
 
 // max (or min, with neg = true) of one int over the CTA
@@ -466,6 +563,7 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
     uint32_t *s_tot = s_run + 256;             // 256: scratch (tile totals)
     uint32_t *s_h4 = s_tot + 256;              // 4 * 256: phase-H histograms, then digit bases
     __shared__ int s_skip;
+    __shared__ uint32_t s_d0;   // a scatter tile's first digit
     __shared__ double s_tab[32];
     exp2_table_init(s_tab);
     pdl_wait();
@@ -549,12 +647,38 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                 uint32_t sor[2] = {0u, 0u}, snot[2] = {0u, 0u};   // per sign class: OR of keys, of ~keys
                 const bool walked = walk_chunk(S, A, nullptr, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
                     const int l0 = warp * 32 * K + lane;
+                    {   // the warp's keys all equal to its first (tied scores in order): one add per digit
+                        const uint32_t k0 = __shfl_sync(FULL, key[0], 0);
+                        bool same = true;
+                        uint32_t nv = 0;
+#pragma unroll
+                        for (int i = 0; i < K; ++i) {
+                            const bool v = l0 + i * 32 < cnt_tile;
+                            same &= !v || key[i] == k0;
+                            nv += v;
+                        }
+                        if (__all_sync(FULL, same)) {
+                            nv = __reduce_add_sync(FULL, nv);   // 0: the warp lies past the end of the tile
+                            if (lane == 0 && nv) {
+#pragma unroll
+                                for (int d = 0; d < 4; ++d) atomicAdd(&s_h4[d * 256 + ((k0 >> (8 * d)) & 0xffu)], nv);
+                                const bool ng = k0 >> 31;
+                                sor[0] |= ng ? 0u : k0;
+                                snot[0] |= ng ? 0u : ~k0;
+                                sor[1] |= ng ? k0 : 0u;
+                                snot[1] |= ng ? ~k0 : 0u;
+                            }
+                            return;
+                        }
+                    }
 #pragma unroll
                     for (int i = 0; i < K; ++i) {
                         if (l0 + i * 32 >= cnt_tile) break;
-                        const int sg = key[i] >> 31;
-                        sor[sg] |= key[i];
-                        snot[sg] |= ~key[i];
+                        const bool ng = key[i] >> 31;
+                        sor[0] |= ng ? 0u : key[i];
+                        snot[0] |= ng ? 0u : ~key[i];
+                        sor[1] |= ng ? key[i] : 0u;
+                        snot[1] |= ng ? ~key[i] : 0u;
 #pragma unroll
                         for (int d = 0; d < 4; ++d) {
                             const uint32_t bin = (key[i] >> (8 * d)) & 0xffu;
@@ -628,8 +752,13 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                 if (c == 0 && tid == 0) solve_equal_run(A, n);
             } else {
                 bool first = true;
+                int uni_tiles = 0;   // this CTA's tiles on one digit in the last pass (the same in every thread)
                 for (int pass = 0; pass < 4; ++pass) {
                     if (skip & (1 << pass)) continue;
+                    // count with whole-warp votes where the last pass mostly met uniform tiles
+                    // (sorted or tied scores); per-key votes otherwise
+                    const bool whole = 2 * uni_tiles >= (int)(t1 - t0);
+                    uni_tiles = 0;
                     const int sh = 8 * pass;
                     const uint32_t *src = cur < 0 ? nullptr : (cur == 0 ? A.keys[0] : A.keys[1]);
                     uint32_t *dst = cur == 0 ? A.keys[1] : A.keys[0];
@@ -638,7 +767,8 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                         for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
                         __syncthreads();
                         if (!walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *) {
-                                warp_count(key, cnt_tile, sh, s_hist + warp * 256);
+                                if (whole) warp_count<K, true>(key, cnt_tile, sh, s_hist + warp * 256);
+                                else warp_count<K, false>(key, cnt_tile, sh, s_hist + warp * 256);
                             })) {
                             if (tid == 0) atomicAdd(A_hist_dirty(A), 1ull);
                             return;
@@ -673,10 +803,11 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                     }
                     __syncthreads();
                     const bool walked = walk_chunk(S, A, src, t0, t1, ph, [&](int64_t, int cnt_tile, const uint32_t (&key)[K], uint32_t *s_keys) {
+                        if (tid == 0) s_d0 = (key[0] >> sh) & 0xffu;   // thread 0 holds the tile's first key
                         for (int i = tid; i < RNW * 256; i += RB) s_hist[i] = 0;
                         __syncthreads();   // every key is in registers: s_keys is free too
                         uint32_t *my_hist = s_hist + warp * 256;
-                        warp_count(key, cnt_tile, sh, my_hist);
+                        warp_count<K, false>(key, cnt_tile, sh, my_hist);
                         __syncthreads();
                         if (tid < 256) {   // per digit: exclusive offsets of the warps, tile total
                             uint32_t tot = 0;
@@ -691,6 +822,18 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
                             s_run[tid] += tot;
                         }
                         __syncthreads();
+                        if (s_tot[s_d0] == (uint32_t)cnt_tile) {   // one digit across the tile (sorted or tied
+                            // scores): it keeps its order, so it is written out as it stands
+                            const uint32_t base0 = s_gofs[s_d0];
+#pragma unroll
+                            for (int i = 0; i < K; ++i) {
+                                const int li = warp * 32 * K + i * 32 + lane;
+                                const uint32_t at = base0 + (uint32_t)li;
+                                if (li < cnt_tile && in_bounds(at < (uint32_t)n, &ctl->status)) dst[at] = key[i];
+                            }
+                            ++uni_tiles;
+                            return;   // walk_chunk's barrier follows
+                        }
                         if (warp == 0) {   // exclusive scan of the 256 tile totals
                             uint32_t v[8], run = 0;
 #pragma unroll
@@ -754,7 +897,11 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
             const Seeds z = locate_seeds(A);
             ChunkRec *crec = reinterpret_cast<ChunkRec *>(A.tilebuf);
             TileRec *rec = reinterpret_cast<TileRec *>(A.tilebuf + 8 * SORT_GMAX);
-            if (skip != 15) locate_tiles<K>(A, sorted, n, t0, t1, z, rec, crec, S.buf, reinterpret_cast<Aff *>(s_hist), s_tab);
+            if (skip != 15 &&
+                !locate_tiles<K>(A, S, ph, sorted, n, t0, t1, z, rec, crec, reinterpret_cast<Aff *>(s_hist), s_tab)) {
+                if (tid == 0) atomicAdd(A_hist_dirty(A), 1ull);
+                return;
+            }
             if (!bar()) return;   // the maps are complete, and every CTA has read the global histograms
             if (c == 0) {
                 for (int i = tid; i < 4 * 256; i += RB) A.hist[i] = 0ull;   // ready for the next sort

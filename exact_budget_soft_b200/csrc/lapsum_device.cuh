@@ -442,42 +442,30 @@ template <int NSRC>
 constexpr int bulk_stages() { return NSRC == 1 ? 4 : 3; }
 
 // Shared memory of a pipeline with NSRC sources (dynamic, 16-byte aligned): the
-// stages, then a full and an empty mbarrier per stage.
+// stages, then one mbarrier per stage.
 template <int NSRC>
 constexpr size_t bulk_smem_bytes() {
-    return (size_t)bulk_stages<NSRC>() * NSRC * BULK_F4 * 16 + 2 * 8 * bulk_stages<NSRC>();
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+    return (size_t)bulk_stages<NSRC>() * NSRC * BULK_F4 * 16 + 8 * bulk_stages<NSRC>();
 }
 
 // Streams the full chunks of NSRC float4 arrays of n4 vectors through shared
 // memory and calls body(const float4 *chunk[NSRC], int64_t first_vector) once
 // per chunk, by every thread of the CTA (each thread reads its own vectors of
-// the chunk; the body may use warp-wide operations, never a CTA barrier).
-// Returns the number of vectors covered by full chunks (the rest is the
-// caller's tail).
-//
-// Producer and consumers meet on two mbarriers per stage, not on a CTA barrier
-// per chunk: "full" counts the bytes of the stage's copy; "empty" counts one
-// arrival per warp done with it.  Warp 0 refills a stage once every warp has
-// released it, one chunk behind, so a warp slowed by rare scores holds the
-// others back only when it falls a whole ring behind.  If a wait gives up (any
-// of them), the CTA stops at the next chunk, sets ST_TIMEOUT, and waits (bounded
-// again) for the copies it has in flight before returning (warps still waiting
-// on a copy that is no longer issued leave when their own bounded wait gives up);
-// the caller's result is then invalid and the error reaches the host through the
-// status word.
+// the chunk).  Returns the number of vectors covered by full chunks (the rest
+// is the caller's tail).  One mbarrier per stage counts the bytes of its copy;
+// a CTA barrier after each chunk frees its stage, and thread 0 refills it with
+// the chunk STAGES ahead.  (Measured against a split full/empty mbarrier ring
+// with one arrival per warp: as fast on random score order, 3.5% faster on the
+// sorted 1e8 row.)  If a wait gives up (in any thread), the CTA sets
+// ST_TIMEOUT, issues no further copy, waits (bounded again) for the copies it
+// has in flight and stops streaming; the caller's result is then invalid and
+// the error reaches the host through the status word.
 template <int NSRC, typename Body>
 __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC], int64_t n4, bool reverse,
                                                unsigned char *smem, int32_t *status, Body &&body) {
-    constexpr int ST = bulk_stages<NSRC>();
+    constexpr int BULK_STAGES = bulk_stages<NSRC>();
     float4 *buf = reinterpret_cast<float4 *>(smem);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)ST * NSRC * BULK_F4 * 16);
-    uint64_t *empty = full + ST;
-    __shared__ int s_stop;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)BULK_STAGES * NSRC * BULK_F4 * 16);
     const int64_t nch = n4 / BULK_F4;
     const int64_t G = gridDim.x;
     const int64_t mine = nch > blockIdx.x ? (nch - 1 - blockIdx.x) / G + 1 : 0;
@@ -486,61 +474,46 @@ __device__ __forceinline__ int64_t bulk_stream(const float4 *const (&src)[NSRC],
         return reverse ? nch - 1 - c : c;
     };
     constexpr uint32_t BYTES = BULK_F4 * 16;
-    auto issue = [&](int64_t j) {   // one thread: chunk j into its stage
-        const int s = (int)(j % ST);
-        fence_proxy_async_smem();
-        mbar_expect_tx(&full[s], BYTES * NSRC);
-        const int64_t c = chunk_of(j);
-#pragma unroll
-        for (int q = 0; q < NSRC; ++q)
-            bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &full[s]);
-    };
-    int64_t issued = 0;   // chunks issued (thread 0)
     if (threadIdx.x == 0) {
-        for (int s = 0; s < ST; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], blockDim.x >> 5);
-        }
+        for (int s = 0; s < BULK_STAGES; ++s) mbar_init(&bars[s], 1);
         mbar_init_fence();
-        s_stop = 0;
     }
     __syncthreads();
-    if (threadIdx.x == 0)
-        for (; issued < ST && issued < mine; ++issued) issue(issued);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < BULK_STAGES && s < mine; ++s) {
+            mbar_expect_tx(&bars[s], BYTES * NSRC);
+            const int64_t c = chunk_of(s);
+#pragma unroll
+            for (int q = 0; q < NSRC; ++q)
+                bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &bars[s]);
+        }
+    }
     for (int64_t i = 0; i < mine; ++i) {
-        if (warp == 0 && i >= 1 && i - 1 + ST < mine) {   // refill the stage chunk i - 1 used
-            const int64_t j = i - 1;
-            const bool ok = __all_sync(FULL, mbar_wait(&empty[j % ST], (uint32_t)((j / ST) & 1), BULK_WAIT_CAP));
-            if (lane == 0) {
-                if (ok) {
-                    issue(j + ST);
-                    issued = j + ST + 1;
-                } else {
-                    s_stop = 1;
-                }
-            }
-            __syncwarp();
-        }
-        const int s = (int)(i % ST);
-        if (!__all_sync(FULL, mbar_wait(&full[s], (uint32_t)((i / ST) & 1), BULK_WAIT_CAP))) {
-            if (lane == 0) s_stop = 1;
-            break;
-        }
+        const int s = (int)(i % BULK_STAGES);
+        const uint32_t parity = (uint32_t)((i / BULK_STAGES) & 1);
+        const bool ok = mbar_wait(&bars[s], parity, BULK_WAIT_CAP);
         const float4 *chunk[NSRC];
 #pragma unroll
         for (int q = 0; q < NSRC; ++q) chunk[q] = buf + ((size_t)s * NSRC + q) * BULK_F4;
         body(chunk, chunk_of(i) * BULK_F4);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    __syncthreads();
-    if (s_stop) {   // a wait gave up: the copies in flight land before the CTA leaves
-        if (threadIdx.x == 0) {
-            if (status) atomicOr(status, ST_TIMEOUT);
-            for (int64_t j = issued > ST ? issued - ST : 0; j < issued; ++j)
-                mbar_wait(&full[j % ST], (uint32_t)((j / ST) & 1), BULK_WAIT_CAP);
+        if (!__syncthreads_and(ok)) {   // every thread is done with stage s; a wait gave up
+            if (threadIdx.x == 0) {
+                if (status) atomicOr(status, ST_TIMEOUT);
+                // the copies issued and not yet consumed: chunks i .. i + STAGES - 1
+                for (int64_t j = i; j < i + BULK_STAGES && j < mine; ++j)
+                    mbar_wait(&bars[j % BULK_STAGES], (uint32_t)((j / BULK_STAGES) & 1), BULK_WAIT_CAP);
+            }
+            __syncthreads();
+            return nch * BULK_F4;
         }
-        __syncthreads();
+        if (threadIdx.x == 0 && i + BULK_STAGES < mine) {
+            fence_proxy_async_smem();
+            mbar_expect_tx(&bars[s], BYTES * NSRC);
+            const int64_t c = chunk_of(i + BULK_STAGES);
+#pragma unroll
+            for (int q = 0; q < NSRC; ++q)
+                bulk_load(buf + ((size_t)s * NSRC + q) * BULK_F4, src[q] + c * BULK_F4, BYTES, &bars[s]);
+        }
     }
     return nch * BULK_F4;
 }
