@@ -523,8 +523,8 @@ def run_case(args):
         r = torch.from_numpy(W.scores(w)).cuda()
         g = torch.from_numpy(W.upstream_grad(w)).cuda()
         opts = None
-    elif args.case in ("random", "laplace"):   # one row in random order: shuffled levels, or Laplace(0,1)
-        w = W.WORKLOADS["levels1e8_shuffled" if args.case == "random" else "laplace1e7"]
+    elif args.case in ("random", "laplace", "pixels"):   # one row in random order
+        w = W.WORKLOADS[{"random": "levels1e8_shuffled", "laplace": "laplace1e7", "pixels": "pixels1m"}[args.case]]
         r = torch.from_numpy(W.scores(w)[0]).cuda()
         g = torch.from_numpy(W.upstream_grad(w)[0]).cuda()
         opts = None
@@ -565,7 +565,7 @@ def main():
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--scale-n", type=int, default=0, help="profiling: same workload at another n")
-    ap.add_argument("--case", choices=["rows", "fallback", "batch", "random", "laplace"], default=None,
+    ap.add_argument("--case", choices=["rows", "fallback", "batch", "random", "laplace", "pixels"], default=None,
                     help="profiling driver: time one non-headline case instead of the benchmark")
     ap.add_argument("--case-rows", type=int, default=0)
     args = ap.parse_args()

@@ -48,12 +48,27 @@ __device__ bool last_block_sum(double (&v)[NV], double *partials, unsigned *tick
     __syncthreads();
     if (!s_last) return false;
     __threadfence();
+    // each thread sums its blocks j = tid, tid + BLOCK, ... in that order; the NV
+    // values of JW of them are loaded together, so the combine waits for one L2
+    // round trip per JW blocks instead of one per block and value
+    constexpr int JW = NV >= 8 ? 1 : 8 / NV;
     double w[NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        double s = 0.0;
-        for (int j = tid; j < G; j += BLOCK) s += __ldcg(partials + (size_t)i * G + j);
-        w[i] = s;
+    for (int i = 0; i < NV; ++i) w[i] = 0.0;
+    for (int j0 = tid; j0 < G; j0 += JW * BLOCK) {
+        double x[NV][JW];
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+#pragma unroll
+            for (int u = 0; u < JW; ++u) {
+                const int j = j0 + u * BLOCK;
+                x[i][u] = j < G ? __ldcg(partials + (size_t)i * G + j) : 0.0;
+            }
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+#pragma unroll
+            for (int u = 0; u < JW; ++u)
+                if (j0 + u * BLOCK < G) w[i] += x[i][u];
     }
     block_sum<BLOCK, NV>(w, scratch);
     if (tid == 0) {
@@ -670,22 +685,26 @@ __device__ __forceinline__ void oob_cheap(float x, int bit, const Ends &E, OobAc
 // large t puts ~40% of the scores within 16 t of an end).
 constexpr int SQ = 32 + 8 * 32;   // staged scores per warp: below 32 between chunks, at most 256 added
 
-// One rare score per lane (act false: nothing), by the whole warp: the fp64 tail
-// term of a score near an end; for a band score its queue slot and/or its two
-// certification terms.  Not-a-number scores take neither (the status reports them).
+// The fp64 tail term of a staged score out of the band (act false, or a band
+// score: nothing).  Branch-free, so that two calls interleave their chains; the
+// term of a score it does not add is formed and dropped.
+__device__ __forceinline__ void special_tail(float x, bool act, const Ends &E, OobAcc &a) {
+    const bool above = act && x >= E.aR, below = act && x < E.aL;
+    const double w = above ? ((double)x - E.daR) * E.s2d : (E.daL - (double)x) * E.s2d;
+    const double e = exp2_neg(fmax(w, 0.0), E.tab);
+    a.SR += above ? e : 0.0;
+    a.SL += below ? e : 0.0;
+}
+
+// One rare score per lane (act false: nothing), by the whole warp, once its tail
+// term is in: for a band score its queue slot and/or its two certification
+// terms.  Not-a-number scores take neither (the status reports them).
 template <int MODE>
-__device__ __forceinline__ void special_one(float x, bool act, const Ends &E, OobAcc &a, const BracketParams &P,
-                                            unsigned long long cap, int lane, float *s_bq, unsigned *s_bn) {
+__device__ __forceinline__ void special_band(float x, bool act, const Ends &E, OobAcc &a, const BracketParams &P,
+                                             unsigned long long cap, int lane, float *s_bq, unsigned *s_bn) {
     constexpr bool CERT = MODE == OOB_CERT;
     constexpr bool BANDTERMS = MODE != OOB_STREAM;
-    const bool above = act && x >= E.aR, below = act && x < E.aL;
-    const bool inb = act && !above && !below && x == x;
-    if (above || below) {   // a score out of the band was staged for its fp64 tail term
-        const double w = above ? ((double)x - E.daR) * E.s2d : (E.daL - (double)x) * E.s2d;
-        const double e = exp2_neg(w, E.tab);
-        if (above) a.SR += e;
-        else a.SL += e;
-    }
+    const bool inb = act && x >= E.aL && x < E.aR;   // false for NaN
     if (BANDTERMS && inb) {   // the band score's two certification terms
         tier2(x, E.aL, (double)x, E.daL, E, a.hL, a.hL2);
         tier2(E.aR, x, E.daR, (double)x, E, a.lR, a.lR2);
@@ -713,13 +732,25 @@ __device__ __forceinline__ void special_batch(const float *q, int cnt, const End
                                               const BracketParams &P, unsigned long long cap, int lane,
                                               float *s_bq, unsigned *s_bn) {
     const bool act = lane < cnt;
-    special_one<MODE>(act ? q[lane] : 0.f, act, E, a, P, cap, lane, s_bq, s_bn);
+    const float x = act ? q[lane] : 0.f;
+    special_tail(x, act, E, a);
+    special_band<MODE>(x, act, E, a, P, cap, lane, s_bq, s_bn);
+}
+// 64 staged scores, two per lane: both tail terms first (independent chains).
+template <int MODE>
+__device__ __forceinline__ void special_batch2(const float *q, const Ends &E, OobAcc &a, const BracketParams &P,
+                                               unsigned long long cap, int lane, float *s_bq, unsigned *s_bn) {
+    const float x0 = q[lane], x1 = q[32 + lane];
+    special_tail(x0, true, E, a);
+    special_tail(x1, true, E, a);
+    special_band<MODE>(x0, true, E, a, P, cap, lane, s_bq, s_bn);
+    special_band<MODE>(x1, true, E, a, P, cap, lane, s_bq, s_bn);
 }
 
 template <int MODE, bool ADAPT>
 __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, const Ends &E, OobAcc &a,
                                           const BracketParams &P, unsigned long long cap, int lane,
-                                          float *s_bq, unsigned *s_bn, float *sq, unsigned *sqc, unsigned &sq_n,
+                                          float *s_bq, unsigned *s_bn, float *sq, unsigned &sq_n,
                                           unsigned &hist, unsigned &tick) {
     constexpr bool CERT = MODE == OOB_CERT;
     constexpr bool BANDTERMS = MODE != OOB_STREAM;
@@ -794,11 +825,18 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
     oob_cheap<MODE>(v1.w, 7, E, a, sp);
     if (CERT) a.np += 8;
     const unsigned cnt = __popc(sp);
-    const unsigned total = __reduce_add_sync(FULL, cnt);
+    // stage them at the warp's fill level, each lane after the lanes below it
+    // (an inclusive scan of the counts: no atomics), then handle them 64 or 32
+    // at a time
+    unsigned incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const unsigned total = __shfl_sync(FULL, incl, 31);
     if (total == 0) return;
-    // stage them (slots from the warp's counter, in any order), then handle full batches of 32
-    unsigned pos = 0;
-    if (cnt) pos = atomicAdd(sqc, cnt);
+    unsigned pos = sq_n + incl - cnt;
     while (sp) {
         if (in_bounds(pos < (unsigned)SQ, &P.ctl->status)) sq[pos] = pick8(v0, v1, __ffs(sp) - 1);
         ++pos;
@@ -806,15 +844,15 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
     }
     __syncwarp();
     sq_n += total;
-    if (sq_n >= 32) {
-        do {
-            sq_n -= 32;
-            special_batch<MODE>(sq + sq_n, 32, E, a, P, cap, lane, s_bq, s_bn);
-        } while (sq_n >= 32);
-        __syncwarp();
-        if (lane == 0) *sqc = sq_n;
-        __syncwarp();
+    while (sq_n >= 64) {
+        sq_n -= 64;
+        special_batch2<MODE>(sq + sq_n, E, a, P, cap, lane, s_bq, s_bn);
     }
+    if (sq_n >= 32) {
+        sq_n -= 32;
+        special_batch<MODE>(sq + sq_n, 32, E, a, P, cap, lane, s_bq, s_bn);
+    }
+    __syncwarp();   // the batch's reads are done before the next chunk stages over them
 }
 
 // The verdict, and for a failed first round with widening enabled the side the
@@ -857,7 +895,6 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
     __shared__ double s_tab[32];
     __shared__ float s_bq[CERT ? 1 : BQ];   // sparse band scores of this CTA
     __shared__ float s_sq[SBLOCK / 32][SQ];   // staged rare scores, per warp
-    __shared__ unsigned s_sqc[SBLOCK / 32];   // and each warp's count of them
     __shared__ unsigned s_bn;
     __shared__ unsigned long long s_bbase;
     exp2_table_init(s_tab);
@@ -876,8 +913,6 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
     const int lane = threadIdx.x & 31;
     const unsigned long long cap = (unsigned long long)P.band_cap;
     OobAcc acc{0, 0, 0, 0, 0u, 0u, 0.0, 0.0, 0.0, 0.0, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (lane == 0) s_sqc[threadIdx.x >> 5] = 0u;
-    __syncwarp();
     const int64_t n = P.n;
     const int64_t gtid = (int64_t)blockIdx.x * SBLOCK + threadIdx.x;
     const int64_t gstride = (int64_t)gridDim.x * SBLOCK;
@@ -891,7 +926,7 @@ __global__ void __launch_bounds__(SBLOCK, MINB) oob_kernel(BracketParams Pg) {
         unsigned sq_n = 0, hist = 0, tick = 0;   // the same in every lane of a warp
         done4 = bulk_stream<1>(src, n4, CERT, dsm, &ctl->status, [&](const float4 *const *ch, int64_t) {
             oob_chunk<MODE, ADAPT>(lds128(ch[0] + threadIdx.x), lds128(ch[0] + threadIdx.x + SBLOCK), E, acc, P, cap,
-                                   lane, s_bq, &s_bn, sq, &s_sqc[threadIdx.x >> 5], sq_n, hist, tick);
+                                   lane, s_bq, &s_bn, sq, sq_n, hist, tick);
         });
         __syncwarp();
         if (sq_n) special_batch<MODE>(sq, (int)sq_n, E, acc, P, cap, lane, s_bq, &s_bn);

@@ -468,6 +468,21 @@ def test_band_select_sizes(L, orc, s, lo, hi):
     check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0])
 
 
+@pytest.mark.parametrize("t", [0.02, 0.05])
+def test_band_select_short_band_of_a_few_tied_levels(L, orc, t):
+    # a short band (at most 4096 scores, copied to shared memory at once) of three
+    # or four whole tied levels: the narrowing ends on one level or on the gap
+    # between two
+    n = 1 << 18
+    r, g = W.small_case("levels256_desc", 1, n, seed=22)
+    k = 1.5 * n / 256
+    p, b, st, grad = run(L, r, k, t, opts=L.options(force_path=L.PATH_BRACKET), g_np=g)
+    assert st["rc"] == 0 and st["path"] == 2 and st["verdict"] == 1
+    band = r[0][(r[0] >= np.float32(st["a_L"])) & (r[0] < np.float32(st["a_R"]))]
+    assert 0 < band.size <= 4096 and np.unique(band).size >= 3 and st["c_band"] == band.size
+    check_row(orc, r[0], g[0], k, t, p[0], b[0], grad[0], exact_sum=False)
+
+
 @pytest.mark.parametrize("certify", [0, 1])
 def test_band_select_band_across_zero(L, orc, certify):
     # k = n/2 puts the band around 0: its keys span both signs (a 31-bit key
