@@ -133,25 +133,69 @@ __device__ __forceinline__ void bitonic_regs(uint32_t (&k)[N]) {
     }
 }
 
+// Merges the 32 lanes' ascending runs of KPT keys (KPT a power of two) into one
+// ascending run of 32 KPT keys, lane l holding positions l KPT .. l KPT + KPT - 1:
+// the phases of a bitonic sorting network, each opening with a stage that
+// compares a key with its mirror image in the phase's block (so that both halves
+// may come in ascending), then half-cleaners -- across lanes by shuffles, then
+// within each lane's registers.  No branch depends on the data.
+template <int KPT>
+__device__ __forceinline__ void warp_bitonic_merge(uint32_t (&k)[KPT]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {   // blocks of 2m lanes
+        const bool lower = (lane & m) == 0;
+#pragma unroll
+        for (int i = 0; i < KPT / 2; ++i) {   // key i against the partner's key KPT - 1 - i, and back
+            const uint32_t a = k[i], b = k[KPT - 1 - i];
+            const uint32_t pa = __shfl_xor_sync(FULL, b, 2 * m - 1), pb = __shfl_xor_sync(FULL, a, 2 * m - 1);
+            k[i] = lower ? min(a, pa) : max(a, pa);
+            k[KPT - 1 - i] = lower ? min(b, pb) : max(b, pb);
+        }
+#pragma unroll
+        for (int h = m >> 1; h > 0; h >>= 1) {   // lanes h apart
+            const bool lo = (lane & h) == 0;
+#pragma unroll
+            for (int i = 0; i < KPT; ++i) {
+                const uint32_t v = __shfl_xor_sync(FULL, k[i], h);
+                k[i] = lo ? min(k[i], v) : max(k[i], v);
+            }
+        }
+#pragma unroll
+        for (int j = KPT >> 1; j > 0; j >>= 1) {   // registers j apart
+#pragma unroll
+            for (int i = 0; i < KPT; ++i) {
+                if ((i & j) == 0) {
+                    const uint32_t a = k[i], b = k[i | j];
+                    k[i] = min(a, b);
+                    k[i | j] = max(a, b);
+                }
+            }
+        }
+    }
+}
+
 // Block-wide merge sort of KPT keys per thread (ascending), the alternative to
-// the radix sort for one CTA's row: each thread sorts its keys in registers,
-// then log2(BLOCK) merge levels double the sorted runs in shared memory.  At a
-// level of runs of L, thread t produces outputs [KPT t, KPT t + KPT) of the
-// merge of its pair of runs: it finds where its outputs start by a binary search
-// on the merge path (the first i with A[i] > B[o - i - 1]) and then merges
-// KPT elements sequentially.  No warp votes: every step is a compare, a select
-// and a shared-memory load.  On return the sorted keys are in s_keys (position
-// j at spad(j)).
+// the radix sort for one CTA's row: each thread sorts its keys in registers
+// (bitonic network), each warp merges its lanes' runs in registers
+// (warp_bitonic_merge), then log2(BLOCK / 32) merge levels double the sorted runs
+// in shared memory.  At a level of runs of L, thread t produces outputs
+// [KPT t, KPT t + KPT) of the merge of its pair of runs: it finds where its
+// outputs start by a binary search on the merge path (the first i with
+// A[i] > B[o - i - 1]) and then merges KPT elements sequentially: a compare, a
+// select and a shared-memory load per output.  On return the sorted keys are in
+// s_keys (position j at spad(j)).
 template <int BLOCK, int KPT>
 __device__ __forceinline__ void block_merge_sort(uint32_t (&key)[KPT], uint32_t *s_keys) {
     constexpr int CAP = BLOCK * KPT;
     const int tid = threadIdx.x;
     bitonic_regs<KPT>(key);
+    warp_bitonic_merge<KPT>(key);
 #pragma unroll
     for (int q = 0; q < KPT; ++q) s_keys[spad(KPT * tid + q)] = key[q];
     __syncthreads();
 #pragma unroll 1
-    for (int L = KPT; L < CAP; L <<= 1) {
+    for (int L = 32 * KPT; L < CAP; L <<= 1) {
         const int out0 = KPT * tid;
         const int base = out0 & ~(2 * L - 1);
         const int o = out0 - base;                 // output offset within the pair's merge
