@@ -779,6 +779,10 @@ __device__ __forceinline__ void oob_chunk(const float4 v0, const float4 v1, cons
         }
         if (__all_sync(FULL, mx < E.midL && fin)) {            // below a_L, fp32 terms
             if (CERT) { a.cB += 8; a.np += 8; } else a.cL += 8;
+            if (__all_sync(FULL, eq0 && eq1)) {   // tied scores: one term per float4 (4a = (a + a) + (a + a))
+                a.SL2 += 4.f * ex2_ftz((v0.x - E.aL) * E.s2) + 4.f * ex2_ftz((v1.x - E.aL) * E.s2);
+                return;
+            }
             a.SL2 += ((ex2_ftz((v0.x - E.aL) * E.s2) + ex2_ftz((v0.y - E.aL) * E.s2)) +
                       (ex2_ftz((v0.z - E.aL) * E.s2) + ex2_ftz((v0.w - E.aL) * E.s2))) +
                      ((ex2_ftz((v1.x - E.aL) * E.s2) + ex2_ftz((v1.y - E.aL) * E.s2)) +
@@ -1071,7 +1075,22 @@ p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restric
     if (aligned) {
         const float4 *src[1] = {r4};
         done4 = bulk_stream<1>(src, n4, false, dsm, &ctl->status, [&](const float4 *const *ch, int64_t base4) {
-            const float4 o0 = p_vec(lds128(ch[0] + threadIdx.x), xf), o1 = p_vec(lds128(ch[0] + threadIdx.x + SBLOCK), xf);
+            const float4 v0 = lds128(ch[0] + threadIdx.x), v1 = lds128(ch[0] + threadIdx.x + SBLOCK);
+            float4 o0, o1;
+            if (__all_sync(FULL, v0.x == v0.y && v0.y == v0.z && v0.z == v0.w && v1.x == v1.y && v1.y == v1.z &&
+                                     v1.z == v1.w)) {   // tied scores (one vote a chunk): one p per float4
+                float q0, q1;
+                const bool m0 = xf.fast(v0.x, q0), m1 = xf.fast(v1.x, q1);
+                if (__any_sync(FULL, m0 || m1)) {
+                    if (m0) q0 = xf.mid(v0.x);
+                    if (m1) q1 = xf.mid(v1.x);
+                }
+                o0 = make_float4(q0, q0, q0, q0);
+                o1 = make_float4(q1, q1, q1, q1);
+            } else {
+                o0 = p_vec(v0, xf);
+                o1 = p_vec(v1, xf);
+            }
             __stcs(p4 + base4 + threadIdx.x, o0);
             __stcs(p4 + base4 + threadIdx.x + SBLOCK, o1);
             ps += (double)(((o0.x + o0.y) + (o0.z + o0.w)) + ((o1.x + o1.y) + (o1.z + o1.w)));
