@@ -280,6 +280,41 @@ def test_levels1e8_workload_and_forced_fallback(L, orc):
     check_large(orc, r, None, w.k, w.t, p2, b2[0], None, rng)
 
 
+@pytest.mark.slow
+def test_levels1e8_in_random_order(L, orc):
+    # the same 1e8 tied scores shuffled (the bench's random-order line): no warp
+    # of the out-of-band passes sees one side of the bracket, a fifth of the
+    # scores take the staged fp64 terms; bracket and counts exact, b, sampled p
+    # and the VJP to tolerance
+    w = W.WORKLOADS["levels1e8_shuffled"]
+    r, g = W.scores(w)[0], W.upstream_grad(w)[0]
+    rng = np.random.default_rng(1)
+    p, b, st, grad = run(L, r, w.k, w.t, g_np=g)
+    assert st["rc"] == 0 and st["path"] == 2 and st["verdict"] == 1 and st["fallback"] == 0
+    plan = L.bracket_plan(w.n, w.k)
+    cert = check_bracket_integers(orc, r, w.k, w.t, st, 0, plan["s"], 1e-6)
+    assert abs(st["G_aL"] - cert["G_aL"]) <= 1e-6 * max(1.0, cert["G_aL"])
+    assert abs(st["G_aR"] - cert["G_aR"]) <= 1e-6 * max(1.0, cert["G_aR"])
+    check_large(orc, r, g, w.k, w.t, p, b[0], grad, rng)
+
+
+@pytest.mark.slow
+def test_batch64x1m_workload(L, orc):
+    # the bench's batched-bracketing line: 64 rows of 2^20 N(0,1) scores, each
+    # with its own bracket (Philox counter word = row), band and certification
+    w = W.WORKLOADS["batch64x1m"]
+    r, g = W.scores(w), W.upstream_grad(w)
+    p, b, sts, grad = run_rows(L, r, w.k, w.t, g_np=g)
+    plan = L.bracket_plan(w.n, w.k)
+    for i in range(w.rows):
+        st = sts[i]
+        e = expected_row(orc, r[i], w.k, w.t, 0, plan["s"], 1e-6, i)
+        assert st["rc"] == 0 and st["verdict"] == e["cert"]["verdict"] == 1
+        assert np.float32(st["a_L"]) == e["br"]["a_L"] and np.float32(st["a_R"]) == e["br"]["a_R"]
+        assert (st["c_L"], st["c_band"], st["c_R"]) == (e["cert"]["c_L"], e["cert"]["c_band"], e["cert"]["c_R"])
+        check_row(orc, r[i], g[i], w.k, w.t, p[i], b[i], grad[i])
+
+
 @pytest.mark.parametrize("certify", [0, 1])
 @pytest.mark.parametrize("level", [0, 1, 2])
 def test_bracketing_band_of_one_tied_level(L, orc, level, certify):
