@@ -1035,19 +1035,35 @@ __device__ __forceinline__ float4 p_vec_lane(const float4 v, const PForm &pf) {
     return make_float4(pf(v.x), pf(v.y), pf(v.z), pf(v.w));
 }
 
-// Four p at once: the fp32 value for all, then -- only in warps where some lane
-// has a mid-range p (one vote) -- the fp64 value for those (PForm).  Every lane
-// of the warp must call it together (the chunks of the bulk pipeline).
-__device__ __forceinline__ float4 p_vec(const float4 v, const PForm &pf) {
-    float4 o;
-    const bool m0 = pf.fast(v.x, o.x), m1 = pf.fast(v.y, o.y), m2 = pf.fast(v.z, o.z), m3 = pf.fast(v.w, o.w);
-    if (__any_sync(FULL, m0 || m1 || m2 || m3)) {
-        if (m0) o.x = pf.mid(v.x);
-        if (m1) o.y = pf.mid(v.y);
-        if (m2) o.z = pf.mid(v.z);
-        if (m3) o.w = pf.mid(v.w);
+// Eight p (one chunk slot pair) at once: the fp32 value for all, then the fp64
+// value of the mid-range ones, one per lane per round (the lane's first pending
+// one), so a warp evaluates the fp64 form as often as its busiest lane has a
+// mid-range score -- usually once -- not once per slot that any lane needs.
+// Every lane of the warp must call it together.
+__device__ __forceinline__ void p_vec8(const float4 v0, const float4 v1, const PForm &pf, float4 &o0, float4 &o1) {
+    unsigned mm = 0;
+    mm |= pf.fast(v0.x, o0.x) ? 1u : 0u;
+    mm |= pf.fast(v0.y, o0.y) ? 2u : 0u;
+    mm |= pf.fast(v0.z, o0.z) ? 4u : 0u;
+    mm |= pf.fast(v0.w, o0.w) ? 8u : 0u;
+    mm |= pf.fast(v1.x, o1.x) ? 16u : 0u;
+    mm |= pf.fast(v1.y, o1.y) ? 32u : 0u;
+    mm |= pf.fast(v1.z, o1.z) ? 64u : 0u;
+    mm |= pf.fast(v1.w, o1.w) ? 128u : 0u;
+    while (__any_sync(FULL, mm != 0u)) {
+        const int i = mm ? __ffs(mm) - 1 : 0;
+        const float q = pf.mid(pick8(v0, v1, i));
+        const unsigned hit = mm & (0u - mm);   // the slot this lane fills (0: none)
+        o0.x = (hit & 1u) ? q : o0.x;
+        o0.y = (hit & 2u) ? q : o0.y;
+        o0.z = (hit & 4u) ? q : o0.z;
+        o0.w = (hit & 8u) ? q : o0.w;
+        o1.x = (hit & 16u) ? q : o1.x;
+        o1.y = (hit & 32u) ? q : o1.y;
+        o1.z = (hit & 64u) ? q : o1.z;
+        o1.w = (hit & 128u) ? q : o1.w;
+        mm &= mm - 1u;
     }
-    return o;
 }
 
 __global__ void __launch_bounds__(SBLOCK, SBLOCKS_PER_SM)
@@ -1088,8 +1104,7 @@ p_kernel(const float *__restrict__ r_, int64_t n, double inv_t, float *__restric
                 o0 = make_float4(q0, q0, q0, q0);
                 o1 = make_float4(q1, q1, q1, q1);
             } else {
-                o0 = p_vec(v0, xf);
-                o1 = p_vec(v1, xf);
+                p_vec8(v0, v1, xf, o0, o1);
             }
             __stcs(p4 + base4 + threadIdx.x, o0);
             __stcs(p4 + base4 + threadIdx.x + SBLOCK, o1);
