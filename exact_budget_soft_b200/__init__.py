@@ -67,7 +67,8 @@ EXPORTS = ["lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get
            "lapsum_strerror", "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read",
            "lapsum_bracket_plan", "lapsum_profile_filter", "lapsum_selftest_math", "lapsum_launch_count",
            "lapsum_backward_noalloc", "lapsum_shard_plan", "lapsum_shard_sample", "lapsum_shard_stream",
-           "lapsum_shard_solve", "lapsum_shard_p", "lapsum_shard_vjp_partial", "lapsum_shard_vjp_apply"]
+           "lapsum_shard_solve", "lapsum_shard_p", "lapsum_shard_vjp_partial", "lapsum_shard_vjp_apply",
+           "lapsum_step_host"]
 SHARD_PART = 10   # doubles in a slice's streaming-pass record (LAPSUM_SHARD_PART)
 
 
@@ -81,6 +82,8 @@ def _load() -> C.CDLL:
     lib.lapsum_forward.argtypes = [vp, i64, i64, dbl, dbl, vp, vp, vp]
     lib.lapsum_forward_ex.argtypes = [vp, i64, i64, dbl, dbl, vp, vp, C.POINTER(Options), vp]
     lib.lapsum_backward.argtypes = [vp, vp, vp, i64, i64, dbl, vp, vp]
+    lib.lapsum_step_host.argtypes = [vp, vp, i64, i64, dbl, dbl, vp, vp, vp, C.POINTER(Options),
+                                     vp, vp, vp, vp, vp, vp]
     lib.lapsum_get_stats.argtypes = [C.POINTER(Stats), vp]
     lib.lapsum_get_stats_rows.argtypes = [C.POINTER(Stats), i64, C.POINTER(i64), vp]
     lib.lapsum_strerror.restype = C.c_char_p
@@ -107,7 +110,7 @@ def _load() -> C.CDLL:
     for name in ("lapsum_shard_plan", "lapsum_shard_sample", "lapsum_shard_stream", "lapsum_shard_solve",
                  "lapsum_shard_p", "lapsum_shard_vjp_partial", "lapsum_shard_vjp_apply"):
         getattr(lib, name).restype = C.c_int
-    for name in ("lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_get_stats",
+    for name in ("lapsum_forward", "lapsum_forward_ex", "lapsum_backward", "lapsum_step_host", "lapsum_get_stats",
                  "lapsum_release", "lapsum_profile_enable", "lapsum_profile_read"):
         getattr(lib, name).restype = C.c_int
     return lib
@@ -265,6 +268,38 @@ def forward_host(scores_host: torch.Tensor, k: float, t: float, device="cuda", o
     d = scores_host.to(device, non_blocking=True)
     p, b = forward(d, k, t, opts=opts, stream=stream)
     return p.to("cpu", non_blocking=False), b.to("cpu", non_blocking=False)
+
+
+def step_host(scores_h: torch.Tensor, g_h: torch.Tensor, k: float, t: float, p_h: torch.Tensor,
+              b_h: torch.Tensor, grad_h: torch.Tensor, scores_d: torch.Tensor, g_d: torch.Tensor,
+              p_d: torch.Tensor, b_d: torch.Tensor, grad_d: torch.Tensor, opts: Options | None = None,
+              stream=None) -> None:
+    """One forward + VJP step on host tensors (lapsum_step_host): scores_h and g_h
+    in, p_h, b_h and grad_h out, through the caller's device buffers; the copies
+    overlap the work where the data allow.  Asynchronous on `stream`: the host
+    results are there once it has been synchronised.  Pinned host tensors let the
+    copies run asynchronously."""
+    rows, n = _as_rows(scores_h)
+    for x, name, dt in ((scores_h, "scores_h", torch.float32), (g_h, "g_h", torch.float32),
+                        (p_h, "p_h", torch.float32), (b_h, "b_h", torch.float64),
+                        (grad_h, "grad_h", torch.float32)):
+        if x.is_cuda or x.dtype != dt or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor of {dt}")
+    for x, name, dt in ((scores_d, "scores_d", torch.float32), (g_d, "g_d", torch.float32),
+                        (p_d, "p_d", torch.float32), (b_d, "b_d", torch.float64),
+                        (grad_d, "grad_d", torch.float32)):
+        _need(x, name, dt)
+    for x, name in ((g_h, "g_h"), (p_h, "p_h"), (grad_h, "grad_h"), (scores_d, "scores_d"), (g_d, "g_d"),
+                    (p_d, "p_d"), (grad_d, "grad_d")):
+        if x.numel() != rows * n:
+            raise ValueError(f"{name} must hold rows x n = {rows} x {n} values")
+    if b_h.numel() != rows or b_d.numel() != rows:
+        raise ValueError("b_h and b_d must hold one threshold per row")
+    rc = lib.lapsum_step_host(scores_h.data_ptr(), g_h.data_ptr(), rows, n, float(k), float(t), p_h.data_ptr(),
+                              b_h.data_ptr(), grad_h.data_ptr(), C.byref(opts) if opts is not None else None,
+                              scores_d.data_ptr(), g_d.data_ptr(), p_d.data_ptr(), b_d.data_ptr(),
+                              grad_d.data_ptr(), _stream(stream))
+    _check(rc, "lapsum_step_host")
 
 
 class _SoftTopK(torch.autograd.Function):

@@ -627,6 +627,80 @@ int lapsum_backward(const float *scores, const double *b, const float *g, int64_
     return w->verify_guards(st);
 }
 
+// ---- one step on host buffers: copies on two side streams per device ----
+namespace {
+struct SideStreams {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+};
+std::mutex g_side_mu;
+std::map<int, SideStreams> g_side;
+
+cudaError_t side_streams(SideStreams *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStreams &s = g_side[dev];
+    if (!s.h2d && (e = cudaStreamCreateWithFlags(&s.h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if (!s.d2h && (e = cudaStreamCreateWithFlags(&s.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    *out = s;
+    return cudaSuccess;
+}
+
+// Events of one call: released when the call returns (the device keeps an
+// event it still has to complete).
+struct StepEvents {
+    cudaEvent_t e[6] = {};
+    cudaError_t create() {
+        for (auto &x : e) {
+            const cudaError_t r = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+            if (r != cudaSuccess) return r;
+        }
+        return cudaSuccess;
+    }
+    ~StepEvents() {
+        for (auto &x : e)
+            if (x) cudaEventDestroy(x);
+    }
+};
+}  // namespace
+
+int lapsum_step_host(const float *scores_h, const float *g_h, int64_t rows, int64_t n, double k, double t,
+                     float *p_h, double *b_h, float *grad_h, const lapsum_options *opt, float *scores_dev,
+                     float *g_dev, float *p_dev, double *b_dev, float *grad_dev, struct CUstream_st *stream_in) {
+    if (!scores_h || !g_h || !p_h || !b_h || !grad_h || !g_dev || !p_dev || !b_dev || !grad_dev) return LAPSUM_ERR_ARG;
+    const int rc0 = check_args(scores_dev, rows, n, k, t);
+    if (rc0 != LAPSUM_OK) return rc0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
+    const size_t bytes = (size_t)rows * (size_t)n * sizeof(float);
+    SideStreams ss;
+    LAPSUM_TRY(side_streams(&ss));
+    StepEvents ev;   // 0 start, 1 scores in, 2 g in, 3 forward done, 4 backward done, 5 copies out
+    LAPSUM_TRY(ev.create());
+    LAPSUM_TRY(cudaEventRecord(ev.e[0], st));   // after the caller's earlier work on `stream`
+    LAPSUM_TRY(cudaStreamWaitEvent(ss.h2d, ev.e[0], 0));
+    LAPSUM_TRY(cudaMemcpyAsync(scores_dev, scores_h, bytes, cudaMemcpyHostToDevice, ss.h2d));
+    LAPSUM_TRY(cudaEventRecord(ev.e[1], ss.h2d));
+    LAPSUM_TRY(cudaMemcpyAsync(g_dev, g_h, bytes, cudaMemcpyHostToDevice, ss.h2d));
+    LAPSUM_TRY(cudaEventRecord(ev.e[2], ss.h2d));
+    LAPSUM_TRY(cudaStreamWaitEvent(st, ev.e[1], 0));
+    int rc = lapsum_forward_ex(scores_dev, rows, n, k, t, p_dev, b_dev, opt, stream_in);
+    if (rc != LAPSUM_OK) return rc;
+    LAPSUM_TRY(cudaEventRecord(ev.e[3], st));
+    LAPSUM_TRY(cudaStreamWaitEvent(ss.d2h, ev.e[3], 0));   // p and b leave while g arrives
+    LAPSUM_TRY(cudaMemcpyAsync(p_h, p_dev, bytes, cudaMemcpyDeviceToHost, ss.d2h));
+    LAPSUM_TRY(cudaMemcpyAsync(b_h, b_dev, (size_t)rows * sizeof(double), cudaMemcpyDeviceToHost, ss.d2h));
+    LAPSUM_TRY(cudaStreamWaitEvent(st, ev.e[2], 0));
+    rc = lapsum_backward(scores_dev, b_dev, g_dev, rows, n, t, grad_dev, stream_in);
+    if (rc != LAPSUM_OK) return rc;
+    LAPSUM_TRY(cudaEventRecord(ev.e[4], st));
+    LAPSUM_TRY(cudaStreamWaitEvent(ss.d2h, ev.e[4], 0));
+    LAPSUM_TRY(cudaMemcpyAsync(grad_h, grad_dev, bytes, cudaMemcpyDeviceToHost, ss.d2h));
+    LAPSUM_TRY(cudaEventRecord(ev.e[5], ss.d2h));
+    LAPSUM_TRY(cudaStreamWaitEvent(st, ev.e[5], 0));   // `stream` completes once every copy has
+    return LAPSUM_OK;
+}
+
 static void fill_stats(const Ctl &c, lapsum_stats *out) {
     std::memset(out, 0, sizeof(*out));
     out->path = c.path == 2 ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;

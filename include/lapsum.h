@@ -191,6 +191,33 @@ LAPSUM_API int lapsum_backward(const float *scores_dev, const double *b_dev, con
                     int64_t rows, int64_t n, double t, float *grad_out_dev,
                     struct CUstream_st *stream);
 
+/*
+ * One forward + VJP step on HOST buffers: copies the scores and g to the
+ * device, runs lapsum_forward_ex and lapsum_backward, and copies p, b and grad
+ * back, the copies overlapping the work where the data allow ("Fast LapSum",
+ * technical summary sections 2.1-2.2):
+ *
+ *   scores in -> forward -> [p, b out  |  g in] -> backward -> grad out
+ *
+ * Host buffers (fp32 [rows][n], b fp64 [rows]): scores_h, g_h read; p_h, b_h,
+ * grad_h written.  Page-locked host memory (cudaHostAlloc / pinned tensors)
+ * lets the copies run asynchronously and in both directions at once; pageable
+ * memory works, with synchronous copies.
+ * Device buffers, caller-owned, of the same shapes: scores_dev, g_dev, p_dev,
+ * grad_dev, b_dev (grad_dev may alias g_dev; nothing else may alias).
+ * Enqueued on `stream` (the copies on two side streams of the library, ordered
+ * against `stream` by events): the call returns at once, and the host buffers
+ * hold the results once `stream` has been synchronised; until then they must
+ * stay valid and untouched.
+ * Returns: LAPSUM_ERR_ARG for a null pointer or the forward's argument errors
+ * (checked before anything is enqueued), LAPSUM_ERR_CUDA if a copy, stream or
+ * event call fails, else the forward's and backward's own codes.
+ */
+LAPSUM_API int lapsum_step_host(const float *scores_h, const float *g_h, int64_t rows, int64_t n, double k,
+                                double t, float *p_h, double *b_h, float *grad_h, const lapsum_options *opt,
+                                float *scores_dev, float *g_dev, float *p_dev, double *b_dev, float *grad_dev,
+                                struct CUstream_st *stream);
+
 /* Copies the last forward's diagnostics to *out. Synchronises `stream`.
  * Returns the device error as a LAPSUM_ERR_* code (LAPSUM_OK if none). */
 LAPSUM_API int lapsum_get_stats(lapsum_stats *out, struct CUstream_st *stream);

@@ -76,6 +76,28 @@ def test_null_pointers_rejected(lib):
     assert lib.lapsum_forward(None, 1, 10, 2.0, 1.0, None, None, None) == -1
 
 
+STEP_HOST_ARGS = [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_double, C.c_double, C.c_void_p, C.c_void_p,
+                  C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+
+
+@pytest.mark.parametrize("null_at", range(10))
+def test_step_host_rejects_a_null_buffer(lib, null_at):
+    # lapsum_step_host: any null host or device buffer is refused before anything is enqueued
+    lib.lapsum_step_host.argtypes = STEP_HOST_ARGS
+    bufs = [C.c_void_p(0x1000 + 0x100 * i) for i in range(10)]   # never dereferenced
+    bufs[null_at] = None
+    sh, gh, ph, bh, grh, sd, gd, pd, bd, grd = bufs
+    assert lib.lapsum_step_host(sh, gh, 1, 10, 2.0, 1.0, ph, bh, grh, None, sd, gd, pd, bd, grd, None) == -1
+
+
+@pytest.mark.parametrize("rows,n,k,t", [(0, 10, 1.0, 1.0), (1, 10, 10.0, 1.0), (1, 10, 2.0, 0.0),
+                                        (1, 10, float("nan"), 1.0), (1, 10, 2.0, 1e37)])
+def test_step_host_rejects_bad_sizes(lib, rows, n, k, t):
+    lib.lapsum_step_host.argtypes = STEP_HOST_ARGS
+    f = C.c_void_p(0x1000)
+    assert lib.lapsum_step_host(f, f, rows, n, k, t, f, f, f, None, f, f, f, f, f, None) == -1
+
+
 class Options(C.Structure):
     _fields_ = [("seed", C.c_uint64), ("sample_size", C.c_int64), ("delta", C.c_double),
                 ("band_cap", C.c_int64), ("spin_cap", C.c_int32), ("force_path", C.c_int32),
