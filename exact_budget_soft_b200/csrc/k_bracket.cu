@@ -655,8 +655,8 @@ __device__ __forceinline__ float pick8(const float4 &u, const float4 &w, int i) 
 // The common part of the general path for one score: the counts, and the fp32
 // tail term of a score more than 16 t beyond its end (the bulk of a long row);
 // every other score -- near an end (fp64 term), in the band, or not a number --
-// only sets its bit in sp_m for special_one.  About sixteen instructions, with
-// the two ends' sums kept apart by predicated adds.
+// only sets its bit in sp_m, to be staged (special_tail, special_band).  About
+// sixteen instructions, with the two ends' sums kept apart by predicated adds.
 template <int MODE>
 __device__ __forceinline__ void oob_cheap(float x, int bit, const Ends &E, OobAcc &a, uint32_t &sp_m) {
     constexpr bool CERT = MODE == OOB_CERT;
