@@ -565,8 +565,22 @@ __global__ void __launch_bounds__(RB, 2) radix_sort_kernel(SortArgs Ag) {
     __shared__ int s_skip;
     __shared__ uint32_t s_d0;   // a scatter tile's first digit
     __shared__ double s_tab[32];
-    exp2_table_init(s_tab);
     pdl_wait();
+    {   // every row's gate closed (the certification passed everywhere): nothing to do,
+        // and nothing else is touched (a clean-up owed by an earlier give-up waits for
+        // the next launch that sorts)
+        bool open = false;
+        for (int64_t r = threadIdx.x; r < Ag.rows; r += RB) {
+            SortArgs A = Ag;
+            A.ctl = Ag.ctl + r;
+            open |= gated_n(A) >= 0;
+        }
+        if (!__syncthreads_or(open)) {
+            pdl_trigger();
+            return;
+        }
+    }
+    exp2_table_init(s_tab);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x, c = blockIdx.x;
     TileStage<K> S;
