@@ -11,10 +11,11 @@
 //   p_kernel        p = F((r - b)/t)
 //   vjp_*_kernel    <g,f>/sum f, then grad = (f/t)(g - <g,f>/sum f)
 //
-// The long passes are persistent grid-stride loops over 16-byte vectors with a
-// fixed grid, so every per-block partial covers a fixed set of elements and the
-// "last block" combine (one atomic ticket, fixed summation order) makes every
-// reduction bitwise reproducible.
+// The long passes are persistent grids that walk the row in 8 KB chunks staged
+// in shared memory by bulk copies (bulk_stream), chunk c to block c mod grid, so
+// every per-block partial covers a fixed set of elements and the "last block"
+// combine (one atomic ticket, fixed summation order) makes every reduction
+// bitwise reproducible.
 #include <cstdint>
 
 #include "lapsum_device.cuh"

@@ -6,9 +6,12 @@
 //   full sort, n <= 32768      one launch: one CTA per row sorts, scans, solves
 //                              and writes p
 //   full sort, longer rows     device radix sort -> locate-scan -> p pass
-//   bracketing (rows == 1,     sample -> select -> streaming pass -> band solve
-//   n >= 2^20 by default)      (one CTA, or device sort + locate) -> certification
-//                              -> gated full-sort fallback -> p pass
+//   bracketing (n >= 2^20 by   sample -> select -> streaming pass -> band select
+//   default; rows of a batch   (one CTA per row) -> certification (or folded into
+//   each bracketed)            the streaming pass) -> optional widening round ->
+//                              gated full-sort fallback -> p pass
+//   VJP                        one CTA per short row, else reduce -> apply
+//   host buffers               lapsum_step_host: the copies on two side streams
 // No step synchronises the host: the band size and the verdict live in device
 // memory and every gated kernel returns at once when it has nothing to do.
 #include <algorithm>
