@@ -1,10 +1,8 @@
 // k_noalloc.cu -- a backward (VJP) entry point that allocates no device memory.
 //
-// Who needs it: code that must not call cudaMalloc on the hot path -- e.g. a
-// caller in the middle of recording work into a CUDA graph with a strict
-// capture mode (allocation calls are illegal there), an inference plugin whose
-// host framework owns all device memory, or a process running under a fixed
-// memory budget.  lapsum_backward keeps per-stream scratch that it grows with
+// Who needs it: code that must not call cudaMalloc on the hot path -- e.g. an
+// inference plugin whose host framework owns all device memory, or a process
+// running under a fixed memory budget.  lapsum_backward keeps per-stream scratch that it grows with
 // cudaMalloc on first use; this variant instead uses one fixed array compiled
 // into the library (LAPSUM_NOALLOC_SCRATCH_BYTES per GPU, held for the life of
 // the process by every GPU that loads the library).

@@ -274,10 +274,8 @@ LAPSUM_API int lapsum_selftest_math(int which, const double *in_dev, double *out
 /*
  * Backward without any device allocation.  The method's pages have no
  * counterpart of this entry point: it exists for callers that may not call
- * cudaMalloc while they run -- for instance code recording work into a CUDA
- * graph under a strict capture mode (allocation is illegal there), a plugin
- * inside a host framework that owns all device memory, or a process held to a
- * fixed memory budget.  lapsum_backward grows a per-stream workspace with
+ * cudaMalloc while they run -- for instance a plugin inside a host framework
+ * that owns all device memory, or a process held to a fixed memory budget.  lapsum_backward grows a per-stream workspace with
  * cudaMalloc on first use; this variant keeps its scratch (per-block partial
  * sums, one lambda and one counter per row) in a single array compiled into
  * the library, LAPSUM_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that
@@ -294,7 +292,7 @@ LAPSUM_API int lapsum_selftest_math(int which, const double *in_dev, double *out
  * LAPSUM_ERR_ARG before anything is enqueued.
  *
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * (cudaGetSymbolAddress) and keeps it for later calls.
  * All calls on a device share the one array: each call clears the counters it
  * needs, but two calls that overlap on the GPU (different streams, or host
  * threads) race on it -- order them on one stream.

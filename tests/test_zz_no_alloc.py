@@ -1,9 +1,8 @@
 """The allocation-free backward entry point (lapsum_backward_noalloc).
 
-It serves callers that may not call cudaMalloc while they run -- code recording
-into a CUDA graph under a strict capture mode, plugins inside a framework that
-owns all device memory, processes held to a fixed memory budget -- by keeping
-its scratch in an array compiled into the library.  These tests call it through
+It serves callers that may not call cudaMalloc while they run -- plugins inside
+a framework that owns all device memory, processes held to a fixed memory
+budget -- by keeping its scratch in an array compiled into the library.  These tests call it through
 the C ABI and compare it with lapsum_backward on the same inputs, two calls in a
 row (the second call must not see the first call's leftovers), and check that a
 call too large for the array is refused.  The file is named to be collected
