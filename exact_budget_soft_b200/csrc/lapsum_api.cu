@@ -165,8 +165,13 @@ constexpr size_t GUARD_BYTES = 0;
 #endif
 constexpr unsigned char GUARD_FILL = 0xA5;
 
+// A new buffer is zeroed (and its guard filled) on the caller's stream st, so the
+// call's kernels, queued after it on st, see the zeros whatever kind of stream st
+// is (a plain cudaMemset runs on the legacy default stream, which a non-blocking
+// stream is not ordered after).  cudaFree of an outgrown buffer waits for the
+// device, so no queued kernel still reads it.
 template <typename T>
-cudaError_t grow(T *&p, size_t &have, size_t need) {
+cudaError_t grow(T *&p, size_t &have, size_t need, cudaStream_t st) {
     if (need <= have && p) return cudaSuccess;
     if (p) {
         cudaFree(p);
@@ -176,9 +181,9 @@ cudaError_t grow(T *&p, size_t &have, size_t need) {
     size_t n = need < 64 ? 64 : need;
     cudaError_t e = cudaMalloc(reinterpret_cast<void **>(&p), n * sizeof(T) + GUARD_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaMemset(p, 0, n * sizeof(T));
+    e = cudaMemsetAsync(p, 0, n * sizeof(T), st);
     if (e == cudaSuccess && GUARD_BYTES)
-        e = cudaMemset(reinterpret_cast<char *>(p) + n * sizeof(T), GUARD_FILL, GUARD_BYTES);
+        e = cudaMemsetAsync(reinterpret_cast<char *>(p) + n * sizeof(T), GUARD_FILL, GUARD_BYTES, st);
     have = n;
     return e;
 }
@@ -242,20 +247,20 @@ Workspace *get_ws(cudaStream_t st) {
 }
 
 // Control blocks and per-block partials for a batch of rows.
-cudaError_t ws_base(Workspace *w, int64_t rows) {
-    cudaError_t e = grow(w->ctl, w->ctl_n, (size_t)rows);
-    if (e == cudaSuccess) e = grow(w->partials, w->partials_n, (size_t)(rows * partial_stride(rows)));
+cudaError_t ws_base(Workspace *w, int64_t rows, cudaStream_t st) {
+    cudaError_t e = grow(w->ctl, w->ctl_n, (size_t)rows, st);
+    if (e == cudaSuccess) e = grow(w->partials, w->partials_n, (size_t)(rows * partial_stride(rows)), st);
     return e;
 }
 
 // The device sort's buffers.  Its second key buffer is the caller's p output
 // (n floats per row, written only by the p pass after the sort), so the
 // workspace holds one key buffer of the row, not two.
-cudaError_t ws_sort(Workspace *w, int64_t cap) {
-    cudaError_t e = grow(w->keys0, w->keys0_n, (size_t)cap);
-    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256 + 6);   // + give-up/clean-up counts, per-sign varying bits
-    if (e == cudaSuccess) e = grow(w->chunkcnt, w->chunkcnt_n, (size_t)4 * 256 * sort_grid_max());
-    if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, (size_t)sort_record_doubles(cap));
+cudaError_t ws_sort(Workspace *w, int64_t cap, cudaStream_t st) {
+    cudaError_t e = grow(w->keys0, w->keys0_n, (size_t)cap, st);
+    if (e == cudaSuccess) e = grow(w->hist, w->hist_n, 4 * 256 + 6, st);   // + give-up/clean-up counts, per-sign varying bits
+    if (e == cudaSuccess) e = grow(w->chunkcnt, w->chunkcnt_n, (size_t)4 * 256 * sort_grid_max(), st);
+    if (e == cudaSuccess) e = grow(w->tilebuf, w->tilebuf_n, (size_t)sort_record_doubles(cap), st);
     return e;
 }
 
@@ -391,7 +396,7 @@ int check_args(const float *scores, int64_t rows, int64_t n, double k, double t)
 // cooperative kernel walks the rows, each gated by its own control block.
 int full_sort_rows(Workspace *w, const float *r, float *p_out, int64_t rows, int64_t n, double k, double t,
                    int32_t gate, int32_t spin_cap, cudaStream_t st) {
-    LAPSUM_TRY(ws_sort(w, n));
+    LAPSUM_TRY(ws_sort(w, n, st));
     SortArgs A = sort_args(w, r, p_out, n, n, gate, spin_cap, k, t);
     A.rows = rows;
     A.src_stride = n;
@@ -419,11 +424,11 @@ int shard_workspace(struct CUstream_st *stream, int64_t s, int64_t band_cap, Sha
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     Workspace *w = get_ws(st);
     w->rows = 1;
-    LAPSUM_TRY(ws_base(w, 1));
-    LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)std::max<int64_t>(s, 1)));
-    LAPSUM_TRY(grow(w->hist1, w->hist1_n, (size_t)HIST_WORDS));
-    LAPSUM_TRY(grow(w->selcand, w->selcand_n, (size_t)SEL_CAND_WORDS));
-    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)std::max<int64_t>(band_cap, 1)));
+    LAPSUM_TRY(ws_base(w, 1, st));
+    LAPSUM_TRY(grow(w->skeys, w->skeys_n, (size_t)std::max<int64_t>(s, 1), st));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, (size_t)HIST_WORDS, st));
+    LAPSUM_TRY(grow(w->selcand, w->selcand_n, (size_t)SEL_CAND_WORDS, st));
+    LAPSUM_TRY(grow(w->band, w->band_n, (size_t)std::max<int64_t>(band_cap, 1), st));
     *out = ShardWs{w->ctl, w->partials, w->skeys, w->hist1, w->selcand, w->band, (int64_t)w->band_n};
     return LAPSUM_OK;
 }
@@ -482,7 +487,7 @@ static int forward_impl(const float *scores, int64_t rows, int64_t n, double k, 
         path = n >= (int64_t(1) << 20) ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
     if (path == LAPSUM_PATH_BRACKET && rows > 65535) return LAPSUM_ERR_ARG;   // grid.y holds the row
     w->rows = path == LAPSUM_PATH_FULLSORT && n <= rowsolve_capacity() ? 1 : rows;
-    LAPSUM_TRY(ws_base(w, w->rows));
+    LAPSUM_TRY(ws_base(w, w->rows, st));
 
     if (path == LAPSUM_PATH_FULLSORT) {
         if (n <= rowsolve_capacity()) {
@@ -542,11 +547,11 @@ static int forward_impl(const float *scores, int64_t rows, int64_t n, double k, 
     }
     const int64_t band_buf = std::max(band_cap, opt.widen ? P2.band_cap : int64_t(0));
     const size_t R = (size_t)rows;
-    LAPSUM_TRY(grow(w->skeys, w->skeys_n, R * (size_t)s));
-    LAPSUM_TRY(grow(w->hist1, w->hist1_n, R * (size_t)HIST_WORDS));
-    LAPSUM_TRY(grow(w->selcand, w->selcand_n, R * (size_t)SEL_CAND_WORDS));
-    LAPSUM_TRY(grow(w->band, w->band_n, R * (size_t)band_buf));
-    LAPSUM_TRY(ws_sort(w, n));   // the fallback may sort a whole row (rows one after another)
+    LAPSUM_TRY(grow(w->skeys, w->skeys_n, R * (size_t)s, st));
+    LAPSUM_TRY(grow(w->hist1, w->hist1_n, R * (size_t)HIST_WORDS, st));
+    LAPSUM_TRY(grow(w->selcand, w->selcand_n, R * (size_t)SEL_CAND_WORDS, st));
+    LAPSUM_TRY(grow(w->band, w->band_n, R * (size_t)band_buf, st));
+    LAPSUM_TRY(ws_sort(w, n, st));   // the fallback may sort a whole row (rows one after another)
 
     P2.band = P.band = w->band;
     P2.keys = P.keys = w->skeys;
@@ -624,7 +629,7 @@ int lapsum_backward(const float *scores, const double *b, const float *g, int64_
     }
     // long rows: the streaming passes, the rows of a batch sharing the grid
     Workspace *w = get_ws(st);
-    LAPSUM_TRY(ws_base(w, rows));
+    LAPSUM_TRY(ws_base(w, rows, st));
     { Launch L("vjp_reduce", st); LAPSUM_TRY(launch_vjp_reduce(scores, b, g, rows, n, t, w->ctl, w->partials, st)); }
     { Launch L("vjp_apply", st); LAPSUM_TRY(launch_vjp_apply(scores, b, g, rows, n, t, w->ctl, grad_out, st)); }
     return w->verify_guards(st);

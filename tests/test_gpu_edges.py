@@ -11,7 +11,9 @@ technical summary sections 2.1-2.2; tolerances as in test_gpu_parity.py):
 * every row of the 1024 x 32768 workload;
 * the plain lapsum_forward entry point on device buffers;
 * a grid-barrier wait of the device-wide sort made to give up at once: the
-  call reports the timeout and the next call is clean.
+  call reports the timeout and the next call is clean;
+* calls on a non-blocking stream whose workspace is new (zeroed on that stream):
+  bit-equal to the same calls on the default stream.
 """
 import ctypes as C
 import math
@@ -245,3 +247,34 @@ def test_grid_barrier_timeout_is_reported_and_the_next_call_is_clean(L, orc):
         bref = orc.solve(r[0], k, t, method=1)
         assert abs(float(b[0]) - bref) <= TOL_B * t
         assert np.max(np.abs(p.cpu().numpy()[0].astype(np.float64) - orc.p(r[0], bref, t))) <= TOL_P
+
+
+# ------------------------------------ a new workspace on a non-blocking stream --
+def test_new_workspace_on_a_nonblocking_stream_matches_the_default_stream(L):
+    # The workspace of a (device, stream) pair is allocated and zeroed on the
+    # first call on that stream; the zeros (the sampler's select histograms, the
+    # device sort's digit histograms, the tickets) must be ordered before the
+    # call's kernels on a stream that does not wait for the legacy default stream.
+    cases = [("normal", 4096, 64.0, 0.05, None),                                   # one-CTA row solve
+             ("normal", 1 << 20, 1000.0, 0.05, None),                              # bracketing + streaming VJP
+             ("laplace", 1 << 20, 3000.0, 0.02, L.options(force_path=L.PATH_FULLSORT))]   # device sort
+    data = []
+    for seed, (dist, n, k, t, opts) in enumerate(cases):
+        r_np, g_np = W.small_case(dist, 1, n, seed=40 + seed)
+        r, g = torch.from_numpy(r_np).cuda(), torch.from_numpy(g_np).cuda()
+        p, b = L.forward(r, k, t, opts=opts)
+        grad = L.backward(r, b, g, t)
+        data.append((r, g, k, t, opts, p.clone(), b.clone(), grad.clone()))
+    torch.cuda.synchronize()
+    L.release()   # every workspace of this device: the calls below grow new ones
+    s = torch.cuda.Stream()   # PyTorch's pool streams are non-blocking
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        outs = []
+        for r, g, k, t, opts, _, _, _ in data:
+            p, b = L.forward(r, k, t, opts=opts)
+            outs.append((p, b, L.backward(r, b, g, t)))
+    s.synchronize()
+    for (_, _, _, _, _, p0, b0, g0), (p, b, grad) in zip(data, outs):
+        assert torch.equal(b, b0) and torch.equal(p, p0) and torch.equal(grad, g0)
+    torch.cuda.synchronize()
