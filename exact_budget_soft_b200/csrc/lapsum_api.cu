@@ -392,6 +392,22 @@ int check_args(const float *scores, int64_t rows, int64_t n, double k, double t)
     return LAPSUM_OK;
 }
 
+// The options a forward accepts for `rows` rows of n scores (opt null: the
+// defaults), and the solver path they select.
+int check_options(const lapsum_options &opt, int64_t rows, int64_t n, int *path_out) {
+    if (opt.delta != 0.0 && !(opt.delta > 0.0 && opt.delta < 1.0)) return LAPSUM_ERR_ARG;
+    if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < -1) return LAPSUM_ERR_ARG;
+    if (opt.force_path < 0 || opt.force_path > 2) return LAPSUM_ERR_ARG;
+    if (opt.certify != LAPSUM_CERTIFY_PASS && opt.certify != LAPSUM_CERTIFY_FUSED) return LAPSUM_ERR_ARG;
+    if (opt.widen != 0 && opt.widen != 1) return LAPSUM_ERR_ARG;
+    int path = opt.force_path;
+    if (path == LAPSUM_PATH_AUTO)   // long rows bracket, one or many (a batch shares the kernels)
+        path = n >= (int64_t(1) << 20) ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
+    if (path == LAPSUM_PATH_BRACKET && rows > 65535) return LAPSUM_ERR_ARG;   // grid.y holds the row
+    if (path_out) *path_out = path;
+    return LAPSUM_OK;
+}
+
 // Full sort of long rows on the device (also the certification fallback): one
 // cooperative kernel walks the rows, each gated by its own control block.
 int full_sort_rows(Workspace *w, const float *r, float *p_out, int64_t rows, int64_t n, double k, double t,
@@ -472,20 +488,13 @@ static int forward_impl(const float *scores, int64_t rows, int64_t n, double k, 
     if (!p_out || !b_out) return LAPSUM_ERR_ARG;
     lapsum_options opt{};
     if (opt_in) opt = *opt_in;
-    if (opt.delta != 0.0 && !(opt.delta > 0.0 && opt.delta < 1.0)) return LAPSUM_ERR_ARG;
-    if (opt.sample_size < 0 || opt.band_cap < 0 || opt.spin_cap < -1) return LAPSUM_ERR_ARG;
-    if (opt.force_path < 0 || opt.force_path > 2) return LAPSUM_ERR_ARG;
-    if (opt.certify != LAPSUM_CERTIFY_PASS && opt.certify != LAPSUM_CERTIFY_FUSED) return LAPSUM_ERR_ARG;
-    if (opt.widen != 0 && opt.widen != 1) return LAPSUM_ERR_ARG;
+    int path = LAPSUM_PATH_AUTO;
+    rc = check_options(opt, rows, n, &path);
+    if (rc) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
     // spin_cap -1: grid-barrier waits give up at their first poll (exercises the timeout path)
     const int32_t spin_cap = opt.spin_cap > 0 ? opt.spin_cap : (opt.spin_cap == 0 ? (1 << 20) : 0);
     Workspace *w = get_ws(st);
-
-    int path = opt.force_path;
-    if (path == LAPSUM_PATH_AUTO)   // long rows bracket, one or many (a batch shares the kernels)
-        path = n >= (int64_t(1) << 20) ? LAPSUM_PATH_BRACKET : LAPSUM_PATH_FULLSORT;
-    if (path == LAPSUM_PATH_BRACKET && rows > 65535) return LAPSUM_ERR_ARG;   // grid.y holds the row
     w->rows = path == LAPSUM_PATH_FULLSORT && n <= rowsolve_capacity() ? 1 : rows;
     LAPSUM_TRY(ws_base(w, w->rows, st));
 
@@ -677,8 +686,14 @@ int lapsum_step_host(const float *scores_h, const float *g_h, int64_t rows, int6
                      float *p_h, double *b_h, float *grad_h, const lapsum_options *opt, float *scores_dev,
                      float *g_dev, float *p_dev, double *b_dev, float *grad_dev, struct CUstream_st *stream_in) {
     if (!scores_h || !g_h || !p_h || !b_h || !grad_h || !g_dev || !p_dev || !b_dev || !grad_dev) return LAPSUM_ERR_ARG;
-    const int rc0 = check_args(scores_dev, rows, n, k, t);
-    if (rc0 != LAPSUM_OK) return rc0;
+    int rc = check_args(scores_dev, rows, n, k, t);
+    if (rc != LAPSUM_OK) return rc;
+    {
+        lapsum_options o{};
+        if (opt) o = *opt;
+        rc = check_options(o, rows, n, nullptr);
+        if (rc != LAPSUM_OK) return rc;
+    }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_in);
     const size_t bytes = (size_t)rows * (size_t)n * sizeof(float);
     SideStreams ss;
@@ -692,15 +707,22 @@ int lapsum_step_host(const float *scores_h, const float *g_h, int64_t rows, int6
     LAPSUM_TRY(cudaMemcpyAsync(g_dev, g_h, bytes, cudaMemcpyHostToDevice, ss.h2d));
     LAPSUM_TRY(cudaEventRecord(ev.e[2], ss.h2d));
     LAPSUM_TRY(cudaStreamWaitEvent(st, ev.e[1], 0));
-    int rc = lapsum_forward_ex(scores_dev, rows, n, k, t, p_dev, b_dev, opt, stream_in);
-    if (rc != LAPSUM_OK) return rc;
+    // a call that fails past this point still leaves `stream` waiting for every
+    // copy it queued, so the caller may reuse the buffers once the stream is done
+    auto fail = [&](int code) {
+        cudaStreamWaitEvent(st, ev.e[2], 0);
+        if (cudaEventRecord(ev.e[5], ss.d2h) == cudaSuccess) cudaStreamWaitEvent(st, ev.e[5], 0);
+        return code;
+    };
+    rc = lapsum_forward_ex(scores_dev, rows, n, k, t, p_dev, b_dev, opt, stream_in);
+    if (rc != LAPSUM_OK) return fail(rc);
     LAPSUM_TRY(cudaEventRecord(ev.e[3], st));
     LAPSUM_TRY(cudaStreamWaitEvent(ss.d2h, ev.e[3], 0));   // p and b leave while g arrives
     LAPSUM_TRY(cudaMemcpyAsync(p_h, p_dev, bytes, cudaMemcpyDeviceToHost, ss.d2h));
     LAPSUM_TRY(cudaMemcpyAsync(b_h, b_dev, (size_t)rows * sizeof(double), cudaMemcpyDeviceToHost, ss.d2h));
     LAPSUM_TRY(cudaStreamWaitEvent(st, ev.e[2], 0));
     rc = lapsum_backward(scores_dev, b_dev, g_dev, rows, n, t, grad_dev, stream_in);
-    if (rc != LAPSUM_OK) return rc;
+    if (rc != LAPSUM_OK) return fail(rc);
     LAPSUM_TRY(cudaEventRecord(ev.e[4], st));
     LAPSUM_TRY(cudaStreamWaitEvent(ss.d2h, ev.e[4], 0));
     LAPSUM_TRY(cudaMemcpyAsync(grad_h, grad_dev, bytes, cudaMemcpyDeviceToHost, ss.d2h));

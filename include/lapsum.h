@@ -209,9 +209,12 @@ LAPSUM_API int lapsum_backward(const float *scores_dev, const double *b_dev, con
  * against `stream` by events): the call returns at once, and the host buffers
  * hold the results once `stream` has been synchronised; until then they must
  * stay valid and untouched.
- * Returns: LAPSUM_ERR_ARG for a null pointer or the forward's argument errors
- * (checked before anything is enqueued), LAPSUM_ERR_CUDA if a copy, stream or
- * event call fails, else the forward's and backward's own codes.
+ * Returns: LAPSUM_ERR_ARG for a null pointer or the forward's argument and
+ * option errors (all checked before anything is enqueued), LAPSUM_ERR_CUDA if a
+ * copy, stream or event call fails, else the forward's and backward's own
+ * codes; a forward or backward that fails once the copies are queued still
+ * leaves `stream` waiting for every copy queued, so the buffers may be reused
+ * once `stream` has been synchronised.
  */
 LAPSUM_API int lapsum_step_host(const float *scores_h, const float *g_h, int64_t rows, int64_t n, double k,
                                 double t, float *p_h, double *b_h, float *grad_h, const lapsum_options *opt,

@@ -101,7 +101,28 @@ def test_step_host_rejects_bad_sizes(lib, rows, n, k, t):
 class Options(C.Structure):
     _fields_ = [("seed", C.c_uint64), ("sample_size", C.c_int64), ("delta", C.c_double),
                 ("band_cap", C.c_int64), ("spin_cap", C.c_int32), ("force_path", C.c_int32),
-                ("certify", C.c_int32), ("reserved", C.c_int32 * 3)]
+                ("certify", C.c_int32), ("widen", C.c_int32), ("reserved", C.c_int32 * 2)]
+
+
+@pytest.mark.parametrize("field,value", [("force_path", 7), ("certify", 2), ("widen", 2), ("delta", 1.5),
+                                         ("sample_size", -1), ("band_cap", -5), ("spin_cap", -2)])
+def test_step_host_rejects_bad_options_before_enqueueing(lib, field, value):
+    # an invalid option is refused before any copy is queued (the pointers are
+    # never dereferenced, and no device is needed to get the answer)
+    lib.lapsum_step_host.argtypes = STEP_HOST_ARGS
+    f = C.c_void_p(0x1000)
+    o = Options()
+    setattr(o, field, value)
+    assert lib.lapsum_step_host(f, f, 1, 10, 2.0, 1.0, f, f, f, C.byref(o), f, f, f, f, f, None) == -1
+
+
+def test_step_host_rejects_a_batch_too_tall_for_the_bracketing_grid(lib):
+    lib.lapsum_step_host.argtypes = STEP_HOST_ARGS
+    f = C.c_void_p(0x1000)
+    o = Options()
+    o.force_path = 2   # bracketing: one grid slice per row, at most 65535 rows
+    assert lib.lapsum_step_host(f, f, 65536, 16, 2.0, 1.0, f, f, f, C.byref(o), f, f, f, f, f, None) == -1
+
 
 
 def _plan(lib, n, k, s=0, delta=0.0):
