@@ -15,6 +15,7 @@ unique threshold with sum_i p_i = k; grad = (f/t)(g - <g,f>/sum f).
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes as C
 import os
 
@@ -125,6 +126,14 @@ def _stream(stream) -> int:
     return stream.cuda_stream
 
 
+def _on(dev: torch.device):
+    """The library works on the current device: make it the tensors' device for
+    the call (no switch, and no cost beyond one query, when it already is)."""
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
+
+
 def _check(rc: int, where: str):
     if rc != 0:
         raise LapSumError(rc, where)
@@ -138,11 +147,19 @@ def _as_rows(x: torch.Tensor) -> tuple[int, int]:
     raise ValueError("scores must be [n] or [rows, n]")
 
 
-def _need(x: torch.Tensor, name: str, dtype=torch.float32):
+def _need(x: torch.Tensor, name: str, dtype=torch.float32, numel: int | None = None,
+          device: torch.device | None = None):
+    """A contiguous CUDA tensor of `dtype` (of `numel` values and on `device` when
+    given): the library writes and reads exactly that many, so a short buffer is
+    refused here rather than overrun on the device."""
     if not x.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
     if x.dtype != dtype or not x.is_contiguous():
         raise ValueError(f"{name} must be contiguous {dtype}")
+    if numel is not None and x.numel() != numel:
+        raise ValueError(f"{name} must hold {numel} values, not {x.numel()}")
+    if device is not None and x.device != device:
+        raise ValueError(f"{name} is on {x.device}, the scores on {device}")
 
 
 def options(seed: int = 0, sample_size: int = 0, delta: float = 0.0, band_cap: int = 0,
@@ -160,33 +177,38 @@ def forward(scores: torch.Tensor, k: float, t: float, p_out: torch.Tensor | None
     """p (float32, like scores) and b (float64 [rows]) of lapsum_forward_ex."""
     _need(scores, "scores")
     rows, n = _as_rows(scores)
+    dev = scores.device
     if p_out is None:
         p_out = torch.empty_like(scores)
     if b_out is None:
-        b_out = torch.empty(rows, dtype=torch.float64, device=scores.device)
-    _need(p_out, "p_out")
-    _need(b_out, "b_out", torch.float64)
-    rc = lib.lapsum_forward_ex(scores.data_ptr(), rows, n, float(k), float(t), p_out.data_ptr(),
-                               b_out.data_ptr(), C.byref(opts) if opts is not None else None,
-                               _stream(stream))
-    _check(rc, "lapsum_forward")
-    if CHECKED:   # the checked build reports an out-of-bounds index through the device status
-        st = Stats()
-        if lib.lapsum_get_stats(C.byref(st), _stream(stream)) == ERR_BOUNDS:
-            raise LapSumError(ERR_BOUNDS, "lapsum_forward")
+        b_out = torch.empty(rows, dtype=torch.float64, device=dev)
+    _need(p_out, "p_out", numel=rows * n, device=dev)
+    _need(b_out, "b_out", torch.float64, numel=rows, device=dev)
+    with _on(dev):
+        rc = lib.lapsum_forward_ex(scores.data_ptr(), rows, n, float(k), float(t), p_out.data_ptr(),
+                                   b_out.data_ptr(), C.byref(opts) if opts is not None else None,
+                                   _stream(stream))
+        _check(rc, "lapsum_forward")
+        if CHECKED:   # the checked build reports an out-of-bounds index through the device status
+            st = Stats()
+            if lib.lapsum_get_stats(C.byref(st), _stream(stream)) == ERR_BOUNDS:
+                raise LapSumError(ERR_BOUNDS, "lapsum_forward")
     return p_out, b_out
 
 
 def backward(scores: torch.Tensor, b: torch.Tensor, g: torch.Tensor, t: float,
              grad_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     _need(scores, "scores")
-    _need(g, "g")
-    _need(b, "b", torch.float64)
     rows, n = _as_rows(scores)
+    dev = scores.device
+    _need(g, "g", numel=rows * n, device=dev)
+    _need(b, "b", torch.float64, numel=rows, device=dev)
     if grad_out is None:
         grad_out = torch.empty_like(scores)
-    rc = lib.lapsum_backward(scores.data_ptr(), b.data_ptr(), g.data_ptr(), rows, n, float(t),
-                             grad_out.data_ptr(), _stream(stream))
+    _need(grad_out, "grad_out", numel=rows * n, device=dev)
+    with _on(dev):
+        rc = lib.lapsum_backward(scores.data_ptr(), b.data_ptr(), g.data_ptr(), rows, n, float(t),
+                                 grad_out.data_ptr(), _stream(stream))
     _check(rc, "lapsum_backward")
     return grad_out
 
@@ -263,11 +285,12 @@ def profile_read() -> dict:
 
 def forward_host(scores_host: torch.Tensor, k: float, t: float, device="cuda", opts=None,
                  stream=None) -> tuple[torch.Tensor, torch.Tensor]:
-    """End-to-end call on host tensors: copy in, solve on the GPU, copy p and b back."""
-    rows, n = _as_rows(scores_host)
-    d = scores_host.to(device, non_blocking=True)
-    p, b = forward(d, k, t, opts=opts, stream=stream)
-    return p.to("cpu", non_blocking=False), b.to("cpu", non_blocking=False)
+    """End-to-end call on host tensors: copy in, solve on the GPU, copy p and b back
+    (the copies and the solve all on `stream`, default the current stream)."""
+    with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+        d = scores_host.to(device, non_blocking=True)
+        p, b = forward(d, k, t, opts=opts)
+        return p.to("cpu", non_blocking=False), b.to("cpu", non_blocking=False)
 
 
 def step_host(scores_h: torch.Tensor, g_h: torch.Tensor, k: float, t: float, p_h: torch.Tensor,
@@ -288,17 +311,19 @@ def step_host(scores_h: torch.Tensor, g_h: torch.Tensor, k: float, t: float, p_h
     for x, name, dt in ((scores_d, "scores_d", torch.float32), (g_d, "g_d", torch.float32),
                         (p_d, "p_d", torch.float32), (b_d, "b_d", torch.float64),
                         (grad_d, "grad_d", torch.float32)):
-        _need(x, name, dt)
+        _need(x, name, dt, device=scores_d.device)
     for x, name in ((g_h, "g_h"), (p_h, "p_h"), (grad_h, "grad_h"), (scores_d, "scores_d"), (g_d, "g_d"),
                     (p_d, "p_d"), (grad_d, "grad_d")):
         if x.numel() != rows * n:
             raise ValueError(f"{name} must hold rows x n = {rows} x {n} values")
     if b_h.numel() != rows or b_d.numel() != rows:
         raise ValueError("b_h and b_d must hold one threshold per row")
-    rc = lib.lapsum_step_host(scores_h.data_ptr(), g_h.data_ptr(), rows, n, float(k), float(t), p_h.data_ptr(),
-                              b_h.data_ptr(), grad_h.data_ptr(), C.byref(opts) if opts is not None else None,
-                              scores_d.data_ptr(), g_d.data_ptr(), p_d.data_ptr(), b_d.data_ptr(),
-                              grad_d.data_ptr(), _stream(stream))
+    with _on(scores_d.device):
+        rc = lib.lapsum_step_host(scores_h.data_ptr(), g_h.data_ptr(), rows, n, float(k), float(t),
+                                  p_h.data_ptr(), b_h.data_ptr(), grad_h.data_ptr(),
+                                  C.byref(opts) if opts is not None else None, scores_d.data_ptr(),
+                                  g_d.data_ptr(), p_d.data_ptr(), b_d.data_ptr(), grad_d.data_ptr(),
+                                  _stream(stream))
     _check(rc, "lapsum_step_host")
 
 

@@ -13,7 +13,9 @@ technical summary sections 2.1-2.2; tolerances as in test_gpu_parity.py):
 * a grid-barrier wait of the device-wide sort made to give up at once: the
   call reports the timeout and the next call is clean;
 * calls on a non-blocking stream whose workspace is new (zeroed on that stream):
-  bit-equal to the same calls on the default stream.
+  bit-equal to the same calls on the default stream;
+* the binding refusing output and input buffers of the wrong size before any
+  launch.
 """
 import ctypes as C
 import math
@@ -278,3 +280,31 @@ def test_new_workspace_on_a_nonblocking_stream_matches_the_default_stream(L):
     for (_, _, _, _, _, p0, b0, g0), (p, b, grad) in zip(data, outs):
         assert torch.equal(b, b0) and torch.equal(p, p0) and torch.equal(grad, g0)
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------- buffers of the wrong size --
+def test_binding_refuses_buffers_of_the_wrong_size(L):
+    # the library writes and reads exactly rows x n values (rows thresholds): a
+    # buffer of another size is refused by the binding, before anything runs
+    rows, n = 2, 4096
+    r = torch.randn(rows, n, device="cuda")
+    g = torch.randn(rows, n, device="cuda")
+    short = torch.empty(rows * n - 1, device="cuda")
+    n0 = L.launch_count()
+    with pytest.raises(ValueError):
+        L.forward(r, 64.0, 0.1, p_out=short)
+    with pytest.raises(ValueError):
+        L.forward(r, 64.0, 0.1, b_out=torch.empty(rows - 1, dtype=torch.float64, device="cuda"))
+    assert L.launch_count() == n0
+    p, b = L.forward(r, 64.0, 0.1)
+    n1 = L.launch_count()
+    with pytest.raises(ValueError):
+        L.backward(r, b, short, 0.1)
+    with pytest.raises(ValueError):
+        L.backward(r, b, g, 0.1, grad_out=short)
+    with pytest.raises(ValueError):
+        L.backward(r, b[:1], g, 0.1)
+    assert L.launch_count() == n1
+    grad = L.backward(r, b, g, 0.1)
+    torch.cuda.synchronize()
+    assert torch.isfinite(grad).all() and torch.isfinite(p).all()

@@ -61,3 +61,17 @@ def test_step_host_grad_may_overwrite_g_on_the_device(L):
     r2, g2 = torch.from_numpy(r).cuda(), torch.from_numpy(g).cuda()
     p2, b2 = L.forward(r2, k, t)
     assert torch.equal(grh, L.backward(r2, b2, g2, t).cpu())
+
+
+@pytest.mark.parametrize("on_side_stream", [False, True])
+def test_forward_host_equals_the_device_call(L, on_side_stream):
+    # forward_host: the copy in, the solve and the copies out all on one stream
+    r, _ = W.small_case("normal", 1, 1 << 20, seed=67)
+    p0, b0 = L.forward(torch.from_numpy(r).cuda(), 1000.0, 0.05)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream() if on_side_stream else None
+    if s is not None:
+        s.wait_stream(torch.cuda.current_stream())
+    p, b = L.forward_host(host(r, True), 1000.0, 0.05, stream=s)
+    assert not p.is_cuda and not b.is_cuda
+    assert torch.equal(p, p0.cpu()) and torch.equal(b, b0.cpu())
