@@ -50,12 +50,6 @@ __device__ __forceinline__ float desc_key_to_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? k : (k ^ 0x7fffffffu));
 }
 
-// Band of one tied value: its largest and smallest keys agree (the streaming
-// pass keeps the largest key and the largest complemented key of the band).
-__device__ __forceinline__ bool band_tied(const Ctl *c) {
-    return c->c_band > 0 && (c->band_kmax ^ c->band_kinv) == 0xffffffffu;
-}
-
 // Folds a CTA's band-key maxima (per thread; 0 for none) into those two words:
 // one shared and one global atomic per CTA.  Every thread of the CTA calls it.
 __device__ __forceinline__ void band_range_flush(Ctl *c, uint32_t kmax, uint32_t kinv, uint32_t *s_two) {
@@ -74,15 +68,6 @@ __device__ __forceinline__ void band_range_flush(Ctl *c, uint32_t kmax, uint32_t
     }
 }
 
-// ------------------------------------------------------------ exp tiers --
-// e^{-z}, z >= 0.  Terms that can move G by more than ~1e-7 relative to one
-// unit (z <= 16) are formed in fp64; farther terms (< 1.2e-7 each) in fp32,
-// whose error is then below ~1.4e-14 absolute per term.
-constexpr double EXP_TIER = 16.0;
-__device__ __forceinline__ double exp_neg_tiered(double z) {
-    return z <= EXP_TIER ? exp(-z) : (double)expf(-(float)z);
-}
-
 // ------------------------------------------------------- affine maps --
 struct Aff {
     double a, s;   // x -> a x + s
@@ -95,9 +80,6 @@ __device__ __forceinline__ Aff shfl_up_aff(Aff v, int o) {
 }
 __device__ __forceinline__ Aff shfl_down_aff(Aff v, int o) {
     return {__shfl_down_sync(FULL, v.a, o), __shfl_down_sync(FULL, v.s, o)};
-}
-__device__ __forceinline__ Aff shfl_aff(Aff v, int src) {
-    return {__shfl_sync(FULL, v.a, src), __shfl_sync(FULL, v.s, src)};
 }
 // Inclusive warp scan in lane order: lane l gets map_0 then ... then map_l.
 __device__ __forceinline__ Aff warp_scan_fwd(Aff v, int lane) {
@@ -158,11 +140,6 @@ __device__ __forceinline__ void block_scan_excl_both(Aff fwd, Aff bwd, Aff &fwd_
 
 // ------------------------------------------------------- reductions --
 __device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-    return v;
-}
-__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
     return v;
@@ -243,12 +220,6 @@ __device__ __forceinline__ double solve_equal_run_values(double c, double nn, do
     }
     *above_run = false;
     return solve_interval(top, c, m0, P_top, nn + d_bot * Q_bot, d_top, k, t);
-}
-
-// Laplace CDF of an fp32 argument, F(x) = e^x/2 (x < 0), 1 - e^{-x}/2 (x >= 0).
-__device__ __forceinline__ float laplace_cdf_f(float x) {
-    float e = 0.5f * expf(-fabsf(x));
-    return x < 0.0f ? e : 1.0f - e;
 }
 
 // ----------------------------------------------- fp32 elementwise math --
@@ -531,14 +502,6 @@ __device__ __forceinline__ void pdl_enter() {
 }
 
 // ------------------------------------------------ bounded device waits --
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -589,17 +552,6 @@ __device__ __forceinline__ bool grid_sync(unsigned *count, unsigned *gen, int ca
     }
     __syncthreads();
     return s_gave_up == 0;
-}
-
-// Relaxed (but coherent at GPU scope) 64-bit accesses, for words that carry their
-// own flag and value and guard no other data.
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 }  // namespace lapsum

@@ -1,4 +1,4 @@
-// scan_solve.cuh -- in-CTA radix sort and the threshold-curve scan/solve
+// scan_solve.cuh -- in-CTA merge sort and the threshold-curve scan/solve
 // (full-sort solver of "Fast LapSum: Exact Differentiable Top-k at Million
 // Scale", technical summary section 2.2), shared by the one-CTA row solver and
 // the last CTA of the device-wide locate kernel.
@@ -14,17 +14,6 @@ namespace lapsum {
 // neighbours (the scan reads runs; unpadded, all 32 lanes would share a bank).
 __device__ __forceinline__ int spad(int j) { return j + (j >> 5); }
 
-// Lanes of the warp holding the same 8-bit digit: eight ballots, one per bit.
-__device__ __forceinline__ unsigned digit_peers(uint32_t d) {
-    unsigned peers = FULL;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-        const unsigned m = __ballot_sync(FULL, (d >> b) & 1u);
-        peers &= ((d >> b) & 1u) ? m : ~m;
-    }
-    return peers;
-}
-
 template <int BLOCK, int KPT>
 struct RowCfg {
     static constexpr int NW = BLOCK / 32;
@@ -34,83 +23,6 @@ struct RowCfg {
     static constexpr size_t SMEM_HIST = size_t(NW) * 256 * 4;
     static constexpr size_t SMEM = SMEM_KEYS + SMEM_HIST + 256 * 4 + 2048;
 };
-
-// Block-wide LSD radix sort of warp-striped register keys (ascending).  On
-// return the sorted keys are in s_keys (position j at spad(j)).
-template <int BLOCK, int KPT>
-__device__ __forceinline__ void block_radix_sort(uint32_t (&key)[KPT], uint32_t *s_keys,
-                                                 uint32_t *s_hist, uint32_t *s_dbase,
-                                                 uint32_t diff) {
-    using C = RowCfg<BLOCK, KPT>;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    uint32_t *my_hist = s_hist + warp * 256;
-    bool sorted_in_smem = false;
-#pragma unroll 1
-    for (int sh = 0; sh < 32; sh += 8) {
-        if (((diff >> sh) & 0xffu) == 0u) continue;   // every key has this digit
-        for (int i = tid; i < C::NW * 256; i += BLOCK) s_hist[i] = 0;
-        __syncthreads();
-        // count: per-warp digit histograms.  Counts need no order: one shared
-        // atomic per key (lanes on one counter serialise, the rest run in
-        // parallel).
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) atomicAdd(&my_hist[(key[i] >> sh) & 0xffu], 1u);
-        __syncthreads();
-        if (tid < 256) {   // per digit: exclusive prefix over warps, and total
-            uint32_t sum = 0;
-            for (int w = 0; w < C::NW; ++w) {
-                uint32_t c = s_hist[w * 256 + tid];
-                s_hist[w * 256 + tid] = sum;
-                sum += c;
-            }
-            s_dbase[tid] = sum;
-        }
-        __syncthreads();
-        if (warp == 0) {   // exclusive scan of the 256 digit totals
-            uint32_t v[8], run = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { v[j] = s_dbase[lane * 8 + j]; run += v[j]; }
-            uint32_t inc = run;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                uint32_t p = __shfl_up_sync(FULL, inc, o);
-                if (lane >= o) inc += p;
-            }
-            uint32_t ex = inc - run;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { uint32_t c = v[j]; s_dbase[lane * 8 + j] = ex; ex += c; }
-        }
-        __syncthreads();
-        for (int i = tid; i < C::NW * 256; i += BLOCK) s_hist[i] += s_dbase[i & 255];
-        __syncthreads();
-        // scatter: the same traversal again hands out consecutive slots (stable)
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const uint32_t d = (key[i] >> sh) & 0xffu;
-            const unsigned peers = digit_peers(d);
-            const int leader = __ffs(peers) - 1;
-            uint32_t base = 0;
-            if (lane == leader) {
-                base = my_hist[d];
-                my_hist[d] = base + __popc(peers);
-            }
-            base = __shfl_sync(FULL, base, leader) + __popc(peers & lt_mask);
-            if (in_bounds(base < (uint32_t)C::CAP, nullptr)) s_keys[spad((int)base)] = key[i];
-            __syncwarp();
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) key[i] = s_keys[spad(warp * C::SEG + i * 32 + lane)];
-        sorted_in_smem = true;
-        __syncthreads();
-    }
-    if (!sorted_in_smem) {   // all keys identical: any order is sorted
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) s_keys[spad(warp * C::SEG + i * 32 + lane)] = key[i];
-        __syncthreads();
-    }
-}
 
 // Ascending sorting network on N keys in registers (bitonic: log2 N (log2 N + 1)/2
 // stages of N/2 compare-exchanges; every index is a compile-time constant).
