@@ -232,18 +232,3 @@ def certify(r, k: float, t: float, a_L: float, a_R: float, band_cap: int) -> dic
                             C.byref(gl), C.byref(gr), C.byref(cl), C.byref(cb), C.byref(cr))
     return {"verdict": int(v), "G_aL": gl.value, "G_aR": gr.value,
             "c_L": cl.value, "c_band": cb.value, "c_R": cr.value}
-
-
-def forward(r, k: float, t: float, method: int = 0) -> tuple[np.ndarray, np.ndarray]:
-    """(p [rows,n] fp64, b [rows] fp64) for a [rows, n] score matrix."""
-    r2 = np.atleast_2d(np.asarray(r, dtype=np.float32))
-    b = solve_rows(r2, k, t, method)
-    pp = np.stack([p(row, bb, t) for row, bb in zip(r2, b)])
-    return pp, b
-
-
-def backward(r, g, b, t: float) -> np.ndarray:
-    r2 = np.atleast_2d(np.asarray(r, dtype=np.float32))
-    g2 = np.atleast_2d(np.asarray(g, dtype=np.float32))
-    b = np.atleast_1d(np.asarray(b, dtype=np.float64))
-    return np.stack([vjp(rr, gg, bb, t)[0] for rr, gg, bb in zip(r2, g2, b)])

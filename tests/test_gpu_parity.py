@@ -7,7 +7,6 @@ Differentiable Top-k at Million Scale", technical summary section 2.1):
 Integer results of the bracketing path (ranks, bracket ends, membership
 counts, certification verdict) must equal the oracle's restatement exactly.
 """
-import math
 
 import numpy as np
 import pytest

@@ -4,7 +4,6 @@ draw different replica inputs.  The solver's data path has no collective."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
