@@ -211,7 +211,7 @@ def _check(orc, res, case, want_verdict, flat=False):
     return r, k, t, opts, res[0][6]
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_sharded_row_matches_the_whole_row(orc, world):
     res = _run(world, case_normal)
     r, k, t, _, (aL, aR, jR, jL) = _check(orc, res, case_normal, 1)
@@ -223,8 +223,9 @@ def test_sharded_row_matches_the_whole_row(orc, world):
     assert res[0][5]["band"] == cert["c_band"]
 
 
-def test_sharded_row_falls_back_over_the_gathered_row(orc):
-    res = _run(2, case_fallback)
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_row_falls_back_over_the_gathered_row(orc, world):
+    res = _run(world, case_fallback)
     _check(orc, res, case_fallback, 0)
     assert all(x[5]["fallback"] == 1 for x in res)
 
