@@ -161,3 +161,64 @@ def test_bracket_plan_ranks_fuzz(lib, orc):
         n = 10 ** 9
         _, jR, jL, _ = _plan(lib, n, pi * n, s, delta)
         assert (jR, jL) == orc.binom_ranks(s, pi, delta)
+
+
+FWD_EX_ARGS = [C.c_void_p, C.c_int64, C.c_int64, C.c_double, C.c_double, C.c_void_p, C.c_void_p, C.c_void_p,
+               C.c_void_p]
+
+
+@pytest.mark.parametrize("field,value", [("force_path", 3), ("certify", 2), ("widen", 2), ("delta", 1.0),
+                                         ("delta", -0.1), ("sample_size", -1), ("band_cap", -1),
+                                         ("spin_cap", -2)])
+def test_forward_rejects_bad_options_on_host(lib, field, value):
+    lib.lapsum_forward_ex.argtypes = FWD_EX_ARGS
+    f = C.c_void_p(0x1000)   # never dereferenced: the options are checked first
+    o = Options()
+    setattr(o, field, value)
+    assert lib.lapsum_forward_ex(f, 1, 10, 2.0, 1.0, f, f, C.byref(o), None) == -1
+
+
+def test_forward_rejects_a_batch_too_tall_for_the_bracketing_grid(lib):
+    lib.lapsum_forward_ex.argtypes = FWD_EX_ARGS
+    f = C.c_void_p(0x1000)
+    assert lib.lapsum_forward_ex(f, 65536, 1 << 20, 1000.0, 0.1, f, f, None, None) == -1   # auto: bracketing
+
+
+SHARD_SAMPLE_ARGS = [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_double, C.c_double, C.c_void_p,
+                     C.c_void_p, C.c_void_p]
+SHARD_STREAM_ARGS = [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_double, C.c_double, C.c_void_p,
+                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+
+
+@pytest.mark.parametrize("n_local,offset,n_total,field,value",
+                         [(10, -1, 100, None, 0),           # a slice before the row
+                          (60, 50, 100, None, 0),           # a slice past the row's end
+                          (0, 0, 100, None, 0),             # an empty slice
+                          (1, 0, 1, None, 0),               # a row of one score
+                          (10, 0, 100, "widen", 1),         # no widening round on a split row
+                          (10, 0, 100, "force_path", 1)])   # nor the full-sort path
+def test_split_row_calls_reject_bad_slices_on_host(lib, n_local, offset, n_total, field, value):
+    lib.lapsum_shard_sample.argtypes = SHARD_SAMPLE_ARGS
+    lib.lapsum_shard_stream.argtypes = SHARD_STREAM_ARGS
+    f = C.c_void_p(0x1000)
+    o = Options()
+    if field:
+        setattr(o, field, value)
+    assert lib.lapsum_shard_sample(f, n_local, offset, n_total, 2.0 if n_total > 2 else 0.5, 1.0, C.byref(o),
+                                   f, None) == -1
+    assert lib.lapsum_shard_stream(f, n_local, offset, n_total, 2.0 if n_total > 2 else 0.5, 1.0, C.byref(o),
+                                   f, f, f, None) == -1
+
+
+@pytest.mark.parametrize("n_total,k", [(1 << 20, 1000.0), (100_000_000, 1e6), (3_000_000, 0.5)])
+def test_split_row_plan_sizes_the_exchange_buffers(lib, n_total, k):
+    # the sample exchange buffer holds the s sample keys and the select's
+    # histograms (65536 top-16-bit bins + 256 top-8-bit bins); the band capacity
+    # is the one-GPU plan's
+    lib.lapsum_shard_plan.argtypes = [C.c_int64, C.c_double, C.POINTER(Options), C.POINTER(C.c_int64),
+                                      C.POINTER(C.c_int64)]
+    words, cap = C.c_int64(), C.c_int64()
+    assert lib.lapsum_shard_plan(n_total, k, None, C.byref(words), C.byref(cap)) == 0
+    s, _, _, band_cap = _plan(lib, n_total, k)
+    assert words.value == s + 65536 + 256
+    assert cap.value == band_cap
