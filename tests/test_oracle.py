@@ -8,9 +8,11 @@ a limit that the pages state (the zero-temperature limit of section 2.3).
 """
 import math
 
+import hypothesis.strategies as hyp
 import numpy as np
 import pytest
 import scipy.stats as st
+from hypothesis import given, settings
 
 import workloads as W
 
@@ -69,7 +71,10 @@ def test_G_and_p_match_scipy_laplace(orc):
 def brute_force_b(r, k, t):
     """Enumerate the n+1 intervals between sorted scores and solve, in each,
     1/2 S- u^2 + (k - m) u - 1/2 S+ = 0 with u = e^{b/t}, S- = sum_{above} e^{-r/t},
-    S+ = sum_{below} e^{r/t}; keep the root that lies inside its interval."""
+    S+ = sum_{below} e^{r/t}; keep the root that lies inside its interval.  The
+    positive root (A >= 0 >= C) is taken in the form that subtracts nothing:
+    (-B + sqrt(disc)) / 2A for B < 0, and -2C / (B + sqrt(disc)) for B >= 0 (the
+    same number; the first form loses digits to cancellation when 4AC << B^2)."""
     c = sorted((float(v) for v in r), reverse=True)
     n = len(c)
     roots = []
@@ -81,7 +86,7 @@ def brute_force_b(r, k, t):
             u = -Cc / B if B != 0 else None
         else:
             disc = B * B - 4 * A * Cc
-            u = (-B + math.sqrt(disc)) / (2 * A)
+            u = (-B + math.sqrt(disc)) / (2 * A) if B < 0 else -2 * Cc / (B + math.sqrt(disc))
         if u is None or u <= 0:
             continue
         b = t * math.log(u)
@@ -106,6 +111,22 @@ def test_bisection_matches_interval_enumeration(orc, seed):
     b = orc.solve(r, k, t)
     assert min(abs(b - x) for x in roots) <= 1e-10 * t
     assert max(roots) - min(roots) <= 1e-9 * t             # unique root (ties repeat it)
+
+
+@settings(max_examples=300, derandomize=True, deadline=None)
+@given(data=hyp.data())
+def test_bisection_matches_interval_enumeration_on_generated_rows(orc, data):
+    # generated rows on a coarse grid (many ties, up to all equal), budgets from
+    # near 0 to near n, temperatures across an order of magnitude
+    n = data.draw(hyp.integers(1, 12))
+    r = np.array(data.draw(hyp.lists(hyp.integers(-10, 10), min_size=n, max_size=n)), np.float32) * np.float32(0.1)
+    t = data.draw(hyp.floats(0.05, 0.6))
+    k = data.draw(hyp.floats(0.01, n - 0.01)) if n > 1 else data.draw(hyp.floats(0.01, 0.99))
+    roots = brute_force_b(r, k, t)
+    assert roots, "brute force found no root"
+    b = orc.solve(r, k, t)
+    assert min(abs(b - x) for x in roots) <= 1e-10 * t
+    assert max(roots) - min(roots) <= 1e-9 * t
 
 
 def test_newton_and_bisection_agree(orc):
