@@ -176,6 +176,23 @@ def test_translation_scale_permutation_reflection(orc):
     np.testing.assert_allclose(orc.p(-r, br, t), 1 - p, atol=1e-12)
 
 
+@settings(max_examples=100, derandomize=True, deadline=None)
+@given(data=hyp.data())
+def test_invariances_on_generated_rows(orc, data):
+    # generated rows on a 2^-12 grid in (-3, 3) (r + 0.5, 4 r and -r stay exact in
+    # fp32), any budget in (0, n), temperatures from 0.02 to 1
+    n = data.draw(hyp.integers(2, 200))
+    r = (np.array(data.draw(hyp.lists(hyp.integers(-3 * 4096, 3 * 4096), min_size=n, max_size=n)),
+                  np.float64) / 4096).astype(np.float32)
+    k = data.draw(hyp.floats(0.05, n - 0.05))
+    t = data.draw(hyp.floats(0.02, 1.0))
+    b = orc.solve(r, k, t)
+    assert abs(orc.solve(r + np.float32(0.5), k, t) - (b + 0.5)) <= 1e-12 * max(1.0, abs(b))
+    assert abs(orc.solve(r * np.float32(4.0), k, 4 * t) - 4 * b) <= 4e-12 * max(1.0, abs(b))
+    assert abs(orc.solve(-r, n - k, t) + b) <= 1e-12 * max(1.0, abs(b))
+    assert abs(orc.p(r, b, t).sum() - k) <= 1e-9 * max(k, 1.0)
+
+
 # ------------------------------------------- zero-temperature (DFTopK) limit
 @pytest.mark.parametrize("k", [1, 5, 40])
 @pytest.mark.parametrize("ratio", [10.0, 20.0, 30.0])
