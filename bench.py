@@ -190,7 +190,7 @@ def run_ours(args):
     L.profile_filter(None)
     L.profile_enable(2)
     L.profile_enable(1)
-    time_steps(torch, step, 3, 1)
+    time_steps(torch, step, 3, 3)
     L.profile_enable(0)
     calib = L.profile_read()
     per_kernel = {k: {"launches": v[0], "avg_ms": v[1] / max(v[0], 1)} for k, v in calib.items()}
@@ -211,7 +211,7 @@ def run_ours(args):
     launches = (L.launch_count() - l0) // (args.steps + args.warmup)
     prof = L.profile_read()
     L.profile_filter(None)
-    fwd_ms = time_steps(torch, fwd, args.steps, 2)
+    fwd_ms = time_steps(torch, fwd, args.steps, 3)
     med = statistics.median(ms)
     med_f = statistics.median(fwd_ms)
     tot = sum(ms)
@@ -358,7 +358,7 @@ def run_ours(args):
                 L.forward(r, w.k, w.t, p_out=p, b_out=b, opts=of)
                 L.backward(r, b, g, w.t, grad_out=grad)
 
-            msf = time_steps(torch, st_fb, max(5, args.steps // 4), 2)
+            msf = time_steps(torch, st_fb, max(5, args.steps // 4), 3)
             st_fb_stats = L.get_stats()
             assert st_fb_stats["fallback"] == 1 and st_fb_stats["rc"] == 0
             out["forced_fallback"] = {"median_ms_fwd_vjp": round(statistics.median(msf), 4),
@@ -371,7 +371,7 @@ def run_ours(args):
                 L.forward(r, w.k, w.t, p_out=p, b_out=b, opts=ow)
                 L.backward(r, b, g, w.t, grad_out=grad)
 
-            msw = time_steps(torch, st_w, max(5, args.steps // 4), 2)
+            msw = time_steps(torch, st_w, max(5, args.steps // 4), 3)
             sw = L.get_stats()
             assert sw["rc"] == 0 and sw["widened"] == 1
             out["forced_widening"] = {"median_ms_fwd_vjp": round(statistics.median(msw), 4),
