@@ -190,7 +190,7 @@ def run_ours(args):
     L.profile_filter(None)
     L.profile_enable(2)
     L.profile_enable(1)
-    time_steps(torch, step, 3, 3)
+    time_steps(torch, step, 3, 3)   # 6 steps recorded: nsteps below
     L.profile_enable(0)
     calib = L.profile_read()
     per_kernel = {k: {"launches": v[0], "avg_ms": v[1] / max(v[0], 1)} for k, v in calib.items()}
@@ -220,7 +220,7 @@ def run_ours(args):
         med, tot, med_f, dom_ms = max_over_ranks(dist, [med, tot, med_f, dom_ms])
         dist.barrier()
 
-    nsteps = 4   # calibration: 1 warm-up + 3 steps
+    nsteps = 6   # calibration: 3 warm-ups + 3 steps, every launch recorded
     peak, peak_kind = peaks()
     alg_bytes = KERNEL_BYTES[dom] * w.n
     achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
@@ -258,7 +258,7 @@ def run_ours(args):
                      "traffic": traffic, "alg_bytes_per_launch": alg_bytes},
         "kernels": {k: {"launches_per_step": round(v["launches"] / nsteps, 2), "avg_ms": round(v["avg_ms"], 4)}
                     for k, v in per_kernel.items()},
-        "kernels_note": "per-kernel averages from a 4-step calibration run with every launch bracketed by events; "
+        "kernels_note": "per-kernel averages from a 6-step calibration run with every launch bracketed by events; "
                         "the timed region brackets only the roofline kernel",
         "gpu_launches": int(launches) * args.steps,
         "clocks": clk.summary(),
