@@ -28,8 +28,11 @@
  *    library's own workspace.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point synchronises the host except
- *    lapsum_get_stats* / lapsum_profile_read (documented) and the first call on
- *    a stream, which may allocate the workspace with cudaMalloc.
+ *    lapsum_get_stats* / lapsum_profile_read (documented) and a call that
+ *    grows the stream's workspace (the first on a stream, or one needing more
+ *    room): cudaMalloc, and cudaFree of what it replaces, which waits for the
+ *    device.  New workspace is zeroed on `stream` itself, so any stream,
+ *    non-blocking ones included, sees it ready.
  *  - Return value: LAPSUM_OK (0) or a negative LAPSUM_ERR_* code.  Argument
  *    errors are detected on the host before anything is enqueued.  Errors
  *    found on the device (non-finite scores, a grid-barrier wait that gave
