@@ -222,3 +222,39 @@ def test_split_row_plan_sizes_the_exchange_buffers(lib, n_total, k):
     s, _, _, band_cap = _plan(lib, n_total, k)
     assert words.value == s + 65536 + 256
     assert cap.value == band_cap
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "lapsum.h"
+
+int main(void) {
+    lapsum_options o;
+    memset(&o, 0, sizeof o);
+    int64_t s = 0, jR = 0, jL = 0, cap = 0;
+    if (strcmp(lapsum_strerror(LAPSUM_OK), "ok") != 0) return 1;
+    if (lapsum_bracket_plan(100000000, 1e6, &o, &s, &jR, &jL, &cap) != LAPSUM_OK) return 2;
+    if (!(s == 65536 && 0 < jR && jR < jL && jL <= s && cap > 0)) return 3;
+    /* argument errors come back before any device work */
+    if (lapsum_forward(NULL, 1, 10, 2.0, 1.0, NULL, NULL, NULL) != LAPSUM_ERR_ARG) return 4;
+    if (lapsum_backward(NULL, NULL, NULL, 1, 10, 1.0, NULL, NULL) != LAPSUM_ERR_ARG) return 5;
+    printf("%lld %lld %lld %lld\n", (long long)s, (long long)jR, (long long)jL, (long long)cap);
+    return 0;
+}
+"""
+
+
+def test_header_serves_a_plain_c_program(lib, tmp_path):
+    # the boundary is a C ABI: a C11 program compiles against include/lapsum.h
+    # with warnings as errors, links to the library and calls its host-side entry
+    # points; its bracket plan equals the one ctypes sees
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(_lib_path())
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-o", str(exe), "-L", libdir, "-llapsum", f"-Wl,-rpath,{libdir}"])
+    out = subprocess.check_output([str(exe)]).decode().split()
+    s, jR, jL, cap = (int(x) for x in out)
+    assert [s, jR, jL, cap] == _plan(lib, 100_000_000, 1e6)
