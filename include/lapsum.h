@@ -241,7 +241,10 @@ LAPSUM_API int lapsum_get_stats_rows(lapsum_stats *out, int64_t max_rows, int64_
 /* Static string for a return code. */
 LAPSUM_API const char *lapsum_strerror(int code);
 
-/* Frees every workspace of the current device (synchronises the device). */
+/* Frees every workspace of the current device (synchronises the device first).
+ * No other host thread may be inside a call on that device meanwhile; the
+ * stats of earlier calls are gone, and the next call on a stream allocates its
+ * workspace again. */
 LAPSUM_API int lapsum_release(void);
 
 /*
