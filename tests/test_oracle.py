@@ -454,3 +454,19 @@ def test_tail_sums_match_scipy_logsumexp(orc):
         SR = math.exp(logsumexp(-(hi - float(aR)) / t)) if hi.size else 0.0
         assert abs(got["S_L"] - SL) <= 1e-12 * max(SL, 1e-300)
         assert abs(got["S_R"] - SR) <= 1e-12 * max(SR, 1e-300)
+
+
+# ------------------------------------------------------ stored expected values
+def test_golden_forced_fallback_is_reproduced_by_the_oracle(orc):
+    # tests/golden/forced_fallback.json holds values written by the oracle alone
+    # (tests/golden/make_golden.py): running the script's computation again gives
+    # every stored field exactly (seed, ranks, bracket ends, counts, G values, b)
+    import importlib.util
+    import json
+    import os
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(here, "make_golden.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    stored = json.load(open(os.path.join(here, "forced_fallback.json")))
+    assert mod.forced_fallback() == stored
