@@ -161,6 +161,14 @@ def test_bracket_plan_ranks_fuzz(lib, orc):
         n = 10 ** 9
         _, jR, jL, _ = _plan(lib, n, pi * n, s, delta)
         assert (jR, jL) == orc.binom_ranks(s, pi, delta)
+    # budgets near n and far below one sample's worth, confidence down to 1e-12
+    for i in range(300):
+        s = int(rng.choice([50, 333, 4096, 5000, 65536]))
+        pi = float(1 - 10 ** rng.uniform(-6, -0.31)) if i % 2 else float(10 ** rng.uniform(-8, -6))
+        delta = float(10 ** rng.uniform(-12, -0.3))
+        n = 10 ** 9
+        _, jR, jL, _ = _plan(lib, n, pi * n, s, delta)
+        assert (jR, jL) == orc.binom_ranks(s, pi * n / n, delta)
 
 
 FWD_EX_ARGS = [C.c_void_p, C.c_int64, C.c_int64, C.c_double, C.c_double, C.c_void_p, C.c_void_p, C.c_void_p,
