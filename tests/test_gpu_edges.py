@@ -154,13 +154,14 @@ def test_select_walks_every_key_when_candidates_overflow(L, orc, band_cap):
 def tail_tolerance(r, a, t, S, S_far, n):
     """Bound on |S_gpu - S| for a tail sum of the streaming pass.  Terms with
     z = |r - a|/t <= 16 are fp64 (relative error ~1e-15, summed in fp64); terms
-    with 16 < z <= 40 are fp32: argument rounding (z up to 40, s = log2(e)/t and
-    r - a each rounded once: <= 2 * 40 * 2^-24 * ln 2 relative) plus ex2.approx
-    (< 2^-21), and each thread sums at most m of them in fp32 before one fp64
-    add (<= m 2^-24 relative); terms beyond z = 40 (< 4.3e-18 each) are dropped.
-    Scores within 0.01 t of z = 16 may fall in either tier."""
+    with 16 < z <= 40 are fp32, 2^{-z2} with z2 = z log2(e) formed in fp32 from
+    three roundings (r - a, the scale log2(e)/t, their product: |dz2| <= 3 z2 2^-24),
+    so the term's relative error ln2 |dz2| is at most 3 z 2^-24 (z <= 40), plus
+    ex2.approx (< 2^-21); each thread sums at most m of them in fp32 before one
+    fp64 add (<= m 2^-24 relative); terms beyond z = 40 (< 4.3e-18 each) are
+    dropped.  Scores within 0.01 t of z = 16 may fall in either tier."""
     m = math.ceil(n / (3 * 148 * 256)) + 8
-    per_far = 2 * 40 * 2.0**-24 * math.log(2) + 2.0**-21 + m * 2.0**-24
+    per_far = 3 * 40 * 2.0**-24 + 2.0**-21 + m * 2.0**-24
     z = np.abs(r.astype(np.float64) - float(a)) / t
     edge = np.count_nonzero(np.abs(z - 16.0) < 0.01) * math.exp(-15.99)
     return 1e-12 * S + per_far * (S_far + edge) + np.count_nonzero(z > 39.9) * 4.3e-18
